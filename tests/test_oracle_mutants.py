@@ -1,0 +1,144 @@
+"""Planted mistakes: each plausible slip in the oracle must fail one of its pins.
+
+Every mutant is a one-line edit of a temporary copy of oracle/qsgd_oracle.c,
+compiled on the CPU.  The battery below re-runs the pins (Philox known answers,
+textbook omega codewords, omega round trip, hand-derived golden streams, the
+decode-accumulate hand values, unbiasedness on a small sweep).
+"""
+
+import os
+import shutil
+
+import numpy as np
+import pytest
+
+import oracle as oracle_mod
+from helpers import (bits_to_words, fixture_decoded, fixture_vector, load_kat,
+                     load_omega_codewords, load_streams, words_to_bits)
+import stats_common as sc
+
+SRC = os.path.join(os.path.dirname(oracle_mod.__file__), "qsgd_oracle.c")
+
+MUTANTS = {
+    "philox_swap_hi_lo": ("uint32_t y1 = lo1;", "uint32_t y1 = hi1;"),
+    "philox_no_key_bump": ("k1 += W1;", ""),
+    "philox_wrong_multiplier_operand": ("(uint64_t)M1 * (uint64_t)x2", "(uint64_t)M1 * (uint64_t)x1"),
+    "random_word_wrong_lane": ("return out[i % 4];", "return out[(i + 1) % 4];"),
+    "uniform_wrong_shift": ("(float)(r >> 9) * 0x1p-23f", "(float)(r >> 8) * 0x1p-23f"),
+    "omega_len_off_by_one": ("len += b;", "len += b - 1;"),
+    "omega_groups_reversed": ("for (int g = ngroups - 1; g >= 0; --g) {", "for (int g = 0; g < ngroups; ++g) {"),
+    "omega_get_group_width": ("for (uint64_t t = 0; t < value; ++t) {", "for (uint64_t t = 1; t < value; ++t) {"),
+    "round_up_direction": ("if (u < p) k += 1;", "if (u > p) k += 1;"),
+    "round_to_nearest": ("float l = floorf(t);", "float l = roundf(t);"),
+    "scale_inverted": ("float sinv = (float)s / norm;", "float sinv = norm / (float)s;"),
+    "l1_norm": ("sum += (double)v[i] * (double)v[i];", "sum += fabs((double)v[i]);"),
+    "gap_origin_zero": ("int64_t prev = -1;\n        for (uint64_t i = 0; i < m && err == 0; ++i) {",
+                        "int64_t prev = 0;\n        for (uint64_t i = 0; i < m && err == 0; ++i) {"),
+    "gap_not_updated": ("prev = (int64_t)i;\n            uint32_t k", "uint32_t k"),
+    "sign_inverted": ("put_bit(words, cap_words, &pos, levels[i] < 0);",
+                      "put_bit(words, cap_words, &pos, levels[i] > 0);"),
+    "fields_swapped": ("err |= qo_omega_put(words, cap_words, &pos, gap);\n            err |= put_bit(words, cap_words, &pos, levels[i] < 0);\n            err |= qo_omega_put(words, cap_words, &pos, k);",
+                       "err |= qo_omega_put(words, cap_words, &pos, k);\n            err |= put_bit(words, cap_words, &pos, levels[i] < 0);\n            err |= qo_omega_put(words, cap_words, &pos, gap);"),
+    "bit_order_lsb_first": ("if (bit) words[w] |= (uint32_t)1u << (31 - (unsigned)(*pos % 32));",
+                            "if (bit) words[w] |= (uint32_t)1u << ((unsigned)(*pos % 32));"),
+    "decode_scale_inverted": ("float scale = norm / (float)s;", "float scale = (float)s / norm;"),
+    "decode_sign_dropped": ("if (q < 0) value = -value;", ""),
+    "accumulate_overwrites": ("out[i] = out[i] + q[i];", "out[i] = q[i];"),
+    "decode_index_not_advanced": ("idx += (int64_t)gap;", "idx += 1;"),
+}
+
+
+# Survives every CPU pin: all CPU pins use seeds below 2^32 and no published
+# known-answer vector has a non-zero key with counter (j, 0, 0, 0).  It is caught
+# by the GPU test that runs curand's Philox4_32_10 generator
+# (tests/test_gpu_philox_curand.py).
+GPU_PINNED_MUTANTS = {
+    "random_word_key_halves_swapped": (
+        "uint32_t key[2] = {(uint32_t)(seed & 0xFFFFFFFFu), (uint32_t)(seed >> 32)};",
+        "uint32_t key[2] = {(uint32_t)(seed >> 32), (uint32_t)(seed & 0xFFFFFFFFu)};"),
+}
+
+
+def _build_mutant(tmp_path, name, old, new):
+    src = open(SRC).read()
+    assert src.count(old) == 1, name
+    d = tmp_path / name
+    d.mkdir()
+    shutil.copy(os.path.join(os.path.dirname(SRC), "qsgd_oracle.h"), d / "qsgd_oracle.h")
+    (d / "qsgd_oracle.c").write_text(src.replace(old, new))
+    out = oracle_mod.build(force=True, src=str(d / "qsgd_oracle.c"), out=str(d / "lib.so"))
+    return oracle_mod.Oracle(oracle_mod.load(out))
+
+
+def pin_battery(o) -> list:
+    """Names of the pins that fail for oracle o."""
+    failed = []
+    for ctr, key, expect in load_kat():
+        if [int(x) for x in o.philox(ctr, key)] != expect:
+            failed.append("philox_kat")
+            break
+    for N, code in load_omega_codewords():
+        if o.omega_bits(N) != code or o.omega_len(N) != len(code):
+            failed.append("omega_textbook")
+            break
+    vals = np.arange(1, 4097, dtype=np.uint64)
+    try:
+        words, nbits = o.omega_put_many(vals)
+        dec, pos = o.omega_get_many(words, len(vals), nbits)
+        if pos != nbits or list(dec) != [int(x) for x in vals]:
+            failed.append("omega_round_trip")
+    except (ValueError, AssertionError):
+        failed.append("omega_round_trip")
+    for case in load_streams():
+        v = fixture_vector(case["v"])
+        bits = "".join(case["bits"]).replace(" ", "")
+        try:
+            w, off, _, st = o.encode(v, case["d"], case["s"], case["seed"])
+            ok = ([int(x) for x in off] == case["offsets"] and words_to_bits(w, len(bits)) == bits
+                  and st == case["status"])
+        except RuntimeError:
+            ok = False
+        if not ok:
+            failed.append("golden_encode")
+            break
+    for case in load_streams():
+        out, st = o.decode(bits_to_words("".join(case["bits"]).replace(" ", "")),
+                           np.array(case["offsets"], np.uint64), len(case["v"]), case["d"], case["s"])
+        if out.view(np.uint32).tolist() != fixture_decoded(case["decoded"]).view(np.uint32).tolist():
+            failed.append("golden_decode")
+            break
+    a = bits_to_words("01000000101000000000000000000000" + "00110" + "00101000")
+    b = bits_to_words("01000000000000000000000000000000" + "100" + "1" + "0")
+    out = np.array([0.5, -0.0], dtype=np.float32)
+    o.decode_accumulate([(a, np.array([0, 45], np.uint64)), (b, np.array([0, 37], np.uint64))],
+                        2, 2, 5, out)
+    f = np.float32
+    expect = np.array([f(f(0.5) + f(3)) + f(0), f(f(-0.0) + f(4)) + f(-0.4)], np.float32)
+    if out.view(np.uint32).tolist() != expect.view(np.uint32).tolist():
+        failed.append("accumulate_hand")
+    # small unbiasedness sweep: 4096 N(0,1) coordinates, s = 8, 400 seeds
+    from quantized_gradient_compression_b200 import workloads
+    v = workloads.normal(4096, 1)
+    sums = sc.Sums(v.size)
+    v64 = v.astype(np.float64)
+    for seed in range(400):
+        levels, norms, _ = o.quantize(v, v.size, 8, seed)
+        sums.add_levels(v64, levels, norms[0], 8)
+    try:
+        sc.check_unbiased(v, 8, sums, max_beyond_4se=10)
+    except AssertionError:
+        failed.append("unbiased")
+    return failed
+
+
+def test_unmutated_oracle_passes_battery(tmp_path):
+    o = _build_mutant(tmp_path, "identity", "int qo_omega_len(uint64_t N) {", "int qo_omega_len(uint64_t N) {")
+    assert pin_battery(o) == []
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(tmp_path, name):
+    old, new = MUTANTS[name]
+    o = _build_mutant(tmp_path, name, old, new)
+    failed = pin_battery(o)
+    assert failed, "mutant %s survived every pin" % name
