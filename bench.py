@@ -1,0 +1,422 @@
+"""QSGD codec benchmark on B200: encode, decode and decode-accumulate throughput.
+
+One step is the whole hot path over one synthetic ResNet-50-sized gradient
+(n = 25,557,032 fp32 in 54 Gaussian layers, bucket d = 512, s = 16):
+  qsgd_encode (bucket norm, Philox stochastic rounding, Elias-omega packing,
+  look-back scan) -> qsgd_decode (dense fp32) -> qsgd_decode_accumulate (the
+  step's stream summed into a receiver buffer).
+The metric is GB/s of fp32 gradient input (4n bytes per step) and the fraction of
+the measured HBM roofline.  The L2 (126 MB, larger than the 110 MB working set of
+a step) is flushed before every timed step by writing a 512 MB buffer.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun (N > 1) every rank runs an independent replica (the codec does not
+shard); the step time is the maximum over ranks and `value` counts all ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "QSGD encode & decode GB/s of fp32 gradient input; % of B200 HBM roofline"
+FALLBACK_HBM_GBS = 6650.0
+
+# DRAM traffic of the dominant kernel from one ncu capture (dram__bytes_read.sum +
+# dram__bytes_write.sum per launch, full workload), with the hash of the kernel
+# sources it was taken on; reported as null once the sources differ.
+TRAFFIC = {"kernel": None, "bytes_per_launch": None, "sources_sha256": None}
+
+
+def sources_sha256() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "quantized_gradient_compression_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def workload():
+    from quantized_gradient_compression_b200 import workloads as W
+
+    return W.C2
+
+
+def config_dict(w, extra=None):
+    c = {"workload": w.name, "n": w.n, "bucket_d": w.d, "s": w.s, "philox_seed": w.seed,
+         "data": "54 Gaussian layers, Dirichlet(1) lengths, log10 sigma ~ U[-4,-1], data seed %d"
+                 % w.data_seed,
+         "step": "encode -> decode -> decode_accumulate(K=1)",
+         "l2": "flushed before every timed step (512 MB write)"}
+    if extra:
+        c.update(extra)
+    return c
+
+
+# --------------------------------------------------------------------------
+# clocks sampled during the timed region
+# --------------------------------------------------------------------------
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_index), "--query-gpu=" + self.QUERY,
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.15)
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append({"sm": float(parts[1]), "max": float(parts[2]), "power": float(parts[3]),
+                             "hw": parts[5], "hw_thermal": parts[6], "sw_thermal": parts[7],
+                             "sw_power": parts[8]})
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        load = [r for r in rows if r["power"] > 200.0] or rows
+        reasons = set()
+        for r in rows:
+            for key, name in (("hw", "hw_slowdown"), ("hw_thermal", "hw_thermal_slowdown"),
+                              ("sw_thermal", "sw_thermal_slowdown"), ("sw_power", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in load),
+                "sm_max_mhz": max(r["max"] for r in rows), "reasons": sorted(reasons),
+                "samples": len(rows), "samples_under_load": len(load)}
+
+
+# --------------------------------------------------------------------------
+# distributed plumbing (replicas; timing only)
+# --------------------------------------------------------------------------
+def init_dist(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+# --------------------------------------------------------------------------
+# the oracle as the CPU baseline / reference arm
+# --------------------------------------------------------------------------
+def time_oracle(v: np.ndarray, w, min_seconds: float = 10.0, max_reps: int = 3):
+    import oracle
+
+    o = oracle.default()
+    reps, total = 0, 0.0
+    while reps < max_reps and (reps == 0 or total < min_seconds):
+        t0 = time.perf_counter()
+        words, offsets, _, _ = o.encode(v, w.d, w.s, w.seed)
+        o.decode(words, offsets, v.size, w.d, w.s)
+        acc = np.zeros(v.size, dtype=np.float32)
+        o.decode_accumulate([(words, offsets)], v.size, w.d, w.s, acc)
+        total += time.perf_counter() - t0
+        reps += 1
+    per_step = total / reps
+    return {"value": 4.0 * v.size / per_step / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": "full workload vector (n=%d), %d step(s) of encode+decode+decode_accumulate, "
+                      "single-threaded C oracle" % (v.size, reps),
+            "seconds_per_step": per_step}
+
+
+def run_reference(args, w):
+    """The reference arm: the oracle (single-threaded C) on the host, as it stands.
+
+    Every step encodes, decodes and decode-accumulates a bounded sample of the
+    workload, sized from a probe so that the K timed steps take about a minute."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    v = w.generate()
+    import oracle
+
+    o = oracle.default()
+
+    def step(vs):
+        words, offsets, _, _ = o.encode(vs, w.d, w.s, w.seed)
+        o.decode(words, offsets, vs.size, w.d, w.s)
+        acc = np.zeros(vs.size, dtype=np.float32)
+        o.decode_accumulate([(words, offsets)], vs.size, w.d, w.s, acc)
+
+    probe_n = min(w.n, 1 << 20)
+    t0 = time.perf_counter()
+    step(np.ascontiguousarray(v[:probe_n]))
+    rate = probe_n / (time.perf_counter() - t0)  # coordinates per second
+    K = max(1, args.steps)
+    sample_n = int(min(w.n, max(w.d, 60.0 / K * rate)))
+    sample_n -= sample_n % w.d if sample_n > w.d else 0
+    vs = np.ascontiguousarray(v[:sample_n])
+    for _ in range(min(args.warmup, 3)):
+        step(vs)
+    t0 = time.perf_counter()
+    for _ in range(K):
+        step(vs)
+    per_step = (time.perf_counter() - t0) / K
+    value = 4.0 * sample_n / per_step / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": K, "warmup": min(args.warmup, 3), "ms_per_step": per_step * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic", "config": config_dict(w, {"sample_n": sample_n}),
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": "first %d coordinates of the workload per step" % sample_n},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------
+# our arm
+# --------------------------------------------------------------------------
+def run_ours(args, w):
+    import torch
+    from quantized_gradient_compression_b200 import binding as B
+
+    rank, world, local = init_dist(args)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+
+    v_host = w.generate()
+    n, d, s = w.n, w.d, w.s
+    seed = w.seed + rank
+    nb = B.qsgd_num_buckets(n, d)
+    cap = B.qsgd_max_encoded_words(n, d, s)
+    x = torch.from_numpy(v_host).to(dev)
+    words = torch.empty(cap, dtype=torch.int32, device=dev)
+    offsets = torch.empty(nb + 1, dtype=torch.int64, device=dev)
+    out = torch.empty(n, dtype=torch.float32, device=dev)
+    acc = torch.zeros(n, dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    ws_bytes = B.qsgd_encode_workspace_bytes(n, d, s)
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def check(code, what):
+        if code != 0:
+            raise RuntimeError("%s failed: %s" % (what, B.qsgd_error_string(code)))
+
+    def encode():
+        check(B.qsgd_encode(x.data_ptr(), n, d, s, seed, words.data_ptr(), cap, offsets.data_ptr(),
+                            ws.data_ptr(), ws_bytes, status.data_ptr(), sh), "qsgd_encode")
+
+    def decode():
+        check(B.qsgd_decode(words.data_ptr(), cap, offsets.data_ptr(), n, d, s, out.data_ptr(),
+                            status.data_ptr(), sh), "qsgd_decode")
+
+    def accumulate():
+        check(B.qsgd_decode_accumulate([words.data_ptr()], [cap], [offsets.data_ptr()], 1, n, d, s,
+                                       acc.data_ptr(), status.data_ptr(), sh), "qsgd_decode_accumulate")
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        encode()
+        decode()
+        accumulate()
+    torch.cuda.synchronize()
+    st = int(status.item())
+    if st != 0:
+        raise RuntimeError("device status %d after warm-up" % st)
+    total_bits = int(offsets[-1].item())
+    comp_bytes = 4 * ((total_bits + 31) // 32) + 8 * (nb + 1)
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        for k in range(K):
+            flush.zero_()
+            ev[k][0].record(stream)
+            encode()
+            ev[k][1].record(stream)
+            decode()
+            ev[k][2].record(stream)
+            accumulate()
+            ev[k][3].record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    t_enc = sum(ev[k][0].elapsed_time(ev[k][1]) for k in range(K)) / K
+    t_dec = sum(ev[k][1].elapsed_time(ev[k][2]) for k in range(K)) / K
+    t_acc = sum(ev[k][2].elapsed_time(ev[k][3]) for k in range(K)) / K
+    t_step = sum(ev[k][0].elapsed_time(ev[k][3]) for k in range(K)) / K
+    t_step_max = max_over_ranks(t_step, world)
+    if int(status.item()) != 0:
+        raise RuntimeError("device status %d in the timed region" % int(status.item()))
+
+    # end to end through the C ABI with host buffers: pinned H2D of the input,
+    # the three calls, D2H of the accumulated result
+    h_in = torch.from_numpy(v_host).pin_memory()
+    h_out = torch.empty(n, dtype=torch.float32).pin_memory()
+    E = args.e2e_steps
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    for it in range(E + 2):
+        if it == 2:
+            e0.record(stream)
+        x.copy_(h_in, non_blocking=True)
+        encode()
+        decode()
+        accumulate()
+        h_out.copy_(acc, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t_e2e = max_over_ranks(e0.elapsed_time(e1) / E, world)
+
+    peak, peak_kind = measured_peaks()
+    in_bytes = 4.0 * n
+    enc_bytes = in_bytes + comp_bytes            # read fp32, write stream + header
+    dec_bytes = comp_bytes + in_bytes            # read stream + header, write fp32
+    acc_bytes = comp_bytes + 2 * in_bytes        # read stream, read + write the sum
+    phases = {
+        "encode": {"ms": t_enc, "input_gbs": in_bytes / t_enc / 1e6,
+                   "algorithmic_gbs": enc_bytes / t_enc / 1e6, "roofline_frac": enc_bytes / t_enc / 1e6 / peak},
+        "decode": {"ms": t_dec, "input_gbs": in_bytes / t_dec / 1e6,
+                   "algorithmic_gbs": dec_bytes / t_dec / 1e6, "roofline_frac": dec_bytes / t_dec / 1e6 / peak},
+        "decode_accumulate": {"ms": t_acc, "input_gbs": in_bytes / t_acc / 1e6,
+                              "algorithmic_gbs": acc_bytes / t_acc / 1e6,
+                              "roofline_frac": acc_bytes / t_acc / 1e6 / peak},
+    }
+    dominant = max(phases, key=lambda k: phases[k]["ms"])
+    dom = phases[dominant]
+    traffic = None
+    if TRAFFIC["bytes_per_launch"] is not None and TRAFFIC["sources_sha256"] == sources_sha256():
+        traffic = TRAFFIC["bytes_per_launch"]
+
+    result = {
+        "metric": METRIC,
+        "value": world * in_bytes / t_step_max / 1e6,
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": t_step_max,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic",
+        "config": config_dict(w, {"parallelism": "replicas x%d" % world}),
+        "bits_per_coord": total_bits / n,
+        "compressed_bytes": comp_bytes,
+        "phases": phases,
+        "roofline": {"bound": "hbm", "kernel": {"encode": "qsgd encode (encode_fast<4>)",
+                                                  "decode": "qsgd decode (decode_buckets<false>)",
+                                                  "decode_accumulate": "qsgd decode_accumulate"}[dominant],
+                     "achieved": dom["algorithmic_gbs"], "peak": peak, "unit": "GB/s",
+                     "frac": dom["algorithmic_gbs"] / peak, "traffic": traffic,
+                     "peak_source": "%s hbm_gbs (burst copy)" % peak_kind,
+                     "algorithmic_bytes_per_launch": {"encode": enc_bytes, "decode": dec_bytes,
+                                                      "decode_accumulate": acc_bytes}[dominant]},
+        "e2e": {"value": world * in_bytes / t_e2e / 1e6, "unit": "GB/s",
+                "h2d_bytes_per_step": int(in_bytes), "d2h_bytes_per_step": int(in_bytes),
+                "ms_per_step": t_e2e},
+        "gpu_launches": 3 * K,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = time_oracle(v_host, w)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse_args()
+    w = workload()
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

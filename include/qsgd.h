@@ -1,0 +1,149 @@
+/*
+ * qsgd.h -- C ABI of the B200 (sm_100a) QSGD gradient codec.
+ *
+ * The method is the one of the page "QSGD (Quantized Stochastic Gradient Descent)
+ * with Elias Coding" (AIMech curated entry):
+ *   - definition paragraph: Q_s(v)_i = ||v||_2 * sgn(v_i) * xi_i(v, s), where
+ *     xi_i = (l_i + 1)/s with probability p_i = s|v_i|/||v||_2 - l_i, else l_i/s,
+ *     l_i = floor(s|v_i|/||v||_2); the sparse tuple (||v||_2, signs, run-length
+ *     gaps, levels k_i = s*xi_i) is sent with Elias recursive (omega) codes;
+ *   - claim "Elias coding communication complexity tradeoff": F = 32 bits for the
+ *     norm, index gaps between non-zeros, levels k_i in {1..s};
+ *   - claim "QSVRG, non-convex and multi-GPU bucketed training": d-block
+ *     bucketing, each bucket quantised with its own norm;
+ *   - definition paragraph ("distributed data-parallel optimization"): a receiver
+ *     decodes its peers' streams and sums them.
+ *
+ * Wire format (the same one the test oracle implements, independently):
+ *   bucket b = coordinates [b*d, min(n,(b+1)*d)); per bucket: 32 raw bits of the
+ *   fp32 norm, then per coordinate with k >= 1 in ascending index:
+ *   omega(gap) || sign (1 = negative) || omega(k); gap = i - prev, prev = -1 at the
+ *   bucket start.  Bits MSB-first within uint32 words; buckets back to back.
+ *   offsets[b] = first bit of bucket b; offsets[nb] = total bits.
+ *   Random source: u_i = floor(r_i / 2^9) * 2^-23 with r_i word (i mod 4) of
+ *   Philox4x32-10(counter = (lo32(i/4), hi32(i/4), 0, 0), key = (lo32(seed),
+ *   hi32(seed))), i the global coordinate index.  Quantiser arithmetic in fp32,
+ *   round-to-nearest-even: sinv = s / norm (once per bucket), t = |v_i| * sinv,
+ *   l = floor(t), p = t - l, k = min(l + [u_i < p], s).  Decoder: fl(fl(norm/s)*k),
+ *   sign applied last, +0.0 off the support.
+ *
+ * Conventions for every call below:
+ *   - "d_" pointers are device pointers on the current CUDA device; "h_" pointers
+ *     are host pointers.  The caller owns every buffer.  The library allocates no
+ *     memory.
+ *   - All work is enqueued on `stream` (0 = legacy default stream) and the call
+ *     returns without synchronising.
+ *   - The return value (qsgd_err) reports argument and launch errors found on the
+ *     host.  Data-dependent conditions found on the device are OR-ed into the
+ *     device word *d_status (QSGD_ST_* bits); the caller zeroes it beforehand and
+ *     reads it after synchronising.  d_status may not be NULL.
+ *   - Limits: 0 <= n <= 2^34, 1 <= d <= 2^31, 1 <= s <= 2^22, and the size bound
+ *     of the stream (qsgd_max_encoded_words * 32) below 2^38 bits.
+ *   - Kernels never trap and never wait without a bound.
+ */
+#ifndef QSGD_H
+#define QSGD_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define QSGD_API __attribute__((visibility("default")))
+#else
+#define QSGD_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Host return codes. */
+typedef enum {
+    QSGD_OK = 0,
+    QSGD_ERR_ARG = 1,       /* a pointer, size or parameter out of range */
+    QSGD_ERR_CAPACITY = 2,  /* output buffer smaller than qsgd_max_encoded_words */
+    QSGD_ERR_CUDA = 3,      /* a CUDA runtime call or kernel launch failed */
+    QSGD_ERR_WORKSPACE = 4  /* workspace smaller than qsgd_encode_workspace_bytes */
+} qsgd_err;
+
+/* Device status bits, OR-ed into *d_status. */
+enum {
+    QSGD_ST_NONFINITE = 1,        /* encode: a bucket's norm is not finite; sent as zero */
+    QSGD_ST_BAD_STREAM = 2,       /* decode: malformed bucket (see qsgd_decode) */
+    QSGD_ST_LOOKBACK_TIMEOUT = 4, /* encode: a bounded wait ran out; output invalid */
+    QSGD_ST_OVERFLOW = 8,         /* encode: a write would pass words_capacity */
+    QSGD_ST_RANGE = 16            /* encode: norm > 0 but s/norm overflows fp32; sent as zero */
+};
+
+/* Number of buckets, ceil(n / d) (0 when d == 0). */
+QSGD_API uint64_t qsgd_num_buckets(uint64_t n, uint32_t d);
+
+/* Worst-case stream size in 32-bit words: ceil(sum_b (32 + m_b*(2 + |omega(s)|)) / 32)
+ * with m_b the length of bucket b.  A record of gap g costs at most g*(2+|omega(s)|)
+ * bits and the gaps of a bucket sum to at most m_b.  Returns 0 for invalid d or s. */
+QSGD_API uint64_t qsgd_max_encoded_words(uint64_t n, uint32_t d, uint32_t s);
+
+/* Bytes of device workspace qsgd_encode needs for (n, d, s).  The workspace holds
+ * the scan state of the single-pass encoder (tile descriptors, tail words, per-bucket
+ * norms for large buckets).  It must be zero-filled once before its first use
+ * (qsgd_workspace_init); every encode leaves it ready for the next one.  One
+ * workspace must not be used by two encodes that may run at the same time. */
+QSGD_API size_t qsgd_encode_workspace_bytes(uint64_t n, uint32_t d, uint32_t s);
+
+/* Zero-fills a workspace (cudaMemsetAsync on `stream`). */
+QSGD_API int qsgd_workspace_init(void* d_ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Encoder: QSGD-quantises d_in[0..n) bucket by bucket and writes the Elias-omega
+ * stream.  (Definition paragraph and the two claims cited above.)
+ *   d_in            fp32[n], any alignment (16-byte alignment and d % 4 == 0 take
+ *                   the fast path)
+ *   seed            Philox key of the stochastic rounding
+ *   d_words         uint32[words_capacity]; words past ceil(offsets[nb]/32) are
+ *                   not written
+ *   words_capacity  must be >= qsgd_max_encoded_words(n, d, s), else QSGD_ERR_CAPACITY
+ *   d_offsets       uint64[nb+1] (bit offsets, see above); 8-byte aligned
+ *   d_ws, ws_bytes  workspace of at least qsgd_encode_workspace_bytes(n, d, s)
+ *   d_status        NONFINITE / RANGE per degenerate bucket (sent as 32 zero bits),
+ *                   LOOKBACK_TIMEOUT or OVERFLOW if the output is not valid.
+ * The stream is a deterministic function of (d_in, n, d, s, seed). */
+QSGD_API int qsgd_encode(const float* d_in, uint64_t n, uint32_t d, uint32_t s, uint64_t seed,
+                uint32_t* d_words, uint64_t words_capacity, uint64_t* d_offsets,
+                void* d_ws, size_t ws_bytes, uint32_t* d_status, cudaStream_t stream);
+
+/* Decoder: writes Q_s(v) as dense fp32 d_out[0..n) (definition paragraph:
+ * ||v||_2 * sgn(v_i) * k_i / s, evaluated as fl(fl(norm/s) * k), sign last; +0.0 off
+ * the support).  Buckets are decoded in parallel from d_offsets.
+ *   d_words, num_words  the stream and its length in words (bounds every read)
+ *   d_offsets           uint64[nb+1] as written by qsgd_encode
+ * Sets QSGD_ST_BAD_STREAM for a bucket whose bits overrun offsets[b+1], whose header
+ * range is shorter than 32 bits or passes 32*num_words, or that holds an index
+ * >= bucket length, a level k > s or 0, or a negative / non-finite norm, or a zero
+ * norm with records.  A malformed bucket's outputs are unspecified; nothing outside
+ * that bucket's range of d_out is written. */
+QSGD_API int qsgd_decode(const uint32_t* d_words, uint64_t num_words, const uint64_t* d_offsets,
+                uint64_t n, uint32_t d, uint32_t s, float* d_out, uint32_t* d_status,
+                cudaStream_t stream);
+
+/* Receiver aggregation: d_out[i] <- (((d_out[i] + q^0_i) + q^1_i) + ... + q^{K-1}_i),
+ * fp32 adds in stream order j = 0..K-1, q^j the decoded stream j (+0.0 off its
+ * support).  All K streams were encoded with the same (n, d, s).
+ *   h_words, h_num_words, h_offsets  host arrays of K entries holding device
+ *                                    pointers / word counts (copied at the call)
+ *   1 <= K <= 1024
+ * Status bits as for qsgd_decode. */
+QSGD_API int qsgd_decode_accumulate(const uint32_t* const* h_words, const uint64_t* h_num_words,
+                           const uint64_t* const* h_offsets, int K, uint64_t n, uint32_t d,
+                           uint32_t s, float* d_out, uint32_t* d_status, cudaStream_t stream);
+
+/* Static description of a host return code. */
+QSGD_API const char* qsgd_error_string(int code);
+
+/* Library version string. */
+QSGD_API const char* qsgd_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -68,6 +68,9 @@ def _declare(lib):
         "qo_capacity_words": (c_u64, [c_u64, c_u64, c_u32]),
         "qo_encode": (c_int, [f32p, c_u64, c_u64, c_u32, c_u64, f32p, u32p, c_u64, u64p,
                               f32p, u32p]),
+        "qo_encode_bucket": (c_int, [f32p, c_u64, c_u64, c_u32, c_u64, f32p, u32p, c_u64, u64p,
+                                     f32p, i32p, u32p]),
+        "qo_decode_bucket": (c_int, [u32p, c_u64, c_u64, c_u64, c_u32, f32p, u32p]),
         "qo_decode": (c_int, [u32p, u64p, c_u64, c_u64, c_u32, f32p, u32p]),
         "qo_decode_levels": (c_int, [u32p, u64p, c_u64, c_u64, c_u32, i32p, f32p, u32p]),
         "qo_decode_accumulate": (c_int, [ctypes.POINTER(u32p), ctypes.POINTER(u64p), c_int,
@@ -198,6 +201,34 @@ class Oracle:
             raise RuntimeError("oracle encode failed (status %d)" % st.value)
         nwords = (int(offsets[nb]) + 31) // 32
         return words[:nwords].copy(), offsets, norms[:nb], st.value
+
+    def encode_bucket(self, vb: np.ndarray, base: int, s: int, seed: int, norm_in=None):
+        """One bucket at global index `base` as a standalone bit string (words, nbits)."""
+        vb = np.ascontiguousarray(vb, dtype=np.float32)
+        m = vb.size
+        cap = (32 + m * (2 + self.omega_len(s))) // 32 + 2
+        words = np.zeros(cap, dtype=np.uint32)
+        levels = np.zeros(max(m, 1), dtype=np.int32)
+        pos = ctypes.c_uint64(0)
+        st = ctypes.c_uint32(0)
+        nin = None if norm_in is None else np.asarray([norm_in], dtype=np.float32)
+        norm = np.zeros(1, dtype=np.float32)
+        rc = self.lib.qo_encode_bucket(_ptr(vb, ctypes.c_float), m, base, s, seed,
+                                       _ptr(nin, ctypes.c_float) if nin is not None else None,
+                                       _ptr(words, ctypes.c_uint32), cap, ctypes.byref(pos),
+                                       _ptr(norm, ctypes.c_float), _ptr(levels, ctypes.c_int32),
+                                       ctypes.byref(st))
+        assert rc == 0
+        return words, pos.value, st.value
+
+    def decode_bucket(self, words: np.ndarray, begin: int, end: int, m: int, s: int):
+        words = np.ascontiguousarray(words, dtype=np.uint32)
+        out = np.zeros(max(m, 1), dtype=np.float32)
+        st = ctypes.c_uint32(0)
+        rc = self.lib.qo_decode_bucket(_ptr(words, ctypes.c_uint32), begin, end, m, s,
+                                       _ptr(out, ctypes.c_float), ctypes.byref(st))
+        assert rc == 0
+        return out[:m], st.value
 
     def decode(self, words: np.ndarray, offsets: np.ndarray, n: int, d: int, s: int):
         words = np.ascontiguousarray(words, dtype=np.uint32)

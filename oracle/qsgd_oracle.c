@@ -218,6 +218,28 @@ static int put_bits_msb_first(uint32_t* words, uint64_t cap, uint64_t* pos, uint
     return 0;
 }
 
+int qo_encode_bucket(const float* v, uint64_t m, uint64_t base, uint32_t s, uint64_t seed,
+                     const float* norm_in, uint32_t* words, uint64_t cap_words, uint64_t* pos,
+                     float* norm_out, int32_t* levels, uint32_t* status) {
+    float norm = qo_quantize_bucket(v, m, base, s, seed, norm_in, levels, status);
+    if (norm_out) *norm_out = norm;
+    uint32_t norm_bits;
+    memcpy(&norm_bits, &norm, sizeof norm_bits);
+    int err = put_bits_msb_first(words, cap_words, pos, norm_bits, 32);
+    int64_t prev = -1;
+    for (uint64_t i = 0; i < m && err == 0; ++i) {
+        if (levels[i] == 0) continue;
+        uint64_t gap = (uint64_t)((int64_t)i - prev);
+        prev = (int64_t)i;
+        uint32_t k = (uint32_t)(levels[i] < 0 ? -levels[i] : levels[i]);
+        err |= qo_omega_put(words, cap_words, pos, gap);
+        err |= put_bit(words, cap_words, pos, levels[i] < 0);
+        err |= qo_omega_put(words, cap_words, pos, k);
+    }
+    if (err) *status |= QO_ST_OVERFLOW;
+    return err ? -1 : 0;
+}
+
 int qo_encode(const float* v, uint64_t n, uint64_t d, uint32_t s, uint64_t seed,
               const float* norms_in, uint32_t* words, uint64_t cap_words,
               uint64_t* offsets, float* norms_out, uint32_t* status) {
@@ -231,24 +253,9 @@ int qo_encode(const float* v, uint64_t n, uint64_t d, uint32_t s, uint64_t seed,
         uint64_t base = b * d;
         uint64_t m = (b + 1 == nb) ? n - base : d;
         offsets[b] = pos;
-        float norm = qo_quantize_bucket(v + base, m, base, s, seed,
-                                        norms_in ? norms_in + b : NULL, levels, status);
-        if (norms_out) norms_out[b] = norm;
-        uint32_t norm_bits;
-        memcpy(&norm_bits, &norm, sizeof norm_bits);
-        int err = put_bits_msb_first(words, cap_words, &pos, norm_bits, 32);
-        int64_t prev = -1;
-        for (uint64_t i = 0; i < m && err == 0; ++i) {
-            if (levels[i] == 0) continue;
-            uint64_t gap = (uint64_t)((int64_t)i - prev);
-            prev = (int64_t)i;
-            uint32_t k = (uint32_t)(levels[i] < 0 ? -levels[i] : levels[i]);
-            err |= qo_omega_put(words, cap_words, &pos, gap);
-            err |= put_bit(words, cap_words, &pos, levels[i] < 0);
-            err |= qo_omega_put(words, cap_words, &pos, k);
-        }
-        if (err) {
-            *status |= QO_ST_OVERFLOW;
+        if (qo_encode_bucket(v + base, m, base, s, seed, norms_in ? norms_in + b : NULL, words,
+                             cap_words, &pos, norms_out ? norms_out + b : NULL, levels,
+                             status) != 0) {
             free(levels);
             return -1;
         }
@@ -296,6 +303,26 @@ static int parse_bucket(const uint32_t* words, uint64_t begin, uint64_t end, uin
     return 0;
 }
 
+int qo_decode_bucket(const uint32_t* words, uint64_t begin, uint64_t end, uint64_t m,
+                     uint32_t s, float* out, uint32_t* status) {
+    int32_t* levels = (int32_t*)malloc((size_t)(m ? m : 1) * sizeof(int32_t));
+    if (!levels) return -1;
+    float norm;
+    if (parse_bucket(words, begin, end, m, s, levels, &norm) != 0) *status |= QO_ST_BAD_STREAM;
+    float scale = norm / (float)s;
+    for (uint64_t i = 0; i < m; ++i) {
+        int32_t q = levels[i];
+        float value = 0.0f;
+        if (q != 0) {
+            value = scale * (float)(q < 0 ? -q : q);
+            if (q < 0) value = -value;
+        }
+        out[i] = value;
+    }
+    free(levels);
+    return 0;
+}
+
 int qo_decode_levels(const uint32_t* words, const uint64_t* offsets, uint64_t n,
                      uint64_t d, uint32_t s, int32_t* levels, float* norms,
                      uint32_t* status) {
@@ -316,26 +343,12 @@ int qo_decode(const uint32_t* words, const uint64_t* offsets, uint64_t n, uint64
               uint32_t s, float* out, uint32_t* status) {
     if (d < 1 || s < 1) return -1;
     uint64_t nb = (n + d - 1) / d;
-    int32_t* levels = (int32_t*)malloc((size_t)(d < n ? d : (n ? n : 1)) * sizeof(int32_t));
-    if (!levels) return -1;
     for (uint64_t b = 0; b < nb; ++b) {
         uint64_t base = b * d;
         uint64_t m = (b + 1 == nb) ? n - base : d;
-        float norm;
-        if (parse_bucket(words, offsets[b], offsets[b + 1], m, s, levels, &norm) != 0)
-            *status |= QO_ST_BAD_STREAM;
-        float scale = norm / (float)s;
-        for (uint64_t i = 0; i < m; ++i) {
-            int32_t q = levels[i];
-            float value = 0.0f;
-            if (q != 0) {
-                value = scale * (float)(q < 0 ? -q : q);
-                if (q < 0) value = -value;
-            }
-            out[base + i] = value;
-        }
+        if (qo_decode_bucket(words, offsets[b], offsets[b + 1], m, s, out + base, status) != 0)
+            return -1;
     }
-    free(levels);
     return 0;
 }
 

@@ -80,6 +80,16 @@ int qo_encode(const float* v, uint64_t n, uint64_t d, uint32_t s, uint64_t seed,
               const float* norms_in, uint32_t* words, uint64_t cap_words,
               uint64_t* offsets, float* norms_out, uint32_t* status);
 
+/* Encodes one bucket v[0..m) whose first coordinate has global index base at bit
+ * *pos (advanced); levels[m] is scratch.  Returns 0 or -1 on overflow. */
+int qo_encode_bucket(const float* v, uint64_t m, uint64_t base, uint32_t s, uint64_t seed,
+                     const float* norm_in, uint32_t* words, uint64_t cap_words, uint64_t* pos,
+                     float* norm_out, int32_t* levels, uint32_t* status);
+
+/* Decodes the bucket stored in bits [begin, end) (m coordinates) into out[m]. */
+int qo_decode_bucket(const uint32_t* words, uint64_t begin, uint64_t end, uint64_t m,
+                     uint32_t s, float* out, uint32_t* status);
+
 /* Decoder: out[n]. */
 int qo_decode(const uint32_t* words, const uint64_t* offsets, uint64_t n, uint64_t d,
               uint32_t s, float* out, uint32_t* status);

@@ -1,0 +1,204 @@
+// Host side of the QSGD C ABI (include/qsgd.h): argument checks, workspace layout,
+// kernel selection.  No allocation happens here or anywhere in the library.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <algorithm>
+#include <cstring>
+
+#include "../../include/qsgd.h"
+#include "qsgd_device.cuh"
+#include "qsgd_internal.h"
+
+namespace qsgd {
+
+uint32_t omega_len_host(uint64_t N) {
+    uint32_t len = 1;
+    while (N > 1) {
+        uint32_t b = 0;
+        for (uint64_t x = N; x; x >>= 1) ++b;
+        len += b;
+        N = b - 1;
+    }
+    return len;
+}
+
+namespace {
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+uint64_t ceil_div(uint64_t a, uint64_t b) { return (a + b - 1) / b; }
+
+bool valid_params(uint64_t n, uint32_t d, uint32_t s) {
+    return n <= kMaxN && d >= 1 && static_cast<uint64_t>(d) <= kMaxD && s >= 1 && s <= kMaxS;
+}
+
+uint32_t general_buckets_per_tile(uint32_t d) {
+    return d >= kGeneralTileCoords ? 1u : kGeneralTileCoords / d;
+}
+
+uint64_t max_bits(uint64_t n, uint32_t d, uint32_t s) {
+    if (n == 0) return 0;
+    const uint64_t nb = ceil_div(n, d);
+    const uint64_t per = 2u + omega_len_host(s);
+    // (32 + m_b * per) summed over buckets = 32 nb + n * per
+    return 32u * nb + n * per;
+}
+
+bool fast_eligible(const float* in, uint32_t d) {
+    return d >= kFastMinD && d <= kFastMaxD && d % 4 == 0 &&
+           (reinterpret_cast<uintptr_t>(in) & 15u) == 0;
+}
+
+}  // namespace
+
+WorkspaceLayout workspace_layout(uint64_t n, uint32_t d) {
+    WorkspaceLayout L{};
+    const uint64_t nb = n ? ceil_div(n, d) : 0;
+    const uint64_t per_tile = std::min<uint64_t>(kWarps, general_buckets_per_tile(d));
+    L.max_tiles = nb ? ceil_div(nb, per_tile) : 0;
+    L.desc_off = 256;
+    L.carry_off = L.desc_off + align256(8 * L.max_tiles);
+    L.norms_off = L.carry_off + align256(8 * L.max_tiles);
+    L.total = L.norms_off + align256(8 * nb);
+    return L;
+}
+
+}  // namespace qsgd
+
+using namespace qsgd;
+
+extern "C" {
+
+uint64_t qsgd_num_buckets(uint64_t n, uint32_t d) { return d ? ceil_div(n, d) : 0; }
+
+uint64_t qsgd_max_encoded_words(uint64_t n, uint32_t d, uint32_t s) {
+    if (!valid_params(n, d, s)) return 0;
+    return ceil_div(max_bits(n, d, s), 32);
+}
+
+size_t qsgd_encode_workspace_bytes(uint64_t n, uint32_t d, uint32_t s) {
+    if (!valid_params(n, d, s)) return 0;
+    return workspace_layout(n, d).total;
+}
+
+int qsgd_workspace_init(void* d_ws, size_t ws_bytes, cudaStream_t stream) {
+    if (!d_ws || ws_bytes == 0) return QSGD_ERR_ARG;
+    return cudaMemsetAsync(d_ws, 0, ws_bytes, stream) == cudaSuccess ? QSGD_OK : QSGD_ERR_CUDA;
+}
+
+int qsgd_encode(const float* d_in, uint64_t n, uint32_t d, uint32_t s, uint64_t seed,
+                uint32_t* d_words, uint64_t words_capacity, uint64_t* d_offsets, void* d_ws,
+                size_t ws_bytes, uint32_t* d_status, cudaStream_t stream) {
+    if (!valid_params(n, d, s) || !d_offsets || !d_status) return QSGD_ERR_ARG;
+    if (max_bits(n, d, s) > kMaxStreamBits) return QSGD_ERR_ARG;
+    if ((reinterpret_cast<uintptr_t>(d_offsets) & 7u) != 0 || (reinterpret_cast<uintptr_t>(d_words) & 3u) != 0)
+        return QSGD_ERR_ARG;
+    if (n == 0) {
+        return cudaMemsetAsync(d_offsets, 0, sizeof(uint64_t), stream) == cudaSuccess ? QSGD_OK
+                                                                                      : QSGD_ERR_CUDA;
+    }
+    if (!d_in || !d_words || !d_ws) return QSGD_ERR_ARG;
+    if ((reinterpret_cast<uintptr_t>(d_ws) & 255u) != 0) return QSGD_ERR_ARG;
+    if (words_capacity < qsgd_max_encoded_words(n, d, s)) return QSGD_ERR_CAPACITY;
+    const WorkspaceLayout L = workspace_layout(n, d);
+    if (ws_bytes < L.total) return QSGD_ERR_WORKSPACE;
+
+    char* ws = static_cast<char*>(d_ws);
+    EncodeArgs a{};
+    a.in = d_in;
+    a.n = n;
+    a.d = d;
+    a.s = s;
+    a.key0 = static_cast<uint32_t>(seed);
+    a.key1 = static_cast<uint32_t>(seed >> 32);
+    a.words = d_words;
+    a.cap_words = words_capacity;
+    a.offsets = d_offsets;
+    a.status = d_status;
+    a.ctrl = reinterpret_cast<ScanControl*>(ws);
+    a.desc = reinterpret_cast<uint64_t*>(ws + L.desc_off);
+    a.carry = reinterpret_cast<uint64_t*>(ws + L.carry_off);
+    a.norms = reinterpret_cast<float2*>(ws + L.norms_off);
+    a.nb = ceil_div(n, d);
+    const uint32_t wl = 2u + omega_len_host(s);
+    const bool fast = fast_eligible(d_in, d);
+    if (fast) {
+        a.buckets_per_tile = kWarps;
+        a.ntiles = ceil_div(a.nb, kWarps);
+        const uint64_t tile_bits = static_cast<uint64_t>(kWarps) * (32u + static_cast<uint64_t>(d) * wl);
+        a.smem_words = static_cast<uint32_t>(ceil_div(tile_bits, 32) + 2);
+    } else {
+        a.buckets_per_tile = general_buckets_per_tile(d);
+        a.ntiles = ceil_div(a.nb, a.buckets_per_tile);
+        // one chunk: 31 leading bits, kChunk records bounded by the gap argument plus
+        // one record whose gap reaches back past the chunk (<= 43 + 1 + |omega(s)|),
+        // and a norm for every bucket that starts inside the chunk
+        const uint64_t starts = kChunk / d + 2;
+        const uint64_t chunk_bits = 31u + static_cast<uint64_t>(kChunk) * wl + 44u + omega_len_host(s) + 32u * starts;
+        a.smem_words = static_cast<uint32_t>(ceil_div(chunk_bits, 32) + 2);
+    }
+    if ((kOmegaTab + static_cast<uint64_t>(a.smem_words)) * 4 > 200 * 1024) return QSGD_ERR_ARG;
+    if (a.ntiles > L.max_tiles) return QSGD_ERR_WORKSPACE;
+    const cudaError_t e = launch_encode(a, fast, stream);
+    return e == cudaSuccess ? QSGD_OK : QSGD_ERR_CUDA;
+}
+
+static int decode_impl(const uint32_t* const* words, const uint64_t* num_words,
+                       const uint64_t* const* offsets, int K, uint64_t n, uint32_t d, uint32_t s,
+                       float* d_out, uint32_t* d_status, cudaStream_t stream, bool accumulate) {
+    if (!valid_params(n, d, s) || !d_status || K < 1 || K > 1024) return QSGD_ERR_ARG;
+    if (n == 0) return QSGD_OK;
+    if (!d_out || !words || !num_words || !offsets) return QSGD_ERR_ARG;
+    for (int j = 0; j < K; ++j)
+        if (!words[j] || !offsets[j] || (reinterpret_cast<uintptr_t>(offsets[j]) & 7u) != 0)
+            return QSGD_ERR_ARG;
+    DecodeArgs a{};
+    a.n = n;
+    a.d = d;
+    a.s = s;
+    a.nb = ceil_div(n, d);
+    a.out = d_out;
+    a.status = d_status;
+    for (int j0 = 0; j0 < K; j0 += kMaxStreamsPerLaunch) {
+        a.K = std::min(K - j0, kMaxStreamsPerLaunch);
+        a.first_group = j0 == 0;
+        for (int j = 0; j < a.K; ++j) {
+            a.streams[j].words = words[j0 + j];
+            a.streams[j].num_words = num_words[j0 + j];
+            a.streams[j].offsets = offsets[j0 + j];
+        }
+        const cudaError_t e = launch_decode(a, accumulate, stream);
+        if (e != cudaSuccess) return QSGD_ERR_CUDA;
+    }
+    return QSGD_OK;
+}
+
+int qsgd_decode(const uint32_t* d_words, uint64_t num_words, const uint64_t* d_offsets, uint64_t n,
+                uint32_t d, uint32_t s, float* d_out, uint32_t* d_status, cudaStream_t stream) {
+    const uint32_t* w[1] = {d_words};
+    const uint64_t nw[1] = {num_words};
+    const uint64_t* o[1] = {d_offsets};
+    return decode_impl(w, nw, o, 1, n, d, s, d_out, d_status, stream, false);
+}
+
+int qsgd_decode_accumulate(const uint32_t* const* h_words, const uint64_t* h_num_words,
+                           const uint64_t* const* h_offsets, int K, uint64_t n, uint32_t d,
+                           uint32_t s, float* d_out, uint32_t* d_status, cudaStream_t stream) {
+    return decode_impl(h_words, h_num_words, h_offsets, K, n, d, s, d_out, d_status, stream, true);
+}
+
+const char* qsgd_error_string(int code) {
+    switch (code) {
+        case QSGD_OK: return "ok";
+        case QSGD_ERR_ARG: return "invalid argument";
+        case QSGD_ERR_CAPACITY: return "output capacity below qsgd_max_encoded_words";
+        case QSGD_ERR_CUDA: return "CUDA runtime error";
+        case QSGD_ERR_WORKSPACE: return "workspace below qsgd_encode_workspace_bytes";
+        default: return "unknown error";
+    }
+}
+
+const char* qsgd_version(void) { return "qsgd-b200 1.0 (wire format v1, sm_100a)"; }
+
+}  // extern "C"

@@ -1,0 +1,245 @@
+// Device building blocks of the QSGD codec (sm_100a).
+//
+// Method: "QSGD (Quantized Stochastic Gradient Descent) with Elias Coding" (AIMech
+// curated entry), definition paragraph and the claim "Elias coding communication
+// complexity tradeoff".  Random source: Philox4x32-10 (Salmon, Moraes, Dror, Shaw,
+// "Parallel Random Numbers: As Easy as 1, 2, 3", SC'11).  Integer code: Elias omega
+// (Elias 1975).  The library is compiled with -fmad=false and every rounding-relevant
+// fp32 operation below is an explicit _rn intrinsic.
+#pragma once
+
+#include <cstdint>
+
+#include "qsgd_limits.h"
+
+namespace qsgd {
+
+// ---------------------------------------------------------------------------
+// Philox4x32-10.  One call yields the random words of four consecutive
+// coordinates 4j..4j+3 (counter (lo32(j), hi32(j), 0, 0), key = the seed).
+// ---------------------------------------------------------------------------
+struct PhiloxKey {
+    uint32_t k0, k1;
+};
+
+__device__ __forceinline__ uint4 philox4x32_10(uint64_t j, PhiloxKey key) {
+    uint32_t c0 = static_cast<uint32_t>(j);
+    uint32_t c1 = static_cast<uint32_t>(j >> 32);
+    uint32_t c2 = 0u, c3 = 0u;
+    uint32_t k0 = key.k0, k1 = key.k1;
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+        // S-box: two 32x32 -> 64 products; the high halves are xored with the
+        // other counter words and the round key.
+        const uint32_t lo_a = 0xD2511F53u * c0;
+        const uint32_t hi_a = __umulhi(0xD2511F53u, c0);
+        const uint32_t lo_b = 0xCD9E8D57u * c2;
+        const uint32_t hi_b = __umulhi(0xCD9E8D57u, c2);
+        c0 = hi_b ^ c1 ^ k0;
+        c2 = hi_a ^ c3 ^ k1;
+        c1 = lo_b;
+        c3 = lo_a;
+        k0 += 0x9E3779B9u;  // Weyl key schedule (the bump after the last round is unused)
+        k1 += 0xBB67AE85u;
+    }
+    return make_uint4(c0, c1, c2, c3);
+}
+
+// ---------------------------------------------------------------------------
+// Quantiser of one coordinate (definition paragraph):
+//   t = |v| * (s/||v||), l = floor(t), p = t - l, k = l + [u < p], clamped to s.
+// floor(t) for 0 <= t < 2^23 is taken from the round-to-nearest integer
+// R = (t + 2^23) - 2^23, minus one when R > t; both steps are exact.
+// u = floor(r / 2^9) * 2^-23 is built exactly as (1 + u) - 1.
+// Returns k; the sign is handled by the caller.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t quantize_level(float v, float sinv, uint32_t r, uint32_t s) {
+    const float t = __fmul_rn(fabsf(v), sinv);
+    const float big = __fadd_rn(t, 8388608.0f);        // 2^23 + RN(t)
+    const float rn = __fsub_rn(big, 8388608.0f);       // RN(t), exact
+    const bool above = rn > t;
+    const float lf = above ? __fsub_rn(rn, 1.0f) : rn; // floor(t), exact
+    const float p = __fsub_rn(t, lf);                  // exact
+    const float u = __fsub_rn(__uint_as_float(0x3F800000u | (r >> 9)), 1.0f);
+    uint32_t k = (__float_as_uint(big) - 0x4B000000u) - (above ? 1u : 0u) + (u < p ? 1u : 0u);
+    return k < s ? k : s;
+}
+
+// ---------------------------------------------------------------------------
+// Elias omega code of N >= 1 (Elias 1975): start from "0"; while N > 1, put the
+// binary form of N in front and continue with bitlength(N) - 1.  Returned as a
+// right-aligned value read MSB-first, and its length in bits.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void omega_compute(uint64_t N, uint64_t& code, uint32_t& len) {
+    code = 0;
+    len = 1;
+    while (N > 1) {
+        const uint32_t b = 64u - static_cast<uint32_t>(__clzll(static_cast<long long>(N)));
+        code |= N << len;
+        len += b;
+        N = b - 1;
+    }
+}
+
+// Shared-memory table of omega codes for N < kOmegaTab: entry = (code << 8) | len.
+__device__ __forceinline__ void omega_table_fill(uint32_t* tab, int tid, int nthreads) {
+    for (int N = tid; N < kOmegaTab; N += nthreads) {
+        uint64_t code;
+        uint32_t len;
+        omega_compute(N == 0 ? 1 : N, code, len);
+        tab[N] = (static_cast<uint32_t>(code) << 8) | len;
+    }
+}
+
+__device__ __forceinline__ uint32_t omega_len(const uint32_t* tab, uint64_t N) {
+    if (N < kOmegaTab) return tab[N] & 0xFFu;
+    uint64_t code;
+    uint32_t len;
+    omega_compute(N, code, len);
+    return len;
+}
+
+__device__ __forceinline__ void omega_code(const uint32_t* tab, uint64_t N, uint64_t& code,
+                                           uint32_t& len) {
+    if (N < kOmegaTab) {
+        const uint32_t e = tab[N];
+        code = e >> 8;
+        len = e & 0xFFu;
+        return;
+    }
+    omega_compute(N, code, len);
+}
+
+// ---------------------------------------------------------------------------
+// MSB-first bit packing into a zero-filled shared word buffer.  A lane keeps up
+// to 31 pending bits; full words are OR-ed into the buffer (neighbouring lanes
+// may share a word, so every write is an atomic OR).
+// ---------------------------------------------------------------------------
+struct BitPacker {
+    uint64_t acc;    // pending bits, right-aligned
+    uint32_t nacc;   // number of pending bits (< 32 between calls)
+    uint32_t word;   // index of the word the pending bits start in
+    uint32_t* buf;
+    uint32_t limit;  // number of words in buf
+
+    __device__ __forceinline__ void start(uint32_t* b, uint32_t lim, uint64_t bitpos) {
+        buf = b;
+        limit = lim;
+        word = static_cast<uint32_t>(bitpos >> 5);
+        nacc = static_cast<uint32_t>(bitpos & 31u);  // leading bits owned by earlier writers
+        acc = 0;
+    }
+    __device__ __forceinline__ bool emit(uint32_t w) {
+        if (word >= limit) return false;
+        if (w) atomicOr(&buf[word], w);
+        ++word;
+        return true;
+    }
+    // Appends len <= 32 bits.
+    __device__ __forceinline__ bool put32(uint32_t code, uint32_t len) {
+        acc = (acc << len) | code;
+        nacc += len;
+        if (nacc >= 32) {
+            nacc -= 32;
+            return emit(static_cast<uint32_t>(acc >> nacc));
+        }
+        return true;
+    }
+    __device__ __forceinline__ bool put(uint64_t code, uint32_t len) {
+        bool ok = true;
+        if (len > 32) {
+            ok = put32(static_cast<uint32_t>(code >> 32), len - 32);
+            len = 32;
+        }
+        return put32(static_cast<uint32_t>(code), len) && ok;
+    }
+    __device__ __forceinline__ bool flush() {
+        if (nacc == 0) return true;
+        return emit(static_cast<uint32_t>(acc << (32 - nacc)));
+    }
+};
+
+// ---------------------------------------------------------------------------
+// Inter-CTA scan state (single-pass prefix scan with decoupled look-back,
+// Merrill & Garland 2016).  A descriptor packs [63:40] epoch, [39:38] state,
+// [37:0] value.  Descriptors from an earlier call (other epoch) read as "not
+// ready", so the workspace needs no clearing between calls.
+// ---------------------------------------------------------------------------
+constexpr uint64_t kStateAggregate = 1;
+constexpr uint64_t kStatePrefix = 2;
+constexpr uint64_t kValueMask = (uint64_t(1) << 38) - 1;
+constexpr uint32_t kEpochMask = 0xFFFFFFu;
+
+__device__ __forceinline__ uint64_t make_desc(uint32_t epoch, uint64_t state, uint64_t value) {
+    return (static_cast<uint64_t>(epoch & kEpochMask) << 40) | (state << 38) | (value & kValueMask);
+}
+__device__ __forceinline__ uint32_t desc_epoch(uint64_t d) { return static_cast<uint32_t>(d >> 40); }
+__device__ __forceinline__ uint64_t desc_state(uint64_t d) { return (d >> 38) & 3u; }
+__device__ __forceinline__ uint64_t desc_value(uint64_t d) { return d & kValueMask; }
+
+__device__ __forceinline__ void st_release(uint64_t* p, uint64_t v) {
+    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ uint64_t ld_acquire(const uint64_t* p) {
+    uint64_t v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ uint32_t ld_acquire32(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Control block at the start of the workspace.
+struct ScanControl {
+    uint32_t ticket;  // next tile to hand out
+    uint32_t done;    // CTAs that have finished
+    uint32_t epoch;   // call counter, advanced by the last CTA
+    uint32_t abort;   // set when a bounded wait ran out
+    uint32_t pad[12];
+};
+static_assert(sizeof(ScanControl) == 64, "control block is one 64-byte line");
+
+// Warp-cooperative look-back for tile `tile` (> 0).  All 32 lanes call it; every
+// lane returns the exclusive prefix.  Returns false (and leaves the prefix
+// undefined) when the bounded wait ran out or another tile aborted.
+__device__ __forceinline__ bool lookback(const uint64_t* desc, uint32_t tile, uint32_t epoch,
+                                         const uint32_t* abort_flag, uint64_t& exclusive) {
+    const int lane = threadIdx.x & 31;
+    uint64_t sum = 0;
+    int64_t window_end = static_cast<int64_t>(tile) - 1;  // highest predecessor in the window
+    uint32_t polls = 0;
+    while (window_end >= 0) {
+        const int64_t idx = window_end - lane;
+        uint64_t d = 0;
+        uint64_t st = kStatePrefix;  // lanes past tile 0 act as a zero prefix
+        uint64_t val = 0;
+        if (idx >= 0) {
+            d = ld_acquire(desc + idx);
+            st = (desc_epoch(d) == (epoch & kEpochMask)) ? desc_state(d) : 0;
+            val = desc_value(d);
+        }
+        const uint32_t not_ready = __ballot_sync(0xFFFFFFFFu, st == 0);
+        const uint32_t have_prefix = __ballot_sync(0xFFFFFFFFu, st == kStatePrefix);
+        // first lane (nearest predecessor) holding a prefix
+        const int first_p = have_prefix ? __ffs(have_prefix) - 1 : 32;
+        const uint32_t upto = first_p == 32 ? 0xFFFFFFFFu : ((2u << first_p) - 1u);
+        if (not_ready & upto) {
+            if (++polls > kMaxPolls) return false;
+            if ((polls & 63u) == 0 && ld_acquire32(abort_flag) != 0) return false;
+            __nanosleep(polls < 64 ? 32 : 256);
+            continue;
+        }
+        uint64_t contrib = (lane <= first_p) ? val : 0;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) contrib += __shfl_xor_sync(0xFFFFFFFFu, contrib, o);
+        sum += contrib;
+        if (first_p < 32) break;
+        window_end -= 32;
+    }
+    exclusive = sum;
+    return true;
+}
+
+}  // namespace qsgd

@@ -1,0 +1,90 @@
+"""The C-ABI library loads on the CPU and exports every entry point of include/qsgd.h.
+
+No compute call is made here: only host-side size queries and argument checks
+that return before any CUDA call.
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "qsgd.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^QSGD_API\s+[\w\s\*]+?\b(qsgd_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from quantized_gradient_compression_b200 import build
+
+    path = build.build()
+    return ctypes.CDLL(path)
+
+
+def test_header_declares_the_boundary():
+    names = declared_symbols()
+    for want in ["qsgd_encode", "qsgd_decode", "qsgd_decode_accumulate", "qsgd_max_encoded_words",
+                 "qsgd_encode_workspace_bytes", "qsgd_num_buckets", "qsgd_error_string"]:
+        assert want in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+
+
+def test_binding_exposes_same_names():
+    from quantized_gradient_compression_b200 import binding
+
+    for name in declared_symbols():
+        assert hasattr(binding, name), name
+        assert name in binding.EXPORTED
+
+
+def test_size_queries_match_oracle_bound(oracle_lib):
+    from quantized_gradient_compression_b200 import binding as B
+
+    for n, d, s in [(1, 1, 1), (7, 3, 2), (25_557_032, 512, 16), (60_192_808, 8192, 1),
+                    (65_536, 65_536, 256), (1 << 30, 512, 256), (1000, 7, 1 << 22)]:
+        assert B.qsgd_num_buckets(n, d) == (n + d - 1) // d
+        if n <= 100_000:
+            assert B.qsgd_max_encoded_words(n, d, s) == oracle_lib.capacity_words(n, d, s)
+        else:
+            nb = (n + d - 1) // d
+            bits = 32 * nb + n * (2 + oracle_lib.omega_len(s))
+            assert B.qsgd_max_encoded_words(n, d, s) == (bits + 31) // 32
+        assert B.qsgd_encode_workspace_bytes(n, d, s) >= 256
+
+
+def test_invalid_parameters_are_rejected_on_the_host():
+    from quantized_gradient_compression_b200 import binding as B
+
+    assert B.qsgd_max_encoded_words(10, 0, 4) == 0
+    assert B.qsgd_max_encoded_words(10, 4, 0) == 0
+    assert B.qsgd_max_encoded_words(10, 4, (1 << 22) + 1) == 0
+    # argument errors are detected before any CUDA call
+    assert B.qsgd_encode(0, 10, 0, 4, 0, 0, 0, 8, 0, 0, 8, 0) == B.QSGD_ERR_ARG
+    assert B.qsgd_encode(256, 10, 4, 4, 0, 256, 100, 256, 256, 1 << 20, 0, 0) == B.QSGD_ERR_ARG  # no status
+    assert B.qsgd_encode(256, 100, 4, 4, 0, 256, 1, 256, 256, 1 << 20, 256, 0) == B.QSGD_ERR_CAPACITY
+    assert B.qsgd_encode(256, 100, 4, 4, 0, 256, 1000, 256, 256, 1, 256, 0) == B.QSGD_ERR_WORKSPACE
+    assert B.qsgd_encode(256, 100, 4, 4, 0, 256, 1000, 257, 256, 1 << 20, 256, 0) == B.QSGD_ERR_ARG
+    assert B.qsgd_decode(256, 10, 256, 10, 4, 0, 256, 256, 0) == B.QSGD_ERR_ARG
+    assert B.qsgd_decode_accumulate([], [], [], 0, 10, 4, 4, 256, 256, 0) == B.QSGD_ERR_ARG
+    assert B.qsgd_error_string(B.QSGD_ERR_CAPACITY).startswith("output capacity")
+    assert "sm_100a" in B.qsgd_version()
+
+
+def test_library_is_sm100a_only():
+    from quantized_gradient_compression_b200 import build
+
+    flags = " ".join(build.NVCC_FLAGS)
+    assert "arch=compute_100a,code=sm_100a" in flags
+    assert "-fmad=false" in flags
+    assert "use_fast_math" not in flags

@@ -32,13 +32,13 @@ MUTANTS = {
     "round_to_nearest": ("float l = floorf(t);", "float l = roundf(t);"),
     "scale_inverted": ("float sinv = (float)s / norm;", "float sinv = norm / (float)s;"),
     "l1_norm": ("sum += (double)v[i] * (double)v[i];", "sum += fabs((double)v[i]);"),
-    "gap_origin_zero": ("int64_t prev = -1;\n        for (uint64_t i = 0; i < m && err == 0; ++i) {",
-                        "int64_t prev = 0;\n        for (uint64_t i = 0; i < m && err == 0; ++i) {"),
-    "gap_not_updated": ("prev = (int64_t)i;\n            uint32_t k", "uint32_t k"),
-    "sign_inverted": ("put_bit(words, cap_words, &pos, levels[i] < 0);",
-                      "put_bit(words, cap_words, &pos, levels[i] > 0);"),
-    "fields_swapped": ("err |= qo_omega_put(words, cap_words, &pos, gap);\n            err |= put_bit(words, cap_words, &pos, levels[i] < 0);\n            err |= qo_omega_put(words, cap_words, &pos, k);",
-                       "err |= qo_omega_put(words, cap_words, &pos, k);\n            err |= put_bit(words, cap_words, &pos, levels[i] < 0);\n            err |= qo_omega_put(words, cap_words, &pos, gap);"),
+    "gap_origin_zero": ("int64_t prev = -1;\n    for (uint64_t i = 0; i < m && err == 0; ++i) {",
+                        "int64_t prev = 0;\n    for (uint64_t i = 0; i < m && err == 0; ++i) {"),
+    "gap_not_updated": ("prev = (int64_t)i;\n        uint32_t k", "uint32_t k"),
+    "sign_inverted": ("put_bit(words, cap_words, pos, levels[i] < 0);",
+                      "put_bit(words, cap_words, pos, levels[i] > 0);"),
+    "fields_swapped": ("err |= qo_omega_put(words, cap_words, pos, gap);\n        err |= put_bit(words, cap_words, pos, levels[i] < 0);\n        err |= qo_omega_put(words, cap_words, pos, k);",
+                       "err |= qo_omega_put(words, cap_words, pos, k);\n        err |= put_bit(words, cap_words, pos, levels[i] < 0);\n        err |= qo_omega_put(words, cap_words, pos, gap);"),
     "bit_order_lsb_first": ("if (bit) words[w] |= (uint32_t)1u << (31 - (unsigned)(*pos % 32));",
                             "if (bit) words[w] |= (uint32_t)1u << ((unsigned)(*pos % 32));"),
     "decode_scale_inverted": ("float scale = norm / (float)s;", "float scale = (float)s / norm;"),
