@@ -45,8 +45,8 @@ uint64_t max_bits(uint64_t n, uint32_t d, uint32_t s) {
     return 32u * nb + n * per;
 }
 
-bool fast_eligible(const float* in, uint32_t d) {
-    return d >= kFastMinD && d <= kFastMaxD && d % 4 == 0 &&
+bool fast_eligible(const float* in, uint32_t d, uint32_t s) {
+    return d >= kFastMinD && d <= kFastMaxD && d % 4 == 0 && s <= kFastMaxS &&
            (reinterpret_cast<uintptr_t>(in) & 15u) == 0;
 }
 
@@ -55,11 +55,13 @@ bool fast_eligible(const float* in, uint32_t d) {
 WorkspaceLayout workspace_layout(uint64_t n, uint32_t d) {
     WorkspaceLayout L{};
     const uint64_t nb = n ? ceil_div(n, d) : 0;
+    // fast path: tiles of kWarps buckets; general path: tiles of whole buckets
     const uint64_t per_tile = std::min<uint64_t>(kWarps, general_buckets_per_tile(d));
     L.max_tiles = nb ? ceil_div(nb, per_tile) : 0;
     L.desc_off = 256;
     L.carry_off = L.desc_off + align256(8 * L.max_tiles);
-    L.norms_off = L.carry_off + align256(8 * L.max_tiles);
+    L.rp_off = L.carry_off + align256(8 * L.max_tiles);
+    L.norms_off = L.rp_off + align256(8 * L.max_tiles);
     L.total = L.norms_off + align256(8 * nb);
     return L;
 }
@@ -119,14 +121,15 @@ int qsgd_encode(const float* d_in, uint64_t n, uint32_t d, uint32_t s, uint64_t 
     a.ctrl = reinterpret_cast<ScanControl*>(ws);
     a.desc = reinterpret_cast<uint64_t*>(ws + L.desc_off);
     a.carry = reinterpret_cast<uint64_t*>(ws + L.carry_off);
+    a.round_prefix = reinterpret_cast<uint64_t*>(ws + L.rp_off);
     a.norms = reinterpret_cast<float2*>(ws + L.norms_off);
     a.nb = ceil_div(n, d);
     const uint32_t wl = 2u + omega_len_host(s);
-    const bool fast = fast_eligible(d_in, d);
+    const bool fast = fast_eligible(d_in, d, s);
     if (fast) {
-        a.buckets_per_tile = kWarps;
-        a.ntiles = ceil_div(a.nb, kWarps);
-        const uint64_t tile_bits = static_cast<uint64_t>(kWarps) * (32u + static_cast<uint64_t>(d) * wl);
+        a.buckets_per_tile = kFastWarps;  // one bucket per warp
+        a.ntiles = ceil_div(a.nb, kFastWarps);
+        const uint64_t tile_bits = static_cast<uint64_t>(kFastWarps) * (32u + static_cast<uint64_t>(d) * wl);
         a.smem_words = static_cast<uint32_t>(ceil_div(tile_bits, 32) + 2);
     } else {
         a.buckets_per_tile = general_buckets_per_tile(d);
@@ -138,7 +141,9 @@ int qsgd_encode(const float* d_in, uint64_t n, uint32_t d, uint32_t s, uint64_t 
         const uint64_t chunk_bits = 31u + static_cast<uint64_t>(kChunk) * wl + 44u + omega_len_host(s) + 32u * starts;
         a.smem_words = static_cast<uint32_t>(ceil_div(chunk_bits, 32) + 2);
     }
-    if ((kOmegaTab + static_cast<uint64_t>(a.smem_words)) * 4 > 200 * 1024) return QSGD_ERR_ARG;
+    const uint64_t smem_bytes = fast ? fast_smem_bytes(d, s, a.smem_words)
+                                     : (kOmegaTab + static_cast<uint64_t>(a.smem_words)) * 4;
+    if (smem_bytes > 200 * 1024) return QSGD_ERR_ARG;
     if (a.ntiles > L.max_tiles) return QSGD_ERR_WORKSPACE;
     const cudaError_t e = launch_encode(a, fast, stream);
     return e == cudaSuccess ? QSGD_OK : QSGD_ERR_CUDA;

@@ -8,10 +8,18 @@
 // "distributed data-parallel optimization" (same paragraph) sums the decoded
 // streams of its peers: out_i <- out_i + q^0_i + ... + q^{K-1}_i in stream order.
 //
-// Buckets are independent prefix-code streams located by the offsets header, so
-// every bucket is parsed by its own thread; every read is bounded by the
-// bucket's [offsets[b], offsets[b+1]) range and by the stream length.
+// Layout of the work: buckets are independent prefix-code streams located by the
+// offsets header, so each lane of a warp parses one bucket.  The decoded values of
+// a segment of kSeg coordinates of each of the warp's 32 buckets are scattered into
+// a shared-memory staging tile (zero-filled, or loaded from the output for
+// decode-accumulate) and the tile is written back with coalesced 16-byte stores.
+// A record is normally decoded with one lookup of its first 12 bits in a
+// shared-memory table of complete records; longer records take a bit-serial path.
+// Every read is bounded by the bucket's [offsets[b], offsets[b+1]) range and by
+// the stream length.
 #include <cuda_runtime.h>
+
+#include <algorithm>
 
 #include "../../include/qsgd.h"
 #include "qsgd_device.cuh"
@@ -20,117 +28,513 @@
 namespace qsgd {
 namespace {
 
-// MSB-first reader over [pos, end) of a word array of num_words words.
-struct BitReader {
+constexpr int kLutBits = 12;
+constexpr int kLut = 1 << kLutBits;
+
+// Record table entry for a 12-bit window: [4:0] record length (0: not complete in
+// 12 bits or k > s), [15:6] gap, [25:16] k, [31] sign.
+__device__ __forceinline__ bool omega_from_window(uint32_t w, int nbits, int& pos, uint32_t& value) {
+    uint32_t v = 1;
+    for (;;) {
+        if (pos >= nbits) return false;
+        const uint32_t bit = (w >> (nbits - 1 - pos)) & 1u;
+        ++pos;
+        if (bit == 0) {
+            value = v;
+            return true;
+        }
+        if (pos + static_cast<int>(v) > nbits) return false;
+        const uint32_t rest = (w >> (nbits - pos - v)) & ((1u << v) - 1u);
+        pos += v;
+        v = (1u << v) | rest;
+    }
+}
+
+__device__ void build_record_lut(uint32_t* lut, uint32_t s, int tid, int nthreads) {
+    for (int w = tid; w < kLut; w += nthreads) {
+        int pos = 0;
+        uint32_t gap = 0, k = 0, e = 0;
+        if (omega_from_window(static_cast<uint32_t>(w), kLutBits, pos, gap) && pos < kLutBits) {
+            const uint32_t sign = (static_cast<uint32_t>(w) >> (kLutBits - 1 - pos)) & 1u;
+            ++pos;
+            if (omega_from_window(static_cast<uint32_t>(w), kLutBits, pos, k) && k <= s && gap < 1024 &&
+                k < 1024)
+                e = static_cast<uint32_t>(pos) | (gap << 6) | (k << 16) | (sign << 31);
+        }
+        lut[w] = e;
+    }
+}
+
+// MSB-first reader of one bucket with a 64-bit cache.  `pos` is the bit position
+// of the cache's first unconsumed bit; bits at or past `end` are never used.
+struct Reader {
     const uint32_t* w;
     uint64_t num_words;
     uint64_t pos;
     uint64_t end;
-
-    __device__ __forceinline__ uint32_t peek32() const {
-        const uint64_t wi = pos >> 5;
-        const uint32_t sh = static_cast<uint32_t>(pos & 31u);
-        const uint32_t hi = wi < num_words ? __ldg(w + wi) : 0u;
-        const uint32_t lo = wi + 1 < num_words ? __ldg(w + wi + 1) : 0u;
-        return sh ? (hi << sh) | (lo >> (32 - sh)) : hi;
+    uint64_t cache;     // 64 stream bits starting at bit 32 * cword
+    uint64_t cword;     // word index of the cache's first word
+    __device__ __forceinline__ uint32_t word(uint64_t i) const { return i < num_words ? __ldg(w + i) : 0u; }
+    __device__ __forceinline__ void init(uint64_t p) {
+        pos = p;
+        cword = p >> 5;
+        cache = (static_cast<uint64_t>(word(cword)) << 32) | word(cword + 1);
     }
-    // Reads 1 <= nbits <= 32 bits; false if they pass `end`.
-    __device__ __forceinline__ bool read(uint32_t nbits, uint32_t& v) {
-        if (end - pos < nbits) return false;
-        v = peek32() >> (32 - nbits);
-        pos += nbits;
-        return true;
+    // next 32 bits at pos (zeros past the stream)
+    __device__ __forceinline__ uint32_t peek32() {
+        uint32_t off = static_cast<uint32_t>(pos - (cword << 5));
+        if (off >= 32) {  // advance the cache by one word
+            cache = (cache << 32) | word(cword + 2);
+            ++cword;
+            off -= 32;
+        }
+        return static_cast<uint32_t>((cache << off) >> 32);
     }
-    // Elias omega: a 0 ends the code; a 1 starts a group of (value + 1) bits whose
-    // value becomes the next length.  Values above 2^32 - 1 are rejected.
+    __device__ __forceinline__ uint64_t left() const { return end - pos; }
+    // bit-serial omega (any length up to 2^32 - 1)
     __device__ __forceinline__ bool omega(uint32_t& N) {
-        uint32_t value = 1;
+        uint32_t v = 1;
         for (;;) {
-            uint32_t bit;
-            if (!read(1, bit)) return false;
+            if (pos >= end) return false;
+            const uint32_t bit = peek32() >> 31;
+            ++pos;
             if (bit == 0) {
-                N = value;
+                N = v;
                 return true;
             }
-            if (value > 31) return false;
-            uint32_t rest;
-            if (!read(value, rest)) return false;
-            value = (1u << value) | rest;
+            if (v > 31 || left() < v) return false;
+            const uint32_t rest = peek32() >> (32 - v);
+            pos += v;
+            v = (1u << v) | rest;
         }
     }
 };
 
-template <bool kAccumulate>
-__global__ void __launch_bounds__(kDecodeBlock) decode_buckets(const __grid_constant__ DecodeArgs a) {
-    const uint64_t b = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (b >= a.nb) return;
-    const uint64_t base = b * a.d;
-    const uint32_t m = static_cast<uint32_t>(min(static_cast<uint64_t>(a.d), a.n - base));
-    float* out = a.out + base;
-    const float fs = __uint2float_rn(a.s);
-    if (kAccumulate && a.first_group) {
-        // out + (+0.0): a coordinate off every support turns -0.0 into +0.0, as the
-        // dense sum does; every other value is unchanged.
-        for (uint32_t i = 0; i < m; ++i) out[i] = __fadd_rn(out[i], 0.0f);
+// One decoded record: index within the bucket and signed level.
+struct Record {
+    uint32_t idx;   // bucket-local index; 0xFFFFFFFF when the bucket has no more records
+    uint32_t k;
+    uint32_t sign;
+};
+
+// Decodes the next record of `r`, or marks the end.  Returns false on a
+// malformed stream (the bucket is then finished).
+__device__ __forceinline__ bool next_record(Reader& r, const uint32_t* lut, uint32_t m, uint32_t s,
+                                            uint32_t& next, Record& rec) {
+    if (r.pos >= r.end) {
+        rec.idx = 0xFFFFFFFFu;
+        return true;
     }
-    for (int j = 0; j < a.K; ++j) {
-        const StreamRef st = a.streams[j];
-        const uint64_t begin = st.offsets[b];
-        const uint64_t end = st.offsets[b + 1];
-        bool bad = !(end >= begin && end - begin >= 32 && end <= st.num_words * 32);
-        uint32_t cur = 0;  // next coordinate not yet written (plain decode)
-        if (!bad) {
-            BitReader br{st.words, st.num_words, begin, end};
-            uint32_t nbits = 0;
-            br.read(32, nbits);
-            const float norm = __uint_as_float(nbits);
-            if (nbits == 0) {
-                bad = br.pos != end;
-            } else if (!(isfinite(norm) && norm > 0.f)) {
+    const uint32_t w = r.peek32();
+    const uint32_t e = lut[w >> (32 - kLutBits)];
+    const uint32_t len = e & 31u;
+    uint32_t gap, k, sign;
+    if (len != 0 && len <= r.left()) {
+        r.pos += len;
+        gap = (e >> 6) & 1023u;
+        k = (e >> 16) & 1023u;
+        sign = e >> 31;
+    } else {
+        if (!r.omega(gap)) return false;
+        if (r.pos >= r.end) return false;
+        sign = r.peek32() >> 31;
+        ++r.pos;
+        if (!r.omega(k) || k > s) return false;
+    }
+    if (static_cast<uint64_t>(next) + gap - 1 >= m) return false;
+    rec.idx = next + gap - 1;
+    rec.k = k;
+    rec.sign = sign;
+    next = rec.idx + 1;
+    return true;
+}
+
+constexpr int kSeg = 64;                 // coordinates per bucket per staging round
+constexpr int kStride = kSeg + 4;        // padded row (floats) of the staging tile
+constexpr int kDecWarps = kDecodeBlock / 32;
+
+// Per-lane state of one stream of one bucket between staging rounds (24 bytes):
+// reader position, next free index, the pending record (index, level | sign << 30
+// | malformed << 31) and the bucket's scale norm/s.
+struct LaneStream {
+    uint64_t pos;
+    uint32_t next;
+    uint32_t idx;
+    uint32_t kflags;
+    float scale;
+};
+static_assert(sizeof(LaneStream) == 24, "compact stream state");
+
+__device__ __forceinline__ Record pending(const LaneStream& ls) {
+    return Record{ls.idx, ls.kflags & 0x3FFFFFFFu, (ls.kflags >> 30) & 1u};
+}
+__device__ __forceinline__ void set_pending(LaneStream& ls, const Record& r, bool bad) {
+    ls.idx = bad ? 0xFFFFFFFFu : r.idx;
+    ls.kflags = (r.k & 0x3FFFFFFFu) | (r.sign << 30) | (bad ? 0x80000000u : 0u);
+}
+
+template <bool kAccumulate>
+__global__ void __launch_bounds__(kDecodeBlock) decode_warp(const __grid_constant__ DecodeArgs a) {
+    extern __shared__ __align__(16) uint32_t smem[];
+    uint32_t* lut = smem;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    float* stage = reinterpret_cast<float*>(smem + kLut) + warp * 32 * kStride;
+    LaneStream* lstate = reinterpret_cast<LaneStream*>(smem + kLut + kDecWarps * 32 * kStride) +
+                         (warp * 32 + lane) * a.K;
+    build_record_lut(lut, a.s, tid, kDecodeBlock);
+    __syncthreads();
+
+    const uint64_t ngroups = (a.nb + 31) / 32;
+    const uint64_t gwarps = static_cast<uint64_t>(gridDim.x) * kDecWarps;
+    for (uint64_t g = static_cast<uint64_t>(blockIdx.x) * kDecWarps + warp; g < ngroups; g += gwarps) {
+        const uint64_t b = g * 32 + lane;  // this lane's bucket
+        const bool live = b < a.nb;
+        const uint64_t base = b * a.d;
+        const uint32_t m = live ? static_cast<uint32_t>(min(static_cast<uint64_t>(a.d), a.n - base)) : 0u;
+        bool any_bad = false;
+
+        // open every stream of this lane's bucket: header checks and the norm
+        for (int j = 0; j < a.K; ++j) {
+            LaneStream ls{0, 0, 0xFFFFFFFFu, 0, 0.f};
+            Record rec{0xFFFFFFFFu, 0, 0};
+            bool bad = false;
+            if (live) {
+                const StreamRef st = a.streams[j];
+                const uint64_t begin = st.offsets[b];
+                const uint64_t end = st.offsets[b + 1];
+                if (!(end >= begin && end - begin >= 32 && end <= st.num_words * 32)) {
+                    bad = true;
+                } else {
+                    Reader r{st.words, st.num_words, 0, end, 0, 0};
+                    r.init(begin);
+                    const uint32_t nbits = r.peek32();
+                    r.pos += 32;
+                    const float norm = __uint_as_float(nbits);
+                    if (nbits == 0) {
+                        bad = r.pos != end;
+                    } else if (!(isfinite(norm) && norm > 0.f)) {
+                        bad = true;
+                    } else {
+                        ls.scale = __fdiv_rn(norm, __uint2float_rn(a.s));
+                        bad = !next_record(r, lut, m, a.s, ls.next, rec);
+                    }
+                    ls.pos = r.pos;
+                }
+            }
+            set_pending(ls, rec, bad);
+            any_bad |= bad;
+            lstate[j] = ls;
+        }
+
+        for (uint32_t lo = 0; lo < a.d; lo += kSeg) {
+            // --- fill the staging tile: zeros, or the current output ----------
+            if (kAccumulate) {
+                for (int r = 0; r < 32; ++r) {
+                    const uint64_t bb = g * 32 + r;
+                    if (bb >= a.nb) break;
+                    const uint32_t mm = static_cast<uint32_t>(min(static_cast<uint64_t>(a.d), a.n - bb * a.d));
+                    for (uint32_t c = lane; c < kSeg; c += 32) {
+                        const uint32_t i = lo + c;
+                        float v = 0.f;
+                        if (i < mm) {
+                            v = a.out[bb * a.d + i];
+                            if (a.first_group) v = __fadd_rn(v, 0.0f);  // -0.0 + (+0.0) = +0.0
+                        }
+                        stage[r * kStride + c] = v;
+                    }
+                }
+            } else {
+                for (int q = lane; q < 32 * kStride / 4; q += 32)
+                    reinterpret_cast<float4*>(stage)[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+            __syncwarp();
+
+            // --- scatter this segment's records of every stream, in order ------
+            const uint32_t hi = lo + kSeg;
+            float* row = stage + lane * kStride;
+            for (int j = 0; j < a.K; ++j) {
+                LaneStream ls = lstate[j];
+                if (ls.idx < hi) {
+                    const StreamRef st = a.streams[j];
+                    Reader r{st.words, st.num_words, 0, st.offsets[b + 1], 0, 0};
+                    r.init(ls.pos);
+                    Record rec = pending(ls);
+                    bool bad = false;
+                    while (rec.idx < hi) {
+                        float val = __fmul_rn(ls.scale, __uint2float_rn(rec.k));
+                        if (rec.sign) val = -val;
+                        float* dst = row + (rec.idx - lo);
+                        *dst = kAccumulate ? __fadd_rn(*dst, val) : val;
+                        if (!next_record(r, lut, m, a.s, ls.next, rec)) {
+                            bad = true;
+                            break;
+                        }
+                    }
+                    ls.pos = r.pos;
+                    set_pending(ls, rec, bad);
+                    any_bad |= bad;
+                    lstate[j] = ls;
+                }
+            }
+            __syncwarp();
+
+            // --- write the tile back: row r is bucket g*32 + r -----------------
+            const uint32_t seg_len = min(static_cast<uint32_t>(kSeg), a.d - lo);
+            if ((a.d & 3u) == 0 && (reinterpret_cast<uintptr_t>(a.out) & 15u) == 0) {
+                // 16-byte stores: kSeg/4 per row
+                constexpr int kVec = kSeg / 4;
+                for (int q = lane; q < 32 * kVec; q += 32) {
+                    const int r = q / kVec, c4 = (q % kVec) * 4;
+                    const uint64_t bb = g * 32 + r;
+                    if (bb >= a.nb || static_cast<uint32_t>(c4) >= seg_len) continue;
+                    const uint32_t mm = static_cast<uint32_t>(min(static_cast<uint64_t>(a.d), a.n - bb * a.d));
+                    const uint32_t i = lo + c4;
+                    if (i + 4 <= mm) {
+                        *reinterpret_cast<float4*>(a.out + bb * a.d + i) =
+                            *reinterpret_cast<const float4*>(stage + r * kStride + c4);
+                    } else {
+                        for (int t = 0; t < 4; ++t)
+                            if (i + t < mm) a.out[bb * a.d + i + t] = stage[r * kStride + c4 + t];
+                    }
+                }
+            } else {
+                for (int r = 0; r < 32; ++r) {
+                    const uint64_t bb = g * 32 + r;
+                    if (bb >= a.nb) break;
+                    const uint32_t mm = static_cast<uint32_t>(min(static_cast<uint64_t>(a.d), a.n - bb * a.d));
+                    for (uint32_t c = lane; c < seg_len; c += 32)
+                        if (lo + c < mm) a.out[bb * a.d + lo + c] = stage[r * kStride + c];
+                }
+            }
+            __syncwarp();
+        }
+        if (any_bad) atomicOr(a.status, QSGD_ST_BAD_STREAM);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Fast decoder: d % 4 == 0, d <= kFastDecodeMaxD, s < 1024, 16-byte aligned output,
+// one stream.  Bucket-relative 32-bit reader state: `wp` points at the word that
+// holds the cache's first bit, (hi, lo) are the two cached words, `nx` the word
+// after them, `off` < 32 the bit offset into hi, `left` the bits of the bucket
+// still unread.
+// ---------------------------------------------------------------------------
+struct FastReader {
+    const uint32_t* wp;
+    const uint32_t* wend;  // one past the last word of the stream
+    uint32_t hi, lo, nx;
+    uint32_t off;
+    uint32_t left;
+    __device__ __forceinline__ uint32_t ld(const uint32_t* p) const { return p < wend ? __ldg(p) : 0u; }
+    __device__ __forceinline__ void init(const uint32_t* words, uint64_t num_words, uint64_t begin, uint32_t nbits) {
+        wend = words + num_words;
+        wp = words + (begin >> 5);
+        off = static_cast<uint32_t>(begin & 31u);
+        hi = ld(wp);
+        lo = ld(wp + 1);
+        nx = ld(wp + 2);
+        left = nbits;
+    }
+    __device__ __forceinline__ uint32_t peek() const { return __funnelshift_l(lo, hi, off); }
+    // consumes n <= 32 bits (the caller checked n <= left)
+    __device__ __forceinline__ void skip(uint32_t n) {
+        off += n;
+        left -= n;
+        if (off >= 32) {
+            off -= 32;
+            hi = lo;
+            lo = nx;
+            ++wp;
+            nx = ld(wp + 2);
+        }
+    }
+    __device__ __forceinline__ bool omega(uint32_t& N) {
+        uint32_t v = 1;
+        for (;;) {
+            if (left == 0) return false;
+            const uint32_t bit = peek() >> 31;
+            skip(1);
+            if (bit == 0) {
+                N = v;
+                return true;
+            }
+            if (v > 31 || left < v) return false;
+            const uint32_t rest = peek() >> (32 - v);
+            skip(v);
+            v = (1u << v) | rest;
+        }
+    }
+};
+
+constexpr uint32_t kFastDecodeMaxD = 4096;
+
+// Next record: its index (0xFFFFFFFF at the end of the bucket) and value bits.
+// Returns false on a malformed record.
+__device__ __forceinline__ bool fast_next(FastReader& r, const uint32_t* lut, uint32_t m, uint32_t s,
+                                          float scale, uint32_t& next, uint32_t& idx, uint32_t& vbits) {
+    if (r.left == 0) {
+        idx = 0xFFFFFFFFu;
+        return true;
+    }
+    const uint32_t e = lut[r.peek() >> (32 - kLutBits)];
+    const uint32_t len = e & 31u;
+    uint32_t gap, k, sign;
+    if (len != 0 && len <= r.left) {
+        r.skip(len);
+        gap = (e >> 6) & 1023u;
+        k = (e >> 16) & 1023u;
+        sign = e >> 31;
+    } else {
+        if (!r.omega(gap) || r.left == 0) return false;
+        sign = r.peek() >> 31;
+        r.skip(1);
+        if (!r.omega(k) || k > s) return false;
+    }
+    idx = next + gap - 1;
+    if (gap > m || idx >= m) return false;
+    next = idx + 1;
+    vbits = __float_as_uint(__fmul_rn(scale, __uint2float_rn(k))) | (sign << 31);
+    return true;
+}
+
+__global__ void __launch_bounds__(kDecodeBlock) decode_fast(const __grid_constant__ DecodeArgs a) {
+    extern __shared__ __align__(16) uint32_t smem[];
+    uint32_t* lut = smem;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    float* stage = reinterpret_cast<float*>(smem + kLut) + warp * 32 * kStride;
+    build_record_lut(lut, a.s, tid, kDecodeBlock);
+    __syncthreads();
+    const StreamRef st = a.streams[0];
+    const float fs = __uint2float_rn(a.s);
+    const uint32_t d = a.d;
+    const uint64_t ngroups = (a.nb + 31) / 32;
+    const uint64_t gwarps = static_cast<uint64_t>(gridDim.x) * kDecWarps;
+    for (uint64_t g = static_cast<uint64_t>(blockIdx.x) * kDecWarps + warp; g < ngroups; g += gwarps) {
+        const uint64_t b = g * 32 + lane;
+        const bool live = b < a.nb;
+        const uint32_t m = live ? static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - b * d)) : 0u;
+        bool bad = false;
+        FastReader r;
+        r.left = 0;
+        float scale = 0.f;
+        if (live) {
+            const uint64_t begin = st.offsets[b];
+            const uint64_t end = st.offsets[b + 1];
+            if (!(end >= begin && end - begin >= 32 && end <= st.num_words * 32 && end - begin < (1ull << 31))) {
                 bad = true;
             } else {
-                const float scale = __fdiv_rn(norm, fs);
-                uint32_t next = 0;  // index of the previous record + 1
-                while (br.pos < end) {
-                    uint32_t gap, sign, k;
-                    if (!br.omega(gap) || static_cast<uint64_t>(next) + gap - 1 >= m) {
-                        bad = true;
-                        break;
-                    }
-                    const uint32_t idx = next + gap - 1;
-                    if (!br.read(1, sign) || !br.omega(k) || k > a.s) {
-                        bad = true;
-                        break;
-                    }
-                    float val = __fmul_rn(scale, __uint2float_rn(k));
-                    if (sign) val = -val;
-                    if (kAccumulate) {
-                        out[idx] = __fadd_rn(out[idx], val);
-                    } else {
-                        for (; cur < idx; ++cur) out[cur] = 0.0f;
-                        out[idx] = val;
-                        cur = idx + 1;
-                    }
-                    next = idx + 1;
+                r.init(st.words, st.num_words, begin, static_cast<uint32_t>(end - begin));
+                const uint32_t nbits = r.peek();
+                r.skip(32);
+                const float norm = __uint_as_float(nbits);
+                if (nbits == 0) {
+                    bad = r.left != 0;
+                    r.left = 0;
+                } else if (!(isfinite(norm) && norm > 0.f)) {
+                    bad = true;
+                    r.left = 0;
+                } else {
+                    scale = __fdiv_rn(norm, fs);
                 }
             }
         }
+        uint32_t next = 0, pidx = 0xFFFFFFFFu, pval = 0;
+        if (!bad && !fast_next(r, lut, m, a.s, scale, next, pidx, pval)) {
+            bad = true;
+            pidx = 0xFFFFFFFFu;
+        }
+        float* row = stage + lane * kStride;
+        // write-back geometry: iteration i stores row 2i + (lane >> 4), columns 4 (lane & 15)..+3
+        const uint32_t wrow = static_cast<uint32_t>(lane >> 4), wcol = static_cast<uint32_t>(lane & 15) * 4;
+        const bool full_group = (g + 1) * 32 <= a.nb && (g + 1) * 32 * static_cast<uint64_t>(d) <= a.n;
+        for (uint32_t lo = 0; lo < d; lo += kSeg) {
+            for (int q = lane; q < 32 * kStride / 4; q += 32)
+                reinterpret_cast<float4*>(stage)[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+            __syncwarp();
+            const uint32_t hi = lo + kSeg;
+            while (pidx < hi) {
+                row[pidx - lo] = __uint_as_float(pval);
+                if (!fast_next(r, lut, m, a.s, scale, next, pidx, pval)) {
+                    bad = true;
+                    pidx = 0xFFFFFFFFu;
+                }
+            }
+            __syncwarp();
+            const uint32_t seg_len = min(static_cast<uint32_t>(kSeg), d - lo);
+            if (full_group && seg_len == kSeg) {
+                float* dst = a.out + (g * 32 + wrow) * d + lo + wcol;
+                const float* src = stage + wrow * kStride + wcol;
+#pragma unroll 4
+                for (int i = 0; i < 16; ++i) {
+                    *reinterpret_cast<float4*>(dst) = *reinterpret_cast<const float4*>(src);
+                    dst += 2 * static_cast<uint64_t>(d);
+                    src += 2 * kStride;
+                }
+            } else {
+                for (int rr = 0; rr < 32; ++rr) {
+                    const uint64_t bb = g * 32 + rr;
+                    if (bb >= a.nb) break;
+                    const uint32_t mm = static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - bb * d));
+                    for (uint32_t c = lane; c < seg_len; c += 32)
+                        if (lo + c < mm) a.out[bb * d + lo + c] = stage[rr * kStride + c];
+                }
+            }
+            __syncwarp();
+        }
         if (bad) atomicOr(a.status, QSGD_ST_BAD_STREAM);
-        if (!kAccumulate)
-            for (; cur < m; ++cur) out[cur] = 0.0f;
     }
+}
+
+cudaError_t launch_fast_decode(const DecodeArgs& a, cudaStream_t stream) {
+    const size_t smem = kLut * sizeof(uint32_t) + static_cast<size_t>(kDecWarps) * 32 * kStride * sizeof(float);
+    static bool attr_set[64] = {};
+    int dev = 0, sms = 0, per_sm = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr_set[dev]) {
+        cudaFuncSetAttribute(decode_fast, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+        attr_set[dev] = true;
+    }
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_fast, kDecodeBlock, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    const uint64_t groups = (a.nb + 31) / 32;
+    const uint64_t blocks = std::min<uint64_t>((groups + kDecWarps - 1) / kDecWarps, static_cast<uint64_t>(sms) * per_sm);
+    decode_fast<<<static_cast<unsigned>(blocks), kDecodeBlock, smem, stream>>>(a);
+    return cudaGetLastError();
+}
+
+template <bool kAccumulate>
+cudaError_t launch(const DecodeArgs& a, cudaStream_t stream) {
+    const size_t smem = kLut * sizeof(uint32_t) + static_cast<size_t>(kDecWarps) * 32 * kStride * sizeof(float) +
+                        static_cast<size_t>(kDecodeBlock) * a.K * sizeof(LaneStream);
+    static bool attr_set[64] = {};
+    int dev = 0, sms = 0, per_sm = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr_set[dev]) {
+        cudaFuncSetAttribute(decode_warp<kAccumulate>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+        attr_set[dev] = true;
+    }
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_warp<kAccumulate>,
+                                                                  kDecodeBlock, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    const uint64_t groups = (a.nb + 31) / 32;
+    const uint64_t blocks = std::min<uint64_t>((groups + kDecWarps - 1) / kDecWarps,
+                                               static_cast<uint64_t>(sms) * per_sm);
+    decode_warp<kAccumulate><<<static_cast<unsigned>(blocks), kDecodeBlock, smem, stream>>>(a);
+    return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_decode(const DecodeArgs& a, bool accumulate, cudaStream_t stream) {
-    const uint64_t blocks = (a.nb + kDecodeBlock - 1) / kDecodeBlock;
-    if (blocks == 0) return cudaSuccess;
-    if (accumulate)
-        decode_buckets<true><<<static_cast<unsigned>(blocks), kDecodeBlock, 0, stream>>>(a);
-    else
-        decode_buckets<false><<<static_cast<unsigned>(blocks), kDecodeBlock, 0, stream>>>(a);
-    return cudaGetLastError();
+    if (a.nb == 0) return cudaSuccess;
+    if (!accumulate && a.K == 1 && a.d % 4 == 0 && a.d <= kFastDecodeMaxD && a.s < 1024 &&
+        (reinterpret_cast<uintptr_t>(a.out) & 15u) == 0 && kSeg == 64)
+        return launch_fast_decode(a, stream);
+    return accumulate ? launch<true>(a, stream) : launch<false>(a, stream);
 }
 
 }  // namespace qsgd

@@ -26,21 +26,19 @@ __device__ __forceinline__ uint4 philox4x32_10(uint64_t j, PhiloxKey key) {
     uint32_t c0 = static_cast<uint32_t>(j);
     uint32_t c1 = static_cast<uint32_t>(j >> 32);
     uint32_t c2 = 0u, c3 = 0u;
-    uint32_t k0 = key.k0, k1 = key.k1;
 #pragma unroll
     for (int r = 0; r < 10; ++r) {
+        // round key: the seed advanced r times by the Weyl constants
+        const uint32_t k0 = key.k0 + static_cast<uint32_t>(r) * 0x9E3779B9u;
+        const uint32_t k1 = key.k1 + static_cast<uint32_t>(r) * 0xBB67AE85u;
         // S-box: two 32x32 -> 64 products; the high halves are xored with the
         // other counter words and the round key.
-        const uint32_t lo_a = 0xD2511F53u * c0;
-        const uint32_t hi_a = __umulhi(0xD2511F53u, c0);
-        const uint32_t lo_b = 0xCD9E8D57u * c2;
-        const uint32_t hi_b = __umulhi(0xCD9E8D57u, c2);
-        c0 = hi_b ^ c1 ^ k0;
-        c2 = hi_a ^ c3 ^ k1;
-        c1 = lo_b;
-        c3 = lo_a;
-        k0 += 0x9E3779B9u;  // Weyl key schedule (the bump after the last round is unused)
-        k1 += 0xBB67AE85u;
+        const uint64_t pa = static_cast<uint64_t>(c0) * 0xD2511F53u;
+        const uint64_t pb = static_cast<uint64_t>(c2) * 0xCD9E8D57u;
+        c0 = static_cast<uint32_t>(pb >> 32) ^ c1 ^ k0;
+        c2 = static_cast<uint32_t>(pa >> 32) ^ c3 ^ k1;
+        c1 = static_cast<uint32_t>(pb);
+        c3 = static_cast<uint32_t>(pa);
     }
     return make_uint4(c0, c1, c2, c3);
 }
@@ -48,20 +46,16 @@ __device__ __forceinline__ uint4 philox4x32_10(uint64_t j, PhiloxKey key) {
 // ---------------------------------------------------------------------------
 // Quantiser of one coordinate (definition paragraph):
 //   t = |v| * (s/||v||), l = floor(t), p = t - l, k = l + [u < p], clamped to s.
-// floor(t) for 0 <= t < 2^23 is taken from the round-to-nearest integer
-// R = (t + 2^23) - 2^23, minus one when R > t; both steps are exact.
+// floor(t) is a round-down conversion to integer (t < 2^23, every step exact);
 // u = floor(r / 2^9) * 2^-23 is built exactly as (1 + u) - 1.
 // Returns k; the sign is handled by the caller.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t quantize_level(float v, float sinv, uint32_t r, uint32_t s) {
     const float t = __fmul_rn(fabsf(v), sinv);
-    const float big = __fadd_rn(t, 8388608.0f);        // 2^23 + RN(t)
-    const float rn = __fsub_rn(big, 8388608.0f);       // RN(t), exact
-    const bool above = rn > t;
-    const float lf = above ? __fsub_rn(rn, 1.0f) : rn; // floor(t), exact
-    const float p = __fsub_rn(t, lf);                  // exact
+    const uint32_t l = __float2uint_rd(t);             // floor(t), exact for 0 <= t < 2^23
+    const float p = __fsub_rn(t, __uint2float_rn(l));  // exact
     const float u = __fsub_rn(__uint_as_float(0x3F800000u | (r >> 9)), 1.0f);
-    uint32_t k = (__float_as_uint(big) - 0x4B000000u) - (above ? 1u : 0u) + (u < p ? 1u : 0u);
+    const uint32_t k = l + (u < p ? 1u : 0u);
     return k < s ? k : s;
 }
 
@@ -81,15 +75,77 @@ __device__ __forceinline__ void omega_compute(uint64_t N, uint64_t& code, uint32
     }
 }
 
-// Shared-memory table of omega codes for N < kOmegaTab: entry = (code << 8) | len.
-__device__ __forceinline__ void omega_table_fill(uint32_t* tab, int tid, int nthreads) {
-    for (int N = tid; N < kOmegaTab; N += nthreads) {
-        uint64_t code;
-        uint32_t len;
-        omega_compute(N == 0 ? 1 : N, code, len);
-        tab[N] = (static_cast<uint32_t>(code) << 8) | len;
+// Table of omega codes for N < kOmegaTab: entry = (code << 8) | len (entry 0 is
+// unused).  Built at compile time by the same rule as omega_compute.
+struct OmegaTable {
+    uint32_t v[kOmegaTab];
+};
+constexpr OmegaTable make_omega_table() {
+    OmegaTable t{};
+    for (int N = 0; N < kOmegaTab; ++N) {
+        uint64_t n = N ? static_cast<uint64_t>(N) : 1u;
+        uint64_t code = 0;
+        uint32_t len = 1;
+        while (n > 1) {
+            uint32_t b = 0;
+            for (uint64_t x = n; x; x >>= 1) ++b;
+            code |= n << len;
+            len += b;
+            n = b - 1;
+        }
+        t.v[N] = (static_cast<uint32_t>(code) << 8) | len;
     }
+    return t;
 }
+__device__ const OmegaTable kOmegaTableGlobal = make_omega_table();
+
+// Copies the table into shared memory (16-byte loads).
+__device__ __forceinline__ void omega_table_fill(uint32_t* tab, int tid, int nthreads) {
+    const uint4* src = reinterpret_cast<const uint4*>(kOmegaTableGlobal.v);
+    uint4* dst = reinterpret_cast<uint4*>(tab);
+    for (int i = tid; i < kOmegaTab / 4; i += nthreads) dst[i] = src[i];
+}
+
+// Whole records omega(gap) | sign | omega(k) for gap < 64 and k < 16, indexed by
+// gap << 5 | k << 1 | sign: entry = code << 5 | length (length <= 20 bits).
+struct RecordTable {
+    uint32_t v[kRecordTab];
+};
+constexpr RecordTable make_record_table() {
+    RecordTable t{};
+    const OmegaTable om = make_omega_table();
+    for (uint32_t gap = 1; gap < 64; ++gap)
+        for (uint32_t k = 1; k < 16; ++k)
+            for (uint32_t sign = 0; sign < 2; ++sign) {
+                const uint32_t ge = om.v[gap], ke = om.v[k];
+                const uint32_t kl = ke & 0xFFu;
+                const uint32_t code = ((((ge >> 8) << 1) | sign) << kl) | (ke >> 8);
+                const uint32_t len = (ge & 0xFFu) + 1u + kl;
+                t.v[(gap << 5) | (k << 1) | sign] = (code << 5) | len;
+            }
+    return t;
+}
+__device__ const RecordTable kRecordTableGlobal = make_record_table();
+
+__device__ __forceinline__ void record_table_fill(uint32_t* tab, int tid, int nthreads) {
+    const uint4* src = reinterpret_cast<const uint4*>(kRecordTableGlobal.v);
+    uint4* dst = reinterpret_cast<uint4*>(tab);
+    for (int i = tid; i < kRecordTab / 4; i += nthreads) dst[i] = src[i];
+}
+
+// Omega code of N >= 1 from the global table (N < kOmegaTab) or computed.
+__device__ __forceinline__ void omega_code_global(uint64_t N, uint64_t& code, uint32_t& len) {
+    if (N < kOmegaTab) {
+        const uint32_t e = __ldg(&kOmegaTableGlobal.v[N]);
+        code = e >> 8;
+        len = e & 0xFFu;
+        return;
+    }
+    omega_compute(N, code, len);
+}
+
+// N < kOmegaTab known by the caller
+__device__ __forceinline__ uint32_t omega_len_fast(const uint32_t* tab, uint32_t N) { return tab[N] & 0xFFu; }
 
 __device__ __forceinline__ uint32_t omega_len(const uint32_t* tab, uint64_t N) {
     if (N < kOmegaTab) return tab[N] & 0xFFu;
@@ -160,6 +216,35 @@ struct BitPacker {
 };
 
 // ---------------------------------------------------------------------------
+// MSB-first packing of one lane's records into its private strip of shared
+// memory (word j at base[32 j]; the strips of a warp interleave, so the lanes'
+// stores fall in distinct banks).  32-bit state: the partial word and its fill.
+// ---------------------------------------------------------------------------
+struct LanePacker {
+    uint32_t* base;
+    uint32_t cur;   // partial word, filled from the top
+    uint32_t used;  // bits in cur (0..31)
+    uint32_t nw;    // words stored
+    // Appends the len (1..32) low bits of code.
+    __device__ __forceinline__ void put(uint32_t code, uint32_t len) {
+        const uint32_t x = code << (32u - len);  // left-aligned record
+        const uint32_t filled = cur | (x >> used);
+        const uint32_t tot = used + len;
+        const bool full = tot >= 32u;
+        if (full) base[32u * nw] = filled;
+        nw += full ? 1u : 0u;
+        // leftover bits of the record start the next word (none when tot == 32)
+        const uint32_t rest = (tot > 32u) ? (x << (32u - used)) : 0u;
+        cur = full ? rest : filled;
+        used = tot & 31u;
+    }
+    __device__ __forceinline__ void finish() {
+        if (used) base[32u * nw] = cur;
+    }
+    __device__ __forceinline__ uint32_t bits() const { return 32u * nw + used; }
+};
+
+// ---------------------------------------------------------------------------
 // Inter-CTA scan state (single-pass prefix scan with decoupled look-back,
 // Merrill & Garland 2016).  A descriptor packs [63:40] epoch, [39:38] state,
 // [37:0] value.  Descriptors from an earlier call (other epoch) read as "not
@@ -183,6 +268,11 @@ __device__ __forceinline__ void st_release(uint64_t* p, uint64_t v) {
 __device__ __forceinline__ uint64_t ld_acquire(const uint64_t* p) {
     uint64_t v;
     asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ ulonglong2 ld_relaxed_v2(const uint64_t* p) {
+    ulonglong2 v;
+    asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(v.x), "=l"(v.y) : "l"(p) : "memory");
     return v;
 }
 __device__ __forceinline__ uint32_t ld_acquire32(const uint32_t* p) {

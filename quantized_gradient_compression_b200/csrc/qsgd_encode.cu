@@ -90,29 +90,6 @@ __device__ __forceinline__ float pow2_scale(float maxabs, float& unscale) {
     return __uint_as_float((254u - e) << 23);  // 2^(127-e)
 }
 
-// Waits (bounded) for the tail word of tile `tile - 1`.
-__device__ __forceinline__ bool wait_carry(const EncodeArgs& a, uint32_t tile, uint32_t epoch,
-                                           uint32_t& word) {
-    const uint64_t* slot = a.carry + (tile - 1);
-    for (uint32_t polls = 0;; ++polls) {
-        const uint64_t c = ld_acquire(slot);
-        if ((c >> 63) != 0 && static_cast<uint32_t>((c >> 32) & kEpochMask) == (epoch & kEpochMask)) {
-            word = static_cast<uint32_t>(c);
-            return true;
-        }
-        if (polls > kMaxPolls) return false;
-        if ((polls & 63u) == 63u && ld_acquire32(&a.ctrl->abort) != 0) return false;
-        __nanosleep(polls < 64 ? 32 : 256);
-    }
-}
-
-__device__ __forceinline__ void publish_carry(const EncodeArgs& a, uint32_t tile, uint32_t epoch,
-                                              uint32_t word) {
-    // [63] present, [55:32] epoch, [31:0] the tail word (a zero-filled slot is never "present")
-    st_release(a.carry + tile, (uint64_t(1) << 63) | (static_cast<uint64_t>(epoch & kEpochMask) << 32) |
-                                   static_cast<uint64_t>(word));
-}
-
 __device__ __forceinline__ void abort_all(const EncodeArgs& a) {
     report(a.status, QSGD_ST_LOOKBACK_TIMEOUT);
     atomicExch(&a.ctrl->abort, 1u);
@@ -133,255 +110,422 @@ __device__ __forceinline__ void cta_exit(ScanControl* ctrl, uint32_t epoch) {
     }
 }
 
-// Stores the words of a tile whose bits sit at tile-local offsets in tw[] and
-// whose stream prefix is X.  Word q of the tile's global range is
-// (tw[q] >> sh) | (tw[q-1] << (32 - sh)), sh = X mod 32.  Word 0 (when sh != 0)
-// also holds the predecessor's last bits and is written here after its tail word
-// arrives; the tile's own partial last word is published for the successor (or
-// stored, for the last tile).
-__device__ __forceinline__ void store_tile(const EncodeArgs& a, const uint32_t* tw, uint32_t tile,
-                                           uint64_t X, uint64_t tb, uint32_t epoch) {
+// ---------------------------------------------------------------------------
+// Fast path (128 <= d <= 128*V, d % 4 == 0, s < 2^21, 16-byte aligned input).
+//
+// Tiles of kFastWarps consecutive buckets, one bucket per warp; lane L codes the 4V
+// consecutive coordinates [4VL, 4VL+4V) of its bucket.  CTAs draw tiles from an
+// atomic ticket, in order.  Stream positions come from a two-level scan that never
+// walks a chain: rounds are C consecutive tickets (C = grid size); a tile publishes
+// its bit count A(t) as soon as it is known, and its exclusive prefix is the
+// previous round's total RP(r-1) plus the sum of A over its round's earlier tiles,
+// read in parallel; the round's last tile publishes RP(r).  A tile only waits on
+// tiles with smaller tickets, which are held by running CTAs.  Each CTA codes its
+// next tile into the second of two tile buffers before it waits for the current
+// tile's prefix, and copies the input of the tile after that into shared memory
+// with cp.async while it works.  The one word two neighbouring tiles share is
+// merged through a slot: whichever tile comes second writes it, nobody waits.
+// ---------------------------------------------------------------------------
+struct TileSlot {
+    uint32_t bits[kFastWarps];  // bits of each bucket of the tile
+    uint64_t total;         // bits of the tile
+};
+
+// Slot of the word shared by tiles t-1 and t: [63:40] epoch, [32] present,
+// [31:0] the first writer's bits.  The second writer ORs its bits in and stores
+// the word; a zero-filled slot or one from an earlier call reads as empty.
+__device__ __forceinline__ void merge_shared_word(const EncodeArgs& a, uint64_t* slot, uint64_t gw,
+                                                  uint32_t bits, uint32_t epoch) {
+    const uint64_t mine = (static_cast<uint64_t>(epoch & kEpochMask) << 40) | (uint64_t(1) << 32) | bits;
+    uint64_t cur = ld_acquire(slot);
+    for (int attempt = 0; attempt < 4; ++attempt) {
+        if (static_cast<uint32_t>(cur >> 40) == (epoch & kEpochMask) && ((cur >> 32) & 1u)) {
+            store_word(a, gw, bits | static_cast<uint32_t>(cur));
+            return;
+        }
+        const unsigned long long prev = atomicCAS(reinterpret_cast<unsigned long long*>(slot),
+                                                  static_cast<unsigned long long>(cur),
+                                                  static_cast<unsigned long long>(mine));
+        if (prev == cur) return;  // first: the other tile writes the word
+        cur = prev;
+    }
+    abort_all(a);  // unreachable with two writers per slot
+}
+
+// Copies the input of tile t into `xin` (cp.async, 16 bytes per copy).  Lane L of
+// warp w takes float4 j of its coordinates to slot L*V + (j ^ swz(L)), so that the
+// later 16-byte reads (lane L, slot j) fall in distinct bank groups.
+template <int V>
+__device__ __forceinline__ void prefetch_tile(const EncodeArgs& a, uint64_t t, float4* xin) {
+    if (t >= a.ntiles) return;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint64_t b = t * kFastWarps + warp;
+    if (b >= a.nb) return;
+    const uint64_t base = b * a.d;
+    const uint32_t m = static_cast<uint32_t>(min(static_cast<uint64_t>(a.d), a.n - base));
+    const uint32_t swz = (static_cast<uint32_t>(lane) * V / 8) & (V - 1);
+    float4* dst = xin + warp * 32 * V + lane * V;
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+        const uint32_t i = lane * 4 * V + 4 * j;
+        const uint32_t avail = i < m ? min(16u, (m - i) * 4u) : 0u;
+        const uint32_t saddr = static_cast<uint32_t>(__cvta_generic_to_shared(dst + (j ^ swz)));
+        const float* src = a.in + base + (i < m ? i : 0);
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(saddr), "l"(src), "r"(avail)
+                     : "memory");
+    }
+    asm volatile("cp.async.commit_group;\n" ::: "memory");
+}
+
+// Codes tile t into tbuf (tile-local bit offsets) and publishes A(t).  On entry
+// the tile's input is in flight into xin.  Two CTA barriers.
+template <int V, bool kShort>
+__device__ __forceinline__ void code_tile(const EncodeArgs& a, uint64_t t, uint64_t t_after, const uint32_t* rtab,
+                                          uint32_t* tbuf, uint32_t* pb, float4* xin, TileSlot& slot,
+                                          uint32_t epoch) {
+    // tbuf holds the bits of the tile coded two tiles ago (slot.total, set by that
+    // tile): clear the words it used
+    const uint32_t dirty = min(a.smem_words, static_cast<uint32_t>((slot.total + 31) >> 5) + 2u);
+    constexpr int NC = 4 * V;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint64_t b = t * kFastWarps + warp;
+    const bool live = b < a.nb;
+    const uint64_t base = b * a.d;
+    const uint32_t first = lane * NC;  // first bucket-local coordinate of this lane
+
+    for (uint32_t i = tid; i < dirty; i += kFastBlock) tbuf[i] = 0u;
+    asm volatile("cp.async.wait_all;\n" ::: "memory");
+    __syncthreads();  // B0: the tile's input has landed; the buffer is clear
+
+    // --- input from shared memory ------------------------------------------
+    float x[NC];
+    {
+        const uint32_t swz = (static_cast<uint32_t>(lane) * V / 8) & (V - 1);
+        const float4* src = xin + warp * 32 * V + lane * V;
+#pragma unroll
+        for (int j = 0; j < V; ++j) {
+            const float4 q = live ? src[j ^ swz] : make_float4(0.f, 0.f, 0.f, 0.f);
+            x[4 * j + 0] = q.x;
+            x[4 * j + 1] = q.y;
+            x[4 * j + 2] = q.z;
+            x[4 * j + 3] = q.w;
+        }
+    }
+
+    // --- bucket norm: per-lane FMA chain, butterfly (same value in all lanes) --
+    float ss = 0.f;
+#pragma unroll
+    for (int q = 0; q < NC; ++q) ss = __fmaf_rn(x[q], x[q], ss);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss = __fadd_rn(ss, __shfl_xor_sync(kFull, ss, o));
+    float norm = __fsqrt_rn(ss);
+    if (live && needs_rescale(ss) && !isnan(ss)) {  // uniform in the warp
+        float mx = 0.f;
+#pragma unroll
+        for (int q = 0; q < NC; ++q) mx = fmaxf(mx, fabsf(x[q]));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
+        if (isinf(mx)) {
+            norm = mx;
+        } else if (mx > 0.f) {
+            float unscale;
+            const float scale = pow2_scale(mx, unscale);
+            float s2 = 0.f;
+#pragma unroll
+            for (int q = 0; q < NC; ++q) {
+                const float y = __fmul_rn(x[q], scale);
+                s2 = __fmaf_rn(y, y, s2);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) s2 = __fadd_rn(s2, __shfl_xor_sync(kFull, s2, o));
+            norm = __fmul_rn(__fsqrt_rn(s2), unscale);
+        }
+    }
+    const BucketScale sc = bucket_scale(norm, a.s, live, a.status, lane == 0);
+    if (!sc.good) {
+#pragma unroll
+        for (int q = 0; q < NC; ++q) x[q] = 0.f;
+    }
+
+    // --- stochastic rounding: one Philox block per 4 coordinates ------------
+    uint32_t kq[NC];  // level | sign << 31
+    const uint64_t g0 = base + first;  // a multiple of 4
+    const PhiloxKey key{a.key0, a.key1};
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+        const uint4 r = philox4x32_10((g0 >> 2) + j, key);
+        const uint32_t rw[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const float v = x[4 * j + c];
+            kq[4 * j + c] = quantize_level(v, sc.sinv, rw[c], a.s) | (__float_as_uint(v) & 0x80000000u);
+        }
+    }
+
+    // --- compact the bucket's non-zeros into the warp's record list, which
+    // reuses this warp's slice of the input buffer (free once x is in registers);
+    // entry = index | k << 10 | sign << 31, in index order ---------------------
+    uint32_t* const rec = reinterpret_cast<uint32_t*>(xin + warp * 32 * V);
+    uint32_t cnt = 0;
+#pragma unroll
+    for (int q = 0; q < NC; ++q) cnt += (kq[q] & 0x7FFFFFFFu) != 0u;
+    uint32_t incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t tt = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += tt;
+    }
+    const uint32_t nz = __shfl_sync(kFull, incl, 31);
+    {
+        uint32_t pos = incl - cnt;
+#pragma unroll
+        for (int q = 0; q < NC; ++q) {
+            if (kq[q] & 0x7FFFFFFFu) {
+                rec[pos] = (first + q) | ((kq[q] & 0x7FFFFFFFu) << 10) | (kq[q] & 0x80000000u);
+                ++pos;
+            }
+        }
+    }
+    __syncwarp();
+
+    // --- records omega(gap) | sign | omega(k) of a contiguous run, packed
+    // MSB-first into this lane's private strip (word j at pb[32 j + lane]) ----
+    LanePacker pk{pb + lane, 0u, 0u, 0u};
+    {
+        const uint32_t per = (nz + 31) >> 5;
+        const uint32_t r0 = min(nz, lane * per), r1 = min(nz, r0 + per);
+        uint32_t prev = r0 ? (rec[r0 - 1] & 1023u) : 0xFFFFFFFFu;  // -1 before the first
+        for (uint32_t r = r0; r < r1; ++r) {
+            const uint32_t e = rec[r];
+            const uint32_t i = e & 1023u;
+            const uint32_t k = (e >> 10) & 0x1FFFFFu;
+            const uint32_t gap = i - prev;
+            prev = i;
+            if (gap < 64u && k < 16u) {
+                const uint32_t re = rtab[(gap << 5) | (k << 1) | (e >> 31)];
+                pk.put(re >> 5, re & 31u);
+            } else {
+                uint64_t gc, kc;
+                uint32_t gl, kl;
+                omega_code_global(gap, gc, gl);
+                omega_code_global(k, kc, kl);
+                pk.put((static_cast<uint32_t>(gc) << 1) | (e >> 31), gl + 1u);
+                if (kl > 32) pk.put(static_cast<uint32_t>(kc >> 32), kl - 32u);
+                pk.put(static_cast<uint32_t>(kc), kl > 32 ? 32u : kl);
+            }
+        }
+        pk.finish();
+    }
+    const uint32_t nbits = pk.bits();
+    uint32_t inclb = nbits;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t tt = __shfl_up_sync(kFull, inclb, o);
+        if (lane >= o) inclb += tt;
+    }
+    const uint32_t exclb = inclb - nbits;
+    if (lane == 31) slot.bits[warp] = live ? 32u + inclb : 0u;
+    __syncthreads();  // B1: bucket sizes known; the input buffer is free
+    prefetch_tile<V>(a, t_after, xin);
+    // tile-local start of this warp's bucket and the tile's size (kFastWarps-lane scan)
+    uint32_t bsc = lane < kFastWarps ? slot.bits[lane] : 0u;
+#pragma unroll
+    for (int o = 1; o < kFastWarps; o <<= 1) {
+        const uint32_t tt = __shfl_up_sync(kFull, bsc, o);
+        if (lane >= o) bsc += tt;
+    }
+    const uint64_t tb = __shfl_sync(kFull, bsc, kFastWarps - 1);
+    const uint64_t bstart = warp ? __shfl_sync(kFull, bsc, warp - 1) : 0u;
+    if (tid == 0) {
+        st_release(a.desc + t, make_desc(epoch, kStateAggregate, tb));
+        slot.total = tb;
+    }
+
+    // --- move the bits to their tile-local offsets ----------------------------
+    if (live) {
+        if (lane == 0) {
+            const uint32_t nb32 = __float_as_uint(sc.sent);
+            const uint32_t w = static_cast<uint32_t>(bstart >> 5), sh = static_cast<uint32_t>(bstart & 31u);
+            atomicOr(&tbuf[w], nb32 >> sh);
+            if (sh) atomicOr(&tbuf[w + 1], nb32 << (32 - sh));
+        }
+        const uint32_t pos = static_cast<uint32_t>(bstart) + 32u + exclb;  // first bit of this lane's records
+        const uint32_t w = pos >> 5, sh = pos & 31u;
+        const uint32_t nsrc = (nbits + 31u) >> 5;         // words in the strip
+        const uint32_t ndst = (sh + nbits + 31u) >> 5;    // words touched in the tile buffer
+        if (w + ndst > a.smem_words) {
+            report(a.status, QSGD_ST_OVERFLOW);
+        } else {
+            uint32_t prv = 0;
+            for (uint32_t j = 0; j < ndst; ++j) {
+                const uint32_t cur = j < nsrc ? pb[32 * j + lane] : 0u;
+                const uint32_t v = sh ? (cur >> sh) | (prv << (32 - sh)) : cur;
+                if (v) atomicOr(&tbuf[w + j], v);
+                prv = cur;
+            }
+        }
+    }
+    __syncwarp();
+}
+
+// Exclusive prefix of tile t = r*C + c: RP(r-2) + the bit counts A of every tile
+// of round r-1 + those of round r's tiles before c, all read in parallel.  The A
+// values are published when tiles are coded, well before they are needed, and
+// RP(r-2) one round earlier, so the wait is normally empty.  One CTA barrier;
+// every thread returns the same value.  `acc` is a zeroed shared accumulator;
+// false when a bounded wait ran out (or another CTA aborted).
+__device__ __forceinline__ bool wait_value(const uint64_t* p, uint64_t state, uint32_t epoch,
+                                           const uint32_t* abort_flag, uint64_t& value) {
+    for (uint32_t polls = 0;; ++polls) {
+        const uint64_t d = ld_acquire(p);
+        if (desc_epoch(d) == (epoch & kEpochMask) && desc_state(d) == state) {
+            value = desc_value(d);
+            return true;
+        }
+        if (polls > kMaxPolls || ((polls & 63u) == 63u && ld_acquire32(abort_flag) != 0)) return false;
+        __nanosleep(polls < 16 ? 64 : 512);
+    }
+}
+
+__device__ __forceinline__ bool gather_prefix(const EncodeArgs& a, uint32_t r, uint32_t C, uint32_t c,
+                                              uint32_t epoch, unsigned long long* acc, int* bad,
+                                              uint64_t& prefix) {
+    const int tid = threadIdx.x, lane = tid & 31;
+    uint64_t sum = 0;
+    bool ok = true;
+    // tiles [t_lo, t_hi): all of round r-1 and round r up to c; plus RP(r-2).
+    // Two descriptors per load; the values are the data, so relaxed loads suffice.
+    const uint64_t t_lo = r >= 1 ? static_cast<uint64_t>(r - 1) * C : 0;
+    const uint64_t t_hi = static_cast<uint64_t>(r) * C + c;
+    const uint64_t lo2 = t_lo & ~uint64_t(1);
+    for (uint64_t i = lo2 + 2 * static_cast<uint64_t>(tid); i < t_hi; i += 2 * kFastBlock) {
+        const ulonglong2 dd = ld_relaxed_v2(a.desc + i);
+        const uint64_t d2[2] = {dd.x, dd.y};
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const uint64_t ti = i + h;
+            if (ti < t_lo || ti >= t_hi) continue;
+            uint64_t d = d2[h];
+            if (!(desc_epoch(d) == (epoch & kEpochMask) && desc_state(d) == kStateAggregate)) {
+                uint64_t v = 0;
+                ok = ok && wait_value(a.desc + ti, kStateAggregate, epoch, &a.ctrl->abort, v);
+                d = v;
+            } else {
+                d = desc_value(d);
+            }
+            sum += d;
+        }
+    }
+    if (tid == kFastBlock - 1 && r >= 2 && ok) {
+        uint64_t v = 0;
+        ok = wait_value(a.round_prefix + (r - 2), kStatePrefix, epoch, &a.ctrl->abort, v);
+        sum += v;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(kFull, sum, o);
+    if (!ok) atomicOr(bad, 1);
+    if (lane == 0 && sum) atomicAdd(acc, static_cast<unsigned long long>(sum));
+    __syncthreads();  // Bg
+    prefix = *acc;
+    return *bad == 0;
+}
+
+// Writes tile t (bits at tile-local offsets in tbuf, stream prefix X, tb bits):
+// offsets header, the words it owns alone, and its share of the words it shares
+// with the neighbouring tiles.
+__device__ __forceinline__ void store_tile(const EncodeArgs& a, const uint32_t* tbuf, const TileSlot& slot,
+                                           uint64_t t, uint64_t X, uint64_t tb, uint32_t epoch) {
+    const int tid = threadIdx.x;
     const uint32_t sh = static_cast<uint32_t>(X & 31u);
     const uint64_t w0 = X >> 5;
     const uint64_t end = X + tb;
     const uint32_t qe = static_cast<uint32_t>((end >> 5) - w0);
-    const bool has_tail = (end & 31u) != 0;
     const uint32_t limit = a.smem_words;
     auto word_at = [&](uint32_t q) -> uint32_t {
-        const uint32_t cur = q < limit ? tw[q] : 0u;
+        const uint32_t cur = q < limit ? tbuf[q] : 0u;
         if (sh == 0) return cur;
-        const uint32_t prv = (q > 0 && q - 1 < limit) ? tw[q - 1] : 0u;
+        const uint32_t prv = (q > 0 && q - 1 < limit) ? tbuf[q - 1] : 0u;
         return (cur >> sh) | (prv << (32 - sh));
     };
-    const int tid = threadIdx.x;
-    if (tid == 0 && has_tail) {
-        const uint32_t tv = word_at(qe);
-        if (tile + 1 == a.ntiles)
-            store_word(a, w0 + qe, tv);
-        else
-            publish_carry(a, tile, epoch, tv);
+    if (tid < 32) {
+        uint32_t v = tid < kFastWarps ? slot.bits[tid] : 0u;
+#pragma unroll
+        for (int o = 1; o < kFastWarps; o <<= 1) {
+            const uint32_t tt = __shfl_up_sync(kFull, v, o);
+            if (tid >= o) v += tt;
+        }
+        const uint64_t bb = t * kFastWarps + tid;
+        if (tid < kFastWarps && bb < a.nb) a.offsets[bb] = X + v - slot.bits[tid];
     }
-    for (uint32_t q = (sh ? 1u : 0u) + tid; q < qe; q += kBlock) store_word(a, w0 + q, word_at(q));
-    if (tid == 32 && sh != 0) {  // a lane of warp 1, so warp 0's tail publication is not delayed
-        uint32_t head;
-        if (wait_carry(a, tile, epoch, head))
-            store_word(a, w0, head | word_at(0));
+    if (tid == 0 && (end & 31u) != 0) {
+        if (t + 1 == a.ntiles)
+            store_word(a, w0 + qe, word_at(qe));
         else
-            abort_all(a);
+            merge_shared_word(a, a.carry + (t + 1), w0 + qe, word_at(qe), epoch);
     }
+    if (tid == 32) {
+        if (t + 1 == a.ntiles) a.offsets[a.nb] = end;
+        if (sh != 0) merge_shared_word(a, a.carry + t, w0, word_at(0), epoch);
+    }
+    for (uint32_t q = (sh ? 1u : 0u) + tid; q < qe; q += kFastBlock) store_word(a, w0 + q, word_at(q));
 }
 
-// ---------------------------------------------------------------------------
-// Fast path: one warp per bucket of 128 < d <= 128*V coordinates.
-// ---------------------------------------------------------------------------
-template <int V>
-__global__ void __launch_bounds__(kBlock) encode_fast(const __grid_constant__ EncodeArgs a) {
+template <int V, bool kShort>
+__global__ void __launch_bounds__(kFastBlock, (V <= 4 ? kFastMinBlocks : 1)) encode_fast(const __grid_constant__ EncodeArgs a) {
     extern __shared__ __align__(16) uint32_t smem[];
-    uint32_t* tab = smem;
-    uint32_t* tw = smem + kOmegaTab;
-    __shared__ uint32_t s_tile;
-    __shared__ uint32_t s_bits[kWarps];
-    __shared__ uint64_t s_off[kWarps + 1];
-    __shared__ uint64_t s_prefix;
-    __shared__ int s_ok;
-
-    constexpr int NC = 4 * V;  // coordinates per lane
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    omega_table_fill(tab, tid, kBlock);
+    __shared__ TileSlot s_slot[2];
+    __shared__ unsigned long long s_acc[2];
+    __shared__ int s_bad;
+    __shared__ uint32_t s_ticket[2];
+    const int tid = threadIdx.x;
+    uint32_t* const rtab = smem;                                                 // record table
+    float4* const xin = reinterpret_cast<float4*>(smem + kRecordTab);           // kFastWarps * 128V floats
+    uint32_t* const tbuf0 = smem + kRecordTab + kFastWarps * 128 * V;           // two tile buffers
+    uint32_t* const pb = tbuf0 + 2 * a.smem_words + (tid >> 5) * 32 * fast_lane_words(V, kShort);  // lane strips
+    record_table_fill(rtab, tid, kFastBlock);
     const uint32_t epoch = *reinterpret_cast<volatile uint32_t*>(&a.ctrl->epoch);
-    const PhiloxKey key{a.key0, a.key1};
-
-    for (;;) {
-        if (tid == 0) s_tile = atomicAdd(&a.ctrl->ticket, 1u);
-        for (uint32_t i = tid; i < a.smem_words; i += kBlock) tw[i] = 0u;
-        __syncthreads();
-        const uint32_t tile = s_tile;
-        if (tile >= a.ntiles) break;
-
-        const uint64_t b = static_cast<uint64_t>(tile) * kWarps + warp;
-        const bool live = b < a.nb;
-        const uint64_t base = b * a.d;
-        const uint32_t m = live ? static_cast<uint32_t>(min(static_cast<uint64_t>(a.d), a.n - base)) : 0u;
-        const uint32_t first = lane * NC;  // first bucket-local coordinate of this lane
-
-        // --- load: 4V consecutive coordinates per lane --------------------
-        float x[NC];
-#pragma unroll
-        for (int j = 0; j < V; ++j) {
-            const uint32_t i = first + 4 * j;
-            if (i + 4 <= m) {
-                const float4 q = __ldg(reinterpret_cast<const float4*>(a.in + base + i));
-                x[4 * j + 0] = q.x;
-                x[4 * j + 1] = q.y;
-                x[4 * j + 2] = q.z;
-                x[4 * j + 3] = q.w;
-            } else {
-#pragma unroll
-                for (int c = 0; c < 4; ++c) x[4 * j + c] = (i + c < m) ? __ldg(a.in + base + i + c) : 0.f;
-            }
-        }
-
-        // --- bucket norm: per-lane FMA chain, then a butterfly (identical in all lanes)
-        float ss = 0.f;
-#pragma unroll
-        for (int q = 0; q < NC; ++q) ss = __fmaf_rn(x[q], x[q], ss);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) ss = __fadd_rn(ss, __shfl_xor_sync(kFull, ss, o));
-        float norm = __fsqrt_rn(ss);
-        if (live && needs_rescale(ss) && !isnan(ss)) {  // uniform in the warp
-            float mx = 0.f;
-#pragma unroll
-            for (int q = 0; q < NC; ++q) mx = fmaxf(mx, fabsf(x[q]));
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
-            if (isinf(mx)) {
-                norm = mx;
-            } else if (mx > 0.f) {
-                float unscale;
-                const float scale = pow2_scale(mx, unscale);
-                float s2 = 0.f;
-#pragma unroll
-                for (int q = 0; q < NC; ++q) {
-                    const float y = __fmul_rn(x[q], scale);
-                    s2 = __fmaf_rn(y, y, s2);
-                }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) s2 = __fadd_rn(s2, __shfl_xor_sync(kFull, s2, o));
-                norm = __fmul_rn(__fsqrt_rn(s2), unscale);
-            }
-        }
-        const BucketScale sc = bucket_scale(norm, a.s, live, a.status, lane == 0);
-        if (!sc.good) {
-#pragma unroll
-            for (int q = 0; q < NC; ++q) x[q] = 0.f;
-        }
-
-        // --- stochastic rounding: one Philox block per 4 coordinates --------
-        uint32_t kq[NC];  // level | sign << 31
-        const uint64_t g0 = base + first;  // a multiple of 4
-#pragma unroll
-        for (int j = 0; j < V; ++j) {
-            const uint4 r = philox4x32_10((g0 >> 2) + j, key);
-            const uint32_t rw[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const float v = x[4 * j + c];
-                kq[4 * j + c] = quantize_level(v, sc.sinv, rw[c], a.s) | (__float_as_uint(v) & 0x80000000u);
-            }
-        }
-
-        // --- gaps: previous non-zero before this lane (exclusive max-scan) --
-        int last = -1;
-#pragma unroll
-        for (int q = 0; q < NC; ++q)
-            if (kq[q] & 0x7FFFFFFFu) last = static_cast<int>(first) + q;
-        int incl = last;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int t = __shfl_up_sync(kFull, incl, o);
-            if (lane >= o) incl = max(incl, t);
-        }
-        int prev0 = __shfl_up_sync(kFull, incl, 1);
-        if (lane == 0) prev0 = -1;
-
-        // --- code lengths: omega(gap) + sign + omega(k) per record ----------
-        uint32_t bits = 0;
-        {
-            int prev = prev0;
-#pragma unroll
-            for (int q = 0; q < NC; ++q) {
-                const uint32_t k = kq[q] & 0x7FFFFFFFu;
-                if (k) {
-                    const int i = static_cast<int>(first) + q;
-                    bits += omega_len(tab, static_cast<uint32_t>(i - prev)) + 1u + omega_len(tab, k);
-                    prev = i;
-                }
-            }
-        }
-        uint32_t inclb = bits;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t t = __shfl_up_sync(kFull, inclb, o);
-            if (lane >= o) inclb += t;
-        }
-        const uint32_t total = __shfl_sync(kFull, inclb, 31);
-        const uint32_t exclb = inclb - bits;
-        if (lane == 0) s_bits[warp] = live ? 32u + total : 0u;
-        __syncthreads();
-
-        // --- tile aggregate: publish it (tile 0: the inclusive prefix) ------
-        if (tid == 0) {
-            uint64_t acc = 0;
-#pragma unroll
-            for (int w = 0; w < kWarps; ++w) {
-                s_off[w] = acc;
-                acc += s_bits[w];
-            }
-            s_off[kWarps] = acc;
-            st_release(a.desc + tile, make_desc(epoch, tile == 0 ? kStatePrefix : kStateAggregate, acc));
-        }
-        __syncthreads();
-
-        // --- pack the bucket at its tile-local offset ----------------------
-        if (live) {
-            const uint64_t bstart = s_off[warp];
-            if (lane == 0) {
-                const uint32_t nbits = __float_as_uint(sc.sent);
-                const uint32_t w = static_cast<uint32_t>(bstart >> 5), sh = static_cast<uint32_t>(bstart & 31u);
-                atomicOr(&tw[w], nbits >> sh);
-                if (sh) atomicOr(&tw[w + 1], nbits << (32 - sh));
-            }
-            BitPacker pk;
-            pk.start(tw, a.smem_words, bstart + 32u + exclb);
-            bool ok = true;
-            int prev = prev0;
-#pragma unroll
-            for (int q = 0; q < NC; ++q) {
-                const uint32_t k = kq[q] & 0x7FFFFFFFu;
-                if (k) {
-                    const int i = static_cast<int>(first) + q;
-                    uint64_t gc, kc;
-                    uint32_t gl, kl;
-                    omega_code(tab, static_cast<uint32_t>(i - prev), gc, gl);
-                    omega_code(tab, k, kc, kl);
-                    prev = i;
-                    ok &= pk.put((gc << 1) | (kq[q] >> 31), gl + 1u);
-                    ok &= pk.put(kc, kl);
-                }
-            }
-            ok &= pk.flush();
-            if (!ok) report(a.status, QSGD_ST_OVERFLOW);
-        }
-        __syncthreads();
-
-        // --- look-back (warp 0) -------------------------------------------
-        if (warp == 0) {
-            uint64_t excl = 0;
-            bool ok = true;
-            if (tile > 0) ok = lookback(a.desc, tile, epoch, &a.ctrl->abort, excl);
-            if (lane == 0) {
-                if (!ok)
-                    abort_all(a);
-                else if (tile > 0)
-                    st_release(a.desc + tile, make_desc(epoch, kStatePrefix, excl + s_off[kWarps]));
-                s_prefix = excl;
-                s_ok = ok;
-            }
-        }
-        __syncthreads();
-
-        // --- offsets header and words -------------------------------------
-        if (s_ok) {
-            const uint64_t X = s_prefix;
-            if (tid < kWarps) {
-                const uint64_t bb = static_cast<uint64_t>(tile) * kWarps + tid;
-                if (bb < a.nb) a.offsets[bb] = X + s_off[tid];
-            }
-            if (tid == kWarps && tile + 1 == a.ntiles) a.offsets[a.nb] = X + s_off[kWarps];
-            store_tile(a, tw, tile, X, s_off[kWarps], epoch);
-        }
-        __syncthreads();
+    const uint32_t C = gridDim.x;
+    if (tid == 0) {
+        s_ticket[0] = atomicAdd(&a.ctrl->ticket, 1u);
+        s_ticket[1] = atomicAdd(&a.ctrl->ticket, 1u);
+        s_acc[0] = s_acc[1] = 0;
+        s_bad = 0;
+        s_slot[0].total = s_slot[1].total = static_cast<uint64_t>(a.smem_words) * 32;  // clear all at first use
     }
+    __syncthreads();
+    uint64_t t = s_ticket[0];
+    uint64_t tn = s_ticket[1];
+    int cur = 0;
+    prefetch_tile<V>(a, t, xin);
+    if (t < a.ntiles) code_tile<V, kShort>(a, t, tn, rtab, tbuf0, pb, xin, s_slot[0], epoch);
+    for (int it = 0; t < a.ntiles; ++it) {
+        // the ticket after tn, drawn now so its input can be copied during tn's coding
+        if (tid == 0) s_ticket[it & 1] = atomicAdd(&a.ctrl->ticket, 1u);
+        uint32_t* const tcur = tbuf0 + cur * a.smem_words;
+        uint32_t* const tnext = tbuf0 + (cur ^ 1) * a.smem_words;
+        __syncthreads();
+        const uint64_t tnn = s_ticket[it & 1];
+        // code the next tile first: its work covers this tile's prefix wait
+        if (tn < a.ntiles) code_tile<V, kShort>(a, tn, tnn, rtab, tnext, pb, xin, s_slot[cur ^ 1], epoch);
+        const uint32_t r = static_cast<uint32_t>(t) / C;
+        const uint32_t c = static_cast<uint32_t>(t) - r * C;
+        const uint64_t tb = s_slot[cur].total;
+        uint64_t X = 0;
+        const bool ok = gather_prefix(a, r, C, c, epoch, &s_acc[it & 1], &s_bad, X);
+        if (tid == 0) s_acc[(it + 1) & 1] = 0;  // the next iteration's accumulator
+        if (!ok) {
+            if (tid == 0) abort_all(a);
+        } else {
+            if (tid == 0 && ((c + 1 == C) || (t + 1 == a.ntiles)))
+                st_release(a.round_prefix + r, make_desc(epoch, kStatePrefix, X + tb));
+            store_tile(a, tcur, s_slot[cur], t, X, tb, epoch);
+        }
+        t = tn;
+        tn = tnn;
+        cur ^= 1;
+    }
+    asm volatile("cp.async.wait_all;\n" ::: "memory");
+    __syncthreads();
     cta_exit(a.ctrl, epoch);
 }
 
@@ -691,51 +835,51 @@ __global__ void __launch_bounds__(kBlock) encode_general(const __grid_constant__
                 if (tile + 1 == a.ntiles)
                     store_word(a, end >> 5, s_pending);
                 else
-                    publish_carry(a, tile, epoch, s_pending);
+                    merge_shared_word(a, a.carry + (tile + 1), end >> 5, s_pending, epoch);
             }
             if (tile + 1 == a.ntiles) a.offsets[a.nb] = end;
-            if (head_shared) {
-                uint32_t head;
-                if (wait_carry(a, tile, epoch, head))
-                    store_word(a, head_word, head | s_head);
-                else
-                    abort_all(a);
-            }
+            if (head_shared) merge_shared_word(a, a.carry + tile, head_word, s_head, epoch);
         }
         __syncthreads();
     }
     cta_exit(a.ctrl, epoch);
 }
 
-template <int V>
+template <int V, bool kShort>
 cudaError_t launch_fast(const EncodeArgs& a, cudaStream_t stream) {
-    const size_t smem = (kOmegaTab + a.smem_words) * sizeof(uint32_t);
+    const size_t smem = fast_smem_bytes(a.d, a.s, a.smem_words);
     static bool attr_set[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 64 && !attr_set[dev]) {
-        cudaFuncSetAttribute(encode_fast<V>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+        cudaFuncSetAttribute(encode_fast<V, kShort>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
         attr_set[dev] = true;
     }
     int sms = 0, per_sm = 0;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, encode_fast<V>, kBlock, smem);
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, encode_fast<V, kShort>, kFastBlock, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const uint64_t grid = std::min<uint64_t>(a.ntiles, static_cast<uint64_t>(sms) * per_sm);
-    encode_fast<V><<<static_cast<unsigned>(grid), kBlock, smem, stream>>>(a);
+    encode_fast<V, kShort><<<static_cast<unsigned>(grid), kFastBlock, smem, stream>>>(a);
     return cudaGetLastError();
+}
+
+template <int V>
+cudaError_t launch_fast_v(const EncodeArgs& a, cudaStream_t stream) {
+    return a.s <= 31 ? launch_fast<V, true>(a, stream) : launch_fast<V, false>(a, stream);
 }
 
 }  // namespace
 
 cudaError_t launch_encode(EncodeArgs a, bool fast_path, cudaStream_t stream) {
     if (fast_path) {
-        const uint32_t v = (a.d + 127) / 128;
-        if (v <= 1) return launch_fast<1>(a, stream);
-        if (v <= 2) return launch_fast<2>(a, stream);
-        if (v <= 4) return launch_fast<4>(a, stream);
-        return launch_fast<8>(a, stream);
+        switch (fast_v(a.d)) {
+            case 1: return launch_fast_v<1>(a, stream);
+            case 2: return launch_fast_v<2>(a, stream);
+            case 4: return launch_fast_v<4>(a, stream);
+            default: return launch_fast_v<8>(a, stream);
+        }
     }
     int dev = 0, sms = 0, per_sm = 0;
     cudaGetDevice(&dev);

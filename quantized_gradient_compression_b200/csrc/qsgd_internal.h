@@ -15,10 +15,11 @@ struct ScanControl;
 // Workspace layout (all offsets 256-byte aligned):
 //   [0, 64)          ScanControl
 //   desc[ntiles]     uint64 scan descriptors
-//   carry[ntiles]    uint64 tail-word slots (1 << 63 | epoch << 32 | word)
+//   carry[ntiles]    uint64 shared-word slots (epoch << 40 | present << 32 | bits)
+//   rp[ntiles]       uint64 round prefixes of the fast path
 //   norms[nb]        float2 (sent norm, s/norm) of the general path
 struct WorkspaceLayout {
-    size_t desc_off, carry_off, norms_off, total;
+    size_t desc_off, carry_off, rp_off, norms_off, total;
     uint64_t max_tiles;
 };
 WorkspaceLayout workspace_layout(uint64_t n, uint32_t d);
@@ -36,6 +37,7 @@ struct EncodeArgs {
     ScanControl* ctrl;
     uint64_t* desc;
     uint64_t* carry;
+    uint64_t* round_prefix;  // fast path: RP(r), inclusive prefix after round r
     float2* norms;     // general path only
     uint64_t nb;
     uint64_t ntiles;
@@ -46,6 +48,27 @@ struct EncodeArgs {
 // Chooses the kernel, sets the launch shape and enqueues it.  Returns a CUDA
 // error code (cudaSuccess on success).
 cudaError_t launch_encode(EncodeArgs a, bool fast_path, cudaStream_t stream);
+
+// Float4s per lane of the fast encoder for bucket size d (a power of two >= d/128).
+inline uint32_t fast_v(uint32_t d) {
+    const uint32_t v = (d + 127) / 128;
+    return v <= 1 ? 1 : v <= 2 ? 2 : v <= 4 ? 4 : 8;
+}
+// Words of one lane's private bit strip in the fast encoder: 4V records of at
+// most 30 bits (s <= 31) or 18 + 1 + 32 bits (larger s), plus one.
+__host__ __device__ inline constexpr uint32_t fast_lane_words(uint32_t V, bool short_records) {
+    return (4 * V * (short_records ? 30u : 51u) + 31u) / 32u + 1u;
+}
+// Dynamic shared memory of the fast encoder: record table | one tile of input
+// (kFastWarps * 128V floats; also the warps' record lists) | two tile buffers |
+// the lane strips.
+inline size_t fast_smem_bytes(uint32_t d, uint32_t s, uint32_t smem_words) {
+    const uint32_t v = fast_v(d);
+    return (static_cast<size_t>(kRecordTab) + static_cast<size_t>(kFastWarps) * 128 * v +
+            2 * static_cast<size_t>(smem_words) +
+            static_cast<size_t>(kFastWarps) * 32 * fast_lane_words(v, s <= 31)) *
+           sizeof(uint32_t);
+}
 
 struct StreamRef {
     const uint32_t* words;

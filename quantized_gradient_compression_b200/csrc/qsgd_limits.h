@@ -10,17 +10,31 @@ constexpr uint64_t kMaxD = uint64_t(1) << 31;
 constexpr uint32_t kMaxS = 1u << 22;          // keeps t = |v| s/||v|| below 2^23
 constexpr uint64_t kMaxStreamBits = (uint64_t(1) << 38) - 1;  // scan descriptor value field
 
-constexpr int kOmegaTab = 1024;               // shared-memory omega table entries
+constexpr int kOmegaTab = 2048;               // omega code table entries (N < 2048)
+constexpr int kRecordTab = 2048;              // record table: gap < 64, k < 16, sign
 constexpr uint32_t kMaxPolls = 1u << 22;      // bound of every spin wait (~1 s)
 
 constexpr int kBlock = 256;                   // threads per CTA, every encode kernel
 constexpr int kWarps = kBlock / 32;
 constexpr uint32_t kFastMinD = 128;           // warp-per-bucket path: 128 <= d <= 1024,
-constexpr uint32_t kFastMaxD = 1024;          //   d % 4 == 0, 16-byte aligned input
+constexpr uint32_t kFastMaxD = 1024;          //   d % 4 == 0, 16-byte aligned input,
+constexpr uint32_t kFastMaxS = (1u << 21) - 1;  //   s < 2^21 (a record list entry is 32 bits)
 constexpr uint32_t kChunk = 4 * kBlock;       // coordinates per chunk of the general path
 constexpr uint32_t kGeneralTileCoords = 4096; // general path: buckets per tile = max(1, 4096/d)
 
+// Fast encoder: warps per CTA (one bucket each per tile) and the CTAs per SM the
+// register budget is sized for (64 registers a thread at 32 warps per SM).
+#ifndef QSGD_FAST_WARPS
+#define QSGD_FAST_WARPS 16
+#endif
+#ifndef QSGD_FAST_MIN_BLOCKS
+#define QSGD_FAST_MIN_BLOCKS (32 / QSGD_FAST_WARPS)
+#endif
+constexpr int kFastWarps = QSGD_FAST_WARPS;
+constexpr int kFastBlock = 32 * kFastWarps;
+constexpr int kFastMinBlocks = QSGD_FAST_MIN_BLOCKS;
+
 constexpr int kDecodeBlock = 128;
-constexpr int kMaxStreamsPerLaunch = 64;
+constexpr int kMaxStreamsPerLaunch = 16;  // decode-accumulate streams per launch
 
 }  // namespace qsgd
