@@ -55,14 +55,11 @@ bool fast_eligible(const float* in, uint32_t d, uint32_t s) {
 WorkspaceLayout workspace_layout(uint64_t n, uint32_t d) {
     WorkspaceLayout L{};
     const uint64_t nb = n ? ceil_div(n, d) : 0;
-    // fast path: tiles of kWarps buckets; general path: tiles of whole buckets
-    const uint64_t per_tile = std::min<uint64_t>(kWarps, general_buckets_per_tile(d));
+    // fast path: tiles of kFastWarps buckets; general path: tiles of whole buckets
+    const uint64_t per_tile = std::min<uint64_t>(kFastWarps, general_buckets_per_tile(d));
     L.max_tiles = nb ? ceil_div(nb, per_tile) : 0;
-    L.desc_off = 256;
-    L.carry_off = L.desc_off + align256(8 * L.max_tiles);
-    L.rp_off = L.carry_off + align256(8 * L.max_tiles);
-    L.norms_off = L.rp_off + align256(8 * L.max_tiles);
-    L.total = L.norms_off + align256(8 * nb);
+    L.tiles_off = 256;
+    L.total = L.tiles_off + align256(sizeof(TileState) * L.max_tiles);
     return L;
 }
 
@@ -119,10 +116,7 @@ int qsgd_encode(const float* d_in, uint64_t n, uint32_t d, uint32_t s, uint64_t 
     a.offsets = d_offsets;
     a.status = d_status;
     a.ctrl = reinterpret_cast<ScanControl*>(ws);
-    a.desc = reinterpret_cast<uint64_t*>(ws + L.desc_off);
-    a.carry = reinterpret_cast<uint64_t*>(ws + L.carry_off);
-    a.round_prefix = reinterpret_cast<uint64_t*>(ws + L.rp_off);
-    a.norms = reinterpret_cast<float2*>(ws + L.norms_off);
+    a.ts = reinterpret_cast<TileState*>(ws + L.tiles_off);
     a.nb = ceil_div(n, d);
     const uint32_t wl = 2u + omega_len_host(s);
     const bool fast = fast_eligible(d_in, d, s);
@@ -142,7 +136,7 @@ int qsgd_encode(const float* d_in, uint64_t n, uint32_t d, uint32_t s, uint64_t 
         a.smem_words = static_cast<uint32_t>(ceil_div(chunk_bits, 32) + 2);
     }
     const uint64_t smem_bytes = fast ? fast_smem_bytes(d, s, a.smem_words)
-                                     : (kOmegaTab + static_cast<uint64_t>(a.smem_words)) * 4;
+                                     : general_smem_bytes(a.smem_words, a.buckets_per_tile);
     if (smem_bytes > 200 * 1024) return QSGD_ERR_ARG;
     if (a.ntiles > L.max_tiles) return QSGD_ERR_WORKSPACE;
     const cudaError_t e = launch_encode(a, fast, stream);

@@ -270,9 +270,9 @@ __device__ __forceinline__ uint64_t ld_acquire(const uint64_t* p) {
     asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
     return v;
 }
-__device__ __forceinline__ ulonglong2 ld_relaxed_v2(const uint64_t* p) {
-    ulonglong2 v;
-    asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(v.x), "=l"(v.y) : "l"(p) : "memory");
+__device__ __forceinline__ uint64_t ld_relaxed(const uint64_t* p) {
+    uint64_t v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
     return v;
 }
 __device__ __forceinline__ uint32_t ld_acquire32(const uint32_t* p) {
@@ -291,10 +291,18 @@ struct ScanControl {
 };
 static_assert(sizeof(ScanControl) == 64, "control block is one 64-byte line");
 
+// Per-tile state in the workspace.
+struct TileState {
+    uint64_t desc;   // scan descriptor of the tile
+    uint64_t slot;   // slot of the word shared with the previous tile
+    uint64_t round;  // fast path: RP(r), the stream position after round r (entry r)
+};
+static_assert(sizeof(TileState) == 24, "tile state is three words");
+
 // Warp-cooperative look-back for tile `tile` (> 0).  All 32 lanes call it; every
 // lane returns the exclusive prefix.  Returns false (and leaves the prefix
 // undefined) when the bounded wait ran out or another tile aborted.
-__device__ __forceinline__ bool lookback(const uint64_t* desc, uint32_t tile, uint32_t epoch,
+__device__ __forceinline__ bool lookback(const TileState* ts, uint32_t tile, uint32_t epoch,
                                          const uint32_t* abort_flag, uint64_t& exclusive) {
     const int lane = threadIdx.x & 31;
     uint64_t sum = 0;
@@ -306,7 +314,7 @@ __device__ __forceinline__ bool lookback(const uint64_t* desc, uint32_t tile, ui
         uint64_t st = kStatePrefix;  // lanes past tile 0 act as a zero prefix
         uint64_t val = 0;
         if (idx >= 0) {
-            d = ld_acquire(desc + idx);
+            d = ld_acquire(&ts[idx].desc);
             st = (desc_epoch(d) == (epoch & kEpochMask)) ? desc_state(d) : 0;
             val = desc_value(d);
         }

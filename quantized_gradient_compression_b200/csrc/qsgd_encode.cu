@@ -337,7 +337,7 @@ __device__ __forceinline__ void code_tile(const EncodeArgs& a, uint64_t t, uint6
     const uint64_t tb = __shfl_sync(kFull, bsc, kFastWarps - 1);
     const uint64_t bstart = warp ? __shfl_sync(kFull, bsc, warp - 1) : 0u;
     if (tid == 0) {
-        st_release(a.desc + t, make_desc(epoch, kStateAggregate, tb));
+        st_release(&a.ts[t].desc, make_desc(epoch, kStateAggregate, tb));
         slot.total = tb;
     }
 
@@ -394,31 +394,23 @@ __device__ __forceinline__ bool gather_prefix(const EncodeArgs& a, uint32_t r, u
     uint64_t sum = 0;
     bool ok = true;
     // tiles [t_lo, t_hi): all of round r-1 and round r up to c; plus RP(r-2).
-    // Two descriptors per load; the values are the data, so relaxed loads suffice.
+    // The values are the data, so relaxed loads suffice.
     const uint64_t t_lo = r >= 1 ? static_cast<uint64_t>(r - 1) * C : 0;
     const uint64_t t_hi = static_cast<uint64_t>(r) * C + c;
-    const uint64_t lo2 = t_lo & ~uint64_t(1);
-    for (uint64_t i = lo2 + 2 * static_cast<uint64_t>(tid); i < t_hi; i += 2 * kFastBlock) {
-        const ulonglong2 dd = ld_relaxed_v2(a.desc + i);
-        const uint64_t d2[2] = {dd.x, dd.y};
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const uint64_t ti = i + h;
-            if (ti < t_lo || ti >= t_hi) continue;
-            uint64_t d = d2[h];
-            if (!(desc_epoch(d) == (epoch & kEpochMask) && desc_state(d) == kStateAggregate)) {
-                uint64_t v = 0;
-                ok = ok && wait_value(a.desc + ti, kStateAggregate, epoch, &a.ctrl->abort, v);
-                d = v;
-            } else {
-                d = desc_value(d);
-            }
-            sum += d;
+    for (uint64_t i = t_lo + tid; i < t_hi; i += kFastBlock) {
+        uint64_t d = ld_relaxed(&a.ts[i].desc);
+        if (!(desc_epoch(d) == (epoch & kEpochMask) && desc_state(d) == kStateAggregate)) {
+            uint64_t v = 0;
+            ok = ok && wait_value(&a.ts[i].desc, kStateAggregate, epoch, &a.ctrl->abort, v);
+            d = v;
+        } else {
+            d = desc_value(d);
         }
+        sum += d;
     }
     if (tid == kFastBlock - 1 && r >= 2 && ok) {
         uint64_t v = 0;
-        ok = wait_value(a.round_prefix + (r - 2), kStatePrefix, epoch, &a.ctrl->abort, v);
+        ok = wait_value(&a.ts[r - 2].round, kStatePrefix, epoch, &a.ctrl->abort, v);
         sum += v;
     }
 #pragma unroll
@@ -461,11 +453,11 @@ __device__ __forceinline__ void store_tile(const EncodeArgs& a, const uint32_t* 
         if (t + 1 == a.ntiles)
             store_word(a, w0 + qe, word_at(qe));
         else
-            merge_shared_word(a, a.carry + (t + 1), w0 + qe, word_at(qe), epoch);
+            merge_shared_word(a, &a.ts[t + 1].slot, w0 + qe, word_at(qe), epoch);
     }
     if (tid == 32) {
         if (t + 1 == a.ntiles) a.offsets[a.nb] = end;
-        if (sh != 0) merge_shared_word(a, a.carry + t, w0, word_at(0), epoch);
+        if (sh != 0) merge_shared_word(a, &a.ts[t].slot, w0, word_at(0), epoch);
     }
     for (uint32_t q = (sh ? 1u : 0u) + tid; q < qe; q += kFastBlock) store_word(a, w0 + q, word_at(q));
 }
@@ -517,7 +509,7 @@ __global__ void __launch_bounds__(kFastBlock, (V <= 4 ? kFastMinBlocks : 1)) enc
             if (tid == 0) abort_all(a);
         } else {
             if (tid == 0 && ((c + 1 == C) || (t + 1 == a.ntiles)))
-                st_release(a.round_prefix + r, make_desc(epoch, kStatePrefix, X + tb));
+                st_release(&a.ts[r].round, make_desc(epoch, kStatePrefix, X + tb));
             store_tile(a, tcur, s_slot[cur], t, X, tb, epoch);
         }
         t = tn;
@@ -533,44 +525,90 @@ __global__ void __launch_bounds__(kFastBlock, (V <= 4 ? kFastMinBlocks : 1)) enc
 // General path.
 // ---------------------------------------------------------------------------
 
-// One warp per bucket: norm and s/norm into the workspace.
-__global__ void __launch_bounds__(kBlock) encode_norms(const __grid_constant__ EncodeArgs a) {
-    const int lane = threadIdx.x & 31;
-    const uint64_t warps = static_cast<uint64_t>(gridDim.x) * kWarps;
-    for (uint64_t b = (static_cast<uint64_t>(blockIdx.x) * kBlock + threadIdx.x) >> 5; b < a.nb; b += warps) {
-        const uint64_t base = b * a.d;
-        const uint64_t m = min(static_cast<uint64_t>(a.d), a.n - base);
-        float ss = 0.f;
-        for (uint64_t i = lane; i < m; i += 32) {
-            const float v = __ldg(a.in + base + i);
-            ss = __fmaf_rn(v, v, ss);
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) ss = __fadd_rn(ss, __shfl_xor_sync(kFull, ss, o));
-        float norm = __fsqrt_rn(ss);
-        if (needs_rescale(ss) && !isnan(ss)) {  // uniform in the warp
-            float mx = 0.f;
-            for (uint64_t i = lane; i < m; i += 32) mx = fmaxf(mx, fabsf(__ldg(a.in + base + i)));
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
-            if (isinf(mx)) {
-                norm = mx;
-            } else if (mx > 0.f) {
-                float unscale;
-                const float scale = pow2_scale(mx, unscale);
-                float s2 = 0.f;
-                for (uint64_t i = lane; i < m; i += 32) {
-                    const float y = __fmul_rn(__ldg(a.in + base + i), scale);
-                    s2 = __fmaf_rn(y, y, s2);
-                }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) s2 = __fadd_rn(s2, __shfl_xor_sync(kFull, s2, o));
-                norm = __fmul_rn(__fsqrt_rn(s2), unscale);
-            }
-        }
-        const BucketScale sc = bucket_scale(norm, a.s, true, a.status, lane == 0);
-        if (lane == 0) a.norms[b] = make_float2(sc.sent, sc.good ? sc.sinv : 0.f);
+// Norm of `m` values starting at p, by one warp (lanes take every 32nd value, then
+// a butterfly); the rescaled form when the squares leave the normal range.
+__device__ __forceinline__ float warp_norm(const float* p, uint64_t m, int lane) {
+    float ss = 0.f;
+    for (uint64_t i = lane; i < m; i += 32) {
+        const float v = __ldg(p + i);
+        ss = __fmaf_rn(v, v, ss);
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss = __fadd_rn(ss, __shfl_xor_sync(kFull, ss, o));
+    float norm = __fsqrt_rn(ss);
+    if (needs_rescale(ss) && !isnan(ss)) {  // uniform in the warp
+        float mx = 0.f;
+        for (uint64_t i = lane; i < m; i += 32) mx = fmaxf(mx, fabsf(__ldg(p + i)));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
+        if (isinf(mx)) {
+            norm = mx;
+        } else if (mx > 0.f) {
+            float unscale;
+            const float scale = pow2_scale(mx, unscale);
+            float s2 = 0.f;
+            for (uint64_t i = lane; i < m; i += 32) {
+                const float y = __fmul_rn(__ldg(p + i), scale);
+                s2 = __fmaf_rn(y, y, s2);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) s2 = __fadd_rn(s2, __shfl_xor_sync(kFull, s2, o));
+            norm = __fmul_rn(__fsqrt_rn(s2), unscale);
+        }
+    }
+    return norm;
+}
+
+// Norm of one large bucket by the whole CTA: thread i takes every kBlock-th value,
+// then a butterfly per warp and the warp sums in order (deterministic).
+__device__ __forceinline__ float block_norm(const float* p, uint64_t m, float* red) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    auto block_sum = [&](float x) -> float {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) x = __fadd_rn(x, __shfl_xor_sync(kFull, x, o));
+        __syncthreads();
+        if (lane == 0) red[warp] = x;
+        __syncthreads();
+        float tot = 0.f;
+        for (int w = 0; w < kWarps; ++w) tot = __fadd_rn(tot, red[w]);
+        return tot;
+    };
+    auto block_max = [&](float x) -> float {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(kFull, x, o));
+        __syncthreads();
+        if (lane == 0) red[warp] = x;
+        __syncthreads();
+        float mx = 0.f;
+        for (int w = 0; w < kWarps; ++w) mx = fmaxf(mx, red[w]);
+        return mx;
+    };
+    float ss = 0.f;
+    for (uint64_t i = tid; i < m; i += kBlock) {
+        const float v = __ldg(p + i);
+        ss = __fmaf_rn(v, v, ss);
+    }
+    ss = block_sum(ss);
+    float norm = __fsqrt_rn(ss);
+    if (needs_rescale(ss) && !isnan(ss)) {  // uniform in the block
+        float mx = 0.f;
+        for (uint64_t i = tid; i < m; i += kBlock) mx = fmaxf(mx, fabsf(__ldg(p + i)));
+        mx = block_max(mx);
+        if (isinf(mx)) {
+            norm = mx;
+        } else if (mx > 0.f) {
+            float unscale;
+            const float scale = pow2_scale(mx, unscale);
+            float s2 = 0.f;
+            for (uint64_t i = tid; i < m; i += kBlock) {
+                const float y = __fmul_rn(__ldg(p + i), scale);
+                s2 = __fmaf_rn(y, y, s2);
+            }
+            s2 = block_sum(s2);
+            norm = __fmul_rn(__fsqrt_rn(s2), unscale);
+        }
+    }
+    return norm;
 }
 
 // Block-wide scans for kBlock threads.
@@ -633,7 +671,8 @@ struct Quad {
 };
 
 __device__ __forceinline__ void quantize_quad(const EncodeArgs& a, uint64_t i0, uint64_t c0,
-                                              uint64_t c1, uint64_t b0, PhiloxKey key, Quad& qd) {
+                                              uint64_t c1, uint64_t b0, PhiloxKey key, const float2* norms,
+                                              Quad& qd) {
     const uint4 r = philox4x32_10(i0 >> 2, key);
     const uint32_t rw[4] = {r.x, r.y, r.z, r.w};
 #pragma unroll
@@ -649,7 +688,7 @@ __device__ __forceinline__ void quantize_quad(const EncodeArgs& a, uint64_t i0, 
         const uint32_t rel = static_cast<uint32_t>(i - c0);  // < buckets_per_tile * d <= 2^31
         const uint64_t bl = rel / a.d;
         const uint64_t b = b0 + bl;
-        const float2 ns = a.norms[b];
+        const float2 ns = norms[bl];
         const float v = __ldg(a.in + i);
         qd.bucket[c] = b;
         qd.bstart[c] = b * a.d;
@@ -664,6 +703,8 @@ __global__ void __launch_bounds__(kBlock) encode_general(const __grid_constant__
     extern __shared__ __align__(16) uint32_t smem[];
     uint32_t* tab = smem;
     uint32_t* buf = smem + kOmegaTab;
+    float2* s_norms = reinterpret_cast<float2*>(smem + kOmegaTab + ((a.smem_words + 1) & ~1u));  // (norm, s/norm)
+    __shared__ float s_red[kWarps];
     __shared__ uint32_t s_tile;
     __shared__ BlockScratch s_scr;
     __shared__ uint64_t s_prefix;
@@ -687,12 +728,29 @@ __global__ void __launch_bounds__(kBlock) encode_general(const __grid_constant__
         const uint64_t c1 = min(a.n, b1 * a.d);
         const uint64_t cbase = c0 & ~uint64_t(3);
 
+        // --- bucket norms into shared memory -------------------------------
+        if (b1 - b0 == 1) {
+            const uint64_t m = c1 - c0;
+            const float norm = block_norm(a.in + c0, m, s_red);
+            const BucketScale sc = bucket_scale(norm, a.s, true, a.status, tid == 0);
+            if (tid == 0) s_norms[0] = make_float2(sc.sent, sc.good ? sc.sinv : 0.f);
+        } else {
+            for (uint64_t bl = warp; bl < b1 - b0; bl += kWarps) {
+                const uint64_t base = (b0 + bl) * a.d;
+                const uint64_t m = min(static_cast<uint64_t>(a.d), a.n - base);
+                const float norm = warp_norm(a.in + base, m, lane);
+                const BucketScale sc = bucket_scale(norm, a.s, true, a.status, lane == 0);
+                if (lane == 0) s_norms[bl] = make_float2(sc.sent, sc.good ? sc.sinv : 0.f);
+            }
+        }
+        __syncthreads();
+
         // --- pass 1: bit count of the tile --------------------------------
         uint64_t tb = 0;
         int64_t carry_prev = -1;
         for (uint64_t cb = cbase; cb < c1; cb += kChunk) {
             Quad qd;
-            quantize_quad(a, cb + 4ull * tid, c0, c1, b0, key, qd);
+            quantize_quad(a, cb + 4ull * tid, c0, c1, b0, key, s_norms, qd);
             int64_t last = -1;
 #pragma unroll
             for (int c = 0; c < 4; ++c)
@@ -718,18 +776,18 @@ __global__ void __launch_bounds__(kBlock) encode_general(const __grid_constant__
             tb += total;
         }
         if (tid == 0)
-            st_release(a.desc + tile, make_desc(epoch, tile == 0 ? kStatePrefix : kStateAggregate, tb));
+            st_release(&a.ts[tile].desc, make_desc(epoch, tile == 0 ? kStatePrefix : kStateAggregate, tb));
 
         // --- look-back ------------------------------------------------------
         if (warp == 0) {
             uint64_t excl = 0;
             bool ok = true;
-            if (tile > 0) ok = lookback(a.desc, tile, epoch, &a.ctrl->abort, excl);
+            if (tile > 0) ok = lookback(a.ts, tile, epoch, &a.ctrl->abort, excl);
             if (lane == 0) {
                 if (!ok)
                     abort_all(a);
                 else if (tile > 0)
-                    st_release(a.desc + tile, make_desc(epoch, kStatePrefix, excl + tb));
+                    st_release(&a.ts[tile].desc, make_desc(epoch, kStatePrefix, excl + tb));
                 s_prefix = excl;
                 s_ok = ok;
                 s_pending = 0;
@@ -750,7 +808,7 @@ __global__ void __launch_bounds__(kBlock) encode_general(const __grid_constant__
         carry_prev = -1;
         for (uint64_t cb = cbase; cb < c1; cb += kChunk) {
             Quad qd;
-            quantize_quad(a, cb + 4ull * tid, c0, c1, b0, key, qd);
+            quantize_quad(a, cb + 4ull * tid, c0, c1, b0, key, s_norms, qd);
             int64_t last = -1;
 #pragma unroll
             for (int c = 0; c < 4; ++c)
@@ -835,10 +893,10 @@ __global__ void __launch_bounds__(kBlock) encode_general(const __grid_constant__
                 if (tile + 1 == a.ntiles)
                     store_word(a, end >> 5, s_pending);
                 else
-                    merge_shared_word(a, a.carry + (tile + 1), end >> 5, s_pending, epoch);
+                    merge_shared_word(a, &a.ts[tile + 1].slot, end >> 5, s_pending, epoch);
             }
             if (tile + 1 == a.ntiles) a.offsets[a.nb] = end;
-            if (head_shared) merge_shared_word(a, a.carry + tile, head_word, s_head, epoch);
+            if (head_shared) merge_shared_word(a, &a.ts[tile].slot, head_word, s_head, epoch);
         }
         __syncthreads();
     }
@@ -884,14 +942,7 @@ cudaError_t launch_encode(EncodeArgs a, bool fast_path, cudaStream_t stream) {
     int dev = 0, sms = 0, per_sm = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    // norms pre-pass: one warp per bucket
-    {
-        const uint64_t blocks = std::min<uint64_t>((a.nb + kWarps - 1) / kWarps, static_cast<uint64_t>(sms) * 64);
-        encode_norms<<<static_cast<unsigned>(blocks), kBlock, 0, stream>>>(a);
-        const cudaError_t e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
-    }
-    const size_t smem = (kOmegaTab + a.smem_words) * sizeof(uint32_t);
+    const size_t smem = general_smem_bytes(a.smem_words, a.buckets_per_tile);
     static bool attr_set[64] = {};
     if (dev < 64 && !attr_set[dev]) {
         cudaFuncSetAttribute(encode_general, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);

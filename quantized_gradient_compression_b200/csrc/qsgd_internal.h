@@ -11,15 +11,14 @@
 namespace qsgd {
 
 struct ScanControl;
+struct TileState;
 
-// Workspace layout (all offsets 256-byte aligned):
-//   [0, 64)          ScanControl
-//   desc[ntiles]     uint64 scan descriptors
-//   carry[ntiles]    uint64 shared-word slots (epoch << 40 | present << 32 | bits)
-//   rp[ntiles]       uint64 round prefixes of the fast path
-//   norms[nb]        float2 (sent norm, s/norm) of the general path
+// Workspace layout: [0, 256) ScanControl, then TileState[max_tiles] (24 bytes per
+// tile: scan descriptor, shared-word slot, round prefix).  Every entry carries the
+// call's epoch and sits at the same place whatever (n, d, s) a call uses, so one
+// workspace serves calls of any shape without clearing.
 struct WorkspaceLayout {
-    size_t desc_off, carry_off, rp_off, norms_off, total;
+    size_t tiles_off, total;
     uint64_t max_tiles;
 };
 WorkspaceLayout workspace_layout(uint64_t n, uint32_t d);
@@ -35,10 +34,7 @@ struct EncodeArgs {
     uint64_t* offsets;
     uint32_t* status;
     ScanControl* ctrl;
-    uint64_t* desc;
-    uint64_t* carry;
-    uint64_t* round_prefix;  // fast path: RP(r), inclusive prefix after round r
-    float2* norms;     // general path only
+    TileState* ts;
     uint64_t nb;
     uint64_t ntiles;
     uint32_t buckets_per_tile;
@@ -48,6 +44,13 @@ struct EncodeArgs {
 // Chooses the kernel, sets the launch shape and enqueues it.  Returns a CUDA
 // error code (cudaSuccess on success).
 cudaError_t launch_encode(EncodeArgs a, bool fast_path, cudaStream_t stream);
+
+// Dynamic shared memory of the general encoder: omega table | chunk buffer |
+// (norm, s/norm) of the tile's buckets.
+inline size_t general_smem_bytes(uint32_t smem_words, uint32_t buckets_per_tile) {
+    return (static_cast<size_t>(kOmegaTab) + ((smem_words + 1) & ~1u) + 2 * static_cast<size_t>(buckets_per_tile)) *
+           sizeof(uint32_t);
+}
 
 // Float4s per lane of the fast encoder for bucket size d (a power of two >= d/128).
 inline uint32_t fast_v(uint32_t d) {
