@@ -65,7 +65,9 @@ typedef enum {
     QSGD_ERR_ARG = 1,       /* a pointer, size or parameter out of range */
     QSGD_ERR_CAPACITY = 2,  /* output buffer smaller than qsgd_max_encoded_words */
     QSGD_ERR_CUDA = 3,      /* a CUDA runtime call or kernel launch failed */
-    QSGD_ERR_WORKSPACE = 4  /* workspace smaller than qsgd_encode_workspace_bytes */
+    QSGD_ERR_WORKSPACE = 4,   /* workspace smaller than qsgd_encode_workspace_bytes */
+    QSGD_ERR_STATIC_LIMIT = 5 /* qsgd_encode_static_ws: the problem needs more scan state than
+                                 the library's fixed device workspace */
 } qsgd_err;
 
 /* Device status bits, OR-ed into *d_status. */
@@ -136,6 +138,38 @@ QSGD_API int qsgd_decode(const uint32_t* d_words, uint64_t num_words, const uint
 QSGD_API int qsgd_decode_accumulate(const uint32_t* const* h_words, const uint64_t* h_num_words,
                            const uint64_t* const* h_offsets, int K, uint64_t n, uint32_t d,
                            uint32_t s, float* d_out, uint32_t* d_status, cudaStream_t stream);
+
+/* Encoder for callers that cannot allocate device memory.  (The paper has no
+ * counterpart: this is a deployment variant of qsgd_encode.)
+ *
+ * Who needs it: code that compresses a gradient at a point where it may not call
+ * cudaMalloc -- inside a caching allocator's own callbacks, in a communication
+ * library's progress thread that must not take the allocator's lock, or in an
+ * embedding that only passes the codec its input and output buffers.  The output
+ * buffers are still the caller's; only the encoder's scan state (the workspace of
+ * qsgd_encode) moves into a fixed array of device memory owned by the library.
+ *
+ * Same arguments and results as qsgd_encode without d_ws / ws_bytes; the stream
+ * is bit-identical to qsgd_encode's for the same (d_in, n, d, s, seed).
+ *   - The array is qsgd_static_workspace_limit() bytes (4 MiB).  Every GPU that
+ *     loads the library holds it until the process exits.  A problem whose
+ *     qsgd_encode_workspace_bytes(n, d, s) exceeds it is rejected with
+ *     QSGD_ERR_STATIC_LIMIT before anything is enqueued (about 1.4 million
+ *     buckets at d = 512).
+ *   - The first call on a device looks up the array's device address (once per
+ *     device, with that device current).  Make that first call before any stream
+ *     capture.
+ *   - Every call shares the one array.  Its state is tagged with a call counter
+ *     and reset by the end of each call, so no call needs to clear it, but calls
+ *     that may overlap on the GPU (different streams, or different host threads)
+ *     race and must be serialised by the caller.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library routine. */
+QSGD_API int qsgd_encode_static_ws(const float* d_in, uint64_t n, uint32_t d, uint32_t s, uint64_t seed,
+                                   uint32_t* d_words, uint64_t words_capacity, uint64_t* d_offsets,
+                                   uint32_t* d_status, cudaStream_t stream);
+
+/* Bytes of the fixed device workspace behind qsgd_encode_static_ws. */
+QSGD_API size_t qsgd_static_workspace_limit(void);
 
 /* Static description of a host return code. */
 QSGD_API const char* qsgd_error_string(int code);

@@ -30,6 +30,7 @@ QSGD_ERR_ARG = 1
 QSGD_ERR_CAPACITY = 2
 QSGD_ERR_CUDA = 3
 QSGD_ERR_WORKSPACE = 4
+QSGD_ERR_STATIC_LIMIT = 5
 
 QSGD_ST_NONFINITE = 1
 QSGD_ST_BAD_STREAM = 2
@@ -48,6 +49,8 @@ _SIGS = {
     "qsgd_decode": (_int, [_vp, _u64, _vp, _u64, _u32, _u32, _vp, _vp, _vp]),
     "qsgd_decode_accumulate": (_int, [ctypes.POINTER(_vp), ctypes.POINTER(_u64), ctypes.POINTER(_vp),
                                       _int, _u64, _u32, _u32, _vp, _vp, _vp]),
+    "qsgd_encode_static_ws": (_int, [_vp, _u64, _u32, _u32, _u64, _vp, _u64, _vp, _vp, _vp]),
+    "qsgd_static_workspace_limit": (_sz, []),
     "qsgd_error_string": (ctypes.c_char_p, [_int]),
     "qsgd_version": (ctypes.c_char_p, []),
 }
@@ -106,6 +109,17 @@ def qsgd_decode_accumulate(h_words, h_num_words, h_offsets, K: int, n: int, d: i
     nw = (_u64 * K)(*h_num_words)
     o = (_vp * K)(*h_offsets)
     return int(_lib.qsgd_decode_accumulate(w, nw, o, K, n, d, s, d_out, d_status, stream))
+
+
+def qsgd_encode_static_ws(d_in: int, n: int, d: int, s: int, seed: int, d_words: int, words_capacity: int,
+                          d_offsets: int, d_status: int, stream: int) -> int:
+    """qsgd_encode without a caller workspace (for callers that cannot allocate)."""
+    return int(_lib.qsgd_encode_static_ws(d_in, n, d, s, seed & 0xFFFFFFFFFFFFFFFF, d_words, words_capacity,
+                                          d_offsets, d_status, stream))
+
+
+def qsgd_static_workspace_limit() -> int:
+    return int(_lib.qsgd_static_workspace_limit())
 
 
 def qsgd_error_string(code: int) -> str:

@@ -194,6 +194,9 @@ const char* qsgd_error_string(int code) {
         case QSGD_ERR_CAPACITY: return "output capacity below qsgd_max_encoded_words";
         case QSGD_ERR_CUDA: return "CUDA runtime error";
         case QSGD_ERR_WORKSPACE: return "workspace below qsgd_encode_workspace_bytes";
+        case QSGD_ERR_STATIC_LIMIT:
+            return "problem needs more scan state than the fixed device workspace of qsgd_encode_static_ws; "
+                   "call qsgd_encode with a caller workspace";
         default: return "unknown error";
     }
 }
