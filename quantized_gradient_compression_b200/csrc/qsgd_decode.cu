@@ -313,90 +313,120 @@ __global__ void __launch_bounds__(kDecodeBlock) decode_warp(const __grid_constan
 }
 
 // ---------------------------------------------------------------------------
-// Fast decoder: d % 4 == 0, d <= kFastDecodeMaxD, s < 1024, 16-byte aligned output,
-// one stream.  Bucket-relative 32-bit reader state: `wp` points at the word that
-// holds the cache's first bit, (hi, lo) are the two cached words, `nx` the word
-// after them, `off` < 32 the bit offset into hi, `left` the bits of the bucket
-// still unread.
+// Fast decoder (one stream; d % 4 == 0, d <= kFastDecodeMaxD, s < 1024, 16-byte
+// aligned output), plain or accumulating.
+//
+// Reader: a 64-bit left-aligned bit buffer -- the next unread bits of the bucket
+// are the top `valid` bits of `buf` (valid >= 32 after every refill) -- plus the
+// next stream word `nx`, loaded one word ahead.  `left` counts the bits of the
+// bucket not yet consumed; a record that would run past the bucket end is only
+// detected when the bucket ends (the staging writes stay inside the segment by
+// construction), so the common path has no per-record bounds checks.
 // ---------------------------------------------------------------------------
-struct FastReader {
-    const uint32_t* wp;
-    const uint32_t* wend;  // one past the last word of the stream
-    uint32_t hi, lo, nx;
-    uint32_t off;
+constexpr uint32_t kFastDecodeMaxD = 4096;
+constexpr uint32_t kFullMask = 0xFFFFFFFFu;
+
+struct BitBuf {
+    const uint32_t* base;  // word holding the bucket's first bit
+    uint32_t wi;           // next word to fetch, relative to base
+    uint32_t wlim;         // words available from base to the end of the stream
+    uint64_t buf;
+    uint32_t valid;
+    uint32_t nx;
     uint32_t left;
-    __device__ __forceinline__ uint32_t ld(const uint32_t* p) const { return p < wend ? __ldg(p) : 0u; }
-    __device__ __forceinline__ void init(const uint32_t* words, uint64_t num_words, uint64_t begin, uint32_t nbits) {
-        wend = words + num_words;
-        wp = words + (begin >> 5);
-        off = static_cast<uint32_t>(begin & 31u);
-        hi = ld(wp);
-        lo = ld(wp + 1);
-        nx = ld(wp + 2);
-        left = nbits;
+    __device__ __forceinline__ uint32_t fetch() {
+        const uint32_t w = wi < wlim ? __ldg(base + wi) : 0u;
+        ++wi;
+        return w;
     }
-    __device__ __forceinline__ uint32_t peek() const { return __funnelshift_l(lo, hi, off); }
-    // consumes n <= 32 bits (the caller checked n <= left)
-    __device__ __forceinline__ void skip(uint32_t n) {
-        off += n;
-        left -= n;
-        if (off >= 32) {
-            off -= 32;
-            hi = lo;
-            lo = nx;
-            ++wp;
-            nx = ld(wp + 2);
+    __device__ __forceinline__ void init(const uint32_t* words, uint64_t num_words, uint64_t begin, uint32_t nbits) {
+        const uint64_t w0 = begin >> 5;
+        base = words + w0;
+        wlim = static_cast<uint32_t>(min(num_words - w0, static_cast<uint64_t>(0xFFFFFFFFu)));
+        wi = 0;
+        const uint32_t a0 = fetch(), a1 = fetch();
+        nx = fetch();
+        const uint32_t sh = static_cast<uint32_t>(begin & 31u);
+        buf = ((static_cast<uint64_t>(a0) << 32) | a1) << sh;
+        valid = 64u - sh;
+        left = nbits;
+        refill();
+    }
+    __device__ __forceinline__ void refill() {
+        if (valid < 32u) {
+            buf |= static_cast<uint64_t>(nx) << (32u - valid);
+            valid += 32u;
+            nx = fetch();
         }
     }
+    // consumes n <= 32 bits
+    __device__ __forceinline__ void consume(uint32_t n) {
+        buf <<= n;
+        valid -= n;
+        left -= n;
+        refill();
+    }
+    __device__ __forceinline__ uint32_t top(uint32_t n) const { return static_cast<uint32_t>(buf >> (64u - n)); }
+    // bit-serial omega for codes the record table does not hold
     __device__ __forceinline__ bool omega(uint32_t& N) {
         uint32_t v = 1;
         for (;;) {
             if (left == 0) return false;
-            const uint32_t bit = peek() >> 31;
-            skip(1);
+            const uint32_t bit = static_cast<uint32_t>(buf >> 63);
+            consume(1);
             if (bit == 0) {
                 N = v;
                 return true;
             }
             if (v > 31 || left < v) return false;
-            const uint32_t rest = peek() >> (32 - v);
-            skip(v);
+            const uint32_t rest = top(v);
+            consume(v);
             v = (1u << v) | rest;
         }
     }
 };
 
-constexpr uint32_t kFastDecodeMaxD = 4096;
+constexpr uint32_t kNoRecord = 0xFFFFFFFFu;  // no record left in the bucket
+constexpr uint32_t kParked = 0xFFFFFFFEu;    // the next record needs the bit-serial path
 
-// Next record: its index (0xFFFFFFFF at the end of the bucket) and value bits.
-// Returns false on a malformed record.
-__device__ __forceinline__ bool fast_next(FastReader& r, const uint32_t* lut, uint32_t m, uint32_t s,
-                                          float scale, uint32_t& next, uint32_t& idx, uint32_t& vbits) {
-    if (r.left == 0) {
-        idx = 0xFFFFFFFFu;
-        return true;
+// Next record through the table: its bucket-local index and value bits, or
+// kParked when the record is longer than the table's window, or kNoRecord at the
+// end of the bucket.  A record that overruns the bucket leaves `left` negative,
+// which the end-of-bucket check reports.
+__device__ __forceinline__ void table_next(BitBuf& r, const uint32_t* lut, float scale, uint32_t& next,
+                                           uint32_t& idx, uint32_t& vbits) {
+    if (static_cast<int32_t>(r.left) <= 0) {
+        idx = kNoRecord;
+        return;
     }
-    const uint32_t e = lut[r.peek() >> (32 - kLutBits)];
+    const uint32_t e = lut[static_cast<uint32_t>(r.buf >> (64 - kLutBits))];
     const uint32_t len = e & 31u;
-    uint32_t gap, k, sign;
-    if (len != 0 && len <= r.left) {
-        r.skip(len);
-        gap = (e >> 6) & 1023u;
-        k = (e >> 16) & 1023u;
-        sign = e >> 31;
-    } else {
-        if (!r.omega(gap) || r.left == 0) return false;
-        sign = r.peek() >> 31;
-        r.skip(1);
-        if (!r.omega(k) || k > s) return false;
+    if (len == 0) {
+        idx = kParked;
+        return;
     }
-    idx = next + gap - 1;
-    if (gap > m || idx >= m) return false;
-    next = idx + 1;
-    vbits = __float_as_uint(__fmul_rn(scale, __uint2float_rn(k))) | (sign << 31);
+    r.consume(len);
+    next += (e >> 6) & 1023u;
+    idx = next - 1;
+    vbits = __float_as_uint(__fmul_rn(scale, __uint2float_rn((e >> 16) & 1023u))) | (e & 0x80000000u);
+}
+
+// The record at the reader through the bit-serial path.  Returns false on a
+// malformed record.
+__device__ __forceinline__ bool slow_next(BitBuf& r, uint32_t s, float scale, uint32_t& next, uint32_t& idx,
+                                       uint32_t& vbits) {
+    uint32_t gap, k;
+    if (!r.omega(gap) || r.left == 0 || gap > 0xFFFFu) return false;
+    const uint32_t sign = static_cast<uint32_t>(r.buf >> 63) << 31;
+    r.consume(1);
+    if (!r.omega(k) || k > s) return false;
+    next += gap;
+    idx = next - 1;
+    vbits = __float_as_uint(__fmul_rn(scale, __uint2float_rn(k))) | sign;
     return true;
 }
 
+template <bool kAccumulate>
 __global__ void __launch_bounds__(kDecodeBlock) decode_fast(const __grid_constant__ DecodeArgs a) {
     extern __shared__ __align__(16) uint32_t smem[];
     uint32_t* lut = smem;
@@ -409,23 +439,27 @@ __global__ void __launch_bounds__(kDecodeBlock) decode_fast(const __grid_constan
     const uint32_t d = a.d;
     const uint64_t ngroups = (a.nb + 31) / 32;
     const uint64_t gwarps = static_cast<uint64_t>(gridDim.x) * kDecWarps;
+    // write-back geometry: step i moves row 2i + (lane >> 4), columns 4 (lane & 15) .. +3
+    const uint32_t wrow = static_cast<uint32_t>(lane >> 4), wcol = static_cast<uint32_t>(lane & 15) * 4;
+    float* row = stage + lane * kStride;
     for (uint64_t g = static_cast<uint64_t>(blockIdx.x) * kDecWarps + warp; g < ngroups; g += gwarps) {
         const uint64_t b = g * 32 + lane;
         const bool live = b < a.nb;
         const uint32_t m = live ? static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - b * d)) : 0u;
+        const bool full_group = (g + 1) * 32 <= a.nb && (g + 1) * 32 * static_cast<uint64_t>(d) <= a.n;
         bool bad = false;
-        FastReader r;
+        BitBuf r;
         r.left = 0;
         float scale = 0.f;
         if (live) {
             const uint64_t begin = st.offsets[b];
             const uint64_t end = st.offsets[b + 1];
-            if (!(end >= begin && end - begin >= 32 && end <= st.num_words * 32 && end - begin < (1ull << 31))) {
+            if (!(end >= begin && end - begin >= 32 && end <= st.num_words * 32 && end - begin < (1ull << 30))) {
                 bad = true;
             } else {
                 r.init(st.words, st.num_words, begin, static_cast<uint32_t>(end - begin));
-                const uint32_t nbits = r.peek();
-                r.skip(32);
+                const uint32_t nbits = r.top(32);
+                r.consume(32);
                 const float norm = __uint_as_float(nbits);
                 if (nbits == 0) {
                     bad = r.left != 0;
@@ -438,30 +472,73 @@ __global__ void __launch_bounds__(kDecodeBlock) decode_fast(const __grid_constan
                 }
             }
         }
-        uint32_t next = 0, pidx = 0xFFFFFFFFu, pval = 0;
-        if (!bad && !fast_next(r, lut, m, a.s, scale, next, pidx, pval)) {
-            bad = true;
-            pidx = 0xFFFFFFFFu;
-        }
-        float* row = stage + lane * kStride;
-        // write-back geometry: iteration i stores row 2i + (lane >> 4), columns 4 (lane & 15)..+3
-        const uint32_t wrow = static_cast<uint32_t>(lane >> 4), wcol = static_cast<uint32_t>(lane & 15) * 4;
-        const bool full_group = (g + 1) * 32 <= a.nb && (g + 1) * 32 * static_cast<uint64_t>(d) <= a.n;
+        uint32_t next = 0, pidx = kNoRecord, pval = 0;
+        if (!bad) table_next(r, lut, scale, next, pidx, pval);
         for (uint32_t lo = 0; lo < d; lo += kSeg) {
-            for (int q = lane; q < 32 * kStride / 4; q += 32)
-                reinterpret_cast<float4*>(stage)[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+            const uint32_t seg_len = min(static_cast<uint32_t>(kSeg), d - lo);
+            const bool vec = full_group && seg_len == kSeg;
+            // --- staging tile: zeros, or the current output (+0.0 turns -0.0 into +0.0)
+            if (kAccumulate) {
+                if (vec) {
+                    const float* src = a.out + (g * 32 + wrow) * d + lo + wcol;
+                    float* dst = stage + wrow * kStride + wcol;
+#pragma unroll 4
+                    for (int i = 0; i < 16; ++i) {
+                        float4 v = *reinterpret_cast<const float4*>(src);
+                        if (a.first_group) {
+                            v.x = __fadd_rn(v.x, 0.0f);
+                            v.y = __fadd_rn(v.y, 0.0f);
+                            v.z = __fadd_rn(v.z, 0.0f);
+                            v.w = __fadd_rn(v.w, 0.0f);
+                        }
+                        *reinterpret_cast<float4*>(dst) = v;
+                        src += 2 * static_cast<uint64_t>(d);
+                        dst += 2 * kStride;
+                    }
+                } else {
+                    for (int rr = 0; rr < 32; ++rr) {
+                        const uint64_t bb = g * 32 + rr;
+                        const uint32_t mm = bb < a.nb ? static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - bb * d)) : 0u;
+                        for (uint32_t c = lane; c < kSeg; c += 32) {
+                            float v = 0.f;
+                            if (lo + c < mm) {
+                                v = a.out[bb * d + lo + c];
+                                if (a.first_group) v = __fadd_rn(v, 0.0f);
+                            }
+                            stage[rr * kStride + c] = v;
+                        }
+                    }
+                }
+            } else {
+                for (int q = lane; q < 32 * kStride / 4; q += 32)
+                    reinterpret_cast<float4*>(stage)[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
             __syncwarp();
+            // --- scatter this segment's records -------------------------------
+            // Lanes whose next record is too long for the table park; the
+            // bit-serial path runs only when no lane has table work left, so the
+            // parked lanes of a warp are resolved together.
             const uint32_t hi = lo + kSeg;
-            while (pidx < hi) {
-                row[pidx - lo] = __uint_as_float(pval);
-                if (!fast_next(r, lut, m, a.s, scale, next, pidx, pval)) {
-                    bad = true;
-                    pidx = 0xFFFFFFFFu;
+            for (;;) {
+                const bool place = pidx < hi;
+                if (__any_sync(kFullMask, place)) {
+                    if (place) {
+                        float* dst = row + (pidx - lo);
+                        *dst = kAccumulate ? __fadd_rn(*dst, __uint_as_float(pval)) : __uint_as_float(pval);
+                        table_next(r, lut, scale, next, pidx, pval);
+                    }
+                } else if (__any_sync(kFullMask, pidx == kParked)) {
+                    if (pidx == kParked && !slow_next(r, a.s, scale, next, pidx, pval)) {
+                        bad = true;
+                        pidx = kNoRecord;
+                    }
+                } else {
+                    break;
                 }
             }
             __syncwarp();
-            const uint32_t seg_len = min(static_cast<uint32_t>(kSeg), d - lo);
-            if (full_group && seg_len == kSeg) {
+            // --- write the tile back: row r is bucket g*32 + r -----------------
+            if (vec) {
                 float* dst = a.out + (g * 32 + wrow) * d + lo + wcol;
                 const float* src = stage + wrow * kStride + wcol;
 #pragma unroll 4
@@ -481,26 +558,29 @@ __global__ void __launch_bounds__(kDecodeBlock) decode_fast(const __grid_constan
             }
             __syncwarp();
         }
+        // every record index below m, and the bucket consumed exactly
+        if (live && !bad && (next > m || r.left != 0 || pidx != kNoRecord)) bad = true;
         if (bad) atomicOr(a.status, QSGD_ST_BAD_STREAM);
     }
 }
 
+template <bool kAccumulate>
 cudaError_t launch_fast_decode(const DecodeArgs& a, cudaStream_t stream) {
     const size_t smem = kLut * sizeof(uint32_t) + static_cast<size_t>(kDecWarps) * 32 * kStride * sizeof(float);
     static bool attr_set[64] = {};
     int dev = 0, sms = 0, per_sm = 0;
     cudaGetDevice(&dev);
     if (dev < 64 && !attr_set[dev]) {
-        cudaFuncSetAttribute(decode_fast, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+        cudaFuncSetAttribute(decode_fast<kAccumulate>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
         attr_set[dev] = true;
     }
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_fast, kDecodeBlock, smem);
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_fast<kAccumulate>, kDecodeBlock, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const uint64_t groups = (a.nb + 31) / 32;
     const uint64_t blocks = std::min<uint64_t>((groups + kDecWarps - 1) / kDecWarps, static_cast<uint64_t>(sms) * per_sm);
-    decode_fast<<<static_cast<unsigned>(blocks), kDecodeBlock, smem, stream>>>(a);
+    decode_fast<kAccumulate><<<static_cast<unsigned>(blocks), kDecodeBlock, smem, stream>>>(a);
     return cudaGetLastError();
 }
 
@@ -531,9 +611,9 @@ cudaError_t launch(const DecodeArgs& a, cudaStream_t stream) {
 
 cudaError_t launch_decode(const DecodeArgs& a, bool accumulate, cudaStream_t stream) {
     if (a.nb == 0) return cudaSuccess;
-    if (!accumulate && a.K == 1 && a.d % 4 == 0 && a.d <= kFastDecodeMaxD && a.s < 1024 &&
-        (reinterpret_cast<uintptr_t>(a.out) & 15u) == 0 && kSeg == 64)
-        return launch_fast_decode(a, stream);
+    if (a.K == 1 && a.d % 4 == 0 && a.d <= kFastDecodeMaxD && a.s < 1024 &&
+        (reinterpret_cast<uintptr_t>(a.out) & 15u) == 0)
+        return accumulate ? launch_fast_decode<true>(a, stream) : launch_fast_decode<false>(a, stream);
     return accumulate ? launch<true>(a, stream) : launch<false>(a, stream);
 }
 
