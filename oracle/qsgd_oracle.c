@@ -288,6 +288,9 @@ static int parse_bucket(const uint32_t* words, uint64_t begin, uint64_t end, uin
     *norm_out = norm;
     if (!isfinite(norm) || signbit(norm)) return -1;
     if (norm == 0.0f) return pos == end ? 0 : -1;
+    /* a norm whose scale norm/s rounds to zero: no conforming encoder sends records
+       under it (s/norm overflows, so the bucket goes out as a zero bucket) */
+    if (norm / (float)s == 0.0f && pos < end) return -1;
     int64_t idx = -1;
     while (pos < end) {
         uint64_t gap, k;

@@ -134,6 +134,24 @@ def test_decode_accumulate_hand_values(oracle_lib):
     assert res.view(np.uint32).tolist() == expect.view(np.uint32).tolist()
 
 
+def test_underflowing_scale_with_records_is_flagged(oracle_lib):
+    # norm = 2^-149 (bit pattern 1) and s = 8: fl(norm / s) = 0, and s / norm overflows,
+    # so no encoder sends records under this norm.  One record gap 1, sign 0, k 1 = "000".
+    s = 8
+    tiny = bits_to_words("0" * 31 + "1" + "000")
+    off = np.array([0, 35], dtype=np.uint64)
+    out, st = oracle_lib.decode(tiny, off, 1, 1, s)
+    assert st & oracle_mod.ST_BAD_STREAM
+    assert np.float32(np.uint32(1).view(np.float32)) / np.float32(s) == 0
+    # the same norm with no record is a valid (all-zero) bucket
+    out, st = oracle_lib.decode(bits_to_words("0" * 31 + "1"), np.array([0, 32], np.uint64), 1, 1, s)
+    assert st == 0 and out.view(np.uint32).tolist() == [0]
+    # the smallest normal norm 2^-126 keeps a non-zero scale: the record decodes
+    normal = bits_to_words("00000000100000000000000000000000" + "000")
+    out, st = oracle_lib.decode(normal, off, 1, 1, s)
+    assert st == 0 and out[0] == np.float32(2.0 ** -126) / np.float32(s) and out[0] > 0
+
+
 def test_decode_accumulate_negative_zero_becomes_positive(oracle_lib):
     # -0.0 + (+0.0) = +0.0: a coordinate off every support turns -0 into +0
     z = bits_to_words("0" * 32)
