@@ -34,10 +34,11 @@ sys.path.insert(0, ROOT)
 METRIC = "QSGD encode & decode GB/s of fp32 gradient input; % of B200 HBM roofline"
 FALLBACK_HBM_GBS = 6650.0
 
-# DRAM traffic of the dominant kernel from one ncu capture (dram__bytes_read.sum +
-# dram__bytes_write.sum per launch, full workload), with the hash of the kernel
-# sources it was taken on; reported as null once the sources differ.
-TRAFFIC = {"kernel": None, "bytes_per_launch": None, "sources_sha256": None}
+# DRAM traffic per launch of each phase's kernel (dram__bytes_read.sum +
+# dram__bytes_write.sum) from one ncu capture of this workload, with the hash of
+# the kernel sources it was taken on; reported as null once the sources differ.
+TRAFFIC = {"bytes_per_launch": {"encode": None, "decode": None, "decode_accumulate": None},
+           "sources_sha256": None}
 
 
 def sources_sha256() -> str:
@@ -365,8 +366,8 @@ def run_ours(args, w):
     dominant = max(phases, key=lambda k: phases[k]["ms"])
     dom = phases[dominant]
     traffic = None
-    if TRAFFIC["bytes_per_launch"] is not None and TRAFFIC["sources_sha256"] == sources_sha256():
-        traffic = TRAFFIC["bytes_per_launch"]
+    if TRAFFIC["sources_sha256"] == sources_sha256():
+        traffic = TRAFFIC["bytes_per_launch"][dominant]
 
     result = {
         "metric": METRIC,
@@ -385,9 +386,9 @@ def run_ours(args, w):
         "bits_per_coord": total_bits / n,
         "compressed_bytes": comp_bytes,
         "phases": phases,
-        "roofline": {"bound": "hbm", "kernel": {"encode": "qsgd encode (encode_fast<4>)",
-                                                  "decode": "qsgd decode (decode_buckets<false>)",
-                                                  "decode_accumulate": "qsgd decode_accumulate"}[dominant],
+        "roofline": {"bound": "hbm", "kernel": {"encode": "encode_fast<4, true> (qsgd_encode)",
+                                                  "decode": "decode_fast<false> (qsgd_decode)",
+                                                  "decode_accumulate": "decode_fast<true> (qsgd_decode_accumulate)"}[dominant],
                      "achieved": dom["algorithmic_gbs"], "peak": peak, "unit": "GB/s",
                      "frac": dom["algorithmic_gbs"] / peak, "traffic": traffic,
                      "peak_source": "%s hbm_gbs (burst copy)" % peak_kind,

@@ -32,7 +32,8 @@ constexpr int kLutBits = 12;
 constexpr int kLut = 1 << kLutBits;
 
 // Record table entry for a 12-bit window: [4:0] record length (0: not complete in
-// 12 bits or k > s), [15:6] gap, [25:16] k, [31] sign.
+// 12 bits or k > s), [5] the window holds a complete record with k > s, [15:6] gap,
+// [25:16] k, [31] sign.
 __device__ __forceinline__ bool omega_from_window(uint32_t w, int nbits, int& pos, uint32_t& value) {
     uint32_t v = 1;
     for (;;) {
@@ -57,9 +58,12 @@ __device__ void build_record_lut(uint32_t* lut, uint32_t s, int tid, int nthread
         if (omega_from_window(static_cast<uint32_t>(w), kLutBits, pos, gap) && pos < kLutBits) {
             const uint32_t sign = (static_cast<uint32_t>(w) >> (kLutBits - 1 - pos)) & 1u;
             ++pos;
-            if (omega_from_window(static_cast<uint32_t>(w), kLutBits, pos, k) && k <= s && gap < 1024 &&
-                k < 1024)
-                e = static_cast<uint32_t>(pos) | (gap << 6) | (k << 16) | (sign << 31);
+            if (omega_from_window(static_cast<uint32_t>(w), kLutBits, pos, k)) {
+                if (k <= s && gap < 1024 && k < 1024)
+                    e = static_cast<uint32_t>(pos) | (gap << 6) | (k << 16) | (sign << 31);
+                else if (k > s)
+                    e = 32u;
+            }
         }
         lut[w] = e;
     }
@@ -216,7 +220,8 @@ __global__ void __launch_bounds__(kDecodeBlock) decode_warp(const __grid_constan
                         bad = true;
                     } else {
                         ls.scale = __fdiv_rn(norm, __uint2float_rn(a.s));
-                        bad = !next_record(r, lut, m, a.s, ls.next, rec);
+                        // a scale that rounds to zero carries no records (wire format)
+                        bad = !(ls.scale > 0.f) ? r.pos != end : !next_record(r, lut, m, a.s, ls.next, rec);
                     }
                     ls.pos = r.pos;
                 }
@@ -386,6 +391,9 @@ struct BitBuf {
     }
 };
 
+// The decoders' loops end by construction (each step consumes at least one bit of a
+// bounded range); kLoopGuard is a second, explicit bound that marks the bucket bad.
+constexpr uint32_t kLoopGuard = 1u << 20;
 constexpr uint32_t kNoRecord = 0xFFFFFFFFu;  // no record left in the bucket
 constexpr uint32_t kParked = 0xFFFFFFFEu;    // the next record needs the bit-serial path
 
@@ -469,6 +477,10 @@ __global__ void __launch_bounds__(kDecodeBlock) decode_fast(const __grid_constan
                     r.left = 0;
                 } else {
                     scale = __fdiv_rn(norm, fs);
+                    if (!(scale > 0.f) && r.left != 0) {  // a zero scale carries no records
+                        bad = true;
+                        r.left = 0;
+                    }
                 }
             }
         }
@@ -480,21 +492,18 @@ __global__ void __launch_bounds__(kDecodeBlock) decode_fast(const __grid_constan
             // --- staging tile: zeros, or the current output (+0.0 turns -0.0 into +0.0)
             if (kAccumulate) {
                 if (vec) {
+                    // all 16 copies in flight at once; the first group's +0.0 is
+                    // applied at write-back instead ((x + 0) + v == (x + v) + 0 for
+                    // every x and every v, -0.0 included)
                     const float* src = a.out + (g * 32 + wrow) * d + lo + wcol;
-                    float* dst = stage + wrow * kStride + wcol;
-#pragma unroll 4
+                    uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(stage + wrow * kStride + wcol));
+#pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        float4 v = *reinterpret_cast<const float4*>(src);
-                        if (a.first_group) {
-                            v.x = __fadd_rn(v.x, 0.0f);
-                            v.y = __fadd_rn(v.y, 0.0f);
-                            v.z = __fadd_rn(v.z, 0.0f);
-                            v.w = __fadd_rn(v.w, 0.0f);
-                        }
-                        *reinterpret_cast<float4*>(dst) = v;
+                        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src) : "memory");
                         src += 2 * static_cast<uint64_t>(d);
-                        dst += 2 * kStride;
+                        dst += 2 * kStride * sizeof(float);
                     }
+                    asm volatile("cp.async.wait_all;\n" ::: "memory");
                 } else {
                     for (int rr = 0; rr < 32; ++rr) {
                         const uint64_t bb = g * 32 + rr;
@@ -519,9 +528,13 @@ __global__ void __launch_bounds__(kDecodeBlock) decode_fast(const __grid_constan
             // bit-serial path runs only when no lane has table work left, so the
             // parked lanes of a warp are resolved together.
             const uint32_t hi = lo + kSeg;
-            for (;;) {
+            for (uint32_t it = 0;; ++it) {
                 const bool place = pidx < hi;
-                if (__any_sync(kFullMask, place)) {
+                if (it == kLoopGuard) {
+                    bad = true;
+                    pidx = kNoRecord;
+                }
+                if (__any_sync(kFullMask, place) && it < kLoopGuard) {
                     if (place) {
                         float* dst = row + (pidx - lo);
                         *dst = kAccumulate ? __fadd_rn(*dst, __uint_as_float(pval)) : __uint_as_float(pval);
@@ -541,9 +554,17 @@ __global__ void __launch_bounds__(kDecodeBlock) decode_fast(const __grid_constan
             if (vec) {
                 float* dst = a.out + (g * 32 + wrow) * d + lo + wcol;
                 const float* src = stage + wrow * kStride + wcol;
+                const bool plus_zero = kAccumulate && a.first_group;
 #pragma unroll 4
                 for (int i = 0; i < 16; ++i) {
-                    *reinterpret_cast<float4*>(dst) = *reinterpret_cast<const float4*>(src);
+                    float4 v = *reinterpret_cast<const float4*>(src);
+                    if (plus_zero) {
+                        v.x = __fadd_rn(v.x, 0.0f);
+                        v.y = __fadd_rn(v.y, 0.0f);
+                        v.z = __fadd_rn(v.z, 0.0f);
+                        v.w = __fadd_rn(v.w, 0.0f);
+                    }
+                    *reinterpret_cast<float4*>(dst) = v;
                     dst += 2 * static_cast<uint64_t>(d);
                     src += 2 * kStride;
                 }
@@ -562,6 +583,327 @@ __global__ void __launch_bounds__(kDecodeBlock) decode_fast(const __grid_constan
         if (live && !bad && (next > m || r.left != 0 || pidx != kNoRecord)) bad = true;
         if (bad) atomicOr(a.status, QSGD_ST_BAD_STREAM);
     }
+}
+
+// ---------------------------------------------------------------------------
+// Split decoder: P lanes per bucket (one stream; the fast decoder's conditions).
+//
+// One lane per bucket leaves a B200 with a few hundred latency-bound chains of
+// dependent table lookups.  Here the record bits [R0, B1) of a bucket (after the
+// 32-bit norm) are cut into P equal parts and lane j of the bucket's P lanes parses
+// from the start S_j of part j.  Only S_0 is known to be a record boundary; the
+// others start mid-record, but a prefix code of this kind falls back into step
+// with the true record boundaries within a few records.  So:
+//   1. each lane parses its part speculatively up to the first record start
+//      E_j >= S_{j+1}, summing the gaps G_j; an invalid or overrunning record
+//      counts as one bit with gap 0, so the parse is a fixed function of its start
+//      position and never passes B1;
+//   2. lane j continues its parse from E_j ("walker") while lane j+1 parses its own
+//      part again from S_{j+1} ("follower"); whichever of the two is behind takes
+//      the next step, until they stand on the same bit X_j.  The walker sums the
+//      gaps WG_j of its records in [E_j, X_j), the follower the gaps FG_{j+1} of
+//      lane j+1's records in [S_{j+1}, X_j).  From X_j on the two parses coincide,
+//      so by induction from S_0 the true records are lane j's records in
+//      [X_{j-1}, X_j) (X_{-1} = S_0, X_{P-1} = B1), whose gaps sum to
+//      T_j = G_j - FG_j + WG_j;
+//   3. an exclusive scan of T_j over the P lanes gives each lane the index of its
+//      first coordinate, so lane j owns the columns [base_j, base_j + T_j) (the
+//      last lane up to the bucket end).  It initialises them (16-byte stores) and
+//      decodes its range [X_{j-1}, X_j) strictly, storing each value straight to
+//      its column; no two lanes write the same column and nothing is staged.
+// The strict pass in 3 checks everything the serial decoder checks, and that each
+// lane's records end exactly at X_j with gaps summing to T_j; ranges that tile
+// [R0, B1) and parse strictly are the serial parse, so the output is the serial
+// decoder's.  A bucket whose walks do not meet within kMaxMergeSteps, or meet out of
+// order, or that is too short to split, is decoded whole by its lane 0.
+// ---------------------------------------------------------------------------
+constexpr uint32_t kMinPartBits = 64;
+constexpr int kMaxMergeSteps = 1024;
+
+// One step of a speculative parse (left > 0): a valid record through the table or
+// the bit-serial path, else one bit with gap 0.
+__device__ __forceinline__ void spec_step(BitBuf& r, const uint32_t* lut, uint32_t s, uint32_t& gsum) {
+    const uint32_t e = lut[static_cast<uint32_t>(r.buf >> (64 - kLutBits))];
+    uint32_t len = e & 31u;
+    uint32_t gap = (e >> 6) & 1023u;
+    if (len == 0 || len > r.left) {
+        len = 1;
+        gap = 0;
+        if ((e & 63u) == 0) {  // longer than the table window
+            BitBuf t = r;
+            uint32_t g, k;
+            if (t.omega(g) && t.left != 0) {
+                t.consume(1);
+                if (t.omega(k) && k <= s) {
+                    r = t;
+                    gsum += g;
+                    return;
+                }
+            }
+        }
+    }
+    r.consume(len);
+    gsum += gap;
+}
+
+// 32 stream bits starting at bit `pos` (zeros past the stream).
+__device__ __forceinline__ uint32_t read32(const uint32_t* words, uint64_t num_words, uint64_t pos) {
+    const uint64_t w0 = pos >> 5;
+    const uint32_t a0 = w0 < num_words ? __ldg(words + w0) : 0u;
+    const uint32_t a1 = w0 + 1 < num_words ? __ldg(words + w0 + 1) : 0u;
+    return __funnelshift_l(a1, a0, static_cast<uint32_t>(pos & 31u));
+}
+
+#ifndef QSGD_SPLIT_BATCH
+#define QSGD_SPLIT_BATCH 4
+#endif
+constexpr int kBatch = QSGD_SPLIT_BATCH;  // records a lane stores per step of the split decoder
+
+// Columns [lo, hi) of one bucket row g (16-byte aligned): zeros, or x + 0.
+template <bool kAccumulate>
+__device__ __forceinline__ void init_columns(float* g, uint32_t lo, uint32_t hi) {
+    if (lo >= hi) return;
+    const uint32_t a4 = min((lo + 3u) & ~3u, hi);
+    const uint32_t b4 = max(a4, hi & ~3u);
+    for (uint32_t c = lo; c < a4; ++c) g[c] = kAccumulate ? __fadd_rn(g[c], 0.0f) : 0.0f;
+    if (kAccumulate) {
+        for (uint32_t c = a4; c < b4; c += 16) {
+            float4 v[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                if (c + 4 * q < b4) v[q] = *reinterpret_cast<const float4*>(g + c + 4 * q);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                if (c + 4 * q < b4) {
+                    v[q].x = __fadd_rn(v[q].x, 0.0f);
+                    v[q].y = __fadd_rn(v[q].y, 0.0f);
+                    v[q].z = __fadd_rn(v[q].z, 0.0f);
+                    v[q].w = __fadd_rn(v[q].w, 0.0f);
+                    *reinterpret_cast<float4*>(g + c + 4 * q) = v[q];
+                }
+            }
+        }
+    } else {
+        for (uint32_t c = a4; c < b4; c += 4) *reinterpret_cast<float4*>(g + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    for (uint32_t c = b4; c < hi; ++c) g[c] = kAccumulate ? __fadd_rn(g[c], 0.0f) : 0.0f;
+}
+
+template <bool kAccumulate, int P>
+__global__ void __launch_bounds__(kDecodeBlock) decode_split(const __grid_constant__ DecodeArgs a) {
+    static_assert(P >= 2 && P <= 8 && (P & (P - 1)) == 0, "P is 2, 4 or 8");
+    extern __shared__ __align__(16) uint32_t smem[];
+    uint32_t* lut = smem;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    build_record_lut(lut, a.s, tid, kDecodeBlock);
+    __syncthreads();
+    const StreamRef st = a.streams[0];
+    const float fs = __uint2float_rn(a.s);
+    const uint32_t d = a.d;
+    constexpr int kPerWarp = 32 / P;
+    const uint32_t j = static_cast<uint32_t>(lane) & (P - 1);
+    const uint32_t gmask = ((1u << P) - 1u) << (static_cast<uint32_t>(lane) & ~static_cast<uint32_t>(P - 1));
+    const uint64_t ngroups = (a.nb + kPerWarp - 1) / kPerWarp;
+    const uint64_t gwarps = static_cast<uint64_t>(gridDim.x) * kDecWarps;
+    for (uint64_t g = static_cast<uint64_t>(blockIdx.x) * kDecWarps + warp; g < ngroups; g += gwarps) {
+        const uint64_t b = g * kPerWarp + static_cast<uint64_t>(lane / P);
+        const bool live = b < a.nb;
+        const uint32_t m = live ? static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - b * d)) : 0u;
+        bool bad = false;
+        uint64_t R0 = 0;
+        uint32_t L = 0;  // record bits of the bucket
+        float scale = 0.f;
+        if (live) {
+            const uint64_t begin = st.offsets[b];
+            const uint64_t end = st.offsets[b + 1];
+            if (!(end >= begin && end - begin >= 32 && end <= st.num_words * 32 && end - begin < (1ull << 30))) {
+                bad = true;
+            } else {
+                const uint32_t nbits = read32(st.words, st.num_words, begin);
+                const float norm = __uint_as_float(nbits);
+                R0 = begin + 32;
+                L = static_cast<uint32_t>(end - begin - 32);
+                if (nbits == 0) {
+                    bad = L != 0;
+                    L = 0;
+                } else if (!(isfinite(norm) && norm > 0.f)) {
+                    bad = true;
+                    L = 0;
+                } else {
+                    scale = __fdiv_rn(norm, fs);
+                    if (!(scale > 0.f) && L != 0) {  // a zero scale carries no records
+                        bad = true;
+                        L = 0;
+                    }
+                }
+            }
+        }
+        const bool split = L >= P * kMinPartBits;  // the same in all P lanes of a bucket
+        const uint32_t s_lo = split ? static_cast<uint32_t>(static_cast<uint64_t>(L) * j / P) : 0u;
+        const uint32_t s_hi = split ? static_cast<uint32_t>(static_cast<uint64_t>(L) * (j + 1) / P) : L;
+
+        // --- 1. speculative parse of part j (`left` counts the bits to B1) ------
+        BitBuf w;
+        w.left = 0;
+        uint32_t G = 0;
+        if (split) w.init(st.words, st.num_words, R0 + s_lo, L - s_lo);
+        const uint32_t lim = L - s_hi;
+        for (uint32_t it = 0;; ++it) {
+            const bool go = split && w.left > lim;
+            if (!__any_sync(kFullMask, go)) break;
+            if (it == kLoopGuard) {
+                bad = true;
+                break;
+            }
+            if (go) spec_step(w, lut, a.s, G);
+        }
+
+        // --- 2. merge walks: walker of lane j against follower of lane j+1 ------
+        const bool has_w = split && j < P - 1;
+        const bool has_f = split && j > 0;
+        BitBuf f;
+        f.left = 0;
+        if (has_f) f.init(st.words, st.num_words, R0 + s_lo, L - s_lo);
+        if (!has_w) w.left = 0;
+        uint32_t WG = 0, FG = 0;
+        bool met = true;
+        for (int it = 0;; ++it) {
+            const uint32_t y_next = __shfl_down_sync(kFullMask, f.left, 1, P);
+            const uint32_t x_prev = __shfl_up_sync(kFullMask, w.left, 1, P);
+            const bool wa = has_w && w.left > y_next;  // the walker is behind
+            const bool fa = has_f && f.left > x_prev;  // the follower is behind
+            if (!__any_sync(kFullMask, wa || fa)) break;
+            if (it == kMaxMergeSteps) {
+                met = !(wa || fa);
+                break;
+            }
+            if (wa) spec_step(w, lut, a.s, WG);
+            if (fa) spec_step(f, lut, a.s, FG);
+        }
+        // lane j's range [X_{j-1}, X_j) as `left` values
+        const uint32_t x_lo = has_f ? f.left : L;
+        const uint32_t x_hi = has_w ? w.left : 0u;
+        const bool ok = met && x_lo >= x_hi;
+        // (the ballot is taken by all lanes: never inside a short-circuit condition)
+        const uint32_t not_ok = __ballot_sync(kFullMask, !ok);
+        const bool serial = !split || (not_ok & gmask) != 0u;
+        const uint32_t T = G - FG + WG;
+        uint32_t incl = T;
+#pragma unroll
+        for (int o = 1; o < P; o <<= 1) {
+            const uint32_t t = __shfl_up_sync(kFullMask, incl, o, P);
+            if (j >= static_cast<uint32_t>(o)) incl += t;
+        }
+        uint32_t own_lo, own_hi, r_start, r_bits;
+        if (serial) {
+            own_lo = j == 0 ? 0u : m;
+            own_hi = m;
+            r_start = 0;
+            r_bits = j == 0 ? L : 0u;
+        } else {
+            own_lo = min(incl - T, m);
+            own_hi = j == P - 1 ? m : max(own_lo, min(incl, m));
+            r_start = L - x_lo;
+            r_bits = x_lo - x_hi;
+        }
+
+        // --- 3. strict decode of the lane's range, stored straight to its columns
+        // The lane first initialises the columns it owns (zeros; for the first
+        // stream of an accumulation x + 0, which turns -0.0 into +0.0 off the
+        // support and changes nothing under a record, whose value is never zero),
+        // then writes its records; no other lane touches these columns.
+        float* gout = a.out + (live ? b * d : 0);
+        if (!kAccumulate || a.first_group) init_columns<kAccumulate>(gout, own_lo, own_hi);
+        BitBuf r;
+        r.left = 0;
+        if (r_bits != 0) r.init(st.words, st.num_words, R0 + r_start, r_bits);
+        uint32_t next = own_lo, pidx = kNoRecord, pval = 0;
+        table_next(r, lut, scale, next, pidx, pval);
+        for (uint32_t it = 0;; ++it) {
+            if (it == kLoopGuard) {
+                bad = true;
+                pidx = kNoRecord;
+            }
+            const bool ready = pidx < kParked;
+            if (__any_sync(kFullMask, ready) && it < kLoopGuard) {
+                if (ready) {
+                    // up to kBatch records through the table, then their stores (and,
+                    // accumulating, their loads) issued together
+                    uint32_t bi[kBatch];
+                    uint32_t bv[kBatch];
+                    uint32_t cnt = 0;
+#pragma unroll
+                    for (int t = 0; t < kBatch; ++t) {
+                        if (pidx < kParked) {
+                            if (pidx >= own_hi) {  // outside the lane's columns
+                                bad = true;
+                                pidx = kNoRecord;
+                            } else {
+                                bi[t] = pidx;
+                                bv[t] = pval;
+                                cnt = t + 1;
+                                table_next(r, lut, scale, next, pidx, pval);
+                            }
+                        }
+                    }
+                    if (kAccumulate) {
+                        float x[kBatch];
+#pragma unroll
+                        for (int t = 0; t < kBatch; ++t)
+                            if (t < static_cast<int>(cnt)) x[t] = gout[bi[t]];
+#pragma unroll
+                        for (int t = 0; t < kBatch; ++t)
+                            if (t < static_cast<int>(cnt)) gout[bi[t]] = __fadd_rn(x[t], __uint_as_float(bv[t]));
+                    } else {
+#pragma unroll
+                        for (int t = 0; t < kBatch; ++t)
+                            if (t < static_cast<int>(cnt)) gout[bi[t]] = __uint_as_float(bv[t]);
+                    }
+                }
+            } else if (__any_sync(kFullMask, pidx == kParked)) {
+                if (pidx == kParked && !slow_next(r, a.s, scale, next, pidx, pval)) {
+                    bad = true;
+                    pidx = kNoRecord;
+                }
+            } else {
+                break;
+            }
+        }
+        // every record stored, the range consumed exactly, the gaps as scanned
+        if (live && !bad) {
+            if (pidx != kNoRecord || r.left != 0 || next > m) bad = true;
+            if (!serial && j < P - 1 && next != incl) bad = true;
+        }
+        if (bad) atomicOr(a.status, QSGD_ST_BAD_STREAM);
+    }
+}
+
+template <bool kAccumulate, int P>
+cudaError_t launch_split_decode(const DecodeArgs& a, cudaStream_t stream) {
+    const size_t smem = kLut * sizeof(uint32_t);
+    static bool attr_set[64] = {};
+    int dev = 0, sms = 0, per_sm = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr_set[dev]) {
+        cudaFuncSetAttribute(decode_split<kAccumulate, P>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+        attr_set[dev] = true;
+    }
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_split<kAccumulate, P>,
+                                                                  kDecodeBlock, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    const uint64_t groups = (a.nb + 32 / P - 1) / (32 / P);
+    const uint64_t blocks = std::min<uint64_t>((groups + kDecWarps - 1) / kDecWarps, static_cast<uint64_t>(sms) * per_sm);
+    decode_split<kAccumulate, P><<<static_cast<unsigned>(blocks), kDecodeBlock, smem, stream>>>(a);
+    return cudaGetLastError();
+}
+
+template <bool kAccumulate>
+cudaError_t launch_split_decode_p(const DecodeArgs& a, cudaStream_t stream) {
+    if (a.d >= 1024) return launch_split_decode<kAccumulate, 8>(a, stream);
+    if (a.d >= 256) return launch_split_decode<kAccumulate, 4>(a, stream);
+    return launch_split_decode<kAccumulate, 2>(a, stream);
 }
 
 template <bool kAccumulate>
@@ -611,8 +953,27 @@ cudaError_t launch(const DecodeArgs& a, cudaStream_t stream) {
 
 cudaError_t launch_decode(const DecodeArgs& a, bool accumulate, cudaStream_t stream) {
     if (a.nb == 0) return cudaSuccess;
-    if (a.K == 1 && a.d % 4 == 0 && a.d <= kFastDecodeMaxD && a.s < 1024 &&
-        (reinterpret_cast<uintptr_t>(a.out) & 15u) == 0)
+    const bool fast = a.d % 4 == 0 && a.d <= kFastDecodeMaxD && a.s < 1024 &&
+                      (reinterpret_cast<uintptr_t>(a.out) & 15u) == 0;
+#ifndef QSGD_NO_SPLIT_DECODE
+    if (fast && a.d >= 128) {
+        if (a.K == 1)
+            return accumulate ? launch_split_decode_p<true>(a, stream) : launch_split_decode_p<false>(a, stream);
+        // several streams (decode-accumulate): one launch per stream, in stream
+        // order on the one CUDA stream, so every coordinate still sees its adds
+        // left to right; between launches the output stays in L2
+        DecodeArgs one = a;
+        one.K = 1;
+        for (int j = 0; j < a.K; ++j) {
+            one.streams[0] = a.streams[j];
+            one.first_group = a.first_group && j == 0;
+            const cudaError_t e = launch_split_decode_p<true>(one, stream);
+            if (e != cudaSuccess) return e;
+        }
+        return cudaSuccess;
+    }
+#endif
+    if (a.K == 1 && fast)
         return accumulate ? launch_fast_decode<true>(a, stream) : launch_fast_decode<false>(a, stream);
     return accumulate ? launch<true>(a, stream) : launch<false>(a, stream);
 }

@@ -46,14 +46,18 @@ __device__ __forceinline__ uint4 philox4x32_10(uint64_t j, PhiloxKey key) {
 // ---------------------------------------------------------------------------
 // Quantiser of one coordinate (definition paragraph):
 //   t = |v| * (s/||v||), l = floor(t), p = t - l, k = l + [u < p], clamped to s.
-// floor(t) is a round-down conversion to integer (t < 2^23, every step exact);
+// floor(t) comes from one round-down add: for 0 <= t < 2^23 the sum t + 2^23 lies
+// in [2^23, 2^24), where fp32 spacing is 1, so rounding it down gives exactly
+// 2^23 + floor(t); its low mantissa bits are floor(t) and subtracting 2^23 back is
+// exact.  p = t - floor(t) is exact (Sterbenz for t >= 1, trivially below).
 // u = floor(r / 2^9) * 2^-23 is built exactly as (1 + u) - 1.
 // Returns k; the sign is handled by the caller.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t quantize_level(float v, float sinv, uint32_t r, uint32_t s) {
     const float t = __fmul_rn(fabsf(v), sinv);
-    const uint32_t l = __float2uint_rd(t);             // floor(t), exact for 0 <= t < 2^23
-    const float p = __fsub_rn(t, __uint2float_rn(l));  // exact
+    const float f = __fadd_rd(t, 8388608.0f);                 // 2^23 + floor(t)
+    const uint32_t l = __float_as_uint(f) - 0x4B000000u;      // floor(t)
+    const float p = __fsub_rn(t, __fsub_rn(f, 8388608.0f));   // exact
     const float u = __fsub_rn(__uint_as_float(0x3F800000u | (r >> 9)), 1.0f);
     const uint32_t k = l + (u < p ? 1u : 0u);
     return k < s ? k : s;

@@ -37,6 +37,11 @@ CASES = [
     ("normal", 513, 512, 16),
     ("normal", 20_000, 512, 1 << 22),      # largest s
     ("normal", 20_000, 100, 7),            # d < 128: general
+    # decoder with P lanes per bucket: P = 2 (d < 256, d not a multiple of 64),
+    # P = 8 (d >= 1024), and sparse buckets too short to split (decoded whole)
+    ("normal", 100_000, 132, 3),
+    ("normal", 200_000, 2048, 64),
+    ("heavy_tailed_sparse", 300_000, 512, 2),
 ]
 
 

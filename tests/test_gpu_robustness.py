@@ -53,7 +53,7 @@ def _decode_guarded(words, offs, n, d, s, accumulate=False):
 @pytest.mark.parametrize("d", [512, 3, 8192])
 @pytest.mark.parametrize("accumulate", [False, True])
 @pytest.mark.parametrize("kind", ["truncate", "swap", "beyond_stream", "short_bucket", "nan_norm",
-                                  "negative_norm", "level_above_s"])
+                                  "negative_norm", "level_above_s", "underflowing_scale"])
 def test_flagged_corruption(kind, d, accumulate):
     n, s = 50_000, 8
     enc, words, offs = _encode(n, d, s)
@@ -67,7 +67,7 @@ def test_flagged_corruption(kind, d, accumulate):
         offs[nb] = np.uint64(words.size * 32 + 64)
     elif kind == "short_bucket":
         offs[b + 1] = offs[b] + np.uint64(16)
-    elif kind in ("nan_norm", "negative_norm", "level_above_s"):
+    elif kind in ("nan_norm", "negative_norm", "level_above_s", "underflowing_scale"):
         # rebuild bucket b as a hand-made bucket of exactly 32 + len bits
         start = int(offs[b])
         end = int(offs[b + 1])
@@ -76,6 +76,9 @@ def test_flagged_corruption(kind, d, accumulate):
             body = "01111111110000000000000000000000"
         elif kind == "negative_norm":
             body = "10111111100000000000000000000000"  # -1.0f with records after it
+        elif kind == "underflowing_scale":
+            # norm 2^-149: norm / s rounds to zero; record gap 1, sign 1, k 1
+            body = "0" * 31 + "1" + "0" + "1" + "0"
         else:
             # norm 1.0, record gap 1, sign 0, k = 9 > s = 8: omega(9) = 1110010
             body = "00111111100000000000000000000000" + "0" + "0" + "1110010"
@@ -98,6 +101,30 @@ def test_random_bit_flips_terminate_in_bounds(d):
         idx = rng.integers(0, used, size=20)
         w[idx] ^= np.uint32(1) << rng.integers(0, 32, size=20).astype(np.uint32)
         _decode_guarded(w, offs, n, d, s)  # status may or may not be set; bounds are checked
+
+
+@pytest.mark.parametrize("d", [512, 132, 2048])
+def test_corruption_stays_in_its_buckets(oracle_lib, d):
+    """Bit flips inside some buckets leave every other bucket exactly as the oracle
+    decodes the intact stream (the decoders read a bucket's bits only)."""
+    rng = np.random.default_rng(d)
+    n, s = 60_000, 16
+    enc, words, offs = _encode(n, d, s)
+    ref, _ = oracle_lib.decode(words, offs, n, d, s)
+    nb = offs.size - 1
+    hit = np.unique(rng.integers(0, nb, size=max(2, nb // 8)))
+    w = words.copy()
+    for b in hit:
+        lo, hi = int(offs[b]) + 32, int(offs[b + 1])
+        if hi <= lo:
+            continue
+        for pos in rng.integers(lo, hi, size=3):
+            w[pos >> 5] ^= np.uint32(1) << np.uint32(31 - (pos & 31))
+    out, st = _decode_guarded(w, offs, n, d, s)
+    keep = np.ones(n, dtype=bool)
+    for b in hit:
+        keep[b * d:min(n, (b + 1) * d)] = False
+    assert np.array_equal(out[keep].view(np.uint32), ref[keep].view(np.uint32))
 
 
 def test_capacity_and_workspace_errors():
