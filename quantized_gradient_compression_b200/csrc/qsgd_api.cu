@@ -119,12 +119,14 @@ int qsgd_encode(const float* d_in, uint64_t n, uint32_t d, uint32_t s, uint64_t 
     a.ts = reinterpret_cast<TileState*>(ws + L.tiles_off);
     a.nb = ceil_div(n, d);
     const uint32_t wl = 2u + omega_len_host(s);
-    const bool fast = fast_eligible(d_in, d, s);
+    // the fast path when its tile fits in shared memory, else the general one
+    const uint64_t fast_tile_bits = static_cast<uint64_t>(kFastWarps) * (32u + static_cast<uint64_t>(d) * wl);
+    const uint32_t fast_words = static_cast<uint32_t>(std::min<uint64_t>(ceil_div(fast_tile_bits, 32) + 2, 1u << 24));
+    const bool fast = fast_eligible(d_in, d, s) && fast_smem_bytes(d, s, fast_words) <= 200 * 1024;
     if (fast) {
         a.buckets_per_tile = kFastWarps;  // one bucket per warp
         a.ntiles = ceil_div(a.nb, kFastWarps);
-        const uint64_t tile_bits = static_cast<uint64_t>(kFastWarps) * (32u + static_cast<uint64_t>(d) * wl);
-        a.smem_words = static_cast<uint32_t>(ceil_div(tile_bits, 32) + 2);
+        a.smem_words = fast_words;
     } else {
         a.buckets_per_tile = general_buckets_per_tile(d);
         a.ntiles = ceil_div(a.nb, a.buckets_per_tile);

@@ -691,7 +691,7 @@ __device__ __forceinline__ void init_columns(float* g, uint32_t lo, uint32_t hi)
 
 template <bool kAccumulate, int P>
 __global__ void __launch_bounds__(kDecodeBlock) decode_split(const __grid_constant__ DecodeArgs a) {
-    static_assert(P >= 2 && P <= 8 && (P & (P - 1)) == 0, "P is 2, 4 or 8");
+    static_assert(P >= 1 && P <= 8 && (P & (P - 1)) == 0, "P is 1, 2, 4 or 8");
     extern __shared__ __align__(16) uint32_t smem[];
     uint32_t* lut = smem;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -738,7 +738,7 @@ __global__ void __launch_bounds__(kDecodeBlock) decode_split(const __grid_consta
                 }
             }
         }
-        const bool split = L >= P * kMinPartBits;  // the same in all P lanes of a bucket
+        const bool split = P > 1 && L >= P * kMinPartBits;  // the same in all P lanes of a bucket
         const uint32_t s_lo = split ? static_cast<uint32_t>(static_cast<uint64_t>(L) * j / P) : 0u;
         const uint32_t s_hi = split ? static_cast<uint32_t>(static_cast<uint64_t>(L) * (j + 1) / P) : L;
 
@@ -878,6 +878,23 @@ __global__ void __launch_bounds__(kDecodeBlock) decode_split(const __grid_consta
     }
 }
 
+// Dynamic shared memory for a one-wave launch of `blocks` CTAs that needs `base`
+// bytes: padded so that no SM can hold more than ceil(blocks / SMs) CTAs.  The
+// hardware otherwise stacks up to the occupancy limit on some SMs and leaves
+// others short, and those SMs' issue-bound warps set the kernel's time.
+inline size_t balanced_smem(size_t base, uint64_t blocks, int dev, int sms, int per_sm) {
+    if (sms <= 0 || per_sm <= 1 || blocks == 0) return base;
+    const uint64_t target = (blocks + sms - 1) / sms;
+    if (target >= static_cast<uint64_t>(per_sm)) return base;
+    int per_sm_bytes = 0, reserved = 0;
+    cudaDeviceGetAttribute(&per_sm_bytes, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+    cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+    // target + 1 CTAs must not fit; target CTAs must
+    const size_t pad = static_cast<size_t>(per_sm_bytes) / (target + 1) - static_cast<size_t>(reserved) + 1;
+    if (pad <= base || target * (pad + reserved) > static_cast<size_t>(per_sm_bytes)) return base;
+    return pad;
+}
+
 template <bool kAccumulate, int P>
 cudaError_t launch_split_decode(const DecodeArgs& a, cudaStream_t stream) {
     const size_t smem = kLut * sizeof(uint32_t);
@@ -894,13 +911,19 @@ cudaError_t launch_split_decode(const DecodeArgs& a, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const uint64_t groups = (a.nb + 32 / P - 1) / (32 / P);
-    const uint64_t blocks = std::min<uint64_t>((groups + kDecWarps - 1) / kDecWarps, static_cast<uint64_t>(sms) * per_sm);
+    // one group per warp while the grid stays modest, so that the hardware hands
+    // out the CTAs as SMs free up; beyond that the warps stride over groups
+    const uint64_t blocks = std::min<uint64_t>((groups + kDecWarps - 1) / kDecWarps,
+                                               static_cast<uint64_t>(sms) * per_sm * 8);
     decode_split<kAccumulate, P><<<static_cast<unsigned>(blocks), kDecodeBlock, smem, stream>>>(a);
     return cudaGetLastError();
 }
 
 template <bool kAccumulate>
 cudaError_t launch_split_decode_p(const DecodeArgs& a, cudaStream_t stream) {
+#ifdef QSGD_SPLIT_P
+    return launch_split_decode<kAccumulate, QSGD_SPLIT_P>(a, stream);
+#endif
     if (a.d >= 1024) return launch_split_decode<kAccumulate, 8>(a, stream);
     if (a.d >= 256) return launch_split_decode<kAccumulate, 4>(a, stream);
     return launch_split_decode<kAccumulate, 2>(a, stream);
@@ -922,7 +945,12 @@ cudaError_t launch_fast_decode(const DecodeArgs& a, cudaStream_t stream) {
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const uint64_t groups = (a.nb + 31) / 32;
     const uint64_t blocks = std::min<uint64_t>((groups + kDecWarps - 1) / kDecWarps, static_cast<uint64_t>(sms) * per_sm);
-    decode_fast<kAccumulate><<<static_cast<unsigned>(blocks), kDecodeBlock, smem, stream>>>(a);
+#ifndef QSGD_NO_BALANCE
+    const size_t smem_launch = balanced_smem(smem, blocks, dev, sms, per_sm);
+#else
+    const size_t smem_launch = smem;
+#endif
+    decode_fast<kAccumulate><<<static_cast<unsigned>(blocks), kDecodeBlock, smem_launch, stream>>>(a);
     return cudaGetLastError();
 }
 
@@ -955,8 +983,12 @@ cudaError_t launch_decode(const DecodeArgs& a, bool accumulate, cudaStream_t str
     if (a.nb == 0) return cudaSuccess;
     const bool fast = a.d % 4 == 0 && a.d <= kFastDecodeMaxD && a.s < 1024 &&
                       (reinterpret_cast<uintptr_t>(a.out) & 15u) == 0;
-#ifndef QSGD_NO_SPLIT_DECODE
-    if (fast && a.d >= 128) {
+#ifndef QSGD_SPLIT_MODE
+#define QSGD_SPLIT_MODE 1
+#endif
+    // split decoder: 0 never, 1 for decode-accumulate, 2 for both
+    const bool use_split = QSGD_SPLIT_MODE == 2 || (QSGD_SPLIT_MODE == 1 && accumulate);
+    if (fast && a.d >= 128 && use_split) {
         if (a.K == 1)
             return accumulate ? launch_split_decode_p<true>(a, stream) : launch_split_decode_p<false>(a, stream);
         // several streams (decode-accumulate): one launch per stream, in stream
@@ -972,7 +1004,6 @@ cudaError_t launch_decode(const DecodeArgs& a, bool accumulate, cudaStream_t str
         }
         return cudaSuccess;
     }
-#endif
     if (a.K == 1 && fast)
         return accumulate ? launch_fast_decode<true>(a, stream) : launch_fast_decode<false>(a, stream);
     return accumulate ? launch<true>(a, stream) : launch<false>(a, stream);

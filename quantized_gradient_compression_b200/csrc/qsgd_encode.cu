@@ -157,10 +157,13 @@ __device__ __forceinline__ void merge_shared_word(const EncodeArgs& a, uint64_t*
 // later 16-byte reads (lane L, slot j) fall in distinct bank groups.
 template <int V>
 __device__ __forceinline__ void prefetch_tile(const EncodeArgs& a, uint64_t t, float4* xin) {
-    if (t >= a.ntiles) return;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint64_t b = t * kFastWarps + warp;
-    if (b >= a.nb) return;
+    // a group is committed in every case, so that the waits can count groups
+    if (t >= a.ntiles || b >= a.nb) {
+        asm volatile("cp.async.commit_group;\n" ::: "memory");
+        return;
+    }
     const uint64_t base = b * a.d;
     const uint32_t m = static_cast<uint32_t>(min(static_cast<uint64_t>(a.d), a.n - base));
     const uint32_t swz = (static_cast<uint32_t>(lane) * V / 8) & (V - 1);
@@ -182,7 +185,7 @@ __device__ __forceinline__ void prefetch_tile(const EncodeArgs& a, uint64_t t, f
 template <int V, bool kShort>
 __device__ __forceinline__ void code_tile(const EncodeArgs& a, uint64_t t, uint64_t t_after, const uint32_t* rtab,
                                           uint32_t* tbuf, uint32_t* pb, float4* xin, TileSlot& slot,
-                                          uint32_t epoch) {
+                                          uint32_t epoch, bool desc_pending) {
     // tbuf holds the bits of the tile coded two tiles ago (slot.total, set by that
     // tile): clear the words it used
     const uint32_t dirty = min(a.smem_words, static_cast<uint32_t>((slot.total + 31) >> 5) + 2u);
@@ -194,7 +197,12 @@ __device__ __forceinline__ void code_tile(const EncodeArgs& a, uint64_t t, uint6
     const uint32_t first = lane * NC;  // first bucket-local coordinate of this lane
 
     for (uint32_t i = tid; i < dirty; i += kFastBlock) tbuf[i] = 0u;
-    asm volatile("cp.async.wait_all;\n" ::: "memory");
+    // the tile's input is the oldest pending copy group; the descriptor copies of
+    // the prefix gather, when issued, are the one group after it
+    if (desc_pending)
+        asm volatile("cp.async.wait_group 1;\n" ::: "memory");
+    else
+        asm volatile("cp.async.wait_all;\n" ::: "memory");
     __syncthreads();  // B0: the tile's input has landed; the buffer is clear
 
     // --- input from shared memory ------------------------------------------
@@ -387,18 +395,53 @@ __device__ __forceinline__ bool wait_value(const uint64_t* p, uint64_t state, ui
     }
 }
 
+// Copies the descriptors the prefix gather of tile t = r*C + c will read (tiles
+// [t_lo, t_hi), see gather_prefix) into dpre -- entry i - t_lo, thread (i - t_lo)
+// mod kFastBlock -- and RP(r-2) into *dround, as one cp.async group.  Issued before
+// the CTA codes its next tile, so the copies travel while it works.  The values
+// are plain data (relaxed reads); an entry that is not ready yet is polled later.
+__device__ __forceinline__ void gather_issue(const EncodeArgs& a, uint32_t r, uint32_t C, uint32_t c,
+                                             uint64_t* dpre, uint64_t* dround) {
+    const int tid = threadIdx.x;
+    const uint64_t t_lo = r >= 1 ? static_cast<uint64_t>(r - 1) * C : 0;
+    const uint64_t t_hi = static_cast<uint64_t>(r) * C + c;
+#pragma unroll
+    for (int k = 0; k < static_cast<int>(kGatherPre / kFastBlock); ++k) {
+        const uint64_t i = t_lo + tid + k * kFastBlock;
+        if (i < t_hi) {
+            const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(dpre + tid + k * kFastBlock));
+            asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(dst), "l"(&a.ts[i].desc) : "memory");
+        }
+    }
+    if (tid == kFastBlock - 1 && r >= 2) {
+        const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(dround));
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(dst), "l"(&a.ts[r - 2].round) : "memory");
+    }
+    asm volatile("cp.async.commit_group;\n" ::: "memory");
+}
+
+// Exclusive prefix of tile t = r*C + c: RP(r-2) + the bit counts A of every tile
+// of round r-1 + those of round r's tiles before c, all read in parallel, from the
+// copies gather_issue made (entries past kGatherPre, and any copy that was not
+// ready yet, are read from global memory, waiting if needed).  `newer_group`:
+// another copy group was committed after gather_issue's.  One CTA barrier; every
+// thread returns the same value.  `acc` is a zeroed shared accumulator; false when
+// a bounded wait ran out (or another CTA aborted).
 __device__ __forceinline__ bool gather_prefix(const EncodeArgs& a, uint32_t r, uint32_t C, uint32_t c,
-                                              uint32_t epoch, unsigned long long* acc, int* bad,
+                                              uint32_t epoch, const uint64_t* dpre, const uint64_t* dround,
+                                              bool newer_group, unsigned long long* acc, int* bad,
                                               uint64_t& prefix) {
     const int tid = threadIdx.x, lane = tid & 31;
+    if (newer_group)
+        asm volatile("cp.async.wait_group 1;\n" ::: "memory");
+    else
+        asm volatile("cp.async.wait_all;\n" ::: "memory");
     uint64_t sum = 0;
     bool ok = true;
-    // tiles [t_lo, t_hi): all of round r-1 and round r up to c; plus RP(r-2).
-    // The values are the data, so relaxed loads suffice.
     const uint64_t t_lo = r >= 1 ? static_cast<uint64_t>(r - 1) * C : 0;
     const uint64_t t_hi = static_cast<uint64_t>(r) * C + c;
     for (uint64_t i = t_lo + tid; i < t_hi; i += kFastBlock) {
-        uint64_t d = ld_relaxed(&a.ts[i].desc);
+        uint64_t d = i - t_lo < kGatherPre ? dpre[i - t_lo] : ld_relaxed(&a.ts[i].desc);
         if (!(desc_epoch(d) == (epoch & kEpochMask) && desc_state(d) == kStateAggregate)) {
             uint64_t v = 0;
             ok = ok && wait_value(&a.ts[i].desc, kStateAggregate, epoch, &a.ctrl->abort, v);
@@ -409,8 +452,12 @@ __device__ __forceinline__ bool gather_prefix(const EncodeArgs& a, uint32_t r, u
         sum += d;
     }
     if (tid == kFastBlock - 1 && r >= 2 && ok) {
+        const uint64_t d = *dround;
         uint64_t v = 0;
-        ok = wait_value(&a.ts[r - 2].round, kStatePrefix, epoch, &a.ctrl->abort, v);
+        if (desc_epoch(d) == (epoch & kEpochMask) && desc_state(d) == kStatePrefix)
+            v = desc_value(d);
+        else
+            ok = wait_value(&a.ts[r - 2].round, kStatePrefix, epoch, &a.ctrl->abort, v);
         sum += v;
     }
 #pragma unroll
@@ -469,10 +516,12 @@ __global__ void __launch_bounds__(kFastBlock, (V <= 4 ? kFastMinBlocks : 1)) enc
     __shared__ unsigned long long s_acc[2];
     __shared__ int s_bad;
     __shared__ uint32_t s_ticket[2];
+    __shared__ uint64_t s_round;  // prefetched RP(r-2)
     const int tid = threadIdx.x;
-    uint32_t* const rtab = smem;                                                 // record table
-    float4* const xin = reinterpret_cast<float4*>(smem + kRecordTab);           // kFastWarps * 128V floats
-    uint32_t* const tbuf0 = smem + kRecordTab + kFastWarps * 128 * V;           // two tile buffers
+    uint64_t* const dpre = reinterpret_cast<uint64_t*>(smem);                    // prefetched descriptors
+    uint32_t* const rtab = smem + 2 * kGatherPre;                                // record table
+    float4* const xin = reinterpret_cast<float4*>(rtab + kRecordTab);           // kFastWarps * 128V floats
+    uint32_t* const tbuf0 = rtab + kRecordTab + kFastWarps * 128 * V;           // two tile buffers
     uint32_t* const pb = tbuf0 + 2 * a.smem_words + (tid >> 5) * 32 * fast_lane_words(V, kShort);  // lane strips
     record_table_fill(rtab, tid, kFastBlock);
     const uint32_t epoch = *reinterpret_cast<volatile uint32_t*>(&a.ctrl->epoch);
@@ -489,7 +538,7 @@ __global__ void __launch_bounds__(kFastBlock, (V <= 4 ? kFastMinBlocks : 1)) enc
     uint64_t tn = s_ticket[1];
     int cur = 0;
     prefetch_tile<V>(a, t, xin);
-    if (t < a.ntiles) code_tile<V, kShort>(a, t, tn, rtab, tbuf0, pb, xin, s_slot[0], epoch);
+    if (t < a.ntiles) code_tile<V, kShort>(a, t, tn, rtab, tbuf0, pb, xin, s_slot[0], epoch, false);
     for (int it = 0; t < a.ntiles; ++it) {
         // the ticket after tn, drawn now so its input can be copied during tn's coding
         if (tid == 0) s_ticket[it & 1] = atomicAdd(&a.ctrl->ticket, 1u);
@@ -497,13 +546,14 @@ __global__ void __launch_bounds__(kFastBlock, (V <= 4 ? kFastMinBlocks : 1)) enc
         uint32_t* const tnext = tbuf0 + (cur ^ 1) * a.smem_words;
         __syncthreads();
         const uint64_t tnn = s_ticket[it & 1];
-        // code the next tile first: its work covers this tile's prefix wait
-        if (tn < a.ntiles) code_tile<V, kShort>(a, tn, tnn, rtab, tnext, pb, xin, s_slot[cur ^ 1], epoch);
         const uint32_t r = static_cast<uint32_t>(t) / C;
         const uint32_t c = static_cast<uint32_t>(t) - r * C;
+        // this tile's prefix descriptors travel while the next tile is coded
+        gather_issue(a, r, C, c, dpre, &s_round);
+        if (tn < a.ntiles) code_tile<V, kShort>(a, tn, tnn, rtab, tnext, pb, xin, s_slot[cur ^ 1], epoch, true);
         const uint64_t tb = s_slot[cur].total;
         uint64_t X = 0;
-        const bool ok = gather_prefix(a, r, C, c, epoch, &s_acc[it & 1], &s_bad, X);
+        const bool ok = gather_prefix(a, r, C, c, epoch, dpre, &s_round, tn < a.ntiles, &s_acc[it & 1], &s_bad, X);
         if (tid == 0) s_acc[(it + 1) & 1] = 0;  // the next iteration's accumulator
         if (!ok) {
             if (tid == 0) abort_all(a);

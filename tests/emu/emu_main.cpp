@@ -84,9 +84,9 @@ int main(int argc, char** argv) {
         a.streams[0].num_words = ws[j].size() / 4;
         a.streams[0].offsets = reinterpret_cast<const uint64_t*>(os[j].data());
         if (acc) {
-            if (P == 2) run_kernel<true, 2>(a, grid); else if (P == 4) run_kernel<true, 4>(a, grid); else run_kernel<true, 8>(a, grid);
+            if (P == 1) run_kernel<true, 1>(a, grid); else if (P == 2) run_kernel<true, 2>(a, grid); else if (P == 4) run_kernel<true, 4>(a, grid); else run_kernel<true, 8>(a, grid);
         } else {
-            if (P == 2) run_kernel<false, 2>(a, grid); else if (P == 4) run_kernel<false, 4>(a, grid); else run_kernel<false, 8>(a, grid);
+            if (P == 1) run_kernel<false, 1>(a, grid); else if (P == 2) run_kernel<false, 2>(a, grid); else if (P == 4) run_kernel<false, 4>(a, grid); else run_kernel<false, 8>(a, grid);
         }
         if (g_emu_error) return 4;
     }

@@ -28,7 +28,9 @@ CSRC = os.path.join(ROOT, "quantized_gradient_compression_b200", "csrc")
 
 def _kernel_source() -> str:
     src = open(os.path.join(CSRC, "qsgd_decode.cu")).read()
-    cut = src.index("template <bool kAccumulate, int P>\ncudaError_t launch_split_decode")
+    # everything from the first host-side launch helper on is cut
+    cut = min(src.index(m) for m in ("template <bool kAccumulate, int P>\ncudaError_t launch_split_decode",
+                                     "// Dynamic shared memory for a one-wave launch") if m in src)
     s = src[:cut] + "}  // namespace\n}  // namespace qsgd\n"
     s = s.replace('#include "../../include/qsgd.h"', '#include "%s"' % os.path.join(ROOT, "include", "qsgd.h"))
     s = s.replace('#include "qsgd_internal.h"', '#include "%s"' % os.path.join(CSRC, "qsgd_internal.h"))
@@ -91,7 +93,7 @@ def _run(exe, tmp, oracle_lib, n, d, s, K, P, accumulate, kind, corrupt=False):
     return got, status, streams, base
 
 
-# (n, d, s, K, P, accumulate, input): P = 2 / 4 / 8, sparse buckets decoded whole,
+# (n, d, s, K, P, accumulate, input): P = 1 / 2 / 4 / 8, sparse buckets decoded whole,
 # layered data (buckets too short to split next to split ones), ragged tails
 CASES = [
     (40_000, 132, 3, 3, 2, True, "normal"),
@@ -101,6 +103,8 @@ CASES = [
     (40_000, 2048, 64, 2, 8, True, "normal"),
     (9_001, 4096, 1000, 1, 8, False, "normal"),
     (513, 512, 16, 2, 4, True, "normal"),
+    (30_001, 512, 16, 1, 1, False, "layered"),   # P = 1: one lane per bucket, direct stores
+    (20_000, 132, 3, 2, 1, True, "normal"),
 ]
 
 
