@@ -454,7 +454,6 @@ __global__ void __launch_bounds__(kDecodeBlock) decode_fast(const __grid_constan
         const uint64_t b = g * 32 + lane;
         const bool live = b < a.nb;
         const uint32_t m = live ? static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - b * d)) : 0u;
-        const bool full_group = (g + 1) * 32 <= a.nb && (g + 1) * 32 * static_cast<uint64_t>(d) <= a.n;
         bool bad = false;
         BitBuf r;
         r.left = 0;
@@ -487,37 +486,28 @@ __global__ void __launch_bounds__(kDecodeBlock) decode_fast(const __grid_constan
         uint32_t next = 0, pidx = kNoRecord, pval = 0;
         if (!bad) table_next(r, lut, scale, next, pidx, pval);
         for (uint32_t lo = 0; lo < d; lo += kSeg) {
-            const uint32_t seg_len = min(static_cast<uint32_t>(kSeg), d - lo);
-            const bool vec = full_group && seg_len == kSeg;
-            // --- staging tile: zeros, or the current output (+0.0 turns -0.0 into +0.0)
+            // --- staging tile: zeros, or the current output ---------------------
+            // Step i covers row 2i + wrow (bucket g*32 + 2i + wrow), columns
+            // lo + wcol .. +3.  Rows past the last bucket and columns past a
+            // bucket's end are neither read nor written back (the ragged last
+            // group takes the same unrolled path, only masked).
             if (kAccumulate) {
-                if (vec) {
-                    // all 16 copies in flight at once; the first group's +0.0 is
-                    // applied at write-back instead ((x + 0) + v == (x + v) + 0 for
-                    // every x and every v, -0.0 included)
-                    const float* src = a.out + (g * 32 + wrow) * d + lo + wcol;
-                    uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(stage + wrow * kStride + wcol));
+                uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(stage + wrow * kStride + wcol));
+                const uint32_t c = lo + wcol;
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
+                for (int i = 0; i < 16; ++i, dst += 2 * kStride * sizeof(float)) {
+                    const uint64_t bb = g * 32 + wrow + 2 * i;
+                    const uint32_t mm = bb < a.nb ? static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - bb * d)) : 0u;
+                    if (c + 4 <= mm) {
+                        const float* src = a.out + bb * d + c;
                         asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src) : "memory");
-                        src += 2 * static_cast<uint64_t>(d);
-                        dst += 2 * kStride * sizeof(float);
-                    }
-                    asm volatile("cp.async.wait_all;\n" ::: "memory");
-                } else {
-                    for (int rr = 0; rr < 32; ++rr) {
-                        const uint64_t bb = g * 32 + rr;
-                        const uint32_t mm = bb < a.nb ? static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - bb * d)) : 0u;
-                        for (uint32_t c = lane; c < kSeg; c += 32) {
-                            float v = 0.f;
-                            if (lo + c < mm) {
-                                v = a.out[bb * d + lo + c];
-                                if (a.first_group) v = __fadd_rn(v, 0.0f);
-                            }
-                            stage[rr * kStride + c] = v;
-                        }
+                    } else if (c < mm) {
+                        float* sp = stage + (wrow + 2 * i) * kStride + wcol;
+                        for (uint32_t e = 0; e < 4; ++e)
+                            if (c + e < mm) sp[e] = a.out[bb * d + c + e];
                     }
                 }
+                asm volatile("cp.async.wait_all;\n" ::: "memory");
             } else {
                 for (int q = lane; q < 32 * kStride / 4; q += 32)
                     reinterpret_cast<float4*>(stage)[q] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -550,31 +540,33 @@ __global__ void __launch_bounds__(kDecodeBlock) decode_fast(const __grid_constan
                 }
             }
             __syncwarp();
-            // --- write the tile back: row r is bucket g*32 + r -----------------
-            if (vec) {
-                float* dst = a.out + (g * 32 + wrow) * d + lo + wcol;
-                const float* src = stage + wrow * kStride + wcol;
+            // --- write the tile back (the first stream of an accumulation adds +0.0:
+            // (x + 0) + v == (x + v) + 0 for every x and v, -0.0 included) ------
+            {
+                const float* sp = stage + wrow * kStride + wcol;
+                const uint32_t c = lo + wcol;
                 const bool plus_zero = kAccumulate && a.first_group;
 #pragma unroll 4
-                for (int i = 0; i < 16; ++i) {
-                    float4 v = *reinterpret_cast<const float4*>(src);
-                    if (plus_zero) {
-                        v.x = __fadd_rn(v.x, 0.0f);
-                        v.y = __fadd_rn(v.y, 0.0f);
-                        v.z = __fadd_rn(v.z, 0.0f);
-                        v.w = __fadd_rn(v.w, 0.0f);
+                for (int i = 0; i < 16; ++i, sp += 2 * kStride) {
+                    const uint64_t bb = g * 32 + wrow + 2 * i;
+                    const uint32_t mm = bb < a.nb ? static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - bb * d)) : 0u;
+                    if (c < mm) {
+                        float4 v = *reinterpret_cast<const float4*>(sp);
+                        if (plus_zero) {
+                            v.x = __fadd_rn(v.x, 0.0f);
+                            v.y = __fadd_rn(v.y, 0.0f);
+                            v.z = __fadd_rn(v.z, 0.0f);
+                            v.w = __fadd_rn(v.w, 0.0f);
+                        }
+                        float* gp = a.out + bb * d + c;
+                        if (c + 4 <= mm) {
+                            *reinterpret_cast<float4*>(gp) = v;
+                        } else {
+                            const float e4[4] = {v.x, v.y, v.z, v.w};
+                            for (uint32_t e = 0; e < 4; ++e)
+                                if (c + e < mm) gp[e] = e4[e];
+                        }
                     }
-                    *reinterpret_cast<float4*>(dst) = v;
-                    dst += 2 * static_cast<uint64_t>(d);
-                    src += 2 * kStride;
-                }
-            } else {
-                for (int rr = 0; rr < 32; ++rr) {
-                    const uint64_t bb = g * 32 + rr;
-                    if (bb >= a.nb) break;
-                    const uint32_t mm = static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - bb * d));
-                    for (uint32_t c = lane; c < seg_len; c += 32)
-                        if (lo + c < mm) a.out[bb * d + lo + c] = stage[rr * kStride + c];
                 }
             }
             __syncwarp();
@@ -983,30 +975,29 @@ cudaError_t launch_decode(const DecodeArgs& a, bool accumulate, cudaStream_t str
     if (a.nb == 0) return cudaSuccess;
     const bool fast = a.d % 4 == 0 && a.d <= kFastDecodeMaxD && a.s < 1024 &&
                       (reinterpret_cast<uintptr_t>(a.out) & 15u) == 0;
+    if (!fast) return accumulate ? launch<true>(a, stream) : launch<false>(a, stream);
 #ifndef QSGD_SPLIT_MODE
-#define QSGD_SPLIT_MODE 1
+#define QSGD_SPLIT_MODE 0
 #endif
-    // split decoder: 0 never, 1 for decode-accumulate, 2 for both
-    const bool use_split = QSGD_SPLIT_MODE == 2 || (QSGD_SPLIT_MODE == 1 && accumulate);
-    if (fast && a.d >= 128 && use_split) {
-        if (a.K == 1)
-            return accumulate ? launch_split_decode_p<true>(a, stream) : launch_split_decode_p<false>(a, stream);
-        // several streams (decode-accumulate): one launch per stream, in stream
-        // order on the one CUDA stream, so every coordinate still sees its adds
-        // left to right; between launches the output stays in L2
-        DecodeArgs one = a;
-        one.K = 1;
-        for (int j = 0; j < a.K; ++j) {
-            one.streams[0] = a.streams[j];
-            one.first_group = a.first_group && j == 0;
-            const cudaError_t e = launch_split_decode_p<true>(one, stream);
-            if (e != cudaSuccess) return e;
-        }
-        return cudaSuccess;
+    // split decoder: 0 never, 1 for decode-accumulate, 2 for both (d >= 128)
+    const bool split = a.d >= 128 && (QSGD_SPLIT_MODE == 2 || (QSGD_SPLIT_MODE == 1 && accumulate));
+    auto one = [&](const DecodeArgs& x) -> cudaError_t {
+        if (split) return accumulate ? launch_split_decode_p<true>(x, stream) : launch_split_decode_p<false>(x, stream);
+        return accumulate ? launch_fast_decode<true>(x, stream) : launch_fast_decode<false>(x, stream);
+    };
+    if (a.K == 1) return one(a);
+    // several streams (decode-accumulate): one launch per stream, in stream order
+    // on the one CUDA stream, so every coordinate still sees its adds left to
+    // right; between launches the output stays in L2
+    DecodeArgs o = a;
+    o.K = 1;
+    for (int j = 0; j < a.K; ++j) {
+        o.streams[0] = a.streams[j];
+        o.first_group = a.first_group && j == 0;
+        const cudaError_t e = one(o);
+        if (e != cudaSuccess) return e;
     }
-    if (a.K == 1 && fast)
-        return accumulate ? launch_fast_decode<true>(a, stream) : launch_fast_decode<false>(a, stream);
-    return accumulate ? launch<true>(a, stream) : launch<false>(a, stream);
+    return cudaSuccess;
 }
 
 }  // namespace qsgd

@@ -1,6 +1,7 @@
-"""The split decoder's kernel source run on the CPU under a warp emulator (no GPU).
+"""The decoders' kernel source run on the CPU under a warp emulator (no GPU).
 
-`tests/emu/inc/warp_emu.h` stands in for the CUDA features `decode_split` uses:
+`tests/emu/inc/warp_emu.h` stands in for the CUDA features `decode_fast` (P = 0
+below) and `decode_split` (P >= 1) use:
 every thread of a block is a host thread, and each warp primitive gathers the 32
 lanes and checks that they call the same primitive at the same source line.  A lane
 that skips a primitive the others wait in (a deadlock on a GPU) fails the test here,
@@ -93,7 +94,8 @@ def _run(exe, tmp, oracle_lib, n, d, s, K, P, accumulate, kind, corrupt=False):
     return got, status, streams, base
 
 
-# (n, d, s, K, P, accumulate, input): P = 1 / 2 / 4 / 8, sparse buckets decoded whole,
+# (n, d, s, K, P, accumulate, input): P = 0 (decode_fast) / 1 / 2 / 4 / 8, sparse
+# buckets decoded whole,
 # layered data (buckets too short to split next to split ones), ragged tails
 CASES = [
     (40_000, 132, 3, 3, 2, True, "normal"),
@@ -105,6 +107,11 @@ CASES = [
     (513, 512, 16, 2, 4, True, "normal"),
     (30_001, 512, 16, 1, 1, False, "layered"),   # P = 1: one lane per bucket, direct stores
     (20_000, 132, 3, 2, 1, True, "normal"),
+    # P = 0: the one-lane staged decoder (decode_fast), ragged last group and d % 64 != 0
+    (30_001, 512, 16, 1, 0, False, "layered"),
+    (30_001, 512, 16, 2, 0, True, "layered"),
+    (20_000, 100, 7, 2, 0, True, "normal"),
+    (9_000, 132, 3, 1, 0, False, "normal"),
 ]
 
 
