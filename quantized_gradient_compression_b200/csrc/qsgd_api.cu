@@ -58,7 +58,8 @@ WorkspaceLayout workspace_layout(uint64_t n, uint32_t d) {
     // fast path: tiles of kFastWarps buckets; general path: tiles of whole buckets
     const uint64_t per_tile = std::min<uint64_t>(kFastWarps, general_buckets_per_tile(d));
     L.max_tiles = nb ? ceil_div(nb, per_tile) : 0;
-    L.tiles_off = 256;
+    L.desc_off = 256;
+    L.tiles_off = L.desc_off + align256(sizeof(uint64_t) * ((L.max_tiles + 1) & ~uint64_t(1)));
     L.total = L.tiles_off + align256(sizeof(TileState) * L.max_tiles);
     return L;
 }
@@ -116,6 +117,7 @@ int qsgd_encode(const float* d_in, uint64_t n, uint32_t d, uint32_t s, uint64_t 
     a.offsets = d_offsets;
     a.status = d_status;
     a.ctrl = reinterpret_cast<ScanControl*>(ws);
+    a.tdesc = reinterpret_cast<uint64_t*>(ws + L.desc_off);
     a.ts = reinterpret_cast<TileState*>(ws + L.tiles_off);
     a.nb = ceil_div(n, d);
     const uint32_t wl = 2u + omega_len_host(s);

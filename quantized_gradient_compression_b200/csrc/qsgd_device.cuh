@@ -295,18 +295,18 @@ struct ScanControl {
 };
 static_assert(sizeof(ScanControl) == 64, "control block is one 64-byte line");
 
-// Per-tile state in the workspace.
+// Per-tile state in the workspace besides the scan descriptor (which lives in its
+// own contiguous array, so that descriptor pairs can be copied 16 bytes at a time).
 struct TileState {
-    uint64_t desc;   // scan descriptor of the tile
     uint64_t slot;   // slot of the word shared with the previous tile
     uint64_t round;  // fast path: RP(r), the stream position after round r (entry r)
 };
-static_assert(sizeof(TileState) == 24, "tile state is three words");
+static_assert(sizeof(TileState) == 16, "tile state is two words");
 
 // Warp-cooperative look-back for tile `tile` (> 0).  All 32 lanes call it; every
 // lane returns the exclusive prefix.  Returns false (and leaves the prefix
 // undefined) when the bounded wait ran out or another tile aborted.
-__device__ __forceinline__ bool lookback(const TileState* ts, uint32_t tile, uint32_t epoch,
+__device__ __forceinline__ bool lookback(const uint64_t* desc, uint32_t tile, uint32_t epoch,
                                          const uint32_t* abort_flag, uint64_t& exclusive) {
     const int lane = threadIdx.x & 31;
     uint64_t sum = 0;
@@ -318,7 +318,7 @@ __device__ __forceinline__ bool lookback(const TileState* ts, uint32_t tile, uin
         uint64_t st = kStatePrefix;  // lanes past tile 0 act as a zero prefix
         uint64_t val = 0;
         if (idx >= 0) {
-            d = ld_acquire(&ts[idx].desc);
+            d = ld_acquire(&desc[idx]);
             st = (desc_epoch(d) == (epoch & kEpochMask)) ? desc_state(d) : 0;
             val = desc_value(d);
         }

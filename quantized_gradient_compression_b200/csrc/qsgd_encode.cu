@@ -174,8 +174,11 @@ __device__ __forceinline__ void prefetch_tile(const EncodeArgs& a, uint64_t t, f
         const uint32_t avail = i < m ? min(16u, (m - i) * 4u) : 0u;
         const uint32_t saddr = static_cast<uint32_t>(__cvta_generic_to_shared(dst + (j ^ swz)));
         const float* src = a.in + base + (i < m ? i : 0);
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(saddr), "l"(src), "r"(avail)
-                     : "memory");
+        if (avail == 16u)
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(saddr), "l"(src) : "memory");
+        else  // the ragged end of the last bucket: zero-filled past m
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(saddr), "l"(src), "r"(avail)
+                         : "memory");
     }
     asm volatile("cp.async.commit_group;\n" ::: "memory");
 }
@@ -183,7 +186,7 @@ __device__ __forceinline__ void prefetch_tile(const EncodeArgs& a, uint64_t t, f
 // Codes tile t into tbuf (tile-local bit offsets) and publishes A(t).  On entry
 // the tile's input is in flight into xin.  Two CTA barriers.
 template <int V, bool kShort>
-__device__ __forceinline__ void code_tile(const EncodeArgs& a, uint64_t t, uint64_t t_after, const uint32_t* rtab,
+__device__ __forceinline__ void code_tile(const EncodeArgs& a, uint64_t t, const uint32_t* t_after_slot, const uint32_t* rtab,
                                           uint32_t* tbuf, uint32_t* pb, float4* xin, TileSlot& slot,
                                           uint32_t epoch, bool desc_pending) {
     // tbuf holds the bits of the tile coded two tiles ago (slot.total, set by that
@@ -196,14 +199,15 @@ __device__ __forceinline__ void code_tile(const EncodeArgs& a, uint64_t t, uint6
     const uint64_t base = b * a.d;
     const uint32_t first = lane * NC;  // first bucket-local coordinate of this lane
 
-    for (uint32_t i = tid; i < dirty; i += kFastBlock) tbuf[i] = 0u;
     // the tile's input is the oldest pending copy group; the descriptor copies of
     // the prefix gather, when issued, are the one group after it
     if (desc_pending)
         asm volatile("cp.async.wait_group 1;\n" ::: "memory");
     else
         asm volatile("cp.async.wait_all;\n" ::: "memory");
-    __syncthreads();  // B0: the tile's input has landed; the buffer is clear
+    __syncthreads();  // B0: the tile's input has landed; every warp is done with tbuf's last tile
+    // clear the words tbuf's last tile used (nothing writes tbuf before B1)
+    for (uint32_t i = tid; i < dirty; i += kFastBlock) tbuf[i] = 0u;
 
     // --- input from shared memory ------------------------------------------
     float x[NC];
@@ -334,7 +338,7 @@ __device__ __forceinline__ void code_tile(const EncodeArgs& a, uint64_t t, uint6
     const uint32_t exclb = inclb - nbits;
     if (lane == 31) slot.bits[warp] = live ? 32u + inclb : 0u;
     __syncthreads();  // B1: bucket sizes known; the input buffer is free
-    prefetch_tile<V>(a, t_after, xin);
+    prefetch_tile<V>(a, *t_after_slot, xin);  // the ticket was stored before B0
     // tile-local start of this warp's bucket and the tile's size (kFastWarps-lane scan)
     uint32_t bsc = lane < kFastWarps ? slot.bits[lane] : 0u;
 #pragma unroll
@@ -345,7 +349,7 @@ __device__ __forceinline__ void code_tile(const EncodeArgs& a, uint64_t t, uint6
     const uint64_t tb = __shfl_sync(kFull, bsc, kFastWarps - 1);
     const uint64_t bstart = warp ? __shfl_sync(kFull, bsc, warp - 1) : 0u;
     if (tid == 0) {
-        st_release(&a.ts[t].desc, make_desc(epoch, kStateAggregate, tb));
+        st_release(&a.tdesc[t], make_desc(epoch, kStateAggregate, tb));
         slot.total = tb;
     }
 
@@ -396,37 +400,37 @@ __device__ __forceinline__ bool wait_value(const uint64_t* p, uint64_t state, ui
 }
 
 // Copies the descriptors the prefix gather of tile t = r*C + c will read (tiles
-// [t_lo, t_hi), see gather_prefix) into dpre -- entry i - t_lo, thread (i - t_lo)
-// mod kFastBlock -- and RP(r-2) into *dround, as one cp.async group.  Issued before
-// the CTA codes its next tile, so the copies travel while it works.  The values
-// are plain data (relaxed reads); an entry that is not ready yet is polled later.
+// [t_lo, t_hi), see gather_prefix) into dpre, as 16-byte pairs: thread k takes the
+// pair (2(p0+k), 2(p0+k)+1), p0 = t_lo / 2, to entries 2k and 2k+1; and RP(r-2)
+// (16 bytes of TileState r-2) into dround.  One cp.async group, issued before the
+// CTA codes its next tile, so the copies travel while it works.  The copies go to
+// L2 only (.cg); the values are plain data, and one that is not ready yet is
+// polled later.
 __device__ __forceinline__ void gather_issue(const EncodeArgs& a, uint32_t r, uint32_t C, uint32_t c,
                                              uint64_t* dpre, uint64_t* dround) {
     const int tid = threadIdx.x;
     const uint64_t t_lo = r >= 1 ? static_cast<uint64_t>(r - 1) * C : 0;
     const uint64_t t_hi = static_cast<uint64_t>(r) * C + c;
-#pragma unroll
-    for (int k = 0; k < static_cast<int>(kGatherPre / kFastBlock); ++k) {
-        const uint64_t i = t_lo + tid + k * kFastBlock;
-        if (i < t_hi) {
-            const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(dpre + tid + k * kFastBlock));
-            asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(dst), "l"(&a.ts[i].desc) : "memory");
-        }
+    const uint64_t p = (t_lo >> 1) + tid;
+    if (2 * p < t_hi && 2 * tid + 1 < kGatherPre) {
+        const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(dpre + 2 * tid));
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(a.tdesc + 2 * p) : "memory");
     }
     if (tid == kFastBlock - 1 && r >= 2) {
         const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(dround));
-        asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(dst), "l"(&a.ts[r - 2].round) : "memory");
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(&a.ts[r - 2]) : "memory");
     }
     asm volatile("cp.async.commit_group;\n" ::: "memory");
 }
 
 // Exclusive prefix of tile t = r*C + c: RP(r-2) + the bit counts A of every tile
-// of round r-1 + those of round r's tiles before c, all read in parallel, from the
-// copies gather_issue made (entries past kGatherPre, and any copy that was not
-// ready yet, are read from global memory, waiting if needed).  `newer_group`:
-// another copy group was committed after gather_issue's.  One CTA barrier; every
-// thread returns the same value.  `acc` is a zeroed shared accumulator; false when
-// a bounded wait ran out (or another CTA aborted).
+// of round r-1 + those of round r's tiles before c, all read in parallel.  Thread
+// k sums the pairs p0+k, p0+k+kFastBlock, ...: the first from the copy
+// gather_issue made, the others (and any copy that was not ready yet) from global
+// memory, waiting if needed.  `newer_group`: another copy group was committed after
+// gather_issue's.  One CTA barrier; every thread returns the same value.  `acc` is
+// a zeroed shared accumulator; false when a bounded wait ran out (or another CTA
+// aborted).
 __device__ __forceinline__ bool gather_prefix(const EncodeArgs& a, uint32_t r, uint32_t C, uint32_t c,
                                               uint32_t epoch, const uint64_t* dpre, const uint64_t* dround,
                                               bool newer_group, unsigned long long* acc, int* bad,
@@ -440,19 +444,25 @@ __device__ __forceinline__ bool gather_prefix(const EncodeArgs& a, uint32_t r, u
     bool ok = true;
     const uint64_t t_lo = r >= 1 ? static_cast<uint64_t>(r - 1) * C : 0;
     const uint64_t t_hi = static_cast<uint64_t>(r) * C + c;
-    for (uint64_t i = t_lo + tid; i < t_hi; i += kFastBlock) {
-        uint64_t d = i - t_lo < kGatherPre ? dpre[i - t_lo] : ld_relaxed(&a.ts[i].desc);
-        if (!(desc_epoch(d) == (epoch & kEpochMask) && desc_state(d) == kStateAggregate)) {
-            uint64_t v = 0;
-            ok = ok && wait_value(&a.ts[i].desc, kStateAggregate, epoch, &a.ctrl->abort, v);
-            d = v;
-        } else {
-            d = desc_value(d);
+    for (uint64_t p = (t_lo >> 1) + tid; 2 * p < t_hi; p += kFastBlock) {
+        const bool copied = p == (t_lo >> 1) + tid && 2 * tid + 1 < kGatherPre;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const uint64_t i = 2 * p + h;
+            if (i < t_lo || i >= t_hi) continue;
+            uint64_t d = copied ? dpre[2 * tid + h] : ld_relaxed(&a.tdesc[i]);
+            if (!(desc_epoch(d) == (epoch & kEpochMask) && desc_state(d) == kStateAggregate)) {
+                uint64_t v = 0;
+                ok = ok && wait_value(&a.tdesc[i], kStateAggregate, epoch, &a.ctrl->abort, v);
+                d = v;
+            } else {
+                d = desc_value(d);
+            }
+            sum += d;
         }
-        sum += d;
     }
     if (tid == kFastBlock - 1 && r >= 2 && ok) {
-        const uint64_t d = *dround;
+        const uint64_t d = dround[1];
         uint64_t v = 0;
         if (desc_epoch(d) == (epoch & kEpochMask) && desc_state(d) == kStatePrefix)
             v = desc_value(d);
@@ -515,8 +525,8 @@ __global__ void __launch_bounds__(kFastBlock, (V <= 4 ? kFastMinBlocks : 1)) enc
     __shared__ TileSlot s_slot[2];
     __shared__ unsigned long long s_acc[2];
     __shared__ int s_bad;
-    __shared__ uint32_t s_ticket[2];
-    __shared__ uint64_t s_round;  // prefetched RP(r-2)
+    __shared__ uint32_t s_ticket[2];  // [0] the first tile; then the ticket drawn each iteration
+    __shared__ __align__(16) uint64_t s_round[2];  // prefetched TileState r-2
     const int tid = threadIdx.x;
     uint64_t* const dpre = reinterpret_cast<uint64_t*>(smem);                    // prefetched descriptors
     uint32_t* const rtab = smem + 2 * kGatherPre;                                // record table
@@ -538,22 +548,28 @@ __global__ void __launch_bounds__(kFastBlock, (V <= 4 ? kFastMinBlocks : 1)) enc
     uint64_t tn = s_ticket[1];
     int cur = 0;
     prefetch_tile<V>(a, t, xin);
-    if (t < a.ntiles) code_tile<V, kShort>(a, t, tn, rtab, tbuf0, pb, xin, s_slot[0], epoch, false);
+    // the first tile's coding prefetches tn's input: read from s_ticket[1]
+    if (t < a.ntiles) code_tile<V, kShort>(a, t, &s_ticket[1], rtab, tbuf0, pb, xin, s_slot[0], epoch, false);
+    __syncthreads();  // every thread has read s_ticket before the loop reuses it
+    // Per iteration: draw the ticket tnn, code tile tn (its B1 starts the input
+    // copy of tnn; B0 publishes tnn), then gather tile t's prefix and store t.
+    // CTA barriers: B0 and B1 inside the coding, Bg inside the gather.
     for (int it = 0; t < a.ntiles; ++it) {
-        // the ticket after tn, drawn now so its input can be copied during tn's coding
         if (tid == 0) s_ticket[it & 1] = atomicAdd(&a.ctrl->ticket, 1u);
         uint32_t* const tcur = tbuf0 + cur * a.smem_words;
         uint32_t* const tnext = tbuf0 + (cur ^ 1) * a.smem_words;
-        __syncthreads();
-        const uint64_t tnn = s_ticket[it & 1];
         const uint32_t r = static_cast<uint32_t>(t) / C;
         const uint32_t c = static_cast<uint32_t>(t) - r * C;
         // this tile's prefix descriptors travel while the next tile is coded
-        gather_issue(a, r, C, c, dpre, &s_round);
-        if (tn < a.ntiles) code_tile<V, kShort>(a, tn, tnn, rtab, tnext, pb, xin, s_slot[cur ^ 1], epoch, true);
+        gather_issue(a, r, C, c, dpre, s_round);
+        if (tn < a.ntiles)
+            code_tile<V, kShort>(a, tn, &s_ticket[it & 1], rtab, tnext, pb, xin, s_slot[cur ^ 1], epoch, true);
+        else
+            __syncthreads();  // orders the ticket, the accumulator reset and store_tile
+        const uint64_t tnn = s_ticket[it & 1];
         const uint64_t tb = s_slot[cur].total;
         uint64_t X = 0;
-        const bool ok = gather_prefix(a, r, C, c, epoch, dpre, &s_round, tn < a.ntiles, &s_acc[it & 1], &s_bad, X);
+        const bool ok = gather_prefix(a, r, C, c, epoch, dpre, s_round, tn < a.ntiles, &s_acc[it & 1], &s_bad, X);
         if (tid == 0) s_acc[(it + 1) & 1] = 0;  // the next iteration's accumulator
         if (!ok) {
             if (tid == 0) abort_all(a);
@@ -826,18 +842,18 @@ __global__ void __launch_bounds__(kBlock) encode_general(const __grid_constant__
             tb += total;
         }
         if (tid == 0)
-            st_release(&a.ts[tile].desc, make_desc(epoch, tile == 0 ? kStatePrefix : kStateAggregate, tb));
+            st_release(&a.tdesc[tile], make_desc(epoch, tile == 0 ? kStatePrefix : kStateAggregate, tb));
 
         // --- look-back ------------------------------------------------------
         if (warp == 0) {
             uint64_t excl = 0;
             bool ok = true;
-            if (tile > 0) ok = lookback(a.ts, tile, epoch, &a.ctrl->abort, excl);
+            if (tile > 0) ok = lookback(a.tdesc, tile, epoch, &a.ctrl->abort, excl);
             if (lane == 0) {
                 if (!ok)
                     abort_all(a);
                 else if (tile > 0)
-                    st_release(&a.ts[tile].desc, make_desc(epoch, kStatePrefix, excl + tb));
+                    st_release(&a.tdesc[tile], make_desc(epoch, kStatePrefix, excl + tb));
                 s_prefix = excl;
                 s_ok = ok;
                 s_pending = 0;

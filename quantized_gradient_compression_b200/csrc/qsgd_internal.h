@@ -13,12 +13,13 @@ namespace qsgd {
 struct ScanControl;
 struct TileState;
 
-// Workspace layout: [0, 256) ScanControl, then TileState[max_tiles] (24 bytes per
-// tile: scan descriptor, shared-word slot, round prefix).  Every entry carries the
-// call's epoch and sits at the same place whatever (n, d, s) a call uses, so one
-// workspace serves calls of any shape without clearing.
+// Workspace layout: [0, 256) ScanControl; from 256 the tile scan descriptors
+// (uint64 per tile, the count rounded up to an even number); then TileState per
+// tile (shared-word slot, round prefix).  Every entry carries the call's epoch, so
+// values left by an earlier call -- of any shape, wherever they now fall -- read as
+// "not ready", and one workspace serves calls of any shape without clearing.
 struct WorkspaceLayout {
-    size_t tiles_off, total;
+    size_t desc_off, tiles_off, total;
     uint64_t max_tiles;
 };
 WorkspaceLayout workspace_layout(uint64_t n, uint32_t d);
@@ -34,6 +35,7 @@ struct EncodeArgs {
     uint64_t* offsets;
     uint32_t* status;
     ScanControl* ctrl;
+    uint64_t* tdesc;  // scan descriptor per tile (16-byte aligned)
     TileState* ts;
     uint64_t nb;
     uint64_t ntiles;
