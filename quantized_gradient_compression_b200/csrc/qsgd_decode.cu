@@ -454,6 +454,8 @@ __global__ void __launch_bounds__(kDecodeBlock) decode_fast(const __grid_constan
         const uint64_t b = g * 32 + lane;
         const bool live = b < a.nb;
         const uint32_t m = live ? static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - b * d)) : 0u;
+        // every row of the group is a whole bucket of d: no masks in the staging
+        const bool full = (g + 1) * 32 <= a.nb && (g + 1) * 32 * static_cast<uint64_t>(d) <= a.n;
         bool bad = false;
         BitBuf r;
         r.left = 0;
@@ -497,7 +499,7 @@ __global__ void __launch_bounds__(kDecodeBlock) decode_fast(const __grid_constan
 #pragma unroll
                 for (int i = 0; i < 16; ++i, dst += 2 * kStride * sizeof(float)) {
                     const uint64_t bb = g * 32 + wrow + 2 * i;
-                    const uint32_t mm = bb < a.nb ? static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - bb * d)) : 0u;
+                    const uint32_t mm = full ? d : bb < a.nb ? static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - bb * d)) : 0u;
                     if (c + 4 <= mm) {
                         const float* src = a.out + bb * d + c;
                         asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src) : "memory");
@@ -549,7 +551,7 @@ __global__ void __launch_bounds__(kDecodeBlock) decode_fast(const __grid_constan
 #pragma unroll 4
                 for (int i = 0; i < 16; ++i, sp += 2 * kStride) {
                     const uint64_t bb = g * 32 + wrow + 2 * i;
-                    const uint32_t mm = bb < a.nb ? static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - bb * d)) : 0u;
+                    const uint32_t mm = full ? d : bb < a.nb ? static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - bb * d)) : 0u;
                     if (c < mm) {
                         float4 v = *reinterpret_cast<const float4*>(sp);
                         if (plus_zero) {

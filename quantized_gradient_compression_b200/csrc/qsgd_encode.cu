@@ -188,7 +188,7 @@ __device__ __forceinline__ void prefetch_tile(const EncodeArgs& a, uint64_t t, f
 template <int V, bool kShort>
 __device__ __forceinline__ void code_tile(const EncodeArgs& a, uint64_t t, const uint32_t* t_after_slot, const uint32_t* rtab,
                                           uint32_t* tbuf, uint32_t* pb, float4* xin, TileSlot& slot,
-                                          uint32_t epoch, bool desc_pending) {
+                                          uint32_t epoch) {
     // tbuf holds the bits of the tile coded two tiles ago (slot.total, set by that
     // tile): clear the words it used
     const uint32_t dirty = min(a.smem_words, static_cast<uint32_t>((slot.total + 31) >> 5) + 2u);
@@ -199,12 +199,7 @@ __device__ __forceinline__ void code_tile(const EncodeArgs& a, uint64_t t, const
     const uint64_t base = b * a.d;
     const uint32_t first = lane * NC;  // first bucket-local coordinate of this lane
 
-    // the tile's input is the oldest pending copy group; the descriptor copies of
-    // the prefix gather, when issued, are the one group after it
-    if (desc_pending)
-        asm volatile("cp.async.wait_group 1;\n" ::: "memory");
-    else
-        asm volatile("cp.async.wait_all;\n" ::: "memory");
+    asm volatile("cp.async.wait_all;\n" ::: "memory");  // the tile's input
     __syncthreads();  // B0: the tile's input has landed; every warp is done with tbuf's last tile
     // clear the words tbuf's last tile used (nothing writes tbuf before B1)
     for (uint32_t i = tid; i < dirty; i += kFastBlock) tbuf[i] = 0u;
@@ -399,75 +394,36 @@ __device__ __forceinline__ bool wait_value(const uint64_t* p, uint64_t state, ui
     }
 }
 
-// Copies the descriptors the prefix gather of tile t = r*C + c will read (tiles
-// [t_lo, t_hi), see gather_prefix) into dpre, as 16-byte pairs: thread k takes the
-// pair (2(p0+k), 2(p0+k)+1), p0 = t_lo / 2, to entries 2k and 2k+1; and RP(r-2)
-// (16 bytes of TileState r-2) into dround.  One cp.async group, issued before the
-// CTA codes its next tile, so the copies travel while it works.  The copies go to
-// L2 only (.cg); the values are plain data, and one that is not ready yet is
-// polled later.
-__device__ __forceinline__ void gather_issue(const EncodeArgs& a, uint32_t r, uint32_t C, uint32_t c,
-                                             uint64_t* dpre, uint64_t* dround) {
-    const int tid = threadIdx.x;
-    const uint64_t t_lo = r >= 1 ? static_cast<uint64_t>(r - 1) * C : 0;
-    const uint64_t t_hi = static_cast<uint64_t>(r) * C + c;
-    const uint64_t p = (t_lo >> 1) + tid;
-    if (2 * p < t_hi && 2 * tid + 1 < kGatherPre) {
-        const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(dpre + 2 * tid));
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(a.tdesc + 2 * p) : "memory");
-    }
-    if (tid == kFastBlock - 1 && r >= 2) {
-        const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(dround));
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(&a.ts[r - 2]) : "memory");
-    }
-    asm volatile("cp.async.commit_group;\n" ::: "memory");
-}
-
 // Exclusive prefix of tile t = r*C + c: RP(r-2) + the bit counts A of every tile
-// of round r-1 + those of round r's tiles before c, all read in parallel.  Thread
-// k sums the pairs p0+k, p0+k+kFastBlock, ...: the first from the copy
-// gather_issue made, the others (and any copy that was not ready yet) from global
-// memory, waiting if needed.  `newer_group`: another copy group was committed after
-// gather_issue's.  One CTA barrier; every thread returns the same value.  `acc` is
-// a zeroed shared accumulator; false when a bounded wait ran out (or another CTA
-// aborted).
+// of round r-1 + those of round r's tiles before c, all read in parallel.  The A
+// values are published when tiles are coded, normally well before they are needed,
+// and RP(r-2) one round earlier.  One CTA barrier; every thread returns the same
+// value.  `acc` is a zeroed shared accumulator; false when a bounded wait ran out
+// (or another CTA aborted).
 __device__ __forceinline__ bool gather_prefix(const EncodeArgs& a, uint32_t r, uint32_t C, uint32_t c,
-                                              uint32_t epoch, const uint64_t* dpre, const uint64_t* dround,
-                                              bool newer_group, unsigned long long* acc, int* bad,
+                                              uint32_t epoch, unsigned long long* acc, int* bad,
                                               uint64_t& prefix) {
     const int tid = threadIdx.x, lane = tid & 31;
-    if (newer_group)
-        asm volatile("cp.async.wait_group 1;\n" ::: "memory");
-    else
-        asm volatile("cp.async.wait_all;\n" ::: "memory");
     uint64_t sum = 0;
     bool ok = true;
+    // tiles [t_lo, t_hi): all of round r-1 and round r up to c; the values are
+    // the data, so relaxed loads suffice
     const uint64_t t_lo = r >= 1 ? static_cast<uint64_t>(r - 1) * C : 0;
     const uint64_t t_hi = static_cast<uint64_t>(r) * C + c;
-    for (uint64_t p = (t_lo >> 1) + tid; 2 * p < t_hi; p += kFastBlock) {
-        const bool copied = p == (t_lo >> 1) + tid && 2 * tid + 1 < kGatherPre;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const uint64_t i = 2 * p + h;
-            if (i < t_lo || i >= t_hi) continue;
-            uint64_t d = copied ? dpre[2 * tid + h] : ld_relaxed(&a.tdesc[i]);
-            if (!(desc_epoch(d) == (epoch & kEpochMask) && desc_state(d) == kStateAggregate)) {
-                uint64_t v = 0;
-                ok = ok && wait_value(&a.tdesc[i], kStateAggregate, epoch, &a.ctrl->abort, v);
-                d = v;
-            } else {
-                d = desc_value(d);
-            }
-            sum += d;
+    for (uint64_t i = t_lo + tid; i < t_hi; i += kFastBlock) {
+        uint64_t d = ld_relaxed(&a.tdesc[i]);
+        if (!(desc_epoch(d) == (epoch & kEpochMask) && desc_state(d) == kStateAggregate)) {
+            uint64_t v = 0;
+            ok = ok && wait_value(&a.tdesc[i], kStateAggregate, epoch, &a.ctrl->abort, v);
+            d = v;
+        } else {
+            d = desc_value(d);
         }
+        sum += d;
     }
     if (tid == kFastBlock - 1 && r >= 2 && ok) {
-        const uint64_t d = dround[1];
         uint64_t v = 0;
-        if (desc_epoch(d) == (epoch & kEpochMask) && desc_state(d) == kStatePrefix)
-            v = desc_value(d);
-        else
-            ok = wait_value(&a.ts[r - 2].round, kStatePrefix, epoch, &a.ctrl->abort, v);
+        ok = wait_value(&a.ts[r - 2].round, kStatePrefix, epoch, &a.ctrl->abort, v);
         sum += v;
     }
 #pragma unroll
@@ -521,66 +477,75 @@ __device__ __forceinline__ void store_tile(const EncodeArgs& a, const uint32_t* 
 
 template <int V, bool kShort>
 __global__ void __launch_bounds__(kFastBlock, (V <= 4 ? kFastMinBlocks : 1)) encode_fast(const __grid_constant__ EncodeArgs a) {
+    constexpr int kEncDepth = enc_depth(V);
+    constexpr int kEncBufs = kEncDepth + 1;
     extern __shared__ __align__(16) uint32_t smem[];
-    __shared__ TileSlot s_slot[2];
+    __shared__ TileSlot s_slot[kEncBufs];
     __shared__ unsigned long long s_acc[2];
     __shared__ int s_bad;
-    __shared__ uint32_t s_ticket[2];  // [0] the first tile; then the ticket drawn each iteration
-    __shared__ __align__(16) uint64_t s_round[2];  // prefetched TileState r-2
+    __shared__ uint32_t s_ticket[kEncDepth + 1];  // the first tickets; then [it & 1] each iteration
     const int tid = threadIdx.x;
-    uint64_t* const dpre = reinterpret_cast<uint64_t*>(smem);                    // prefetched descriptors
-    uint32_t* const rtab = smem + 2 * kGatherPre;                                // record table
-    float4* const xin = reinterpret_cast<float4*>(rtab + kRecordTab);           // kFastWarps * 128V floats
-    uint32_t* const tbuf0 = rtab + kRecordTab + kFastWarps * 128 * V;           // two tile buffers
-    uint32_t* const pb = tbuf0 + 2 * a.smem_words + (tid >> 5) * 32 * fast_lane_words(V, kShort);  // lane strips
+    uint32_t* const rtab = smem;                                                 // record table
+    float4* const xin = reinterpret_cast<float4*>(smem + kRecordTab);           // kFastWarps * 128V floats
+    uint32_t* const tbuf0 = smem + kRecordTab + kFastWarps * 128 * V;           // kEncBufs tile buffers
+    uint32_t* const pb = tbuf0 + kEncBufs * a.smem_words + (tid >> 5) * 32 * fast_lane_words(V, kShort);  // lane strips
     record_table_fill(rtab, tid, kFastBlock);
     const uint32_t epoch = *reinterpret_cast<volatile uint32_t*>(&a.ctrl->epoch);
     const uint32_t C = gridDim.x;
     if (tid == 0) {
-        s_ticket[0] = atomicAdd(&a.ctrl->ticket, 1u);
-        s_ticket[1] = atomicAdd(&a.ctrl->ticket, 1u);
+#pragma unroll
+        for (int j = 0; j <= kEncDepth; ++j) s_ticket[j] = atomicAdd(&a.ctrl->ticket, 1u);
         s_acc[0] = s_acc[1] = 0;
         s_bad = 0;
-        s_slot[0].total = s_slot[1].total = static_cast<uint64_t>(a.smem_words) * 32;  // clear all at first use
+#pragma unroll
+        for (int j = 0; j < kEncBufs; ++j) s_slot[j].total = static_cast<uint64_t>(a.smem_words) * 32;  // clear all at first use
     }
     __syncthreads();
-    uint64_t t = s_ticket[0];
-    uint64_t tn = s_ticket[1];
-    int cur = 0;
-    prefetch_tile<V>(a, t, xin);
-    // the first tile's coding prefetches tn's input: read from s_ticket[1]
-    if (t < a.ntiles) code_tile<V, kShort>(a, t, &s_ticket[1], rtab, tbuf0, pb, xin, s_slot[0], epoch, false);
+    // Prologue: code the first kEncDepth tiles (each coding starts the input copy of
+    // the next ticket at its B1).  held[] are the coded tiles not yet stored, oldest
+    // first; tile number q (in coding order) lives in buffer q mod kEncBufs.
+    uint64_t held[kEncDepth];
+    prefetch_tile<V>(a, s_ticket[0], xin);
+#pragma unroll
+    for (int j = 0; j < kEncDepth; ++j) {
+        held[j] = s_ticket[j];
+        if (held[j] < a.ntiles)
+            code_tile<V, kShort>(a, held[j], &s_ticket[j + 1], rtab, tbuf0 + j * a.smem_words, pb, xin, s_slot[j], epoch);
+    }
+    uint64_t tn = s_ticket[kEncDepth];
     __syncthreads();  // every thread has read s_ticket before the loop reuses it
-    // Per iteration: draw the ticket tnn, code tile tn (its B1 starts the input
-    // copy of tnn; B0 publishes tnn), then gather tile t's prefix and store t.
-    // CTA barriers: B0 and B1 inside the coding, Bg inside the gather.
-    for (int it = 0; t < a.ntiles; ++it) {
+    // Per iteration: draw the ticket tnn; code tile tn (its B1 starts the input copy
+    // of tnn; B0 publishes tnn); gather the prefix of the oldest coded tile and store
+    // it.  CTA barriers: B0 and B1 inside the coding, Bg inside the gather.  Coding
+    // runs kEncDepth tiles ahead of storing, so the tiles a gather waits for have had
+    // kEncDepth iterations to publish their sizes.
+    for (uint32_t it = 0; held[0] < a.ntiles; ++it) {
         if (tid == 0) s_ticket[it & 1] = atomicAdd(&a.ctrl->ticket, 1u);
-        uint32_t* const tcur = tbuf0 + cur * a.smem_words;
-        uint32_t* const tnext = tbuf0 + (cur ^ 1) * a.smem_words;
+        const uint64_t t = held[0];
+        const uint32_t bs = it % kEncBufs;                // buffer of t
+        const uint32_t bn = (it + kEncDepth) % kEncBufs;  // buffer for tn
         const uint32_t r = static_cast<uint32_t>(t) / C;
         const uint32_t c = static_cast<uint32_t>(t) - r * C;
-        // this tile's prefix descriptors travel while the next tile is coded
-        gather_issue(a, r, C, c, dpre, s_round);
         if (tn < a.ntiles)
-            code_tile<V, kShort>(a, tn, &s_ticket[it & 1], rtab, tnext, pb, xin, s_slot[cur ^ 1], epoch, true);
+            code_tile<V, kShort>(a, tn, &s_ticket[it & 1], rtab, tbuf0 + bn * a.smem_words, pb, xin, s_slot[bn], epoch);
         else
             __syncthreads();  // orders the ticket, the accumulator reset and store_tile
         const uint64_t tnn = s_ticket[it & 1];
-        const uint64_t tb = s_slot[cur].total;
+        const uint64_t tb = s_slot[bs].total;
         uint64_t X = 0;
-        const bool ok = gather_prefix(a, r, C, c, epoch, dpre, s_round, tn < a.ntiles, &s_acc[it & 1], &s_bad, X);
+        const bool ok = gather_prefix(a, r, C, c, epoch, &s_acc[it & 1], &s_bad, X);
         if (tid == 0) s_acc[(it + 1) & 1] = 0;  // the next iteration's accumulator
         if (!ok) {
             if (tid == 0) abort_all(a);
         } else {
             if (tid == 0 && ((c + 1 == C) || (t + 1 == a.ntiles)))
                 st_release(&a.ts[r].round, make_desc(epoch, kStatePrefix, X + tb));
-            store_tile(a, tcur, s_slot[cur], t, X, tb, epoch);
+            store_tile(a, tbuf0 + bs * a.smem_words, s_slot[bs], t, X, tb, epoch);
         }
-        t = tn;
+#pragma unroll
+        for (int j = 0; j + 1 < kEncDepth; ++j) held[j] = held[j + 1];
+        held[kEncDepth - 1] = tn;
         tn = tnn;
-        cur ^= 1;
     }
     asm volatile("cp.async.wait_all;\n" ::: "memory");
     __syncthreads();

@@ -64,19 +64,15 @@ inline uint32_t fast_v(uint32_t d) {
 __host__ __device__ inline constexpr uint32_t fast_lane_words(uint32_t V, bool short_records) {
     return (4 * V * (short_records ? 30u : 51u) + 31u) / 32u + 1u;
 }
-// Tile descriptors the fast encoder copies into shared memory ahead of its prefix
-// gather (two per thread); a gather over more tiles reads the rest directly.
-constexpr uint32_t kGatherPre = 2 * kFastBlock;
-// Dynamic shared memory of the fast encoder: prefetched descriptors (uint64) |
-// record table | one tile of input (kFastWarps * 128V floats; also the warps'
-// record lists) | two tile buffers | the lane strips.
+// Dynamic shared memory of the fast encoder: record table | one tile of input
+// (kFastWarps * 128V floats; also the warps' record lists) | kEncBufs tile buffers |
+// the lane strips.
 inline size_t fast_smem_bytes(uint32_t d, uint32_t s, uint32_t smem_words) {
     const uint32_t v = fast_v(d);
-    return static_cast<size_t>(kGatherPre) * sizeof(uint64_t) +
-           (static_cast<size_t>(kRecordTab) + static_cast<size_t>(kFastWarps) * 128 * v +
-            2 * static_cast<size_t>(smem_words) +
+    return (static_cast<size_t>(kRecordTab) + static_cast<size_t>(kFastWarps) * 128 * v +
+            static_cast<size_t>(enc_depth(v) + 1) * smem_words +
             static_cast<size_t>(kFastWarps) * 32 * fast_lane_words(v, s <= 31)) *
-               sizeof(uint32_t);
+           sizeof(uint32_t);
 }
 
 struct StreamRef {
