@@ -75,6 +75,12 @@ def _declare(lib):
         "qo_decode_levels": (c_int, [u32p, u64p, c_u64, c_u64, c_u32, i32p, f32p, u32p]),
         "qo_decode_accumulate": (c_int, [ctypes.POINTER(u32p), ctypes.POINTER(u64p), c_int,
                                          c_u64, c_u64, c_u32, f32p, u32p]),
+        "qo_bbit_levels": (c_u32, [c_u32]),
+        "qo_bbit_code_words": (c_u64, [c_u64, c_u32]),
+        "qo_bbit_encode": (c_int, [f32p, c_u64, c_u64, c_u32, c_u64, f32p, f32p, u32p, u32p]),
+        "qo_bbit_decode": (c_int, [f32p, u32p, c_u64, c_u64, c_u32, f32p, u32p]),
+        "qo_bbit_decode_accumulate": (c_int, [ctypes.POINTER(f32p), ctypes.POINTER(u32p), c_int,
+                                              c_u64, c_u64, c_u32, f32p, u32p]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -273,6 +279,68 @@ class Oracle:
         buf = out if n else np.zeros(1, np.float32)
         rc = self.lib.qo_decode_accumulate(wp, op, K, n, d, s, _ptr(buf, ctypes.c_float),
                                            ctypes.byref(st))
+        assert rc == 0
+        return out, st.value
+
+
+    # ---- fixed-width b-bit variant ----------------------------------------------
+    def bbit_levels(self, b: int) -> int:
+        return int(self.lib.qo_bbit_levels(b))
+
+    def bbit_code_words(self, n: int, b: int) -> int:
+        return int(self.lib.qo_bbit_code_words(n, b))
+
+    def bbit_encode(self, v: np.ndarray, d: int, b: int, seed: int, norms_in=None):
+        """Returns (codes uint32[ceil(n*b/32)], norms float32[nb], status)."""
+        v = np.ascontiguousarray(v, dtype=np.float32)
+        n = v.size
+        nb = (n + d - 1) // d
+        codes = np.zeros(max(self.bbit_code_words(n, b), 1), dtype=np.uint32)
+        norms = np.zeros(max(nb, 1), dtype=np.float32)
+        st = ctypes.c_uint32(0)
+        nin = None
+        if norms_in is not None:
+            nin = np.ascontiguousarray(norms_in, dtype=np.float32)
+            assert nin.size == nb
+        vv = v if n else np.zeros(1, np.float32)
+        rc = self.lib.qo_bbit_encode(_ptr(vv, ctypes.c_float), n, d, b, seed,
+                                     _ptr(nin, ctypes.c_float) if nin is not None else None,
+                                     _ptr(norms, ctypes.c_float), _ptr(codes, ctypes.c_uint32),
+                                     ctypes.byref(st))
+        if rc != 0:
+            raise ValueError("oracle b-bit encode rejected b=%d d=%d" % (b, d))
+        return codes[:self.bbit_code_words(n, b)].copy(), norms[:nb].copy(), st.value
+
+    def bbit_decode(self, norms: np.ndarray, codes: np.ndarray, n: int, d: int, b: int):
+        norms = np.ascontiguousarray(norms, dtype=np.float32)
+        codes = np.ascontiguousarray(codes, dtype=np.uint32)
+        if codes.size == 0:
+            codes = np.zeros(1, np.uint32)
+        if norms.size == 0:
+            norms = np.zeros(1, np.float32)
+        out = np.zeros(max(n, 1), dtype=np.float32)
+        st = ctypes.c_uint32(0)
+        rc = self.lib.qo_bbit_decode(_ptr(norms, ctypes.c_float), _ptr(codes, ctypes.c_uint32), n, d, b,
+                                     _ptr(out, ctypes.c_float), ctypes.byref(st))
+        assert rc == 0
+        return out[:n], st.value
+
+    def bbit_decode_accumulate(self, streams, n: int, d: int, b: int, out: np.ndarray):
+        """streams: list of (norms, codes).  out is updated in place and returned."""
+        K = len(streams)
+        ns = [np.ascontiguousarray(x if x.size else np.zeros(1, np.float32), dtype=np.float32)
+              for x, _ in streams]
+        cs = [np.ascontiguousarray(c if c.size else np.zeros(1, np.uint32), dtype=np.uint32)
+              for _, c in streams]
+        f32p = ctypes.POINTER(ctypes.c_float)
+        u32p = ctypes.POINTER(ctypes.c_uint32)
+        npp = (f32p * K)(*[_ptr(x, ctypes.c_float) for x in ns])
+        cpp = (u32p * K)(*[_ptr(c, ctypes.c_uint32) for c in cs])
+        assert out.dtype == np.float32 and out.flags["C_CONTIGUOUS"] and out.size == n
+        st = ctypes.c_uint32(0)
+        buf = out if n else np.zeros(1, np.float32)
+        rc = self.lib.qo_bbit_decode_accumulate(npp, cpp, K, n, d, b, _ptr(buf, ctypes.c_float),
+                                                ctypes.byref(st))
         assert rc == 0
         return out, st.value
 

@@ -371,3 +371,98 @@ int qo_decode_accumulate(const uint32_t* const* words, const uint64_t* const* of
     free(q);
     return 0;
 }
+
+/* ------------------------------------------------------------------------- */
+/* Fixed-width b-bit variant: the quantiser above with s = 2^(b-1) - 1, each  */
+/* coordinate's level and sign in b bits at a fixed place; no gaps, no omega. */
+/* ------------------------------------------------------------------------- */
+
+uint32_t qo_bbit_levels(uint32_t b) {
+    return (b == 2 || b == 4 || b == 8) ? (1u << (b - 1)) - 1u : 0u;
+}
+
+uint64_t qo_bbit_code_words(uint64_t n, uint32_t b) {
+    return (n * (uint64_t)b + 31u) / 32u;
+}
+
+int qo_bbit_encode(const float* v, uint64_t n, uint64_t d, uint32_t b, uint64_t seed,
+                   const float* norms_in, float* norms_out, uint32_t* codes, uint32_t* status) {
+    uint32_t s = qo_bbit_levels(b);
+    if (s == 0 || d < 1) return -1;
+    uint64_t nw = qo_bbit_code_words(n, b);
+    for (uint64_t w = 0; w < nw; ++w) codes[w] = 0;
+    uint64_t nb = (n + d - 1) / d;
+    int32_t* levels = (int32_t*)malloc((size_t)(d ? d : 1) * sizeof(int32_t));
+    if (!levels) return -1;
+    for (uint64_t bk = 0; bk < nb; ++bk) {
+        uint64_t base = bk * d;
+        uint64_t m = (bk + 1 == nb) ? n - base : d;
+        float norm = qo_quantize_bucket(v + base, m, base, s, seed, norms_in ? norms_in + bk : 0, levels, status);
+        norms_out[bk] = norm;
+        for (uint64_t i = 0; i < m; ++i) {
+            uint32_t k = (uint32_t)(levels[i] < 0 ? -levels[i] : levels[i]);
+            uint32_t code = ((levels[i] < 0 ? 1u : 0u) << (b - 1)) | k;
+            uint64_t pos = (base + i) * b;
+            put_bits_msb_first(codes, nw, &pos, code, (int)b);
+        }
+    }
+    free(levels);
+    return 0;
+}
+
+int qo_bbit_decode(const float* norms, const uint32_t* codes, uint64_t n, uint64_t d, uint32_t b,
+                   float* out, uint32_t* status) {
+    uint32_t s = qo_bbit_levels(b);
+    if (s == 0 || d < 1) return -1;
+    uint64_t nw = qo_bbit_code_words(n, b);
+    uint64_t nb = (n + d - 1) / d;
+    for (uint64_t bk = 0; bk < nb; ++bk) {
+        uint64_t base = bk * d;
+        uint64_t m = (bk + 1 == nb) ? n - base : d;
+        float norm = norms[bk];
+        float scale = norm / (float)s;
+        int bad = !isfinite(norm) || signbit(norm);
+        for (uint64_t i = 0; i < m; ++i) {
+            uint64_t pos = (base + i) * b;
+            uint32_t code = 0;
+            for (uint32_t t = 0; t < b; ++t) {
+                int bit = 0;
+                get_bit(codes, &pos, nw * 32u, &bit);
+                code = (code << 1) | (uint32_t)bit;
+            }
+            uint32_t sign = code >> (b - 1);
+            uint32_t k = code & s;
+            float value = 0.0f;
+            if (k == 0) {
+                if (sign) bad = 1; /* a sign on a zero level: no encoder writes it */
+            } else if (norm == 0.0f || scale == 0.0f) {
+                bad = 1; /* levels under a norm that carries none */
+            } else {
+                value = scale * (float)k;
+                if (sign) value = -value;
+            }
+            out[base + i] = value;
+        }
+        if (bad) {
+            *status |= QO_ST_BAD_STREAM;
+            for (uint64_t i = 0; i < m; ++i) out[base + i] = 0.0f;
+        }
+    }
+    return 0;
+}
+
+int qo_bbit_decode_accumulate(const float* const* norms, const uint32_t* const* codes, int K,
+                              uint64_t n, uint64_t d, uint32_t b, float* out, uint32_t* status) {
+    if (K < 1) return -1;
+    float* q = (float*)malloc((size_t)(n ? n : 1) * sizeof(float));
+    if (!q) return -1;
+    for (int j = 0; j < K; ++j) {
+        if (qo_bbit_decode(norms[j], codes[j], n, d, b, q, status) != 0) {
+            free(q);
+            return -1;
+        }
+        for (uint64_t i = 0; i < n; ++i) out[i] = out[i] + q[i];
+    }
+    free(q);
+    return 0;
+}

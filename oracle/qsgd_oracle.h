@@ -104,6 +104,33 @@ int qo_decode_accumulate(const uint32_t* const* words, const uint64_t* const* of
                          int K, uint64_t n, uint64_t d, uint32_t s, float* out,
                          uint32_t* status);
 
+/* ---- Fixed-width b-bit variant (b = 2, 4, 8) ----------------------------------
+ * The "4-bit and 2-bit QSGD" of the claim "QSVRG, non-convex and multi-GPU bucketed
+ * training" (and the 4/8-bit of the curated limitations): s = 2^(b-1) - 1 levels, the
+ * same quantiser and random words as above, and per coordinate a b-bit code
+ * (sign << (b-1)) | k packed densely at bits [i*b, i*b + b) of the code words,
+ * MSB-first; one fp32 norm per bucket in its own array. */
+
+/* s = 2^(b-1) - 1 for b in {2, 4, 8}; 0 otherwise. */
+uint32_t qo_bbit_levels(uint32_t b);
+
+/* Words of the code array for n coordinates: ceil(n*b / 32). */
+uint64_t qo_bbit_code_words(uint64_t n, uint32_t b);
+
+/* codes must hold qo_bbit_code_words(n, b) words (cleared here); norms_out[nb]
+ * receives the sent norms.  norms_in (nullable) replaces the computed norms. */
+int qo_bbit_encode(const float* v, uint64_t n, uint64_t d, uint32_t b, uint64_t seed,
+                   const float* norms_in, float* norms_out, uint32_t* codes, uint32_t* status);
+
+/* Dense decode; BAD_STREAM for a negative or non-finite norm, a non-zero code under
+ * a zero norm or a zero scale fl(norm/s), or a code with sign 1 and k = 0. */
+int qo_bbit_decode(const float* norms, const uint32_t* codes, uint64_t n, uint64_t d, uint32_t b,
+                   float* out, uint32_t* status);
+
+/* out[i] <- out[i] + q^0[i] + ... + q^{K-1}[i], left to right. */
+int qo_bbit_decode_accumulate(const float* const* norms, const uint32_t* const* codes, int K,
+                              uint64_t n, uint64_t d, uint32_t b, float* out, uint32_t* status);
+
 #ifdef __cplusplus
 }
 #endif
