@@ -420,7 +420,7 @@ int qo_bbit_decode(const float* norms, const uint32_t* codes, uint64_t n, uint64
         uint64_t base = bk * d;
         uint64_t m = (bk + 1 == nb) ? n - base : d;
         float norm = norms[bk];
-        float scale = norm / (float)s;
+        float bscale = norm / (float)s; /* fl(norm / s) */
         int bad = !isfinite(norm) || signbit(norm);
         for (uint64_t i = 0; i < m; ++i) {
             uint64_t pos = (base + i) * b;
@@ -435,10 +435,10 @@ int qo_bbit_decode(const float* norms, const uint32_t* codes, uint64_t n, uint64
             float value = 0.0f;
             if (k == 0) {
                 if (sign) bad = 1; /* a sign on a zero level: no encoder writes it */
-            } else if (norm == 0.0f || scale == 0.0f) {
+            } else if (norm == 0.0f || bscale == 0.0f) {
                 bad = 1; /* levels under a norm that carries none */
             } else {
-                value = scale * (float)k;
+                value = bscale * (float)k;
                 if (sign) value = -value;
             }
             out[base + i] = value;
@@ -461,7 +461,7 @@ int qo_bbit_decode_accumulate(const float* const* norms, const uint32_t* const* 
             free(q);
             return -1;
         }
-        for (uint64_t i = 0; i < n; ++i) out[i] = out[i] + q[i];
+        for (uint64_t i = 0; i < n; ++i) out[i] += q[i]; /* one fp32 add, as above */
     }
     free(q);
     return 0;

@@ -32,11 +32,14 @@ def test_levels_per_width(oracle_lib, b, s):
 #  b=4, v = (2, -3, 6, 0..): ||v|| = 7, k = (2, 3, 6) -> codes 0010 1011 0110
 #  b=2, v = (0, -1, 0, 0): s = 1, ||v|| = 1, k_1 = 1, sign 1 -> code 11 at bits 2..3
 #  b=8, v = (127, 0, 0, 0): s = 127 = ||v||, k_0 = 127 -> code 0111 1111
+#  b=4, v = (0, 14, 0..): ||v|| = 14, s/||v|| = 0.5, k_1 = 7 -> code 0111; decodes to
+#       fl(14/7) * 7 = 14 (a norm other than s, so the decode's scale is pinned too)
 GOLDEN = [
     (4, [0, -7, 0, 0, 0, 0, 0, 0], 8, [0x0F000000], [7.0]),
     (4, [2, -3, 6, 0, 0, 0, 0, 0], 8, [0x2B600000], [7.0]),
     (2, [0, -1, 0, 0], 4, [0x30000000], [1.0]),
     (8, [127, 0, 0, 0], 4, [0x7F000000], [127.0]),
+    (4, [0, 14, 0, 0, 0, 0, 0, 0], 8, [0x07000000], [14.0]),
     # two buckets of 4 (b = 4): (0, 0, 7, 0) and (0, -7, 0, 0) -> 0000 0000 0111 0000 | 0000 1111 ...
     (4, [0, 0, 7, 0, 0, -7, 0, 0], 4, [0x00700F00], [7.0, 7.0]),
 ]

@@ -45,6 +45,16 @@ MUTANTS = {
     "decode_sign_dropped": ("if (q < 0) value = -value;", ""),
     "accumulate_overwrites": ("out[i] = out[i] + q[i];", "out[i] = q[i];"),
     "decode_index_not_advanced": ("idx += (int64_t)gap;", "idx += 1;"),
+    # fixed-width b-bit variant
+    "bbit_sign_in_low_bit": ("uint32_t code = ((levels[i] < 0 ? 1u : 0u) << (b - 1)) | k;",
+                             "uint32_t code = (k << 1) | (levels[i] < 0 ? 1u : 0u);"),
+    "bbit_levels_full_width": ("(1u << (b - 1)) - 1u : 0u;", "(1u << b) - 1u : 0u;"),
+    "bbit_decode_sign_dropped": ("if (sign) value = -value;", ""),
+    "bbit_decode_scale_inverted": ("float bscale = norm / (float)s;", "float bscale = (float)s / norm;"),
+    "bbit_sign_on_zero_accepted": ("if (sign) bad = 1; /* a sign on a zero level: no encoder writes it */", ""),
+    "bbit_accumulate_overwrites": ("out[i] += q[i];", "out[i] = q[i];"),
+    "bbit_code_shifted": ("uint64_t pos = (base + i) * b;\n            put_bits_msb_first",
+                          "uint64_t pos = (base + i) * b + 1;\n            put_bits_msb_first"),
 }
 
 
@@ -116,8 +126,39 @@ def pin_battery(o) -> list:
     expect = np.array([f(f(0.5) + f(3)) + f(0), f(f(-0.0) + f(4)) + f(-0.4)], np.float32)
     if out.view(np.uint32).tolist() != expect.view(np.uint32).tolist():
         failed.append("accumulate_hand")
-    # small unbiasedness sweep: 4096 N(0,1) coordinates, s = 8, 400 seeds
     from quantized_gradient_compression_b200 import workloads
+
+    # b-bit variant: hand-derived words, the Elias path's levels, malformed codes,
+    # decode-accumulate
+    try:
+        for bw, vv, dd, words_expect in [(4, [2, -3, 6, 0, 0, 0, 0, 0], 8, [0x2B600000]),
+                                          (4, [0, 14, 0, 0, 0, 0, 0, 0], 8, [0x07000000]),
+                                          (2, [0, -1, 0, 0], 4, [0x30000000]),
+                                          (4, [0, 0, 7, 0, 0, -7, 0, 0], 4, [0x00700F00])]:
+            vv = np.array(vv, np.float32)
+            codes, nrm, _ = o.bbit_encode(vv, dd, bw, 3)
+            dec, st = o.bbit_decode(nrm, codes, vv.size, dd, bw)
+            if [int(x) for x in codes] != words_expect or st != 0 or not np.array_equal(dec, vv):
+                failed.append("bbit_golden")
+                break
+        vv = workloads.normal(300, 5)
+        lv, _, _ = o.quantize(vv, 100, 7, 2)
+        codes, nrm, _ = o.bbit_encode(vv, 100, 4, 2)
+        bits = np.unpackbits(codes.astype(">u4").view(np.uint8))[:1200].reshape(300, 4)
+        code = (bits * np.array([8, 4, 2, 1])).sum(axis=1)
+        if not (np.array_equal(code & 7, np.abs(lv)) and np.array_equal(code >> 3, (lv < 0).astype(int))):
+            failed.append("bbit_levels")
+        _, st = o.bbit_decode(np.array([7.0], np.float32), np.array([0x2B680000], np.uint32), 8, 8, 4)
+        if not st & oracle_mod.ST_BAD_STREAM:
+            failed.append("bbit_malformed")
+        acc = np.array([0.25] * 8, np.float32)
+        c1, n1, _ = o.bbit_encode(np.array([2, -3, 6, 0, 0, 0, 0, 0], np.float32), 8, 4, 1)
+        o.bbit_decode_accumulate([(n1, c1), (n1, c1)], 8, 8, 4, acc)
+        if acc.tolist() != [4.25, -5.75, 12.25, 0.25, 0.25, 0.25, 0.25, 0.25]:
+            failed.append("bbit_accumulate")
+    except (ValueError, AssertionError):
+        failed.append("bbit")
+    # small unbiasedness sweep: 4096 N(0,1) coordinates, s = 8, 400 seeds
     v = workloads.normal(4096, 1)
     sums = sc.Sums(v.size)
     v64 = v.astype(np.float64)
