@@ -397,6 +397,53 @@ def run_ours(args, w):
     if int(status.item()) != 0:
         raise RuntimeError("device status %d in the end-to-end run" % int(status.item()))
 
+    # fixed-width b-bit variant on the same vector: each call timed alone, L2 flushed
+    bbit = {}
+    for bw in (2, 4, 8):
+        cw = B.qsgd_bbit_code_words(n, bw)
+        norms_b = torch.empty(nb, dtype=torch.float32, device=dev)
+        codes_b = torch.empty(max(cw, 1), dtype=torch.int32, device=dev)
+        out_b = torch.empty(n, dtype=torch.float32, device=dev)
+        acc_b = torch.zeros(n, dtype=torch.float32, device=dev)
+
+        def b_enc():
+            check(B.qsgd_bbit_encode(x.data_ptr(), n, d, bw, seed, norms_b.data_ptr(), codes_b.data_ptr(),
+                                     status.data_ptr(), sh), "qsgd_bbit_encode")
+
+        def b_dec():
+            check(B.qsgd_bbit_decode(norms_b.data_ptr(), codes_b.data_ptr(), n, d, bw, out_b.data_ptr(),
+                                     status.data_ptr(), sh), "qsgd_bbit_decode")
+
+        def b_acc():
+            check(B.qsgd_bbit_decode_accumulate([norms_b.data_ptr()], [codes_b.data_ptr()], 1, n, d, bw,
+                                                acc_b.data_ptr(), status.data_ptr(), sh),
+                  "qsgd_bbit_decode_accumulate")
+
+        times = {}
+        for name, fn in (("encode", b_enc), ("decode", b_dec), ("decode_accumulate", b_acc)):
+            for _ in range(3):
+                fn()
+            ts = []
+            for _ in range(max(3, min(K, 50))):
+                flush.zero_()
+                e_a, e_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e_a.record(stream)
+                fn()
+                e_b.record(stream)
+                torch.cuda.synchronize()
+                ts.append(e_a.elapsed_time(e_b))
+            times[name] = statistics.median(ts)
+        if int(status.item()) != 0:
+            raise RuntimeError("device status %d in the b-bit runs" % int(status.item()))
+        cbytes = 4.0 * nb + 4.0 * cw
+        alg = {"encode": 4.0 * n + cbytes, "decode": cbytes + 4.0 * n, "decode_accumulate": cbytes + 8.0 * n}
+        bbit["b%d" % bw] = {
+            "s": (1 << (bw - 1)) - 1, "bits_per_coord": bw + 32.0 * nb / n,
+            "us": {k: 1e3 * v for k, v in times.items()},
+            "algorithmic_gbs": {k: alg[k] / times[k] / 1e6 for k in times},
+            "roofline_frac": {k: alg[k] / times[k] / 1e6 / measured_peaks()[0] for k in times},
+        }
+
     peak, peak_kind = measured_peaks()
     in_bytes = 4.0 * n
     enc_bytes = in_bytes + comp_bytes            # read fp32, write stream + header
@@ -448,6 +495,7 @@ def run_ours(args, w):
                 "how": "qsgd_encode/decode/decode_accumulate on host-pinned data; per step H2D of the "
                        "input and D2H of the result, pipelined over copy-in / compute / copy-out streams"},
         "gpu_launches": 3 * K,
+        "bbit": bbit,
         "clocks": clocks.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -171,6 +171,42 @@ QSGD_API int qsgd_encode_static_ws(const float* d_in, uint64_t n, uint32_t d, ui
 /* Bytes of the fixed device workspace behind qsgd_encode_static_ws. */
 QSGD_API size_t qsgd_static_workspace_limit(void);
 
+/* ---- Fixed-width b-bit QSGD (b = 2, 4, 8) ---------------------------------------
+ * The "4-bit and 2-bit QSGD" of the claim "QSVRG, non-convex and multi-GPU bucketed
+ * training" (and the 4/8-bit of the curated limitations): s = 2^(b-1) - 1 levels with
+ * the quantiser, random words and bucket norms of qsgd_encode; no Elias coding.  The
+ * page gives no layout; this library's (its "Fixed-width b-bit variant" section):
+ *   d_norms  float32[nb], the sent norm of every bucket (0 for a zero, non-finite or
+ *            out-of-range bucket, which also sets NONFINITE / RANGE);
+ *   d_codes  uint32[qsgd_bbit_code_words(n, b)]: coordinate i has the code
+ *            (sign << (b-1)) | k at bits [i*b, i*b + b), MSB-first in each word (bit j
+ *            is bit 31 - j%32 of word j/32); the sign bit is 1 only for k >= 1 and a
+ *            negative v_i; bits past n*b are 0.
+ * Every code sits at a fixed place, so both directions are data-parallel passes. */
+
+/* Words of the code array: ceil(n * b / 32). */
+QSGD_API uint64_t qsgd_bbit_code_words(uint64_t n, uint32_t b);
+
+/* b-bit encoder.  b in {2, 4, 8}, else QSGD_ERR_ARG; d_norms 4-byte aligned, d_codes
+ * 4-byte aligned with qsgd_bbit_code_words(n, b) words.  Allocates nothing; one or two
+ * kernel launches on `stream`.  Codes are a deterministic function of
+ * (d_in, n, d, b, seed); norms within 1e-6 relative of the exactly rounded norm. */
+QSGD_API int qsgd_bbit_encode(const float* d_in, uint64_t n, uint32_t d, uint32_t b, uint64_t seed,
+                              float* d_norms, uint32_t* d_codes, uint32_t* d_status, cudaStream_t stream);
+
+/* b-bit decoder: d_out[0..n) = fl(fl(norm/s) * k), negated for sign 1, +0.0 for k = 0.
+ * Sets QSGD_ST_BAD_STREAM for a negative or non-finite norm, a non-zero code under a
+ * zero norm or a zero scale, or a code with sign 1 and k = 0 (that bucket's output is
+ * then unspecified; nothing outside d_out[0..n) is written). */
+QSGD_API int qsgd_bbit_decode(const float* d_norms, const uint32_t* d_codes, uint64_t n, uint32_t d,
+                              uint32_t b, float* d_out, uint32_t* d_status, cudaStream_t stream);
+
+/* b-bit receiver aggregation: d_out[i] <- ((d_out[i] + q^0_i) + ...) + q^{K-1}_i, fp32
+ * adds in stream order.  h_norms, h_codes: host arrays of K device pointers; 1 <= K. */
+QSGD_API int qsgd_bbit_decode_accumulate(const float* const* h_norms, const uint32_t* const* h_codes, int K,
+                                         uint64_t n, uint32_t d, uint32_t b, float* d_out, uint32_t* d_status,
+                                         cudaStream_t stream);
+
 /* Static description of a host return code. */
 QSGD_API const char* qsgd_error_string(int code);
 

@@ -51,6 +51,11 @@ _SIGS = {
                                       _int, _u64, _u32, _u32, _vp, _vp, _vp]),
     "qsgd_encode_static_ws": (_int, [_vp, _u64, _u32, _u32, _u64, _vp, _u64, _vp, _vp, _vp]),
     "qsgd_static_workspace_limit": (_sz, []),
+    "qsgd_bbit_code_words": (_u64, [_u64, _u32]),
+    "qsgd_bbit_encode": (_int, [_vp, _u64, _u32, _u32, _u64, _vp, _vp, _vp, _vp]),
+    "qsgd_bbit_decode": (_int, [_vp, _vp, _u64, _u32, _u32, _vp, _vp, _vp]),
+    "qsgd_bbit_decode_accumulate": (_int, [ctypes.POINTER(_vp), ctypes.POINTER(_vp), _int, _u64, _u32, _u32,
+                                           _vp, _vp, _vp]),
     "qsgd_error_string": (ctypes.c_char_p, [_int]),
     "qsgd_version": (ctypes.c_char_p, []),
 }
@@ -120,6 +125,27 @@ def qsgd_encode_static_ws(d_in: int, n: int, d: int, s: int, seed: int, d_words:
 
 def qsgd_static_workspace_limit() -> int:
     return int(_lib.qsgd_static_workspace_limit())
+
+
+def qsgd_bbit_code_words(n: int, b: int) -> int:
+    return int(_lib.qsgd_bbit_code_words(n, b))
+
+
+def qsgd_bbit_encode(d_in: int, n: int, d: int, b: int, seed: int, d_norms: int, d_codes: int, d_status: int,
+                     stream: int) -> int:
+    return int(_lib.qsgd_bbit_encode(d_in, n, d, b, seed & 0xFFFFFFFFFFFFFFFF, d_norms, d_codes, d_status, stream))
+
+
+def qsgd_bbit_decode(d_norms: int, d_codes: int, n: int, d: int, b: int, d_out: int, d_status: int,
+                     stream: int) -> int:
+    return int(_lib.qsgd_bbit_decode(d_norms, d_codes, n, d, b, d_out, d_status, stream))
+
+
+def qsgd_bbit_decode_accumulate(h_norms, h_codes, K: int, n: int, d: int, b: int, d_out: int, d_status: int,
+                                stream: int) -> int:
+    nn = (_vp * K)(*h_norms)
+    cc = (_vp * K)(*h_codes)
+    return int(_lib.qsgd_bbit_decode_accumulate(nn, cc, K, n, d, b, d_out, d_status, stream))
 
 
 def qsgd_error_string(code: int) -> str:
@@ -211,4 +237,60 @@ def decode_accumulate(encs, out, status=None):
     _check(qsgd_decode_accumulate([e.words.data_ptr() for e in encs], [e.num_words for e in encs],
                                   [e.offsets.data_ptr() for e in encs], len(encs), e0.n, e0.d, e0.s,
                                   out.data_ptr(), status.data_ptr(), stream), "qsgd_decode_accumulate")
+    return out, status
+
+
+# --- fixed-width b-bit variant -------------------------------------------------
+
+@dataclass
+class BbitEncoded:
+    norms: "object"   # torch.float32 tensor [nb]
+    codes: "object"   # torch.int32 tensor [qsgd_bbit_code_words(n, b)] (uint32 bit patterns)
+    n: int
+    d: int
+    b: int
+    seed: int
+    status: "object"  # torch.int32 tensor [1]
+
+
+def bbit_encode(x, d: int, b: int, seed: int, norms=None, codes=None, status=None) -> BbitEncoded:
+    torch = _torch()
+    assert x.is_cuda and x.dtype == torch.float32 and x.is_contiguous()
+    n = x.numel()
+    dev = x.device
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    if norms is None:
+        norms = torch.empty(max(qsgd_num_buckets(n, d), 1), dtype=torch.float32, device=dev)
+    if codes is None:
+        codes = torch.empty(max(qsgd_bbit_code_words(n, b), 1), dtype=torch.int32, device=dev)
+    if status is None:
+        status = torch.zeros(1, dtype=torch.int32, device=dev)
+    _check(qsgd_bbit_encode(x.data_ptr(), n, d, b, seed, norms.data_ptr(), codes.data_ptr(), status.data_ptr(),
+                            stream), "qsgd_bbit_encode")
+    return BbitEncoded(norms, codes, n, d, b, seed, status)
+
+
+def bbit_decode(enc: BbitEncoded, out=None, status=None):
+    torch = _torch()
+    dev = enc.codes.device
+    if out is None:
+        out = torch.empty(enc.n, dtype=torch.float32, device=dev)
+    if status is None:
+        status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    _check(qsgd_bbit_decode(enc.norms.data_ptr(), enc.codes.data_ptr(), enc.n, enc.d, enc.b, out.data_ptr(),
+                            status.data_ptr(), stream), "qsgd_bbit_decode")
+    return out, status
+
+
+def bbit_decode_accumulate(encs, out, status=None):
+    torch = _torch()
+    e0 = encs[0]
+    dev = out.device
+    if status is None:
+        status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    _check(qsgd_bbit_decode_accumulate([e.norms.data_ptr() for e in encs], [e.codes.data_ptr() for e in encs],
+                                       len(encs), e0.n, e0.d, e0.b, out.data_ptr(), status.data_ptr(), stream),
+           "qsgd_bbit_decode_accumulate")
     return out, status

@@ -191,6 +191,48 @@ int qsgd_decode_accumulate(const uint32_t* const* h_words, const uint64_t* h_num
     return decode_impl(h_words, h_num_words, h_offsets, K, n, d, s, d_out, d_status, stream, true);
 }
 
+uint64_t qsgd_bbit_code_words(uint64_t n, uint32_t b) { return (n * static_cast<uint64_t>(b) + 31u) / 32u; }
+
+static bool valid_bbit(uint64_t n, uint32_t d, uint32_t b) {
+    return (b == 2 || b == 4 || b == 8) && d >= 1 && d <= kMaxD && n <= kMaxN;
+}
+
+int qsgd_bbit_encode(const float* d_in, uint64_t n, uint32_t d, uint32_t b, uint64_t seed, float* d_norms,
+                     uint32_t* d_codes, uint32_t* d_status, cudaStream_t stream) {
+    if (!valid_bbit(n, d, b) || !d_status) return QSGD_ERR_ARG;
+    if (n == 0) return QSGD_OK;
+    if (!d_in || !d_norms || !d_codes || (reinterpret_cast<uintptr_t>(d_in) & 3u) != 0 ||
+        (reinterpret_cast<uintptr_t>(d_norms) & 3u) != 0 || (reinterpret_cast<uintptr_t>(d_codes) & 3u) != 0)
+        return QSGD_ERR_ARG;
+    return launch_bbit_encode(d_in, n, d, b, seed, d_norms, d_codes, d_status, stream) == cudaSuccess ? QSGD_OK
+                                                                                                     : QSGD_ERR_CUDA;
+}
+
+int qsgd_bbit_decode(const float* d_norms, const uint32_t* d_codes, uint64_t n, uint32_t d, uint32_t b,
+                     float* d_out, uint32_t* d_status, cudaStream_t stream) {
+    if (!valid_bbit(n, d, b) || !d_status) return QSGD_ERR_ARG;
+    if (n == 0) return QSGD_OK;
+    if (!d_norms || !d_codes || !d_out || (reinterpret_cast<uintptr_t>(d_out) & 3u) != 0) return QSGD_ERR_ARG;
+    return launch_bbit_decode(d_norms, d_codes, n, d, b, d_out, false, d_status, stream) == cudaSuccess
+               ? QSGD_OK
+               : QSGD_ERR_CUDA;
+}
+
+int qsgd_bbit_decode_accumulate(const float* const* h_norms, const uint32_t* const* h_codes, int K, uint64_t n,
+                                uint32_t d, uint32_t b, float* d_out, uint32_t* d_status, cudaStream_t stream) {
+    if (!valid_bbit(n, d, b) || !d_status || K < 1 || !h_norms || !h_codes) return QSGD_ERR_ARG;
+    if (n == 0) return QSGD_OK;
+    if (!d_out || (reinterpret_cast<uintptr_t>(d_out) & 3u) != 0) return QSGD_ERR_ARG;
+    for (int j = 0; j < K; ++j)
+        if (!h_norms[j] || !h_codes[j]) return QSGD_ERR_ARG;
+    // one launch per stream, in order on `stream`: every coordinate's adds run left
+    // to right
+    for (int j = 0; j < K; ++j)
+        if (launch_bbit_decode(h_norms[j], h_codes[j], n, d, b, d_out, true, d_status, stream) != cudaSuccess)
+            return QSGD_ERR_CUDA;
+    return QSGD_OK;
+}
+
 const char* qsgd_error_string(int code) {
     switch (code) {
         case QSGD_OK: return "ok";

@@ -37,57 +37,11 @@ namespace {
 
 constexpr uint32_t kFull = 0xFFFFFFFFu;
 
-__device__ __forceinline__ void report(uint32_t* status, uint32_t bits) { atomicOr(status, bits); }
-
 __device__ __forceinline__ void store_word(const EncodeArgs& a, uint64_t gw, uint32_t v) {
     if (gw < a.cap_words)
         a.words[gw] = v;
     else
         report(a.status, QSGD_ST_OVERFLOW);
-}
-
-// Bucket norm and the reciprocal scale s/norm (definition paragraph: the levels
-// are s|v_i|/||v||_2).  Degenerate buckets (zero, non-finite, or s/norm beyond
-// fp32) are sent as a zero norm with no record.
-struct BucketScale {
-    float sent;
-    float sinv;
-    bool good;
-};
-
-__device__ __forceinline__ BucketScale bucket_scale(float norm, uint32_t s, bool live,
-                                                    uint32_t* status, bool reporter) {
-    BucketScale r{0.f, 0.f, false};
-    if (!live) return r;
-    if (!isfinite(norm)) {
-        if (reporter) report(status, QSGD_ST_NONFINITE);
-        return r;
-    }
-    if (norm == 0.f) return r;
-    const float sinv = __fdiv_rn(__uint2float_rn(s), norm);
-    if (isinf(sinv)) {
-        if (reporter) report(status, QSGD_ST_RANGE);
-        return r;
-    }
-    r.sent = norm;
-    r.sinv = sinv;
-    r.good = true;
-    return r;
-}
-
-// A plain fp32 sum of squares loses accuracy when squares leave the normal range.
-// Such buckets (sum below 2^-60, infinite, or NaN) are recomputed with every
-// value multiplied by 2^(127-E), E the exponent field of max|v| (clamped to
-// [1, 253]), so the largest scaled value lies in [1, 2); the root is scaled
-// back by the exact power of two 2^(E-127).
-__device__ __forceinline__ bool needs_rescale(float sumsq) {
-    return !(sumsq >= 0x1p-60f) || isinf(sumsq);
-}
-__device__ __forceinline__ float pow2_scale(float maxabs, float& unscale) {
-    uint32_t e = (__float_as_uint(maxabs) >> 23) & 0xFFu;
-    e = e < 1u ? 1u : (e > 253u ? 253u : e);
-    unscale = __uint_as_float(e << 23);        // 2^(e-127)
-    return __uint_as_float((254u - e) << 23);  // 2^(127-e)
 }
 
 __device__ __forceinline__ void abort_all(const EncodeArgs& a) {
@@ -220,34 +174,7 @@ __device__ __forceinline__ void code_tile(const EncodeArgs& a, uint64_t t, const
     }
 
     // --- bucket norm: per-lane FMA chain, butterfly (same value in all lanes) --
-    float ss = 0.f;
-#pragma unroll
-    for (int q = 0; q < NC; ++q) ss = __fmaf_rn(x[q], x[q], ss);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss = __fadd_rn(ss, __shfl_xor_sync(kFull, ss, o));
-    float norm = __fsqrt_rn(ss);
-    if (live && needs_rescale(ss) && !isnan(ss)) {  // uniform in the warp
-        float mx = 0.f;
-#pragma unroll
-        for (int q = 0; q < NC; ++q) mx = fmaxf(mx, fabsf(x[q]));
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
-        if (isinf(mx)) {
-            norm = mx;
-        } else if (mx > 0.f) {
-            float unscale;
-            const float scale = pow2_scale(mx, unscale);
-            float s2 = 0.f;
-#pragma unroll
-            for (int q = 0; q < NC; ++q) {
-                const float y = __fmul_rn(x[q], scale);
-                s2 = __fmaf_rn(y, y, s2);
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) s2 = __fadd_rn(s2, __shfl_xor_sync(kFull, s2, o));
-            norm = __fmul_rn(__fsqrt_rn(s2), unscale);
-        }
-    }
+    const float norm = warp_bucket_norm<NC>(x, live);
     const BucketScale sc = bucket_scale(norm, a.s, live, a.status, lane == 0);
     if (!sc.good) {
 #pragma unroll

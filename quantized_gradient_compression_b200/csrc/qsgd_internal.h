@@ -95,6 +95,12 @@ struct DecodeArgs {
 
 cudaError_t launch_decode(const DecodeArgs& a, bool accumulate, cudaStream_t stream);
 
+// Fixed-width b-bit variant (b in {2, 4, 8}, checked by the caller).
+cudaError_t launch_bbit_encode(const float* in, uint64_t n, uint32_t d, uint32_t b, uint64_t seed, float* norms,
+                               uint32_t* codes, uint32_t* status, cudaStream_t stream);
+cudaError_t launch_bbit_decode(const float* norms, const uint32_t* codes, uint64_t n, uint32_t d, uint32_t b,
+                               float* out, bool accumulate, uint32_t* status, cudaStream_t stream);
+
 // Omega code length on the host (for the size bound).
 uint32_t omega_len_host(uint64_t N);
 

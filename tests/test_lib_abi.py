@@ -31,7 +31,8 @@ def lib():
 def test_header_declares_the_boundary():
     names = declared_symbols()
     for want in ["qsgd_encode", "qsgd_decode", "qsgd_decode_accumulate", "qsgd_max_encoded_words",
-                 "qsgd_encode_workspace_bytes", "qsgd_num_buckets", "qsgd_error_string"]:
+                 "qsgd_encode_workspace_bytes", "qsgd_num_buckets", "qsgd_error_string",
+                 "qsgd_bbit_encode", "qsgd_bbit_decode", "qsgd_bbit_decode_accumulate", "qsgd_bbit_code_words"]:
         assert want in names
 
 
@@ -88,3 +89,16 @@ def test_library_is_sm100a_only():
     assert "arch=compute_100a,code=sm_100a" in flags
     assert "-fmad=false" in flags
     assert "use_fast_math" not in flags
+
+
+def test_bbit_size_query_and_argument_checks(oracle_lib):
+    from quantized_gradient_compression_b200 import binding as B
+
+    for n in (0, 1, 15, 16, 17, 25_557_032):
+        for b in (2, 4, 8):
+            assert B.qsgd_bbit_code_words(n, b) == oracle_lib.bbit_code_words(n, b)
+    # widths other than 2, 4, 8 and null pointers are refused before any CUDA call
+    assert B.qsgd_bbit_encode(256, 10, 4, 3, 0, 256, 256, 256, 0) == B.QSGD_ERR_ARG
+    assert B.qsgd_bbit_encode(0, 10, 4, 4, 0, 256, 256, 256, 0) == B.QSGD_ERR_ARG
+    assert B.qsgd_bbit_decode(256, 256, 10, 4, 16, 256, 256, 0) == B.QSGD_ERR_ARG
+    assert B.qsgd_bbit_decode_accumulate([], [], 0, 10, 4, 4, 256, 256, 0) == B.QSGD_ERR_ARG
