@@ -62,6 +62,7 @@ def _declare(lib):
         "qo_omega_put": (c_int, [u32p, c_u64, u64p, c_u64]),
         "qo_omega_get": (c_int, [u32p, u64p, c_u64, u64p]),
         "qo_bucket_norm": (ctypes.c_float, [f32p, c_u64]),
+        "qo_bucket_maxnorm": (ctypes.c_float, [f32p, c_u64]),
         "qo_quantize_bucket": (ctypes.c_float,
                                [f32p, c_u64, c_u64, c_u32, c_u64, f32p, i32p, u32p]),
         "qo_bucket_bit_bound": (c_u64, [c_u64, c_u32]),
@@ -156,6 +157,18 @@ class Oracle:
     def bucket_norm(self, v: np.ndarray) -> np.float32:
         v = np.ascontiguousarray(v, dtype=np.float32)
         return np.float32(self.lib.qo_bucket_norm(_ptr(v, ctypes.c_float), v.size))
+
+    def bucket_maxnorm(self, v: np.ndarray) -> np.float32:
+        v = np.ascontiguousarray(v, dtype=np.float32)
+        if v.size == 0:
+            return np.float32(0.0)
+        return np.float32(self.lib.qo_bucket_maxnorm(_ptr(v, ctypes.c_float), v.size))
+
+    def maxnorms(self, v: np.ndarray, d: int) -> np.ndarray:
+        """The max-norm of every bucket: norms_in for the QSGDinf variant."""
+        v = np.ascontiguousarray(v, dtype=np.float32)
+        nb = (v.size + d - 1) // d
+        return np.array([self.bucket_maxnorm(v[b * d:(b + 1) * d]) for b in range(nb)], dtype=np.float32)
 
     def capacity_words(self, n: int, d: int, s: int) -> int:
         return int(self.lib.qo_capacity_words(n, d, s))

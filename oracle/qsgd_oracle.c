@@ -160,6 +160,18 @@ float qo_bucket_norm(const float* v, uint64_t m) {
     return (float)sqrt(sum);
 }
 
+/* The max-norm ||v||_inf of a bucket: the scale of the QSGDinf heuristic (named
+   in the NUQSGD abstract; the name gives the norm).  NaN when any value is NaN, so
+   that such a bucket is non-finite like under the L2 norm. */
+float qo_bucket_maxnorm(const float* v, uint64_t m) {
+    float mx = 0.0f;
+    for (uint64_t i = 0; i < m; ++i) {
+        if (isnan(v[i])) return NAN;
+        if (fabsf(v[i]) > mx) mx = fabsf(v[i]);
+    }
+    return mx;
+}
+
 float qo_quantize_bucket(const float* v, uint64_t m, uint64_t base, uint32_t s,
                          uint64_t seed, const float* norm_in, int32_t* levels,
                          uint32_t* status) {

@@ -58,6 +58,10 @@ int qo_omega_get(const uint32_t* words, uint64_t* pos, uint64_t end_bit, uint64_
 /* fp32 L2 norm of one bucket: exact-ish sum of squares in double, rounded once. */
 float qo_bucket_norm(const float* v, uint64_t m);
 
+/* max_i |v_i| of m values (NaN if any value is NaN): the QSGDinf scale.  Passed to
+ * the encoders as norms_in, it gives the max-norm variant of either format. */
+float qo_bucket_maxnorm(const float* v, uint64_t m);
+
 /* Quantises one bucket v[0..m) that starts at global index base.  Writes the
  * signed levels (+k or -k; 0 off the support) to levels[0..m) and returns the
  * norm that is sent (0 for a degenerate bucket).  norm_in: if non-NULL, this

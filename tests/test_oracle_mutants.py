@@ -53,6 +53,9 @@ MUTANTS = {
     "bbit_decode_scale_inverted": ("float bscale = norm / (float)s;", "float bscale = (float)s / norm;"),
     "bbit_sign_on_zero_accepted": ("if (sign) bad = 1; /* a sign on a zero level: no encoder writes it */", ""),
     "bbit_accumulate_overwrites": ("out[i] += q[i];", "out[i] = q[i];"),
+    # max-norm (QSGDinf) scale
+    "maxnorm_drops_nan": ("if (isnan(v[i])) return NAN;", ""),
+    "maxnorm_signed": ("if (fabsf(v[i]) > mx) mx = fabsf(v[i]);", "if (v[i] > mx) mx = v[i];"),
     "bbit_code_shifted": ("uint64_t pos = (base + i) * b;\n            put_bits_msb_first",
                           "uint64_t pos = (base + i) * b + 1;\n            put_bits_msb_first"),
 }
@@ -158,6 +161,13 @@ def pin_battery(o) -> list:
             failed.append("bbit_accumulate")
     except (ValueError, AssertionError):
         failed.append("bbit")
+    # max-norm scale: numpy's max |v| per bucket, NaN propagated
+    vm = workloads.normal(1000, 4)
+    ref = np.array([np.max(np.abs(vm[b * 100:(b + 1) * 100])) for b in range(10)], np.float32)
+    vn = vm.copy()
+    vn[5] = np.nan
+    if not (np.array_equal(o.maxnorms(vm, 100), ref) and np.isnan(o.maxnorms(vn, 100)[0])):
+        failed.append("maxnorm")
     # small unbiasedness sweep: 4096 N(0,1) coordinates, s = 8, 400 seeds
     v = workloads.normal(4096, 1)
     sums = sc.Sums(v.size)
