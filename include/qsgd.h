@@ -79,6 +79,13 @@ enum {
     QSGD_ST_RANGE = 16            /* encode: norm > 0 but s/norm overflows fp32; sent as zero */
 };
 
+/* Bucket scale of the encoders' _ex forms.  QSGD_NORM_L2 is the definition
+ * paragraph's ||v||_2 (what qsgd_encode and qsgd_bbit_encode use).  QSGD_NORM_MAX is
+ * max_i |v_i|, the QSGDinf heuristic that the NUQSGD abstract names (no formula on
+ * the page: the name gives the norm); a NaN in a bucket makes it non-finite.  The
+ * scale is sent in the norm field, so the decoders are the same for both. */
+enum { QSGD_NORM_L2 = 0, QSGD_NORM_MAX = 1 };
+
 /* Number of buckets, ceil(n / d) (0 when d == 0). */
 QSGD_API uint64_t qsgd_num_buckets(uint64_t n, uint32_t d);
 
@@ -113,6 +120,14 @@ QSGD_API int qsgd_workspace_init(void* d_ws, size_t ws_bytes, cudaStream_t strea
 QSGD_API int qsgd_encode(const float* d_in, uint64_t n, uint32_t d, uint32_t s, uint64_t seed,
                 uint32_t* d_words, uint64_t words_capacity, uint64_t* d_offsets,
                 void* d_ws, size_t ws_bytes, uint32_t* d_status, cudaStream_t stream);
+
+/* qsgd_encode with the bucket scale chosen by norm_kind (QSGD_NORM_L2 or
+ * QSGD_NORM_MAX, else QSGD_ERR_ARG).  Under QSGD_NORM_MAX the sent norm is exactly
+ * max_i |v_i| and the largest value of a bucket gets level s. */
+QSGD_API int qsgd_encode_ex(const float* d_in, uint64_t n, uint32_t d, uint32_t s, uint64_t seed,
+                            uint32_t norm_kind, uint32_t* d_words, uint64_t words_capacity,
+                            uint64_t* d_offsets, void* d_ws, size_t ws_bytes, uint32_t* d_status,
+                            cudaStream_t stream);
 
 /* Decoder: writes Q_s(v) as dense fp32 d_out[0..n) (definition paragraph:
  * ||v||_2 * sgn(v_i) * k_i / s, evaluated as fl(fl(norm/s) * k), sign last; +0.0 off
@@ -193,6 +208,12 @@ QSGD_API uint64_t qsgd_bbit_code_words(uint64_t n, uint32_t b);
  * (d_in, n, d, b, seed); norms within 1e-6 relative of the exactly rounded norm. */
 QSGD_API int qsgd_bbit_encode(const float* d_in, uint64_t n, uint32_t d, uint32_t b, uint64_t seed,
                               float* d_norms, uint32_t* d_codes, uint32_t* d_status, cudaStream_t stream);
+
+/* qsgd_bbit_encode with the bucket scale chosen by norm_kind (QSGD_NORM_L2 or
+ * QSGD_NORM_MAX, else QSGD_ERR_ARG). */
+QSGD_API int qsgd_bbit_encode_ex(const float* d_in, uint64_t n, uint32_t d, uint32_t b, uint64_t seed,
+                                 uint32_t norm_kind, float* d_norms, uint32_t* d_codes, uint32_t* d_status,
+                                 cudaStream_t stream);
 
 /* b-bit decoder: d_out[0..n) = fl(fl(norm/s) * k), negated for sign 1, +0.0 for k = 0.
  * Sets QSGD_ST_BAD_STREAM for a negative or non-finite norm, a non-zero code under a

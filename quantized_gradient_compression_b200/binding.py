@@ -38,6 +38,9 @@ QSGD_ST_LOOKBACK_TIMEOUT = 4
 QSGD_ST_OVERFLOW = 8
 QSGD_ST_RANGE = 16
 
+QSGD_NORM_L2 = 0
+QSGD_NORM_MAX = 1
+
 _u64, _u32, _int, _sz, _vp = ctypes.c_uint64, ctypes.c_uint32, ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
 
 _SIGS = {
@@ -46,6 +49,7 @@ _SIGS = {
     "qsgd_encode_workspace_bytes": (_sz, [_u64, _u32, _u32]),
     "qsgd_workspace_init": (_int, [_vp, _sz, _vp]),
     "qsgd_encode": (_int, [_vp, _u64, _u32, _u32, _u64, _vp, _u64, _vp, _vp, _sz, _vp, _vp]),
+    "qsgd_encode_ex": (_int, [_vp, _u64, _u32, _u32, _u64, _u32, _vp, _u64, _vp, _vp, _sz, _vp, _vp]),
     "qsgd_decode": (_int, [_vp, _u64, _vp, _u64, _u32, _u32, _vp, _vp, _vp]),
     "qsgd_decode_accumulate": (_int, [ctypes.POINTER(_vp), ctypes.POINTER(_u64), ctypes.POINTER(_vp),
                                       _int, _u64, _u32, _u32, _vp, _vp, _vp]),
@@ -53,6 +57,7 @@ _SIGS = {
     "qsgd_static_workspace_limit": (_sz, []),
     "qsgd_bbit_code_words": (_u64, [_u64, _u32]),
     "qsgd_bbit_encode": (_int, [_vp, _u64, _u32, _u32, _u64, _vp, _vp, _vp, _vp]),
+    "qsgd_bbit_encode_ex": (_int, [_vp, _u64, _u32, _u32, _u64, _u32, _vp, _vp, _vp, _vp]),
     "qsgd_bbit_decode": (_int, [_vp, _vp, _u64, _u32, _u32, _vp, _vp, _vp]),
     "qsgd_bbit_decode_accumulate": (_int, [ctypes.POINTER(_vp), ctypes.POINTER(_vp), _int, _u64, _u32, _u32,
                                            _vp, _vp, _vp]),
@@ -103,6 +108,12 @@ def qsgd_encode(d_in: int, n: int, d: int, s: int, seed: int, d_words: int, word
                                 d_offsets, d_ws, ws_bytes, d_status, stream))
 
 
+def qsgd_encode_ex(d_in: int, n: int, d: int, s: int, seed: int, norm_kind: int, d_words: int,
+                   words_capacity: int, d_offsets: int, d_ws: int, ws_bytes: int, d_status: int, stream: int) -> int:
+    return int(_lib.qsgd_encode_ex(d_in, n, d, s, seed & 0xFFFFFFFFFFFFFFFF, norm_kind, d_words, words_capacity,
+                                   d_offsets, d_ws, ws_bytes, d_status, stream))
+
+
 def qsgd_decode(d_words: int, num_words: int, d_offsets: int, n: int, d: int, s: int, d_out: int,
                 d_status: int, stream: int) -> int:
     return int(_lib.qsgd_decode(d_words, num_words, d_offsets, n, d, s, d_out, d_status, stream))
@@ -134,6 +145,12 @@ def qsgd_bbit_code_words(n: int, b: int) -> int:
 def qsgd_bbit_encode(d_in: int, n: int, d: int, b: int, seed: int, d_norms: int, d_codes: int, d_status: int,
                      stream: int) -> int:
     return int(_lib.qsgd_bbit_encode(d_in, n, d, b, seed & 0xFFFFFFFFFFFFFFFF, d_norms, d_codes, d_status, stream))
+
+
+def qsgd_bbit_encode_ex(d_in: int, n: int, d: int, b: int, seed: int, norm_kind: int, d_norms: int, d_codes: int,
+                        d_status: int, stream: int) -> int:
+    return int(_lib.qsgd_bbit_encode_ex(d_in, n, d, b, seed & 0xFFFFFFFFFFFFFFFF, norm_kind, d_norms, d_codes,
+                                        d_status, stream))
 
 
 def qsgd_bbit_decode(d_norms: int, d_codes: int, n: int, d: int, b: int, d_out: int, d_status: int,
@@ -194,7 +211,8 @@ def workspace(n: int, d: int, s: int, device, stream_handle: int):
     return ws
 
 
-def encode(x, d: int, s: int, seed: int, words=None, offsets=None, status=None) -> Encoded:
+def encode(x, d: int, s: int, seed: int, words=None, offsets=None, status=None,
+           norm_kind: int = QSGD_NORM_L2) -> Encoded:
     torch = _torch()
     assert x.is_cuda and x.dtype == torch.float32 and x.is_contiguous()
     n = x.numel()
@@ -209,8 +227,8 @@ def encode(x, d: int, s: int, seed: int, words=None, offsets=None, status=None) 
     if status is None:
         status = torch.zeros(1, dtype=torch.int32, device=dev)
     ws = workspace(n, d, s, dev, stream)
-    _check(qsgd_encode(x.data_ptr(), n, d, s, seed, words.data_ptr(), words.numel(), offsets.data_ptr(),
-                       ws.data_ptr(), ws.numel(), status.data_ptr(), stream), "qsgd_encode")
+    _check(qsgd_encode_ex(x.data_ptr(), n, d, s, seed, norm_kind, words.data_ptr(), words.numel(),
+                          offsets.data_ptr(), ws.data_ptr(), ws.numel(), status.data_ptr(), stream), "qsgd_encode_ex")
     return Encoded(words, offsets, n, d, s, seed, status)
 
 
@@ -253,7 +271,8 @@ class BbitEncoded:
     status: "object"  # torch.int32 tensor [1]
 
 
-def bbit_encode(x, d: int, b: int, seed: int, norms=None, codes=None, status=None) -> BbitEncoded:
+def bbit_encode(x, d: int, b: int, seed: int, norms=None, codes=None, status=None,
+                norm_kind: int = QSGD_NORM_L2) -> BbitEncoded:
     torch = _torch()
     assert x.is_cuda and x.dtype == torch.float32 and x.is_contiguous()
     n = x.numel()
@@ -265,8 +284,8 @@ def bbit_encode(x, d: int, b: int, seed: int, norms=None, codes=None, status=Non
         codes = torch.empty(max(qsgd_bbit_code_words(n, b), 1), dtype=torch.int32, device=dev)
     if status is None:
         status = torch.zeros(1, dtype=torch.int32, device=dev)
-    _check(qsgd_bbit_encode(x.data_ptr(), n, d, b, seed, norms.data_ptr(), codes.data_ptr(), status.data_ptr(),
-                            stream), "qsgd_bbit_encode")
+    _check(qsgd_bbit_encode_ex(x.data_ptr(), n, d, b, seed, norm_kind, norms.data_ptr(), codes.data_ptr(),
+                               status.data_ptr(), stream), "qsgd_bbit_encode_ex")
     return BbitEncoded(norms, codes, n, d, b, seed, status)
 
 

@@ -87,9 +87,10 @@ int qsgd_workspace_init(void* d_ws, size_t ws_bytes, cudaStream_t stream) {
     return cudaMemsetAsync(d_ws, 0, ws_bytes, stream) == cudaSuccess ? QSGD_OK : QSGD_ERR_CUDA;
 }
 
-int qsgd_encode(const float* d_in, uint64_t n, uint32_t d, uint32_t s, uint64_t seed,
-                uint32_t* d_words, uint64_t words_capacity, uint64_t* d_offsets, void* d_ws,
-                size_t ws_bytes, uint32_t* d_status, cudaStream_t stream) {
+int qsgd_encode_ex(const float* d_in, uint64_t n, uint32_t d, uint32_t s, uint64_t seed, uint32_t norm_kind,
+                   uint32_t* d_words, uint64_t words_capacity, uint64_t* d_offsets, void* d_ws, size_t ws_bytes,
+                   uint32_t* d_status, cudaStream_t stream) {
+    if (norm_kind != QSGD_NORM_L2 && norm_kind != QSGD_NORM_MAX) return QSGD_ERR_ARG;
     if (!valid_params(n, d, s) || !d_offsets || !d_status) return QSGD_ERR_ARG;
     if (max_bits(n, d, s) > kMaxStreamBits) return QSGD_ERR_ARG;
     if ((reinterpret_cast<uintptr_t>(d_offsets) & 7u) != 0 || (reinterpret_cast<uintptr_t>(d_words) & 3u) != 0)
@@ -116,6 +117,7 @@ int qsgd_encode(const float* d_in, uint64_t n, uint32_t d, uint32_t s, uint64_t 
     a.cap_words = words_capacity;
     a.offsets = d_offsets;
     a.status = d_status;
+    a.norm_kind = norm_kind;
     a.ctrl = reinterpret_cast<ScanControl*>(ws);
     a.tdesc = reinterpret_cast<uint64_t*>(ws + L.desc_off);
     a.ts = reinterpret_cast<TileState*>(ws + L.tiles_off);
@@ -145,6 +147,13 @@ int qsgd_encode(const float* d_in, uint64_t n, uint32_t d, uint32_t s, uint64_t 
     if (a.ntiles > L.max_tiles) return QSGD_ERR_WORKSPACE;
     const cudaError_t e = launch_encode(a, fast, stream);
     return e == cudaSuccess ? QSGD_OK : QSGD_ERR_CUDA;
+}
+
+int qsgd_encode(const float* d_in, uint64_t n, uint32_t d, uint32_t s, uint64_t seed, uint32_t* d_words,
+                uint64_t words_capacity, uint64_t* d_offsets, void* d_ws, size_t ws_bytes, uint32_t* d_status,
+                cudaStream_t stream) {
+    return qsgd_encode_ex(d_in, n, d, s, seed, QSGD_NORM_L2, d_words, words_capacity, d_offsets, d_ws, ws_bytes,
+                          d_status, stream);
 }
 
 static int decode_impl(const uint32_t* const* words, const uint64_t* num_words,
@@ -197,15 +206,22 @@ static bool valid_bbit(uint64_t n, uint32_t d, uint32_t b) {
     return (b == 2 || b == 4 || b == 8) && d >= 1 && d <= kMaxD && n <= kMaxN;
 }
 
-int qsgd_bbit_encode(const float* d_in, uint64_t n, uint32_t d, uint32_t b, uint64_t seed, float* d_norms,
-                     uint32_t* d_codes, uint32_t* d_status, cudaStream_t stream) {
+int qsgd_bbit_encode_ex(const float* d_in, uint64_t n, uint32_t d, uint32_t b, uint64_t seed, uint32_t norm_kind,
+                        float* d_norms, uint32_t* d_codes, uint32_t* d_status, cudaStream_t stream) {
     if (!valid_bbit(n, d, b) || !d_status) return QSGD_ERR_ARG;
+    if (norm_kind != QSGD_NORM_L2 && norm_kind != QSGD_NORM_MAX) return QSGD_ERR_ARG;
     if (n == 0) return QSGD_OK;
     if (!d_in || !d_norms || !d_codes || (reinterpret_cast<uintptr_t>(d_in) & 3u) != 0 ||
         (reinterpret_cast<uintptr_t>(d_norms) & 3u) != 0 || (reinterpret_cast<uintptr_t>(d_codes) & 3u) != 0)
         return QSGD_ERR_ARG;
-    return launch_bbit_encode(d_in, n, d, b, seed, d_norms, d_codes, d_status, stream) == cudaSuccess ? QSGD_OK
-                                                                                                     : QSGD_ERR_CUDA;
+    return launch_bbit_encode(d_in, n, d, b, seed, norm_kind, d_norms, d_codes, d_status, stream) == cudaSuccess
+               ? QSGD_OK
+               : QSGD_ERR_CUDA;
+}
+
+int qsgd_bbit_encode(const float* d_in, uint64_t n, uint32_t d, uint32_t b, uint64_t seed, float* d_norms,
+                     uint32_t* d_codes, uint32_t* d_status, cudaStream_t stream) {
+    return qsgd_bbit_encode_ex(d_in, n, d, b, seed, QSGD_NORM_L2, d_norms, d_codes, d_status, stream);
 }
 
 int qsgd_bbit_decode(const float* d_norms, const uint32_t* d_codes, uint64_t n, uint32_t d, uint32_t b,

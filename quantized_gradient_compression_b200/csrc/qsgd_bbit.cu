@@ -36,8 +36,8 @@ __device__ __forceinline__ uint32_t bbit_code(float v, float sinv, uint32_t r, u
 // ---------------------------------------------------------------------------
 template <int V, int B>
 __global__ void __launch_bounds__(kBbitBlock) bbit_encode_fast(const float* __restrict__ in, uint64_t n,
-                                                               uint32_t d, uint64_t seed, float* norms,
-                                                               uint32_t* codes, uint32_t* status) {
+                                                               uint32_t d, uint64_t seed, uint32_t norm_kind,
+                                                               float* norms, uint32_t* codes, uint32_t* status) {
     constexpr int NC = 4 * V;
     constexpr uint32_t S = (1u << (B - 1)) - 1u;
     constexpr int kLaneBits = NC * B;  // 8 .. 256
@@ -69,7 +69,7 @@ __global__ void __launch_bounds__(kBbitBlock) bbit_encode_fast(const float* __re
             x[4 * j + 2] = q.z;
             x[4 * j + 3] = q.w;
         }
-        const float norm = warp_bucket_norm<NC>(x, true);
+        const float norm = norm_kind == QSGD_NORM_MAX ? warp_bucket_maxnorm<NC>(x) : warp_bucket_norm<NC>(x, true);
         const BucketScale sc = bucket_scale(norm, S, true, status, lane == 0);
         if (lane == 0) norms[bk] = sc.sent;
         uint32_t part[kLaneWords];
@@ -117,7 +117,8 @@ __global__ void __launch_bounds__(kBbitBlock) bbit_encode_fast(const float* __re
 // scales (its first coordinate is a multiple of 4: one Philox block per 4).
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kBbitBlock) bbit_norms(const float* __restrict__ in, uint64_t n, uint32_t d,
-                                                         uint32_t s, float* norms, uint32_t* status) {
+                                                         uint32_t s, uint32_t norm_kind, float* norms,
+                                                         uint32_t* status) {
     const int lane = threadIdx.x & 31;
     const uint64_t nb = (n + d - 1) / d;
     const uint64_t gwarps = static_cast<uint64_t>(gridDim.x) * (kBbitBlock / 32);
@@ -125,6 +126,11 @@ __global__ void __launch_bounds__(kBbitBlock) bbit_norms(const float* __restrict
          bk += gwarps) {
         const float* p = in + bk * d;
         const uint64_t m = min(static_cast<uint64_t>(d), n - bk * d);
+        if (norm_kind == QSGD_NORM_MAX) {  // uniform in the grid
+            const BucketScale sc = bucket_scale(warp_maxnorm(p, m, lane), s, true, status, lane == 0);
+            if (lane == 0) norms[bk] = sc.sent;
+            continue;
+        }
         float ss = 0.f;
         for (uint64_t i = lane; i < m; i += 32) ss = __fmaf_rn(p[i], p[i], ss);
 #pragma unroll
@@ -285,23 +291,23 @@ int grid_for(uint64_t items, int per_sm_blocks = 8) {
 }
 
 template <int B>
-cudaError_t launch_bbit_encode_b(const float* in, uint64_t n, uint32_t d, uint64_t seed, float* norms,
+cudaError_t launch_bbit_encode_b(const float* in, uint64_t n, uint32_t d, uint64_t seed, uint32_t nk, float* norms,
                                  uint32_t* codes, uint32_t* status, cudaStream_t stream) {
     const uint64_t nb = (n + d - 1) / d;
     const bool fast = d % 128 == 0 && d <= 1024 && (reinterpret_cast<uintptr_t>(in) & 15u) == 0;
     if (fast) {
         const int grid = grid_for(nb * 32);
         switch (d / 128) {
-            case 1: bbit_encode_fast<1, B><<<grid, kBbitBlock, 0, stream>>>(in, n, d, seed, norms, codes, status); break;
-            case 2: bbit_encode_fast<2, B><<<grid, kBbitBlock, 0, stream>>>(in, n, d, seed, norms, codes, status); break;
-            case 4: bbit_encode_fast<4, B><<<grid, kBbitBlock, 0, stream>>>(in, n, d, seed, norms, codes, status); break;
-            case 8: bbit_encode_fast<8, B><<<grid, kBbitBlock, 0, stream>>>(in, n, d, seed, norms, codes, status); break;
+            case 1: bbit_encode_fast<1, B><<<grid, kBbitBlock, 0, stream>>>(in, n, d, seed, nk, norms, codes, status); break;
+            case 2: bbit_encode_fast<2, B><<<grid, kBbitBlock, 0, stream>>>(in, n, d, seed, nk, norms, codes, status); break;
+            case 4: bbit_encode_fast<4, B><<<grid, kBbitBlock, 0, stream>>>(in, n, d, seed, nk, norms, codes, status); break;
+            case 8: bbit_encode_fast<8, B><<<grid, kBbitBlock, 0, stream>>>(in, n, d, seed, nk, norms, codes, status); break;
             default: goto general;  // d = 384, 640, 768, 896: the general path
         }
         return cudaGetLastError();
     }
 general:
-    bbit_norms<<<grid_for(nb * 32), kBbitBlock, 0, stream>>>(in, n, d, (1u << (B - 1)) - 1u, norms, status);
+    bbit_norms<<<grid_for(nb * 32), kBbitBlock, 0, stream>>>(in, n, d, (1u << (B - 1)) - 1u, nk, norms, status);
     bbit_pack<B><<<grid_for((n * B + 31) / 32), kBbitBlock, 0, stream>>>(in, n, d, seed, norms, codes);
     return cudaGetLastError();
 }
@@ -318,12 +324,13 @@ cudaError_t launch_bbit_decode_b(const float* norms, const uint32_t* codes, uint
 
 }  // namespace
 
-cudaError_t launch_bbit_encode(const float* in, uint64_t n, uint32_t d, uint32_t b, uint64_t seed, float* norms,
-                               uint32_t* codes, uint32_t* status, cudaStream_t stream) {
+cudaError_t launch_bbit_encode(const float* in, uint64_t n, uint32_t d, uint32_t b, uint64_t seed,
+                               uint32_t norm_kind, float* norms, uint32_t* codes, uint32_t* status,
+                               cudaStream_t stream) {
     switch (b) {
-        case 2: return launch_bbit_encode_b<2>(in, n, d, seed, norms, codes, status, stream);
-        case 4: return launch_bbit_encode_b<4>(in, n, d, seed, norms, codes, status, stream);
-        default: return launch_bbit_encode_b<8>(in, n, d, seed, norms, codes, status, stream);
+        case 2: return launch_bbit_encode_b<2>(in, n, d, seed, norm_kind, norms, codes, status, stream);
+        case 4: return launch_bbit_encode_b<4>(in, n, d, seed, norm_kind, norms, codes, status, stream);
+        default: return launch_bbit_encode_b<8>(in, n, d, seed, norm_kind, norms, codes, status, stream);
     }
 }
 

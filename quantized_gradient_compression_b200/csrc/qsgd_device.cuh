@@ -149,6 +149,39 @@ __device__ __forceinline__ float warp_bucket_norm(const float (&x)[NC], bool liv
     return norm;
 }
 
+// Max-norm max_i |v_i| of a bucket held by one warp (NC values per lane): the
+// scale of the QSGDinf variant.  NaN when any value is NaN, so that the bucket is
+// non-finite as under the L2 norm.  Exact: no rounding.
+template <int NC>
+__device__ __forceinline__ float warp_bucket_maxnorm(const float (&x)[NC]) {
+    constexpr uint32_t kAll = 0xFFFFFFFFu;
+    float mx = 0.f;
+    bool nan = false;
+#pragma unroll
+    for (int q = 0; q < NC; ++q) {
+        nan |= isnan(x[q]);
+        mx = fmaxf(mx, fabsf(x[q]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kAll, mx, o));
+    return __any_sync(kAll, nan) ? __uint_as_float(0x7FC00000u) : mx;
+}
+
+// The same over m values at p, read by one warp (lanes take every 32nd value).
+__device__ __forceinline__ float warp_maxnorm(const float* p, uint64_t m, int lane) {
+    constexpr uint32_t kAll = 0xFFFFFFFFu;
+    float mx = 0.f;
+    bool nan = false;
+    for (uint64_t i = lane; i < m; i += 32) {
+        const float v = __ldg(p + i);
+        nan |= isnan(v);
+        mx = fmaxf(mx, fabsf(v));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kAll, mx, o));
+    return __any_sync(kAll, nan) ? __uint_as_float(0x7FC00000u) : mx;
+}
+
 // ---------------------------------------------------------------------------
 // Elias omega code of N >= 1 (Elias 1975): start from "0"; while N > 1, put the
 // binary form of N in front and continue with bitlength(N) - 1.  Returned as a

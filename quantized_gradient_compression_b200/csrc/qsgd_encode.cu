@@ -174,7 +174,7 @@ __device__ __forceinline__ void code_tile(const EncodeArgs& a, uint64_t t, const
     }
 
     // --- bucket norm: per-lane FMA chain, butterfly (same value in all lanes) --
-    const float norm = warp_bucket_norm<NC>(x, live);
+    const float norm = a.norm_kind == QSGD_NORM_MAX ? warp_bucket_maxnorm<NC>(x) : warp_bucket_norm<NC>(x, live);
     const BucketScale sc = bucket_scale(norm, a.s, live, a.status, lane == 0);
     if (!sc.good) {
 #pragma unroll
@@ -569,6 +569,27 @@ __device__ __forceinline__ float block_norm(const float* p, uint64_t m, float* r
     return norm;
 }
 
+// Max-norm of m values at p by the whole CTA (NaN if any value is NaN).
+__device__ __forceinline__ float block_maxnorm(const float* p, uint64_t m, float* red) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    float mx = 0.f;
+    bool nan = false;
+    for (uint64_t i = tid; i < m; i += kBlock) {
+        const float v = __ldg(p + i);
+        nan |= isnan(v);
+        mx = fmaxf(mx, fabsf(v));
+    }
+    if (__syncthreads_or(nan)) return __uint_as_float(0x7FC00000u);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
+    if (lane == 0) red[warp] = mx;
+    __syncthreads();
+    float tot = 0.f;
+    for (int w = 0; w < kWarps; ++w) tot = fmaxf(tot, red[w]);
+    __syncthreads();  // red is reused by the next call
+    return tot;
+}
+
 // Block-wide scans for kBlock threads.
 struct BlockScratch {
     int64_t i64[kWarps];
@@ -689,14 +710,16 @@ __global__ void __launch_bounds__(kBlock) encode_general(const __grid_constant__
         // --- bucket norms into shared memory -------------------------------
         if (b1 - b0 == 1) {
             const uint64_t m = c1 - c0;
-            const float norm = block_norm(a.in + c0, m, s_red);
+            const float norm = a.norm_kind == QSGD_NORM_MAX ? block_maxnorm(a.in + c0, m, s_red)
+                                                            : block_norm(a.in + c0, m, s_red);
             const BucketScale sc = bucket_scale(norm, a.s, true, a.status, tid == 0);
             if (tid == 0) s_norms[0] = make_float2(sc.sent, sc.good ? sc.sinv : 0.f);
         } else {
             for (uint64_t bl = warp; bl < b1 - b0; bl += kWarps) {
                 const uint64_t base = (b0 + bl) * a.d;
                 const uint64_t m = min(static_cast<uint64_t>(a.d), a.n - base);
-                const float norm = warp_norm(a.in + base, m, lane);
+                const float norm = a.norm_kind == QSGD_NORM_MAX ? warp_maxnorm(a.in + base, m, lane)
+                                                                : warp_norm(a.in + base, m, lane);
                 const BucketScale sc = bucket_scale(norm, a.s, true, a.status, lane == 0);
                 if (lane == 0) s_norms[bl] = make_float2(sc.sent, sc.good ? sc.sinv : 0.f);
             }

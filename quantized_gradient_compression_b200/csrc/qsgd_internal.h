@@ -41,6 +41,7 @@ struct EncodeArgs {
     uint64_t ntiles;
     uint32_t buckets_per_tile;
     uint32_t smem_words;  // words of the per-tile (or per-chunk) bit buffer
+    uint32_t norm_kind;   // QSGD_NORM_L2 or QSGD_NORM_MAX
 };
 
 // Chooses the kernel, sets the launch shape and enqueues it.  Returns a CUDA
@@ -96,8 +97,9 @@ struct DecodeArgs {
 cudaError_t launch_decode(const DecodeArgs& a, bool accumulate, cudaStream_t stream);
 
 // Fixed-width b-bit variant (b in {2, 4, 8}, checked by the caller).
-cudaError_t launch_bbit_encode(const float* in, uint64_t n, uint32_t d, uint32_t b, uint64_t seed, float* norms,
-                               uint32_t* codes, uint32_t* status, cudaStream_t stream);
+cudaError_t launch_bbit_encode(const float* in, uint64_t n, uint32_t d, uint32_t b, uint64_t seed,
+                               uint32_t norm_kind, float* norms, uint32_t* codes, uint32_t* status,
+                               cudaStream_t stream);
 cudaError_t launch_bbit_decode(const float* norms, const uint32_t* codes, uint64_t n, uint32_t d, uint32_t b,
                                float* out, bool accumulate, uint32_t* status, cudaStream_t stream);
 

@@ -102,3 +102,12 @@ def test_bbit_size_query_and_argument_checks(oracle_lib):
     assert B.qsgd_bbit_encode(0, 10, 4, 4, 0, 256, 256, 256, 0) == B.QSGD_ERR_ARG
     assert B.qsgd_bbit_decode(256, 256, 10, 4, 16, 256, 256, 0) == B.QSGD_ERR_ARG
     assert B.qsgd_bbit_decode_accumulate([], [], 0, 10, 4, 4, 256, 256, 0) == B.QSGD_ERR_ARG
+
+
+def test_norm_kind_checked():
+    from quantized_gradient_compression_b200 import binding as B
+
+    assert B.QSGD_NORM_L2 == 0 and B.QSGD_NORM_MAX == 1
+    # an unknown norm kind is refused before any CUDA call
+    assert B.qsgd_encode_ex(256, 10, 4, 4, 0, 2, 256, 100, 256, 256, 4096, 256, 0) == B.QSGD_ERR_ARG
+    assert B.qsgd_bbit_encode_ex(256, 10, 4, 4, 0, 7, 256, 256, 256, 0) == B.QSGD_ERR_ARG

@@ -31,9 +31,11 @@ def test_maxnorm_special_values(oracle_lib):
 
 
 def test_maxnorm_scale_reaches_level_s_and_flags(oracle_lib):
-    # the largest |v_i| of a bucket has t = s exactly: level s, whatever the random word
+    # the largest |v_i| of a bucket has t = fl(max * fl(s / max)); for this vector that
+    # product rounds to s itself, so its level is s whatever the random word
     v = W.normal(512, 3)
     mx = oracle_lib.maxnorms(v, 512)
+    assert np.float32(mx[0]) * np.float32(np.float32(16) / mx[0]) == np.float32(16)
     for seed in range(5):
         levels, norms, st = oracle_lib.quantize(v, 512, 16, seed, norms_in=mx)
         assert st == 0 and np.abs(levels[np.argmax(np.abs(v))]) == 16
