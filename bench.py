@@ -397,6 +397,21 @@ def run_ours(args, w):
     if int(status.item()) != 0:
         raise RuntimeError("device status %d in the end-to-end run" % int(status.item()))
 
+    def time_alone(fn):
+        """Median device time (ms) of one call, L2 flushed before each."""
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(max(3, min(K, 50))):
+            flush.zero_()
+            e_a, e_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e_a.record(stream)
+            fn()
+            e_b.record(stream)
+            torch.cuda.synchronize()
+            ts.append(e_a.elapsed_time(e_b))
+        return statistics.median(ts)
+
     # fixed-width b-bit variant on the same vector: each call timed alone, L2 flushed
     bbit = {}
     for bw in (2, 4, 8):
@@ -419,20 +434,8 @@ def run_ours(args, w):
                                                 acc_b.data_ptr(), status.data_ptr(), sh),
                   "qsgd_bbit_decode_accumulate")
 
-        times = {}
-        for name, fn in (("encode", b_enc), ("decode", b_dec), ("decode_accumulate", b_acc)):
-            for _ in range(3):
-                fn()
-            ts = []
-            for _ in range(max(3, min(K, 50))):
-                flush.zero_()
-                e_a, e_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e_a.record(stream)
-                fn()
-                e_b.record(stream)
-                torch.cuda.synchronize()
-                ts.append(e_a.elapsed_time(e_b))
-            times[name] = statistics.median(ts)
+        times = {name: time_alone(fn) for name, fn in
+                 (("encode", b_enc), ("decode", b_dec), ("decode_accumulate", b_acc))}
         if int(status.item()) != 0:
             raise RuntimeError("device status %d in the b-bit runs" % int(status.item()))
         cbytes = 4.0 * nb + 4.0 * cw
@@ -443,6 +446,27 @@ def run_ours(args, w):
             "algorithmic_gbs": {k: alg[k] / times[k] / 1e6 for k in times},
             "roofline_frac": {k: alg[k] / times[k] / 1e6 / measured_peaks()[0] for k in times},
         }
+
+    # QSGDinf (max-norm scale) on the same vector, Elias coded at the same (d, s): the
+    # encoder and decoder timed alone, L2 flushed
+    def i_enc():
+        check(B.qsgd_encode_ex(x.data_ptr(), n, d, s, seed, B.QSGD_NORM_MAX, words.data_ptr(), cap,
+                               offsets.data_ptr(), ws.data_ptr(), ws_bytes, status.data_ptr(), sh), "qsgd_encode_ex")
+
+    def i_dec():
+        check(B.qsgd_decode(words.data_ptr(), cap, offsets.data_ptr(), n, d, s, out.data_ptr(),
+                            status.data_ptr(), sh), "qsgd_decode")
+
+    i_times = {"encode": time_alone(i_enc), "decode": time_alone(i_dec)}
+    if int(status.item()) != 0:
+        raise RuntimeError("device status %d in the max-norm runs" % int(status.item()))
+    i_bits = int(offsets[-1].item())
+    i_comp = 4 * ((i_bits + 31) // 32) + 8 * (nb + 1)
+    i_alg = {"encode": 4.0 * n + i_comp, "decode": i_comp + 4.0 * n}
+    qsgdinf = {"s": s, "bits_per_coord": i_bits / n, "compressed_bytes": i_comp,
+               "us": {k: 1e3 * v for k, v in i_times.items()},
+               "algorithmic_gbs": {k: i_alg[k] / i_times[k] / 1e6 for k in i_times},
+               "roofline_frac": {k: i_alg[k] / i_times[k] / 1e6 / measured_peaks()[0] for k in i_times}}
 
     peak, peak_kind = measured_peaks()
     in_bytes = 4.0 * n
@@ -496,6 +520,7 @@ def run_ours(args, w):
                        "input and D2H of the result, pipelined over copy-in / compute / copy-out streams"},
         "gpu_launches": 3 * K,
         "bbit": bbit,
+        "qsgdinf": qsgdinf,
         "clocks": clocks.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
