@@ -79,6 +79,9 @@ def _declare(lib):
         "qo_bbit_levels": (c_u32, [c_u32]),
         "qo_bbit_code_words": (c_u64, [c_u64, c_u32]),
         "qo_bbit_encode": (c_int, [f32p, c_u64, c_u64, c_u32, c_u64, f32p, f32p, u32p, u32p]),
+        "qo_encode_ef": (c_int, [f32p, f32p, c_u64, c_u64, c_u32, c_u64, c_int, f32p, u32p, c_u64, u64p,
+                                 f32p, u32p]),
+        "qo_bbit_encode_ef": (c_int, [f32p, f32p, c_u64, c_u64, c_u32, c_u64, c_int, f32p, f32p, u32p, u32p]),
         "qo_bbit_decode": (c_int, [f32p, u32p, c_u64, c_u64, c_u32, f32p, u32p]),
         "qo_bbit_decode_accumulate": (c_int, [ctypes.POINTER(f32p), ctypes.POINTER(u32p), c_int,
                                               c_u64, c_u64, c_u32, f32p, u32p]),
@@ -323,6 +326,56 @@ class Oracle:
         if rc != 0:
             raise ValueError("oracle b-bit encode rejected b=%d d=%d" % (b, d))
         return codes[:self.bbit_code_words(n, b)].copy(), norms[:nb].copy(), st.value
+
+    # --- error feedback ("Sparsified SGD with Memory") ----------------------
+    def encode_ef(self, g: np.ndarray, e: np.ndarray, d: int, s: int, seed: int, max_norm: bool = False,
+                  norms_in=None):
+        """p = e + g is encoded; returns (words, offsets, norms, status, e_new) with
+        e_new = p - Q(p) (p where no record was sent).  e is not modified."""
+        g = np.ascontiguousarray(g, dtype=np.float32)
+        e_new = np.array(e, dtype=np.float32, copy=True)
+        n = g.size
+        assert e_new.size == n
+        nb = (n + d - 1) // d
+        cap = self.capacity_words(n, d, s)
+        words = np.zeros(max(cap, 1), dtype=np.uint32)
+        offsets = np.zeros(nb + 1, dtype=np.uint64)
+        norms = np.zeros(max(nb, 1), dtype=np.float32)
+        st = ctypes.c_uint32(0)
+        nin = None if norms_in is None else np.ascontiguousarray(norms_in, dtype=np.float32)
+        gg = g if n else np.zeros(1, np.float32)
+        ee = e_new if n else np.zeros(1, np.float32)
+        rc = self.lib.qo_encode_ef(_ptr(gg, ctypes.c_float), _ptr(ee, ctypes.c_float), n, d, s, seed,
+                                   int(bool(max_norm)), _ptr(nin, ctypes.c_float) if nin is not None else None,
+                                   _ptr(words, ctypes.c_uint32), cap, _ptr(offsets, ctypes.c_uint64),
+                                   _ptr(norms, ctypes.c_float), ctypes.byref(st))
+        if rc != 0:
+            raise RuntimeError("oracle error-feedback encode failed (status %d)" % st.value)
+        nwords = (int(offsets[nb]) + 31) // 32
+        return words[:nwords].copy(), offsets, norms[:nb].copy(), st.value, e_new[:n]
+
+    def bbit_encode_ef(self, g: np.ndarray, e: np.ndarray, d: int, b: int, seed: int, max_norm: bool = False,
+                       norms_in=None):
+        """b-bit codes of p = e + g; returns (codes, norms, status, e_new)."""
+        g = np.ascontiguousarray(g, dtype=np.float32)
+        e_new = np.array(e, dtype=np.float32, copy=True)
+        n = g.size
+        assert e_new.size == n
+        nb = (n + d - 1) // d
+        codes = np.zeros(max(self.bbit_code_words(n, b), 1), dtype=np.uint32)
+        norms = np.zeros(max(nb, 1), dtype=np.float32)
+        st = ctypes.c_uint32(0)
+        nin = None if norms_in is None else np.ascontiguousarray(norms_in, dtype=np.float32)
+        gg = g if n else np.zeros(1, np.float32)
+        ee = e_new if n else np.zeros(1, np.float32)
+        rc = self.lib.qo_bbit_encode_ef(_ptr(gg, ctypes.c_float), _ptr(ee, ctypes.c_float), n, d, b, seed,
+                                        int(bool(max_norm)),
+                                        _ptr(nin, ctypes.c_float) if nin is not None else None,
+                                        _ptr(norms, ctypes.c_float), _ptr(codes, ctypes.c_uint32),
+                                        ctypes.byref(st))
+        if rc != 0:
+            raise ValueError("oracle b-bit error-feedback encode rejected b=%d d=%d" % (b, d))
+        return codes[:self.bbit_code_words(n, b)].copy(), norms[:nb].copy(), st.value, e_new[:n]
 
     def bbit_decode(self, norms: np.ndarray, codes: np.ndarray, n: int, d: int, b: int):
         norms = np.ascontiguousarray(norms, dtype=np.float32)

@@ -478,3 +478,76 @@ int qo_bbit_decode_accumulate(const float* const* norms, const uint32_t* const* 
     free(q);
     return 0;
 }
+
+/* ---- Error feedback ------------------------------------------------------------
+ * "Sparsified SGD with Memory" (abstract): the compressor keeps what it did not send
+ * in a memory and adds it to the next gradient.  Step by step: p = e + g, the stream
+ * carries Q(p), and the memory becomes p minus Q(p) as a receiver decodes it.  A
+ * coordinate with no record decodes to 0 and keeps p in the memory unchanged. */
+
+/* p[i] = e[i] + g[i] (one fp32 add); the caller frees p. */
+static float* ef_sum(const float* g, const float* e, uint64_t n) {
+    float* p = (float*)malloc((size_t)(n ? n : 1) * sizeof(float));
+    if (!p) return NULL;
+    for (uint64_t i = 0; i < n; ++i) p[i] = e[i] + g[i];
+    return p;
+}
+
+/* max_i |p_i| of every bucket (the QSGDinf scale of p); the caller frees it. */
+static float* ef_max_norms(const float* p, uint64_t n, uint64_t d) {
+    const uint64_t nb = (n + d - 1) / d;
+    float* mx = (float*)malloc((size_t)(nb ? nb : 1) * sizeof(float));
+    if (!mx) return NULL;
+    for (uint64_t b = 0; b < nb; ++b) {
+        const uint64_t m = (b + 1) * d <= n ? d : n - b * d;
+        mx[b] = qo_bucket_maxnorm(p + b * d, m);
+    }
+    return mx;
+}
+
+/* e[i] <- p[i] - q[i] where a record was sent (q[i] != 0), else p[i]. */
+static void ef_update(float* e, const float* p, const float* q, uint64_t n) {
+    for (uint64_t i = 0; i < n; ++i) e[i] = q[i] != 0.0f ? p[i] - q[i] : p[i];
+}
+
+int qo_encode_ef(const float* g, float* e, uint64_t n, uint64_t d, uint32_t s, uint64_t seed,
+                 int max_norm, const float* norms_in, uint32_t* words, uint64_t cap_words,
+                 uint64_t* offsets, float* norms_out, uint32_t* status) {
+    if (d == 0) return -1;
+    int rc = -1;
+    float* p = ef_sum(g, e, n);
+    float* q = (float*)malloc((size_t)(n ? n : 1) * sizeof(float));
+    float* mx = (p && max_norm && !norms_in) ? ef_max_norms(p, n, d) : NULL;
+    const float* nin = norms_in ? norms_in : mx;
+    if (!p || !q || (max_norm && !nin)) goto done;
+    if (qo_encode(p, n, d, s, seed, nin, words, cap_words, offsets, norms_out, status) != 0) goto done;
+    if (qo_decode(words, offsets, n, d, s, q, status) != 0) goto done;
+    ef_update(e, p, q, n);
+    rc = 0;
+done:
+    free(mx);
+    free(q);
+    free(p);
+    return rc;
+}
+
+int qo_bbit_encode_ef(const float* g, float* e, uint64_t n, uint64_t d, uint32_t b, uint64_t seed,
+                      int max_norm, const float* norms_in, float* norms_out, uint32_t* codes,
+                      uint32_t* status) {
+    if (d == 0) return -1;
+    int rc = -1;
+    float* p = ef_sum(g, e, n);
+    float* q = (float*)malloc((size_t)(n ? n : 1) * sizeof(float));
+    float* mx = (p && max_norm && !norms_in) ? ef_max_norms(p, n, d) : NULL;
+    const float* nin = norms_in ? norms_in : mx;
+    if (!p || !q || (max_norm && !nin)) goto done;
+    if (qo_bbit_encode(p, n, d, b, seed, nin, norms_out, codes, status) != 0) goto done;
+    if (qo_bbit_decode(norms_out, codes, n, d, b, q, status) != 0) goto done;
+    ef_update(e, p, q, n);
+    rc = 0;
+done:
+    free(mx);
+    free(q);
+    free(p);
+    return rc;
+}

@@ -17,7 +17,9 @@
  * Pins (tests/test_oracle_*.py): Philox known-answer vectors; omega code brute
  * force over 1..2^20 and textbook codewords; hand-derived golden bitstreams;
  * unbiasedness, the closed-form variance, the sparsity bound and the 2.818n+32
- * bit bound from the page's claims; the size bound by brute force.
+ * bit bound from the page's claims; the size bound by brute force.  Error feedback
+ * ("Sparsified SGD with Memory", abstract): exact steps, closed-form outcomes and the
+ * telescoping sum of sent values plus memory (tests/test_oracle_ef.py).
  */
 #ifndef QSGD_ORACLE_H
 #define QSGD_ORACLE_H
@@ -135,6 +137,16 @@ int qo_bbit_decode(const float* norms, const uint32_t* codes, uint64_t n, uint64
 int qo_bbit_decode_accumulate(const float* const* norms, const uint32_t* const* codes, int K,
                               uint64_t n, uint64_t d, uint32_t b, float* out, uint32_t* status);
 
+/* ---- Error feedback ("Sparsified SGD with Memory", abstract) -------------------
+ * p = e + g; the stream (or codes) carries Q(p); e <- p - Q(p), Q(p) as decoded, and
+ * e <- p where a coordinate has no record.  max_norm: scale by the max-norms of p
+ * (QSGDinf) when norms_in is NULL.  e[n] is read and overwritten. */
+int qo_encode_ef(const float* g, float* e, uint64_t n, uint64_t d, uint32_t s, uint64_t seed,
+                 int max_norm, const float* norms_in, uint32_t* words, uint64_t cap_words,
+                 uint64_t* offsets, float* norms_out, uint32_t* status);
+int qo_bbit_encode_ef(const float* g, float* e, uint64_t n, uint64_t d, uint32_t b, uint64_t seed,
+                      int max_norm, const float* norms_in, float* norms_out, uint32_t* codes,
+                      uint32_t* status);
 #ifdef __cplusplus
 }
 #endif

@@ -56,6 +56,10 @@ MUTANTS = {
     # max-norm (QSGDinf) scale
     "maxnorm_drops_nan": ("if (isnan(v[i])) return NAN;", ""),
     "maxnorm_signed": ("if (fabsf(v[i]) > mx) mx = fabsf(v[i]);", "if (v[i] > mx) mx = v[i];"),
+    # error feedback
+    "ef_residual_sign": ("e[i] = q[i] != 0.0f ? p[i] - q[i] : p[i];", "e[i] = q[i] != 0.0f ? q[i] - p[i] : p[i];"),
+    "ef_forgets_memory": ("p[i] = e[i] + g[i];", "p[i] = g[i];"),
+    "ef_drops_unsent": ("e[i] = q[i] != 0.0f ? p[i] - q[i] : p[i];", "e[i] = q[i] != 0.0f ? p[i] - q[i] : 0.0f;"),
     "bbit_code_shifted": ("uint64_t pos = (base + i) * b;\n            put_bits_msb_first",
                           "uint64_t pos = (base + i) * b + 1;\n            put_bits_msb_first"),
 }
@@ -168,6 +172,28 @@ def pin_battery(o) -> list:
     vn[5] = np.nan
     if not (np.array_equal(o.maxnorms(vm, 100), ref) and np.isnan(o.maxnorms(vn, 100)[0])):
         failed.append("maxnorm")
+    # error feedback: an exact step, the two outcomes of a fractional one, e = 0
+    try:
+        g = np.array([1, 4, 0, 0, 0, 0, 0, 0], np.float32)
+        e = np.array([2, 0, 0, 0, 0, 0, 0, 0], np.float32)
+        w, off, _, _, e_new = o.encode_ef(g, e, 8, 5, 1)
+        pw, _, _, _ = o.encode(g + e, 8, 5, 1)
+        if not (np.array_equal(w, pw) and e_new.view(np.uint32).tolist() == [0] * 8):
+            failed.append("ef_exact")
+        for seed in range(40):
+            _, _, _, _, e_new = o.encode_ef(np.array([-3, 4, 0, 0], np.float32), np.zeros(4, np.float32),
+                                            4, 1, seed)
+            if e_new[0] not in (-3.0, 2.0) or e_new[1] not in (4.0, -1.0):
+                failed.append("ef_outcomes")
+                break
+        g = workloads.normal(300, 12)
+        _, _, _, _, e_new = o.encode_ef(g, np.zeros(300, np.float32), 100, 2, 4)
+        w, off, _, _ = o.encode(g, 100, 2, 4)
+        q, _ = o.decode(w, off, 300, 100, 2)
+        if not np.array_equal(e_new[q == 0], g[q == 0]):
+            failed.append("ef_unsent")
+    except (RuntimeError, ValueError, AssertionError):
+        failed.append("ef")
     # small unbiasedness sweep: 4096 N(0,1) coordinates, s = 8, 400 seeds
     v = workloads.normal(4096, 1)
     sums = sc.Sums(v.size)
