@@ -468,6 +468,24 @@ def run_ours(args, w):
                "algorithmic_gbs": {k: i_alg[k] / i_times[k] / 1e6 for k in i_times},
                "roofline_frac": {k: i_alg[k] / i_times[k] / 1e6 / measured_peaks()[0] for k in i_times}}
 
+    # error feedback on the same gradient: the fused one-pass encode that reads g and
+    # the memory e and writes the stream and e (L2 scale), timed alone, L2 flushed
+    e_mem = torch.zeros(n, dtype=torch.float32, device=dev)
+
+    def f_enc():
+        check(B.qsgd_encode_ef(x.data_ptr(), e_mem.data_ptr(), n, d, s, seed, B.QSGD_NORM_L2, words.data_ptr(), cap,
+                               offsets.data_ptr(), ws.data_ptr(), ws_bytes, status.data_ptr(), sh), "qsgd_encode_ef")
+
+    f_ms = time_alone(f_enc)
+    if int(status.item()) != 0:
+        raise RuntimeError("device status %d in the error-feedback runs" % int(status.item()))
+    f_bits = int(offsets[-1].item())
+    f_comp = 4 * ((f_bits + 31) // 32) + 8 * (nb + 1)
+    f_alg = 12.0 * n + f_comp  # read g and e, write e and the stream
+    error_feedback = {"s": s, "bits_per_coord": f_bits / n, "us": {"encode": 1e3 * f_ms},
+                      "algorithmic_bytes": f_alg, "algorithmic_gbs": {"encode": f_alg / f_ms / 1e6},
+                      "roofline_frac": {"encode": f_alg / f_ms / 1e6 / measured_peaks()[0]}}
+
     peak, peak_kind = measured_peaks()
     in_bytes = 4.0 * n
     enc_bytes = in_bytes + comp_bytes            # read fp32, write stream + header
@@ -521,6 +539,7 @@ def run_ours(args, w):
         "gpu_launches": 3 * K,
         "bbit": bbit,
         "qsgdinf": qsgdinf,
+        "error_feedback": error_feedback,
         "clocks": clocks.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -123,8 +123,28 @@ QSGD_API int qsgd_encode(const float* d_in, uint64_t n, uint32_t d, uint32_t s, 
 
 /* qsgd_encode with the bucket scale chosen by norm_kind (QSGD_NORM_L2 or
  * QSGD_NORM_MAX, else QSGD_ERR_ARG).  Under QSGD_NORM_MAX the sent norm is exactly
- * max_i |v_i| and the largest value of a bucket gets level s. */
+ * max_i |v_i|, and the largest value of a bucket gets level s whenever
+ * fl(max * fl(s / max)) rounds to s. */
 QSGD_API int qsgd_encode_ex(const float* d_in, uint64_t n, uint32_t d, uint32_t s, uint64_t seed,
+                            uint32_t norm_kind, uint32_t* d_words, uint64_t words_capacity,
+                            uint64_t* d_offsets, void* d_ws, size_t ws_bytes, uint32_t* d_status,
+                            cudaStream_t stream);
+
+/* Error feedback around the Elias codec ("Sparsified SGD with Memory", abstract: the
+ * compressor keeps what it did not send in memory and adds it to the next gradient).
+ * Per coordinate, p = fl(e + g); the stream is qsgd_encode_ex of p (same d, s, seed,
+ * norm_kind, words, offsets, workspace and status rules); then e becomes
+ * fl(p - q), where q is the value qsgd_decode gives the coordinate.  Where no record
+ * was sent (q = +0), e keeps p bit for bit.  The learning rate is the caller's: scale
+ * g first.
+ *   d_g  [n] fp32, device, read only.
+ *   d_e  [n] fp32, device, read and overwritten.  It must not overlap d_g
+ *        (QSGD_ERR_ARG).  Both are 4-byte aligned.
+ * The encode is one fused kernel when the fast encoder takes the shape and both
+ * arrays are 16-byte aligned.  Otherwise it is three kernels: e <- e + g, the encoder
+ * on e, and a pass that subtracts the decoded values.  After a non-zero status
+ * (overflow, abort), d_e is unspecified. */
+QSGD_API int qsgd_encode_ef(const float* d_g, float* d_e, uint64_t n, uint32_t d, uint32_t s, uint64_t seed,
                             uint32_t norm_kind, uint32_t* d_words, uint64_t words_capacity,
                             uint64_t* d_offsets, void* d_ws, size_t ws_bytes, uint32_t* d_status,
                             cudaStream_t stream);
@@ -214,6 +234,15 @@ QSGD_API int qsgd_bbit_encode(const float* d_in, uint64_t n, uint32_t d, uint32_
 QSGD_API int qsgd_bbit_encode_ex(const float* d_in, uint64_t n, uint32_t d, uint32_t b, uint64_t seed,
                                  uint32_t norm_kind, float* d_norms, uint32_t* d_codes, uint32_t* d_status,
                                  cudaStream_t stream);
+
+/* Error feedback around the b-bit codec: p = fl(e + g) is coded as qsgd_bbit_encode_ex
+ * would code it, and e becomes fl(p - q) (q as qsgd_bbit_decode gives it), or p where
+ * the code's level is 0.  The argument rules are those of qsgd_encode_ef: d_g is read,
+ * d_e is overwritten, and the two must not overlap.  The encode is one kernel for
+ * d in {128, 256, 512, 1024} with d_g and d_e 16-byte aligned, else three. */
+QSGD_API int qsgd_bbit_encode_ef(const float* d_g, float* d_e, uint64_t n, uint32_t d, uint32_t b,
+                                 uint64_t seed, uint32_t norm_kind, float* d_norms, uint32_t* d_codes,
+                                 uint32_t* d_status, cudaStream_t stream);
 
 /* b-bit decoder: d_out[0..n) = fl(fl(norm/s) * k), negated for sign 1, +0.0 for k = 0.
  * Sets QSGD_ST_BAD_STREAM for a negative or non-finite norm, a non-zero code under a

@@ -50,6 +50,7 @@ _SIGS = {
     "qsgd_workspace_init": (_int, [_vp, _sz, _vp]),
     "qsgd_encode": (_int, [_vp, _u64, _u32, _u32, _u64, _vp, _u64, _vp, _vp, _sz, _vp, _vp]),
     "qsgd_encode_ex": (_int, [_vp, _u64, _u32, _u32, _u64, _u32, _vp, _u64, _vp, _vp, _sz, _vp, _vp]),
+    "qsgd_encode_ef": (_int, [_vp, _vp, _u64, _u32, _u32, _u64, _u32, _vp, _u64, _vp, _vp, _sz, _vp, _vp]),
     "qsgd_decode": (_int, [_vp, _u64, _vp, _u64, _u32, _u32, _vp, _vp, _vp]),
     "qsgd_decode_accumulate": (_int, [ctypes.POINTER(_vp), ctypes.POINTER(_u64), ctypes.POINTER(_vp),
                                       _int, _u64, _u32, _u32, _vp, _vp, _vp]),
@@ -58,6 +59,7 @@ _SIGS = {
     "qsgd_bbit_code_words": (_u64, [_u64, _u32]),
     "qsgd_bbit_encode": (_int, [_vp, _u64, _u32, _u32, _u64, _vp, _vp, _vp, _vp]),
     "qsgd_bbit_encode_ex": (_int, [_vp, _u64, _u32, _u32, _u64, _u32, _vp, _vp, _vp, _vp]),
+    "qsgd_bbit_encode_ef": (_int, [_vp, _vp, _u64, _u32, _u32, _u64, _u32, _vp, _vp, _vp, _vp]),
     "qsgd_bbit_decode": (_int, [_vp, _vp, _u64, _u32, _u32, _vp, _vp, _vp]),
     "qsgd_bbit_decode_accumulate": (_int, [ctypes.POINTER(_vp), ctypes.POINTER(_vp), _int, _u64, _u32, _u32,
                                            _vp, _vp, _vp]),
@@ -114,6 +116,12 @@ def qsgd_encode_ex(d_in: int, n: int, d: int, s: int, seed: int, norm_kind: int,
                                    d_offsets, d_ws, ws_bytes, d_status, stream))
 
 
+def qsgd_encode_ef(d_g: int, d_e: int, n: int, d: int, s: int, seed: int, norm_kind: int, d_words: int,
+                   words_capacity: int, d_offsets: int, d_ws: int, ws_bytes: int, d_status: int, stream: int) -> int:
+    return int(_lib.qsgd_encode_ef(d_g, d_e, n, d, s, seed & 0xFFFFFFFFFFFFFFFF, norm_kind, d_words, words_capacity,
+                                   d_offsets, d_ws, ws_bytes, d_status, stream))
+
+
 def qsgd_decode(d_words: int, num_words: int, d_offsets: int, n: int, d: int, s: int, d_out: int,
                 d_status: int, stream: int) -> int:
     return int(_lib.qsgd_decode(d_words, num_words, d_offsets, n, d, s, d_out, d_status, stream))
@@ -150,6 +158,12 @@ def qsgd_bbit_encode(d_in: int, n: int, d: int, b: int, seed: int, d_norms: int,
 def qsgd_bbit_encode_ex(d_in: int, n: int, d: int, b: int, seed: int, norm_kind: int, d_norms: int, d_codes: int,
                         d_status: int, stream: int) -> int:
     return int(_lib.qsgd_bbit_encode_ex(d_in, n, d, b, seed & 0xFFFFFFFFFFFFFFFF, norm_kind, d_norms, d_codes,
+                                        d_status, stream))
+
+
+def qsgd_bbit_encode_ef(d_g: int, d_e: int, n: int, d: int, b: int, seed: int, norm_kind: int, d_norms: int,
+                        d_codes: int, d_status: int, stream: int) -> int:
+    return int(_lib.qsgd_bbit_encode_ef(d_g, d_e, n, d, b, seed & 0xFFFFFFFFFFFFFFFF, norm_kind, d_norms, d_codes,
                                         d_status, stream))
 
 
@@ -232,6 +246,30 @@ def encode(x, d: int, s: int, seed: int, words=None, offsets=None, status=None,
     return Encoded(words, offsets, n, d, s, seed, status)
 
 
+def encode_ef(g, e, d: int, s: int, seed: int, words=None, offsets=None, status=None,
+              norm_kind: int = QSGD_NORM_L2) -> Encoded:
+    """Error feedback: encodes p = e + g and leaves p minus its decoded value in e."""
+    torch = _torch()
+    for t in (g, e):
+        assert t.is_cuda and t.dtype == torch.float32 and t.is_contiguous()
+    n = g.numel()
+    assert e.numel() == n
+    nb = qsgd_num_buckets(n, d)
+    cap = qsgd_max_encoded_words(n, d, s)
+    dev = g.device
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    if words is None:
+        words = torch.empty(max(cap, 1), dtype=torch.int32, device=dev)
+    if offsets is None:
+        offsets = torch.empty(nb + 1, dtype=torch.int64, device=dev)
+    if status is None:
+        status = torch.zeros(1, dtype=torch.int32, device=dev)
+    ws = workspace(n, d, s, dev, stream)
+    _check(qsgd_encode_ef(g.data_ptr(), e.data_ptr(), n, d, s, seed, norm_kind, words.data_ptr(), words.numel(),
+                          offsets.data_ptr(), ws.data_ptr(), ws.numel(), status.data_ptr(), stream), "qsgd_encode_ef")
+    return Encoded(words, offsets, n, d, s, seed, status)
+
+
 def decode(enc: Encoded, out=None, status=None):
     torch = _torch()
     dev = enc.words.device
@@ -286,6 +324,27 @@ def bbit_encode(x, d: int, b: int, seed: int, norms=None, codes=None, status=Non
         status = torch.zeros(1, dtype=torch.int32, device=dev)
     _check(qsgd_bbit_encode_ex(x.data_ptr(), n, d, b, seed, norm_kind, norms.data_ptr(), codes.data_ptr(),
                                status.data_ptr(), stream), "qsgd_bbit_encode_ex")
+    return BbitEncoded(norms, codes, n, d, b, seed, status)
+
+
+def bbit_encode_ef(g, e, d: int, b: int, seed: int, norms=None, codes=None, status=None,
+                   norm_kind: int = QSGD_NORM_L2) -> BbitEncoded:
+    """Error feedback: codes p = e + g and leaves p minus its decoded value in e."""
+    torch = _torch()
+    for t in (g, e):
+        assert t.is_cuda and t.dtype == torch.float32 and t.is_contiguous()
+    n = g.numel()
+    assert e.numel() == n
+    dev = g.device
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    if norms is None:
+        norms = torch.empty(max(qsgd_num_buckets(n, d), 1), dtype=torch.float32, device=dev)
+    if codes is None:
+        codes = torch.empty(max(qsgd_bbit_code_words(n, b), 1), dtype=torch.int32, device=dev)
+    if status is None:
+        status = torch.zeros(1, dtype=torch.int32, device=dev)
+    _check(qsgd_bbit_encode_ef(g.data_ptr(), e.data_ptr(), n, d, b, seed, norm_kind, norms.data_ptr(),
+                               codes.data_ptr(), status.data_ptr(), stream), "qsgd_bbit_encode_ef")
     return BbitEncoded(norms, codes, n, d, b, seed, status)
 
 

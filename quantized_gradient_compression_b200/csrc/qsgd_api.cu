@@ -87,16 +87,24 @@ int qsgd_workspace_init(void* d_ws, size_t ws_bytes, cudaStream_t stream) {
     return cudaMemsetAsync(d_ws, 0, ws_bytes, stream) == cudaSuccess ? QSGD_OK : QSGD_ERR_CUDA;
 }
 
-int qsgd_encode_ex(const float* d_in, uint64_t n, uint32_t d, uint32_t s, uint64_t seed, uint32_t norm_kind,
+}  // extern "C"
+
+namespace {
+
+constexpr int kNothingToDo = -1;  // n == 0: only the end of the header is written (no QSGD_* code is negative)
+
+// Checks the arguments of an encode of d_in and fills the kernel arguments.
+// Returns QSGD_OK, kNothingToDo (n == 0, header written) or a QSGD_ERR_* code.
+int prepare_encode(const float* d_in, uint64_t n, uint32_t d, uint32_t s, uint64_t seed, uint32_t norm_kind,
                    uint32_t* d_words, uint64_t words_capacity, uint64_t* d_offsets, void* d_ws, size_t ws_bytes,
-                   uint32_t* d_status, cudaStream_t stream) {
+                   uint32_t* d_status, cudaStream_t stream, EncodeArgs& a, bool& fast) {
     if (norm_kind != QSGD_NORM_L2 && norm_kind != QSGD_NORM_MAX) return QSGD_ERR_ARG;
     if (!valid_params(n, d, s) || !d_offsets || !d_status) return QSGD_ERR_ARG;
     if (max_bits(n, d, s) > kMaxStreamBits) return QSGD_ERR_ARG;
     if ((reinterpret_cast<uintptr_t>(d_offsets) & 7u) != 0 || (reinterpret_cast<uintptr_t>(d_words) & 3u) != 0)
         return QSGD_ERR_ARG;
     if (n == 0) {
-        return cudaMemsetAsync(d_offsets, 0, sizeof(uint64_t), stream) == cudaSuccess ? QSGD_OK
+        return cudaMemsetAsync(d_offsets, 0, sizeof(uint64_t), stream) == cudaSuccess ? kNothingToDo
                                                                                       : QSGD_ERR_CUDA;
     }
     if (!d_in || !d_words || !d_ws) return QSGD_ERR_ARG;
@@ -106,7 +114,7 @@ int qsgd_encode_ex(const float* d_in, uint64_t n, uint32_t d, uint32_t s, uint64
     if (ws_bytes < L.total) return QSGD_ERR_WORKSPACE;
 
     char* ws = static_cast<char*>(d_ws);
-    EncodeArgs a{};
+    a = EncodeArgs{};
     a.in = d_in;
     a.n = n;
     a.d = d;
@@ -118,6 +126,7 @@ int qsgd_encode_ex(const float* d_in, uint64_t n, uint32_t d, uint32_t s, uint64
     a.offsets = d_offsets;
     a.status = d_status;
     a.norm_kind = norm_kind;
+    a.ef = nullptr;
     a.ctrl = reinterpret_cast<ScanControl*>(ws);
     a.tdesc = reinterpret_cast<uint64_t*>(ws + L.desc_off);
     a.ts = reinterpret_cast<TileState*>(ws + L.tiles_off);
@@ -126,7 +135,7 @@ int qsgd_encode_ex(const float* d_in, uint64_t n, uint32_t d, uint32_t s, uint64
     // the fast path when its tile fits in shared memory, else the general one
     const uint64_t fast_tile_bits = static_cast<uint64_t>(kFastWarps) * (32u + static_cast<uint64_t>(d) * wl);
     const uint32_t fast_words = static_cast<uint32_t>(std::min<uint64_t>(ceil_div(fast_tile_bits, 32) + 2, 1u << 24));
-    const bool fast = fast_eligible(d_in, d, s) && fast_smem_bytes(d, s, fast_words) <= 200 * 1024;
+    fast = fast_eligible(d_in, d, s) && fast_smem_bytes(d, s, fast_words) <= 200 * 1024;
     if (fast) {
         a.buckets_per_tile = kFastWarps;  // one bucket per warp
         a.ntiles = ceil_div(a.nb, kFastWarps);
@@ -145,8 +154,58 @@ int qsgd_encode_ex(const float* d_in, uint64_t n, uint32_t d, uint32_t s, uint64
                                      : general_smem_bytes(a.smem_words, a.buckets_per_tile);
     if (smem_bytes > 200 * 1024) return QSGD_ERR_ARG;
     if (a.ntiles > L.max_tiles) return QSGD_ERR_WORKSPACE;
-    const cudaError_t e = launch_encode(a, fast, stream);
-    return e == cudaSuccess ? QSGD_OK : QSGD_ERR_CUDA;
+    return QSGD_OK;
+}
+
+// Whether [a, a + n) and [b, b + n) share a float.
+bool overlaps(const float* a, const float* b, uint64_t n) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    const uint64_t bytes = n * sizeof(float);
+    return x < y + bytes && y < x + bytes;
+}
+
+}  // namespace
+
+extern "C" {
+
+int qsgd_encode_ex(const float* d_in, uint64_t n, uint32_t d, uint32_t s, uint64_t seed, uint32_t norm_kind,
+                   uint32_t* d_words, uint64_t words_capacity, uint64_t* d_offsets, void* d_ws, size_t ws_bytes,
+                   uint32_t* d_status, cudaStream_t stream) {
+    EncodeArgs a;
+    bool fast = false;
+    const int rc = prepare_encode(d_in, n, d, s, seed, norm_kind, d_words, words_capacity, d_offsets, d_ws, ws_bytes,
+                                  d_status, stream, a, fast);
+    if (rc != QSGD_OK) return rc == kNothingToDo ? QSGD_OK : rc;
+    return launch_encode(a, fast, stream) == cudaSuccess ? QSGD_OK : QSGD_ERR_CUDA;
+}
+
+int qsgd_encode_ef(const float* d_g, float* d_e, uint64_t n, uint32_t d, uint32_t s, uint64_t seed,
+                   uint32_t norm_kind, uint32_t* d_words, uint64_t words_capacity, uint64_t* d_offsets, void* d_ws,
+                   size_t ws_bytes, uint32_t* d_status, cudaStream_t stream) {
+    if (n > 0) {
+        if (!d_g || !d_e || ((reinterpret_cast<uintptr_t>(d_g) | reinterpret_cast<uintptr_t>(d_e)) & 3u) != 0)
+            return QSGD_ERR_ARG;
+        if (overlaps(d_g, d_e, n)) return QSGD_ERR_ARG;
+    }
+    EncodeArgs a;
+    bool fast = false;
+    int rc = prepare_encode(d_g, n, d, s, seed, norm_kind, d_words, words_capacity, d_offsets, d_ws, ws_bytes,
+                            d_status, stream, a, fast);
+    if (rc != QSGD_OK) return rc == kNothingToDo ? QSGD_OK : rc;
+    if (fast && (reinterpret_cast<uintptr_t>(d_e) & 15u) == 0) {
+        // one pass: the fast encoder reads g and e and writes the stream and e
+        a.ef = d_e;
+        return launch_encode(a, true, stream) == cudaSuccess ? QSGD_OK : QSGD_ERR_CUDA;
+    }
+    // three passes: e <- e + g; encode p from e; e <- p - decoded
+    rc = prepare_encode(d_e, n, d, s, seed, norm_kind, d_words, words_capacity, d_offsets, d_ws, ws_bytes, d_status,
+                        stream, a, fast);
+    if (rc != QSGD_OK) return rc;
+    if (launch_ef_add(d_g, d_e, n, stream) != cudaSuccess) return QSGD_ERR_CUDA;
+    if (launch_encode(a, fast, stream) != cudaSuccess) return QSGD_ERR_CUDA;
+    return launch_ef_residual(d_e, d_words, words_capacity, d_offsets, n, d, s, seed, stream) == cudaSuccess
+               ? QSGD_OK
+               : QSGD_ERR_CUDA;
 }
 
 int qsgd_encode(const float* d_in, uint64_t n, uint32_t d, uint32_t s, uint64_t seed, uint32_t* d_words,
@@ -214,9 +273,34 @@ int qsgd_bbit_encode_ex(const float* d_in, uint64_t n, uint32_t d, uint32_t b, u
     if (!d_in || !d_norms || !d_codes || (reinterpret_cast<uintptr_t>(d_in) & 3u) != 0 ||
         (reinterpret_cast<uintptr_t>(d_norms) & 3u) != 0 || (reinterpret_cast<uintptr_t>(d_codes) & 3u) != 0)
         return QSGD_ERR_ARG;
-    return launch_bbit_encode(d_in, n, d, b, seed, norm_kind, d_norms, d_codes, d_status, stream) == cudaSuccess
+    return launch_bbit_encode(d_in, nullptr, n, d, b, seed, norm_kind, d_norms, d_codes, d_status, stream) ==
+                   cudaSuccess
                ? QSGD_OK
                : QSGD_ERR_CUDA;
+}
+
+int qsgd_bbit_encode_ef(const float* d_g, float* d_e, uint64_t n, uint32_t d, uint32_t b, uint64_t seed,
+                        uint32_t norm_kind, float* d_norms, uint32_t* d_codes, uint32_t* d_status,
+                        cudaStream_t stream) {
+    if (!valid_bbit(n, d, b) || !d_status) return QSGD_ERR_ARG;
+    if (norm_kind != QSGD_NORM_L2 && norm_kind != QSGD_NORM_MAX) return QSGD_ERR_ARG;
+    if (n == 0) return QSGD_OK;
+    if (!d_g || !d_e || !d_norms || !d_codes ||
+        ((reinterpret_cast<uintptr_t>(d_g) | reinterpret_cast<uintptr_t>(d_e) | reinterpret_cast<uintptr_t>(d_norms) |
+          reinterpret_cast<uintptr_t>(d_codes)) & 3u) != 0)
+        return QSGD_ERR_ARG;
+    if (overlaps(d_g, d_e, n)) return QSGD_ERR_ARG;
+    if (bbit_fast_shape(d_g, d_e, d))  // one pass
+        return launch_bbit_encode(d_g, d_e, n, d, b, seed, norm_kind, d_norms, d_codes, d_status, stream) ==
+                       cudaSuccess
+                   ? QSGD_OK
+                   : QSGD_ERR_CUDA;
+    // three passes: e <- e + g; encode p from e; e <- p - decoded
+    if (launch_ef_add(d_g, d_e, n, stream) != cudaSuccess) return QSGD_ERR_CUDA;
+    if (launch_bbit_encode(d_e, nullptr, n, d, b, seed, norm_kind, d_norms, d_codes, d_status, stream) !=
+        cudaSuccess)
+        return QSGD_ERR_CUDA;
+    return launch_bbit_ef_residual(d_e, d_norms, d_codes, n, d, b, stream) == cudaSuccess ? QSGD_OK : QSGD_ERR_CUDA;
 }
 
 int qsgd_bbit_encode(const float* d_in, uint64_t n, uint32_t d, uint32_t b, uint64_t seed, float* d_norms,

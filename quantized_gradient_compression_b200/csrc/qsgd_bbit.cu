@@ -34,10 +34,11 @@ __device__ __forceinline__ uint32_t bbit_code(float v, float sinv, uint32_t r, u
 // NC codes.  When NC*b < 32, G = 32 / (NC b) neighbouring lanes share a word and
 // OR their parts together with shuffles.
 // ---------------------------------------------------------------------------
-template <int V, int B>
-__global__ void __launch_bounds__(kBbitBlock) bbit_encode_fast(const float* __restrict__ in, uint64_t n,
-                                                               uint32_t d, uint64_t seed, uint32_t norm_kind,
-                                                               float* norms, uint32_t* codes, uint32_t* status) {
+template <int V, int B, bool kEF>
+__global__ void __launch_bounds__(kBbitBlock) bbit_encode_fast(const float* __restrict__ in, float* __restrict__ ef,
+                                                               uint64_t n, uint32_t d, uint64_t seed,
+                                                               uint32_t norm_kind, float* norms, uint32_t* codes,
+                                                               uint32_t* status) {
     constexpr int NC = 4 * V;
     constexpr uint32_t S = (1u << (B - 1)) - 1u;
     constexpr int kLaneBits = NC * B;  // 8 .. 256
@@ -52,6 +53,8 @@ __global__ void __launch_bounds__(kBbitBlock) bbit_encode_fast(const float* __re
         const uint64_t base = bk * d;
         const uint32_t m = static_cast<uint32_t>(min(static_cast<uint64_t>(d), n - base));
         const uint32_t first = static_cast<uint32_t>(lane) * NC;
+        float ev[kEF ? NC : 1];  // error feedback: the memory of these coordinates
+        if constexpr (kEF) ef_load<V>(ef + base, first, m, ev);
         float x[NC];
 #pragma unroll
         for (int j = 0; j < V; ++j) {
@@ -69,6 +72,10 @@ __global__ void __launch_bounds__(kBbitBlock) bbit_encode_fast(const float* __re
             x[4 * j + 2] = q.z;
             x[4 * j + 3] = q.w;
         }
+        if constexpr (kEF) {  // p = e + g
+#pragma unroll
+            for (int q = 0; q < NC; ++q) x[q] = __fadd_rn(ev[q], x[q]);
+        }
         const float norm = norm_kind == QSGD_NORM_MAX ? warp_bucket_maxnorm<NC>(x) : warp_bucket_norm<NC>(x, true);
         const BucketScale sc = bucket_scale(norm, S, true, status, lane == 0);
         if (lane == 0) norms[bk] = sc.sent;
@@ -76,6 +83,7 @@ __global__ void __launch_bounds__(kBbitBlock) bbit_encode_fast(const float* __re
 #pragma unroll
         for (int w = 0; w < kLaneWords; ++w) part[w] = 0u;
         if (sc.good) {
+            const float scale = kEF ? __fdiv_rn(sc.sent, static_cast<float>(S)) : 0.f;
 #pragma unroll
             for (int j = 0; j < V; ++j) {
                 const uint4 rr = philox4x32_10(((base + first) >> 2) + j, key);
@@ -84,6 +92,7 @@ __global__ void __launch_bounds__(kBbitBlock) bbit_encode_fast(const float* __re
                 for (int c = 0; c < 4; ++c) {
                     const int q = 4 * j + c;
                     const uint32_t code = first + q < m ? bbit_code(x[q], sc.sinv, rw[c], S, B) : 0u;
+                    if constexpr (kEF) ev[q] = ef_residual(x[q], code & S, code >> (B - 1), scale);
                     const int bit = q * B;  // offset of the code inside the lane's bits
                     if (kLaneBits >= 32)
                         part[bit / 32] |= code << (32 - B - bit % 32);
@@ -91,6 +100,12 @@ __global__ void __launch_bounds__(kBbitBlock) bbit_encode_fast(const float* __re
                         part[0] |= code << (kLaneBits - B - bit);
                 }
             }
+        }
+        if constexpr (kEF) {  // the memory keeps p minus what a receiver decodes (p where nothing was sent)
+            if (sc.good)
+                ef_store<V>(ef + base, first, m, ev);
+            else
+                ef_store<V>(ef + base, first, m, x);
         }
         // the bucket's codes start on a word: d * b is a multiple of 32
         uint32_t* out = codes + (base * B) / 32;
@@ -290,23 +305,32 @@ int grid_for(uint64_t items, int per_sm_blocks = 8) {
     return static_cast<int>(std::max<uint64_t>(1, std::min<uint64_t>(want, static_cast<uint64_t>(sms) * per_sm_blocks)));
 }
 
-template <int B>
-cudaError_t launch_bbit_encode_b(const float* in, uint64_t n, uint32_t d, uint64_t seed, uint32_t nk, float* norms,
-                                 uint32_t* codes, uint32_t* status, cudaStream_t stream) {
-    const uint64_t nb = (n + d - 1) / d;
-    const bool fast = d % 128 == 0 && d <= 1024 && (reinterpret_cast<uintptr_t>(in) & 15u) == 0;
-    if (fast) {
-        const int grid = grid_for(nb * 32);
-        switch (d / 128) {
-            case 1: bbit_encode_fast<1, B><<<grid, kBbitBlock, 0, stream>>>(in, n, d, seed, nk, norms, codes, status); break;
-            case 2: bbit_encode_fast<2, B><<<grid, kBbitBlock, 0, stream>>>(in, n, d, seed, nk, norms, codes, status); break;
-            case 4: bbit_encode_fast<4, B><<<grid, kBbitBlock, 0, stream>>>(in, n, d, seed, nk, norms, codes, status); break;
-            case 8: bbit_encode_fast<8, B><<<grid, kBbitBlock, 0, stream>>>(in, n, d, seed, nk, norms, codes, status); break;
-            default: goto general;  // d = 384, 640, 768, 896: the general path
-        }
-        return cudaGetLastError();
+bool fast_shape(const float* in, const float* ef, uint32_t d) {
+    const bool pow2v = d == 128 || d == 256 || d == 512 || d == 1024;
+    return pow2v && ((reinterpret_cast<uintptr_t>(in) | reinterpret_cast<uintptr_t>(ef)) & 15u) == 0;
+}
+
+template <int B, bool kEF>
+cudaError_t launch_bbit_fast(const float* in, float* ef, uint64_t n, uint32_t d, uint64_t seed, uint32_t nk,
+                             float* norms, uint32_t* codes, uint32_t* status, cudaStream_t stream) {
+    const int grid = grid_for(((n + d - 1) / d) * 32);
+    switch (d / 128) {
+        case 1: bbit_encode_fast<1, B, kEF><<<grid, kBbitBlock, 0, stream>>>(in, ef, n, d, seed, nk, norms, codes, status); break;
+        case 2: bbit_encode_fast<2, B, kEF><<<grid, kBbitBlock, 0, stream>>>(in, ef, n, d, seed, nk, norms, codes, status); break;
+        case 4: bbit_encode_fast<4, B, kEF><<<grid, kBbitBlock, 0, stream>>>(in, ef, n, d, seed, nk, norms, codes, status); break;
+        default: bbit_encode_fast<8, B, kEF><<<grid, kBbitBlock, 0, stream>>>(in, ef, n, d, seed, nk, norms, codes, status); break;
     }
-general:
+    return cudaGetLastError();
+}
+
+template <int B>
+cudaError_t launch_bbit_encode_b(const float* in, float* ef, uint64_t n, uint32_t d, uint64_t seed, uint32_t nk,
+                                 float* norms, uint32_t* codes, uint32_t* status, cudaStream_t stream) {
+    // one pass: one warp per bucket of d = 128, 256, 512 or 1024, 16-byte aligned input
+    if (fast_shape(in, ef, d))
+        return ef ? launch_bbit_fast<B, true>(in, ef, n, d, seed, nk, norms, codes, status, stream)
+                  : launch_bbit_fast<B, false>(in, ef, n, d, seed, nk, norms, codes, status, stream);
+    const uint64_t nb = (n + d - 1) / d;
     bbit_norms<<<grid_for(nb * 32), kBbitBlock, 0, stream>>>(in, n, d, (1u << (B - 1)) - 1u, nk, norms, status);
     bbit_pack<B><<<grid_for((n * B + 31) / 32), kBbitBlock, 0, stream>>>(in, n, d, seed, norms, codes);
     return cudaGetLastError();
@@ -324,13 +348,16 @@ cudaError_t launch_bbit_decode_b(const float* norms, const uint32_t* codes, uint
 
 }  // namespace
 
-cudaError_t launch_bbit_encode(const float* in, uint64_t n, uint32_t d, uint32_t b, uint64_t seed,
+bool bbit_fast_shape(const float* in, const float* ef, uint32_t d) { return fast_shape(in, ef, d); }
+
+cudaError_t launch_bbit_encode(const float* in, float* ef, uint64_t n, uint32_t d, uint32_t b, uint64_t seed,
                                uint32_t norm_kind, float* norms, uint32_t* codes, uint32_t* status,
                                cudaStream_t stream) {
+    if (ef && !fast_shape(in, ef, d)) return cudaErrorInvalidValue;
     switch (b) {
-        case 2: return launch_bbit_encode_b<2>(in, n, d, seed, norm_kind, norms, codes, status, stream);
-        case 4: return launch_bbit_encode_b<4>(in, n, d, seed, norm_kind, norms, codes, status, stream);
-        default: return launch_bbit_encode_b<8>(in, n, d, seed, norm_kind, norms, codes, status, stream);
+        case 2: return launch_bbit_encode_b<2>(in, ef, n, d, seed, norm_kind, norms, codes, status, stream);
+        case 4: return launch_bbit_encode_b<4>(in, ef, n, d, seed, norm_kind, norms, codes, status, stream);
+        default: return launch_bbit_encode_b<8>(in, ef, n, d, seed, norm_kind, norms, codes, status, stream);
     }
 }
 

@@ -183,6 +183,57 @@ __device__ __forceinline__ float warp_maxnorm(const float* p, uint64_t m, int la
 }
 
 // ---------------------------------------------------------------------------
+// Error-feedback memory ("Sparsified SGD with Memory", abstract: the compressor
+// keeps what it did not send and adds it to the next gradient).  One lane's NC = 4V
+// coordinates [first, first + NC) of a bucket of m values at p: loads give zeros
+// past m, stores write nothing past m.  The memory is read once and written once
+// per step, so both stream past L1 (.cs).  p + first is 16-byte aligned.
+// ---------------------------------------------------------------------------
+template <int V>
+__device__ __forceinline__ void ef_load(const float* p, uint32_t first, uint32_t m, float (&v)[4 * V]) {
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+        const uint32_t i = first + 4 * j;
+        float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (i + 4 <= m) {
+            q = __ldcs(reinterpret_cast<const float4*>(p + i));
+        } else if (i < m) {
+            q.x = __ldcs(p + i);
+            if (i + 1 < m) q.y = __ldcs(p + i + 1);
+            if (i + 2 < m) q.z = __ldcs(p + i + 2);
+        }
+        v[4 * j + 0] = q.x;
+        v[4 * j + 1] = q.y;
+        v[4 * j + 2] = q.z;
+        v[4 * j + 3] = q.w;
+    }
+}
+
+template <int V>
+__device__ __forceinline__ void ef_store(float* p, uint32_t first, uint32_t m, const float (&v)[4 * V]) {
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+        const uint32_t i = first + 4 * j;
+        if (i + 4 <= m) {
+            __stcs(reinterpret_cast<float4*>(p + i), make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
+        } else if (i < m) {
+            __stcs(p + i, v[4 * j]);
+            if (i + 1 < m) __stcs(p + i + 1, v[4 * j + 1]);
+            if (i + 2 < m) __stcs(p + i + 2, v[4 * j + 2]);
+        }
+    }
+}
+
+// The memory left by one coordinate p = e + g sent as level k (sign `neg`) of step
+// `scale` = fl(norm / s): p minus the value a receiver decodes, fl(scale * k) with
+// the sign applied last; p itself when no record was sent.
+__device__ __forceinline__ float ef_residual(float p, uint32_t k, bool neg, float scale) {
+    if (k == 0u) return p;
+    const float q = __fmul_rn(scale, __uint2float_rn(k));
+    return __fsub_rn(p, neg ? -q : q);
+}
+
+// ---------------------------------------------------------------------------
 // Elias omega code of N >= 1 (Elias 1975): start from "0"; while N > 1, put the
 // binary form of N in front and continue with bitlength(N) - 1.  Returned as a
 // right-aligned value read MSB-first, and its length in bits.

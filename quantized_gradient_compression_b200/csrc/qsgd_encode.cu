@@ -139,7 +139,7 @@ __device__ __forceinline__ void prefetch_tile(const EncodeArgs& a, uint64_t t, f
 
 // Codes tile t into tbuf (tile-local bit offsets) and publishes A(t).  On entry
 // the tile's input is in flight into xin.  Two CTA barriers.
-template <int V, bool kShort>
+template <int V, bool kShort, bool kEF>
 __device__ __forceinline__ void code_tile(const EncodeArgs& a, uint64_t t, const uint32_t* t_after_slot, const uint32_t* rtab,
                                           uint32_t* tbuf, uint32_t* pb, float4* xin, TileSlot& slot,
                                           uint32_t epoch) {
@@ -152,6 +152,11 @@ __device__ __forceinline__ void code_tile(const EncodeArgs& a, uint64_t t, const
     const bool live = b < a.nb;
     const uint64_t base = b * a.d;
     const uint32_t first = lane * NC;  // first bucket-local coordinate of this lane
+
+    // error feedback: the memory of this lane's coordinates, loaded before the wait
+    const uint32_t mlen = live ? static_cast<uint32_t>(min(static_cast<uint64_t>(a.d), a.n - base)) : 0u;
+    float ev[kEF ? NC : 1];
+    if constexpr (kEF) ef_load<V>(a.ef + base, first, mlen, ev);
 
     asm volatile("cp.async.wait_all;\n" ::: "memory");  // the tile's input
     __syncthreads();  // B0: the tile's input has landed; every warp is done with tbuf's last tile
@@ -172,11 +177,16 @@ __device__ __forceinline__ void code_tile(const EncodeArgs& a, uint64_t t, const
             x[4 * j + 3] = q.w;
         }
     }
+    if constexpr (kEF) {  // p = e + g
+#pragma unroll
+        for (int q = 0; q < NC; ++q) x[q] = __fadd_rn(ev[q], x[q]);
+    }
 
     // --- bucket norm: per-lane FMA chain, butterfly (same value in all lanes) --
     const float norm = a.norm_kind == QSGD_NORM_MAX ? warp_bucket_maxnorm<NC>(x) : warp_bucket_norm<NC>(x, live);
     const BucketScale sc = bucket_scale(norm, a.s, live, a.status, lane == 0);
     if (!sc.good) {
+        if constexpr (kEF) ef_store<V>(a.ef + base, first, mlen, x);  // nothing sent: the memory keeps p
 #pragma unroll
         for (int q = 0; q < NC; ++q) x[q] = 0.f;
     }
@@ -193,6 +203,14 @@ __device__ __forceinline__ void code_tile(const EncodeArgs& a, uint64_t t, const
         for (int c = 0; c < 4; ++c) {
             const float v = x[4 * j + c];
             kq[4 * j + c] = quantize_level(v, sc.sinv, rw[c], a.s) | (__float_as_uint(v) & 0x80000000u);
+        }
+    }
+    if constexpr (kEF) {  // the memory keeps p minus what a receiver decodes
+        if (sc.good) {
+            const float scale = __fdiv_rn(sc.sent, __uint2float_rn(a.s));
+#pragma unroll
+            for (int q = 0; q < NC; ++q) ev[q] = ef_residual(x[q], kq[q] & 0x7FFFFFFFu, kq[q] >> 31, scale);
+            ef_store<V>(a.ef + base, first, mlen, ev);
         }
     }
 
@@ -402,7 +420,7 @@ __device__ __forceinline__ void store_tile(const EncodeArgs& a, const uint32_t* 
     for (uint32_t q = (sh ? 1u : 0u) + tid; q < qe; q += kFastBlock) store_word(a, w0 + q, word_at(q));
 }
 
-template <int V, bool kShort>
+template <int V, bool kShort, bool kEF>
 __global__ void __launch_bounds__(kFastBlock, (V <= 4 ? kFastMinBlocks : 1)) encode_fast(const __grid_constant__ EncodeArgs a) {
     constexpr int kEncDepth = enc_depth(V);
     constexpr int kEncBufs = kEncDepth + 1;
@@ -437,7 +455,7 @@ __global__ void __launch_bounds__(kFastBlock, (V <= 4 ? kFastMinBlocks : 1)) enc
     for (int j = 0; j < kEncDepth; ++j) {
         held[j] = s_ticket[j];
         if (held[j] < a.ntiles)
-            code_tile<V, kShort>(a, held[j], &s_ticket[j + 1], rtab, tbuf0 + j * a.smem_words, pb, xin, s_slot[j], epoch);
+            code_tile<V, kShort, kEF>(a, held[j], &s_ticket[j + 1], rtab, tbuf0 + j * a.smem_words, pb, xin, s_slot[j], epoch);
     }
     uint64_t tn = s_ticket[kEncDepth];
     __syncthreads();  // every thread has read s_ticket before the loop reuses it
@@ -454,7 +472,7 @@ __global__ void __launch_bounds__(kFastBlock, (V <= 4 ? kFastMinBlocks : 1)) enc
         const uint32_t r = static_cast<uint32_t>(t) / C;
         const uint32_t c = static_cast<uint32_t>(t) - r * C;
         if (tn < a.ntiles)
-            code_tile<V, kShort>(a, tn, &s_ticket[it & 1], rtab, tbuf0 + bn * a.smem_words, pb, xin, s_slot[bn], epoch);
+            code_tile<V, kShort, kEF>(a, tn, &s_ticket[it & 1], rtab, tbuf0 + bn * a.smem_words, pb, xin, s_slot[bn], epoch);
         else
             __syncthreads();  // orders the ticket, the accumulator reset and store_tile
         const uint64_t tnn = s_ticket[it & 1];
@@ -884,29 +902,30 @@ __global__ void __launch_bounds__(kBlock) encode_general(const __grid_constant__
     cta_exit(a.ctrl, epoch);
 }
 
-template <int V, bool kShort>
+template <int V, bool kShort, bool kEF>
 cudaError_t launch_fast(const EncodeArgs& a, cudaStream_t stream) {
     const size_t smem = fast_smem_bytes(a.d, a.s, a.smem_words);
     static bool attr_set[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 64 && !attr_set[dev]) {
-        cudaFuncSetAttribute(encode_fast<V, kShort>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+        cudaFuncSetAttribute(encode_fast<V, kShort, kEF>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
         attr_set[dev] = true;
     }
     int sms = 0, per_sm = 0;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, encode_fast<V, kShort>, kFastBlock, smem);
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, encode_fast<V, kShort, kEF>, kFastBlock, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const uint64_t grid = std::min<uint64_t>(a.ntiles, static_cast<uint64_t>(sms) * per_sm);
-    encode_fast<V, kShort><<<static_cast<unsigned>(grid), kFastBlock, smem, stream>>>(a);
+    encode_fast<V, kShort, kEF><<<static_cast<unsigned>(grid), kFastBlock, smem, stream>>>(a);
     return cudaGetLastError();
 }
 
 template <int V>
 cudaError_t launch_fast_v(const EncodeArgs& a, cudaStream_t stream) {
-    return a.s <= 31 ? launch_fast<V, true>(a, stream) : launch_fast<V, false>(a, stream);
+    if (a.ef) return a.s <= 31 ? launch_fast<V, true, true>(a, stream) : launch_fast<V, false, true>(a, stream);
+    return a.s <= 31 ? launch_fast<V, true, false>(a, stream) : launch_fast<V, false, false>(a, stream);
 }
 
 }  // namespace

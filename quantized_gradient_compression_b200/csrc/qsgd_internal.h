@@ -42,6 +42,7 @@ struct EncodeArgs {
     uint32_t buckets_per_tile;
     uint32_t smem_words;  // words of the per-tile (or per-chunk) bit buffer
     uint32_t norm_kind;   // QSGD_NORM_L2 or QSGD_NORM_MAX
+    float* ef;            // error-feedback memory fused into the fast encoder, or null
 };
 
 // Chooses the kernel, sets the launch shape and enqueues it.  Returns a CUDA
@@ -97,9 +98,19 @@ struct DecodeArgs {
 cudaError_t launch_decode(const DecodeArgs& a, bool accumulate, cudaStream_t stream);
 
 // Fixed-width b-bit variant (b in {2, 4, 8}, checked by the caller).
-cudaError_t launch_bbit_encode(const float* in, uint64_t n, uint32_t d, uint32_t b, uint64_t seed,
+cudaError_t launch_bbit_encode(const float* in, float* ef, uint64_t n, uint32_t d, uint32_t b, uint64_t seed,
                                uint32_t norm_kind, float* norms, uint32_t* codes, uint32_t* status,
                                cudaStream_t stream);
+// Whether launch_bbit_encode fuses error feedback for this shape (else ef must be null).
+bool bbit_fast_shape(const float* in, const float* ef, uint32_t d);
+
+// Error feedback for the shapes the fused encoders do not take (qsgd_ef.cu):
+// e <- e + g; then, after the encoder has read p from e, the residual passes.
+cudaError_t launch_ef_add(const float* g, float* e, uint64_t n, cudaStream_t stream);
+cudaError_t launch_ef_residual(float* e, const uint32_t* words, uint64_t cap_words, const uint64_t* offsets,
+                               uint64_t n, uint32_t d, uint32_t s, uint64_t seed, cudaStream_t stream);
+cudaError_t launch_bbit_ef_residual(float* e, const float* norms, const uint32_t* codes, uint64_t n, uint32_t d,
+                                    uint32_t b, cudaStream_t stream);
 cudaError_t launch_bbit_decode(const float* norms, const uint32_t* codes, uint64_t n, uint32_t d, uint32_t b,
                                float* out, bool accumulate, uint32_t* status, cudaStream_t stream);
 

@@ -111,3 +111,18 @@ def test_norm_kind_checked():
     # an unknown norm kind is refused before any CUDA call
     assert B.qsgd_encode_ex(256, 10, 4, 4, 0, 2, 256, 100, 256, 256, 4096, 256, 0) == B.QSGD_ERR_ARG
     assert B.qsgd_bbit_encode_ex(256, 10, 4, 4, 0, 7, 256, 256, 256, 0) == B.QSGD_ERR_ARG
+
+
+def test_error_feedback_arguments_checked():
+    from quantized_gradient_compression_b200 import binding as B
+
+    A = 1 << 20  # fake device addresses: every call below is refused before a CUDA call
+    # g and e overlap
+    assert B.qsgd_encode_ef(A, A + 64, 100, 4, 4, 0, 0, A * 8, 10_000, A * 16, A * 32, 1 << 20, A * 64, 0) \
+        == B.QSGD_ERR_ARG
+    assert B.qsgd_bbit_encode_ef(A, A + 64, 100, 4, 4, 0, 0, A * 8, A * 16, A * 64, 0) == B.QSGD_ERR_ARG
+    # a null memory, a misaligned gradient, an unknown norm kind
+    assert B.qsgd_encode_ef(A, 0, 100, 4, 4, 0, 0, A * 8, 10_000, A * 16, A * 32, 1 << 20, A * 64, 0) \
+        == B.QSGD_ERR_ARG
+    assert B.qsgd_bbit_encode_ef(A + 2, A * 4, 100, 4, 4, 0, 0, A * 8, A * 16, A * 64, 0) == B.QSGD_ERR_ARG
+    assert B.qsgd_bbit_encode_ef(A, A * 4, 100, 4, 4, 0, 5, A * 8, A * 16, A * 64, 0) == B.QSGD_ERR_ARG
