@@ -85,6 +85,10 @@ def _declare(lib):
         "qo_bbit_decode": (c_int, [f32p, u32p, c_u64, c_u64, c_u32, f32p, u32p]),
         "qo_bbit_decode_accumulate": (c_int, [ctypes.POINTER(f32p), ctypes.POINTER(u32p), c_int,
                                               c_u64, c_u64, c_u32, f32p, u32p]),
+        "qo_decode_mean": (c_int, [ctypes.POINTER(u32p), ctypes.POINTER(u64p), c_int,
+                                   c_u64, c_u64, c_u32, f32p, u32p]),
+        "qo_bbit_decode_mean": (c_int, [ctypes.POINTER(f32p), ctypes.POINTER(u32p), c_int,
+                                        c_u64, c_u64, c_u32, f32p, u32p]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -299,6 +303,22 @@ class Oracle:
         return out, st.value
 
 
+    def decode_mean(self, streams, n: int, d: int, s: int):
+        """Mean of the K decoded streams (list of (words, offsets)): (sum from +0) / K."""
+        K = len(streams)
+        ws = [np.ascontiguousarray(w if w.size else np.zeros(1, np.uint32), dtype=np.uint32)
+              for w, _ in streams]
+        os_ = [np.ascontiguousarray(o, dtype=np.uint64) for _, o in streams]
+        u32p = ctypes.POINTER(ctypes.c_uint32)
+        u64p = ctypes.POINTER(ctypes.c_uint64)
+        wp = (u32p * K)(*[_ptr(w, ctypes.c_uint32) for w in ws])
+        op = (u64p * K)(*[_ptr(o, ctypes.c_uint64) for o in os_])
+        out = np.zeros(max(n, 1), np.float32)
+        st = ctypes.c_uint32(0)
+        rc = self.lib.qo_decode_mean(wp, op, K, n, d, s, _ptr(out, ctypes.c_float), ctypes.byref(st))
+        assert rc == 0
+        return out[:n], st.value
+
     # ---- fixed-width b-bit variant ----------------------------------------------
     def bbit_levels(self, b: int) -> int:
         return int(self.lib.qo_bbit_levels(b))
@@ -409,6 +429,24 @@ class Oracle:
                                                 ctypes.byref(st))
         assert rc == 0
         return out, st.value
+
+
+    def bbit_decode_mean(self, streams, n: int, d: int, b: int):
+        """Mean of the K decoded b-bit streams (list of (norms, codes))."""
+        K = len(streams)
+        ns = [np.ascontiguousarray(x if x.size else np.zeros(1, np.float32), dtype=np.float32)
+              for x, _ in streams]
+        cs = [np.ascontiguousarray(c if c.size else np.zeros(1, np.uint32), dtype=np.uint32)
+              for _, c in streams]
+        f32p = ctypes.POINTER(ctypes.c_float)
+        u32p = ctypes.POINTER(ctypes.c_uint32)
+        npp = (f32p * K)(*[_ptr(x, ctypes.c_float) for x in ns])
+        cpp = (u32p * K)(*[_ptr(c, ctypes.c_uint32) for c in cs])
+        out = np.zeros(max(n, 1), np.float32)
+        st = ctypes.c_uint32(0)
+        rc = self.lib.qo_bbit_decode_mean(npp, cpp, K, n, d, b, _ptr(out, ctypes.c_float), ctypes.byref(st))
+        assert rc == 0
+        return out[:n], st.value
 
 
 _default = None

@@ -551,3 +551,26 @@ done:
     free(p);
     return rc;
 }
+
+/* ---- Data-parallel exchange: the mean of K received streams ---------------------
+ * "for distributed data-parallel optimization" (definition paragraph): every node
+ * quantises its gradient and the nodes exchange the encodings; a node's update is
+ * the mean of the K decoded gradients.  The sum runs left to right from +0 as in
+ * decode-accumulate, then one fp32 division by K per coordinate. */
+int qo_decode_mean(const uint32_t* const* words, const uint64_t* const* offsets, int K, uint64_t n,
+                   uint64_t d, uint32_t s, float* out, uint32_t* status) {
+    if (K < 1) return -1;
+    for (uint64_t i = 0; i < n; ++i) out[i] = 0.0f;
+    if (qo_decode_accumulate(words, offsets, K, n, d, s, out, status) != 0) return -1;
+    for (uint64_t i = 0; i < n; ++i) out[i] = out[i] / (float)K;
+    return 0;
+}
+
+int qo_bbit_decode_mean(const float* const* norms, const uint32_t* const* codes, int K, uint64_t n,
+                        uint64_t d, uint32_t b, float* out, uint32_t* status) {
+    if (K < 1) return -1;
+    for (uint64_t i = 0; i < n; ++i) out[i] = 0.0f;
+    if (qo_bbit_decode_accumulate(norms, codes, K, n, d, b, out, status) != 0) return -1;
+    for (uint64_t i = 0; i < n; ++i) out[i] = out[i] / (float)K;
+    return 0;
+}

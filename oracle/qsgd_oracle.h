@@ -19,7 +19,9 @@
  * unbiasedness, the closed-form variance, the sparsity bound and the 2.818n+32
  * bit bound from the page's claims; the size bound by brute force.  Error feedback
  * ("Sparsified SGD with Memory", abstract): exact steps, closed-form outcomes and the
- * telescoping sum of sent values plus memory (tests/test_oracle_ef.py).
+ * telescoping sum of sent values plus memory (tests/test_oracle_ef.py).  The mean of
+ * K received streams: hand values, K = 1 and 2, the rounding bound, unbiasedness
+ * (tests/test_oracle_mean.py).
  */
 #ifndef QSGD_ORACLE_H
 #define QSGD_ORACLE_H
@@ -147,6 +149,13 @@ int qo_encode_ef(const float* g, float* e, uint64_t n, uint64_t d, uint32_t s, u
 int qo_bbit_encode_ef(const float* g, float* e, uint64_t n, uint64_t d, uint32_t b, uint64_t seed,
                       int max_norm, const float* norms_in, float* norms_out, uint32_t* codes,
                       uint32_t* status);
+/* ---- Data-parallel exchange ("for distributed data-parallel optimization") -------
+ * out[i] = (q^0[i] + ... + q^{K-1}[i]) / K: the sum left to right from +0, then one
+ * fp32 division by K. */
+int qo_decode_mean(const uint32_t* const* words, const uint64_t* const* offsets, int K, uint64_t n,
+                   uint64_t d, uint32_t s, float* out, uint32_t* status);
+int qo_bbit_decode_mean(const float* const* norms, const uint32_t* const* codes, int K, uint64_t n,
+                        uint64_t d, uint32_t b, float* out, uint32_t* status);
 #ifdef __cplusplus
 }
 #endif

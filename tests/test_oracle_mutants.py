@@ -60,6 +60,13 @@ MUTANTS = {
     "ef_residual_sign": ("e[i] = q[i] != 0.0f ? p[i] - q[i] : p[i];", "e[i] = q[i] != 0.0f ? q[i] - p[i] : p[i];"),
     "ef_forgets_memory": ("p[i] = e[i] + g[i];", "p[i] = g[i];"),
     "ef_drops_unsent": ("e[i] = q[i] != 0.0f ? p[i] - q[i] : p[i];", "e[i] = q[i] != 0.0f ? p[i] - q[i] : 0.0f;"),
+    # mean of K streams
+    "mean_not_divided": ("if (qo_decode_accumulate(words, offsets, K, n, d, s, out, status) != 0) return -1;\n    for (uint64_t i = 0; i < n; ++i) out[i] = out[i] / (float)K;",
+                         "if (qo_decode_accumulate(words, offsets, K, n, d, s, out, status) != 0) return -1;"),
+    "mean_wrong_count": ("if (qo_decode_accumulate(words, offsets, K, n, d, s, out, status) != 0) return -1;\n    for (uint64_t i = 0; i < n; ++i) out[i] = out[i] / (float)K;",
+                         "if (qo_decode_accumulate(words, offsets, K, n, d, s, out, status) != 0) return -1;\n    for (uint64_t i = 0; i < n; ++i) out[i] = out[i] / (float)(K + 1);"),
+    "bbit_mean_not_divided": ("if (qo_bbit_decode_accumulate(norms, codes, K, n, d, b, out, status) != 0) return -1;\n    for (uint64_t i = 0; i < n; ++i) out[i] = out[i] / (float)K;",
+                              "if (qo_bbit_decode_accumulate(norms, codes, K, n, d, b, out, status) != 0) return -1;"),
     "bbit_code_shifted": ("uint64_t pos = (base + i) * b;\n            put_bits_msb_first",
                           "uint64_t pos = (base + i) * b + 1;\n            put_bits_msb_first"),
 }
@@ -194,6 +201,17 @@ def pin_battery(o) -> list:
             failed.append("ef_unsent")
     except (RuntimeError, ValueError, AssertionError):
         failed.append("ef")
+    # mean of K streams: hand values, and two equal b-bit streams give their decode
+    mo, _ = o.decode_mean([(a, np.array([0, 45], np.uint64)), (b, np.array([0, 37], np.uint64))], 2, 2, 5)
+    if mo.tolist() != [1.5, float(np.float32(np.float32(4) + np.float32(-0.4)) / np.float32(2))]:
+        failed.append("mean_hand")
+    try:
+        c1, n1, _ = o.bbit_encode(np.array([2, -3, 6, 0, 0, 0, 0, 0], np.float32), 8, 4, 1)
+        bm, _ = o.bbit_decode_mean([(n1, c1), (n1, c1)], 8, 8, 4)
+        if bm.tolist() != [2, -3, 6, 0, 0, 0, 0, 0]:
+            failed.append("bbit_mean")
+    except (ValueError, AssertionError):
+        failed.append("bbit_mean")
     # small unbiasedness sweep: 4096 N(0,1) coordinates, s = 8, 400 seeds
     v = workloads.normal(4096, 1)
     sums = sc.Sums(v.size)
