@@ -489,6 +489,44 @@ def run_ours(args, w):
                       "algorithmic_bytes": f_alg, "algorithmic_gbs": {"encode": f_alg / f_ms / 1e6},
                       "roofline_frac": {"encode": f_alg / f_ms / 1e6 / measured_peaks()[0]}}
 
+    # data-parallel exchange, every rank: encode, all-gather the lengths, headers and
+    # padded streams (NCCL), decode the mean of the N streams; timed per step on the
+    # device, max over ranks.  And the receiver's side of an 8-GPU node on this GPU: the
+    # mean of 8 streams (this rank's stream 8 times), timed alone.
+    from quantized_gradient_compression_b200 import exchange as X
+
+    xch = X.EliasExchange(X.LibraryCodec(n, d, s, dev))
+    xout = torch.empty(n, dtype=torch.float32, device=dev)
+    for k in range(3):
+        xch.step(x, seed + 1000 + k, out=xout)
+    x_ts = []
+    for k in range(max(3, min(K, 20))):
+        flush.zero_()
+        barrier(world)
+        e_a, e_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e_a.record(stream)
+        xch.step(x, seed + 2000 + k, out=xout)
+        e_b.record(stream)
+        torch.cuda.synchronize()
+        x_ts.append(e_a.elapsed_time(e_b))
+    x_ms = max_over_ranks(statistics.median(x_ts), world)
+    if int(xch.codec.status.item()) != 0:
+        raise RuntimeError("device status %d in the exchange" % int(xch.codec.status.item()))
+    R = 8
+    xw, xo = xch.codec.words, xch.codec.offsets
+
+    def r_mean():
+        check(B.qsgd_decode_mean([xw.data_ptr()] * R, [xw.numel()] * R, [xo.data_ptr()] * R, R, n, d, s,
+                                 xout.data_ptr(), status.data_ptr(), sh), "qsgd_decode_mean")
+
+    r_ms = time_alone(r_mean)
+    r_comp = 4 * ((int(xo[-1].item()) + 31) // 32) + 8 * (nb + 1)
+    exchange = {"ranks": world, "collective": "all_gather_into_tensor x3 (%s)" % (
+                    "nccl" if world > 1 else "nccl, one rank" if torch.distributed.is_initialized() else "none"),
+                "ms_per_step": x_ms, "sent_bytes_per_rank": xch.last.sent_bytes,
+                "receiver_mean_of_8": {"us": 1e3 * r_ms, "algorithmic_bytes": R * r_comp + 4.0 * n,
+                                       "roofline_frac": (R * r_comp + 4.0 * n) / r_ms / 1e6 / measured_peaks()[0]}}
+
     peak, peak_kind = measured_peaks()
     in_bytes = 4.0 * n
     enc_bytes = in_bytes + comp_bytes            # read fp32, write stream + header
@@ -543,6 +581,7 @@ def run_ours(args, w):
         "bbit": bbit,
         "qsgdinf": qsgdinf,
         "error_feedback": error_feedback,
+        "exchange": exchange,
         "clocks": clocks.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -174,6 +174,18 @@ QSGD_API int qsgd_decode_accumulate(const uint32_t* const* h_words, const uint64
                            const uint64_t* const* h_offsets, int K, uint64_t n, uint32_t d,
                            uint32_t s, float* d_out, uint32_t* d_status, cudaStream_t stream);
 
+/* The mean of K received streams, the update of a node in data-parallel training (the
+ * definition paragraph places QSGD in distributed data-parallel optimisation).
+ *   d_out[i] = (q^0[i] + q^1[i] + ... + q^{K-1}[i]) / K
+ * The sum runs left to right from +0, in fp32, as in qsgd_decode_accumulate; then one
+ * IEEE division by K per coordinate.  d_out is overwritten, not accumulated.  The
+ * arguments and the status are those of qsgd_decode_accumulate (1 <= K <= 1024, host
+ * arrays of device pointers).  Every stream is checked before the first launch.  The
+ * work is K decode launches and one division pass. */
+QSGD_API int qsgd_decode_mean(const uint32_t* const* h_words, const uint64_t* h_num_words,
+                              const uint64_t* const* h_offsets, int K, uint64_t n, uint32_t d,
+                              uint32_t s, float* d_out, uint32_t* d_status, cudaStream_t stream);
+
 /* Encoder for callers that cannot allocate device memory.  (The paper has no
  * counterpart: this is a deployment variant of qsgd_encode.)
  *
@@ -256,6 +268,12 @@ QSGD_API int qsgd_bbit_decode(const float* d_norms, const uint32_t* d_codes, uin
 QSGD_API int qsgd_bbit_decode_accumulate(const float* const* h_norms, const uint32_t* const* h_codes, int K,
                                          uint64_t n, uint32_t d, uint32_t b, float* d_out, uint32_t* d_status,
                                          cudaStream_t stream);
+
+/* The mean of K b-bit streams: d_out[i] = (q^0[i] + ... + q^{K-1}[i]) / K, with the
+ * order, rounding and arguments of qsgd_decode_mean. */
+QSGD_API int qsgd_bbit_decode_mean(const float* const* h_norms, const uint32_t* const* h_codes, int K,
+                                   uint64_t n, uint32_t d, uint32_t b, float* d_out, uint32_t* d_status,
+                                   cudaStream_t stream);
 
 /* Static description of a host return code. */
 QSGD_API const char* qsgd_error_string(int code);

@@ -54,6 +54,8 @@ _SIGS = {
     "qsgd_decode": (_int, [_vp, _u64, _vp, _u64, _u32, _u32, _vp, _vp, _vp]),
     "qsgd_decode_accumulate": (_int, [ctypes.POINTER(_vp), ctypes.POINTER(_u64), ctypes.POINTER(_vp),
                                       _int, _u64, _u32, _u32, _vp, _vp, _vp]),
+    "qsgd_decode_mean": (_int, [ctypes.POINTER(_vp), ctypes.POINTER(_u64), ctypes.POINTER(_vp),
+                                _int, _u64, _u32, _u32, _vp, _vp, _vp]),
     "qsgd_encode_static_ws": (_int, [_vp, _u64, _u32, _u32, _u64, _vp, _u64, _vp, _vp, _vp]),
     "qsgd_static_workspace_limit": (_sz, []),
     "qsgd_bbit_code_words": (_u64, [_u64, _u32]),
@@ -63,6 +65,8 @@ _SIGS = {
     "qsgd_bbit_decode": (_int, [_vp, _vp, _u64, _u32, _u32, _vp, _vp, _vp]),
     "qsgd_bbit_decode_accumulate": (_int, [ctypes.POINTER(_vp), ctypes.POINTER(_vp), _int, _u64, _u32, _u32,
                                            _vp, _vp, _vp]),
+    "qsgd_bbit_decode_mean": (_int, [ctypes.POINTER(_vp), ctypes.POINTER(_vp), _int, _u64, _u32, _u32,
+                                     _vp, _vp, _vp]),
     "qsgd_error_string": (ctypes.c_char_p, [_int]),
     "qsgd_version": (ctypes.c_char_p, []),
 }
@@ -135,6 +139,14 @@ def qsgd_decode_accumulate(h_words, h_num_words, h_offsets, K: int, n: int, d: i
     return int(_lib.qsgd_decode_accumulate(w, nw, o, K, n, d, s, d_out, d_status, stream))
 
 
+def qsgd_decode_mean(h_words, h_num_words, h_offsets, K: int, n: int, d: int, s: int,
+                     d_out: int, d_status: int, stream: int) -> int:
+    w = (_vp * K)(*h_words)
+    nw = (_u64 * K)(*h_num_words)
+    o = (_vp * K)(*h_offsets)
+    return int(_lib.qsgd_decode_mean(w, nw, o, K, n, d, s, d_out, d_status, stream))
+
+
 def qsgd_encode_static_ws(d_in: int, n: int, d: int, s: int, seed: int, d_words: int, words_capacity: int,
                           d_offsets: int, d_status: int, stream: int) -> int:
     """qsgd_encode without a caller workspace (for callers that cannot allocate)."""
@@ -177,6 +189,13 @@ def qsgd_bbit_decode_accumulate(h_norms, h_codes, K: int, n: int, d: int, b: int
     nn = (_vp * K)(*h_norms)
     cc = (_vp * K)(*h_codes)
     return int(_lib.qsgd_bbit_decode_accumulate(nn, cc, K, n, d, b, d_out, d_status, stream))
+
+
+def qsgd_bbit_decode_mean(h_norms, h_codes, K: int, n: int, d: int, b: int, d_out: int, d_status: int,
+                          stream: int) -> int:
+    nn = (_vp * K)(*h_norms)
+    cc = (_vp * K)(*h_codes)
+    return int(_lib.qsgd_bbit_decode_mean(nn, cc, K, n, d, b, d_out, d_status, stream))
 
 
 def qsgd_error_string(code: int) -> str:

@@ -253,6 +253,24 @@ int qsgd_decode(const uint32_t* d_words, uint64_t num_words, const uint64_t* d_o
     return decode_impl(w, nw, o, 1, n, d, s, d_out, d_status, stream, false);
 }
 
+int qsgd_decode_mean(const uint32_t* const* h_words, const uint64_t* h_num_words,
+                     const uint64_t* const* h_offsets, int K, uint64_t n, uint32_t d, uint32_t s, float* d_out,
+                     uint32_t* d_status, cudaStream_t stream) {
+    if (!h_words || !h_num_words || !h_offsets || K < 1 || K > 1024) return QSGD_ERR_ARG;
+    if (!valid_params(n, d, s) || !d_status) return QSGD_ERR_ARG;
+    for (int j = 0; j < K; ++j)  // every stream is checked before the first launch
+        if (!h_words[j] || !h_offsets[j] || (reinterpret_cast<uintptr_t>(h_offsets[j]) & 7u) != 0)
+            return QSGD_ERR_ARG;
+    // stream 0 decoded into d_out, the others added in order, then the division
+    int rc = decode_impl(h_words, h_num_words, h_offsets, 1, n, d, s, d_out, d_status, stream, false);
+    if (rc != QSGD_OK || n == 0) return rc;
+    if (K > 1) {
+        rc = decode_impl(h_words + 1, h_num_words + 1, h_offsets + 1, K - 1, n, d, s, d_out, d_status, stream, true);
+        if (rc != QSGD_OK) return rc;
+    }
+    return launch_div(d_out, n, static_cast<uint32_t>(K), stream) == cudaSuccess ? QSGD_OK : QSGD_ERR_CUDA;
+}
+
 int qsgd_decode_accumulate(const uint32_t* const* h_words, const uint64_t* h_num_words,
                            const uint64_t* const* h_offsets, int K, uint64_t n, uint32_t d,
                            uint32_t s, float* d_out, uint32_t* d_status, cudaStream_t stream) {
@@ -331,6 +349,19 @@ int qsgd_bbit_decode_accumulate(const float* const* h_norms, const uint32_t* con
         if (launch_bbit_decode(h_norms[j], h_codes[j], n, d, b, d_out, true, d_status, stream) != cudaSuccess)
             return QSGD_ERR_CUDA;
     return QSGD_OK;
+}
+
+int qsgd_bbit_decode_mean(const float* const* h_norms, const uint32_t* const* h_codes, int K, uint64_t n,
+                          uint32_t d, uint32_t b, float* d_out, uint32_t* d_status, cudaStream_t stream) {
+    if (!valid_bbit(n, d, b) || !d_status || K < 1 || K > 1024 || !h_norms || !h_codes) return QSGD_ERR_ARG;
+    if (n == 0) return QSGD_OK;
+    if (!d_out || (reinterpret_cast<uintptr_t>(d_out) & 3u) != 0) return QSGD_ERR_ARG;
+    for (int j = 0; j < K; ++j)
+        if (!h_norms[j] || !h_codes[j]) return QSGD_ERR_ARG;
+    for (int j = 0; j < K; ++j)
+        if (launch_bbit_decode(h_norms[j], h_codes[j], n, d, b, d_out, j > 0, d_status, stream) != cudaSuccess)
+            return QSGD_ERR_CUDA;
+    return launch_div(d_out, n, static_cast<uint32_t>(K), stream) == cudaSuccess ? QSGD_OK : QSGD_ERR_CUDA;
 }
 
 const char* qsgd_error_string(int code) {

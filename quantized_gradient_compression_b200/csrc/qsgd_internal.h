@@ -104,6 +104,9 @@ cudaError_t launch_bbit_encode(const float* in, float* ef, uint64_t n, uint32_t 
 // Whether launch_bbit_encode fuses error feedback for this shape (else ef must be null).
 bool bbit_fast_shape(const float* in, const float* ef, uint32_t d);
 
+// out[i] <- fl(out[i] / K): the last step of the mean of K streams (qsgd_mean.cu).
+cudaError_t launch_div(float* out, uint64_t n, uint32_t K, cudaStream_t stream);
+
 // Error feedback for the shapes the fused encoders do not take (qsgd_ef.cu):
 // e <- e + g; then, after the encoder has read p from e, the residual passes.
 cudaError_t launch_ef_add(const float* g, float* e, uint64_t n, cudaStream_t stream);

@@ -126,3 +126,17 @@ def test_error_feedback_arguments_checked():
         == B.QSGD_ERR_ARG
     assert B.qsgd_bbit_encode_ef(A + 2, A * 4, 100, 4, 4, 0, 0, A * 8, A * 16, A * 64, 0) == B.QSGD_ERR_ARG
     assert B.qsgd_bbit_encode_ef(A, A * 4, 100, 4, 4, 0, 5, A * 8, A * 16, A * 64, 0) == B.QSGD_ERR_ARG
+
+
+def test_mean_arguments_checked():
+    from quantized_gradient_compression_b200 import binding as B
+
+    A = 1 << 20
+    # K out of range, a null stream among valid ones, a misaligned offsets array:
+    # refused before any launch
+    assert B.qsgd_decode_mean([], [], [], 0, 100, 4, 4, A, A, 0) == B.QSGD_ERR_ARG
+    assert B.qsgd_decode_mean([A, 0], [10, 10], [A * 2, A * 2], 2, 100, 4, 4, A * 4, A * 8, 0) == B.QSGD_ERR_ARG
+    assert B.qsgd_decode_mean([A, A], [10, 10], [A * 2, A * 2 + 4], 2, 100, 4, 4, A * 4, A * 8, 0) \
+        == B.QSGD_ERR_ARG
+    assert B.qsgd_bbit_decode_mean([A, 0], [A, A], 2, 100, 4, 4, A * 4, A * 8, 0) == B.QSGD_ERR_ARG
+    assert B.qsgd_bbit_decode_mean([A], [A], 1, 100, 4, 3, A * 4, A * 8, 0) == B.QSGD_ERR_ARG
