@@ -217,7 +217,8 @@ int qsgd_encode(const float* d_in, uint64_t n, uint32_t d, uint32_t s, uint64_t 
 
 static int decode_impl(const uint32_t* const* words, const uint64_t* num_words,
                        const uint64_t* const* offsets, int K, uint64_t n, uint32_t d, uint32_t s,
-                       float* d_out, uint32_t* d_status, cudaStream_t stream, bool accumulate) {
+                       float* d_out, uint32_t* d_status, cudaStream_t stream, bool accumulate,
+                       bool mean = false) {
     if (!valid_params(n, d, s) || !d_status || K < 1 || K > 1024) return QSGD_ERR_ARG;
     if (n == 0) return QSGD_OK;
     if (!d_out || !words || !num_words || !offsets) return QSGD_ERR_ARG;
@@ -234,6 +235,8 @@ static int decode_impl(const uint32_t* const* words, const uint64_t* num_words,
     for (int j0 = 0; j0 < K; j0 += kMaxStreamsPerLaunch) {
         a.K = std::min(K - j0, kMaxStreamsPerLaunch);
         a.first_group = j0 == 0;
+        a.start_zero = mean && j0 == 0;  // the mean: the sum starts from +0 ...
+        a.div = mean && j0 + a.K == K ? static_cast<float>(K) : 0.f;  // ... and is divided at the end
         for (int j = 0; j < a.K; ++j) {
             a.streams[j].words = words[j0 + j];
             a.streams[j].num_words = num_words[j0 + j];
@@ -261,7 +264,10 @@ int qsgd_decode_mean(const uint32_t* const* h_words, const uint64_t* h_num_words
     for (int j = 0; j < K; ++j)  // every stream is checked before the first launch
         if (!h_words[j] || !h_offsets[j] || (reinterpret_cast<uintptr_t>(h_offsets[j]) & 7u) != 0)
             return QSGD_ERR_ARG;
-    // stream 0 decoded into d_out, the others added in order, then the division
+    // the several-stream kernel: sum from +0 in stream order, divided in its last launch
+    if (decode_fast_shape(d, s, d_out))
+        return decode_impl(h_words, h_num_words, h_offsets, K, n, d, s, d_out, d_status, stream, true, true);
+    // other shapes: stream 0 decoded into d_out, the others added in order, then the division
     int rc = decode_impl(h_words, h_num_words, h_offsets, 1, n, d, s, d_out, d_status, stream, false);
     if (rc != QSGD_OK || n == 0) return rc;
     if (K > 1) {

@@ -580,6 +580,155 @@ __global__ void __launch_bounds__(kDecodeBlock) decode_fast(const __grid_constan
 }
 
 // ---------------------------------------------------------------------------
+// Decode-accumulate and mean of several streams in one launch.
+//
+// The one-stream decoder leaves about ten warps on an SM, each one chain of
+// dependent table lookups, so K streams decoded one launch after another wait K
+// times on that latency and move the output 2K times.  Here a CTA of kMultiWarps
+// warps takes one group of 32 buckets, and warp w decodes stream c * kMultiWarps + w
+// of chunk c into its own staging tile, so the chunk's streams are decoded side by
+// side.  Each stream puts at most one value on a coordinate, so a tile holds q_j
+// (+0 off the support).  After each segment the CTA adds the tiles onto the output
+// in stream order, every coordinate and every stream:
+//   out <- ((out + q_c0) + q_c0+1) + ...
+// which is the decode-accumulate order.  With start_zero the first chunk starts from
+// +0 instead of the output; with div != 0 the last chunk divides the sum by div (the
+// mean of the streams).  The output is read and written once per chunk.
+// ---------------------------------------------------------------------------
+constexpr int kMultiWarps = 8;
+constexpr int kMultiBlock = 32 * kMultiWarps;
+
+__global__ void __launch_bounds__(kMultiBlock) decode_multi(const __grid_constant__ DecodeArgs a) {
+    extern __shared__ __align__(16) uint32_t smem[];
+    uint32_t* lut = smem;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    float* const tiles = reinterpret_cast<float*>(smem + kLut);
+    float* const stage = tiles + warp * 32 * kStride;
+    float* const row = stage + lane * kStride;
+    build_record_lut(lut, a.s, tid, kMultiBlock);
+    __syncthreads();
+    const float fs = __uint2float_rn(a.s);
+    const uint32_t d = a.d;
+    const uint64_t ngroups = (a.nb + 31) / 32;
+    for (uint64_t g = blockIdx.x; g < ngroups; g += gridDim.x) {
+        const uint64_t b = g * 32 + lane;
+        const bool live = b < a.nb;
+        const uint32_t m = live ? static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - b * d)) : 0u;
+        for (int c0 = 0; c0 < a.K; c0 += kMultiWarps) {
+            const int nt = min(kMultiWarps, a.K - c0);  // streams in this chunk
+            const bool mine = warp < nt;                // uniform in the warp
+            const bool last_chunk = c0 + nt == a.K;
+            // --- open this lane's bucket of stream c0 + warp --------------------
+            bool bad = false;
+            BitBuf r;
+            r.left = 0;
+            float scale = 0.f;
+            if (mine && live) {
+                const StreamRef st = a.streams[c0 + warp];
+                const uint64_t begin = st.offsets[b];
+                const uint64_t end = st.offsets[b + 1];
+                if (!(end >= begin && end - begin >= 32 && end <= st.num_words * 32 && end - begin < (1ull << 30))) {
+                    bad = true;
+                } else {
+                    r.init(st.words, st.num_words, begin, static_cast<uint32_t>(end - begin));
+                    const uint32_t nbits = r.top(32);
+                    r.consume(32);
+                    const float norm = __uint_as_float(nbits);
+                    if (nbits == 0) {
+                        bad = r.left != 0;
+                        r.left = 0;
+                    } else if (!(isfinite(norm) && norm > 0.f)) {
+                        bad = true;
+                        r.left = 0;
+                    } else {
+                        scale = __fdiv_rn(norm, fs);
+                        if (!(scale > 0.f) && r.left != 0) {  // a zero scale carries no records
+                            bad = true;
+                            r.left = 0;
+                        }
+                    }
+                }
+            }
+            uint32_t next = 0, pidx = kNoRecord, pval = 0;
+            if (mine && !bad) table_next(r, lut, scale, next, pidx, pval);
+            for (uint32_t lo = 0; lo < d; lo += kSeg) {
+                if (mine) {
+                    // --- this stream's values of the segment into a zeroed tile ----
+                    for (int q = lane; q < 32 * kStride / 4; q += 32)
+                        reinterpret_cast<float4*>(stage)[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    __syncwarp();
+                    const uint32_t hi = lo + kSeg;
+                    for (uint32_t it = 0;; ++it) {
+                        const bool place = pidx < hi;
+                        if (it == kLoopGuard) {
+                            bad = true;
+                            pidx = kNoRecord;
+                        }
+                        if (__any_sync(kFullMask, place) && it < kLoopGuard) {
+                            if (place) {
+                                row[pidx - lo] = __uint_as_float(pval);
+                                table_next(r, lut, scale, next, pidx, pval);
+                            }
+                        } else if (__any_sync(kFullMask, pidx == kParked)) {
+                            if (pidx == kParked && !slow_next(r, a.s, scale, next, pidx, pval)) {
+                                bad = true;
+                                pidx = kNoRecord;
+                            }
+                        } else {
+                            break;
+                        }
+                    }
+                }
+                __syncthreads();  // every tile of the chunk holds its segment
+                // --- the CTA adds the tiles onto the output in stream order ------
+                for (int q = tid; q < 32 * (kSeg / 4); q += kMultiBlock) {
+                    const uint32_t rr = static_cast<uint32_t>(q) / (kSeg / 4);
+                    const uint32_t cc = (static_cast<uint32_t>(q) % (kSeg / 4)) * 4;
+                    const uint64_t bb = g * 32 + rr;
+                    const uint32_t mm = bb < a.nb ? static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - bb * d)) : 0u;
+                    const uint32_t c = lo + cc;
+                    if (c >= mm) continue;
+                    float* gp = a.out + bb * d + c;
+                    const bool whole = c + 4 <= mm;
+                    float v[4] = {0.f, 0.f, 0.f, 0.f};
+                    if (!(a.start_zero && c0 == 0)) {
+                        if (whole) {
+                            const float4 o = *reinterpret_cast<const float4*>(gp);
+                            v[0] = o.x;
+                            v[1] = o.y;
+                            v[2] = o.z;
+                            v[3] = o.w;
+                        } else {
+                            for (uint32_t e = 0; c + e < mm; ++e) v[e] = gp[e];
+                        }
+                    }
+                    for (int t = 0; t < nt; ++t) {
+                        const float4 w = *reinterpret_cast<const float4*>(tiles + (t * 32 + rr) * kStride + cc);
+                        v[0] = __fadd_rn(v[0], w.x);
+                        v[1] = __fadd_rn(v[1], w.y);
+                        v[2] = __fadd_rn(v[2], w.z);
+                        v[3] = __fadd_rn(v[3], w.w);
+                    }
+                    if (last_chunk && a.div != 0.f) {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) v[e] = __fdiv_rn(v[e], a.div);
+                    }
+                    if (whole) {
+                        *reinterpret_cast<float4*>(gp) = make_float4(v[0], v[1], v[2], v[3]);
+                    } else {
+                        for (uint32_t e = 0; c + e < mm; ++e) gp[e] = v[e];
+                    }
+                }
+                __syncthreads();  // the tiles are free for the next segment
+            }
+            // every record index below m, and the bucket consumed exactly
+            if (mine && live && !bad && (next > m || r.left != 0 || pidx != kNoRecord)) bad = true;
+            if (mine && bad) atomicOr(a.status, QSGD_ST_BAD_STREAM);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Split decoder: P lanes per bucket (one stream; the fast decoder's conditions).
 //
 // One lane per bucket leaves a B200 with a few hundred latency-bound chains of
@@ -948,6 +1097,25 @@ cudaError_t launch_fast_decode(const DecodeArgs& a, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
+cudaError_t launch_multi(const DecodeArgs& a, cudaStream_t stream) {
+    const size_t smem = kLut * sizeof(uint32_t) + static_cast<size_t>(kMultiWarps) * 32 * kStride * sizeof(float);
+    static bool attr_set[64] = {};
+    int dev = 0, sms = 0, per_sm = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr_set[dev]) {
+        cudaFuncSetAttribute(decode_multi, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+        attr_set[dev] = true;
+    }
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_multi, kMultiBlock, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    const uint64_t groups = (a.nb + 31) / 32;
+    const uint64_t blocks = std::min<uint64_t>(groups, static_cast<uint64_t>(sms) * per_sm);
+    decode_multi<<<static_cast<unsigned>(blocks), kMultiBlock, smem, stream>>>(a);
+    return cudaGetLastError();
+}
+
 template <bool kAccumulate>
 cudaError_t launch(const DecodeArgs& a, cudaStream_t stream) {
     const size_t smem = kLut * sizeof(uint32_t) + static_cast<size_t>(kDecWarps) * 32 * kStride * sizeof(float) +
@@ -973,11 +1141,20 @@ cudaError_t launch(const DecodeArgs& a, cudaStream_t stream) {
 
 }  // namespace
 
+bool decode_fast_shape(uint32_t d, uint32_t s, const float* out) {
+    return d % 4 == 0 && d <= kFastDecodeMaxD && s < 1024 && (reinterpret_cast<uintptr_t>(out) & 15u) == 0;
+}
+
 cudaError_t launch_decode(const DecodeArgs& a, bool accumulate, cudaStream_t stream) {
     if (a.nb == 0) return cudaSuccess;
-    const bool fast = a.d % 4 == 0 && a.d <= kFastDecodeMaxD && a.s < 1024 &&
-                      (reinterpret_cast<uintptr_t>(a.out) & 15u) == 0;
+    const bool fast = decode_fast_shape(a.d, a.s, a.out);
+    if (a.start_zero || a.div != 0.f) return fast ? launch_multi(a, stream) : cudaErrorInvalidValue;
     if (!fast) return accumulate ? launch<true>(a, stream) : launch<false>(a, stream);
+#ifndef QSGD_MULTI
+#define QSGD_MULTI 1
+#endif
+    // several streams: decoded side by side, the output moved once
+    if (QSGD_MULTI && accumulate && a.K >= 2) return launch_multi(a, stream);
 #ifndef QSGD_SPLIT_MODE
 #define QSGD_SPLIT_MODE 0
 #endif

@@ -93,9 +93,14 @@ struct DecodeArgs {
     float* out;
     uint32_t* status;
     int first_group;  // decode-accumulate: this launch holds stream 0
+    int start_zero;   // several-stream kernel: the sum starts from +0, not from out
+    float div;        // several-stream kernel: divide the finished sum by div (0: no)
 };
 
 cudaError_t launch_decode(const DecodeArgs& a, bool accumulate, cudaStream_t stream);
+// Whether the one-lane-per-bucket decoders (and the several-stream kernel, which
+// start_zero / div need) take this shape.
+bool decode_fast_shape(uint32_t d, uint32_t s, const float* out);
 
 // Fixed-width b-bit variant (b in {2, 4, 8}, checked by the caller).
 cudaError_t launch_bbit_encode(const float* in, float* ef, uint64_t n, uint32_t d, uint32_t b, uint64_t seed,

@@ -1,9 +1,11 @@
-// Runs the decoder kernels decode_fast (P = 0) and decode_split (P >= 1), compiled
-// for the host under warp_emu.h,
-// over streams read from files.  argv: dir P accumulate [grid]
+// Runs the decoder kernels decode_fast (P = 0), decode_split (P >= 1) and
+// decode_multi (P = -1), compiled for the host under warp_emu.h, over streams read
+// from files.  argv: dir P accumulate [grid [mean]]
 // dir holds params.bin (u64 n, d, s, K), out_in.bin (fp32[n]), w<j>.bin / o<j>.bin
 // (words, offsets of stream j); the result goes to out.bin and the status to stdout.
-// K streams are decoded one launch each, in order, as the library does.
+// For P >= 0 the K streams are decoded one launch each, in order.  For P = -1 they
+// go 16 to a launch, as the library sends them to decode_multi; with mean = 1 the
+// first launch starts from +0 and the last divides by K.
 #include "warp_emu.h"
 thread_local dim3e threadIdx, blockIdx;
 dim3e gridDim, blockDim;
@@ -63,6 +65,28 @@ template <bool A, int P> void run_kernel(const qsgd::DecodeArgs& a, unsigned gri
         for (auto& x : th) x.join();
     }
 }
+static void run_multi(const qsgd::DecodeArgs& a, unsigned grid) {
+    const int kBlock = qsgd::kMultiBlock;
+    const size_t smem = qsgd::kLut * 4 + (size_t)qsgd::kMultiWarps * 32 * qsgd::kStride * 4;
+    gridDim = {grid, 1, 1};
+    blockDim = {(unsigned)kBlock, 1, 1};
+    std::vector<unsigned char> sm(smem + 64);
+    std::vector<WarpSync> warps(kBlock / 32);
+    for (unsigned b = 0; b < grid; ++b) {
+        g_emu_smem = sm.data();
+        std::memset(sm.data(), 0xAB, sm.size());
+        g_warps = warps.data();
+        std::vector<std::thread> th;
+        for (int t = 0; t < kBlock; ++t)
+            th.emplace_back([&, t, b] {
+                threadIdx = {(unsigned)t, 0, 0};
+                blockIdx = {b, 0, 0};
+                qsgd::decode_multi(a);
+            });
+        for (auto& x : th) x.join();
+    }
+}
+
 int main(int argc, char** argv) {
     const std::string dir = argv[1];
     const int P = std::atoi(argv[2]);
@@ -79,6 +103,33 @@ int main(int argc, char** argv) {
     std::memcpy(out.data(), outb.data(), 4 * n);
     uint32_t status = 0;
     std::vector<std::vector<unsigned char>> ws(K), os(K);
+    if (P < 0) {
+        const bool mean = argc > 5 && std::atoi(argv[5]) != 0;
+        for (int j = 0; j < K; ++j) {
+            ws[j] = slurp(dir + "/w" + std::to_string(j) + ".bin");
+            os[j] = slurp(dir + "/o" + std::to_string(j) + ".bin");
+        }
+        for (int j0 = 0; j0 < K; j0 += qsgd::kMaxStreamsPerLaunch) {
+            qsgd::DecodeArgs a{};
+            a.n = n; a.d = d; a.s = s; a.nb = (n + d - 1) / d; a.out = out.data(); a.status = &status;
+            a.K = std::min(K - j0, qsgd::kMaxStreamsPerLaunch);
+            a.first_group = j0 == 0;
+            a.start_zero = mean && j0 == 0;
+            a.div = mean && j0 + a.K == K ? (float)K : 0.f;
+            for (int j = 0; j < a.K; ++j) {
+                a.streams[j].words = reinterpret_cast<const uint32_t*>(ws[j0 + j].data());
+                a.streams[j].num_words = ws[j0 + j].size() / 4;
+                a.streams[j].offsets = reinterpret_cast<const uint64_t*>(os[j0 + j].data());
+            }
+            run_multi(a, grid);
+            if (g_emu_error) return 4;
+        }
+        FILE* f = std::fopen((dir + "/out.bin").c_str(), "wb");
+        std::fwrite(out.data(), 4, n, f);
+        std::fclose(f);
+        std::printf("status %u\n", status);
+        return 0;
+    }
     for (int j = 0; j < K; ++j) {
         ws[j] = slurp(dir + "/w" + std::to_string(j) + ".bin");
         os[j] = slurp(dir + "/o" + std::to_string(j) + ".bin");

@@ -69,7 +69,7 @@ def _flip_bits(words, offsets, rng):
                 words[pos >> 5] ^= np.uint32(1) << np.uint32(31 - (pos & 31))
 
 
-def _run(exe, tmp, oracle_lib, n, d, s, K, P, accumulate, kind, corrupt=False):
+def _run(exe, tmp, oracle_lib, n, d, s, K, P, accumulate, kind, corrupt=False, mean=False):
     streams = []
     for j in range(K):
         v = W.GENERATORS[kind](n, 300 + j)
@@ -86,7 +86,7 @@ def _run(exe, tmp, oracle_lib, n, d, s, K, P, accumulate, kind, corrupt=False):
         base[:] = np.float32(np.nan)  # every coordinate must be written
     base.tofile(tmp / "out_in.bin")
     np.array([n, d, s, K], np.uint64).tofile(tmp / "params.bin")
-    r = subprocess.run([exe, str(tmp), str(P), "1" if accumulate else "0", "3"],
+    r = subprocess.run([exe, str(tmp), str(P), "1" if accumulate else "0", "3", "1" if mean else "0"],
                        capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, (r.stdout[-500:], r.stderr[-2000:])
     status = int(r.stdout.split()[-1])
@@ -149,5 +149,56 @@ def test_split_decoder_corrupt_streams(emu_exe, tmp_path, oracle_lib, d, P):
         w0, w1 = int(offs[b]) >> 5, (int(offs[b + 1]) + 31) >> 5
         if flipped[w0:w1].any():
             keep[b * d:min(n, (b + 1) * d)] = False
+    assert keep.any()
+    assert np.array_equal(got[keep].view(np.uint32), ref[keep].view(np.uint32))
+
+
+# decode_multi (P = -1): K streams side by side in one launch (16 to a launch), for
+# decode-accumulate and for the mean; ragged tails, d % 64 != 0, K past one chunk of
+# eight warps and past one launch
+MULTI = [
+    (20_000, 512, 16, 3, True, False, "layered"),
+    (20_000, 512, 16, 8, True, False, "normal"),
+    (9_001, 100, 7, 11, True, False, "normal"),
+    (5_000, 132, 3, 17, True, False, "normal"),
+    (20_000, 512, 16, 5, False, True, "layered"),
+    (7_000, 100, 7, 18, False, True, "normal"),
+    (4_000, 512, 16, 1, False, True, "normal"),
+]
+
+
+@pytest.mark.parametrize("n,d,s,K,accumulate,mean,kind", MULTI, ids=["n%d-d%d-s%d-K%d-acc%d-mean%d-%s" % c for c in MULTI])
+def test_multi_stream_kernel_matches_oracle(emu_exe, tmp_path, oracle_lib, n, d, s, K, accumulate, mean, kind):
+    got, status, streams, base = _run(emu_exe, tmp_path, oracle_lib, n, d, s, K, -1, accumulate, kind, mean=mean)
+    assert status == 0
+    if mean:
+        ref, rst = oracle_lib.decode_mean(streams, n, d, s)
+    else:
+        ref = base.copy()
+        _, rst = oracle_lib.decode_accumulate(streams, n, d, s, ref)
+    assert rst == 0
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+
+
+def test_multi_stream_kernel_corrupt_stream(emu_exe, tmp_path, oracle_lib):
+    """Bit flips in stream 1 of 3: the kernel finishes, flags the input, and every
+    bucket that no flip touched equals the oracle's sum."""
+    n, d, s = 20_000, 512, 16
+    got, status, streams, base = _run(emu_exe, tmp_path, oracle_lib, n, d, s, 3, -1, True, "normal", corrupt=True)
+    assert status & 2
+    intact = []
+    for j in range(3):
+        words, offsets, _, _ = oracle_lib.encode(W.GENERATORS["normal"](n, 300 + j), d, s, seed=77 + j)
+        intact.append((words, offsets))
+    ref = base.copy()
+    oracle_lib.decode_accumulate(intact, n, d, s, ref)
+    keep = np.ones(n, dtype=bool)
+    for j in range(3):
+        flipped = streams[j][0] != intact[j][0]
+        offs = intact[j][1]
+        for b in range(offs.size - 1):
+            w0, w1 = int(offs[b]) >> 5, (int(offs[b + 1]) + 31) >> 5
+            if flipped[w0:w1].any():
+                keep[b * d:min(n, (b + 1) * d)] = False
     assert keep.any()
     assert np.array_equal(got[keep].view(np.uint32), ref[keep].view(np.uint32))
