@@ -215,6 +215,11 @@ int qsgd_encode(const float* d_in, uint64_t n, uint32_t d, uint32_t s, uint64_t 
                           d_status, stream);
 }
 
+// Streams from which the several-stream decode kernel beats one launch per stream
+// (measured on B200 at n = 25.6 M, d = 512, s = 16: 2 streams 498 against 267 us,
+// 4 streams 523 against 525 us, 8 streams 563 against 1036 us).
+constexpr int kMultiMinStreams = 4;
+
 static int decode_impl(const uint32_t* const* words, const uint64_t* num_words,
                        const uint64_t* const* offsets, int K, uint64_t n, uint32_t d, uint32_t s,
                        float* d_out, uint32_t* d_status, cudaStream_t stream, bool accumulate,
@@ -242,6 +247,17 @@ static int decode_impl(const uint32_t* const* words, const uint64_t* num_words,
             a.streams[j].num_words = num_words[j0 + j];
             a.streams[j].offsets = offsets[j0 + j];
         }
+        if (accumulate && !mean && a.K > 1 && a.K < kMultiMinStreams) {
+            // a few streams: one launch each, in order
+            DecodeArgs o = a;
+            o.K = 1;
+            for (int j = 0; j < a.K; ++j) {
+                o.streams[0] = a.streams[j];
+                o.first_group = a.first_group && j == 0;
+                if (launch_decode(o, true, stream) != cudaSuccess) return QSGD_ERR_CUDA;
+            }
+            continue;
+        }
         const cudaError_t e = launch_decode(a, accumulate, stream);
         if (e != cudaSuccess) return QSGD_ERR_CUDA;
     }
@@ -265,9 +281,10 @@ int qsgd_decode_mean(const uint32_t* const* h_words, const uint64_t* h_num_words
         if (!h_words[j] || !h_offsets[j] || (reinterpret_cast<uintptr_t>(h_offsets[j]) & 7u) != 0)
             return QSGD_ERR_ARG;
     // the several-stream kernel: sum from +0 in stream order, divided in its last launch
-    if (decode_fast_shape(d, s, d_out))
+    if (decode_fast_shape(d, s, d_out) && K >= kMultiMinStreams)
         return decode_impl(h_words, h_num_words, h_offsets, K, n, d, s, d_out, d_status, stream, true, true);
-    // other shapes: stream 0 decoded into d_out, the others added in order, then the division
+    // other shapes and a few streams: stream 0 decoded into d_out, the others added in
+    // order, then the division
     int rc = decode_impl(h_words, h_num_words, h_offsets, 1, n, d, s, d_out, d_status, stream, false);
     if (rc != QSGD_OK || n == 0) return rc;
     if (K > 1) {
