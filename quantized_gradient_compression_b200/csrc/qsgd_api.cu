@@ -216,9 +216,10 @@ int qsgd_encode(const float* d_in, uint64_t n, uint32_t d, uint32_t s, uint64_t 
 }
 
 // Streams from which the several-stream decode kernel beats one launch per stream
-// (measured on B200 at n = 25.6 M, d = 512, s = 16: 2 streams 498 against 267 us,
-// 4 streams 523 against 525 us, 8 streams 563 against 1036 us).
-constexpr int kMultiMinStreams = 4;
+// (measured on B200 at n = 25.6 M, d = 512, s = 16: 2 streams 173 against 263 us,
+// 4 streams 269 against 525 us, 8 streams 451 against 1036 us; one stream 209
+// against 133 us, so one stream stays on the one-stream kernel).
+constexpr int kMultiMinStreams = 2;
 
 static int decode_impl(const uint32_t* const* words, const uint64_t* num_words,
                        const uint64_t* const* offsets, int K, uint64_t n, uint32_t d, uint32_t s,

@@ -584,47 +584,56 @@ __global__ void __launch_bounds__(kDecodeBlock) decode_fast(const __grid_constan
 //
 // The one-stream decoder leaves about ten warps on an SM, each one chain of
 // dependent table lookups, so K streams decoded one launch after another wait K
-// times on that latency and move the output 2K times.  Here a CTA of kMultiWarps
-// warps takes one group of 32 buckets, and warp w decodes stream c * kMultiWarps + w
-// of chunk c into its own staging tile, so the chunk's streams are decoded side by
-// side.  Each stream puts at most one value on a coordinate, so a tile holds q_j
-// (+0 off the support).  After each segment the CTA adds the tiles onto the output
-// in stream order, every coordinate and every stream:
-//   out <- ((out + q_c0) + q_c0+1) + ...
+// times on that latency and move the output 2K times.  Here the kMultiWarps warps of
+// a CTA decode side by side: with W = min(K, kMultiWarps) streams to a chunk, the CTA
+// takes G = kMultiWarps / W groups of 32 buckets at once, and warp w decodes stream
+// c * W + (w mod W) of chunk c for group w div W into its own staging tile.  Each
+// stream puts at most one value on a coordinate, so a tile holds q_j (+0 off the
+// support).  After each segment the CTA adds a group's tiles onto the output in
+// stream order, every coordinate and every stream:
+//   out <- ((out + q_cW) + q_cW+1) + ...
 // which is the decode-accumulate order.  With start_zero the first chunk starts from
 // +0 instead of the output; with div != 0 the last chunk divides the sum by div (the
-// mean of the streams).  The output is read and written once per chunk.
+// mean of the streams).  The output is read and written once per chunk.  Segments
+// are 32 columns wide, so that four CTAs fit on an SM.
 // ---------------------------------------------------------------------------
 constexpr int kMultiWarps = 8;
 constexpr int kMultiBlock = 32 * kMultiWarps;
+constexpr int kMSeg = 32;              // coordinates per bucket per staging round
+constexpr int kMStride = kMSeg + 4;    // padded row (floats) of a staging tile
 
 __global__ void __launch_bounds__(kMultiBlock) decode_multi(const __grid_constant__ DecodeArgs a) {
     extern __shared__ __align__(16) uint32_t smem[];
     uint32_t* lut = smem;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     float* const tiles = reinterpret_cast<float*>(smem + kLut);
-    float* const stage = tiles + warp * 32 * kStride;
-    float* const row = stage + lane * kStride;
+    float* const stage = tiles + warp * 32 * kMStride;
+    float* const row = stage + lane * kMStride;
     build_record_lut(lut, a.s, tid, kMultiBlock);
     __syncthreads();
     const float fs = __uint2float_rn(a.s);
     const uint32_t d = a.d;
     const uint64_t ngroups = (a.nb + 31) / 32;
-    for (uint64_t g = blockIdx.x; g < ngroups; g += gridDim.x) {
+    const int W = min(a.K, kMultiWarps);  // streams to a chunk
+    const int G = kMultiWarps / W;        // groups a CTA takes at once
+    const int gi = warp / W;              // this warp's group of the G (G when idle)
+    const int wj = warp - gi * W;         // this warp's stream within a chunk
+    for (uint64_t g0 = static_cast<uint64_t>(blockIdx.x) * G; g0 < ngroups; g0 += static_cast<uint64_t>(gridDim.x) * G) {
+        const uint64_t g = g0 + gi;
         const uint64_t b = g * 32 + lane;
-        const bool live = b < a.nb;
+        const bool live = gi < G && b < a.nb;
         const uint32_t m = live ? static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - b * d)) : 0u;
-        for (int c0 = 0; c0 < a.K; c0 += kMultiWarps) {
-            const int nt = min(kMultiWarps, a.K - c0);  // streams in this chunk
-            const bool mine = warp < nt;                // uniform in the warp
+        for (int c0 = 0; c0 < a.K; c0 += W) {
+            const int nt = min(W, a.K - c0);              // streams in this chunk
+            const bool mine = gi < G && g < ngroups && wj < nt;  // uniform in the warp
             const bool last_chunk = c0 + nt == a.K;
-            // --- open this lane's bucket of stream c0 + warp --------------------
+            // --- open this lane's bucket of stream c0 + wj ----------------------
             bool bad = false;
             BitBuf r;
             r.left = 0;
             float scale = 0.f;
             if (mine && live) {
-                const StreamRef st = a.streams[c0 + warp];
+                const StreamRef st = a.streams[c0 + wj];
                 const uint64_t begin = st.offsets[b];
                 const uint64_t end = st.offsets[b + 1];
                 if (!(end >= begin && end - begin >= 32 && end <= st.num_words * 32 && end - begin < (1ull << 30))) {
@@ -651,13 +660,13 @@ __global__ void __launch_bounds__(kMultiBlock) decode_multi(const __grid_constan
             }
             uint32_t next = 0, pidx = kNoRecord, pval = 0;
             if (mine && !bad) table_next(r, lut, scale, next, pidx, pval);
-            for (uint32_t lo = 0; lo < d; lo += kSeg) {
+            for (uint32_t lo = 0; lo < d; lo += kMSeg) {
                 if (mine) {
                     // --- this stream's values of the segment into a zeroed tile ----
-                    for (int q = lane; q < 32 * kStride / 4; q += 32)
+                    for (int q = lane; q < 32 * kMStride / 4; q += 32)
                         reinterpret_cast<float4*>(stage)[q] = make_float4(0.f, 0.f, 0.f, 0.f);
                     __syncwarp();
-                    const uint32_t hi = lo + kSeg;
+                    const uint32_t hi = lo + kMSeg;
                     for (uint32_t it = 0;; ++it) {
                         const bool place = pidx < hi;
                         if (it == kLoopGuard) {
@@ -680,11 +689,13 @@ __global__ void __launch_bounds__(kMultiBlock) decode_multi(const __grid_constan
                     }
                 }
                 __syncthreads();  // every tile of the chunk holds its segment
-                // --- the CTA adds the tiles onto the output in stream order ------
-                for (int q = tid; q < 32 * (kSeg / 4); q += kMultiBlock) {
-                    const uint32_t rr = static_cast<uint32_t>(q) / (kSeg / 4);
-                    const uint32_t cc = (static_cast<uint32_t>(q) % (kSeg / 4)) * 4;
-                    const uint64_t bb = g * 32 + rr;
+                // --- the CTA adds each group's tiles onto the output in stream order
+                for (int q = tid; q < G * 32 * (kMSeg / 4); q += kMultiBlock) {
+                    const int qg = q / (32 * (kMSeg / 4));
+                    const int qr = q - qg * (32 * (kMSeg / 4));
+                    const uint32_t rr = static_cast<uint32_t>(qr) / (kMSeg / 4);
+                    const uint32_t cc = (static_cast<uint32_t>(qr) % (kMSeg / 4)) * 4;
+                    const uint64_t bb = (g0 + qg) * 32 + rr;
                     const uint32_t mm = bb < a.nb ? static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - bb * d)) : 0u;
                     const uint32_t c = lo + cc;
                     if (c >= mm) continue;
@@ -698,12 +709,14 @@ __global__ void __launch_bounds__(kMultiBlock) decode_multi(const __grid_constan
                             v[1] = o.y;
                             v[2] = o.z;
                             v[3] = o.w;
-                        } else {
-                            for (uint32_t e = 0; c + e < mm; ++e) v[e] = gp[e];
+                        } else {  // c < mm <= c + 3
+                            v[0] = gp[0];
+                            if (c + 1 < mm) v[1] = gp[1];
+                            if (c + 2 < mm) v[2] = gp[2];
                         }
                     }
                     for (int t = 0; t < nt; ++t) {
-                        const float4 w = *reinterpret_cast<const float4*>(tiles + (t * 32 + rr) * kStride + cc);
+                        const float4 w = *reinterpret_cast<const float4*>(tiles + ((qg * W + t) * 32 + rr) * kMStride + cc);
                         v[0] = __fadd_rn(v[0], w.x);
                         v[1] = __fadd_rn(v[1], w.y);
                         v[2] = __fadd_rn(v[2], w.z);
@@ -716,7 +729,9 @@ __global__ void __launch_bounds__(kMultiBlock) decode_multi(const __grid_constan
                     if (whole) {
                         *reinterpret_cast<float4*>(gp) = make_float4(v[0], v[1], v[2], v[3]);
                     } else {
-                        for (uint32_t e = 0; c + e < mm; ++e) gp[e] = v[e];
+                        gp[0] = v[0];
+                        if (c + 1 < mm) gp[1] = v[1];
+                        if (c + 2 < mm) gp[2] = v[2];
                     }
                 }
                 __syncthreads();  // the tiles are free for the next segment
@@ -1098,7 +1113,7 @@ cudaError_t launch_fast_decode(const DecodeArgs& a, cudaStream_t stream) {
 }
 
 cudaError_t launch_multi(const DecodeArgs& a, cudaStream_t stream) {
-    const size_t smem = kLut * sizeof(uint32_t) + static_cast<size_t>(kMultiWarps) * 32 * kStride * sizeof(float);
+    const size_t smem = kLut * sizeof(uint32_t) + static_cast<size_t>(kMultiWarps) * 32 * kMStride * sizeof(float);
     static bool attr_set[64] = {};
     int dev = 0, sms = 0, per_sm = 0;
     cudaGetDevice(&dev);
@@ -1110,8 +1125,9 @@ cudaError_t launch_multi(const DecodeArgs& a, cudaStream_t stream) {
     cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_multi, kMultiBlock, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
-    const uint64_t groups = (a.nb + 31) / 32;
-    const uint64_t blocks = std::min<uint64_t>(groups, static_cast<uint64_t>(sms) * per_sm);
+    const uint64_t G = static_cast<uint64_t>(kMultiWarps / std::min(a.K, kMultiWarps));  // groups a CTA takes at once
+    const uint64_t sets = ((a.nb + 31) / 32 + G - 1) / G;
+    const uint64_t blocks = std::min<uint64_t>(sets, static_cast<uint64_t>(sms) * per_sm);
     decode_multi<<<static_cast<unsigned>(blocks), kMultiBlock, smem, stream>>>(a);
     return cudaGetLastError();
 }

@@ -67,7 +67,7 @@ template <bool A, int P> void run_kernel(const qsgd::DecodeArgs& a, unsigned gri
 }
 static void run_multi(const qsgd::DecodeArgs& a, unsigned grid) {
     const int kBlock = qsgd::kMultiBlock;
-    const size_t smem = qsgd::kLut * 4 + (size_t)qsgd::kMultiWarps * 32 * qsgd::kStride * 4;
+    const size_t smem = qsgd::kLut * 4 + (size_t)qsgd::kMultiWarps * 32 * qsgd::kMStride * 4;
     gridDim = {grid, 1, 1};
     blockDim = {(unsigned)kBlock, 1, 1};
     std::vector<unsigned char> sm(smem + 64);

@@ -157,6 +157,13 @@ def test_split_decoder_corrupt_streams(emu_exe, tmp_path, oracle_lib, d, P):
 # decode-accumulate and for the mean; ragged tails, d % 64 != 0, K past one chunk of
 # eight warps and past one launch
 MULTI = [
+    # one, two, three and four streams: 8, 4, 2 and 2 groups to a CTA (3 leaves two
+    # warps idle); bucket counts that leave the last set of groups part-filled
+    (20_000, 512, 16, 1, True, False, "layered"),
+    (70_001, 256, 16, 2, True, False, "normal"),
+    (50_000, 100, 7, 4, True, False, "normal"),
+    (33_000, 128, 5, 1, False, True, "normal"),
+    (61_001, 256, 16, 2, False, True, "layered"),
     (20_000, 512, 16, 3, True, False, "layered"),
     (20_000, 512, 16, 8, True, False, "normal"),
     (9_001, 100, 7, 11, True, False, "normal"),
