@@ -152,6 +152,32 @@ def _rank_main(rank, world, port, out_dir):
         streams.append((nr, c))
     ref, _ = o.bbit_decode_mean(streams, N, D, BW)
     res["ok"].append(bool(np.array_equal(out.numpy().view(np.uint32), ref.view(np.uint32))))
+    # b-bit with the memory, two steps
+    bmem = torch.zeros(N, dtype=torch.float32)
+    bmems = [np.zeros(N, np.float32) for _ in range(world)]
+    for step in range(2):
+        out = xb.step(torch.from_numpy(_grad(rank, step)), seed=80 + step, memory=bmem)
+        streams = []
+        for j in range(world):
+            c, nr, _, bmems[j] = o.bbit_encode_ef(_grad(j, step), bmems[j], D, BW, X.rank_seed(80 + step, j))
+            streams.append((nr, c))
+        ref, _ = o.bbit_decode_mean(streams, N, D, BW)
+        res["ok"].append(bool(np.array_equal(out.numpy().view(np.uint32), ref.view(np.uint32))))
+        res["ok"].append(bool(np.array_equal(bmem.numpy().view(np.uint32), bmems[rank].view(np.uint32))))
+    # uneven streams: rank 0 sends an all-zero gradient (norms only), the others a
+    # gradient with a non-finite bucket
+    def odd(j):
+        g = np.zeros(N, np.float32) if j == 0 else _grad(j, 9)
+        if j > 0:
+            g[D + 3] = np.inf
+        return g
+    out = xe.step(torch.from_numpy(odd(rank)), seed=99)
+    streams = []
+    for j in range(world):
+        w, off, _, _ = o.encode(odd(j), D, S, X.rank_seed(99, j))
+        streams.append((w, off))
+    ref, _ = o.decode_mean(streams, N, D, S)
+    res["ok"].append(bool(np.array_equal(out.numpy().view(np.uint32), ref.view(np.uint32))))
     res["mean0"] = float(out[0])
     dist.barrier()
     dist.destroy_process_group()
