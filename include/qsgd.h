@@ -169,7 +169,10 @@ QSGD_API int qsgd_decode(const uint32_t* d_words, uint64_t num_words, const uint
  *   h_words, h_num_words, h_offsets  host arrays of K entries holding device
  *                                    pointers / word counts (copied at the call)
  *   1 <= K <= 1024
- * Status bits as for qsgd_decode. */
+ * Status bits as for qsgd_decode.  Two or more streams (d % 4 == 0, d <= 4096,
+ * s < 1024, 16-byte aligned d_out) are decoded side by side, up to 16 to a launch, and
+ * d_out is read and written once per eight streams.  Other cases take one launch per
+ * stream.  The result is the same either way. */
 QSGD_API int qsgd_decode_accumulate(const uint32_t* const* h_words, const uint64_t* h_num_words,
                            const uint64_t* const* h_offsets, int K, uint64_t n, uint32_t d,
                            uint32_t s, float* d_out, uint32_t* d_status, cudaStream_t stream);
@@ -180,8 +183,10 @@ QSGD_API int qsgd_decode_accumulate(const uint32_t* const* h_words, const uint64
  * The sum runs left to right from +0, in fp32, as in qsgd_decode_accumulate; then one
  * IEEE division by K per coordinate.  d_out is overwritten, not accumulated.  The
  * arguments and the status are those of qsgd_decode_accumulate (1 <= K <= 1024, host
- * arrays of device pointers).  Every stream is checked before the first launch.  The
- * work is K decode launches and one division pass. */
+ * arrays of device pointers).  Every stream is checked before the first launch.  Two
+ * or more streams on the shapes qsgd_decode_accumulate decodes side by side divide in
+ * the same pass.  One stream, or another shape, is decoded, accumulated and then
+ * divided in a separate pass. */
 QSGD_API int qsgd_decode_mean(const uint32_t* const* h_words, const uint64_t* h_num_words,
                               const uint64_t* const* h_offsets, int K, uint64_t n, uint32_t d,
                               uint32_t s, float* d_out, uint32_t* d_status, cudaStream_t stream);
