@@ -120,6 +120,16 @@ class LibraryBbitCodec:
 # ---------------------------------------------------------------------------
 # The exchange
 # ---------------------------------------------------------------------------
+def _all_gather(out, inp, group):
+    """out = the ranks' inp, rank-major (a copy in a process without a group)."""
+    import torch.distributed as dist
+
+    if dist.is_initialized():
+        dist.all_gather_into_tensor(out, inp, group=group)
+    else:
+        out.copy_(inp)
+
+
 @dataclass
 class StepInfo:
     """What one exchange step moved (bytes this rank sent into the gathers)."""
@@ -141,12 +151,7 @@ class EliasExchange:
         self.last = StepInfo(0, 0)
 
     def _gather(self, out, inp):
-        import torch.distributed as dist
-
-        if dist.is_initialized():
-            dist.all_gather_into_tensor(out, inp, group=self.group)
-        else:  # a single process without a process group
-            out.copy_(inp)
+        _all_gather(out, inp, self.group)
 
     def step(self, grad, seed: int, memory=None, out=None):
         """Exchanges this rank's encoding of grad; returns the mean of all ranks' decodes."""
@@ -181,12 +186,7 @@ class BbitExchange:
         self.rank = dist.get_rank(group) if dist.is_initialized() else 0
 
     def _gather(self, out, inp):
-        import torch.distributed as dist
-
-        if dist.is_initialized():
-            dist.all_gather_into_tensor(out, inp, group=self.group)
-        else:  # a single process without a process group
-            out.copy_(inp)
+        _all_gather(out, inp, self.group)
 
     def step(self, grad, seed: int, memory=None, out=None):
         torch = _torch()
