@@ -1,0 +1,2 @@
+#pragma once
+#include "block_emu.h"
