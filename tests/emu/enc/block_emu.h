@@ -90,6 +90,10 @@ inline unsigned long long atomicCAS(unsigned long long* p, unsigned long long cm
     return cmp;
 }
 inline void __threadfence() { __atomic_thread_fence(__ATOMIC_SEQ_CST); }
+// host helpers that size grids ask for the device: one B200-sized answer
+enum { cudaDevAttrMultiProcessorCount = 16 };
+inline cudaError_t cudaGetDevice(int* dev) { *dev = 0; return cudaSuccess; }
+inline cudaError_t cudaDeviceGetAttribute(int* v, int, int) { *v = 148; return cudaSuccess; }
 inline void __nanosleep(unsigned) { std::this_thread::yield(); }
 
 // ---- one block's state ---------------------------------------------------------
