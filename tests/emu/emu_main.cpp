@@ -1,11 +1,11 @@
-// Runs the decoder kernels decode_fast (P = 0), decode_split (P >= 1) and
-// decode_multi (P = -1), compiled for the host under warp_emu.h, over streams read
-// from files.  argv: dir P accumulate [grid [mean]]
+// Runs the decoder kernels decode_fast (P = 0), decode_split (P >= 1), decode_multi
+// (P = -1) and decode_warp (P = -2), compiled for the host under warp_emu.h, over
+// streams read from files.  argv: dir P accumulate [grid [mean]]
 // dir holds params.bin (u64 n, d, s, K), out_in.bin (fp32[n]), w<j>.bin / o<j>.bin
 // (words, offsets of stream j); the result goes to out.bin and the status to stdout.
-// For P >= 0 the K streams are decoded one launch each, in order.  For P = -1 they
-// go 16 to a launch, as the library sends them to decode_multi; with mean = 1 the
-// first launch starts from +0 and the last divides by K.
+// For P >= 0 the K streams are decoded one launch each, in order.  For P < 0 they
+// go 16 to a launch, as the library sends them; with mean = 1 (decode_multi only)
+// the first launch starts from +0 and the last divides by K.
 #include "warp_emu.h"
 thread_local dim3e threadIdx, blockIdx;
 dim3e gridDim, blockDim;
@@ -65,6 +65,29 @@ template <bool A, int P> void run_kernel(const qsgd::DecodeArgs& a, unsigned gri
         for (auto& x : th) x.join();
     }
 }
+template <bool A> static void run_warp(const qsgd::DecodeArgs& a, unsigned grid) {
+    const int kBlock = qsgd::kDecodeBlock;
+    const size_t smem = qsgd::kLut * 4 + (size_t)qsgd::kDecWarps * 32 * qsgd::kStride * 4 +
+                        (size_t)kBlock * a.K * sizeof(qsgd::LaneStream);
+    gridDim = {grid, 1, 1};
+    blockDim = {(unsigned)kBlock, 1, 1};
+    std::vector<unsigned char> sm(smem + 64);
+    std::vector<WarpSync> warps(kBlock / 32);
+    for (unsigned b = 0; b < grid; ++b) {
+        g_emu_smem = sm.data();
+        std::memset(sm.data(), 0xAB, sm.size());
+        g_warps = warps.data();
+        std::vector<std::thread> th;
+        for (int t = 0; t < kBlock; ++t)
+            th.emplace_back([&, t, b] {
+                threadIdx = {(unsigned)t, 0, 0};
+                blockIdx = {b, 0, 0};
+                qsgd::decode_warp<A>(a);
+            });
+        for (auto& x : th) x.join();
+    }
+}
+
 static void run_multi(const qsgd::DecodeArgs& a, unsigned grid) {
     const int kBlock = qsgd::kMultiBlock;
     const size_t smem = qsgd::kLut * 4 + (size_t)qsgd::kMultiWarps * 32 * qsgd::kMStride * 4;
@@ -121,7 +144,12 @@ int main(int argc, char** argv) {
                 a.streams[j].num_words = ws[j0 + j].size() / 4;
                 a.streams[j].offsets = reinterpret_cast<const uint64_t*>(os[j0 + j].data());
             }
-            run_multi(a, grid);
+            if (P == -1)
+                run_multi(a, grid);
+            else if (acc)
+                run_warp<true>(a, grid);
+            else
+                run_warp<false>(a, grid);
             if (g_emu_error) return 4;
         }
         FILE* f = std::fopen((dir + "/out.bin").c_str(), "wb");

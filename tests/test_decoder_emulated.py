@@ -209,3 +209,27 @@ def test_multi_stream_kernel_corrupt_stream(emu_exe, tmp_path, oracle_lib):
                 keep[b * d:min(n, (b + 1) * d)] = False
     assert keep.any()
     assert np.array_equal(got[keep].view(np.uint32), ref[keep].view(np.uint32))
+
+
+# decode_warp (P = -2): the decoder of every other shape (d % 4 != 0, d > 4096,
+# s >= 1024), up to 16 streams to a launch with per-lane state in shared memory
+WARP = [
+    (20_000, 100, 7, 1, False, "normal"),
+    (20_001, 130, 3, 3, True, "layered"),
+    (9_001, 5_000, 2_000, 1, False, "normal"),
+    (6_000, 99, 16, 17, True, "normal"),
+    (30_000, 512, 16, 2, True, "heavy_tailed_sparse"),
+]
+
+
+@pytest.mark.parametrize("n,d,s,K,accumulate,kind", WARP, ids=["n%d-d%d-s%d-K%d-acc%d-%s" % c for c in WARP])
+def test_general_decoder_matches_oracle(emu_exe, tmp_path, oracle_lib, n, d, s, K, accumulate, kind):
+    got, status, streams, base = _run(emu_exe, tmp_path, oracle_lib, n, d, s, K, -2, accumulate, kind)
+    assert status == 0
+    if accumulate:
+        ref = base.copy()
+        _, rst = oracle_lib.decode_accumulate(streams, n, d, s, ref)
+    else:
+        ref, rst = oracle_lib.decode(streams[-1][0], streams[-1][1], n, d, s)
+    assert rst == 0
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
