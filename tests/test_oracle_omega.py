@@ -13,7 +13,8 @@ def test_textbook_codewords(oracle_lib, N, code):
 
 
 def test_textbook_lengths(oracle_lib):
-    # lengths quoted in the survey of the method's coding step
+    # lengths worked out by hand from the omega construction (Elias 1975), e.g.
+    # 16 -> 10 100 10000 0 (11 bits), 512 -> 11 1001 1000000000 0 (17 bits)
     expect = {1: 1, 2: 3, 3: 3, 4: 6, 8: 7, 16: 11, 256: 16, 512: 17, 8192: 21, 1 << 20: 32}
     for N, ln in expect.items():
         assert oracle_lib.omega_len(N) == ln
