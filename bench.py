@@ -186,6 +186,11 @@ def replica_seed(w, rank: int) -> int:
     return w.seed + rank
 
 
+def spread(times) -> dict:
+    """Median and minimum of per-step device times (ms)."""
+    return {"ms_median": statistics.median(times), "ms_min": min(times)}
+
+
 def job_value(world: int, bytes_per_rank: float, ms_max: float) -> float:
     """Whole-job GB/s: every rank's bytes over the slowest rank's time."""
     return world * bytes_per_rank / ms_max / 1e6
@@ -341,6 +346,8 @@ def run_ours(args, w):
     t_dec = sum(ev[k][1].elapsed_time(ev[k][2]) for k in range(K)) / K
     t_acc = sum(ev[k][2].elapsed_time(ev[k][3]) for k in range(K)) / K
     t_step = sum(ev[k][0].elapsed_time(ev[k][3]) for k in range(K)) / K
+    per_step = {name: [ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(K)]
+                for i, name in enumerate(("encode", "decode", "decode_accumulate"))}
     t_step_max = max_over_ranks(t_step, world)
     if int(status.item()) != 0:
         raise RuntimeError("device status %d in the timed region" % int(status.item()))
@@ -541,6 +548,8 @@ def run_ours(args, w):
                               "algorithmic_gbs": acc_bytes / t_acc / 1e6,
                               "roofline_frac": acc_bytes / t_acc / 1e6 / peak},
     }
+    for name, ts in per_step.items():
+        phases[name].update(spread(ts))  # "ms" is the mean over the timed steps
     dominant = max(phases, key=lambda k: phases[k]["ms"])
     dom = phases[dominant]
     traffic = None

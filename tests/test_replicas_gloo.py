@@ -66,3 +66,11 @@ def test_two_gloo_replicas(tmp_path):
     n = 25_557_032
     assert r[0]["value"] == pytest.approx(2 * 4.0 * n / 2.5 / 1e6)  # all ranks' bytes / max time
     assert r[1]["ref_output"] == "" and r[1]["ref_ret"] is None     # non-zero ranks do no work
+
+
+def test_phase_spread():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    assert bench.spread([3.0, 1.0, 2.0, 10.0]) == {"ms_median": 2.5, "ms_min": 1.0}
+    assert bench.spread([0.5]) == {"ms_median": 0.5, "ms_min": 0.5}
