@@ -77,9 +77,14 @@ uint64_t qsgd_max_encoded_words(uint64_t n, uint32_t d, uint32_t s) {
     return ceil_div(max_bits(n, d, s), 32);
 }
 
+#ifndef QSGD_ENCODER_TWO_PASS
+#define QSGD_ENCODER_TWO_PASS 0  // 1: the fast shapes go to the two-pass encoder
+#endif
+
 size_t qsgd_encode_workspace_bytes(uint64_t n, uint32_t d, uint32_t s) {
     if (!valid_params(n, d, s)) return 0;
-    return workspace_layout(n, d).total;
+    const size_t total = workspace_layout(n, d).total;
+    return QSGD_ENCODER_TWO_PASS ? align256(total) + encode2_scratch_bytes(n, d) : total;
 }
 
 int qsgd_workspace_init(void* d_ws, size_t ws_bytes, cudaStream_t stream) {
@@ -176,6 +181,11 @@ int qsgd_encode_ex(const float* d_in, uint64_t n, uint32_t d, uint32_t s, uint64
     const int rc = prepare_encode(d_in, n, d, s, seed, norm_kind, d_words, words_capacity, d_offsets, d_ws, ws_bytes,
                                   d_status, stream, a, fast);
     if (rc != QSGD_OK) return rc == kNothingToDo ? QSGD_OK : rc;
+    if (QSGD_ENCODER_TWO_PASS && fast) {
+        const size_t off = align256(workspace_layout(n, d).total);
+        if (ws_bytes < off + encode2_scratch_bytes(n, d)) return QSGD_ERR_WORKSPACE;
+        return launch_encode2(a, static_cast<char*>(d_ws) + off, stream) == cudaSuccess ? QSGD_OK : QSGD_ERR_CUDA;
+    }
     return launch_encode(a, fast, stream) == cudaSuccess ? QSGD_OK : QSGD_ERR_CUDA;
 }
 

@@ -49,6 +49,11 @@ struct EncodeArgs {
 // error code (cudaSuccess on success).
 cudaError_t launch_encode(EncodeArgs a, bool fast_path, cudaStream_t stream);
 
+// The two-pass encoder (qsgd_encode2.cu; used when QSGD_ENCODER_TWO_PASS is set):
+// its scratch (record lists, counts, sizes, norms) and its three launches.
+size_t encode2_scratch_bytes(uint64_t n, uint32_t d);
+cudaError_t launch_encode2(const EncodeArgs& a, void* scratch, cudaStream_t stream);
+
 // Dynamic shared memory of the general encoder: omega table | chunk buffer |
 // (norm, s/norm) of the tile's buckets.
 inline size_t general_smem_bytes(uint32_t smem_words, uint32_t buckets_per_tile) {
