@@ -181,7 +181,7 @@ int qsgd_encode_ex(const float* d_in, uint64_t n, uint32_t d, uint32_t s, uint64
     const int rc = prepare_encode(d_in, n, d, s, seed, norm_kind, d_words, words_capacity, d_offsets, d_ws, ws_bytes,
                                   d_status, stream, a, fast);
     if (rc != QSGD_OK) return rc == kNothingToDo ? QSGD_OK : rc;
-    if (QSGD_ENCODER_TWO_PASS && fast) {
+    if (QSGD_ENCODER_TWO_PASS && fast && encode2_fits(d, s)) {
         const size_t off = align256(workspace_layout(n, d).total);
         if (ws_bytes < off + encode2_scratch_bytes(n, d)) return QSGD_ERR_WORKSPACE;
         return launch_encode2(a, static_cast<char*>(d_ws) + off, stream) == cudaSuccess ? QSGD_OK : QSGD_ERR_CUDA;

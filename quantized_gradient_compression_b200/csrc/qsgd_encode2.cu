@@ -43,7 +43,7 @@ struct Enc2Args {
     uint32_t* words;
     uint64_t cap_words;
     uint32_t* status;
-    uint32_t bucket_words;  // words of one bucket's staging buffer
+    uint32_t bucket_words;  // words of one bucket's staging buffer (its bits, or its record list)
 };
 
 // Pass A: one warp per bucket.  Norm, levels, the record list, the bit count.
@@ -53,6 +53,7 @@ __global__ void __launch_bounds__(kE2Block) enc2_levels(const __grid_constant__ 
     uint32_t* const otab = smem;  // omega code table
     constexpr int NC = 4 * V;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    uint32_t* const slist = smem + kOmegaTab + warp * 128 * V;  // this warp's record list
     omega_table_fill(otab, tid, kE2Block);
     __syncthreads();
     const PhiloxKey key{a.key0, a.key1};
@@ -114,14 +115,13 @@ __global__ void __launch_bounds__(kE2Block) enc2_levels(const __grid_constant__ 
         }
         int32_t prev = __shfl_up_sync(kAll2, lmax, 1);  // the last record before this lane's
         if (lane == 0) prev = -1;
-        uint32_t* rec = a.recs + base;
         uint32_t pos = incl - cnt, lbits = 0;
 #pragma unroll
         for (int q = 0; q < NC; ++q) {
             const uint32_t k = kq[q] & 0x7FFFFFFFu;
             if (k) {
                 const uint32_t i = first + q;
-                rec[pos++] = i | (k << 10) | (kq[q] & 0x80000000u);
+                slist[pos++] = i | (k << 10) | (kq[q] & 0x80000000u);
                 lbits += omega_len(otab, static_cast<uint64_t>(static_cast<int32_t>(i) - prev)) + 1u + omega_len(otab, k);
                 prev = static_cast<int32_t>(i);
             }
@@ -129,6 +129,10 @@ __global__ void __launch_bounds__(kE2Block) enc2_levels(const __grid_constant__ 
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) lbits += __shfl_xor_sync(kAll2, lbits, o);
         const uint32_t nzb = __shfl_sync(kAll2, incl, 31);
+        __syncwarp();  // the list is complete
+        uint32_t* rec = a.recs + base;
+        for (uint32_t r = lane; r < nzb; r += 32) rec[r] = slist[r];
+        __syncwarp();  // the list is free for the next bucket
         if (lane == 0) {
             a.nz[b] = nzb;
             a.bits[b] = 32u + lbits;
@@ -186,7 +190,10 @@ __global__ void __launch_bounds__(kE2Block) enc2_pack(const __grid_constant__ En
         const uint32_t nz = a.nz[b];
         const uint32_t nbits = a.bits[b];
         const uint64_t o = a.offsets[b];
-        const uint32_t* rec = a.recs + b * a.d;
+        const uint32_t* grec = a.recs + b * a.d;
+        for (uint32_t r = lane; r < nz; r += 32) buf[r] = grec[r];  // the list, staged in buf
+        __syncwarp();
+        const uint32_t* rec = buf;
         // this lane's run of records into its strip
         LanePacker pk{pb, 0u, 0u, 0u};
         const uint32_t per = (nz + 31) >> 5;
@@ -213,6 +220,7 @@ __global__ void __launch_bounds__(kE2Block) enc2_pack(const __grid_constant__ En
         }
         pk.finish();
         const uint32_t lb = pk.bits();
+        __syncwarp();  // every lane has read its run: buf takes the bucket's bits next
         uint32_t incl = lb;
 #pragma unroll
         for (int s = 1; s < 32; s <<= 1) {
@@ -264,7 +272,9 @@ template <int V>
 cudaError_t launch_v(const Enc2Args& a, int grid, cudaStream_t stream) {
     int dev = 0;
     cudaGetDevice(&dev);
-    enc2_levels<V><<<grid, kE2Block, kOmegaTab * sizeof(uint32_t), stream>>>(a);
+    const size_t smem_a = (static_cast<size_t>(kOmegaTab) + static_cast<size_t>(kE2Warps) * 128 * V) * sizeof(uint32_t);
+    cudaFuncSetAttribute(enc2_levels<V>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    enc2_levels<V><<<grid, kE2Block, smem_a, stream>>>(a);
     enc2_scan<<<1, kScanBlock, 0, stream>>>(a);
     const bool sh = a.s <= 31;
     const size_t smem = (static_cast<size_t>(kRecordTab) + static_cast<size_t>(kE2Warps) * a.bucket_words +
@@ -281,6 +291,14 @@ cudaError_t launch_v(const Enc2Args& a, int grid, cudaStream_t stream) {
 }
 
 }  // namespace
+
+bool encode2_fits(uint32_t d, uint32_t s) {
+    const uint32_t V = fast_v(d);
+    const uint64_t bw = std::max<uint64_t>((32u + static_cast<uint64_t>(d) * (2u + omega_len_host(s)) + 31) / 32 + 1, d);
+    const uint64_t words_c = kRecordTab + kE2Warps * bw + static_cast<uint64_t>(kE2Warps) * 32 * fast_lane_words(V, s <= 31);
+    const uint64_t words_a = kOmegaTab + static_cast<uint64_t>(kE2Warps) * 128 * V;
+    return std::max(words_a, words_c) * sizeof(uint32_t) <= 200 * 1024;
+}
 
 size_t encode2_scratch_bytes(uint64_t n, uint32_t d) {
     const uint64_t nb = (n + d - 1) / d;
@@ -306,7 +324,9 @@ cudaError_t launch_encode2(const EncodeArgs& e, void* scratch, cudaStream_t stre
     a.words = e.words;
     a.cap_words = e.cap_words;
     a.status = e.status;
-    a.bucket_words = static_cast<uint32_t>((32u + static_cast<uint64_t>(e.d) * (2u + omega_len_host(e.s)) + 31) / 32 + 1);
+    // a bucket's bits, or its record list before them
+    a.bucket_words = static_cast<uint32_t>(std::max<uint64_t>(
+        (32u + static_cast<uint64_t>(e.d) * (2u + omega_len_host(e.s)) + 31) / 32 + 1, e.d));
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

@@ -51,6 +51,7 @@ cudaError_t launch_encode(EncodeArgs a, bool fast_path, cudaStream_t stream);
 
 // The two-pass encoder (qsgd_encode2.cu; used when QSGD_ENCODER_TWO_PASS is set):
 // its scratch (record lists, counts, sizes, norms) and its three launches.
+bool encode2_fits(uint32_t d, uint32_t s);  // its shared memory fits this shape
 size_t encode2_scratch_bytes(uint64_t n, uint32_t d);
 cudaError_t launch_encode2(const EncodeArgs& a, void* scratch, cudaStream_t stream);
 

@@ -35,7 +35,7 @@ template <class Kernel> static void run_grid(unsigned grid, unsigned block, size
 }
 using namespace qsgd;
 template <int V> static void passes(const Enc2Args& a, unsigned grid) {
-    run_grid(grid, kE2Block, kOmegaTab * 4, [&] { enc2_levels<V>(a); });
+    run_grid(grid, kE2Block, ((size_t)kOmegaTab + (size_t)kE2Warps * 128 * V) * 4, [&] { enc2_levels<V>(a); });
     run_grid(1, kScanBlock, 0, [&] { enc2_scan(a); });
     const bool sh = a.s <= 31;
     const size_t smem = (kRecordTab + (size_t)kE2Warps * a.bucket_words + (size_t)kE2Warps * 32 * fast_lane_words(V, sh)) * 4;
@@ -58,7 +58,7 @@ int main(int argc, char** argv) {
     a.in = in.data(); a.n = n; a.d = d; a.s = s; a.key0 = (uint32_t)seed; a.key1 = (uint32_t)(seed >> 32); a.norm_kind = nk;
     a.nb = nb; a.recs = recs.data(); a.nz = nz.data(); a.bits = bits.data(); a.norms = norms.data();
     a.offsets = offsets.data(); a.words = words.data(); a.cap_words = cap; a.status = &status;
-    a.bucket_words = (uint32_t)((32u + (uint64_t)d * (2u + omega_len_host(s)) + 31) / 32 + 1);
+    a.bucket_words = (uint32_t)std::max<uint64_t>((32u + (uint64_t)d * (2u + omega_len_host(s)) + 31) / 32 + 1, d);
     switch (fast_v(d)) {
         case 1: passes<1>(a, grid); break;
         case 2: passes<2>(a, grid); break;
