@@ -25,7 +25,7 @@
 namespace qsgd {
 namespace {
 
-constexpr uint32_t kAll2 = 0xFFFFFFFFu;
+constexpr uint32_t kWarpAll = 0xFFFFFFFFu;
 constexpr int kE2Warps = 16;
 constexpr int kE2Block = 32 * kE2Warps;
 constexpr int kScanBlock = 1024;
@@ -106,14 +106,14 @@ __global__ void __launch_bounds__(kE2Block) enc2_levels(const __grid_constant__ 
         int32_t lmax = last;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t t = __shfl_up_sync(kAll2, incl, o);
-            const int32_t u = __shfl_up_sync(kAll2, lmax, o);
+            const uint32_t t = __shfl_up_sync(kWarpAll, incl, o);
+            const int32_t u = __shfl_up_sync(kWarpAll, lmax, o);
             if (lane >= o) {
                 incl += t;
                 lmax = max(lmax, u);
             }
         }
-        int32_t prev = __shfl_up_sync(kAll2, lmax, 1);  // the last record before this lane's
+        int32_t prev = __shfl_up_sync(kWarpAll, lmax, 1);  // the last record before this lane's
         if (lane == 0) prev = -1;
         uint32_t pos = incl - cnt, lbits = 0;
 #pragma unroll
@@ -127,8 +127,8 @@ __global__ void __launch_bounds__(kE2Block) enc2_levels(const __grid_constant__ 
             }
         }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) lbits += __shfl_xor_sync(kAll2, lbits, o);
-        const uint32_t nzb = __shfl_sync(kAll2, incl, 31);
+        for (int o = 16; o > 0; o >>= 1) lbits += __shfl_xor_sync(kWarpAll, lbits, o);
+        const uint32_t nzb = __shfl_sync(kWarpAll, incl, 31);
         __syncwarp();  // the list is complete
         uint32_t* rec = a.recs + base;
         for (uint32_t r = lane; r < nzb; r += 32) rec[r] = slist[r];
@@ -224,7 +224,7 @@ __global__ void __launch_bounds__(kE2Block) enc2_pack(const __grid_constant__ En
         uint32_t incl = lb;
 #pragma unroll
         for (int s = 1; s < 32; s <<= 1) {
-            const uint32_t t = __shfl_up_sync(kAll2, incl, s);
+            const uint32_t t = __shfl_up_sync(kWarpAll, incl, s);
             if (lane >= s) incl += t;
         }
         const uint32_t pos = 32u + incl - lb;  // bucket-local bit of this lane's first record
@@ -270,8 +270,6 @@ __global__ void __launch_bounds__(kE2Block) enc2_pack(const __grid_constant__ En
 
 template <int V>
 cudaError_t launch_v(const Enc2Args& a, int grid, cudaStream_t stream) {
-    int dev = 0;
-    cudaGetDevice(&dev);
     const size_t smem_a = (static_cast<size_t>(kOmegaTab) + static_cast<size_t>(kE2Warps) * 128 * V) * sizeof(uint32_t);
     cudaFuncSetAttribute(enc2_levels<V>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
     enc2_levels<V><<<grid, kE2Block, smem_a, stream>>>(a);
