@@ -140,3 +140,25 @@ def test_mean_arguments_checked():
         == B.QSGD_ERR_ARG
     assert B.qsgd_bbit_decode_mean([A, 0], [A, A], 2, 100, 4, 4, A * 4, A * 8, 0) == B.QSGD_ERR_ARG
     assert B.qsgd_bbit_decode_mean([A], [A], 1, 100, 4, 3, A * 4, A * 8, 0) == B.QSGD_ERR_ARG
+
+
+def test_product_path_fails_loudly_without_the_library(tmp_path):
+    """No CPU fallback: the binding refuses to import when the CUDA library is absent."""
+    import importlib.util
+    import shutil
+
+    src = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                       "quantized_gradient_compression_b200", "binding.py")
+    shutil.copy(src, tmp_path / "binding.py")  # a package directory with no .so in it
+    spec = importlib.util.spec_from_file_location("binding_without_lib", tmp_path / "binding.py")
+    mod = importlib.util.module_from_spec(spec)
+    with pytest.raises(ImportError, match="not built"):
+        spec.loader.exec_module(mod)
+
+
+def test_library_codec_takes_cuda_tensors_only():
+    import torch
+    from quantized_gradient_compression_b200 import binding as B
+
+    with pytest.raises(AssertionError):
+        B.encode(torch.zeros(1024), 512, 16, 0)
