@@ -573,7 +573,7 @@ def run_ours(args, w):
         "bits_per_coord": total_bits / n,
         "compressed_bytes": comp_bytes,
         "phases": phases,
-        "roofline": {"bound": "hbm", "kernel": {"encode": "encode_fast<4, true> (qsgd_encode)",
+        "roofline": {"bound": "hbm", "kernel": {"encode": "encode_fast<4, true, false> (qsgd_encode)",
                                                   "decode": "decode_fast<false> (qsgd_decode)",
                                                   "decode_accumulate": "decode_fast<true> (qsgd_decode_accumulate)"}[dominant],
                      "achieved": dom["algorithmic_gbs"], "peak": peak, "unit": "GB/s",
