@@ -64,6 +64,19 @@ WorkspaceLayout workspace_layout(uint64_t n, uint32_t d) {
     return L;
 }
 
+StageLayout stage_layout(uint64_t n, uint32_t d, uint32_t s) {
+    StageLayout L{};
+    const uint64_t nb = n ? ceil_div(n, d) : 0;
+    const uint64_t slot_bits = 32u + static_cast<uint64_t>(d) * (2u + omega_len_host(s));
+    L.slot_words = static_cast<uint32_t>(ceil_div(slot_bits, 32));
+    L.ntiles = ceil_div(nb, kCompactBlock);
+    L.desc_off = 256;
+    L.bits_off = L.desc_off + align256(sizeof(uint64_t) * L.ntiles);
+    L.stage_off = L.bits_off + align256(sizeof(uint32_t) * nb);
+    L.total = L.stage_off + align256(sizeof(uint32_t) * nb * L.slot_words);
+    return L;
+}
+
 }  // namespace qsgd
 
 using namespace qsgd;
@@ -81,10 +94,18 @@ uint64_t qsgd_max_encoded_words(uint64_t n, uint32_t d, uint32_t s) {
 #define QSGD_ENCODER_TWO_PASS 0  // 1: the fast shapes go to the two-pass encoder
 #endif
 
-size_t qsgd_encode_workspace_bytes(uint64_t n, uint32_t d, uint32_t s) {
+// Workspace of the one-pass encoders (encode_fast, encode_general) alone: the scan
+// state, a few bytes per tile.
+static size_t one_pass_workspace_bytes(uint64_t n, uint32_t d, uint32_t s) {
     if (!valid_params(n, d, s)) return 0;
     const size_t total = workspace_layout(n, d).total;
     return QSGD_ENCODER_TWO_PASS ? align256(total) + encode2_scratch_bytes(n, d) : total;
+}
+
+size_t qsgd_encode_workspace_bytes(uint64_t n, uint32_t d, uint32_t s) {
+    const size_t one = one_pass_workspace_bytes(n, d, s);
+    if (one == 0 || !stage_shape(d)) return one;
+    return std::max(one, stage_layout(n, d, s).total);
 }
 
 int qsgd_workspace_init(void* d_ws, size_t ws_bytes, cudaStream_t stream) {
@@ -171,51 +192,107 @@ bool overlaps(const float* a, const float* b, uint64_t n) {
 
 }  // namespace
 
+namespace qsgd {
+
+// Fills the two-launch encoder's arguments (after prepare_encode has checked them).
+static StageArgs stage_args(const EncodeArgs& e, float* d_ef, uint64_t seed, void* d_ws) {
+    const StageLayout L = stage_layout(e.n, e.d, e.s);
+    char* ws = static_cast<char*>(d_ws);
+    StageArgs a{};
+    a.in = e.in;
+    a.ef = d_ef;
+    a.n = e.n;
+    a.d = e.d;
+    a.s = e.s;
+    a.norm_kind = e.norm_kind;
+    const uint32_t k0 = static_cast<uint32_t>(seed), k1 = static_cast<uint32_t>(seed >> 32);
+    for (uint32_t r = 0; r < 10; ++r) {
+        a.rk[2 * r] = k0 + r * 0x9E3779B9u;
+        a.rk[2 * r + 1] = k1 + r * 0xBB67AE85u;
+    }
+    a.nb = e.nb;
+    a.slot_words = L.slot_words;
+    a.buf_words = L.slot_words + 1;
+    a.stage = reinterpret_cast<uint32_t*>(ws + L.stage_off);
+    a.bits = reinterpret_cast<uint32_t*>(ws + L.bits_off);
+    a.status = e.status;
+    a.words = e.words;
+    a.cap_words = e.cap_words;
+    a.offsets = e.offsets;
+    a.ctrl = reinterpret_cast<ScanControl*>(ws);
+    a.cdesc = reinterpret_cast<uint64_t*>(ws + L.desc_off);
+    a.ntiles = L.ntiles;
+    return a;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// qsgd_encode_ex / qsgd_encode_ef.  d_ef: the error-feedback memory, or null.  With
+// `strict`, the workspace must hold qsgd_encode_workspace_bytes; otherwise (the static
+// workspace entry point) the two-launch encoder runs when its layout fits, else a
+// one-pass encoder.  Every path writes the same stream.
+int encode_entry(const float* d_in, float* d_ef, uint64_t n, uint32_t d, uint32_t s, uint64_t seed,
+                 uint32_t norm_kind, uint32_t* d_words, uint64_t words_capacity, uint64_t* d_offsets, void* d_ws,
+                 size_t ws_bytes, uint32_t* d_status, cudaStream_t stream, bool strict) {
+    if (d_ef && n > 0) {
+        if (!d_in || ((reinterpret_cast<uintptr_t>(d_in) | reinterpret_cast<uintptr_t>(d_ef)) & 3u) != 0)
+            return QSGD_ERR_ARG;
+        if (overlaps(d_in, d_ef, n)) return QSGD_ERR_ARG;
+    }
+    EncodeArgs a;
+    bool fast = false;
+    int rc = prepare_encode(d_in, n, d, s, seed, norm_kind, d_words, words_capacity, d_offsets, d_ws, ws_bytes,
+                            d_status, stream, a, fast);
+    if (rc != QSGD_OK) return rc == kNothingToDo ? QSGD_OK : rc;
+    if (strict && ws_bytes < qsgd_encode_workspace_bytes(n, d, s)) return QSGD_ERR_WORKSPACE;
+    if (stage_shape(d) && aligned16(d_in) && (!d_ef || aligned16(d_ef)) &&
+        ws_bytes >= stage_layout(n, d, s).total) {
+        // two launches: bucket coder (with the memory fused in), compaction
+        return launch_encode_stage(stage_args(a, d_ef, seed, d_ws), stream) == cudaSuccess ? QSGD_OK : QSGD_ERR_CUDA;
+    }
+    if (!d_ef) {
+        if (QSGD_ENCODER_TWO_PASS && fast && encode2_fits(d, s)) {
+            const size_t off = align256(workspace_layout(n, d).total);
+            if (ws_bytes < off + encode2_scratch_bytes(n, d)) return QSGD_ERR_WORKSPACE;
+            return launch_encode2(a, static_cast<char*>(d_ws) + off, stream) == cudaSuccess ? QSGD_OK : QSGD_ERR_CUDA;
+        }
+        return launch_encode(a, fast, stream) == cudaSuccess ? QSGD_OK : QSGD_ERR_CUDA;
+    }
+    if (fast && aligned16(d_ef)) {
+        // one pass: the fast encoder reads g and e and writes the stream and e
+        a.ef = d_ef;
+        return launch_encode(a, true, stream) == cudaSuccess ? QSGD_OK : QSGD_ERR_CUDA;
+    }
+    // three passes: e <- e + g; encode p from e; e <- p - decoded
+    rc = prepare_encode(d_ef, n, d, s, seed, norm_kind, d_words, words_capacity, d_offsets, d_ws, ws_bytes, d_status,
+                        stream, a, fast);
+    if (rc != QSGD_OK) return rc;
+    if (launch_ef_add(d_in, d_ef, n, stream) != cudaSuccess) return QSGD_ERR_CUDA;
+    if (launch_encode(a, fast, stream) != cudaSuccess) return QSGD_ERR_CUDA;
+    return launch_ef_residual(d_ef, d_words, words_capacity, d_offsets, n, d, s, seed, stream) == cudaSuccess
+               ? QSGD_OK
+               : QSGD_ERR_CUDA;
+}
+
+size_t min_encode_workspace_bytes(uint64_t n, uint32_t d, uint32_t s) { return one_pass_workspace_bytes(n, d, s); }
+
+}  // namespace qsgd
+
 extern "C" {
 
 int qsgd_encode_ex(const float* d_in, uint64_t n, uint32_t d, uint32_t s, uint64_t seed, uint32_t norm_kind,
                    uint32_t* d_words, uint64_t words_capacity, uint64_t* d_offsets, void* d_ws, size_t ws_bytes,
                    uint32_t* d_status, cudaStream_t stream) {
-    EncodeArgs a;
-    bool fast = false;
-    const int rc = prepare_encode(d_in, n, d, s, seed, norm_kind, d_words, words_capacity, d_offsets, d_ws, ws_bytes,
-                                  d_status, stream, a, fast);
-    if (rc != QSGD_OK) return rc == kNothingToDo ? QSGD_OK : rc;
-    if (QSGD_ENCODER_TWO_PASS && fast && encode2_fits(d, s)) {
-        const size_t off = align256(workspace_layout(n, d).total);
-        if (ws_bytes < off + encode2_scratch_bytes(n, d)) return QSGD_ERR_WORKSPACE;
-        return launch_encode2(a, static_cast<char*>(d_ws) + off, stream) == cudaSuccess ? QSGD_OK : QSGD_ERR_CUDA;
-    }
-    return launch_encode(a, fast, stream) == cudaSuccess ? QSGD_OK : QSGD_ERR_CUDA;
+    return encode_entry(d_in, nullptr, n, d, s, seed, norm_kind, d_words, words_capacity, d_offsets, d_ws, ws_bytes,
+                        d_status, stream, true);
 }
 
 int qsgd_encode_ef(const float* d_g, float* d_e, uint64_t n, uint32_t d, uint32_t s, uint64_t seed,
                    uint32_t norm_kind, uint32_t* d_words, uint64_t words_capacity, uint64_t* d_offsets, void* d_ws,
                    size_t ws_bytes, uint32_t* d_status, cudaStream_t stream) {
-    if (n > 0) {
-        if (!d_g || !d_e || ((reinterpret_cast<uintptr_t>(d_g) | reinterpret_cast<uintptr_t>(d_e)) & 3u) != 0)
-            return QSGD_ERR_ARG;
-        if (overlaps(d_g, d_e, n)) return QSGD_ERR_ARG;
-    }
-    EncodeArgs a;
-    bool fast = false;
-    int rc = prepare_encode(d_g, n, d, s, seed, norm_kind, d_words, words_capacity, d_offsets, d_ws, ws_bytes,
-                            d_status, stream, a, fast);
-    if (rc != QSGD_OK) return rc == kNothingToDo ? QSGD_OK : rc;
-    if (fast && (reinterpret_cast<uintptr_t>(d_e) & 15u) == 0) {
-        // one pass: the fast encoder reads g and e and writes the stream and e
-        a.ef = d_e;
-        return launch_encode(a, true, stream) == cudaSuccess ? QSGD_OK : QSGD_ERR_CUDA;
-    }
-    // three passes: e <- e + g; encode p from e; e <- p - decoded
-    rc = prepare_encode(d_e, n, d, s, seed, norm_kind, d_words, words_capacity, d_offsets, d_ws, ws_bytes, d_status,
-                        stream, a, fast);
-    if (rc != QSGD_OK) return rc;
-    if (launch_ef_add(d_g, d_e, n, stream) != cudaSuccess) return QSGD_ERR_CUDA;
-    if (launch_encode(a, fast, stream) != cudaSuccess) return QSGD_ERR_CUDA;
-    return launch_ef_residual(d_e, d_words, words_capacity, d_offsets, n, d, s, seed, stream) == cudaSuccess
-               ? QSGD_OK
-               : QSGD_ERR_CUDA;
+    if (n > 0 && (!d_g || !d_e)) return QSGD_ERR_ARG;
+    return encode_entry(d_g, d_e, n, d, s, seed, norm_kind, d_words, words_capacity, d_offsets, d_ws, ws_bytes,
+                        d_status, stream, true);
 }
 
 int qsgd_encode(const float* d_in, uint64_t n, uint32_t d, uint32_t s, uint64_t seed, uint32_t* d_words,

@@ -1165,6 +1165,8 @@ cudaError_t launch_decode(const DecodeArgs& a, bool accumulate, cudaStream_t str
     if (a.nb == 0) return cudaSuccess;
     const bool fast = decode_fast_shape(a.d, a.s, a.out);
     if (a.start_zero || a.div != 0.f) return fast ? launch_multi(a, stream) : cudaErrorInvalidValue;
+    // one stream: whole bucket rows staged as byte codes when the shape allows
+    if (a.K == 1 && decode_rows_shape(a.d, a.s, a.out)) return launch_decode_rows(a, accumulate, stream);
     if (!fast) return accumulate ? launch<true>(a, stream) : launch<false>(a, stream);
 #ifndef QSGD_MULTI
 #define QSGD_MULTI 1

@@ -1,0 +1,320 @@
+// QSGD decoder for one stream with whole bucket rows staged as byte codes (sm_100a).
+//
+// Method: "QSGD (Quantized Stochastic Gradient Descent) with Elias Coding" (AIMech
+// curated entry).  The definition paragraph calls the coding "lossless prefix
+// coding" of the tuple (||v||_2, signs, run-length gaps, levels k_i); the decoder
+// inverts it and evaluates Q_s(v)_i = ||v||_2 * sgn(v_i) * k_i / s as
+// fl(fl(norm / s) * k), sign last, +0.0 off the support.  Decode-accumulate (a
+// receiver in "distributed data-parallel optimization", same paragraph) adds the
+// decoded stream onto the output: out_i <- fl(out_i + q_i).
+//
+// Work layout: each lane of a warp parses one bucket (buckets are independent
+// prefix-code streams located by the offsets header), 32 consecutive buckets to a
+// warp.  A record is decoded with one lookup of its first 12 bits in a shared-memory
+// table of whole records; longer records take a bit-serial path.  The lane stores the
+// record's code (sign << 7 | k, one byte, so s <= 127) at its index in its bucket's
+// row of a zeroed staging area: 32 rows of d bytes, padded so that the rows start on
+// different banks.  No lane waits for another while parsing.  Then the warp converts
+// the rows to fp32, row by row, and writes each bucket with coalesced 16-byte stores
+// (decode-accumulate first reads the output, which a prefetch to L2 issued before
+// the parse has brought in).
+#include <cuda_runtime.h>
+
+#include <algorithm>
+
+#include "../../include/qsgd.h"
+#include "qsgd_device.cuh"
+#include "qsgd_internal.h"
+
+namespace qsgd {
+namespace {
+
+constexpr uint32_t kWarpAll = 0xFFFFFFFFu;
+constexpr int kLutBits = 12;
+constexpr int kLutSize = 1 << kLutBits;
+constexpr uint32_t kParseGuard = 1u << 20;  // a second, explicit bound of the parse loop
+
+// One omega code from the top of an n-bit window w, starting at bit pos (MSB = 0).
+__device__ __forceinline__ bool window_omega(uint32_t w, int nbits, int& pos, uint32_t& value) {
+    uint32_t v = 1;
+    for (;;) {
+        if (pos >= nbits) return false;
+        const uint32_t bit = (w >> (nbits - 1 - pos)) & 1u;
+        ++pos;
+        if (bit == 0) {
+            value = v;
+            return true;
+        }
+        if (pos + static_cast<int>(v) > nbits) return false;
+        const uint32_t rest = (w >> (nbits - pos - v)) & ((1u << v) - 1u);
+        pos += v;
+        v = (1u << v) | rest;
+    }
+}
+
+// Table of whole records in a 12-bit window: [4:0] length (0: the window holds no
+// whole record with k <= s), [14:5] gap, [23:16] code sign << 7 | k.
+__device__ void build_rows_lut(uint32_t* lut, uint32_t s, int tid, int nthreads) {
+    for (int w = tid; w < kLutSize; w += nthreads) {
+        int pos = 0;
+        uint32_t gap = 0, k = 0, e = 0;
+        if (window_omega(static_cast<uint32_t>(w), kLutBits, pos, gap) && pos < kLutBits) {
+            const uint32_t sign = (static_cast<uint32_t>(w) >> (kLutBits - 1 - pos)) & 1u;
+            ++pos;
+            if (window_omega(static_cast<uint32_t>(w), kLutBits, pos, k) && k <= s && k < 128u && gap < 1024u)
+                e = static_cast<uint32_t>(pos) | (gap << 5) | (((sign << 7) | k) << 16);
+        }
+        lut[w] = e;
+    }
+}
+
+// MSB-first reader of one bucket: the next unread bits are the top `valid` bits of
+// buf (valid >= 32 after every refill), nx is the next stream word, `left` the bits
+// of the bucket not yet consumed (negative, as int32, after a record that overran).
+struct RowReader {
+    const uint32_t* base;  // word holding the bucket's first bit
+    uint32_t wi;           // next word to fetch, relative to base
+    uint32_t wlim;         // words available from base to the end of the stream
+    uint64_t buf;
+    uint32_t valid;
+    uint32_t nx;
+    uint32_t left;
+    __device__ __forceinline__ uint32_t fetch() {
+        const uint32_t w = wi < wlim ? __ldg(base + wi) : 0u;
+        ++wi;
+        return w;
+    }
+    __device__ __forceinline__ void init(const uint32_t* words, uint64_t num_words, uint64_t begin, uint32_t nbits) {
+        const uint64_t w0 = begin >> 5;
+        base = words + w0;
+        wlim = static_cast<uint32_t>(min(num_words - w0, static_cast<uint64_t>(0xFFFFFFFFu)));
+        wi = 0;
+        const uint32_t a0 = fetch(), a1 = fetch();
+        nx = fetch();
+        const uint32_t sh = static_cast<uint32_t>(begin & 31u);
+        buf = ((static_cast<uint64_t>(a0) << 32) | a1) << sh;
+        valid = 64u - sh;
+        left = nbits;
+        refill();
+    }
+    __device__ __forceinline__ void refill() {
+        if (valid < 32u) {
+            buf |= static_cast<uint64_t>(nx) << (32u - valid);
+            valid += 32u;
+            nx = fetch();
+        }
+    }
+    __device__ __forceinline__ void consume(uint32_t n) {  // n <= 32
+        buf <<= n;
+        valid -= n;
+        left -= n;
+        refill();
+    }
+    __device__ __forceinline__ uint32_t top(uint32_t n) const { return static_cast<uint32_t>(buf >> (64u - n)); }
+    __device__ __forceinline__ bool omega(uint32_t& N) {  // bit-serial, any length up to 2^32 - 1
+        uint32_t v = 1;
+        for (;;) {
+            if (static_cast<int32_t>(left) <= 0) return false;
+            const uint32_t bit = static_cast<uint32_t>(buf >> 63);
+            consume(1);
+            if (bit == 0) {
+                N = v;
+                return true;
+            }
+            if (v > 31 || static_cast<int32_t>(left) < static_cast<int32_t>(v)) return false;
+            const uint32_t rest = top(v);
+            consume(v);
+            v = (1u << v) | rest;
+        }
+    }
+};
+
+// A record the table does not hold, bit by bit: false when it is malformed (or its
+// level exceeds s).
+__device__ __forceinline__ bool slow_record(RowReader& r, uint32_t s, uint32_t& gap, uint32_t& code) {
+    uint32_t k;
+    if (!r.omega(gap) || static_cast<int32_t>(r.left) <= 0 || gap > 0xFFFFu) return false;
+    const uint32_t sign = static_cast<uint32_t>(r.buf >> 63);
+    r.consume(1);
+    if (!r.omega(k) || k > s) return false;
+    code = (sign << 7) | k;
+    return true;
+}
+
+template <int V, bool kAcc>
+__global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows(const __grid_constant__ DecodeArgs a,
+                                                                   uint32_t stride_w) {
+    extern __shared__ __align__(16) uint32_t smem[];
+    uint32_t* const lut = smem;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int W = blockDim.x >> 5;
+    uint32_t* const rows = smem + kLutSize + static_cast<uint32_t>(warp) * 32u * stride_w;
+    uint8_t* const myrow = reinterpret_cast<uint8_t*>(rows + static_cast<uint32_t>(lane) * stride_w);
+    build_rows_lut(lut, a.s, tid, blockDim.x);
+    __syncthreads();
+    const StreamRef st = a.streams[0];
+    const float fs = __uint2float_rn(a.s);
+    const uint32_t d = a.d;
+    const uint64_t ngroups = (a.nb + 31) / 32;
+    for (uint64_t g = blockIdx.x + static_cast<uint64_t>(gridDim.x) * warp; g < ngroups;
+         g += static_cast<uint64_t>(gridDim.x) * W) {
+        const uint64_t b = g * 32 + lane;
+        const bool live = b < a.nb;
+        const uint32_t m = live ? static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - b * d)) : 0u;
+        if constexpr (kAcc) {  // bring the group's output into L2 while the records are parsed
+            const float* gp = a.out + g * 32 * d;
+            const uint64_t gbytes = 4 * (min(a.n, (g + 1) * 32 * d) - g * 32 * d);
+            for (uint64_t off = static_cast<uint64_t>(lane) * 128; off < gbytes; off += 32 * 128)
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const char*>(gp) + off));
+        }
+        // zero the warp's rows (32 * stride_w words, a multiple of four)
+        for (uint32_t q = lane; q < 8u * stride_w; q += 32)
+            reinterpret_cast<uint4*>(rows)[q] = make_uint4(0u, 0u, 0u, 0u);
+        // open this lane's bucket: header checks and the norm
+        bool bad = false;
+        RowReader r;
+        r.left = 0;
+        float scale = 0.f;
+        if (live) {
+            const uint64_t begin = st.offsets[b];
+            const uint64_t end = st.offsets[b + 1];
+            if (!(end >= begin && end - begin >= 32 && end <= st.num_words * 32 && end - begin < (1ull << 30))) {
+                bad = true;
+            } else {
+                r.init(st.words, st.num_words, begin, static_cast<uint32_t>(end - begin));
+                const uint32_t nbits = r.top(32);
+                r.consume(32);
+                const float norm = __uint_as_float(nbits);
+                if (nbits == 0) {
+                    bad = r.left != 0;
+                    r.left = 0;
+                } else if (!(isfinite(norm) && norm > 0.f)) {
+                    bad = true;
+                    r.left = 0;
+                } else {
+                    scale = __fdiv_rn(norm, fs);
+                    if (!(scale > 0.f) && r.left != 0) {  // a zero scale carries no records
+                        bad = true;
+                        r.left = 0;
+                    }
+                }
+            }
+        }
+        __syncwarp();
+        // --- parse: every record's code into the lane's row ----------------------
+        uint32_t next = 0;  // bucket-local index after the last record
+        for (uint32_t it = 0;; ++it) {
+            const bool act = static_cast<int32_t>(r.left) > 0 && !bad;
+            if (!__any_sync(kWarpAll, act)) break;
+            if (it == kParseGuard) {
+                bad = bad || act;
+                break;
+            }
+            if (act) {
+                const uint32_t e = lut[static_cast<uint32_t>(r.buf >> (64 - kLutBits))];
+                const uint32_t len = e & 31u;
+                uint32_t gap = (e >> 5) & 1023u, code = e >> 16;
+                if (len != 0u) {
+                    r.consume(len);
+                } else if (!slow_record(r, a.s, gap, code)) {
+                    bad = true;
+                    gap = 0;
+                }
+                next += gap;
+                // a malformed index lands in the row's padding (the bucket is then bad)
+                if (!bad) myrow[min(next - 1u, d)] = static_cast<uint8_t>(code);
+            }
+        }
+        // every record index below m, and the bucket consumed exactly
+        if (live && !bad && (next > m || r.left != 0)) bad = true;
+        __syncwarp();
+        // --- write the rows back: row rr is bucket g*32 + rr -----------------------
+        for (int rr = 0; rr < 32; ++rr) {
+            const uint64_t bb = g * 32 + rr;
+            const float sc = __shfl_sync(kWarpAll, scale, rr);
+            if (bb >= a.nb) break;
+            const uint32_t mm = static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - bb * d));
+            const uint32_t* rowp = rows + static_cast<uint32_t>(rr) * stride_w;
+            float* gp = a.out + bb * d;
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                const uint32_t q = static_cast<uint32_t>(lane) + 32u * i;
+                const uint32_t c = 4u * q;
+                if (c < mm) {
+                    const uint32_t w = rowp[q];
+                    float v[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const uint32_t code = (w >> (8 * j)) & 0xFFu;
+                        // k as fp32 through the 2^23 offset (exact for k < 2^23), times the step
+                        const float kf = __fsub_rn(__uint_as_float(0x4B000000u | (code & 0x7Fu)), 8388608.0f);
+                        v[j] = __uint_as_float(__float_as_uint(__fmul_rn(sc, kf)) | ((code & 0x80u) << 24));
+                    }
+                    if (c + 4 <= mm) {
+                        float4* p4 = reinterpret_cast<float4*>(gp + c);
+                        if constexpr (kAcc) {
+                            const float4 o = *p4;
+                            v[0] = __fadd_rn(o.x, v[0]);
+                            v[1] = __fadd_rn(o.y, v[1]);
+                            v[2] = __fadd_rn(o.z, v[2]);
+                            v[3] = __fadd_rn(o.w, v[3]);
+                        }
+                        __stcs(p4, make_float4(v[0], v[1], v[2], v[3]));
+                    } else {
+                        for (uint32_t j = 0; j < 4 && c + j < mm; ++j)
+                            gp[c + j] = kAcc ? __fadd_rn(gp[c + j], v[j]) : v[j];
+                    }
+                }
+            }
+        }
+        if (bad) atomicOr(a.status, QSGD_ST_BAD_STREAM);
+        __syncwarp();
+    }
+}
+
+// Words of one staging row: room for d codes and a padding byte, rounded so that
+// consecutive rows start on consecutive banks (stride = 1 mod 32).
+uint32_t rows_stride_words(uint32_t d) {
+    const uint32_t need = (d + 4 + 3) / 4;
+    return ((need + 30) / 32) * 32 + 1;
+}
+
+template <int V, bool kAcc>
+cudaError_t launch_rows_v(const DecodeArgs& a, cudaStream_t stream) {
+    const uint32_t stride = rows_stride_words(a.d);
+    int dev = 0, sms = 0, optin = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    const size_t per_warp = static_cast<size_t>(32) * stride * sizeof(uint32_t);
+    const size_t lut_bytes = static_cast<size_t>(kLutSize) * sizeof(uint32_t);
+    const int W = static_cast<int>(std::min<size_t>(kRowsMaxWarps, (static_cast<size_t>(optin) - lut_bytes - 1024) / per_warp));
+    if (W < 1) return cudaErrorInvalidConfiguration;
+    const size_t smem = lut_bytes + W * per_warp;
+    static bool attr_set[64] = {};
+    if (dev < 64 && !attr_set[dev]) {
+        cudaFuncSetAttribute(decode_rows<V, kAcc>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+        attr_set[dev] = true;
+    }
+    const uint64_t groups = (a.nb + 31) / 32;
+    const uint64_t blocks = std::max<uint64_t>(1, std::min<uint64_t>(static_cast<uint64_t>(sms), (groups + W - 1) / W));
+    decode_rows<V, kAcc><<<static_cast<unsigned>(blocks), 32 * W, smem, stream>>>(a, stride);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool decode_rows_shape(uint32_t d, uint32_t s, const float* out) {
+    return d % 4 == 0 && d >= 4 && d <= kRowsMaxD && s <= kRowsMaxS && (reinterpret_cast<uintptr_t>(out) & 15u) == 0;
+}
+
+cudaError_t launch_decode_rows(const DecodeArgs& a, bool accumulate, cudaStream_t stream) {
+    switch (fast_v(a.d)) {
+        case 1: return accumulate ? launch_rows_v<1, true>(a, stream) : launch_rows_v<1, false>(a, stream);
+        case 2: return accumulate ? launch_rows_v<2, true>(a, stream) : launch_rows_v<2, false>(a, stream);
+        case 4: return accumulate ? launch_rows_v<4, true>(a, stream) : launch_rows_v<4, false>(a, stream);
+        default: return accumulate ? launch_rows_v<8, true>(a, stream) : launch_rows_v<8, false>(a, stream);
+    }
+}
+
+}  // namespace qsgd

@@ -1,0 +1,452 @@
+// QSGD encoder in two launches: a bucket coder and a stream compaction (sm_100a).
+//
+// Method: "QSGD (Quantized Stochastic Gradient Descent) with Elias Coding" (AIMech
+// curated entry).  Per bucket (claim "QSVRG, non-convex and multi-GPU bucketed
+// training", section 3.3 bucketing): the L2 norm, unbiased stochastic rounding of
+// every coordinate to one of s+1 levels (definition paragraph), and the Elias-omega
+// coding of the tuple (norm, signs, run-length gaps, levels) (definition paragraph;
+// claim "Elias coding communication complexity tradeoff", F = 32).
+//
+// 1. code_buckets: one warp per bucket, no warp waits for another.  The warp reads
+//    its bucket with coalesced 16-byte loads (lane L holds float4 L + 32j), computes
+//    the norm, draws one Philox block per four coordinates, quantises, and writes the
+//    bucket's bits (norm, then the records in index order) into the bucket's own
+//    slot of a staging area in the workspace, at bucket-local bit offsets, together
+//    with the bucket's bit count.  A slot holds the bucket's largest possible size.
+// 2. compact_stream: one CTA per 256 buckets scans the bit counts (a block scan and a
+//    decoupled look-back over the CTAs, Merrill & Garland 2016), writes the offsets
+//    header, and moves every bucket's bits to their stream position with funnel
+//    shifts.  An output word belongs to the bucket that holds its first bit; that
+//    bucket's warp also reads the first bits of the next bucket, so every word has
+//    exactly one writer and the output needs no clearing.
+// The staging costs two extra passes over the compressed bytes (a few percent of
+// the input bytes) and buys an encoder with no inter-CTA waits in its long kernel.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+
+#include "../../include/qsgd.h"
+#include "qsgd_device.cuh"
+#include "qsgd_internal.h"
+
+namespace qsgd {
+namespace {
+
+constexpr uint32_t kAll = 0xFFFFFFFFu;
+
+// Whole records omega(gap) | sign | omega(k) for gap < 64 and k < 32, indexed by
+// gap << 6 | k << 1 | sign: entry = code << 5 | length (length <= 24 bits).
+struct RecordTable64 {
+    uint32_t v[kRecordTab64];
+};
+constexpr RecordTable64 make_record_table64() {
+    RecordTable64 t{};
+    const OmegaTable om = make_omega_table();
+    for (uint32_t gap = 1; gap < 64; ++gap)
+        for (uint32_t k = 1; k < 32; ++k)
+            for (uint32_t sign = 0; sign < 2; ++sign) {
+                const uint32_t ge = om.v[gap], ke = om.v[k];
+                const uint32_t kl = ke & 0xFFu;
+                const uint32_t code = ((((ge >> 8) << 1) | sign) << kl) | (ke >> 8);
+                const uint32_t len = (ge & 0xFFu) + 1u + kl;
+                t.v[(gap << 6) | (k << 1) | sign] = (code << 5) | len;
+            }
+    return t;
+}
+__device__ const RecordTable64 kRecordTable64Global = make_record_table64();
+
+// Philox4x32-10 of counter (j, 0, 0, 0) with the round keys precomputed on the host
+// (rk[2r], rk[2r+1] = the seed advanced r times by the Weyl constants).  The
+// counter's high words are zero because j = i / 4 < 2^32 for every coordinate.
+__device__ __forceinline__ uint4 philox_rk(uint32_t j, const uint32_t* rk) {
+    uint32_t c0 = j, c1 = 0u, c2 = 0u, c3 = 0u;
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+        const uint64_t pa = static_cast<uint64_t>(c0) * 0xD2511F53u;
+        const uint64_t pb = static_cast<uint64_t>(c2) * 0xCD9E8D57u;
+        c0 = static_cast<uint32_t>(pb >> 32) ^ c1 ^ rk[2 * r];
+        c2 = static_cast<uint32_t>(pa >> 32) ^ c3 ^ rk[2 * r + 1];
+        c1 = static_cast<uint32_t>(pb);
+        c3 = static_cast<uint32_t>(pa);
+    }
+    return make_uint4(c0, c1, c2, c3);
+}
+
+// The level k = min(floor(t) + [u < p], s) of one coordinate, t = fl(|v| sinv),
+// p = t - floor(t), u = floor(r / 2^9) 2^-23 (definition paragraph; fp32 order of
+// the wire format).  Exact rewrite of the comparison: with f = RD(t + 2^23) =
+// 2^23 + floor(t) (exact for 0 <= t < 2^23), the sum t + (2^23 + 1 - f) is exactly
+// 1 + p, and 1 + u lies on the fp32 grid of [1, 2); so u < p holds exactly when
+// 1 + u < RU(1 + p).
+__device__ __forceinline__ uint32_t level_of(float v, float sinv, uint32_t r, uint32_t s) {
+    const float t = __fmul_rn(fabsf(v), sinv);
+    const float f = __fadd_rd(t, 8388608.0f);
+    const float w = __fadd_ru(t, __fsub_rn(8388609.0f, f));
+    const float u1 = __uint_as_float(0x3F800000u | (r >> 9));
+    const uint32_t k = (__float_as_uint(f) - 0x4B000000u) + (u1 < w ? 1u : 0u);
+    return k < s ? k : s;
+}
+
+// ORs the len (1..32) low bits of code, MSB-first, into the zeroed bit buffer at
+// bit position pos.
+__device__ __forceinline__ void put_bits(uint32_t* buf, uint32_t pos, uint32_t code, uint32_t len) {
+    const uint32_t w = pos >> 5, sh = pos & 31u;
+    const uint64_t v = static_cast<uint64_t>(code) << (64u - len - sh);
+    atomicOr(&buf[w], static_cast<uint32_t>(v >> 32));
+    if (static_cast<uint32_t>(v) != 0u) atomicOr(&buf[w + 1], static_cast<uint32_t>(v));
+}
+
+// The same for len (1..64) bits.
+__device__ __forceinline__ void put_bits64(uint32_t* buf, uint32_t pos, uint64_t code, uint32_t len) {
+    if (len > 32) {
+        put_bits(buf, pos, static_cast<uint32_t>(code >> 32), len - 32);
+        pos += len - 32;
+        len = 32;
+    }
+    put_bits(buf, pos, static_cast<uint32_t>(code), len);
+}
+
+// Stores one lane's 4V values (float4 L + 32j of a bucket of m values at p) with
+// streaming stores; nothing past m is written.
+template <int V>
+__device__ __forceinline__ void store_lane(float* p, int lane, uint32_t m, const float (&v)[4 * V]) {
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+        const uint32_t i = 4u * (static_cast<uint32_t>(lane) + 32u * j);
+        if (i + 4 <= m) {
+            __stcs(reinterpret_cast<float4*>(p + i), make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
+        } else if (i < m) {
+            __stcs(p + i, v[4 * j]);
+            if (i + 1 < m) __stcs(p + i + 1, v[4 * j + 1]);
+            if (i + 2 < m) __stcs(p + i + 2, v[4 * j + 2]);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// 1. Bucket coder.  kShort: s <= 31, records of gap < 64 through the whole-record
+// table (the others from the omega table), every record <= 30 bits.  Otherwise every
+// record from the omega table (or computed for k >= 2048), up to 18 + 1 + 34 bits.
+// ---------------------------------------------------------------------------
+template <int V, bool kShort, bool kEF>
+__global__ void __launch_bounds__(kStageBlock) code_buckets(const __grid_constant__ StageArgs a) {
+    extern __shared__ __align__(16) uint32_t smem[];
+    constexpr int NC = 4 * V;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    uint32_t* const otab = smem;                                                  // omega table
+    uint32_t* const rtab = smem + kOmegaTab;                                      // record table (kShort)
+    uint32_t* const buf = smem + kOmegaTab + (kShort ? kRecordTab64 : 0) + warp * a.buf_words;  // this warp's bucket bits
+    omega_table_fill(otab, tid, kStageBlock);
+    if constexpr (kShort) {
+        const uint4* src = reinterpret_cast<const uint4*>(kRecordTable64Global.v);
+        for (int i = tid; i < kRecordTab64 / 4; i += kStageBlock) reinterpret_cast<uint4*>(rtab)[i] = src[i];
+    }
+    for (uint32_t i = lane; i < a.buf_words; i += 32) buf[i] = 0u;
+    // the compaction's scan state for this call: cleared here, before it runs
+    {
+        const uint64_t gt = static_cast<uint64_t>(blockIdx.x) * kStageBlock + tid;
+        for (uint64_t i = gt; i < a.ntiles; i += static_cast<uint64_t>(gridDim.x) * kStageBlock) a.cdesc[i] = 0;
+        if (gt == 0) {
+            a.ctrl->ticket = 0;
+            a.ctrl->abort = 0;
+        }
+    }
+    __syncthreads();
+
+    const uint32_t d = a.d;
+    const uint64_t gwarps = static_cast<uint64_t>(gridDim.x) * kStageWarps;
+    for (uint64_t b = static_cast<uint64_t>(blockIdx.x) * kStageWarps + warp; b < a.nb; b += gwarps) {
+        const uint64_t base = b * d;
+        const uint32_t m = static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - base));
+        // --- the bucket: lane L holds float4 f = L + 32j (coordinates 4f..4f+3) ----
+        float x[NC];
+        float ev[kEF ? NC : 1];
+#pragma unroll
+        for (int j = 0; j < V; ++j) {
+            const uint32_t i = 4u * (static_cast<uint32_t>(lane) + 32u * j);
+            float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
+            float4 e = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (i + 4 <= m) {
+                q = __ldcs(reinterpret_cast<const float4*>(a.in + base + i));
+                if constexpr (kEF) e = __ldcs(reinterpret_cast<const float4*>(a.ef + base + i));
+            } else if (i < m) {  // the ragged end of the last bucket
+                q.x = a.in[base + i];
+                if (i + 1 < m) q.y = a.in[base + i + 1];
+                if (i + 2 < m) q.z = a.in[base + i + 2];
+                if constexpr (kEF) {
+                    e.x = a.ef[base + i];
+                    if (i + 1 < m) e.y = a.ef[base + i + 1];
+                    if (i + 2 < m) e.z = a.ef[base + i + 2];
+                }
+            }
+            x[4 * j + 0] = q.x;
+            x[4 * j + 1] = q.y;
+            x[4 * j + 2] = q.z;
+            x[4 * j + 3] = q.w;
+            if constexpr (kEF) {
+                ev[4 * j + 0] = e.x;
+                ev[4 * j + 1] = e.y;
+                ev[4 * j + 2] = e.z;
+                ev[4 * j + 3] = e.w;
+            }
+        }
+        if constexpr (kEF) {  // p = e + g
+#pragma unroll
+            for (int q = 0; q < NC; ++q) x[q] = __fadd_rn(ev[q], x[q]);
+        }
+        const float norm = a.norm_kind == QSGD_NORM_MAX ? warp_bucket_maxnorm<NC>(x) : warp_bucket_norm<NC>(x, true);
+        const BucketScale sc = bucket_scale(norm, a.s, true, a.status, lane == 0);
+        if (!sc.good) {  // sent as a zero bucket; the memory keeps p
+            if constexpr (kEF) store_lane<V>(a.ef + base, lane, m, x);
+#pragma unroll
+            for (int q = 0; q < NC; ++q) x[q] = 0.f;
+        }
+        // --- levels: one Philox block per float4 ----------------------------------
+        uint32_t kq[NC];  // level | sign << 31
+        const uint32_t j0 = static_cast<uint32_t>(base >> 2) + static_cast<uint32_t>(lane);
+#pragma unroll
+        for (int j = 0; j < V; ++j) {
+            const uint4 r = philox_rk(j0 + 32u * j, a.rk);
+            const uint32_t rw[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const float v = x[4 * j + c];
+                kq[4 * j + c] = level_of(v, sc.sinv, rw[c], a.s) | (__float_as_uint(v) & 0x80000000u);
+            }
+        }
+        if constexpr (kEF) {  // the memory keeps p minus what a receiver decodes
+            if (sc.good) {
+                const float scale = __fdiv_rn(sc.sent, __uint2float_rn(a.s));
+#pragma unroll
+                for (int q = 0; q < NC; ++q) ev[q] = ef_residual(x[q], kq[q] & 0x7FFFFFFFu, kq[q] >> 31, scale);
+                store_lane<V>(a.ef + base, lane, m, ev);
+            }
+        }
+        // --- records, run by run: run j is coordinates [128j, 128j + 128) ----------
+        if (lane == 0) buf[0] = __float_as_uint(sc.sent);
+        uint32_t pos = 32u;      // bucket-local bit where the current run starts
+        int32_t carry = -1;      // last record's index before the current run
+#pragma unroll
+        for (int j = 0; j < V; ++j) {
+            const uint32_t qb = 4u * (static_cast<uint32_t>(lane) + 32u * j);
+            uint32_t m4 = 0;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) m4 |= ((kq[4 * j + c] & 0x7FFFFFFFu) != 0u ? 1u : 0u) << c;
+            const int32_t last = m4 ? static_cast<int32_t>(qb + 31u - __clz(m4)) : -1;
+            const uint32_t B = __ballot_sync(kAll, m4 != 0u);
+            const uint32_t lower = B & ((1u << lane) - 1u);
+            const int32_t pv = __shfl_sync(kAll, last, lower ? 31 - __clz(lower) : 0);
+            int32_t prev = lower ? pv : carry;
+            carry = B ? __shfl_sync(kAll, last, 31 - __clz(B)) : carry;
+            // the lane's records of this run: codes and their total length
+            uint32_t code[4], len[4];
+            uint64_t kcode[kShort ? 1 : 4];
+            uint32_t klen[kShort ? 1 : 4];
+            uint32_t lbits = 0;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const uint32_t kv = kq[4 * j + c];
+                const uint32_t k = kv & 0x7FFFFFFFu;
+                const uint32_t gap = static_cast<uint32_t>(static_cast<int32_t>(qb + c) - prev);
+                code[c] = 0;
+                len[c] = 0;
+                if constexpr (!kShort) {
+                    kcode[c] = 0;
+                    klen[c] = 0;
+                }
+                if (k != 0u) {
+                    prev = static_cast<int32_t>(qb + c);
+                    if constexpr (kShort) {
+                        if (gap < 64u) {
+                            const uint32_t e = rtab[(gap << 6) | __funnelshift_l(kv, kv, 1)];
+                            code[c] = e >> 5;
+                            len[c] = e & 31u;
+                        } else {  // omega(gap) from the table (gap <= d <= 1024), then sign, omega(k)
+                            const uint32_t ge = otab[gap], ke = otab[k];
+                            const uint32_t kl = ke & 0xFFu;
+                            code[c] = ((((ge >> 8) << 1) | (kv >> 31)) << kl) | (ke >> 8);
+                            len[c] = (ge & 0xFFu) + 1u + kl;
+                        }
+                    } else {
+                        const uint32_t ge = otab[gap];
+                        code[c] = ((ge >> 8) << 1) | (kv >> 31);
+                        len[c] = (ge & 0xFFu) + 1u;
+                        if (k < static_cast<uint32_t>(kOmegaTab)) {
+                            const uint32_t ke = otab[k];
+                            kcode[c] = ke >> 8;
+                            klen[c] = ke & 0xFFu;
+                        } else {
+                            omega_compute(k, kcode[c], klen[c]);
+                        }
+                    }
+                }
+                lbits += len[c];
+                if constexpr (!kShort) lbits += klen[c];
+            }
+            // the lane's first bit in the run: exclusive scan of the lane lengths
+            uint32_t incl = lbits;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t t = __shfl_up_sync(kAll, incl, o);
+                if (lane >= o) incl += t;
+            }
+            uint32_t p = pos + incl - lbits;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                if (len[c] != 0u) {
+                    put_bits(buf, p, code[c], len[c]);
+                    p += len[c];
+                    if constexpr (!kShort) {
+                        put_bits64(buf, p, kcode[c], klen[c]);
+                        p += klen[c];
+                    }
+                }
+            }
+            pos += __shfl_sync(kAll, incl, 31);
+        }
+        __syncwarp();
+        // --- the bucket's bits into its staging slot; the buffer cleared again -----
+        uint32_t* const slot = a.stage + b * a.slot_words;
+        const uint32_t nw = (pos + 31u) >> 5;
+        for (uint32_t i = lane; i < nw; i += 32) {
+            slot[i] = buf[i];
+            buf[i] = 0u;
+        }
+        if (lane == 0) a.bits[b] = pos;
+        __syncwarp();
+    }
+}
+
+// ---------------------------------------------------------------------------
+// 2. Compaction: offsets header and the stream at its final bit positions.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kCompactBlock) compact_stream(const __grid_constant__ StageArgs a) {
+    __shared__ uint64_t s_F[kCompactBlock];
+    __shared__ uint32_t s_L[kCompactBlock];
+    __shared__ uint32_t s_warp[kCompactBlock / 32];
+    __shared__ uint32_t s_tile;
+    __shared__ uint64_t s_X;
+    __shared__ int s_ok;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) s_tile = atomicAdd(&a.ctrl->ticket, 1u);  // tiles in scheduling order
+    __syncthreads();
+    const uint64_t tile = s_tile;
+    const uint64_t b0 = tile * kCompactBlock;
+    const uint64_t b = b0 + tid;
+    const uint32_t L = b < a.nb ? a.bits[b] : 0u;
+    // block scan of the bucket sizes (a tile is at most 256 * 2^21 bits... far below 2^32)
+    uint32_t incl = L;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t t = __shfl_up_sync(kAll, incl, o);
+        if (lane >= o) incl += t;
+    }
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    uint32_t before = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < kCompactBlock / 32; ++w) {
+        const uint32_t x = s_warp[w];
+        before += w < warp ? x : 0u;
+        total += x;
+    }
+    const uint32_t excl = before + incl - L;
+    if (warp == 0) {
+        uint64_t X = 0;
+        bool ok = true;
+        if (tile == 0) {
+            if (lane == 0) st_release(&a.cdesc[0], make_desc(0, kStatePrefix, total));
+        } else {
+            if (lane == 0) st_release(&a.cdesc[tile], make_desc(0, kStateAggregate, total));
+            ok = lookback(a.cdesc, static_cast<uint32_t>(tile), 0, &a.ctrl->abort, X);
+            if (lane == 0 && ok) st_release(&a.cdesc[tile], make_desc(0, kStatePrefix, X + total));
+        }
+        if (lane == 0) {
+            s_X = X;
+            s_ok = ok;
+            if (!ok) {
+                report(a.status, QSGD_ST_LOOKBACK_TIMEOUT);
+                atomicExch(&a.ctrl->abort, 1u);
+            }
+        }
+    }
+    __syncthreads();
+    if (!s_ok) return;
+    const uint64_t X = s_X;
+    const uint64_t F = X + excl;
+    s_F[tid] = F;
+    s_L[tid] = L;
+    if (b < a.nb) a.offsets[b] = F;
+    if (b + 1 == a.nb) a.offsets[a.nb] = F + L;
+    __syncthreads();
+    // bucket i of the tile: the words whose first bit lies in it
+    const uint64_t nt = min(static_cast<uint64_t>(kCompactBlock), a.nb - b0);
+    for (uint32_t i = warp; i < nt; i += kCompactBlock / 32) {
+        const uint64_t bb = b0 + i;
+        const uint64_t Fb = s_F[i];
+        const uint32_t Lb = s_L[i];
+        const uint32_t* src = a.stage + bb * a.slot_words;
+        const uint32_t nsw = (Lb + 31u) >> 5;
+        const uint64_t w_begin = (Fb + 31u) >> 5, w_end = (Fb + Lb + 31u) >> 5;
+        for (uint64_t w = w_begin + lane; w < w_end; w += 32) {
+            const uint32_t r = static_cast<uint32_t>(32u * w - Fb);
+            const uint32_t q = r >> 5, sh = r & 31u;
+            const uint32_t a0 = src[q];
+            const uint32_t a1 = q + 1 < nsw ? src[q + 1] : 0u;
+            uint32_t v = __funnelshift_l(a1, a0, sh);
+            if (r + 32u > Lb) {  // the word runs into the next bucket: its first bits
+                const uint32_t hd = bb + 1 < a.nb ? a.stage[(bb + 1) * a.slot_words] : 0u;
+                v |= hd >> (Lb - r);
+            }
+            if (w < a.cap_words)
+                a.words[w] = v;
+            else
+                report(a.status, QSGD_ST_OVERFLOW);
+        }
+    }
+}
+
+template <int V, bool kShort, bool kEF>
+cudaError_t launch_code(const StageArgs& a, cudaStream_t stream) {
+    const size_t smem = stage_smem_bytes(a.s, a.buf_words);
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr_set[dev]) {
+        cudaFuncSetAttribute(code_buckets<V, kShort, kEF>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+        attr_set[dev] = true;
+    }
+    int sms = 0, per_sm = 0;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, code_buckets<V, kShort, kEF>, kStageBlock, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    const uint64_t want = (a.nb + kStageWarps - 1) / kStageWarps;
+    const uint64_t grid = std::max<uint64_t>(1, std::min<uint64_t>(want, static_cast<uint64_t>(sms) * per_sm));
+    code_buckets<V, kShort, kEF><<<static_cast<unsigned>(grid), kStageBlock, smem, stream>>>(a);
+    return cudaGetLastError();
+}
+
+template <int V>
+cudaError_t launch_code_v(const StageArgs& a, cudaStream_t stream) {
+    const bool sh = a.s <= kStageShortMaxS;
+    if (a.ef) return sh ? launch_code<V, true, true>(a, stream) : launch_code<V, false, true>(a, stream);
+    return sh ? launch_code<V, true, false>(a, stream) : launch_code<V, false, false>(a, stream);
+}
+
+}  // namespace
+
+cudaError_t launch_encode_stage(const StageArgs& a, cudaStream_t stream) {
+    cudaError_t e;
+    switch (stage_v(a.d)) {
+        case 1: e = launch_code_v<1>(a, stream); break;
+        case 2: e = launch_code_v<2>(a, stream); break;
+        case 4: e = launch_code_v<4>(a, stream); break;
+        default: e = launch_code_v<8>(a, stream); break;
+    }
+    if (e != cudaSuccess) return e;
+    compact_stream<<<static_cast<unsigned>(a.ntiles), kCompactBlock, 0, stream>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace qsgd

@@ -83,6 +83,59 @@ inline size_t fast_smem_bytes(uint32_t d, uint32_t s, uint32_t smem_words) {
            sizeof(uint32_t);
 }
 
+// Two-launch encoder (qsgd_encode_stage.cu): the bucket coder writes every bucket's
+// bits into its own staging slot and its bit count; the compaction scans the counts
+// and writes the offsets header and the stream.
+struct StageArgs {
+    const float* in;
+    float* ef;            // error-feedback memory fused into the bucket coder, or null
+    uint64_t n;
+    uint32_t d, s, norm_kind;
+    uint32_t rk[20];      // Philox round keys: the seed advanced r times by the Weyl constants
+    uint64_t nb;
+    uint32_t slot_words;  // staging words per bucket (its largest size)
+    uint32_t buf_words;   // shared-memory words of one warp's bucket buffer
+    uint32_t* stage;      // nb * slot_words
+    uint32_t* bits;       // nb bucket sizes in bits
+    uint32_t* status;
+    uint32_t* words;
+    uint64_t cap_words;
+    uint64_t* offsets;
+    ScanControl* ctrl;
+    uint64_t* cdesc;      // compaction scan descriptor per tile of kCompactBlock buckets
+    uint64_t ntiles;
+};
+
+// Workspace of the two-launch encoder: [0, 256) control block; the compaction's
+// descriptors; the bucket sizes; the staging slots.
+struct StageLayout {
+    size_t desc_off, bits_off, stage_off, total;
+    uint64_t ntiles;
+    uint32_t slot_words;
+};
+StageLayout stage_layout(uint64_t n, uint32_t d, uint32_t s);
+
+// Float4s per lane of the bucket coder (a power of two >= d/128).
+inline uint32_t stage_v(uint32_t d) { return fast_v(d); }
+// Dynamic shared memory of the bucket coder: omega table | record table (s <= 31) |
+// one bucket buffer per warp.
+inline size_t stage_smem_bytes(uint32_t s, uint32_t buf_words) {
+    return (static_cast<size_t>(kOmegaTab) + (s <= kStageShortMaxS ? kRecordTab64 : 0) +
+            static_cast<size_t>(kStageWarps) * buf_words) *
+           sizeof(uint32_t);
+}
+inline bool stage_shape(uint32_t d) { return d >= kStageMinD && d <= kStageMaxD && d % 4 == 0; }
+cudaError_t launch_encode_stage(const StageArgs& a, cudaStream_t stream);
+
+// The encode entry behind qsgd_encode_ex and qsgd_encode_ef (d_ef null or the
+// memory).  strict: the workspace must hold qsgd_encode_workspace_bytes; otherwise
+// the one-pass encoders run when the two-launch layout does not fit.
+int encode_entry(const float* d_in, float* d_ef, uint64_t n, uint32_t d, uint32_t s, uint64_t seed,
+                 uint32_t norm_kind, uint32_t* d_words, uint64_t words_capacity, uint64_t* d_offsets, void* d_ws,
+                 size_t ws_bytes, uint32_t* d_status, cudaStream_t stream, bool strict);
+// Workspace of the one-pass encoders alone (their scan state).
+size_t min_encode_workspace_bytes(uint64_t n, uint32_t d, uint32_t s);
+
 struct StreamRef {
     const uint32_t* words;
     uint64_t num_words;
@@ -104,6 +157,9 @@ struct DecodeArgs {
 };
 
 cudaError_t launch_decode(const DecodeArgs& a, bool accumulate, cudaStream_t stream);
+// The one-stream decoder with whole rows staged as byte codes (qsgd_decode_rows.cu).
+bool decode_rows_shape(uint32_t d, uint32_t s, const float* out);
+cudaError_t launch_decode_rows(const DecodeArgs& a, bool accumulate, cudaStream_t stream);
 // Whether the one-lane-per-bucket decoders (and the several-stream kernel, which
 // start_zero / div need) take this shape.
 bool decode_fast_shape(uint32_t d, uint32_t s, const float* out);

@@ -12,6 +12,7 @@ constexpr uint64_t kMaxStreamBits = (uint64_t(1) << 38) - 1;  // scan descriptor
 
 constexpr int kOmegaTab = 2048;               // omega code table entries (N < 2048)
 constexpr int kRecordTab = 2048;              // record table: gap < 64, k < 16, sign
+constexpr int kRecordTab64 = 4096;            // record table of the bucket coder: gap < 64, k < 32, sign
 constexpr uint32_t kMaxPolls = 1u << 22;      // bound of every spin wait (~1 s)
 
 constexpr int kBlock = 256;                   // threads per CTA, every encode kernel
@@ -42,6 +43,23 @@ constexpr int kFastBlock = 32 * kFastWarps;
 #endif
 __host__ __device__ constexpr int enc_depth(unsigned v) { return v <= 4 ? QSGD_ENC_DEPTH : 1; }
 constexpr int kFastMinBlocks = QSGD_FAST_MIN_BLOCKS;
+
+// Two-launch encoder (bucket coder + compaction): 4 <= d <= 1024, d % 4 == 0,
+// 16-byte aligned input; one warp per bucket, kStageWarps warps per CTA; the
+// compaction takes kCompactBlock buckets per CTA.  Whole-record table for s <= 31.
+constexpr int kStageWarps = 8;
+constexpr int kStageBlock = 32 * kStageWarps;
+constexpr int kCompactBlock = 256;
+constexpr uint32_t kStageMinD = 4;
+constexpr uint32_t kStageMaxD = 1024;
+constexpr uint32_t kStageShortMaxS = 31;
+
+// One-stream decoder with byte codes staged in whole bucket rows: d % 4 == 0,
+// 4 <= d <= 1024, s <= 127 (a code is sign << 7 | k), 16-byte aligned output; up to
+// kRowsMaxWarps warps (32 buckets each) to a CTA, as many as the shared memory holds.
+constexpr int kRowsMaxWarps = 16;
+constexpr uint32_t kRowsMaxD = 1024;
+constexpr uint32_t kRowsMaxS = 127;
 
 constexpr int kDecodeBlock = 128;
 constexpr int kMaxStreamsPerLaunch = 16;  // decode-accumulate streams per launch

@@ -52,14 +52,16 @@ size_t qsgd_static_workspace_limit(void) { return kStaticWorkspaceBytes; }
 int qsgd_encode_static_ws(const float* d_in, uint64_t n, uint32_t d, uint32_t s, uint64_t seed,
                           uint32_t* d_words, uint64_t words_capacity, uint64_t* d_offsets,
                           uint32_t* d_status, cudaStream_t stream) {
-    const size_t need = qsgd_encode_workspace_bytes(n, d, s);
+    // the one-pass encoders' scan state must fit; the two-launch encoder runs when its
+    // staging fits as well
+    const size_t need = qsgd::min_encode_workspace_bytes(n, d, s);
     if (need == 0) return QSGD_ERR_ARG;
     if (need > kStaticWorkspaceBytes) return QSGD_ERR_STATIC_LIMIT;
     void* ws = nullptr;
     const int rc = static_ws_address(&ws);
     if (rc != QSGD_OK) return rc;
-    return qsgd_encode(d_in, n, d, s, seed, d_words, words_capacity, d_offsets, ws, kStaticWorkspaceBytes,
-                       d_status, stream);
+    return qsgd::encode_entry(d_in, nullptr, n, d, s, seed, QSGD_NORM_L2, d_words, words_capacity, d_offsets, ws,
+                              kStaticWorkspaceBytes, d_status, stream, false);
 }
 
 }  // extern "C"

@@ -20,6 +20,7 @@
 #include <memory>
 #include <mutex>
 #include <thread>
+#include <type_traits>
 #include <vector>
 
 #define __device__
@@ -59,6 +60,19 @@ inline float __fadd_rd(float a, float b) {
     volatile float r = x + y;
     std::fesetround(old);
     return r;
+}
+inline float __fadd_ru(float a, float b) {
+    const int old = std::fegetround();
+    std::fesetround(FE_UPWARD);
+    volatile float x = a, y = b;
+    volatile float r = x + y;
+    std::fesetround(old);
+    return r;
+}
+// the high word of (hi:lo) << (sh mod 32)
+inline uint32_t __funnelshift_l(uint32_t lo, uint32_t hi, uint32_t sh) {
+    const uint64_t x = (static_cast<uint64_t>(hi) << 32) | lo;
+    return static_cast<uint32_t>((x << (sh & 31u)) >> 32);
 }
 inline float __uint2float_rn(uint32_t u) { return static_cast<float>(u); }
 inline float __uint_as_float(uint32_t u) { float f; std::memcpy(&f, &u, 4); return f; }
@@ -103,6 +117,7 @@ struct WarpSync {
     int arrived = 0;
     uint64_t gen = 0;
     int site[32];
+    int arg[32];
     uint64_t val[32];
     uint64_t out[32];
 };
@@ -150,6 +165,7 @@ inline uint64_t emu_warp(int op, int line, uint64_t v, int arg, int width) {
     const uint64_t my_gen = w.gen;
     w.site[lane] = line * 8 + (op & 7);
     w.val[lane] = v;
+    w.arg[lane] = arg;
     if (++w.arrived == 32) {
         for (int i = 1; i < 32; ++i)
             if (w.site[i] != w.site[0]) {
@@ -169,9 +185,10 @@ inline uint64_t emu_warp(int op, int line, uint64_t v, int arg, int width) {
             switch (op) {
                 case 0: w.out[i] = any; break;
                 case 1: w.out[i] = ballot; break;
-                case 4: w.out[i] = (pos >= arg) ? w.val[i - arg] : w.val[i]; break;
-                case 5: w.out[i] = w.val[seg + (arg % width)]; break;
-                case 7: w.out[i] = ((pos ^ arg) < width) ? w.val[seg + (pos ^ arg)] : w.val[i]; break;
+                // each lane's own offset, source lane or mask
+                case 4: w.out[i] = (pos >= w.arg[i]) ? w.val[i - w.arg[i]] : w.val[i]; break;
+                case 5: w.out[i] = w.val[seg + (w.arg[i] % width)]; break;
+                case 7: w.out[i] = ((pos ^ w.arg[i]) < width) ? w.val[seg + (pos ^ w.arg[i])] : w.val[i]; break;
                 default: w.out[i] = 0;
             }
         }
@@ -184,7 +201,11 @@ inline uint64_t emu_warp(int op, int line, uint64_t v, int arg, int width) {
     }
     return w.out[lane];
 }
-template <class T> inline T emu_cast(uint64_t x) { T t; std::memcpy(&t, &x, sizeof(T)); return t; }
+template <class T> inline std::remove_cv_t<T> emu_cast(uint64_t x) {
+    std::remove_cv_t<T> t;
+    std::memcpy(&t, &x, sizeof(T));
+    return t;
+}
 template <class T> inline uint64_t emu_bits(T v) { uint64_t x = 0; std::memcpy(&x, &v, sizeof(T)); return x; }
 inline int emu_width() { return 32; }
 inline int emu_width(int w) { return w; }

@@ -1,0 +1,100 @@
+// Runs the one-stream row decoder decode_rows, compiled for the host under
+// block_emu.h, with all its CTAs at once.
+// argv: dir accumulate grid warps
+// dir holds params.bin (u64 n, d, s), w0.bin (u32 stream words), o0.bin (u64[nb+1])
+// and out_in.bin (fp32[n], the output before the call).  It writes out.bin and
+// prints the status word.
+#include "block_emu.h"
+thread_local dim3e threadIdx, blockIdx;
+dim3e gridDim, blockDim;
+thread_local BlockCtx* t_blk;
+std::atomic<int> g_emu_error{0};
+#include "rows_emu.inc"  // the kernel source, prepared by the test
+#include <string>
+
+static std::vector<unsigned char> slurp(const std::string& p) {
+    FILE* f = std::fopen(p.c_str(), "rb");
+    if (!f) { std::perror(p.c_str()); std::exit(2); }
+    std::fseek(f, 0, SEEK_END); long n = std::ftell(f); std::fseek(f, 0, SEEK_SET);
+    std::vector<unsigned char> b(n);
+    if (n && std::fread(b.data(), 1, n, f) != (size_t)n) std::exit(2);
+    std::fclose(f);
+    return b;
+}
+static void spit(const std::string& p, const void* data, size_t bytes) {
+    FILE* f = std::fopen(p.c_str(), "wb");
+    std::fwrite(data, 1, bytes, f);
+    std::fclose(f);
+}
+
+template <class Kernel>
+static void run_grid(unsigned grid, unsigned block, size_t smem, Kernel k) {
+    gridDim = {grid, 1, 1};
+    blockDim = {block, 1, 1};
+    std::vector<std::unique_ptr<BlockCtx>> blocks;
+    for (unsigned b = 0; b < grid; ++b) {
+        blocks.emplace_back(new BlockCtx());
+        blocks.back()->smem.assign(smem + 64, 0xAB);  // garbage, like real shared memory
+    }
+    std::vector<std::thread> th;
+    for (unsigned b = 0; b < grid; ++b)
+        for (unsigned t = 0; t < block; ++t)
+            th.emplace_back([&, b, t] {
+                t_blk = blocks[b].get();
+                threadIdx = {t, 0, 0};
+                blockIdx = {b, 0, 0};
+                k();
+            });
+    for (auto& x : th) x.join();
+}
+
+template <int V>
+static void run(const qsgd::DecodeArgs& a, bool acc, unsigned grid, unsigned W, uint32_t stride, size_t smem) {
+    if (acc)
+        run_grid(grid, 32 * W, smem, [&] { qsgd::decode_rows<V, true>(a, stride); });
+    else
+        run_grid(grid, 32 * W, smem, [&] { qsgd::decode_rows<V, false>(a, stride); });
+}
+
+int main(int argc, char** argv) {
+    const std::string dir = argv[1];
+    const bool acc = std::atoi(argv[2]) != 0;
+    const unsigned grid = std::atoi(argv[3]), W = std::atoi(argv[4]);
+    auto prm = slurp(dir + "/params.bin");
+    uint64_t q[3];
+    std::memcpy(q, prm.data(), sizeof q);
+    const uint64_t n = q[0];
+    const uint32_t d = (uint32_t)q[1], s = (uint32_t)q[2];
+    const uint64_t nb = (n + d - 1) / d;
+    auto wb = slurp(dir + "/w0.bin");
+    auto ob = slurp(dir + "/o0.bin");
+    auto xb = slurp(dir + "/out_in.bin");
+    std::vector<uint32_t> words(wb.size() / 4 + 1);
+    std::memcpy(words.data(), wb.data(), wb.size());
+    std::vector<uint64_t> offsets(nb + 1);
+    std::memcpy(offsets.data(), ob.data(), 8 * (nb + 1));
+    std::vector<float> out(n + 4);
+    std::memcpy(out.data(), xb.data(), 4 * n);
+    uint32_t status = 0;
+    qsgd::DecodeArgs a{};
+    a.streams[0].words = words.data();
+    a.streams[0].num_words = wb.size() / 4;
+    a.streams[0].offsets = offsets.data();
+    a.K = 1;
+    a.n = n; a.d = d; a.s = s; a.nb = nb;
+    a.out = out.data();
+    a.status = &status;
+    a.first_group = 1;
+    const uint32_t stride = qsgd::rows_stride_words(d);
+    const size_t smem = 4 * (size_t)qsgd::kLutSize + (size_t)W * 32 * stride * 4;
+    switch (qsgd::fast_v(d)) {
+        case 1: run<1>(a, acc, grid, W, stride, smem); break;
+        case 2: run<2>(a, acc, grid, W, stride, smem); break;
+        case 4: run<4>(a, acc, grid, W, stride, smem); break;
+        default: run<8>(a, acc, grid, W, stride, smem); break;
+    }
+    if (g_emu_error) return 4;
+    spit(dir + "/out.bin", out.data(), 4 * n);
+    std::printf("status %u\n", status);
+    return 0;
+}

@@ -23,6 +23,7 @@ def host_source(text: str) -> str:
          "v = __atomic_load_n(p, __ATOMIC_RELAXED);"),
         (r'asm volatile\("ld\.acquire\.gpu\.global\.u32 %0, \[%1\];" : "=r"\(v\) : "l"\(p\) : "memory"\);',
          "v = __atomic_load_n(p, __ATOMIC_ACQUIRE);"),
+        (r'asm volatile\("prefetch\.global\.L2 \[%0\];" ::"l"\([^;]*\);', ";"),
         (r"extern __shared__ __align__\(16\) uint32_t smem\[\];",
          "uint32_t* smem = reinterpret_cast<uint32_t*>(emu_smem());"),
         (r"__shared__\s+([\w:<> ]+?)\s+(\w+)\s*(\[[^\]]*\])?\s*;", r"auto& \2 = emu_shared<\1\3>(__LINE__);"),

@@ -1,0 +1,132 @@
+"""The one-stream row decoder's exact source (decode_rows) on the CPU block emulator
+(no GPU).
+
+All CTAs of a launch run at once, every CUDA thread a host thread; warp primitives
+check that their 32 lanes meet at the same call site, and shared memory starts as
+garbage.  Streams come from the oracle's encoder; the output is compared bit for bit
+with the oracle's decode (or decode-accumulate onto an output holding -0.0 values).
+Bit flips in some buckets must be flagged, and every bucket no flip touched must
+still decode as the oracle decodes it."""
+
+import os
+import shutil
+import subprocess
+
+import numpy as np
+import pytest
+
+from emu_source import host_source as _host_source
+from quantized_gradient_compression_b200 import workloads as W
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+CSRC = os.path.join(ROOT, "quantized_gradient_compression_b200", "csrc")
+EMU = os.path.join(HERE, "emu", "enc")
+
+
+@pytest.fixture(scope="module")
+def rows_exe(tmp_path_factory):
+    if shutil.which("g++") is None:
+        pytest.skip("g++ not available")
+    d = tmp_path_factory.mktemp("rowsemu")
+    src_dir = d / "pkg" / "csrc"
+    src_dir.mkdir(parents=True)
+    shutil.copytree(os.path.join(ROOT, "include"), d / "include")
+    for h in ("qsgd_internal.h", "qsgd_limits.h"):
+        shutil.copy(os.path.join(CSRC, h), src_dir / h)
+    (src_dir / "qsgd_device.cuh").write_text(_host_source(open(os.path.join(CSRC, "qsgd_device.cuh")).read()))
+    src = open(os.path.join(CSRC, "qsgd_decode_rows.cu")).read()
+    cut = src.index("template <int V, bool kAcc>\ncudaError_t launch_rows_v")
+    (src_dir / "rows_emu.inc").write_text(_host_source(src[:cut]) + "}  // namespace\n}  // namespace qsgd\n")
+    exe = d / "rows_main"
+    r = subprocess.run(["g++", "-O1", "-std=c++17", "-ffp-contract=off", "-pthread", "-I", EMU, "-I", str(src_dir),
+                        os.path.join(EMU, "rows_main.cpp"), "-o", str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr[-4000:]
+    return str(exe)
+
+
+def _flip_bits(words, offsets, rng):
+    nb = offsets.size - 1
+    for b in rng.integers(0, nb, size=max(1, nb // 8)):
+        lo, hi = int(offsets[b]) + 32, int(offsets[b + 1])
+        if hi > lo:
+            for pos in rng.integers(lo, hi, size=3):
+                words[pos >> 5] ^= np.uint32(1) << np.uint32(31 - (pos & 31))
+
+
+def _run(exe, tmp, words, offsets, n, d, s, accumulate, grid, warps, base):
+    np.concatenate([words, np.zeros(1, np.uint32)]).tofile(tmp / "w0.bin")
+    offsets.astype(np.uint64).tofile(tmp / "o0.bin")
+    base.tofile(tmp / "out_in.bin")
+    np.array([n, d, s], np.uint64).tofile(tmp / "params.bin")
+    r = subprocess.run([exe, str(tmp), "1" if accumulate else "0", str(grid), str(warps)],
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, (r.stdout[-500:], r.stderr[-2000:])
+    return np.fromfile(tmp / "out.bin", np.float32), int(r.stdout.split()[-1])
+
+
+def _base(n, d, accumulate):
+    base = (np.random.default_rng(d).standard_normal(n) * 1e-3).astype(np.float32)
+    base[::5] = np.float32(-0.0)
+    if not accumulate:
+        base[:] = np.float32(np.nan)  # every coordinate must be written
+    return base
+
+
+# (n, d, s, accumulate, grid, warps, input): every lane count per row (d = 4 .. 1024),
+# ragged last bucket and last group, sparse streams with long records (bit-serial
+# path), s up to 127, warps that take several groups
+CASES = [
+    (40_003, 512, 16, False, 2, 3, "layered"),
+    (40_003, 512, 16, True, 2, 3, "layered"),
+    (20_000, 128, 4, False, 1, 4, "normal"),
+    (30_001, 1024, 64, True, 2, 2, "normal"),
+    (9_000, 256, 1, False, 2, 2, "heavy_tailed_sparse"),
+    (70_001, 200, 7, True, 3, 2, "normal"),
+    (3_001, 4, 2, False, 2, 2, "normal"),
+    (6_000, 1000, 127, False, 1, 2, "layered"),
+    (1, 512, 16, True, 1, 1, "normal"),
+]
+
+
+@pytest.mark.parametrize("n,d,s,accumulate,grid,warps,kind", CASES,
+                         ids=["n%d-d%d-s%d-acc%d-g%d-w%d-%s" % c for c in CASES])
+def test_row_decoder_matches_oracle(rows_exe, tmp_path, oracle_lib, n, d, s, accumulate, grid, warps, kind):
+    v = W.GENERATORS[kind](n, n % 89)
+    words, offsets, _, st = oracle_lib.encode(v, d, s, seed=11)
+    assert st == 0
+    base = _base(n, d, accumulate)
+    got, status = _run(rows_exe, tmp_path, words, offsets, n, d, s, accumulate, grid, warps, base)
+    assert status == 0
+    if accumulate:
+        ref = base.copy()
+        _, rst = oracle_lib.decode_accumulate([(words, offsets)], n, d, s, ref)
+    else:
+        ref, rst = oracle_lib.decode(words, offsets, n, d, s)
+    assert rst == 0
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("d,accumulate", [(512, False), (128, True), (1000, False)])
+def test_row_decoder_corrupt_streams(rows_exe, tmp_path, oracle_lib, d, accumulate):
+    n, s = 30_000, 16
+    v = W.normal(n, 5)
+    intact, offsets, _, _ = oracle_lib.encode(v, d, s, seed=3)
+    words = intact.copy()
+    _flip_bits(words, offsets, np.random.default_rng(d))
+    base = _base(n, d, accumulate)
+    got, status = _run(rows_exe, tmp_path, words, offsets, n, d, s, accumulate, 2, 2, base)
+    assert status & 2
+    if accumulate:
+        ref = base.copy()
+        oracle_lib.decode_accumulate([(intact, offsets)], n, d, s, ref)
+    else:
+        ref, _ = oracle_lib.decode(intact, offsets, n, d, s)
+    flipped = words != intact
+    keep = np.ones(n, dtype=bool)
+    for b in range(offsets.size - 1):
+        w0, w1 = int(offsets[b]) >> 5, (int(offsets[b + 1]) + 31) >> 5
+        if flipped[w0:w1].any():
+            keep[b * d:min(n, (b + 1) * d)] = False
+    assert keep.any() and not keep.all()
+    assert np.array_equal(got[keep].view(np.uint32), ref[keep].view(np.uint32))
