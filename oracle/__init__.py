@@ -69,6 +69,8 @@ def _declare(lib):
         "qo_capacity_words": (c_u64, [c_u64, c_u64, c_u32]),
         "qo_encode": (c_int, [f32p, c_u64, c_u64, c_u32, c_u64, f32p, u32p, c_u64, u64p,
                               f32p, u32p]),
+        "qo_encode_range": (c_int, [f32p, c_u64, c_u64, c_u32, c_u64, c_u64, c_u64, f32p, u32p, c_u64,
+                                    u64p, f32p, u32p]),
         "qo_encode_bucket": (c_int, [f32p, c_u64, c_u64, c_u32, c_u64, f32p, u32p, c_u64, u64p,
                                      f32p, i32p, u32p]),
         "qo_decode_bucket": (c_int, [u32p, c_u64, c_u64, c_u64, c_u32, f32p, u32p]),
@@ -227,6 +229,32 @@ class Oracle:
             raise RuntimeError("oracle encode failed (status %d)" % st.value)
         nwords = (int(offsets[nb]) + 31) // 32
         return words[:nwords].copy(), offsets, norms[:nb], st.value
+
+    def encode_range(self, v: np.ndarray, d: int, s: int, seed: int, b0: int, b1: int, norms_in=None):
+        """Buckets [b0, b1) of v as a standalone stream: (words, offsets relative to the
+        slice, norms, status); the bits of those buckets in encode()'s stream."""
+        assert v.dtype == np.float32 and v.flags["C_CONTIGUOUS"]
+        n = v.size
+        nb = (n + d - 1) // d
+        assert 0 <= b0 <= b1 <= nb
+        m = min(n, b1 * d) - b0 * d
+        cap = (32 * (b1 - b0) + m * (2 + self.omega_len(s)) + 31) // 32 + 1
+        words = np.zeros(cap, dtype=np.uint32)
+        offsets = np.zeros(b1 - b0 + 1, dtype=np.uint64)
+        norms = np.zeros(max(b1 - b0, 1), dtype=np.float32)
+        st = ctypes.c_uint32(0)
+        nin = None
+        if norms_in is not None:
+            nin = np.ascontiguousarray(norms_in, dtype=np.float32)
+            assert nin.size == b1 - b0
+        rc = self.lib.qo_encode_range(_ptr(v, ctypes.c_float), n, d, s, seed, b0, b1,
+                                      _ptr(nin, ctypes.c_float) if nin is not None else None,
+                                      _ptr(words, ctypes.c_uint32), cap, _ptr(offsets, ctypes.c_uint64),
+                                      _ptr(norms, ctypes.c_float), ctypes.byref(st))
+        if rc != 0:
+            raise RuntimeError("oracle encode_range failed (status %d)" % st.value)
+        nwords = (int(offsets[-1]) + 31) // 32
+        return words[:nwords].copy(), offsets, norms[:b1 - b0], st.value
 
     def encode_bucket(self, vb: np.ndarray, base: int, s: int, seed: int, norm_in=None):
         """One bucket at global index `base` as a standalone bit string (words, nbits)."""

@@ -277,6 +277,32 @@ int qo_encode(const float* v, uint64_t n, uint64_t d, uint32_t s, uint64_t seed,
     return 0;
 }
 
+int qo_encode_range(const float* v, uint64_t n, uint64_t d, uint32_t s, uint64_t seed, uint64_t b0,
+                    uint64_t b1, const float* norms_in, uint32_t* words, uint64_t cap_words,
+                    uint64_t* offsets, float* norms_out, uint32_t* status) {
+    if (d < 1 || s < 1) return -1;
+    uint64_t nb = (n + d - 1) / d;
+    if (b0 > b1 || b1 > nb) return -1;
+    memset(words, 0, cap_words * sizeof(uint32_t));
+    int32_t* levels = (int32_t*)malloc((size_t)(d < n ? d : (n ? n : 1)) * sizeof(int32_t));
+    if (!levels) return -1;
+    uint64_t pos = 0;
+    for (uint64_t b = b0; b < b1; ++b) {
+        uint64_t base = b * d;
+        uint64_t m = (b + 1 == nb) ? n - base : d;
+        offsets[b - b0] = pos;
+        if (qo_encode_bucket(v + base, m, base, s, seed, norms_in ? norms_in + (b - b0) : NULL, words,
+                             cap_words, &pos, norms_out ? norms_out + (b - b0) : NULL, levels,
+                             status) != 0) {
+            free(levels);
+            return -1;
+        }
+    }
+    offsets[b1 - b0] = pos;
+    free(levels);
+    return 0;
+}
+
 /* ------------------------------------------------------------------------- */
 /* Decoder: Q_s(v)_i = ||v||_2 * sgn(v_i) * k_i / s, evaluated as             */
 /* fl(fl(norm / s) * k) with the sign applied last; zeros off the support.   */

@@ -88,6 +88,15 @@ int qo_encode(const float* v, uint64_t n, uint64_t d, uint32_t s, uint64_t seed,
               const float* norms_in, uint32_t* words, uint64_t cap_words,
               uint64_t* offsets, float* norms_out, uint32_t* status);
 
+/* Encoder of the buckets [b0, b1) of the vector v[0..n) as a standalone stream:
+ * the same bits as bits [offsets[b0], offsets[b1]) of qo_encode's stream (every
+ * coordinate keeps its global index, so its Philox word), shifted to start at bit 0.
+ * words[cap_words] (zeroed here), offsets[b1 - b0 + 1] relative to the slice start;
+ * norms_in / norms_out: NULL or b1 - b0 norms of these buckets.  Returns 0 or -1. */
+int qo_encode_range(const float* v, uint64_t n, uint64_t d, uint32_t s, uint64_t seed, uint64_t b0,
+                    uint64_t b1, const float* norms_in, uint32_t* words, uint64_t cap_words,
+                    uint64_t* offsets, float* norms_out, uint32_t* status);
+
 /* Encodes one bucket v[0..m) whose first coordinate has global index base at bit
  * *pos (advanced); levels[m] is scratch.  Returns 0 or -1 on overflow. */
 int qo_encode_bucket(const float* v, uint64_t m, uint64_t base, uint32_t s, uint64_t seed,

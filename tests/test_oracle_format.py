@@ -217,3 +217,28 @@ def test_range_status_for_tiny_norm(oracle_lib):
     words, offsets, norms, st = oracle_lib.encode(v, 4, 1 << 22, seed=0)
     assert st & oracle_mod.ST_RANGE
     assert offsets.tolist() == [0, 32] and int(words[0]) == 0
+
+
+@pytest.mark.parametrize("n,d,s", [(10_007, 100, 16), (4_096, 512, 1), (3_000, 7, 300)])
+def test_encode_range_is_a_slice_of_the_whole_stream(oracle_lib, n, d, s):
+    """encode_range(b0, b1) keeps every coordinate's global index (its Philox word):
+    its stream is bits [offsets[b0], offsets[b1]) of the whole-vector stream, its
+    offsets are the whole offsets shifted, and the slices tile the whole stream."""
+    from gpu_common import extract_bits
+    from quantized_gradient_compression_b200 import workloads as W
+
+    v = W.layered(n, n % 13)
+    words, offsets, norms, st = oracle_lib.encode(v, d, s, 21)
+    nb = offsets.size - 1
+    cuts = [0, 1, nb // 3, nb // 3 + 1, nb - 1, nb]
+    for b0, b1 in zip(cuts[:-1], cuts[1:]):
+        rw, ro, rn, rst = oracle_lib.encode_range(v, d, s, 21, b0, b1)
+        begin, end = int(offsets[b0]), int(offsets[b1])
+        assert np.array_equal(ro, offsets[b0:b1 + 1] - offsets[b0])
+        assert np.array_equal(rn.view(np.uint32), norms[b0:b1].view(np.uint32))
+        assert np.array_equal(rw, extract_bits(words, begin, end))
+    # the GPU-norm form: with norms_in, the same slice as encode(norms_in=...)
+    alt = norms * np.float32(1.0000001)
+    aw, ao, _, _ = oracle_lib.encode(v, d, s, 21, norms_in=alt)
+    rw, ro, _, _ = oracle_lib.encode_range(v, d, s, 21, 1, nb, norms_in=alt[1:])
+    assert np.array_equal(rw, extract_bits(aw, int(ao[1]), int(ao[nb])))
