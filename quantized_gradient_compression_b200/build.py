@@ -13,7 +13,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libqsgd_b200.so")
-SOURCES = ["qsgd_api.cu", "qsgd_encode.cu", "qsgd_decode.cu", "qsgd_static_ws.cu", "qsgd_bbit.cu", "qsgd_ef.cu", "qsgd_mean.cu", "qsgd_encode2.cu", "qsgd_encode_stage.cu", "qsgd_decode_rows.cu"]
+SOURCES = ["qsgd_api.cu", "qsgd_encode.cu", "qsgd_decode.cu", "qsgd_static_ws.cu", "qsgd_bbit.cu", "qsgd_ef.cu", "qsgd_mean.cu", "qsgd_encode_stage.cu", "qsgd_decode_rows.cu"]
 HEADERS = ["qsgd_device.cuh", "qsgd_internal.h", "qsgd_limits.h"]
 
 NVCC_FLAGS = [

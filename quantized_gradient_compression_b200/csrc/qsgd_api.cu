@@ -90,16 +90,11 @@ uint64_t qsgd_max_encoded_words(uint64_t n, uint32_t d, uint32_t s) {
     return ceil_div(max_bits(n, d, s), 32);
 }
 
-#ifndef QSGD_ENCODER_TWO_PASS
-#define QSGD_ENCODER_TWO_PASS 0  // 1: the fast shapes go to the two-pass encoder
-#endif
-
 // Workspace of the one-pass encoders (encode_fast, encode_general) alone: the scan
 // state, a few bytes per tile.
 static size_t one_pass_workspace_bytes(uint64_t n, uint32_t d, uint32_t s) {
     if (!valid_params(n, d, s)) return 0;
-    const size_t total = workspace_layout(n, d).total;
-    return QSGD_ENCODER_TWO_PASS ? align256(total) + encode2_scratch_bytes(n, d) : total;
+    return workspace_layout(n, d).total;
 }
 
 size_t qsgd_encode_workspace_bytes(uint64_t n, uint32_t d, uint32_t s) {
@@ -250,14 +245,11 @@ int encode_entry(const float* d_in, float* d_ef, uint64_t n, uint32_t d, uint32_
         // two launches: bucket coder (with the memory fused in), compaction
         return launch_encode_stage(stage_args(a, d_ef, seed, d_ws), stream) == cudaSuccess ? QSGD_OK : QSGD_ERR_CUDA;
     }
-    if (!d_ef) {
-        if (QSGD_ENCODER_TWO_PASS && fast && encode2_fits(d, s)) {
-            const size_t off = align256(workspace_layout(n, d).total);
-            if (ws_bytes < off + encode2_scratch_bytes(n, d)) return QSGD_ERR_WORKSPACE;
-            return launch_encode2(a, static_cast<char*>(d_ws) + off, stream) == cudaSuccess ? QSGD_OK : QSGD_ERR_CUDA;
-        }
-        return launch_encode(a, fast, stream) == cudaSuccess ? QSGD_OK : QSGD_ERR_CUDA;
-    }
+    // one-pass encoders: their descriptor entries zeroed first (the two-launch encoder
+    // may have left staging data in those bytes)
+    if (cudaMemsetAsync(static_cast<char*>(d_ws) + 256, 0, workspace_layout(n, d).total - 256, stream) != cudaSuccess)
+        return QSGD_ERR_CUDA;
+    if (!d_ef) return launch_encode(a, fast, stream) == cudaSuccess ? QSGD_OK : QSGD_ERR_CUDA;
     if (fast && aligned16(d_ef)) {
         // one pass: the fast encoder reads g and e and writes the stream and e
         a.ef = d_ef;

@@ -743,299 +743,6 @@ __global__ void __launch_bounds__(kMultiBlock) decode_multi(const __grid_constan
     }
 }
 
-// ---------------------------------------------------------------------------
-// Split decoder: P lanes per bucket (one stream; the fast decoder's conditions).
-//
-// One lane per bucket leaves a B200 with a few hundred latency-bound chains of
-// dependent table lookups.  Here the record bits [R0, B1) of a bucket (after the
-// 32-bit norm) are cut into P equal parts and lane j of the bucket's P lanes parses
-// from the start S_j of part j.  Only S_0 is known to be a record boundary; the
-// others start mid-record, but a prefix code of this kind falls back into step
-// with the true record boundaries within a few records.  So:
-//   1. each lane parses its part speculatively up to the first record start
-//      E_j >= S_{j+1}, summing the gaps G_j; an invalid or overrunning record
-//      counts as one bit with gap 0, so the parse is a fixed function of its start
-//      position and never passes B1;
-//   2. lane j continues its parse from E_j ("walker") while lane j+1 parses its own
-//      part again from S_{j+1} ("follower"); whichever of the two is behind takes
-//      the next step, until they stand on the same bit X_j.  The walker sums the
-//      gaps WG_j of its records in [E_j, X_j), the follower the gaps FG_{j+1} of
-//      lane j+1's records in [S_{j+1}, X_j).  From X_j on the two parses coincide,
-//      so by induction from S_0 the true records are lane j's records in
-//      [X_{j-1}, X_j) (X_{-1} = S_0, X_{P-1} = B1), whose gaps sum to
-//      T_j = G_j - FG_j + WG_j;
-//   3. an exclusive scan of T_j over the P lanes gives each lane the index of its
-//      first coordinate, so lane j owns the columns [base_j, base_j + T_j) (the
-//      last lane up to the bucket end).  It initialises them (16-byte stores) and
-//      decodes its range [X_{j-1}, X_j) strictly, storing each value straight to
-//      its column; no two lanes write the same column and nothing is staged.
-// The strict pass in 3 checks everything the serial decoder checks, and that each
-// lane's records end exactly at X_j with gaps summing to T_j; ranges that tile
-// [R0, B1) and parse strictly are the serial parse, so the output is the serial
-// decoder's.  A bucket whose walks do not meet within kMaxMergeSteps, or meet out of
-// order, or that is too short to split, is decoded whole by its lane 0.
-// ---------------------------------------------------------------------------
-constexpr uint32_t kMinPartBits = 64;
-constexpr int kMaxMergeSteps = 1024;
-
-// One step of a speculative parse (left > 0): a valid record through the table or
-// the bit-serial path, else one bit with gap 0.
-__device__ __forceinline__ void spec_step(BitBuf& r, const uint32_t* lut, uint32_t s, uint32_t& gsum) {
-    const uint32_t e = lut[static_cast<uint32_t>(r.buf >> (64 - kLutBits))];
-    uint32_t len = e & 31u;
-    uint32_t gap = (e >> 6) & 1023u;
-    if (len == 0 || len > r.left) {
-        len = 1;
-        gap = 0;
-        if ((e & 63u) == 0) {  // longer than the table window
-            BitBuf t = r;
-            uint32_t g, k;
-            if (t.omega(g) && t.left != 0) {
-                t.consume(1);
-                if (t.omega(k) && k <= s) {
-                    r = t;
-                    gsum += g;
-                    return;
-                }
-            }
-        }
-    }
-    r.consume(len);
-    gsum += gap;
-}
-
-// 32 stream bits starting at bit `pos` (zeros past the stream).
-__device__ __forceinline__ uint32_t read32(const uint32_t* words, uint64_t num_words, uint64_t pos) {
-    const uint64_t w0 = pos >> 5;
-    const uint32_t a0 = w0 < num_words ? __ldg(words + w0) : 0u;
-    const uint32_t a1 = w0 + 1 < num_words ? __ldg(words + w0 + 1) : 0u;
-    return __funnelshift_l(a1, a0, static_cast<uint32_t>(pos & 31u));
-}
-
-#ifndef QSGD_SPLIT_BATCH
-#define QSGD_SPLIT_BATCH 4
-#endif
-constexpr int kBatch = QSGD_SPLIT_BATCH;  // records a lane stores per step of the split decoder
-
-// Columns [lo, hi) of one bucket row g (16-byte aligned): zeros, or x + 0.
-template <bool kAccumulate>
-__device__ __forceinline__ void init_columns(float* g, uint32_t lo, uint32_t hi) {
-    if (lo >= hi) return;
-    const uint32_t a4 = min((lo + 3u) & ~3u, hi);
-    const uint32_t b4 = max(a4, hi & ~3u);
-    for (uint32_t c = lo; c < a4; ++c) g[c] = kAccumulate ? __fadd_rn(g[c], 0.0f) : 0.0f;
-    if (kAccumulate) {
-        for (uint32_t c = a4; c < b4; c += 16) {
-            float4 v[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                if (c + 4 * q < b4) v[q] = *reinterpret_cast<const float4*>(g + c + 4 * q);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                if (c + 4 * q < b4) {
-                    v[q].x = __fadd_rn(v[q].x, 0.0f);
-                    v[q].y = __fadd_rn(v[q].y, 0.0f);
-                    v[q].z = __fadd_rn(v[q].z, 0.0f);
-                    v[q].w = __fadd_rn(v[q].w, 0.0f);
-                    *reinterpret_cast<float4*>(g + c + 4 * q) = v[q];
-                }
-            }
-        }
-    } else {
-        for (uint32_t c = a4; c < b4; c += 4) *reinterpret_cast<float4*>(g + c) = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    for (uint32_t c = b4; c < hi; ++c) g[c] = kAccumulate ? __fadd_rn(g[c], 0.0f) : 0.0f;
-}
-
-template <bool kAccumulate, int P>
-__global__ void __launch_bounds__(kDecodeBlock) decode_split(const __grid_constant__ DecodeArgs a) {
-    static_assert(P >= 1 && P <= 8 && (P & (P - 1)) == 0, "P is 1, 2, 4 or 8");
-    extern __shared__ __align__(16) uint32_t smem[];
-    uint32_t* lut = smem;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    build_record_lut(lut, a.s, tid, kDecodeBlock);
-    __syncthreads();
-    const StreamRef st = a.streams[0];
-    const float fs = __uint2float_rn(a.s);
-    const uint32_t d = a.d;
-    constexpr int kPerWarp = 32 / P;
-    const uint32_t j = static_cast<uint32_t>(lane) & (P - 1);
-    const uint32_t gmask = ((1u << P) - 1u) << (static_cast<uint32_t>(lane) & ~static_cast<uint32_t>(P - 1));
-    const uint64_t ngroups = (a.nb + kPerWarp - 1) / kPerWarp;
-    const uint64_t gwarps = static_cast<uint64_t>(gridDim.x) * kDecWarps;
-    for (uint64_t g = static_cast<uint64_t>(blockIdx.x) * kDecWarps + warp; g < ngroups; g += gwarps) {
-        const uint64_t b = g * kPerWarp + static_cast<uint64_t>(lane / P);
-        const bool live = b < a.nb;
-        const uint32_t m = live ? static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - b * d)) : 0u;
-        bool bad = false;
-        uint64_t R0 = 0;
-        uint32_t L = 0;  // record bits of the bucket
-        float scale = 0.f;
-        if (live) {
-            const uint64_t begin = st.offsets[b];
-            const uint64_t end = st.offsets[b + 1];
-            if (!(end >= begin && end - begin >= 32 && end <= st.num_words * 32 && end - begin < (1ull << 30))) {
-                bad = true;
-            } else {
-                const uint32_t nbits = read32(st.words, st.num_words, begin);
-                const float norm = __uint_as_float(nbits);
-                R0 = begin + 32;
-                L = static_cast<uint32_t>(end - begin - 32);
-                if (nbits == 0) {
-                    bad = L != 0;
-                    L = 0;
-                } else if (!(isfinite(norm) && norm > 0.f)) {
-                    bad = true;
-                    L = 0;
-                } else {
-                    scale = __fdiv_rn(norm, fs);
-                    if (!(scale > 0.f) && L != 0) {  // a zero scale carries no records
-                        bad = true;
-                        L = 0;
-                    }
-                }
-            }
-        }
-        const bool split = P > 1 && L >= P * kMinPartBits;  // the same in all P lanes of a bucket
-        const uint32_t s_lo = split ? static_cast<uint32_t>(static_cast<uint64_t>(L) * j / P) : 0u;
-        const uint32_t s_hi = split ? static_cast<uint32_t>(static_cast<uint64_t>(L) * (j + 1) / P) : L;
-
-        // --- 1. speculative parse of part j (`left` counts the bits to B1) ------
-        BitBuf w;
-        w.left = 0;
-        uint32_t G = 0;
-        if (split) w.init(st.words, st.num_words, R0 + s_lo, L - s_lo);
-        const uint32_t lim = L - s_hi;
-        for (uint32_t it = 0;; ++it) {
-            const bool go = split && w.left > lim;
-            if (!__any_sync(kFullMask, go)) break;
-            if (it == kLoopGuard) {
-                bad = true;
-                break;
-            }
-            if (go) spec_step(w, lut, a.s, G);
-        }
-
-        // --- 2. merge walks: walker of lane j against follower of lane j+1 ------
-        const bool has_w = split && j < P - 1;
-        const bool has_f = split && j > 0;
-        BitBuf f;
-        f.left = 0;
-        if (has_f) f.init(st.words, st.num_words, R0 + s_lo, L - s_lo);
-        if (!has_w) w.left = 0;
-        uint32_t WG = 0, FG = 0;
-        bool met = true;
-        for (int it = 0;; ++it) {
-            const uint32_t y_next = __shfl_down_sync(kFullMask, f.left, 1, P);
-            const uint32_t x_prev = __shfl_up_sync(kFullMask, w.left, 1, P);
-            const bool wa = has_w && w.left > y_next;  // the walker is behind
-            const bool fa = has_f && f.left > x_prev;  // the follower is behind
-            if (!__any_sync(kFullMask, wa || fa)) break;
-            if (it == kMaxMergeSteps) {
-                met = !(wa || fa);
-                break;
-            }
-            if (wa) spec_step(w, lut, a.s, WG);
-            if (fa) spec_step(f, lut, a.s, FG);
-        }
-        // lane j's range [X_{j-1}, X_j) as `left` values
-        const uint32_t x_lo = has_f ? f.left : L;
-        const uint32_t x_hi = has_w ? w.left : 0u;
-        const bool ok = met && x_lo >= x_hi;
-        // (the ballot is taken by all lanes: never inside a short-circuit condition)
-        const uint32_t not_ok = __ballot_sync(kFullMask, !ok);
-        const bool serial = !split || (not_ok & gmask) != 0u;
-        const uint32_t T = G - FG + WG;
-        uint32_t incl = T;
-#pragma unroll
-        for (int o = 1; o < P; o <<= 1) {
-            const uint32_t t = __shfl_up_sync(kFullMask, incl, o, P);
-            if (j >= static_cast<uint32_t>(o)) incl += t;
-        }
-        uint32_t own_lo, own_hi, r_start, r_bits;
-        if (serial) {
-            own_lo = j == 0 ? 0u : m;
-            own_hi = m;
-            r_start = 0;
-            r_bits = j == 0 ? L : 0u;
-        } else {
-            own_lo = min(incl - T, m);
-            own_hi = j == P - 1 ? m : max(own_lo, min(incl, m));
-            r_start = L - x_lo;
-            r_bits = x_lo - x_hi;
-        }
-
-        // --- 3. strict decode of the lane's range, stored straight to its columns
-        // The lane first initialises the columns it owns (zeros; for the first
-        // stream of an accumulation x + 0, which turns -0.0 into +0.0 off the
-        // support and changes nothing under a record, whose value is never zero),
-        // then writes its records; no other lane touches these columns.
-        float* gout = a.out + (live ? b * d : 0);
-        if (!kAccumulate || a.first_group) init_columns<kAccumulate>(gout, own_lo, own_hi);
-        BitBuf r;
-        r.left = 0;
-        if (r_bits != 0) r.init(st.words, st.num_words, R0 + r_start, r_bits);
-        uint32_t next = own_lo, pidx = kNoRecord, pval = 0;
-        table_next(r, lut, scale, next, pidx, pval);
-        for (uint32_t it = 0;; ++it) {
-            if (it == kLoopGuard) {
-                bad = true;
-                pidx = kNoRecord;
-            }
-            const bool ready = pidx < kParked;
-            if (__any_sync(kFullMask, ready) && it < kLoopGuard) {
-                if (ready) {
-                    // up to kBatch records through the table, then their stores (and,
-                    // accumulating, their loads) issued together
-                    uint32_t bi[kBatch];
-                    uint32_t bv[kBatch];
-                    uint32_t cnt = 0;
-#pragma unroll
-                    for (int t = 0; t < kBatch; ++t) {
-                        if (pidx < kParked) {
-                            if (pidx >= own_hi) {  // outside the lane's columns
-                                bad = true;
-                                pidx = kNoRecord;
-                            } else {
-                                bi[t] = pidx;
-                                bv[t] = pval;
-                                cnt = t + 1;
-                                table_next(r, lut, scale, next, pidx, pval);
-                            }
-                        }
-                    }
-                    if (kAccumulate) {
-                        float x[kBatch];
-#pragma unroll
-                        for (int t = 0; t < kBatch; ++t)
-                            if (t < static_cast<int>(cnt)) x[t] = gout[bi[t]];
-#pragma unroll
-                        for (int t = 0; t < kBatch; ++t)
-                            if (t < static_cast<int>(cnt)) gout[bi[t]] = __fadd_rn(x[t], __uint_as_float(bv[t]));
-                    } else {
-#pragma unroll
-                        for (int t = 0; t < kBatch; ++t)
-                            if (t < static_cast<int>(cnt)) gout[bi[t]] = __uint_as_float(bv[t]);
-                    }
-                }
-            } else if (__any_sync(kFullMask, pidx == kParked)) {
-                if (pidx == kParked && !slow_next(r, a.s, scale, next, pidx, pval)) {
-                    bad = true;
-                    pidx = kNoRecord;
-                }
-            } else {
-                break;
-            }
-        }
-        // every record stored, the range consumed exactly, the gaps as scanned
-        if (live && !bad) {
-            if (pidx != kNoRecord || r.left != 0 || next > m) bad = true;
-            if (!serial && j < P - 1 && next != incl) bad = true;
-        }
-        if (bad) atomicOr(a.status, QSGD_ST_BAD_STREAM);
-    }
-}
-
 // Dynamic shared memory for a one-wave launch of `blocks` CTAs that needs `base`
 // bytes: padded so that no SM can hold more than ceil(blocks / SMs) CTAs.  The
 // hardware otherwise stacks up to the occupancy limit on some SMs and leaves
@@ -1051,40 +758,6 @@ inline size_t balanced_smem(size_t base, uint64_t blocks, int dev, int sms, int 
     const size_t pad = static_cast<size_t>(per_sm_bytes) / (target + 1) - static_cast<size_t>(reserved) + 1;
     if (pad <= base || target * (pad + reserved) > static_cast<size_t>(per_sm_bytes)) return base;
     return pad;
-}
-
-template <bool kAccumulate, int P>
-cudaError_t launch_split_decode(const DecodeArgs& a, cudaStream_t stream) {
-    const size_t smem = kLut * sizeof(uint32_t);
-    static bool attr_set[64] = {};
-    int dev = 0, sms = 0, per_sm = 0;
-    cudaGetDevice(&dev);
-    if (dev < 64 && !attr_set[dev]) {
-        cudaFuncSetAttribute(decode_split<kAccumulate, P>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-        attr_set[dev] = true;
-    }
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_split<kAccumulate, P>,
-                                                                  kDecodeBlock, smem);
-    if (e != cudaSuccess) return e;
-    if (per_sm < 1) return cudaErrorInvalidConfiguration;
-    const uint64_t groups = (a.nb + 32 / P - 1) / (32 / P);
-    // one group per warp while the grid stays modest, so that the hardware hands
-    // out the CTAs as SMs free up; beyond that the warps stride over groups
-    const uint64_t blocks = std::min<uint64_t>((groups + kDecWarps - 1) / kDecWarps,
-                                               static_cast<uint64_t>(sms) * per_sm * 8);
-    decode_split<kAccumulate, P><<<static_cast<unsigned>(blocks), kDecodeBlock, smem, stream>>>(a);
-    return cudaGetLastError();
-}
-
-template <bool kAccumulate>
-cudaError_t launch_split_decode_p(const DecodeArgs& a, cudaStream_t stream) {
-#ifdef QSGD_SPLIT_P
-    return launch_split_decode<kAccumulate, QSGD_SPLIT_P>(a, stream);
-#endif
-    if (a.d >= 1024) return launch_split_decode<kAccumulate, 8>(a, stream);
-    if (a.d >= 256) return launch_split_decode<kAccumulate, 4>(a, stream);
-    return launch_split_decode<kAccumulate, 2>(a, stream);
 }
 
 template <bool kAccumulate>
@@ -1173,13 +846,7 @@ cudaError_t launch_decode(const DecodeArgs& a, bool accumulate, cudaStream_t str
 #endif
     // several streams: decoded side by side, the output moved once
     if (QSGD_MULTI && accumulate && a.K >= 2) return launch_multi(a, stream);
-#ifndef QSGD_SPLIT_MODE
-#define QSGD_SPLIT_MODE 0
-#endif
-    // split decoder: 0 never, 1 for decode-accumulate, 2 for both (d >= 128)
-    const bool split = a.d >= 128 && (QSGD_SPLIT_MODE == 2 || (QSGD_SPLIT_MODE == 1 && accumulate));
     auto one = [&](const DecodeArgs& x) -> cudaError_t {
-        if (split) return accumulate ? launch_split_decode_p<true>(x, stream) : launch_split_decode_p<false>(x, stream);
         return accumulate ? launch_fast_decode<true>(x, stream) : launch_fast_decode<false>(x, stream);
     };
     if (a.K == 1) return one(a);

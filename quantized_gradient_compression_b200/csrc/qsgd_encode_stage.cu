@@ -146,10 +146,6 @@ __global__ void __launch_bounds__(kStageBlock) code_buckets(const __grid_constan
     {
         const uint64_t gt = static_cast<uint64_t>(blockIdx.x) * kStageBlock + tid;
         for (uint64_t i = gt; i < a.ntiles; i += static_cast<uint64_t>(gridDim.x) * kStageBlock) a.cdesc[i] = 0;
-        if (gt == 0) {
-            a.ctrl->ticket = 0;
-            a.ctrl->abort = 0;
-        }
     }
     __syncthreads();
 
@@ -317,6 +313,21 @@ __global__ void __launch_bounds__(kStageBlock) code_buckets(const __grid_constan
     }
 }
 
+// The last compaction CTA out returns the control block to its resting state (ticket
+// and completion count zero, no abort), which every encoder of the library expects
+// at the start of a call on this workspace.
+__device__ __forceinline__ void release_control(ScanControl* ctrl) {
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(&ctrl->done, 1u) == gridDim.x - 1) {
+            ctrl->ticket = 0;
+            ctrl->abort = 0;
+            __threadfence();
+            atomicExch(&ctrl->done, 0u);
+        }
+    }
+}
+
 // ---------------------------------------------------------------------------
 // 2. Compaction: offsets header and the stream at its final bit positions.
 // ---------------------------------------------------------------------------
@@ -371,7 +382,10 @@ __global__ void __launch_bounds__(kCompactBlock) compact_stream(const __grid_con
         }
     }
     __syncthreads();
-    if (!s_ok) return;
+    if (!s_ok) {
+        release_control(a.ctrl);
+        return;
+    }
     const uint64_t X = s_X;
     const uint64_t F = X + excl;
     s_F[tid] = F;
@@ -404,6 +418,7 @@ __global__ void __launch_bounds__(kCompactBlock) compact_stream(const __grid_con
                 report(a.status, QSGD_ST_OVERFLOW);
         }
     }
+    release_control(a.ctrl);
 }
 
 template <int V, bool kShort, bool kEF>

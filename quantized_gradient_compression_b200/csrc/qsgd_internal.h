@@ -13,11 +13,12 @@ namespace qsgd {
 struct ScanControl;
 struct TileState;
 
-// Workspace layout: [0, 256) ScanControl; from 256 the tile scan descriptors
-// (uint64 per tile, the count rounded up to an even number); then TileState per
-// tile (shared-word slot, round prefix).  Every entry carries the call's epoch, so
-// values left by an earlier call -- of any shape, wherever they now fall -- read as
-// "not ready", and one workspace serves calls of any shape without clearing.
+// Workspace layout of the one-pass encoders: [0, 256) ScanControl; from 256 the tile
+// scan descriptors (uint64 per tile, the count rounded up to an even number); then
+// TileState per tile (shared-word slot, round prefix).  Every entry carries the
+// call's epoch.  The host zeroes the entries before every one-pass launch, because
+// the two-launch encoder keeps staging data in the same bytes, and data there can
+// look like a descriptor of any epoch.
 struct WorkspaceLayout {
     size_t desc_off, tiles_off, total;
     uint64_t max_tiles;
@@ -48,12 +49,6 @@ struct EncodeArgs {
 // Chooses the kernel, sets the launch shape and enqueues it.  Returns a CUDA
 // error code (cudaSuccess on success).
 cudaError_t launch_encode(EncodeArgs a, bool fast_path, cudaStream_t stream);
-
-// The two-pass encoder (qsgd_encode2.cu; used when QSGD_ENCODER_TWO_PASS is set):
-// its scratch (record lists, counts, sizes, norms) and its three launches.
-bool encode2_fits(uint32_t d, uint32_t s);  // its shared memory fits this shape
-size_t encode2_scratch_bytes(uint64_t n, uint32_t d);
-cudaError_t launch_encode2(const EncodeArgs& a, void* scratch, cudaStream_t stream);
 
 // Dynamic shared memory of the general encoder: omega table | chunk buffer |
 // (norm, s/norm) of the tile's buckets.

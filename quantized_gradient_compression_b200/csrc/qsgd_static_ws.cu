@@ -7,6 +7,7 @@
 // lives in a fixed array of device memory owned by this library.  The array is a
 // file-scope static device variable: every GPU that loads the library holds it
 // (kStaticWorkspaceBytes) until the process exits.  Nothing here allocates.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -25,21 +26,57 @@ static __device__ __align__(256) unsigned char g_static_ws[kStaticWorkspaceBytes
 
 constexpr int kMaxDevices = 64;
 std::mutex g_setup_mutex;
-void* g_ws_ptr[kMaxDevices] = {};
+
+// The array's address is cached per device together with the ID of the CUDA context
+// it was looked up in: after a cudaDeviceReset the device's next context loads the
+// module again, possibly at another address, so a new context ID means a new lookup.
+struct CachedAddress {
+    unsigned long long ctx_id;
+    void* ptr;
+};
+CachedAddress g_ws[kMaxDevices] = {};
+
+// The current context's ID, through the driver entry points the runtime hands out
+// (no link against the driver library).  0 when it cannot be had.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+unsigned long long current_context_id() {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    if (!get_current || !get_id) {
+        cudaDriverEntryPointQueryResult q1, q2;
+        void* f1 = nullptr;
+        void* f2 = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) != cudaSuccess ||
+            cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) != cudaSuccess ||
+            q1 != cudaDriverEntryPointSuccess || q2 != cudaDriverEntryPointSuccess || !f1 || !f2)
+            return 0;
+        get_current = reinterpret_cast<CtxGetCurrentFn>(f1);
+        get_id = reinterpret_cast<CtxGetIdFn>(f2);
+    }
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
 
 // Device address of the array on the current device.  In host code the symbol
-// g_static_ws is only a host-side stand-in, so the address is looked up once per
-// device with that device current.
+// g_static_ws is only a host-side stand-in, so the address is looked up with the
+// device current: once per device and context (twice when the first call comes
+// before the runtime has made the device's context current: that lookup makes it
+// current, and the next call caches the address under the context's ID).
 int static_ws_address(void** ptr) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QSGD_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (g_ws_ptr[dev] == nullptr) {
+    const unsigned long long id = current_context_id();
+    if (g_ws[dev].ptr == nullptr || id == 0 || g_ws[dev].ctx_id != id) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_static_ws) != cudaSuccess || p == nullptr) return QSGD_ERR_CUDA;
-        g_ws_ptr[dev] = p;
+        g_ws[dev].ptr = p;
+        g_ws[dev].ctx_id = id;
     }
-    *ptr = g_ws_ptr[dev];
+    *ptr = g_ws[dev].ptr;
     return QSGD_OK;
 }
 

@@ -1,9 +1,9 @@
-// Runs the decoder kernels decode_fast (P = 0), decode_split (P >= 1), decode_multi
-// (P = -1) and decode_warp (P = -2), compiled for the host under warp_emu.h, over
+// Runs the decoder kernels decode_fast (P = 0), decode_multi (P = -1) and
+// decode_warp (P = -2), compiled for the host under warp_emu.h, over
 // streams read from files.  argv: dir P accumulate [grid [mean]]
 // dir holds params.bin (u64 n, d, s, K), out_in.bin (fp32[n]), w<j>.bin / o<j>.bin
 // (words, offsets of stream j); the result goes to out.bin and the status to stdout.
-// For P >= 0 the K streams are decoded one launch each, in order.  For P < 0 they
+// For P = 0 the K streams are decoded one launch each, in order.  For P < 0 they
 // go 16 to a launch, as the library sends them; with mean = 1 (decode_multi only)
 // the first launch starts from +0 and the last divides by K.
 #include "warp_emu.h"
@@ -40,10 +40,10 @@ static std::vector<unsigned char> slurp(const std::string& p) {
     std::fclose(f);
     return b;
 }
-// P = 0 runs decode_fast (one lane per bucket, staged segments); P >= 1 decode_split.
-template <bool A, int P> void run_kernel(const qsgd::DecodeArgs& a, unsigned grid) {
+// decode_fast (one lane per bucket, staged segments).
+template <bool A> void run_kernel(const qsgd::DecodeArgs& a, unsigned grid) {
     const int kBlock = qsgd::kDecodeBlock;
-    const size_t smem = qsgd::kLut * 4 + (P == 0 ? (size_t)qsgd::kDecWarps * 32 * qsgd::kStride * 4 : 0);
+    const size_t smem = qsgd::kLut * 4 + (size_t)qsgd::kDecWarps * 32 * qsgd::kStride * 4;
     gridDim = {grid, 1, 1};
     blockDim = {(unsigned)kBlock, 1, 1};
     std::vector<unsigned char> sm(smem + 64);
@@ -57,10 +57,7 @@ template <bool A, int P> void run_kernel(const qsgd::DecodeArgs& a, unsigned gri
             th.emplace_back([&, t, b] {
                 threadIdx = {(unsigned)t, 0, 0};
                 blockIdx = {b, 0, 0};
-                if constexpr (P == 0)
-                    qsgd::decode_fast<A>(a);
-                else
-                    qsgd::decode_split<A, P>(a);
+                qsgd::decode_fast<A>(a);
             });
         for (auto& x : th) x.join();
     }
@@ -167,11 +164,10 @@ int main(int argc, char** argv) {
         a.streams[0].words = reinterpret_cast<const uint32_t*>(ws[j].data());
         a.streams[0].num_words = ws[j].size() / 4;
         a.streams[0].offsets = reinterpret_cast<const uint64_t*>(os[j].data());
-        if (acc) {
-            if (P == 0) run_kernel<true, 0>(a, grid); else if (P == 1) run_kernel<true, 1>(a, grid); else if (P == 2) run_kernel<true, 2>(a, grid); else if (P == 4) run_kernel<true, 4>(a, grid); else run_kernel<true, 8>(a, grid);
-        } else {
-            if (P == 0) run_kernel<false, 0>(a, grid); else if (P == 1) run_kernel<false, 1>(a, grid); else if (P == 2) run_kernel<false, 2>(a, grid); else if (P == 4) run_kernel<false, 4>(a, grid); else run_kernel<false, 8>(a, grid);
-        }
+        if (acc)
+            run_kernel<true>(a, grid);
+        else
+            run_kernel<false>(a, grid);
         if (g_emu_error) return 4;
     }
     FILE* f = std::fopen((dir + "/out.bin").c_str(), "wb");

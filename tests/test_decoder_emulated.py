@@ -1,7 +1,7 @@
 """The decoders' kernel source run on the CPU under a warp emulator (no GPU).
 
 `tests/emu/inc/warp_emu.h` stands in for the CUDA features `decode_fast` (P = 0
-below) and `decode_split` (P >= 1) use:
+below), `decode_multi` (P = -1) and `decode_warp` (P = -2) use:
 every thread of a block is a host thread, and each warp primitive gathers the 32
 lanes and checks that they call the same primitive at the same source line.  A lane
 that skips a primitive the others wait in (a deadlock on a GPU) fails the test here,
@@ -30,8 +30,7 @@ CSRC = os.path.join(ROOT, "quantized_gradient_compression_b200", "csrc")
 def _kernel_source() -> str:
     src = open(os.path.join(CSRC, "qsgd_decode.cu")).read()
     # everything from the first host-side launch helper on is cut
-    cut = min(src.index(m) for m in ("template <bool kAccumulate, int P>\ncudaError_t launch_split_decode",
-                                     "// Dynamic shared memory for a one-wave launch") if m in src)
+    cut = src.index("// Dynamic shared memory for a one-wave launch")
     s = src[:cut] + "}  // namespace\n}  // namespace qsgd\n"
     s = s.replace('#include "../../include/qsgd.h"', '#include "%s"' % os.path.join(ROOT, "include", "qsgd.h"))
     s = s.replace('#include "qsgd_internal.h"', '#include "%s"' % os.path.join(CSRC, "qsgd_internal.h"))
@@ -94,30 +93,22 @@ def _run(exe, tmp, oracle_lib, n, d, s, K, P, accumulate, kind, corrupt=False, m
     return got, status, streams, base
 
 
-# (n, d, s, K, P, accumulate, input): P = 0 (decode_fast) / 1 / 2 / 4 / 8, sparse
-# buckets decoded whole,
-# layered data (buckets too short to split next to split ones), ragged tails
+# (n, d, s, K, P, accumulate, input): P = 0, the one-lane staged decoder
+# (decode_fast): ragged last group, d % 64 != 0, several streams one launch each
 CASES = [
-    (40_000, 132, 3, 3, 2, True, "normal"),
-    (30_001, 512, 16, 1, 4, False, "layered"),
-    (30_001, 512, 16, 2, 4, True, "layered"),
-    (20_000, 512, 2, 1, 4, False, "heavy_tailed_sparse"),
-    (40_000, 2048, 64, 2, 8, True, "normal"),
-    (9_001, 4096, 1000, 1, 8, False, "normal"),
-    (513, 512, 16, 2, 4, True, "normal"),
-    (30_001, 512, 16, 1, 1, False, "layered"),   # P = 1: one lane per bucket, direct stores
-    (20_000, 132, 3, 2, 1, True, "normal"),
-    # P = 0: the one-lane staged decoder (decode_fast), ragged last group and d % 64 != 0
     (30_001, 512, 16, 1, 0, False, "layered"),
     (30_001, 512, 16, 2, 0, True, "layered"),
     (20_000, 100, 7, 2, 0, True, "normal"),
     (9_000, 132, 3, 1, 0, False, "normal"),
+    (20_000, 512, 2, 1, 0, False, "heavy_tailed_sparse"),
+    (9_001, 4096, 1000, 1, 0, False, "normal"),
+    (513, 512, 16, 2, 0, True, "normal"),
 ]
 
 
 @pytest.mark.parametrize("n,d,s,K,P,accumulate,kind", CASES,
                          ids=["n%d-d%d-s%d-K%d-P%d-%s-%s" % c for c in CASES])
-def test_split_decoder_matches_oracle(emu_exe, tmp_path, oracle_lib, n, d, s, K, P, accumulate, kind):
+def test_staged_decoder_matches_oracle(emu_exe, tmp_path, oracle_lib, n, d, s, K, P, accumulate, kind):
     got, status, streams, base = _run(emu_exe, tmp_path, oracle_lib, n, d, s, K, P, accumulate, kind)
     assert status == 0
     if accumulate:
@@ -129,24 +120,19 @@ def test_split_decoder_matches_oracle(emu_exe, tmp_path, oracle_lib, n, d, s, K,
     assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
 
 
-@pytest.mark.parametrize("d,P", [(512, 4), (132, 2), (2048, 8)])
-def test_split_decoder_corrupt_streams(emu_exe, tmp_path, oracle_lib, d, P):
+@pytest.mark.parametrize("d", [512, 132, 2048])
+def test_staged_decoder_corrupt_streams(emu_exe, tmp_path, oracle_lib, d):
     """Bit flips in some buckets: the kernel finishes (no lane waits alone), flags
     the stream, and every bucket without a flip decodes as the oracle decodes it."""
     n, s = 30_000, 16
-    got, status, streams, _ = _run(emu_exe, tmp_path, oracle_lib, n, d, s, 1, P, False, "normal", corrupt=True)
+    got, status, streams, _ = _run(emu_exe, tmp_path, oracle_lib, n, d, s, 1, 0, False, "normal", corrupt=True)
     assert status & 2
-    intact = []
-    for j in range(1):
-        v = W.GENERATORS["normal"](n, 300 + j)
-        words, offsets, _, _ = oracle_lib.encode(v, d, s, seed=77 + j)
-        intact.append((words, offsets))
-    ref, _ = oracle_lib.decode(intact[0][0], intact[0][1], n, d, s)
-    flipped = streams[0][0] != intact[0][0]
+    words, offsets, _, _ = oracle_lib.encode(W.GENERATORS["normal"](n, 300), d, s, seed=77)
+    ref, _ = oracle_lib.decode(words, offsets, n, d, s)
+    flipped = streams[0][0] != words
     keep = np.ones(n, dtype=bool)
-    offs = intact[0][1]
-    for b in range(offs.size - 1):
-        w0, w1 = int(offs[b]) >> 5, (int(offs[b + 1]) + 31) >> 5
+    for b in range(offsets.size - 1):
+        w0, w1 = int(offsets[b]) >> 5, (int(offsets[b + 1]) + 31) >> 5
         if flipped[w0:w1].any():
             keep[b * d:min(n, (b + 1) * d)] = False
     assert keep.any()

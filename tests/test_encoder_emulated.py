@@ -134,60 +134,3 @@ def test_special_values(enc_exe, tmp_path, oracle_lib):
         check_norms(gn, own_norms)
         r_words, r_offsets, _, _ = oracle_lib.encode(v, d, 16, 1, norms_in=gn)
         assert np.array_equal(offsets, r_offsets) and np.array_equal(words, r_words)
-
-
-# ---- the two-pass encoder (qsgd_encode2.cu, behind QSGD_ENCODER_TWO_PASS) ----------
-@pytest.fixture(scope="module")
-def enc2_exe(tmp_path_factory):
-    if shutil.which("g++") is None:
-        pytest.skip("g++ not available")
-    d = tmp_path_factory.mktemp("enc2emu")
-    src_dir = d / "pkg" / "csrc"
-    src_dir.mkdir(parents=True)
-    shutil.copytree(os.path.join(ROOT, "include"), d / "include")
-    for h in ("qsgd_internal.h", "qsgd_limits.h"):
-        shutil.copy(os.path.join(CSRC, h), src_dir / h)
-    (src_dir / "qsgd_device.cuh").write_text(_host_source(open(os.path.join(CSRC, "qsgd_device.cuh")).read()))
-    enc = open(os.path.join(CSRC, "qsgd_encode2.cu")).read()
-    cut = enc.index("template <int V>\ncudaError_t launch_v(")
-    (src_dir / "encode2_emu.inc").write_text(_host_source(enc[:cut]) + "}  // namespace\n}  // namespace qsgd\n")
-    exe = d / "enc2_main"
-    r = subprocess.run(["g++", "-O1", "-std=c++17", "-ffp-contract=off", "-pthread", "-I", EMU, "-I", str(src_dir),
-                        os.path.join(EMU, "enc2_main.cpp"), "-o", str(exe)], capture_output=True, text=True)
-    assert r.returncode == 0, r.stderr[-4000:]
-    return str(exe)
-
-
-TWO_PASS = [(40_003, 512, 16, "layered", 0), (20_000, 128, 4, "normal", 0), (30_001, 1024, 64, "normal", 0),
-            (9_000, 256, 1, "heavy_tailed_sparse", 0), (20_000, 512, 16, "special", 1), (1, 512, 16, "normal", 0),
-            (5_000, 384, 3000, "normal", 0)]
-
-
-@pytest.mark.parametrize("n,d,s,kind,nk", TWO_PASS, ids=["n%d-d%d-s%d-%s-nk%d" % c for c in TWO_PASS])
-def test_two_pass_encoder_matches_oracle(enc2_exe, tmp_path, oracle_lib, n, d, s, kind, nk):
-    if kind == "special":
-        v = W.layered(n, 3)
-        v[:512] = 0.0
-        v[700] = np.inf
-        v[1300] = np.nan
-        v[1600:2048] = 1e-30
-        v[2048:2560] = 3e38
-    else:
-        v = W.GENERATORS[kind](n, n % 97)
-    cap = max(1, (32 * ((n + d - 1) // d) + n * (2 + _omega_len(s)) + 31) // 32)
-    np.array([n, d, s, 5, nk, cap], np.uint64).tofile(tmp_path / "params.bin")
-    v.astype(np.float32).tofile(tmp_path / "in.bin")
-    r = subprocess.run([enc2_exe, str(tmp_path), "3"], capture_output=True, text=True, timeout=900)
-    assert r.returncode == 0, r.stderr[-2000:]
-    status = int(r.stdout.split()[-1])
-    offsets = np.fromfile(tmp_path / "offsets.bin", np.uint64)
-    words = np.fromfile(tmp_path / "words.bin", np.uint32)[: (int(offsets[-1]) + 31) // 32]
-    if nk:
-        r_words, r_offsets, _, rst = oracle_lib.encode(v, d, s, 5, norms_in=oracle_lib.maxnorms(v, d))
-    else:
-        _, _, own_norms, rst = oracle_lib.encode(v, d, s, 5)
-        gn = stream_norms(words, offsets)
-        check_norms(gn, own_norms)
-        r_words, r_offsets, _, _ = oracle_lib.encode(v, d, s, 5, norms_in=gn)
-    assert status == rst
-    assert np.array_equal(offsets, r_offsets) and np.array_equal(words, r_words)

@@ -123,3 +123,12 @@ def test_non_default_stream(oracle_lib):
     v = vec("layered", 400_000, 2)
     with torch.cuda.stream(st):
         check_parity(oracle_lib, v, 512, 16, seed=1)
+
+
+def test_one_workspace_serves_every_encoder(oracle_lib):
+    """Calls of the two-launch encoder (d = 512) and of the one-pass encoders (d = 3,
+    d = 8192) alternate on the binding's one shared workspace: each leaves it ready
+    for the next."""
+    for n, d, s, seed in ((70_001, 512, 16, 1), (30_001, 3, 4, 2), (70_001, 512, 16, 3),
+                          (50_000, 8192, 1, 4), (10_000, 128, 64, 5)):
+        check_parity(oracle_lib, W.layered(n, seed), d, s, seed)

@@ -162,3 +162,43 @@ def test_nonfinite_input_status():
     enc = B.encode(torch.from_numpy(v).cuda(), 512, 16, 0)
     torch.cuda.synchronize()
     assert int(enc.status.item()) & B.QSGD_ST_NONFINITE
+
+
+@pytest.mark.parametrize("d,misalign", [(3, 0), (512, 1)])
+def test_epoch_wrap_clears_stale_entries(oracle_lib, d, misalign):
+    """The one-pass encoder tags workspace entries with a 24-bit call epoch.  Entries
+    planted with epoch 0 and the "prefix ready" state would fool the call that runs
+    with epoch 0.  The call that wraps the epoch (epoch 0xFFFFFF) must clear them, so
+    that the next call, with epoch 0, still writes the oracle's stream.  (d = 3, and
+    d = 512 on misaligned input, take the one-pass encoder.)"""
+    import torch
+    from gpu_common import check_norms, device_vector, stream_norms
+    from quantized_gradient_compression_b200 import binding as B
+
+    s, seed = 16, 9
+    ws = torch.zeros(4 << 20, dtype=torch.uint8, device="cuda")
+    ws[256:].view(torch.int64).fill_((2 << 38) | 12345)  # epoch 0, prefix ready, a wrong value
+    ws[8:12].view(torch.int32).fill_(0xFFFFFF)  # the control block's epoch
+    h = torch.cuda.current_stream().cuda_stream
+    # the wrapping call has one tile; the next call's look-back reads entries past it
+    for call, n in enumerate((4_000, 40_000)):
+        v = W.layered(n, 4)
+        x = device_vector(v, misalign)
+        nb = (n + d - 1) // d
+        cap = B.qsgd_max_encoded_words(n, d, s)
+        assert ws.numel() >= B.qsgd_encode_workspace_bytes(n, d, s)
+        words = torch.zeros(cap, dtype=torch.int32, device="cuda")
+        offs = torch.zeros(nb + 1, dtype=torch.int64, device="cuda")
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        assert B.qsgd_encode(x.data_ptr(), n, d, s, seed, words.data_ptr(), cap, offs.data_ptr(), ws.data_ptr(),
+                             ws.numel(), st.data_ptr(), h) == B.QSGD_OK
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        assert int(ws[8:12].view(torch.int32).item()) == call  # 0xFFFFFF + 1 wraps to 0, then 1
+        o = offs.cpu().numpy().view(np.uint64)
+        w = words[:(int(o[-1]) + 31) // 32].cpu().numpy().view(np.uint32)
+        gn = stream_norms(w, o)
+        _, _, onorms, _ = oracle_lib.encode(v, d, s, seed)
+        check_norms(gn, onorms)
+        r_words, r_offsets, _, _ = oracle_lib.encode(v, d, s, seed, norms_in=gn)
+        assert np.array_equal(o, r_offsets) and np.array_equal(w, r_words)

@@ -1,6 +1,6 @@
 """The kernels' source under AddressSanitizer on the CPU emulators (no GPU).
 
-- Decoders (decode_fast, decode_split, decode_multi, decode_warp) on damaged input:
+- Decoders (decode_fast, decode_multi, decode_warp) on damaged input:
   random bit flips anywhere (norm fields included), scrambled offsets headers, and
   word arrays cut short.  They may flag the input, but they must read and write
   nothing outside their buffers, and must end.
@@ -55,7 +55,7 @@ def test_decoders_on_damaged_input(dec_asan, tmp_path, oracle_lib):
         d = int(rng.choice([4, 64, 100, 128, 512, 1000, 4096]))
         s = int(rng.choice([1, 3, 16, 100, 1023]))
         K = int(rng.integers(1, 4))
-        P = int(rng.choice([0, 1, 2, 4, -1, -2]))
+        P = int(rng.choice([0, -1, -2]))
         acc = bool(rng.integers(0, 2)) or P == -1
         t = tmp_path / ("t%d" % trial)
         t.mkdir()
@@ -122,37 +122,3 @@ def test_encoders_stay_in_bounds(enc_asan, tmp_path, oracle_lib, n, d, s, mode, 
     check_norms(gn, own_norms)
     r_words, r_offsets, _, _ = oracle_lib.encode(v, d, s, 2, norms_in=gn)
     assert np.array_equal(offsets, r_offsets) and np.array_equal(words, r_words)
-
-
-@pytest.fixture(scope="module")
-def enc2_asan(tmp_path_factory):
-    d = tmp_path_factory.mktemp("enc2asan")
-    if not _have_asan(d):
-        pytest.skip("no sanitizer")
-    src_dir = d / "pkg" / "csrc"
-    src_dir.mkdir(parents=True)
-    shutil.copytree(os.path.join(ROOT, "include"), d / "include")
-    for h in ("qsgd_internal.h", "qsgd_limits.h"):
-        shutil.copy(os.path.join(CSRC, h), src_dir / h)
-    (src_dir / "qsgd_device.cuh").write_text(host_source(open(os.path.join(CSRC, "qsgd_device.cuh")).read()))
-    enc = open(os.path.join(CSRC, "qsgd_encode2.cu")).read()
-    cut = enc.index("template <int V>\ncudaError_t launch_v(")
-    (src_dir / "encode2_emu.inc").write_text(host_source(enc[:cut]) + "}  // namespace\n}  // namespace qsgd\n")
-    exe = d / "enc2"
-    emu = os.path.join(HERE, "emu", "enc")
-    r = subprocess.run(["g++", *ASAN, "-I", emu, "-I", str(src_dir), os.path.join(emu, "enc2_main.cpp"), "-o", str(exe)],
-                       capture_output=True, text=True)
-    assert r.returncode == 0, r.stderr[-3000:]
-    return str(exe)
-
-
-@pytest.mark.parametrize("n,d,s", [(20_000, 512, 16), (5_000, 384, 3000)])
-def test_two_pass_encoder_asan(enc2_asan, tmp_path, n, d, s):
-    """The two-pass encoder (levels, scan, pack) under the sanitizer."""
-    import test_encoder_emulated as E
-
-    cap = max(1, (32 * ((n + d - 1) // d) + n * (2 + E._omega_len(s)) + 31) // 32)
-    np.array([n, d, s, 5, 0, cap], np.uint64).tofile(tmp_path / "params.bin")
-    W.normal(n, 2).tofile(tmp_path / "in.bin")
-    r = subprocess.run([enc2_asan, str(tmp_path), "3"], capture_output=True, text=True, timeout=1500)
-    assert r.returncode == 0 and "Sanitizer" not in r.stderr, r.stderr[-3000:]
