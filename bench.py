@@ -70,6 +70,8 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5],
+                    help="workload: 2 (default, the headline line) or another of the five configs")
     return ap.parse_args()
 
 
@@ -603,11 +605,211 @@ def run_ours(args, w):
         dist.destroy_process_group()
 
 
+# --------------------------------------------------------------------------
+# the other configurations: one JSON line each (c2 above is the default line)
+# --------------------------------------------------------------------------
+CONFIG_NAMES = {1: "c1_single_bucket_n65536", 3: "c3_resnet152_grad_d8192_s1",
+                4: "c4_receiver_K16_n25557032_d512_s4", 5: "c5_n1073741824_d512_s_sweep"}
+
+
+def config_workloads(cfg: int):
+    from quantized_gradient_compression_b200 import workloads as W
+
+    if cfg == 1:
+        return [W.C1]
+    if cfg == 3:
+        return [W.C3]
+    if cfg == 4:
+        return W.c4_streams()
+    return [W.c5(s) for s in (1, 4, 16, 256)]
+
+
+def run_config(args, cfg: int):
+    """c1 / c3: encode and decode of one vector; c4: the 16 senders' encodes and the
+    receiver's qsgd_decode_accumulate of all 16 streams; c5: encode and decode of the
+    2^30 vector for s = 1, 4, 16, 256.  Every call is timed alone on the device (CUDA
+    events, L2 flushed before each), median over the steps; value = GB/s of fp32
+    gradient input of the config's step."""
+    import torch
+    from quantized_gradient_compression_b200 import binding as B
+
+    rank, world, local = init_dist(args)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+    peak, peak_kind = measured_peaks()
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    K = args.steps
+
+    def check(code, what):
+        if code != 0:
+            raise RuntimeError("%s failed: %s" % (what, B.qsgd_error_string(code)))
+
+    def time_calls(fn):
+        for _ in range(max(3, args.warmup)):
+            flush.zero_()
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(K):
+            flush.zero_()
+            e_a, e_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e_a.record(stream)
+            fn()
+            e_b.record(stream)
+            torch.cuda.synchronize()
+            ts.append(e_a.elapsed_time(e_b))
+        if int(status.item()) != 0:
+            raise RuntimeError("device status %d" % int(status.item()))
+        return statistics.median(ts), min(ts)
+
+    ws_list = config_workloads(cfg)
+    n, d = ws_list[0].n, ws_list[0].d
+    nb = B.qsgd_num_buckets(n, d)
+    lines = []
+    with ClockSampler(local) as clocks:
+        if cfg in (1, 3, 5):
+            v_host = ws_list[0].generate()
+            x = torch.from_numpy(v_host).to(dev)
+            out = torch.empty(n, dtype=torch.float32, device=dev)
+            for w in ws_list:
+                s = w.s
+                cap = B.qsgd_max_encoded_words(n, d, s)
+                words = torch.empty(cap, dtype=torch.int32, device=dev)
+                offsets = torch.empty(nb + 1, dtype=torch.int64, device=dev)
+                ws_bytes = B.qsgd_encode_workspace_bytes(n, d, s)
+                ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
+
+                def enc():
+                    check(B.qsgd_encode(x.data_ptr(), n, d, s, replica_seed(w, rank), words.data_ptr(), cap,
+                                        offsets.data_ptr(), ws.data_ptr(), ws_bytes, status.data_ptr(), sh),
+                          "qsgd_encode")
+
+                def dec():
+                    check(B.qsgd_decode(words.data_ptr(), cap, offsets.data_ptr(), n, d, s, out.data_ptr(),
+                                        status.data_ptr(), sh), "qsgd_decode")
+
+                t_enc, m_enc = time_calls(enc)
+                t_dec, m_dec = time_calls(dec)
+                bits = int(offsets[-1].item())
+                comp = 4 * ((bits + 31) // 32) + 8 * (nb + 1)
+                alg = 4.0 * n + comp
+                lines.append({"s": s, "bits_per_coord": bits / n, "compressed_bytes": comp,
+                              "encode": {"ms_median": t_enc, "ms_min": m_enc, "input_gbs": 4.0 * n / t_enc / 1e6,
+                                         "algorithmic_gbs": alg / t_enc / 1e6, "roofline_frac": alg / t_enc / 1e6 / peak},
+                              "decode": {"ms_median": t_dec, "ms_min": m_dec, "input_gbs": 4.0 * n / t_dec / 1e6,
+                                         "algorithmic_gbs": alg / t_dec / 1e6, "roofline_frac": alg / t_dec / 1e6 / peak}})
+                del words, ws
+            step_ms = sum(r["encode"]["ms_median"] + r["decode"]["ms_median"] for r in lines)
+            value = len(lines) * 4.0 * n / step_ms / 1e6
+            dom = max(((r["encode"]["ms_median"], "encode", r) for r in lines), key=lambda z: z[0])
+            dom2 = max(((r["decode"]["ms_median"], "decode", r) for r in lines), key=lambda z: z[0])
+            dom = max(dom, dom2, key=lambda z: z[0])
+            roof = {"bound": "hbm", "kernel": "%s, s = %d" % (dom[1], dom[2]["s"]),
+                    "achieved": dom[2][dom[1]]["algorithmic_gbs"], "peak": peak, "unit": "GB/s",
+                    "frac": dom[2][dom[1]]["roofline_frac"], "traffic": None,
+                    "peak_source": "%s hbm_gbs (burst copy)" % peak_kind}
+            step = "encode -> decode" + (" for s = 1, 4, 16, 256" if cfg == 5 else "")
+            extra = {"sweep": lines} if cfg == 5 else {"phases": {"encode": lines[0]["encode"], "decode": lines[0]["decode"]},
+                                                       "bits_per_coord": lines[0]["bits_per_coord"],
+                                                       "compressed_bytes": lines[0]["compressed_bytes"]}
+            cpu_sample = v_host[: min(n, 1 << 22)]
+            cpu_w = ws_list[2] if cfg == 5 else ws_list[0]
+        else:  # c4: 16 senders, one receiver
+            Kst = len(ws_list)
+            s = ws_list[0].s
+            cap = B.qsgd_max_encoded_words(n, d, s)
+            ws_bytes = B.qsgd_encode_workspace_bytes(n, d, s)
+            ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
+            words = [torch.empty(cap, dtype=torch.int32, device=dev) for _ in range(Kst)]
+            offsets = [torch.empty(nb + 1, dtype=torch.int64, device=dev) for _ in range(Kst)]
+            xs = [torch.from_numpy(w.generate()).to(dev) for w in ws_list]
+            acc = torch.zeros(n, dtype=torch.float32, device=dev)
+
+            def enc_all():
+                for j, w in enumerate(ws_list):
+                    check(B.qsgd_encode(xs[j].data_ptr(), n, d, s, replica_seed(w, rank), words[j].data_ptr(), cap,
+                                        offsets[j].data_ptr(), ws.data_ptr(), ws_bytes, status.data_ptr(), sh),
+                          "qsgd_encode")
+
+            def receive():
+                check(B.qsgd_decode_accumulate([t.data_ptr() for t in words], [cap] * Kst,
+                                               [t.data_ptr() for t in offsets], Kst, n, d, s, acc.data_ptr(),
+                                               status.data_ptr(), sh), "qsgd_decode_accumulate")
+
+            t_enc, m_enc = time_calls(enc_all)
+            t_acc, m_acc = time_calls(receive)
+            comps = []
+            for o in offsets:
+                bits = int(o[-1].item())
+                comps.append(4 * ((bits + 31) // 32) + 8 * (nb + 1))
+            alg_acc = sum(comps) + 8.0 * n
+            alg_enc = Kst * 4.0 * n + sum(comps)
+            value = Kst * 4.0 * n / t_acc / 1e6
+            roof = {"bound": "hbm", "kernel": "qsgd_decode_accumulate, K = %d" % Kst,
+                    "achieved": alg_acc / t_acc / 1e6, "peak": peak, "unit": "GB/s",
+                    "frac": alg_acc / t_acc / 1e6 / peak, "traffic": None,
+                    "peak_source": "%s hbm_gbs (burst copy)" % peak_kind}
+            step = "decode_accumulate of the K = 16 streams into one fp32 buffer (the senders' encodes timed apart)"
+            extra = {"bits_per_coord": sum(8 * c for c in comps) / Kst / n,
+                     "phases": {"decode_accumulate_K16": {"ms_median": t_acc, "ms_min": m_acc,
+                                                          "algorithmic_bytes": alg_acc,
+                                                          "algorithmic_gbs": alg_acc / t_acc / 1e6,
+                                                          "roofline_frac": alg_acc / t_acc / 1e6 / peak},
+                                "encode_16_senders": {"ms_median": t_enc, "ms_min": m_enc,
+                                                      "algorithmic_bytes": alg_enc,
+                                                      "algorithmic_gbs": alg_enc / t_enc / 1e6,
+                                                      "roofline_frac": alg_enc / t_enc / 1e6 / peak}}}
+            step_ms = t_acc
+            cpu_sample = ws_list[0].generate()[: 1 << 22]
+            cpu_w = ws_list[0]
+    # library launches per timed step: an encode is two (the coder and the compaction,
+    # or the descriptor clear and the one-pass encoder), a decode one, the K = 16
+    # receive one
+    launches = K * (1 if cfg == 4 else 3 * len(ws_list))
+    result = {"metric": METRIC, "value": world * value,
+              "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": step_ms,
+              "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+              "config": {"workload": CONFIG_NAMES[cfg], "n": n, "bucket_d": d,
+                         "s": [w.s for w in ws_list] if cfg == 5 else ws_list[0].s,
+                         "step": step, "l2": "flushed before every timed call (512 MB write)",
+                         "parallelism": "replicas x%d" % world},
+              "roofline": roof, "gpu_launches": launches, "clocks": clocks.summary()}
+    result.update(extra)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+
+        o = oracle.default()
+        t0 = time.perf_counter()
+        reps = 0
+        while reps < 3 and (reps == 0 or time.perf_counter() - t0 < 10.0):
+            wds, offs, _, _ = o.encode(cpu_sample, cpu_w.d, cpu_w.s, cpu_w.seed)
+            o.decode(wds, offs, cpu_sample.size, cpu_w.d, cpu_w.s)
+            reps += 1
+        per = (time.perf_counter() - t0) / reps
+        result["cpu_baseline"] = {"value": 4.0 * cpu_sample.size / per / 1e9, "unit": "GB/s", "cores": 1,
+                                  "kind": "oracle",
+                                  "sample": "first %d coordinates, encode + decode at s = %d, single-threaded C oracle"
+                                            % (cpu_sample.size, cpu_w.s)}
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
 def main():
     args = parse_args()
     w = workload()
     if args.impl == "reference":
+        if args.config != 2:
+            w = config_workloads(args.config)[2 if args.config == 5 else 0]
         run_reference(args, w)
+    elif args.config != 2:
+        run_config(args, args.config)
     else:
         run_ours(args, w)
 

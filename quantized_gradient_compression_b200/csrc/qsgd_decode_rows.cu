@@ -52,33 +52,51 @@ __device__ __forceinline__ bool window_omega(uint32_t w, int nbits, int& pos, ui
     }
 }
 
-// Table of whole records in a 12-bit window: [4:0] length (0: the window holds no
-// whole record with k <= s), [14:5] gap, [23:16] code sign << 7 | k.
+// One whole record (omega(gap) | sign | omega(k)) at bit pos of a 12-bit window with
+// gap <= 15 and 1 <= k <= min(s, 127): its gap, code sign << 7 | k and the bit after it.
+__device__ __forceinline__ bool window_record(uint32_t w, int& pos, uint32_t s, uint32_t& gap, uint32_t& code) {
+    uint32_t k = 0;
+    if (!window_omega(w, kLutBits, pos, gap) || pos >= kLutBits) return false;
+    const uint32_t sign = (w >> (kLutBits - 1 - pos)) & 1u;
+    ++pos;
+    if (!window_omega(w, kLutBits, pos, k) || k > s || k > 127u || gap > 15u) return false;
+    code = (sign << 7) | k;
+    return true;
+}
+
+// Table of the whole records at the start of a 12-bit window, up to two: [3:0] length
+// of the first (0: none, take the bit-serial path), [7:4] length of both (the first's
+// when there is no second), [11:8] first gap, [15:12] second gap, [23:16] first code,
+// [31:24] second code (0: none; a code is never 0, since k >= 1).
 __device__ void build_rows_lut(uint32_t* lut, uint32_t s, int tid, int nthreads) {
     for (int w = tid; w < kLutSize; w += nthreads) {
         int pos = 0;
-        uint32_t gap = 0, k = 0, e = 0;
-        if (window_omega(static_cast<uint32_t>(w), kLutBits, pos, gap) && pos < kLutBits) {
-            const uint32_t sign = (static_cast<uint32_t>(w) >> (kLutBits - 1 - pos)) & 1u;
-            ++pos;
-            if (window_omega(static_cast<uint32_t>(w), kLutBits, pos, k) && k <= s && k < 128u && gap < 1024u)
-                e = static_cast<uint32_t>(pos) | (gap << 5) | (((sign << 7) | k) << 16);
+        uint32_t g1 = 0, c1 = 0, e = 0;
+        if (window_record(static_cast<uint32_t>(w), pos, s, g1, c1)) {
+            const int len1 = pos;
+            uint32_t g2 = 0, c2 = 0;
+            int len2 = len1;
+            if (!window_record(static_cast<uint32_t>(w), len2, s, g2, c2)) {
+                g2 = 0;
+                c2 = 0;
+                len2 = len1;
+            }
+            e = static_cast<uint32_t>(len1) | (static_cast<uint32_t>(len2) << 4) | (g1 << 8) | (g2 << 12) |
+                (c1 << 16) | (c2 << 24);
         }
         lut[w] = e;
     }
 }
 
-// MSB-first reader of one bucket: the next unread bits are the top `valid` bits of
-// buf (valid >= 32 after every refill), nx is the next stream word, `left` the bits
+// MSB-first reader of one bucket over two stream words: the next unread bits are
+// the top bits of funnelshift(nx, cur, off) (0 <= off < 32); `left` counts the bits
 // of the bucket not yet consumed (negative, as int32, after a record that overran).
 struct RowReader {
     const uint32_t* base;  // word holding the bucket's first bit
     uint32_t wi;           // next word to fetch, relative to base
     uint32_t wlim;         // words available from base to the end of the stream
-    uint64_t buf;
-    uint32_t valid;
-    uint32_t nx;
-    uint32_t left;
+    uint32_t cur, nx, off;
+    int32_t left;
     __device__ __forceinline__ uint32_t fetch() {
         const uint32_t w = wi < wlim ? __ldg(base + wi) : 0u;
         ++wi;
@@ -89,41 +107,34 @@ struct RowReader {
         base = words + w0;
         wlim = static_cast<uint32_t>(min(num_words - w0, static_cast<uint64_t>(0xFFFFFFFFu)));
         wi = 0;
-        const uint32_t a0 = fetch(), a1 = fetch();
+        cur = fetch();
         nx = fetch();
-        const uint32_t sh = static_cast<uint32_t>(begin & 31u);
-        buf = ((static_cast<uint64_t>(a0) << 32) | a1) << sh;
-        valid = 64u - sh;
-        left = nbits;
-        refill();
+        off = static_cast<uint32_t>(begin & 31u);
+        left = static_cast<int32_t>(nbits);
     }
-    __device__ __forceinline__ void refill() {
-        if (valid < 32u) {
-            buf |= static_cast<uint64_t>(nx) << (32u - valid);
-            valid += 32u;
+    __device__ __forceinline__ uint32_t peek() const { return __funnelshift_l(nx, cur, off); }
+    __device__ __forceinline__ void advance(uint32_t n) {  // n <= 32
+        off += n;
+        left -= static_cast<int32_t>(n);
+        if (off >= 32u) {
+            cur = nx;
             nx = fetch();
+            off -= 32u;
         }
     }
-    __device__ __forceinline__ void consume(uint32_t n) {  // n <= 32
-        buf <<= n;
-        valid -= n;
-        left -= n;
-        refill();
-    }
-    __device__ __forceinline__ uint32_t top(uint32_t n) const { return static_cast<uint32_t>(buf >> (64u - n)); }
     __device__ __forceinline__ bool omega(uint32_t& N) {  // bit-serial, any length up to 2^32 - 1
         uint32_t v = 1;
         for (;;) {
-            if (static_cast<int32_t>(left) <= 0) return false;
-            const uint32_t bit = static_cast<uint32_t>(buf >> 63);
-            consume(1);
+            if (left <= 0) return false;
+            const uint32_t bit = peek() >> 31;
+            advance(1);
             if (bit == 0) {
                 N = v;
                 return true;
             }
-            if (v > 31 || static_cast<int32_t>(left) < static_cast<int32_t>(v)) return false;
-            const uint32_t rest = top(v);
-            consume(v);
+            if (v > 31 || left < static_cast<int32_t>(v)) return false;
+            const uint32_t rest = peek() >> (32 - v);
+            advance(v);
             v = (1u << v) | rest;
         }
     }
@@ -133,12 +144,32 @@ struct RowReader {
 // level exceeds s).
 __device__ __forceinline__ bool slow_record(RowReader& r, uint32_t s, uint32_t& gap, uint32_t& code) {
     uint32_t k;
-    if (!r.omega(gap) || static_cast<int32_t>(r.left) <= 0 || gap > 0xFFFFu) return false;
-    const uint32_t sign = static_cast<uint32_t>(r.buf >> 63);
-    r.consume(1);
+    if (!r.omega(gap) || r.left <= 0 || gap > 0xFFFFu) return false;
+    const uint32_t sign = r.peek() >> 31;
+    r.advance(1);
     if (!r.omega(k) || k > s) return false;
     code = (sign << 7) | k;
     return true;
+}
+
+// The output of bucket bb as lane `lane` reads it in the write-back: float4 i is
+// coordinates 4 (lane + 32 i) .. + 3, zeros past the bucket's end.
+template <int V>
+__device__ __forceinline__ void load_row(const DecodeArgs& a, uint64_t bb, int lane, float4 (&o)[V]) {
+    const uint32_t mm = static_cast<uint32_t>(min(static_cast<uint64_t>(a.d), a.n - bb * a.d));
+    const float* gp = a.out + bb * a.d;
+#pragma unroll
+    for (int i = 0; i < V; ++i) {
+        const uint32_t c = 4u * (static_cast<uint32_t>(lane) + 32u * i);
+        o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (c + 4 <= mm) {
+            o[i] = __ldcs(reinterpret_cast<const float4*>(gp + c));
+        } else if (c < mm) {
+            o[i].x = gp[c];
+            if (c + 1 < mm) o[i].y = gp[c + 1];
+            if (c + 2 < mm) o[i].z = gp[c + 2];
+        }
+    }
 }
 
 template <int V, bool kAcc>
@@ -182,8 +213,8 @@ __global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows(const __grid_c
                 bad = true;
             } else {
                 r.init(st.words, st.num_words, begin, static_cast<uint32_t>(end - begin));
-                const uint32_t nbits = r.top(32);
-                r.consume(32);
+                const uint32_t nbits = r.peek();
+                r.advance(32);
                 const float norm = __uint_as_float(nbits);
                 if (nbits == 0) {
                     bad = r.left != 0;
@@ -201,38 +232,57 @@ __global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows(const __grid_c
             }
         }
         __syncwarp();
-        // --- parse: every record's code into the lane's row ----------------------
+        // --- parse: every record's code into the lane's row, up to two a lookup ----
         uint32_t next = 0;  // bucket-local index after the last record
-        for (uint32_t it = 0;; ++it) {
-            const bool act = static_cast<int32_t>(r.left) > 0 && !bad;
-            if (!__any_sync(kWarpAll, act)) break;
+        if (bad) r.left = 0;
+        for (uint32_t it = 0; __any_sync(kWarpAll, r.left > 0); ++it) {
             if (it == kParseGuard) {
-                bad = bad || act;
+                bad = bad || r.left > 0;
                 break;
             }
-            if (act) {
-                const uint32_t e = lut[static_cast<uint32_t>(r.buf >> (64 - kLutBits))];
-                const uint32_t len = e & 31u;
-                uint32_t gap = (e >> 5) & 1023u, code = e >> 16;
-                if (len != 0u) {
-                    r.consume(len);
-                } else if (!slow_record(r, a.s, gap, code)) {
-                    bad = true;
-                    gap = 0;
+            if (r.left > 0) {
+                const uint32_t e = lut[r.peek() >> (32 - kLutBits)];
+                const uint32_t len1 = e & 15u;
+                if (len1 != 0u) {
+                    // the second record only when it ends inside the bucket
+                    const uint32_t len2 = (e >> 4) & 15u;
+                    const bool two = static_cast<int32_t>(len2) <= r.left;
+                    r.advance(two ? len2 : len1);
+                    next += (e >> 8) & 15u;
+                    myrow[min(next - 1u, d)] = static_cast<uint8_t>(e >> 16);
+                    const uint32_t c2 = e >> 24;
+                    if (two && c2 != 0u) {
+                        next += (e >> 12) & 15u;
+                        myrow[min(next - 1u, d)] = static_cast<uint8_t>(c2);
+                    }
+                } else {
+                    uint32_t gap = 0, code = 0;
+                    if (slow_record(r, a.s, gap, code)) {
+                        next += gap;
+                        myrow[min(next - 1u, d)] = static_cast<uint8_t>(code);
+                    } else {
+                        bad = true;
+                        r.left = 0;
+                    }
                 }
-                next += gap;
-                // a malformed index lands in the row's padding (the bucket is then bad)
-                if (!bad) myrow[min(next - 1u, d)] = static_cast<uint8_t>(code);
             }
         }
-        // every record index below m, and the bucket consumed exactly
+        // every record index below m, and the bucket consumed exactly (a record that
+        // overran leaves left negative; an index past m lands in the row's padding)
         if (live && !bad && (next > m || r.left != 0)) bad = true;
         __syncwarp();
         // --- write the rows back: row rr is bucket g*32 + rr -----------------------
-        for (int rr = 0; rr < 32; ++rr) {
+        // (decode-accumulate reads the next row's output before it stores this row's,
+        // so that two rows of loads are in flight)
+        const int nrows = static_cast<int>(min(static_cast<uint64_t>(32), a.nb - g * 32));
+        float4 cur[kAcc ? V : 1], nxt[kAcc ? V : 1];
+        if constexpr (kAcc) load_row<V>(a, g * 32, lane, cur);
+        for (int rr = 0; rr < nrows; ++rr) {
             const uint64_t bb = g * 32 + rr;
             const float sc = __shfl_sync(kWarpAll, scale, rr);
-            if (bb >= a.nb) break;
+            if constexpr (kAcc) {
+                if (rr + 1 < nrows) load_row<V>(a, bb + 1, lane, nxt);
+            }
             const uint32_t mm = static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - bb * d));
             const uint32_t* rowp = rows + static_cast<uint32_t>(rr) * stride_w;
             float* gp = a.out + bb * d;
@@ -250,21 +300,22 @@ __global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows(const __grid_c
                         const float kf = __fsub_rn(__uint_as_float(0x4B000000u | (code & 0x7Fu)), 8388608.0f);
                         v[j] = __uint_as_float(__float_as_uint(__fmul_rn(sc, kf)) | ((code & 0x80u) << 24));
                     }
+                    if constexpr (kAcc) {
+                        v[0] = __fadd_rn(cur[i].x, v[0]);
+                        v[1] = __fadd_rn(cur[i].y, v[1]);
+                        v[2] = __fadd_rn(cur[i].z, v[2]);
+                        v[3] = __fadd_rn(cur[i].w, v[3]);
+                    }
                     if (c + 4 <= mm) {
-                        float4* p4 = reinterpret_cast<float4*>(gp + c);
-                        if constexpr (kAcc) {
-                            const float4 o = *p4;
-                            v[0] = __fadd_rn(o.x, v[0]);
-                            v[1] = __fadd_rn(o.y, v[1]);
-                            v[2] = __fadd_rn(o.z, v[2]);
-                            v[3] = __fadd_rn(o.w, v[3]);
-                        }
-                        __stcs(p4, make_float4(v[0], v[1], v[2], v[3]));
+                        __stcs(reinterpret_cast<float4*>(gp + c), make_float4(v[0], v[1], v[2], v[3]));
                     } else {
-                        for (uint32_t j = 0; j < 4 && c + j < mm; ++j)
-                            gp[c + j] = kAcc ? __fadd_rn(gp[c + j], v[j]) : v[j];
+                        for (uint32_t j = 0; j < 4 && c + j < mm; ++j) gp[c + j] = v[j];
                     }
                 }
+            }
+            if constexpr (kAcc) {
+#pragma unroll
+                for (int i = 0; i < V; ++i) cur[i] = nxt[i];
             }
         }
         if (bad) atomicOr(a.status, QSGD_ST_BAD_STREAM);
@@ -288,15 +339,17 @@ cudaError_t launch_rows_v(const DecodeArgs& a, cudaStream_t stream) {
     cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     const size_t per_warp = static_cast<size_t>(32) * stride * sizeof(uint32_t);
     const size_t lut_bytes = static_cast<size_t>(kLutSize) * sizeof(uint32_t);
-    const int W = static_cast<int>(std::min<size_t>(kRowsMaxWarps, (static_cast<size_t>(optin) - lut_bytes - 1024) / per_warp));
-    if (W < 1) return cudaErrorInvalidConfiguration;
+    const int W_fit = static_cast<int>(std::min<size_t>(kRowsMaxWarps, (static_cast<size_t>(optin) - lut_bytes - 1024) / per_warp));
+    if (W_fit < 1) return cudaErrorInvalidConfiguration;
+    // one CTA per SM, its warps one group each where the groups allow: every SM busy
+    const uint64_t groups = (a.nb + 31) / 32;
+    const int W = static_cast<int>(std::max<uint64_t>(1, std::min<uint64_t>(W_fit, (groups + sms - 1) / sms)));
     const size_t smem = lut_bytes + W * per_warp;
     static bool attr_set[64] = {};
     if (dev < 64 && !attr_set[dev]) {
         cudaFuncSetAttribute(decode_rows<V, kAcc>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
         attr_set[dev] = true;
     }
-    const uint64_t groups = (a.nb + 31) / 32;
     const uint64_t blocks = std::max<uint64_t>(1, std::min<uint64_t>(static_cast<uint64_t>(sms), (groups + W - 1) / W));
     decode_rows<V, kAcc><<<static_cast<unsigned>(blocks), 32 * W, smem, stream>>>(a, stride);
     return cudaGetLastError();

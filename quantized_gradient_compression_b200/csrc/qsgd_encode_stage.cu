@@ -123,6 +123,210 @@ __device__ __forceinline__ void store_lane(float* p, int lane, uint32_t m, const
     }
 }
 
+// One record of the short form (s <= 31): the whole-record table for gap < 64, the
+// omega table otherwise (gap <= d <= 1024); code right-aligned, <= 30 bits.
+__device__ __forceinline__ void short_record(const uint32_t* rtab, const uint32_t* otab, uint32_t gap, uint32_t kv,
+                                             uint32_t& code, uint32_t& len) {
+    if (gap < 64u) {
+        const uint32_t e = rtab[(gap << 6) | __funnelshift_l(kv, kv, 1)];
+        code = e >> 5;
+        len = e & 31u;
+    } else {
+        const uint32_t ge = otab[gap], ke = otab[kv & 0x7FFFFFFFu];
+        const uint32_t kl = ke & 0xFFu;
+        code = ((((ge >> 8) << 1) | (kv >> 31)) << kl) | (ke >> 8);
+        len = (ge & 0xFFu) + 1u + kl;
+    }
+}
+
+// Loads one lane's NC = 4V consecutive values [q0, q0 + NC) of a bucket of m values
+// at p (streaming; zeros past m).
+template <int V>
+__device__ __forceinline__ void load_contig(const float* p, uint32_t q0, uint32_t m, float (&x)[4 * V]) {
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+        const uint32_t i = q0 + 4u * j;
+        float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (i + 4 <= m) {
+            q = __ldcs(reinterpret_cast<const float4*>(p + i));
+        } else if (i < m) {
+            q.x = p[i];
+            if (i + 1 < m) q.y = p[i + 1];
+            if (i + 2 < m) q.z = p[i + 2];
+        }
+        x[4 * j + 0] = q.x;
+        x[4 * j + 1] = q.y;
+        x[4 * j + 2] = q.z;
+        x[4 * j + 3] = q.w;
+    }
+}
+
+// Stores one lane's NC consecutive values [q0, q0 + NC) (streaming; nothing past m).
+template <int V>
+__device__ __forceinline__ void store_contig(float* p, uint32_t q0, uint32_t m, const float (&v)[4 * V]) {
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+        const uint32_t i = q0 + 4u * j;
+        if (i + 4 <= m) {
+            __stcs(reinterpret_cast<float4*>(p + i), make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
+        } else if (i < m) {
+            __stcs(p + i, v[4 * j]);
+            if (i + 1 < m) __stcs(p + i + 1, v[4 * j + 1]);
+            if (i + 2 < m) __stcs(p + i + 2, v[4 * j + 2]);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// 1a. Bucket coder for s <= 31 (records <= 30 bits).  Lane L holds the NC = 4V
+// consecutive coordinates [NC L, NC L + NC) of its bucket, so a bucket is one run:
+// one gap chain over the lanes (a ballot and a shuffle) and one scan of the lanes'
+// bit counts.  A lane appends its records to a 96-bit register string as it codes
+// them and ORs the string into the bucket buffer once its position is known.  A
+// bucket where some lane needs more than 96 bits is placed record by record.
+// ---------------------------------------------------------------------------
+template <int V, bool kEF>
+__global__ void __launch_bounds__(kStageBlock) code_buckets_short(const __grid_constant__ StageArgs a) {
+    extern __shared__ __align__(16) uint32_t smem[];
+    constexpr int NC = 4 * V;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    uint32_t* const otab = smem;                                                  // omega table
+    uint32_t* const rtab = smem + kOmegaTab;                                      // record table
+    uint32_t* const buf = smem + kOmegaTab + kRecordTab64 + warp * a.buf_words;   // this warp's bucket bits
+    omega_table_fill(otab, tid, kStageBlock);
+    {
+        const uint4* src = reinterpret_cast<const uint4*>(kRecordTable64Global.v);
+        for (int i = tid; i < kRecordTab64 / 4; i += kStageBlock) reinterpret_cast<uint4*>(rtab)[i] = src[i];
+    }
+    for (uint32_t i = lane; i < a.buf_words; i += 32) buf[i] = 0u;
+    {  // the compaction's scan state for this call: cleared here, before it runs
+        const uint64_t gt = static_cast<uint64_t>(blockIdx.x) * kStageBlock + tid;
+        for (uint64_t i = gt; i < a.ntiles; i += static_cast<uint64_t>(gridDim.x) * kStageBlock) a.cdesc[i] = 0;
+    }
+    __syncthreads();
+
+    const uint32_t d = a.d;
+    const uint32_t q0 = static_cast<uint32_t>(NC * lane);
+    const uint32_t lanes_below = (1u << lane) - 1u;
+    const uint64_t gwarps = static_cast<uint64_t>(gridDim.x) * kStageWarps;
+    for (uint64_t b = static_cast<uint64_t>(blockIdx.x) * kStageWarps + warp; b < a.nb; b += gwarps) {
+        const uint64_t base = b * d;
+        const uint32_t m = static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - base));
+        float x[NC];
+        float ev[kEF ? NC : 1];
+        load_contig<V>(a.in + base, q0, m, x);
+        if constexpr (kEF) {  // p = e + g
+            load_contig<V>(a.ef + base, q0, m, ev);
+#pragma unroll
+            for (int q = 0; q < NC; ++q) x[q] = __fadd_rn(ev[q], x[q]);
+        }
+        const float norm = a.norm_kind == QSGD_NORM_MAX ? warp_bucket_maxnorm<NC>(x) : warp_bucket_norm<NC>(x, true);
+        const BucketScale sc = bucket_scale(norm, a.s, true, a.status, lane == 0);
+        if (!sc.good) {  // sent as a zero bucket; the memory keeps p
+            if constexpr (kEF) store_contig<V>(a.ef + base, q0, m, x);
+#pragma unroll
+            for (int q = 0; q < NC; ++q) x[q] = 0.f;
+        }
+        // --- levels: one Philox block per four coordinates -------------------------
+        uint32_t kq[NC];  // level | sign << 31
+        const uint32_t j0 = static_cast<uint32_t>((base + q0) >> 2);
+#pragma unroll
+        for (int j = 0; j < V; ++j) {
+            const uint4 r = philox_rk(j0 + j, a.rk);
+            const uint32_t rw[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const float v = x[4 * j + c];
+                kq[4 * j + c] = level_of(v, sc.sinv, rw[c], a.s) | (__float_as_uint(v) & 0x80000000u);
+            }
+        }
+        if constexpr (kEF) {  // the memory keeps p minus what a receiver decodes
+            if (sc.good) {
+                const float scale = __fdiv_rn(sc.sent, __uint2float_rn(a.s));
+#pragma unroll
+                for (int q = 0; q < NC; ++q) ev[q] = ef_residual(x[q], kq[q] & 0x7FFFFFFFu, kq[q] >> 31, scale);
+                store_contig<V>(a.ef + base, q0, m, ev);
+            }
+        }
+        // --- gap chain: the last record before this lane's coordinates ----------------
+        uint32_t nzm = 0;
+#pragma unroll
+        for (int c = 0; c < NC; ++c) nzm |= ((kq[c] & 0x7FFFFFFFu) != 0u ? 1u : 0u) << c;
+        const int32_t last = nzm ? static_cast<int32_t>(q0 + 31u - __clz(nzm)) : -1;
+        const uint32_t B = __ballot_sync(kAll, nzm != 0u) & lanes_below;
+        const int32_t pv = __shfl_sync(kAll, last, B ? 31 - __clz(B) : 0);
+        const int32_t prev_in = B ? pv : -1;
+        // --- the lane's records, appended to (w2:w1:w0), right-aligned ---------------
+        uint32_t w0 = 0, w1 = 0, w2 = 0, nbits = 0;
+        {
+            int32_t prev = prev_in;
+#pragma unroll
+            for (int c = 0; c < NC; ++c) {
+                const uint32_t kv = kq[c];
+                uint32_t code = 0, len = 0;
+                if ((kv & 0x7FFFFFFFu) != 0u) {
+                    short_record(rtab, otab, static_cast<uint32_t>(static_cast<int32_t>(q0 + c) - prev), kv, code, len);
+                    prev = static_cast<int32_t>(q0 + c);
+                }
+                w2 = __funnelshift_l(w1, w2, len);
+                w1 = __funnelshift_l(w0, w1, len);
+                w0 = (w0 << len) | code;
+                nbits += len;
+            }
+        }
+        // --- the lane's first bit in the bucket: scan of the bit counts ---------------
+        uint32_t incl = nbits;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t t = __shfl_up_sync(kAll, incl, o);
+            if (lane >= o) incl += t;
+        }
+        const uint32_t P = 32u + incl - nbits;
+        const uint32_t total = 32u + __shfl_sync(kAll, incl, 31);
+        if (lane == 0) buf[0] = __float_as_uint(sc.sent);
+        if (!__any_sync(kAll, nbits > 96u)) {
+            if (nbits != 0u) {
+                // left-align the string in 96 bits, then OR it in at bit P
+                const uint32_t sa = 96u - nbits, bsh = sa & 31u, wsh = sa >> 5;
+                const uint32_t t2 = __funnelshift_l(w1, w2, bsh), t1 = __funnelshift_l(w0, w1, bsh), t0 = w0 << bsh;
+                const uint32_t L0 = wsh == 0 ? t2 : wsh == 1 ? t1 : t0;
+                const uint32_t L1 = wsh == 0 ? t1 : wsh == 1 ? t0 : 0u;
+                const uint32_t L2 = wsh == 0 ? t0 : 0u;
+                const uint32_t wp = P >> 5, sh = P & 31u;
+                const uint32_t nw = (sh + nbits + 31u) >> 5;  // 1..4
+                atomicOr(&buf[wp], L0 >> sh);
+                if (nw > 1) atomicOr(&buf[wp + 1], __funnelshift_r(L1, L0, sh));
+                if (nw > 2) atomicOr(&buf[wp + 2], __funnelshift_r(L2, L1, sh));
+                if (nw > 3) atomicOr(&buf[wp + 3], __funnelshift_r(0u, L2, sh));
+            }
+        } else {  // some lane's string is longer than 96 bits: record by record
+            int32_t prev = prev_in;
+            uint32_t p = P;
+#pragma unroll
+            for (int c = 0; c < NC; ++c) {
+                const uint32_t kv = kq[c];
+                if ((kv & 0x7FFFFFFFu) != 0u) {
+                    uint32_t code, len;
+                    short_record(rtab, otab, static_cast<uint32_t>(static_cast<int32_t>(q0 + c) - prev), kv, code, len);
+                    prev = static_cast<int32_t>(q0 + c);
+                    put_bits(buf, p, code, len);
+                    p += len;
+                }
+            }
+        }
+        __syncwarp();
+        // --- the bucket's bits into its staging slot; the buffer cleared again -------
+        uint32_t* const slot = a.stage + b * a.slot_words;
+        const uint32_t nw = (total + 31u) >> 5;
+        for (uint32_t i = lane; i < nw; i += 32) {
+            slot[i] = buf[i];
+            buf[i] = 0u;
+        }
+        if (lane == 0) a.bits[b] = total;
+        __syncwarp();
+    }
+}
+
 // ---------------------------------------------------------------------------
 // 1. Bucket coder.  kShort: s <= 31, records of gap < 64 through the whole-record
 // table (the others from the omega table), every record <= 30 bits.  Otherwise every
@@ -332,7 +536,7 @@ __device__ __forceinline__ void release_control(ScanControl* ctrl) {
 // 2. Compaction: offsets header and the stream at its final bit positions.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kCompactBlock) compact_stream(const __grid_constant__ StageArgs a) {
-    __shared__ uint64_t s_F[kCompactBlock];
+    __shared__ uint32_t s_R[kCompactBlock];
     __shared__ uint32_t s_L[kCompactBlock];
     __shared__ uint32_t s_warp[kCompactBlock / 32];
     __shared__ uint32_t s_tile;
@@ -388,32 +592,51 @@ __global__ void __launch_bounds__(kCompactBlock) compact_stream(const __grid_con
     }
     const uint64_t X = s_X;
     const uint64_t F = X + excl;
-    s_F[tid] = F;
+    s_R[tid] = excl;  // tile-relative start of each bucket
     s_L[tid] = L;
     if (b < a.nb) a.offsets[b] = F;
     if (b + 1 == a.nb) a.offsets[a.nb] = F + L;
     __syncthreads();
-    // bucket i of the tile: the words whose first bit lies in it
-    const uint64_t nt = min(static_cast<uint64_t>(kCompactBlock), a.nb - b0);
-    for (uint32_t i = warp; i < nt; i += kCompactBlock / 32) {
-        const uint64_t bb = b0 + i;
-        const uint64_t Fb = s_F[i];
-        const uint32_t Lb = s_L[i];
-        const uint32_t* src = a.stage + bb * a.slot_words;
-        const uint32_t nsw = (Lb + 31u) >> 5;
-        const uint64_t w_begin = (Fb + 31u) >> 5, w_end = (Fb + Lb + 31u) >> 5;
-        for (uint64_t w = w_begin + lane; w < w_end; w += 32) {
-            const uint32_t r = static_cast<uint32_t>(32u * w - Fb);
+    // Every thread takes output words w = wb + tid + kCompactBlock i of the tile: the
+    // words whose first bit lies in one of its buckets.  A word's bucket comes from a
+    // binary search over the buckets' starts; its bits are that bucket's staged bits
+    // from the word's offset on, and, past the bucket's end, the first bits of the
+    // next bucket (always >= 32 bits, so one word of it suffices).
+    const uint32_t nt = static_cast<uint32_t>(min(static_cast<uint64_t>(kCompactBlock), a.nb - b0));
+    const uint64_t wb = (X + 31u) >> 5, we = (X + total + 31u) >> 5;
+    constexpr int kUnroll = 4;
+    for (uint64_t w0 = wb + tid; w0 < we; w0 += kUnroll * kCompactBlock) {
+        uint32_t v[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const uint64_t w = w0 + static_cast<uint64_t>(u) * kCompactBlock;
+            v[u] = 0u;
+            if (w >= we) continue;
+            const uint32_t g = static_cast<uint32_t>(32u * w - X);  // tile-relative bit of the word
+            uint32_t lo = 0, hi = nt - 1;  // the last bucket with start <= g
+            while (lo < hi) {
+                const uint32_t mid = (lo + hi + 1) >> 1;
+                if (s_R[mid] <= g) lo = mid; else hi = mid - 1;
+            }
+            const uint64_t bb = b0 + lo;
+            const uint32_t Lb = s_L[lo];
+            const uint32_t r = g - s_R[lo];
             const uint32_t q = r >> 5, sh = r & 31u;
+            const uint32_t* src = a.stage + bb * a.slot_words;
             const uint32_t a0 = src[q];
-            const uint32_t a1 = q + 1 < nsw ? src[q + 1] : 0u;
-            uint32_t v = __funnelshift_l(a1, a0, sh);
+            const uint32_t a1 = q + 1 < ((Lb + 31u) >> 5) ? src[q + 1] : 0u;
+            v[u] = __funnelshift_l(a1, a0, sh);
             if (r + 32u > Lb) {  // the word runs into the next bucket: its first bits
                 const uint32_t hd = bb + 1 < a.nb ? a.stage[(bb + 1) * a.slot_words] : 0u;
-                v |= hd >> (Lb - r);
+                v[u] |= hd >> (Lb - r);
             }
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const uint64_t w = w0 + static_cast<uint64_t>(u) * kCompactBlock;
+            if (w >= we) continue;
             if (w < a.cap_words)
-                a.words[w] = v;
+                a.words[w] = v[u];
             else
                 report(a.status, QSGD_ST_OVERFLOW);
         }
@@ -421,25 +644,33 @@ __global__ void __launch_bounds__(kCompactBlock) compact_stream(const __grid_con
     release_control(a.ctrl);
 }
 
-template <int V, bool kShort, bool kEF>
-cudaError_t launch_code(const StageArgs& a, cudaStream_t stream) {
+template <class Kernel>
+cudaError_t launch_coder(Kernel kernel, const StageArgs& a, cudaStream_t stream) {
     const size_t smem = stage_smem_bytes(a.s, a.buf_words);
     static bool attr_set[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 64 && !attr_set[dev]) {
-        cudaFuncSetAttribute(code_buckets<V, kShort, kEF>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
         attr_set[dev] = true;
     }
     int sms = 0, per_sm = 0;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, code_buckets<V, kShort, kEF>, kStageBlock, smem);
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kStageBlock, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const uint64_t want = (a.nb + kStageWarps - 1) / kStageWarps;
     const uint64_t grid = std::max<uint64_t>(1, std::min<uint64_t>(want, static_cast<uint64_t>(sms) * per_sm));
-    code_buckets<V, kShort, kEF><<<static_cast<unsigned>(grid), kStageBlock, smem, stream>>>(a);
+    kernel<<<static_cast<unsigned>(grid), kStageBlock, smem, stream>>>(a);
     return cudaGetLastError();
+}
+
+template <int V, bool kShort, bool kEF>
+cudaError_t launch_code(const StageArgs& a, cudaStream_t stream) {
+    if constexpr (kShort)
+        return launch_coder(code_buckets_short<V, kEF>, a, stream);
+    else
+        return launch_coder(code_buckets<V, false, kEF>, a, stream);
 }
 
 template <int V>

@@ -74,6 +74,11 @@ inline uint32_t __funnelshift_l(uint32_t lo, uint32_t hi, uint32_t sh) {
     const uint64_t x = (static_cast<uint64_t>(hi) << 32) | lo;
     return static_cast<uint32_t>((x << (sh & 31u)) >> 32);
 }
+// the low word of (hi:lo) >> (sh mod 32)
+inline uint32_t __funnelshift_r(uint32_t lo, uint32_t hi, uint32_t sh) {
+    const uint64_t x = (static_cast<uint64_t>(hi) << 32) | lo;
+    return static_cast<uint32_t>(x >> (sh & 31u));
+}
 inline float __uint2float_rn(uint32_t u) { return static_cast<float>(u); }
 inline float __uint_as_float(uint32_t u) { float f; std::memcpy(&f, &u, 4); return f; }
 inline uint32_t __float_as_uint(float f) { uint32_t u; std::memcpy(&u, &f, 4); return u; }

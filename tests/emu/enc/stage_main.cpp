@@ -65,7 +65,10 @@ static void run_grid(unsigned grid, unsigned block, size_t smem, Kernel k) {
 
 template <int V, bool kShort, bool kEF>
 static void code(const qsgd::StageArgs& a, unsigned grid, size_t smem) {
-    run_grid(grid, qsgd::kStageBlock, smem, [&] { qsgd::code_buckets<V, kShort, kEF>(a); });
+    if constexpr (kShort)
+        run_grid(grid, qsgd::kStageBlock, smem, [&] { qsgd::code_buckets_short<V, kEF>(a); });
+    else
+        run_grid(grid, qsgd::kStageBlock, smem, [&] { qsgd::code_buckets<V, false, kEF>(a); });
 }
 template <int V, bool kEF>
 static void code_v(const qsgd::StageArgs& a, unsigned grid, size_t smem) {

@@ -38,7 +38,7 @@ def stage_exe(tmp_path_factory):
         shutil.copy(os.path.join(CSRC, h), src_dir / h)
     (src_dir / "qsgd_device.cuh").write_text(_host_source(open(os.path.join(CSRC, "qsgd_device.cuh")).read()))
     enc = open(os.path.join(CSRC, "qsgd_encode_stage.cu")).read()
-    cut = enc.index("template <int V, bool kShort, bool kEF>\ncudaError_t launch_code")
+    cut = enc.index("template <class Kernel>\ncudaError_t launch_coder")
     (src_dir / "stage_emu.inc").write_text(_host_source(enc[:cut]) + "}  // namespace\n}  // namespace qsgd\n")
     exe = d / "stage_main"
     r = subprocess.run(["g++", "-O1", "-std=c++17", "-ffp-contract=off", "-pthread", "-I", EMU, "-I", str(src_dir),
@@ -140,3 +140,21 @@ def test_stage_special_values(stage_exe, tmp_path, oracle_lib):
         check_norms(gn, own_norms)
         r_words, r_offsets, _, _ = oracle_lib.encode(v, d, 16, 1, norms_in=gn)
         assert np.array_equal(offsets, r_offsets) and np.array_equal(words, r_words)
+
+
+def test_stage_lane_strings_past_96_bits(stage_exe, tmp_path, oracle_lib):
+    """A lane whose 16 coordinates all carry large levels needs more than 96 bits for
+    its records (the short coder's register string): the bucket is then placed record
+    by record, and the stream must not change."""
+    v = (W.normal(8_192, 3) * np.float32(1e-3)).astype(np.float32)
+    for b in range(0, 8_192, 512):
+        lane = (b // 512) % 32
+        v[b + 16 * lane: b + 16 * lane + 16] = np.float32(1.0)  # norm ~4: levels ~8 at s = 31
+    words, offsets, status, _ = _run(stage_exe, tmp_path, v, 512, 31, 2, 2)
+    _, _, own_norms, own_status = oracle_lib.encode(v, 512, 31, 2)
+    assert status == own_status
+    gn = stream_norms(words, offsets)
+    check_norms(gn, own_norms)
+    r_words, r_offsets, _, _ = oracle_lib.encode(v, 512, 31, 2, norms_in=gn)
+    assert np.array_equal(offsets, r_offsets) and np.array_equal(words, r_words)
+    assert int(np.diff(offsets.astype(np.int64)).max()) > 32 + 96  # some bucket took the record-by-record path
