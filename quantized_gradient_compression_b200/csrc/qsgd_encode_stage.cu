@@ -14,7 +14,8 @@
 //    slot of a staging area in the workspace, at bucket-local bit offsets, together
 //    with the bucket's bit count.  A slot holds the bucket's largest possible size.
 // 2. compact_stream: one CTA per 256 buckets scans the bit counts (a block scan and a
-//    decoupled look-back over the CTAs, Merrill & Garland 2016), writes the offsets
+//    decoupled look-back over the CTAs, Merrill & Garland 2016, read a whole CTA of
+//    predecessors at a time), writes the offsets
 //    header, and moves every bucket's bits to their stream position with funnel
 //    shifts.  An output word belongs to the bucket that holds its first bit; that
 //    bucket's warp also reads the first bits of the next bucket, so every word has
@@ -186,7 +187,7 @@ __device__ __forceinline__ void store_contig(float* p, uint32_t q0, uint32_t m, 
 // bucket where some lane needs more than 96 bits is placed record by record.
 // ---------------------------------------------------------------------------
 template <int V, bool kEF>
-__global__ void __launch_bounds__(kStageBlock) code_buckets_short(const __grid_constant__ StageArgs a) {
+__global__ void __launch_bounds__(kStageBlock, (V <= 4 ? 4 : 2)) code_buckets_short(const __grid_constant__ StageArgs a) {
     extern __shared__ __align__(16) uint32_t smem[];
     constexpr int NC = 4 * V;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -542,6 +543,8 @@ __global__ void __launch_bounds__(kCompactBlock) compact_stream(const __grid_con
     __shared__ uint32_t s_tile;
     __shared__ uint64_t s_X;
     __shared__ int s_ok;
+    __shared__ uint32_t s_first;
+    __shared__ uint64_t s_part[kCompactBlock / 32];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) s_tile = atomicAdd(&a.ctrl->ticket, 1u);  // tiles in scheduling order
     __syncthreads();
@@ -566,23 +569,62 @@ __global__ void __launch_bounds__(kCompactBlock) compact_stream(const __grid_con
         total += x;
     }
     const uint32_t excl = before + incl - L;
-    if (warp == 0) {
-        uint64_t X = 0;
-        bool ok = true;
-        if (tile == 0) {
-            if (lane == 0) st_release(&a.cdesc[0], make_desc(0, kStatePrefix, total));
-        } else {
-            if (lane == 0) st_release(&a.cdesc[tile], make_desc(0, kStateAggregate, total));
-            ok = lookback(a.cdesc, static_cast<uint32_t>(tile), 0, &a.ctrl->abort, X);
-            if (lane == 0 && ok) st_release(&a.cdesc[tile], make_desc(0, kStatePrefix, X + total));
-        }
-        if (lane == 0) {
-            s_X = X;
-            s_ok = ok;
-            if (!ok) {
-                report(a.status, QSGD_ST_LOOKBACK_TIMEOUT);
-                atomicExch(&a.ctrl->abort, 1u);
+    if (tid == 0) st_release(&a.cdesc[tile], make_desc(0, tile == 0 ? kStatePrefix : kStateAggregate, total));
+    // look-back by the whole CTA: thread i reads the descriptor of tile (window end -
+    // i), so one read covers kCompactBlock predecessors; the nearest one holding its
+    // inclusive prefix ends the walk, and every tile between must have published its
+    // bit count.  Bounded: an abort or kMaxPolls empty reads end it with an error.
+    uint64_t Xacc = 0;
+    bool ok = true;
+    if (tile > 0) {
+        int64_t wend = static_cast<int64_t>(tile) - 1;
+        uint32_t polls = 0;
+        while (wend >= 0) {
+            const int64_t idx = wend - tid;
+            uint64_t st = kStatePrefix, val = 0;  // threads past tile 0 act as a zero prefix
+            if (idx >= 0) {
+                const uint64_t dsc = ld_acquire(&a.cdesc[idx]);
+                st = desc_state(dsc);
+                val = desc_value(dsc);
             }
+            // nearest prefix: the smallest thread index holding one
+            if (tid == 0) s_first = kCompactBlock;
+            __syncthreads();
+            if (st == kStatePrefix) atomicMin(&s_first, static_cast<uint32_t>(tid));
+            __syncthreads();
+            const uint32_t first = s_first;
+            const bool wait_here = st == 0 && static_cast<uint32_t>(tid) <= first;
+            if (__syncthreads_or(wait_here)) {
+                ++polls;  // the same count in every thread
+                const bool give_up =
+                    polls > kMaxPolls || (tid == 0 && (polls & 63u) == 0 && ld_acquire32(&a.ctrl->abort) != 0);
+                if (__syncthreads_or(give_up)) {
+                    ok = false;
+                    break;
+                }
+                __nanosleep(polls < 64 ? 32 : 256);
+                continue;
+            }
+            // the window's sum up to (and with) the nearest prefix
+            uint64_t c = static_cast<uint32_t>(tid) <= first ? val : 0;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(kAll, c, o);
+            if (lane == 0) s_part[warp] = c;
+            __syncthreads();
+#pragma unroll
+            for (int w = 0; w < kCompactBlock / 32; ++w) Xacc += s_part[w];
+            __syncthreads();
+            if (first < kCompactBlock) break;
+            wend -= kCompactBlock;
+        }
+        if (tid == 0 && ok) st_release(&a.cdesc[tile], make_desc(0, kStatePrefix, Xacc + total));
+    }
+    if (tid == 0) {
+        s_X = Xacc;
+        s_ok = ok;
+        if (!ok) {
+            report(a.status, QSGD_ST_LOOKBACK_TIMEOUT);
+            atomicExch(&a.ctrl->abort, 1u);
         }
     }
     __syncthreads();
@@ -604,7 +646,7 @@ __global__ void __launch_bounds__(kCompactBlock) compact_stream(const __grid_con
     // next bucket (always >= 32 bits, so one word of it suffices).
     const uint32_t nt = static_cast<uint32_t>(min(static_cast<uint64_t>(kCompactBlock), a.nb - b0));
     const uint64_t wb = (X + 31u) >> 5, we = (X + total + 31u) >> 5;
-    constexpr int kUnroll = 4;
+    constexpr int kUnroll = 8;
     for (uint64_t w0 = wb + tid; w0 < we; w0 += kUnroll * kCompactBlock) {
         uint32_t v[kUnroll];
 #pragma unroll

@@ -49,7 +49,10 @@ constexpr int kFastMinBlocks = QSGD_FAST_MIN_BLOCKS;
 // compaction takes kCompactBlock buckets per CTA.  Whole-record table for s <= 31.
 constexpr int kStageWarps = 8;
 constexpr int kStageBlock = 32 * kStageWarps;
-constexpr int kCompactBlock = 256;
+#ifndef QSGD_COMPACT_BLOCK
+#define QSGD_COMPACT_BLOCK 256
+#endif
+constexpr int kCompactBlock = QSGD_COMPACT_BLOCK;
 constexpr uint32_t kStageMinD = 4;
 constexpr uint32_t kStageMaxD = 1024;
 constexpr uint32_t kStageShortMaxS = 31;

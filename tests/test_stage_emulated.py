@@ -26,11 +26,10 @@ CSRC = os.path.join(ROOT, "quantized_gradient_compression_b200", "csrc")
 EMU = os.path.join(HERE, "emu", "enc")
 
 
-@pytest.fixture(scope="module")
-def stage_exe(tmp_path_factory):
+def _build(tmp_path_factory, name, extra=()):
     if shutil.which("g++") is None:
         pytest.skip("g++ not available")
-    d = tmp_path_factory.mktemp("stageemu")
+    d = tmp_path_factory.mktemp(name)
     src_dir = d / "pkg" / "csrc"
     src_dir.mkdir(parents=True)
     shutil.copytree(os.path.join(ROOT, "include"), d / "include")
@@ -41,10 +40,22 @@ def stage_exe(tmp_path_factory):
     cut = enc.index("template <class Kernel>\ncudaError_t launch_coder")
     (src_dir / "stage_emu.inc").write_text(_host_source(enc[:cut]) + "}  // namespace\n}  // namespace qsgd\n")
     exe = d / "stage_main"
-    r = subprocess.run(["g++", "-O1", "-std=c++17", "-ffp-contract=off", "-pthread", "-I", EMU, "-I", str(src_dir),
-                        os.path.join(EMU, "stage_main.cpp"), "-o", str(exe)], capture_output=True, text=True)
+    r = subprocess.run(["g++", "-O1", "-std=c++17", "-ffp-contract=off", "-pthread", *extra, "-I", EMU, "-I",
+                        str(src_dir), os.path.join(EMU, "stage_main.cpp"), "-o", str(exe)], capture_output=True,
+                       text=True)
     assert r.returncode == 0, r.stderr[-4000:]
     return str(exe)
+
+
+@pytest.fixture(scope="module")
+def stage_exe(tmp_path_factory):
+    return _build(tmp_path_factory, "stageemu")
+
+
+@pytest.fixture(scope="module")
+def stage_exe_small_tiles(tmp_path_factory):
+    # compaction tiles of 32 buckets, so that the look-back walks several windows
+    return _build(tmp_path_factory, "stageemu32", ["-DQSGD_COMPACT_BLOCK=32"])
 
 
 def _omega_len(N):
@@ -158,3 +169,17 @@ def test_stage_lane_strings_past_96_bits(stage_exe, tmp_path, oracle_lib):
     r_words, r_offsets, _, _ = oracle_lib.encode(v, 512, 31, 2, norms_in=gn)
     assert np.array_equal(offsets, r_offsets) and np.array_equal(words, r_words)
     assert int(np.diff(offsets.astype(np.int64)).max()) > 32 + 96  # some bucket took the record-by-record path
+
+
+@pytest.mark.parametrize("n,d,s", [(12_000, 4, 3), (40_003, 128, 16)])
+def test_stage_lookback_over_several_windows(stage_exe_small_tiles, tmp_path, oracle_lib, n, d, s):
+    """Compaction tiles of 32 buckets: 94 and 10 tiles, so a tile's look-back reads
+    up to three windows of predecessors before it meets a prefix."""
+    v = W.layered(n, 5)
+    words, offsets, status, _ = _run(stage_exe_small_tiles, tmp_path, v, d, s, 4, 2)
+    _, _, own_norms, own_status = oracle_lib.encode(v, d, s, 4)
+    assert status == own_status
+    gn = stream_norms(words, offsets)
+    check_norms(gn, own_norms)
+    r_words, r_offsets, _, _ = oracle_lib.encode(v, d, s, 4, norms_in=gn)
+    assert np.array_equal(offsets, r_offsets) and np.array_equal(words, r_words)
