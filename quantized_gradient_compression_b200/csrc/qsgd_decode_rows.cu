@@ -10,11 +10,12 @@
 //
 // Work layout: each lane of a warp parses one bucket (buckets are independent
 // prefix-code streams located by the offsets header), 32 consecutive buckets to a
-// warp.  A record is decoded with one lookup of its first 12 bits in a shared-memory
-// table of whole records; longer records take a bit-serial path.  The lane stores the
-// record's code (sign << 7 | k, one byte, so s <= 127) at its index in its bucket's
-// row of a zeroed staging area: 32 rows of d bytes, padded so that the rows start on
-// different banks.  No lane waits for another while parsing.  Then the warp converts
+// warp.  Records are decoded through a shared-memory table of the whole records at
+// the start of a 12-bit window (up to two per entry), two lookups a step; longer
+// records take a bit-serial path.  The lane stores the
+// record's code (sign << 7 | k in a byte for s <= 127, sign << 15 | k in 16 bits for
+// s <= 32767) at its index in its bucket's row of a zeroed staging area: 32 rows of d
+// codes, padded so that the rows start on different banks.  No lane waits for another while parsing.  Then the warp converts
 // the rows to fp32, row by row, and writes each bucket with coalesced 16-byte stores
 // (decode-accumulate first reads the output, which a prefetch to L2 issued before
 // the parse has brought in).
@@ -142,14 +143,23 @@ struct RowReader {
 
 // A record the table does not hold, bit by bit: false when it is malformed (or its
 // level exceeds s).
-__device__ __forceinline__ bool slow_record(RowReader& r, uint32_t s, uint32_t& gap, uint32_t& code) {
-    uint32_t k;
+__device__ __forceinline__ bool slow_record(RowReader& r, uint32_t s, uint32_t& gap, uint32_t& sign, uint32_t& k) {
     if (!r.omega(gap) || r.left <= 0 || gap > 0xFFFFu) return false;
-    const uint32_t sign = r.peek() >> 31;
+    sign = r.peek() >> 31;
     r.advance(1);
-    if (!r.omega(k) || k > s) return false;
-    code = (sign << 7) | k;
-    return true;
+    return r.omega(k) && k <= s;
+}
+
+// A row code: sign << 7 | k in a byte (s <= 127) or sign << 15 | k in 16 bits.
+template <class T>
+__device__ __forceinline__ T row_code(uint32_t sign, uint32_t k) {
+    return static_cast<T>((sign << (8 * sizeof(T) - 1)) | k);
+}
+// A table code (sign << 7 | k, k <= 15) as a row code.
+template <class T>
+__device__ __forceinline__ T table_code(uint32_t c) {
+    if constexpr (sizeof(T) == 1) return static_cast<T>(c);
+    return static_cast<T>(((c & 0x80u) << 8) | (c & 0x7Fu));
 }
 
 // The output of bucket bb as lane `lane` reads it in the write-back: float4 i is
@@ -172,7 +182,7 @@ __device__ __forceinline__ void load_row(const DecodeArgs& a, uint64_t bb, int l
     }
 }
 
-template <int V, bool kAcc>
+template <int V, bool kAcc, class T>
 __global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows(const __grid_constant__ DecodeArgs a,
                                                                    uint32_t stride_w) {
     extern __shared__ __align__(16) uint32_t smem[];
@@ -180,7 +190,7 @@ __global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows(const __grid_c
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int W = blockDim.x >> 5;
     uint32_t* const rows = smem + kLutSize + static_cast<uint32_t>(warp) * 32u * stride_w;
-    uint8_t* const myrow = reinterpret_cast<uint8_t*>(rows + static_cast<uint32_t>(lane) * stride_w);
+    T* const myrow = reinterpret_cast<T*>(rows + static_cast<uint32_t>(lane) * stride_w);
     build_rows_lut(lut, a.s, tid, blockDim.x);
     __syncthreads();
     const StreamRef st = a.streams[0];
@@ -241,25 +251,45 @@ __global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows(const __grid_c
                 break;
             }
             if (r.left > 0) {
-                const uint32_t e = lut[r.peek() >> (32 - kLutBits)];
+                // up to two table entries a step, each up to two records: the 32 bits at
+                // the cursor hold both 12-bit windows (the first takes at most 12 bits);
+                // a record is taken only when it ends inside the bucket
+                const uint32_t w = r.peek();
+                const uint32_t e = lut[w >> (32 - kLutBits)];
                 const uint32_t len1 = e & 15u;
                 if (len1 != 0u) {
-                    // the second record only when it ends inside the bucket
                     const uint32_t len2 = (e >> 4) & 15u;
                     const bool two = static_cast<int32_t>(len2) <= r.left;
-                    r.advance(two ? len2 : len1);
+                    uint32_t used = two ? len2 : len1;
                     next += (e >> 8) & 15u;
-                    myrow[min(next - 1u, d)] = static_cast<uint8_t>(e >> 16);
+                    myrow[min(next - 1u, d)] = table_code<T>((e >> 16) & 0xFFu);
                     const uint32_t c2 = e >> 24;
                     if (two && c2 != 0u) {
                         next += (e >> 12) & 15u;
-                        myrow[min(next - 1u, d)] = static_cast<uint8_t>(c2);
+                        myrow[min(next - 1u, d)] = table_code<T>(c2);
                     }
+                    if (two) {
+                        const uint32_t f = lut[(w << used) >> (32 - kLutBits)];
+                        const uint32_t flen1 = f & 15u;
+                        if (flen1 != 0u && static_cast<int32_t>(used + flen1) <= r.left) {
+                            const uint32_t flen2 = (f >> 4) & 15u;
+                            const bool ftwo = static_cast<int32_t>(used + flen2) <= r.left;
+                            next += (f >> 8) & 15u;
+                            myrow[min(next - 1u, d)] = table_code<T>((f >> 16) & 0xFFu);
+                            const uint32_t fc2 = f >> 24;
+                            if (ftwo && fc2 != 0u) {
+                                next += (f >> 12) & 15u;
+                                myrow[min(next - 1u, d)] = table_code<T>(fc2);
+                            }
+                            used += ftwo ? flen2 : flen1;
+                        }
+                    }
+                    r.advance(used);
                 } else {
-                    uint32_t gap = 0, code = 0;
-                    if (slow_record(r, a.s, gap, code)) {
+                    uint32_t gap = 0, sign = 0, k = 0;
+                    if (slow_record(r, a.s, gap, sign, k)) {
                         next += gap;
-                        myrow[min(next - 1u, d)] = static_cast<uint8_t>(code);
+                        myrow[min(next - 1u, d)] = row_code<T>(sign, k);
                     } else {
                         bad = true;
                         r.left = 0;
@@ -291,14 +321,25 @@ __global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows(const __grid_c
                 const uint32_t q = static_cast<uint32_t>(lane) + 32u * i;
                 const uint32_t c = 4u * q;
                 if (c < mm) {
-                    const uint32_t w = rowp[q];
+                    uint32_t code[4];
+                    if constexpr (sizeof(T) == 1) {
+                        const uint32_t w = rowp[q];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) code[j] = ((w >> (8 * j)) & 0x7Fu) | (((w >> (8 * j)) & 0x80u) << 24);
+                    } else {
+                        const uint2 w = reinterpret_cast<const uint2*>(rowp)[q];
+                        code[0] = (w.x & 0x7FFFu) | ((w.x & 0x8000u) << 16);
+                        code[1] = (w.x >> 16 & 0x7FFFu) | (w.x & 0x80000000u);
+                        code[2] = (w.y & 0x7FFFu) | ((w.y & 0x8000u) << 16);
+                        code[3] = (w.y >> 16 & 0x7FFFu) | (w.y & 0x80000000u);
+                    }
                     float v[4];
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
-                        const uint32_t code = (w >> (8 * j)) & 0xFFu;
-                        // k as fp32 through the 2^23 offset (exact for k < 2^23), times the step
-                        const float kf = __fsub_rn(__uint_as_float(0x4B000000u | (code & 0x7Fu)), 8388608.0f);
-                        v[j] = __uint_as_float(__float_as_uint(__fmul_rn(sc, kf)) | ((code & 0x80u) << 24));
+                        // code[j] = k | sign << 31: k as fp32 through the 2^23 offset (exact
+                        // for k < 2^23), times the step, the sign last
+                        const float kf = __fsub_rn(__uint_as_float(0x4B000000u | (code[j] & 0x7FFFFFFFu)), 8388608.0f);
+                        v[j] = __uint_as_float(__float_as_uint(__fmul_rn(sc, kf)) | (code[j] & 0x80000000u));
                     }
                     if constexpr (kAcc) {
                         v[0] = __fadd_rn(cur[i].x, v[0]);
@@ -323,16 +364,18 @@ __global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows(const __grid_c
     }
 }
 
-// Words of one staging row: room for d codes and a padding byte, rounded so that
-// consecutive rows start on consecutive banks (stride = 1 mod 32).
-uint32_t rows_stride_words(uint32_t d) {
-    const uint32_t need = (d + 4 + 3) / 4;
-    return ((need + 30) / 32) * 32 + 1;
+// Words of one staging row: room for d codes and a padding code, rounded so that
+// consecutive rows start on different banks: stride = 1 mod 32 for byte codes;
+// for 16-bit codes even (the write-back reads 8 bytes a lane) and 2 mod 32.
+uint32_t rows_stride_words(uint32_t d, uint32_t code_bytes) {
+    const uint32_t need = (code_bytes * (d + 1) + 3) / 4;
+    const uint32_t r = code_bytes == 1 ? 1u : 2u;
+    return ((need + 31 - r) / 32) * 32 + r;
 }
 
-template <int V, bool kAcc>
+template <int V, bool kAcc, class T>
 cudaError_t launch_rows_v(const DecodeArgs& a, cudaStream_t stream) {
-    const uint32_t stride = rows_stride_words(a.d);
+    const uint32_t stride = rows_stride_words(a.d, sizeof(T));
     int dev = 0, sms = 0, optin = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -347,12 +390,22 @@ cudaError_t launch_rows_v(const DecodeArgs& a, cudaStream_t stream) {
     const size_t smem = lut_bytes + W * per_warp;
     static bool attr_set[64] = {};
     if (dev < 64 && !attr_set[dev]) {
-        cudaFuncSetAttribute(decode_rows<V, kAcc>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+        cudaFuncSetAttribute(decode_rows<V, kAcc, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
         attr_set[dev] = true;
     }
     const uint64_t blocks = std::max<uint64_t>(1, std::min<uint64_t>(static_cast<uint64_t>(sms), (groups + W - 1) / W));
-    decode_rows<V, kAcc><<<static_cast<unsigned>(blocks), 32 * W, smem, stream>>>(a, stride);
+    decode_rows<V, kAcc, T><<<static_cast<unsigned>(blocks), 32 * W, smem, stream>>>(a, stride);
     return cudaGetLastError();
+}
+
+template <class T>
+cudaError_t launch_rows_t(const DecodeArgs& a, bool accumulate, cudaStream_t stream) {
+    switch (fast_v(a.d)) {
+        case 1: return accumulate ? launch_rows_v<1, true, T>(a, stream) : launch_rows_v<1, false, T>(a, stream);
+        case 2: return accumulate ? launch_rows_v<2, true, T>(a, stream) : launch_rows_v<2, false, T>(a, stream);
+        case 4: return accumulate ? launch_rows_v<4, true, T>(a, stream) : launch_rows_v<4, false, T>(a, stream);
+        default: return accumulate ? launch_rows_v<8, true, T>(a, stream) : launch_rows_v<8, false, T>(a, stream);
+    }
 }
 
 }  // namespace
@@ -362,12 +415,7 @@ bool decode_rows_shape(uint32_t d, uint32_t s, const float* out) {
 }
 
 cudaError_t launch_decode_rows(const DecodeArgs& a, bool accumulate, cudaStream_t stream) {
-    switch (fast_v(a.d)) {
-        case 1: return accumulate ? launch_rows_v<1, true>(a, stream) : launch_rows_v<1, false>(a, stream);
-        case 2: return accumulate ? launch_rows_v<2, true>(a, stream) : launch_rows_v<2, false>(a, stream);
-        case 4: return accumulate ? launch_rows_v<4, true>(a, stream) : launch_rows_v<4, false>(a, stream);
-        default: return accumulate ? launch_rows_v<8, true>(a, stream) : launch_rows_v<8, false>(a, stream);
-    }
+    return a.s <= kRowsMaxS8 ? launch_rows_t<uint8_t>(a, accumulate, stream) : launch_rows_t<uint16_t>(a, accumulate, stream);
 }
 
 }  // namespace qsgd

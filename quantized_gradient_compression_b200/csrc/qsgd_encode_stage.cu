@@ -36,13 +36,20 @@ namespace {
 constexpr uint32_t kAll = 0xFFFFFFFFu;
 
 // Whole records omega(gap) | sign | omega(k) for gap < 64 and k < 32, indexed by
-// gap << 6 | k << 1 | sign: entry = code << 5 | length (length <= 24 bits).
+// gap << 6 | k << 1 | sign: entry = code << 5 | length (length <= 24 bits).  Gap 0
+// holds the record without its gap, sign | omega(k); k = 0 entries are empty.
 struct RecordTable64 {
     uint32_t v[kRecordTab64];
 };
 constexpr RecordTable64 make_record_table64() {
     RecordTable64 t{};
     const OmegaTable om = make_omega_table();
+    for (uint32_t k = 1; k < 32; ++k)
+        for (uint32_t sign = 0; sign < 2; ++sign) {
+            const uint32_t ke = om.v[k];
+            const uint32_t kl = ke & 0xFFu;
+            t.v[(k << 1) | sign] = (((sign << kl) | (ke >> 8)) << 5) | (1u + kl);
+        }
     for (uint32_t gap = 1; gap < 64; ++gap)
         for (uint32_t k = 1; k < 32; ++k)
             for (uint32_t sign = 0; sign < 2; ++sign) {
@@ -257,22 +264,43 @@ __global__ void __launch_bounds__(kStageBlock, (V <= 4 ? 4 : 2)) code_buckets_sh
         const uint32_t B = __ballot_sync(kAll, nzm != 0u) & lanes_below;
         const int32_t pv = __shfl_sync(kAll, last, B ? 31 - __clz(B) : 0);
         const int32_t prev_in = B ? pv : -1;
-        // --- the lane's records, appended to (w2:w1:w0), right-aligned ---------------
+        // --- the lane's records, appended to (w2:w1:w0), right-aligned: every record
+        // from the whole-record table, the lane's first one without its gap (the gaps
+        // inside a lane are below 64); that gap's omega code goes in front at the end --
         uint32_t w0 = 0, w1 = 0, w2 = 0, nbits = 0;
         {
-            int32_t prev = prev_in;
+            const uint32_t cf = nzm ? static_cast<uint32_t>(__ffs(nzm) - 1) : 0u;
+            uint32_t prev = q0 + cf;
 #pragma unroll
             for (int c = 0; c < NC; ++c) {
                 const uint32_t kv = kq[c];
-                uint32_t code = 0, len = 0;
-                if ((kv & 0x7FFFFFFFu) != 0u) {
-                    short_record(rtab, otab, static_cast<uint32_t>(static_cast<int32_t>(q0 + c) - prev), kv, code, len);
-                    prev = static_cast<int32_t>(q0 + c);
-                }
+                const uint32_t kr = __funnelshift_l(kv, kv, 1);  // k << 1 | sign
+                // below the lane's first record the gap wraps, but k = 0 there: an empty entry
+                const uint32_t e = rtab[(((q0 + c - prev) << 6) | kr) & (kRecordTab64 - 1)];
+                const uint32_t len = e & 31u;
                 w2 = __funnelshift_l(w1, w2, len);
                 w1 = __funnelshift_l(w0, w1, len);
-                w0 = (w0 << len) | code;
+                w0 = (w0 << len) | (e >> 5);
                 nbits += len;
+                prev = kr > 1u ? q0 + c : prev;
+            }
+            if (nzm) {  // omega(gap of the first record) in front of the string
+                const uint32_t ge = otab[q0 + cf - prev_in];  // gap <= d <= 1024
+                const uint32_t gl = ge & 0xFFu, gc = ge >> 8;
+                if (nbits + gl <= 96u) {
+                    const uint32_t sh = nbits & 31u;  // gc lands at bit nbits
+                    const uint32_t lo = sh ? gc << sh : gc, hi = sh ? gc >> (32u - sh) : 0u;
+                    if (nbits < 32u) {
+                        w0 |= lo;
+                        w1 |= hi;
+                    } else if (nbits < 64u) {
+                        w1 |= lo;
+                        w2 |= hi;
+                    } else {
+                        w2 |= lo;
+                    }
+                }
+                nbits += gl;
             }
         }
         // --- the lane's first bit in the bucket: scan of the bit counts ---------------

@@ -58,11 +58,13 @@ constexpr uint32_t kStageMaxD = 1024;
 constexpr uint32_t kStageShortMaxS = 31;
 
 // One-stream decoder with byte codes staged in whole bucket rows: d % 4 == 0,
-// 4 <= d <= 1024, s <= 127 (a code is sign << 7 | k), 16-byte aligned output; up to
+// 4 <= d <= 1024, s <= 32767 (a code is sign << 7 | k in a byte, or sign << 15 | k
+// in 16 bits above s = 127), 16-byte aligned output; up to
 // kRowsMaxWarps warps (32 buckets each) to a CTA, as many as the shared memory holds.
 constexpr int kRowsMaxWarps = 16;
 constexpr uint32_t kRowsMaxD = 1024;
-constexpr uint32_t kRowsMaxS = 127;
+constexpr uint32_t kRowsMaxS8 = 127;     // byte codes up to here, 16-bit codes above
+constexpr uint32_t kRowsMaxS = 32767;
 
 constexpr int kDecodeBlock = 128;
 constexpr int kMaxStreamsPerLaunch = 16;  // decode-accumulate streams per launch

@@ -48,12 +48,23 @@ static void run_grid(unsigned grid, unsigned block, size_t smem, Kernel k) {
     for (auto& x : th) x.join();
 }
 
-template <int V>
+template <int V, class T>
 static void run(const qsgd::DecodeArgs& a, bool acc, unsigned grid, unsigned W, uint32_t stride, size_t smem) {
     if (acc)
-        run_grid(grid, 32 * W, smem, [&] { qsgd::decode_rows<V, true>(a, stride); });
+        run_grid(grid, 32 * W, smem, [&] { qsgd::decode_rows<V, true, T>(a, stride); });
     else
-        run_grid(grid, 32 * W, smem, [&] { qsgd::decode_rows<V, false>(a, stride); });
+        run_grid(grid, 32 * W, smem, [&] { qsgd::decode_rows<V, false, T>(a, stride); });
+}
+template <class T>
+static void run_t(const qsgd::DecodeArgs& a, bool acc, unsigned grid, unsigned W) {
+    const uint32_t stride = qsgd::rows_stride_words(a.d, sizeof(T));
+    const size_t smem = 4 * (size_t)qsgd::kLutSize + (size_t)W * 32 * stride * 4;
+    switch (qsgd::fast_v(a.d)) {
+        case 1: run<1, T>(a, acc, grid, W, stride, smem); break;
+        case 2: run<2, T>(a, acc, grid, W, stride, smem); break;
+        case 4: run<4, T>(a, acc, grid, W, stride, smem); break;
+        default: run<8, T>(a, acc, grid, W, stride, smem); break;
+    }
 }
 
 int main(int argc, char** argv) {
@@ -85,14 +96,10 @@ int main(int argc, char** argv) {
     a.out = out.data();
     a.status = &status;
     a.first_group = 1;
-    const uint32_t stride = qsgd::rows_stride_words(d);
-    const size_t smem = 4 * (size_t)qsgd::kLutSize + (size_t)W * 32 * stride * 4;
-    switch (qsgd::fast_v(d)) {
-        case 1: run<1>(a, acc, grid, W, stride, smem); break;
-        case 2: run<2>(a, acc, grid, W, stride, smem); break;
-        case 4: run<4>(a, acc, grid, W, stride, smem); break;
-        default: run<8>(a, acc, grid, W, stride, smem); break;
-    }
+    if (s <= qsgd::kRowsMaxS8)
+        run_t<uint8_t>(a, acc, grid, W);
+    else
+        run_t<uint16_t>(a, acc, grid, W);
     if (g_emu_error) return 4;
     spit(dir + "/out.bin", out.data(), 4 * n);
     std::printf("status %u\n", status);

@@ -36,7 +36,7 @@ def rows_exe(tmp_path_factory):
         shutil.copy(os.path.join(CSRC, h), src_dir / h)
     (src_dir / "qsgd_device.cuh").write_text(_host_source(open(os.path.join(CSRC, "qsgd_device.cuh")).read()))
     src = open(os.path.join(CSRC, "qsgd_decode_rows.cu")).read()
-    cut = src.index("template <int V, bool kAcc>\ncudaError_t launch_rows_v")
+    cut = src.index("template <int V, bool kAcc, class T>\ncudaError_t launch_rows_v")
     (src_dir / "rows_emu.inc").write_text(_host_source(src[:cut]) + "}  // namespace\n}  // namespace qsgd\n")
     exe = d / "rows_main"
     r = subprocess.run(["g++", "-O1", "-std=c++17", "-ffp-contract=off", "-pthread", "-I", EMU, "-I", str(src_dir),
@@ -86,6 +86,10 @@ CASES = [
     (3_001, 4, 2, False, 2, 2, "normal"),
     (6_000, 1000, 127, False, 1, 2, "layered"),
     (1, 512, 16, True, 1, 1, "normal"),
+    # 16-bit codes (s > 127): large levels, and records the table never holds
+    (20_000, 512, 256, False, 2, 2, "normal"),
+    (20_000, 512, 256, True, 2, 2, "layered"),
+    (9_001, 100, 32767, False, 1, 3, "normal"),
 ]
 
 
@@ -107,9 +111,9 @@ def test_row_decoder_matches_oracle(rows_exe, tmp_path, oracle_lib, n, d, s, acc
     assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
 
 
-@pytest.mark.parametrize("d,accumulate", [(512, False), (128, True), (1000, False)])
-def test_row_decoder_corrupt_streams(rows_exe, tmp_path, oracle_lib, d, accumulate):
-    n, s = 30_000, 16
+@pytest.mark.parametrize("d,accumulate,s", [(512, False, 16), (128, True, 16), (1000, False, 16), (512, True, 300)])
+def test_row_decoder_corrupt_streams(rows_exe, tmp_path, oracle_lib, d, accumulate, s):
+    n = 30_000
     v = W.normal(n, 5)
     intact, offsets, _, _ = oracle_lib.encode(v, d, s, seed=3)
     words = intact.copy()
