@@ -364,6 +364,274 @@ __global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows(const __grid_c
     }
 }
 
+// ---------------------------------------------------------------------------
+// Several streams (decode-accumulate and the mean), K <= 16 to a launch.
+//
+// A warp takes 32 buckets (lane = bucket) and walks their columns in segments of
+// kMSeg.  For every segment it holds an fp32 tile of the 32 buckets' columns in
+// shared memory (the output + 0, or +0 for the first launch of a mean), decodes
+// stream 0's records of the segment and adds each value onto the tile, then stream
+// 1's, and so on: every coordinate gets its adds in stream order, the order of
+// decode-accumulate, and a stream adds nothing off its support.  The tile is then
+// written back (divided by K in the last launch of a mean).  Between segments each
+// stream's parse state (reader, next index, the record read past the segment, the
+// bucket's scale) waits in shared memory.  Records are read through a table of omega
+// gap codes (12-bit window) and one of sign | omega(k) (8-bit window), so gaps up to
+// 63 and levels up to 15 take two lookups; others take the bit-serial path.
+// ---------------------------------------------------------------------------
+constexpr int kMSeg = 64;          // columns per segment
+constexpr int kMTile = kMSeg + 1;  // tile row stride (odd: lanes' rows on different banks)
+constexpr uint32_t kNoPend = 0xFFFFFFFFu;
+
+// omega(gap) at the top of a 12-bit window: [3:0] length (0: not within 12 bits),
+// [9:4] gap (<= 63).
+__device__ void build_gap_lut(uint16_t* glut, int tid, int nthreads) {
+    for (int w = tid; w < kLutSize; w += nthreads) {
+        int pos = 0;
+        uint32_t g = 0;
+        uint32_t e = 0;
+        if (window_omega(static_cast<uint32_t>(w), kLutBits, pos, g) && g <= 63u) e = static_cast<uint32_t>(pos) | (g << 4);
+        glut[w] = static_cast<uint16_t>(e);
+    }
+}
+// sign | omega(k) at the top of an 8-bit window: [3:0] length (0: not within 8 bits,
+// or k > s), [8:4] k (<= 15), [15] sign.
+__device__ void build_level_lut(uint16_t* klut, uint32_t s, int tid, int nthreads) {
+    for (int w = tid; w < 256; w += nthreads) {
+        const uint32_t sign = static_cast<uint32_t>(w) >> 7;
+        int pos = 1;
+        uint32_t k = 0, e = 0;
+        if (window_omega(static_cast<uint32_t>(w), 8, pos, k) && k <= s && k <= 15u)
+            e = static_cast<uint32_t>(pos) | (k << 4) | (sign << 15);
+        klut[w] = static_cast<uint16_t>(e);
+    }
+}
+
+// Parse state of one stream of one bucket, kept in registers while the stream is
+// decoded and in shared memory (one array per field, [stream][lane]) in between.
+struct MsReader {
+    uint64_t wabs;  // absolute index of the next word to fetch
+    uint32_t cur, nx, off;
+    int32_t left;
+    uint32_t next;  // bucket-local index after the last record
+    uint32_t pidx;  // a record read past the segment: its index (kNoPend: none) ...
+    float pval;     // ... and value
+    float scale;
+};
+struct MsState {  // [field][stream][lane]
+    uint32_t v[10][kMaxStreamsPerLaunch][32];
+};
+__device__ __forceinline__ void ms_save(MsState& S, int j, int lane, const MsReader& r) {
+    S.v[0][j][lane] = static_cast<uint32_t>(r.wabs);
+    S.v[1][j][lane] = static_cast<uint32_t>(r.wabs >> 32);
+    S.v[2][j][lane] = r.cur;
+    S.v[3][j][lane] = r.nx;
+    S.v[4][j][lane] = r.off;
+    S.v[5][j][lane] = static_cast<uint32_t>(r.left);
+    S.v[6][j][lane] = r.next;
+    S.v[7][j][lane] = r.pidx;
+    S.v[8][j][lane] = __float_as_uint(r.pval);
+    S.v[9][j][lane] = __float_as_uint(r.scale);
+}
+__device__ __forceinline__ void ms_load(const MsState& S, int j, int lane, MsReader& r) {
+    r.wabs = S.v[0][j][lane] | (static_cast<uint64_t>(S.v[1][j][lane]) << 32);
+    r.cur = S.v[2][j][lane];
+    r.nx = S.v[3][j][lane];
+    r.off = S.v[4][j][lane];
+    r.left = static_cast<int32_t>(S.v[5][j][lane]);
+    r.next = S.v[6][j][lane];
+    r.pidx = S.v[7][j][lane];
+    r.pval = __uint_as_float(S.v[8][j][lane]);
+    r.scale = __uint_as_float(S.v[9][j][lane]);
+}
+__device__ __forceinline__ uint32_t ms_fetch(const StreamRef& st, uint64_t& wabs) {
+    const uint32_t w = wabs < st.num_words ? __ldg(st.words + wabs) : 0u;
+    ++wabs;
+    return w;
+}
+__device__ __forceinline__ void ms_advance(MsReader& r, const StreamRef& st, uint32_t n) {  // n <= 32
+    r.off += n;
+    r.left -= static_cast<int32_t>(n);
+    if (r.off >= 32u) {
+        r.cur = r.nx;
+        r.nx = ms_fetch(st, r.wabs);
+        r.off -= 32u;
+    }
+}
+__device__ __forceinline__ uint32_t ms_peek(const MsReader& r) { return __funnelshift_l(r.nx, r.cur, r.off); }
+__device__ __forceinline__ bool ms_omega(MsReader& r, const StreamRef& st, uint32_t& N) {
+    uint32_t v = 1;
+    for (;;) {
+        if (r.left <= 0) return false;
+        const uint32_t bit = ms_peek(r) >> 31;
+        ms_advance(r, st, 1);
+        if (bit == 0) {
+            N = v;
+            return true;
+        }
+        if (v > 31 || r.left < static_cast<int32_t>(v)) return false;
+        const uint32_t rest = ms_peek(r) >> (32 - v);
+        ms_advance(r, st, v);
+        v = (1u << v) | rest;
+    }
+}
+
+__global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows_multi(const __grid_constant__ DecodeArgs a) {
+    extern __shared__ __align__(16) uint32_t smem[];
+    uint16_t* const glut = reinterpret_cast<uint16_t*>(smem);
+    uint16_t* const klut = glut + kLutSize;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int W = blockDim.x >> 5;
+    char* const wbase = reinterpret_cast<char*>(smem) + (kLutSize + 256) * sizeof(uint16_t) +
+                        static_cast<size_t>(warp) * (sizeof(MsState) + 32 * kMTile * sizeof(float));
+    MsState& S = *reinterpret_cast<MsState*>(wbase);
+    float* const tile = reinterpret_cast<float*>(wbase + sizeof(MsState));
+    float* const myrow = tile + lane * kMTile;
+    build_gap_lut(glut, tid, blockDim.x);
+    build_level_lut(klut, a.s, tid, blockDim.x);
+    __syncthreads();
+    const float fs = __uint2float_rn(a.s);
+    const uint32_t d = a.d;
+    const int K = a.K;
+    const uint64_t ngroups = (a.nb + 31) / 32;
+    for (uint64_t g = blockIdx.x + static_cast<uint64_t>(gridDim.x) * warp; g < ngroups;
+         g += static_cast<uint64_t>(gridDim.x) * W) {
+        const uint64_t b = g * 32 + lane;
+        const bool live = b < a.nb;
+        const uint32_t m = live ? static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - b * d)) : 0u;
+        const int nrows = static_cast<int>(min(static_cast<uint64_t>(32), a.nb - g * 32));
+        bool bad = false;
+        // --- open this lane's bucket in every stream --------------------------------
+        for (int j = 0; j < K; ++j) {
+            const StreamRef st = a.streams[j];
+            MsReader r{0, 0, 0, 0, 0, 0, kNoPend, 0.f, 0.f};
+            if (live) {
+                const uint64_t begin = st.offsets[b];
+                const uint64_t end = st.offsets[b + 1];
+                if (!(end >= begin && end - begin >= 32 && end <= st.num_words * 32 && end - begin < (1ull << 30))) {
+                    bad = true;
+                } else {
+                    r.wabs = begin >> 5;
+                    r.cur = ms_fetch(st, r.wabs);
+                    r.nx = ms_fetch(st, r.wabs);
+                    r.off = static_cast<uint32_t>(begin & 31u);
+                    r.left = static_cast<int32_t>(end - begin);
+                    const uint32_t nbits = ms_peek(r);
+                    ms_advance(r, st, 32);
+                    const float norm = __uint_as_float(nbits);
+                    if (nbits == 0) {
+                        bad = bad || r.left != 0;
+                        r.left = 0;
+                    } else if (!(isfinite(norm) && norm > 0.f)) {
+                        bad = true;
+                        r.left = 0;
+                    } else {
+                        r.scale = __fdiv_rn(norm, fs);
+                        if (!(r.scale > 0.f) && r.left != 0) {  // a zero scale carries no records
+                            bad = true;
+                            r.left = 0;
+                        }
+                    }
+                }
+            }
+            ms_save(S, j, lane, r);
+        }
+        for (uint32_t lo = 0; lo < d; lo += kMSeg) {
+            const uint32_t hi = lo + kMSeg;
+            const uint32_t ncols = min(static_cast<uint32_t>(kMSeg), d - lo);
+            // --- the tile: the output + 0 (canonical zeros), or +0 ---------------------
+            for (int rr = 0; rr < nrows; ++rr) {
+                const uint64_t bb = g * 32 + rr;
+                const uint32_t mm = static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - bb * d));
+                const float* gp = a.out + bb * d + lo;
+#pragma unroll
+                for (int c0 = 0; c0 < kMSeg; c0 += 32) {
+                    const uint32_t c = static_cast<uint32_t>(c0 + lane);
+                    float v = 0.f;
+                    if (!a.start_zero && c < ncols && lo + c < mm) v = __fadd_rn(gp[c], 0.0f);
+                    tile[rr * kMTile + c] = v;
+                }
+            }
+            __syncwarp();
+            // --- the streams, in order --------------------------------------------------
+            for (int j = 0; j < K; ++j) {
+                const StreamRef st = a.streams[j];
+                MsReader r;
+                ms_load(S, j, lane, r);
+                if (r.pidx < hi) {
+                    myrow[r.pidx - lo] = __fadd_rn(myrow[r.pidx - lo], r.pval);
+                    r.pidx = kNoPend;
+                }
+                for (uint32_t it = 0; it < kParseGuard; ++it) {
+                    const bool act = r.pidx == kNoPend && r.left > 0;
+                    if (!__any_sync(kWarpAll, act)) break;
+                    if (act) {
+                        uint32_t gap = 0, k = 0, sign = 0;
+                        bool ok = false;
+                        const uint32_t w = ms_peek(r);
+                        const uint32_t ge = glut[w >> (32 - kLutBits)];
+                        const uint32_t gl = ge & 15u;
+                        const uint32_t ke = gl ? klut[(w << gl) >> 24] : 0u;
+                        const uint32_t kl = ke & 15u;
+                        if (kl != 0u) {
+                            gap = (ge >> 4) & 63u;
+                            k = (ke >> 4) & 31u;
+                            sign = ke >> 15;
+                            ms_advance(r, st, gl + kl);
+                            ok = r.left >= 0;
+                        } else if (ms_omega(r, st, gap) && r.left > 0 && gap <= 0xFFFFu) {
+                            sign = ms_peek(r) >> 31;
+                            ms_advance(r, st, 1);
+                            ok = ms_omega(r, st, k) && k <= a.s;
+                        }
+                        const uint32_t idx = r.next + gap - 1u;
+                        if (!ok || idx >= m) {
+                            bad = true;
+                            r.left = 0;
+                        } else {
+                            r.next = idx + 1u;
+                            const float q = __fmul_rn(r.scale, __uint2float_rn(k));
+                            const float val = sign ? -q : q;
+                            if (idx < hi) {
+                                myrow[idx - lo] = __fadd_rn(myrow[idx - lo], val);
+                            } else {
+                                r.pidx = idx;
+                                r.pval = val;
+                            }
+                        }
+                    }
+                }
+                ms_save(S, j, lane, r);
+            }
+            __syncwarp();
+            // --- the tile back to the output --------------------------------------------
+            const bool last = a.div != 0.f;
+            for (int rr = 0; rr < nrows; ++rr) {
+                const uint64_t bb = g * 32 + rr;
+                const uint32_t mm = static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - bb * d));
+                float* gp = a.out + bb * d + lo;
+#pragma unroll
+                for (int c0 = 0; c0 < kMSeg; c0 += 32) {
+                    const uint32_t c = static_cast<uint32_t>(c0 + lane);
+                    if (c < ncols && lo + c < mm) {
+                        const float v = tile[rr * kMTile + c];
+                        gp[c] = last ? __fdiv_rn(v, a.div) : v;
+                    }
+                }
+            }
+            __syncwarp();
+        }
+        // every stream's bucket consumed exactly, every index below m
+        for (int j = 0; j < K && live && !bad; ++j) {
+            MsReader r;
+            ms_load(S, j, lane, r);
+            if (r.left != 0 || r.next > m || r.pidx != kNoPend) bad = true;
+        }
+        if (bad) atomicOr(a.status, QSGD_ST_BAD_STREAM);
+        __syncwarp();
+    }
+}
+
 // Words of one staging row: room for d codes and a padding code, rounded so that
 // consecutive rows start on different banks: stride = 1 mod 32 for byte codes;
 // for 16-bit codes even (the write-back reads 8 bytes a lane) and 2 mod 32.
@@ -398,6 +666,28 @@ cudaError_t launch_rows_v(const DecodeArgs& a, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
+cudaError_t launch_rows_multi(const DecodeArgs& a, cudaStream_t stream) {
+    int dev = 0, sms = 0, optin = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    const size_t per_warp = sizeof(MsState) + 32 * kMTile * sizeof(float);
+    const size_t luts = (kLutSize + 256) * sizeof(uint16_t);
+    const int W_fit = static_cast<int>(std::min<size_t>(kRowsMaxWarps, (static_cast<size_t>(optin) - luts - 1024) / per_warp));
+    if (W_fit < 1) return cudaErrorInvalidConfiguration;
+    const uint64_t groups = (a.nb + 31) / 32;
+    const int W = static_cast<int>(std::max<uint64_t>(1, std::min<uint64_t>(W_fit, (groups + sms - 1) / sms)));
+    const size_t smem = luts + W * per_warp;
+    static bool attr_set[64] = {};
+    if (dev < 64 && !attr_set[dev]) {
+        cudaFuncSetAttribute(decode_rows_multi, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+        attr_set[dev] = true;
+    }
+    const uint64_t blocks = std::max<uint64_t>(1, std::min<uint64_t>(static_cast<uint64_t>(sms), (groups + W - 1) / W));
+    decode_rows_multi<<<static_cast<unsigned>(blocks), 32 * W, smem, stream>>>(a);
+    return cudaGetLastError();
+}
+
 template <class T>
 cudaError_t launch_rows_t(const DecodeArgs& a, bool accumulate, cudaStream_t stream) {
     switch (fast_v(a.d)) {
@@ -413,6 +703,8 @@ cudaError_t launch_rows_t(const DecodeArgs& a, bool accumulate, cudaStream_t str
 bool decode_rows_shape(uint32_t d, uint32_t s, const float* out) {
     return d % 4 == 0 && d >= 4 && d <= kRowsMaxD && s <= kRowsMaxS && (reinterpret_cast<uintptr_t>(out) & 15u) == 0;
 }
+
+cudaError_t launch_decode_rows_multi(const DecodeArgs& a, cudaStream_t stream) { return launch_rows_multi(a, stream); }
 
 cudaError_t launch_decode_rows(const DecodeArgs& a, bool accumulate, cudaStream_t stream) {
     return a.s <= kRowsMaxS8 ? launch_rows_t<uint8_t>(a, accumulate, stream) : launch_rows_t<uint16_t>(a, accumulate, stream);

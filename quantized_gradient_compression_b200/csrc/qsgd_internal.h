@@ -155,6 +155,8 @@ cudaError_t launch_decode(const DecodeArgs& a, bool accumulate, cudaStream_t str
 // The one-stream decoder with whole rows staged as byte codes (qsgd_decode_rows.cu).
 bool decode_rows_shape(uint32_t d, uint32_t s, const float* out);
 cudaError_t launch_decode_rows(const DecodeArgs& a, bool accumulate, cudaStream_t stream);
+// Several streams (decode-accumulate and the mean) on the same shapes (qsgd_decode_rows.cu).
+cudaError_t launch_decode_rows_multi(const DecodeArgs& a, cudaStream_t stream);
 // Whether the one-lane-per-bucket decoders (and the several-stream kernel, which
 // start_zero / div need) take this shape.
 bool decode_fast_shape(uint32_t d, uint32_t s, const float* out);

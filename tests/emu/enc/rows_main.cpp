@@ -67,10 +67,33 @@ static void run_t(const qsgd::DecodeArgs& a, bool acc, unsigned grid, unsigned W
     }
 }
 
+// Several streams: decode_rows_multi over K streams, 16 to a launch as the library
+// sends them (a mean starts the first launch from +0 and divides in the last).
+static void run_multi(qsgd::DecodeArgs a, const std::vector<std::vector<unsigned char>>& ws,
+                      const std::vector<std::vector<unsigned char>>& os, bool mean, unsigned grid, unsigned W) {
+    const int K = (int)ws.size();
+    const size_t smem = (qsgd::kLutSize + 256) * 2 + (size_t)W * (sizeof(qsgd::MsState) + 32 * qsgd::kMTile * 4);
+    for (int j0 = 0; j0 < K; j0 += qsgd::kMaxStreamsPerLaunch) {
+        a.K = std::min(K - j0, qsgd::kMaxStreamsPerLaunch);
+        a.first_group = j0 == 0;
+        a.start_zero = mean && j0 == 0;
+        a.div = mean && j0 + a.K == K ? (float)K : 0.f;
+        for (int j = 0; j < a.K; ++j) {
+            a.streams[j].words = reinterpret_cast<const uint32_t*>(ws[j0 + j].data());
+            a.streams[j].num_words = ws[j0 + j].size() / 4;
+            a.streams[j].offsets = reinterpret_cast<const uint64_t*>(os[j0 + j].data());
+        }
+        run_grid(grid, 32 * W, smem, [&] { qsgd::decode_rows_multi(a); });
+        if (g_emu_error) return;
+    }
+}
+
 int main(int argc, char** argv) {
     const std::string dir = argv[1];
     const bool acc = std::atoi(argv[2]) != 0;
     const unsigned grid = std::atoi(argv[3]), W = std::atoi(argv[4]);
+    const int K = argc > 5 ? std::atoi(argv[5]) : 1;
+    const bool mean = argc > 6 && std::atoi(argv[6]) != 0;
     auto prm = slurp(dir + "/params.bin");
     uint64_t q[3];
     std::memcpy(q, prm.data(), sizeof q);
@@ -87,6 +110,20 @@ int main(int argc, char** argv) {
     std::vector<float> out(n + 4);
     std::memcpy(out.data(), xb.data(), 4 * n);
     uint32_t status = 0;
+    if (K > 1 || mean) {
+        std::vector<std::vector<unsigned char>> ws(K), os(K);
+        for (int j = 0; j < K; ++j) {
+            ws[j] = slurp(dir + "/w" + std::to_string(j) + ".bin");
+            os[j] = slurp(dir + "/o" + std::to_string(j) + ".bin");
+        }
+        qsgd::DecodeArgs a{};
+        a.n = n; a.d = d; a.s = s; a.nb = nb; a.out = out.data(); a.status = &status;
+        run_multi(a, ws, os, mean, grid, W);
+        if (g_emu_error) return 4;
+        spit(dir + "/out.bin", out.data(), 4 * n);
+        std::printf("status %u\n", status);
+        return 0;
+    }
     qsgd::DecodeArgs a{};
     a.streams[0].words = words.data();
     a.streams[0].num_words = wb.size() / 4;

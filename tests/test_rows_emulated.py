@@ -134,3 +134,73 @@ def test_row_decoder_corrupt_streams(rows_exe, tmp_path, oracle_lib, d, accumula
             keep[b * d:min(n, (b + 1) * d)] = False
     assert keep.any() and not keep.all()
     assert np.array_equal(got[keep].view(np.uint32), ref[keep].view(np.uint32))
+
+
+# decode_rows_multi: K streams added onto fp32 tiles in stream order, decode-accumulate
+# and the mean; past one launch (16 streams); sparse and dense streams, ragged shapes
+MULTI = [
+    (20_003, 512, 4, 3, False, "small_normal"),
+    (20_003, 512, 16, 2, True, "layered"),
+    (9_001, 128, 4, 17, False, "small_normal"),
+    (7_000, 100, 7, 5, True, "normal"),
+    (5_000, 1000, 300, 3, False, "normal"),
+    (3_000, 512, 1, 18, True, "heavy_tailed_sparse"),
+]
+
+
+def _run_multi(exe, tmp, streams, n, d, s, mean, base, grid=2, warps=2):
+    for j, (w, o) in enumerate(streams):
+        np.concatenate([w, np.zeros(1, np.uint32)]).tofile(tmp / ("w%d.bin" % j))
+        o.astype(np.uint64).tofile(tmp / ("o%d.bin" % j))
+    base.tofile(tmp / "out_in.bin")
+    np.array([n, d, s], np.uint64).tofile(tmp / "params.bin")
+    r = subprocess.run([exe, str(tmp), "1", str(grid), str(warps), str(len(streams)), "1" if mean else "0"],
+                       capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, (r.stdout[-500:], r.stderr[-2000:])
+    return np.fromfile(tmp / "out.bin", np.float32), int(r.stdout.split()[-1])
+
+
+@pytest.mark.parametrize("n,d,s,K,mean,kind", MULTI, ids=["n%d-d%d-s%d-K%d-mean%d-%s" % c for c in MULTI])
+def test_row_multi_decoder_matches_oracle(rows_exe, tmp_path, oracle_lib, n, d, s, K, mean, kind):
+    streams = []
+    for j in range(K):
+        v = W.GENERATORS[kind](n, 50 + j)
+        w, o, _, st = oracle_lib.encode(v, d, s, seed=j)
+        assert st == 0
+        streams.append((w, o))
+    base = _base(n, d, True)
+    got, status = _run_multi(rows_exe, tmp_path, streams, n, d, s, mean, base)
+    assert status == 0
+    if mean:
+        ref, rst = oracle_lib.decode_mean(streams, n, d, s)
+    else:
+        ref = base.copy()
+        _, rst = oracle_lib.decode_accumulate(streams, n, d, s, ref)
+    assert rst == 0
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+
+
+def test_row_multi_decoder_corrupt_stream(rows_exe, tmp_path, oracle_lib):
+    n, d, s, K = 20_000, 512, 4, 3
+    intact, streams = [], []
+    for j in range(K):
+        w, o, _, _ = oracle_lib.encode(W.small_normal(n, 70 + j), d, s, seed=j)
+        intact.append((w, o))
+        w2 = w.copy()
+        if j == 1:
+            _flip_bits(w2, o, np.random.default_rng(9))
+        streams.append((w2, o))
+    base = _base(n, d, True)
+    got, status = _run_multi(rows_exe, tmp_path, streams, n, d, s, False, base)
+    assert status & 2
+    ref = base.copy()
+    oracle_lib.decode_accumulate(intact, n, d, s, ref)
+    keep = np.ones(n, dtype=bool)
+    flipped = streams[1][0] != intact[1][0]
+    offs = intact[1][1]
+    for b in range(offs.size - 1):
+        w0, w1 = int(offs[b]) >> 5, (int(offs[b + 1]) + 31) >> 5
+        if flipped[w0:w1].any():
+            keep[b * d:min(n, (b + 1) * d)] = False
+    assert keep.any() and not keep.all()
+    assert np.array_equal(got[keep].view(np.uint32), ref[keep].view(np.uint32))
