@@ -64,6 +64,12 @@ WorkspaceLayout workspace_layout(uint64_t n, uint32_t d) {
     return L;
 }
 
+bool stage_shape(uint32_t d, uint32_t s) {
+    if (d < kStageMinD || d % 4 != 0 || d > (s <= kStageShortMaxS ? kStageShortMaxD : kStageMaxD)) return false;
+    const uint64_t slot_bits = 32u + static_cast<uint64_t>(d) * (2u + omega_len_host(s));
+    return stage_smem_bytes(s, static_cast<uint32_t>(ceil_div(slot_bits, 32)) + 1u) <= 200 * 1024;
+}
+
 StageLayout stage_layout(uint64_t n, uint32_t d, uint32_t s) {
     StageLayout L{};
     const uint64_t nb = n ? ceil_div(n, d) : 0;
@@ -99,7 +105,7 @@ static size_t one_pass_workspace_bytes(uint64_t n, uint32_t d, uint32_t s) {
 
 size_t qsgd_encode_workspace_bytes(uint64_t n, uint32_t d, uint32_t s) {
     const size_t one = one_pass_workspace_bytes(n, d, s);
-    if (one == 0 || !stage_shape(d)) return one;
+    if (one == 0 || !stage_shape(d, s)) return one;
     return std::max(one, stage_layout(n, d, s).total);
 }
 
@@ -240,7 +246,7 @@ int encode_entry(const float* d_in, float* d_ef, uint64_t n, uint32_t d, uint32_
                             d_status, stream, a, fast);
     if (rc != QSGD_OK) return rc == kNothingToDo ? QSGD_OK : rc;
     if (strict && ws_bytes < qsgd_encode_workspace_bytes(n, d, s)) return QSGD_ERR_WORKSPACE;
-    if (stage_shape(d) && aligned16(d_in) && (!d_ef || aligned16(d_ef)) &&
+    if (stage_shape(d, s) && aligned16(d_in) && (!d_ef || aligned16(d_ef)) &&
         ws_bytes >= stage_layout(n, d, s).total) {
         // two launches: bucket coder (with the memory fused in), compaction
         return launch_encode_stage(stage_args(a, d_ef, seed, d_ws), stream) == cudaSuccess ? QSGD_OK : QSGD_ERR_CUDA;

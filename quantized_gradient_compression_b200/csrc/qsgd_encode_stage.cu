@@ -193,10 +193,169 @@ __device__ __forceinline__ void store_contig(float* p, uint32_t q0, uint32_t m, 
 // them and ORs the string into the bucket buffer once its position is known.  A
 // bucket where some lane needs more than 96 bits is placed record by record.
 // ---------------------------------------------------------------------------
+// Codes one chunk of a bucket for the short coder: lane L holds the values x[] (p,
+// for error feedback) of the NC = 4V consecutive coordinates lo + NC L + c; their
+// global index is base + that.  carry: the bucket-local index of the last record
+// before the chunk (-1 before the first); pos: the bucket-local bit where the chunk's
+// records start.  Both advance past the chunk.  The chunk's bits are ORed into the
+// zeroed bucket buffer.
+template <int V, bool kEF>
+__device__ __forceinline__ void code_chunk(const StageArgs& a, const uint32_t* rtab, const uint32_t* otab, uint32_t* buf,
+                                           float (&x)[4 * V], float (&ev)[kEF ? 4 * V : 1], const BucketScale& sc,
+                                           uint64_t base, uint32_t lo, uint32_t m, int lane, int32_t& carry,
+                                           uint32_t& pos) {
+    constexpr int NC = 4 * V;
+    const uint32_t q0 = lo + static_cast<uint32_t>(NC * lane);  // bucket-local index of x[0]
+    const uint32_t lanes_below = (1u << lane) - 1u;
+    // --- levels: one Philox block per four coordinates ---------------------------------
+    uint32_t kq[NC];  // level | sign << 31
+    const uint32_t j0 = static_cast<uint32_t>((base + q0) >> 2);
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+        const uint4 r = philox_rk(j0 + j, a.rk);
+        const uint32_t rw[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const float v = x[4 * j + c];
+            kq[4 * j + c] = level_of(v, sc.sinv, rw[c], a.s) | (__float_as_uint(v) & 0x80000000u);
+        }
+    }
+    if constexpr (kEF) {  // the memory keeps p minus what a receiver decodes
+        if (sc.good) {
+            const float scale = __fdiv_rn(sc.sent, __uint2float_rn(a.s));
+#pragma unroll
+            for (int q = 0; q < NC; ++q) ev[q] = ef_residual(x[q], kq[q] & 0x7FFFFFFFu, kq[q] >> 31, scale);
+            store_contig<V>(a.ef + base, q0, m, ev);
+        }
+    }
+    // --- gap chain: the last record before this lane's coordinates ------------------------
+    uint32_t nzm = 0;
+#pragma unroll
+    for (int c = 0; c < NC; ++c) nzm |= ((kq[c] & 0x7FFFFFFFu) != 0u ? 1u : 0u) << c;
+    const int32_t last = nzm ? static_cast<int32_t>(q0 + 31u - __clz(nzm)) : -1;
+    const uint32_t any = __ballot_sync(kAll, nzm != 0u);
+    const uint32_t B = any & lanes_below;
+    const int32_t pv = __shfl_sync(kAll, last, B ? 31 - __clz(B) : 0);
+    const int32_t prev_in = B ? pv : carry;
+    const int32_t top = __shfl_sync(kAll, last, any ? 31 - __clz(any) : 0);
+    carry = any ? top : carry;
+    // --- the lane's records, appended to (w2:w1:w0), right-aligned: every record from the
+    // whole-record table, the lane's first one without its gap (the gaps inside a lane
+    // are below 64); that gap's omega code goes in front at the end -----------------------
+    uint32_t w0 = 0, w1 = 0, w2 = 0, nbits = 0;
+    {
+        const uint32_t cf = nzm ? static_cast<uint32_t>(__ffs(nzm) - 1) : 0u;
+        uint32_t prev = q0 + cf;
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
+            const uint32_t kv = kq[c];
+            const uint32_t kr = __funnelshift_l(kv, kv, 1);  // k << 1 | sign
+            // below the lane's first record the gap wraps, but k = 0 there: an empty entry
+            const uint32_t e = rtab[(((q0 + c - prev) << 6) | kr) & (kRecordTab64 - 1)];
+            const uint32_t len = e & 31u;
+            w2 = __funnelshift_l(w1, w2, len);
+            w1 = __funnelshift_l(w0, w1, len);
+            w0 = (w0 << len) | (e >> 5);
+            nbits += len;
+            prev = kr > 1u ? q0 + c : prev;
+        }
+        if (nzm) {  // omega(gap of the first record) in front of the string
+            const uint32_t gap = static_cast<uint32_t>(static_cast<int32_t>(q0 + cf) - prev_in);
+            uint32_t gl, gc;
+            if (gap < static_cast<uint32_t>(kOmegaTab)) {
+                const uint32_t ge = otab[gap];
+                gl = ge & 0xFFu;
+                gc = ge >> 8;
+            } else {  // gap <= d <= 16384: omega code of at most 22 bits
+                uint64_t c64;
+                omega_compute(gap, c64, gl);
+                gc = static_cast<uint32_t>(c64);
+            }
+            if (nbits + gl <= 96u) {
+                const uint32_t sh = nbits & 31u;  // gc lands at bit nbits
+                const uint32_t glo = sh ? gc << sh : gc, ghi = sh ? gc >> (32u - sh) : 0u;
+                if (nbits < 32u) {
+                    w0 |= glo;
+                    w1 |= ghi;
+                } else if (nbits < 64u) {
+                    w1 |= glo;
+                    w2 |= ghi;
+                } else {
+                    w2 |= glo;
+                }
+            }
+            nbits += gl;
+        }
+    }
+    // --- the lane's first bit: scan of the bit counts --------------------------------------
+    uint32_t incl = nbits;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t t = __shfl_up_sync(kAll, incl, o);
+        if (lane >= o) incl += t;
+    }
+    const uint32_t P = pos + incl - nbits;
+    pos += __shfl_sync(kAll, incl, 31);
+    if (!__any_sync(kAll, nbits > 96u)) {
+        if (nbits != 0u) {
+            // left-align the string in 96 bits, then OR it in at bit P
+            const uint32_t sa = 96u - nbits, bsh = sa & 31u, wsh = sa >> 5;
+            const uint32_t t2 = __funnelshift_l(w1, w2, bsh), t1 = __funnelshift_l(w0, w1, bsh), t0 = w0 << bsh;
+            const uint32_t L0 = wsh == 0 ? t2 : wsh == 1 ? t1 : t0;
+            const uint32_t L1 = wsh == 0 ? t1 : wsh == 1 ? t0 : 0u;
+            const uint32_t L2 = wsh == 0 ? t0 : 0u;
+            const uint32_t wp = P >> 5, sh = P & 31u;
+            const uint32_t nw = (sh + nbits + 31u) >> 5;  // 1..4
+            atomicOr(&buf[wp], L0 >> sh);
+            if (nw > 1) atomicOr(&buf[wp + 1], __funnelshift_r(L1, L0, sh));
+            if (nw > 2) atomicOr(&buf[wp + 2], __funnelshift_r(L2, L1, sh));
+            if (nw > 3) atomicOr(&buf[wp + 3], __funnelshift_r(0u, L2, sh));
+        }
+    } else {  // some lane's string is longer than 96 bits: record by record
+        int32_t prev = prev_in;
+        uint32_t p = P;
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
+            const uint32_t kv = kq[c];
+            if ((kv & 0x7FFFFFFFu) != 0u) {
+                const uint32_t gap = static_cast<uint32_t>(static_cast<int32_t>(q0 + c) - prev);
+                prev = static_cast<int32_t>(q0 + c);
+                if (gap < static_cast<uint32_t>(kOmegaTab)) {
+                    uint32_t code, len;
+                    short_record(rtab, otab, gap, kv, code, len);
+                    put_bits(buf, p, code, len);
+                    p += len;
+                } else {  // a gap past the omega table: its code, then sign | omega(k)
+                    uint64_t gcode;
+                    uint32_t glen;
+                    omega_compute(gap, gcode, glen);
+                    put_bits64(buf, p, gcode, glen);
+                    p += glen;
+                    const uint32_t ke = otab[kv & 0x7FFFFFFFu];
+                    const uint32_t kl = ke & 0xFFu;
+                    put_bits(buf, p, ((kv >> 31) << kl) | (ke >> 8), 1u + kl);
+                    p += 1u + kl;
+                }
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// 1a. Bucket coder for s <= 31 (records of up to 30 bits, plus a first gap up to d).
+// Lane L holds NC = 4V consecutive coordinates of a chunk of 128V, so a chunk is one
+// run: one gap chain over the lanes (a ballot and a shuffle) and one scan of the
+// lanes' bit counts.  A lane appends its records to a 96-bit register string as it
+// codes them and ORs the string into the bucket buffer once its position is known; a
+// chunk where some lane needs more than 96 bits is placed record by record.  A bucket
+// of one chunk keeps its values in registers; a longer one (d > 128V) is read twice:
+// for its norm, then chunk by chunk for its records.
+// ---------------------------------------------------------------------------
 template <int V, bool kEF>
 __global__ void __launch_bounds__(kStageBlock, (V <= 4 ? 4 : 2)) code_buckets_short(const __grid_constant__ StageArgs a) {
     extern __shared__ __align__(16) uint32_t smem[];
     constexpr int NC = 4 * V;
+    constexpr uint32_t kChunkCoords = 128u * V;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     uint32_t* const otab = smem;                                                  // omega table
     uint32_t* const rtab = smem + kOmegaTab;                                      // record table
@@ -214,137 +373,108 @@ __global__ void __launch_bounds__(kStageBlock, (V <= 4 ? 4 : 2)) code_buckets_sh
     __syncthreads();
 
     const uint32_t d = a.d;
-    const uint32_t q0 = static_cast<uint32_t>(NC * lane);
-    const uint32_t lanes_below = (1u << lane) - 1u;
+    const uint32_t ql = static_cast<uint32_t>(NC * lane);  // lane offset inside a chunk
     const uint64_t gwarps = static_cast<uint64_t>(gridDim.x) * kStageWarps;
     for (uint64_t b = static_cast<uint64_t>(blockIdx.x) * kStageWarps + warp; b < a.nb; b += gwarps) {
         const uint64_t base = b * d;
         const uint32_t m = static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - base));
         float x[NC];
         float ev[kEF ? NC : 1];
-        load_contig<V>(a.in + base, q0, m, x);
-        if constexpr (kEF) {  // p = e + g
-            load_contig<V>(a.ef + base, q0, m, ev);
+        int32_t carry = -1;
+        uint32_t pos = 32u;
+        if (m <= kChunkCoords) {
+            // --- one chunk: the values stay in registers ---------------------------------
+            load_contig<V>(a.in + base, ql, m, x);
+            if constexpr (kEF) {  // p = e + g
+                load_contig<V>(a.ef + base, ql, m, ev);
 #pragma unroll
-            for (int q = 0; q < NC; ++q) x[q] = __fadd_rn(ev[q], x[q]);
-        }
-        const float norm = a.norm_kind == QSGD_NORM_MAX ? warp_bucket_maxnorm<NC>(x) : warp_bucket_norm<NC>(x, true);
-        const BucketScale sc = bucket_scale(norm, a.s, true, a.status, lane == 0);
-        if (!sc.good) {  // sent as a zero bucket; the memory keeps p
-            if constexpr (kEF) store_contig<V>(a.ef + base, q0, m, x);
-#pragma unroll
-            for (int q = 0; q < NC; ++q) x[q] = 0.f;
-        }
-        // --- levels: one Philox block per four coordinates -------------------------
-        uint32_t kq[NC];  // level | sign << 31
-        const uint32_t j0 = static_cast<uint32_t>((base + q0) >> 2);
-#pragma unroll
-        for (int j = 0; j < V; ++j) {
-            const uint4 r = philox_rk(j0 + j, a.rk);
-            const uint32_t rw[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const float v = x[4 * j + c];
-                kq[4 * j + c] = level_of(v, sc.sinv, rw[c], a.s) | (__float_as_uint(v) & 0x80000000u);
+                for (int q = 0; q < NC; ++q) x[q] = __fadd_rn(ev[q], x[q]);
             }
-        }
-        if constexpr (kEF) {  // the memory keeps p minus what a receiver decodes
-            if (sc.good) {
-                const float scale = __fdiv_rn(sc.sent, __uint2float_rn(a.s));
+            const float norm =
+                a.norm_kind == QSGD_NORM_MAX ? warp_bucket_maxnorm<NC>(x) : warp_bucket_norm<NC>(x, true);
+            const BucketScale sc = bucket_scale(norm, a.s, true, a.status, lane == 0);
+            if (!sc.good) {  // sent as a zero bucket; the memory keeps p
+                if constexpr (kEF) store_contig<V>(a.ef + base, ql, m, x);
 #pragma unroll
-                for (int q = 0; q < NC; ++q) ev[q] = ef_residual(x[q], kq[q] & 0x7FFFFFFFu, kq[q] >> 31, scale);
-                store_contig<V>(a.ef + base, q0, m, ev);
+                for (int q = 0; q < NC; ++q) x[q] = 0.f;
             }
-        }
-        // --- gap chain: the last record before this lane's coordinates ----------------
-        uint32_t nzm = 0;
+            code_chunk<V, kEF>(a, rtab, otab, buf, x, ev, sc, base, 0u, m, lane, carry, pos);
+            if (lane == 0) buf[0] = __float_as_uint(sc.sent);
+        } else {
+            // --- several chunks: the norm over the whole bucket first ---------------------
+            float ss = 0.f, mx = 0.f;
+            bool nan = false;
+            for (uint32_t lo = 0; lo < m; lo += kChunkCoords) {
+                load_contig<V>(a.in + base, lo + ql, m, x);
+                if constexpr (kEF) {
+                    load_contig<V>(a.ef + base, lo + ql, m, ev);
 #pragma unroll
-        for (int c = 0; c < NC; ++c) nzm |= ((kq[c] & 0x7FFFFFFFu) != 0u ? 1u : 0u) << c;
-        const int32_t last = nzm ? static_cast<int32_t>(q0 + 31u - __clz(nzm)) : -1;
-        const uint32_t B = __ballot_sync(kAll, nzm != 0u) & lanes_below;
-        const int32_t pv = __shfl_sync(kAll, last, B ? 31 - __clz(B) : 0);
-        const int32_t prev_in = B ? pv : -1;
-        // --- the lane's records, appended to (w2:w1:w0), right-aligned: every record
-        // from the whole-record table, the lane's first one without its gap (the gaps
-        // inside a lane are below 64); that gap's omega code goes in front at the end --
-        uint32_t w0 = 0, w1 = 0, w2 = 0, nbits = 0;
-        {
-            const uint32_t cf = nzm ? static_cast<uint32_t>(__ffs(nzm) - 1) : 0u;
-            uint32_t prev = q0 + cf;
+                    for (int q = 0; q < NC; ++q) x[q] = __fadd_rn(ev[q], x[q]);
+                }
 #pragma unroll
-            for (int c = 0; c < NC; ++c) {
-                const uint32_t kv = kq[c];
-                const uint32_t kr = __funnelshift_l(kv, kv, 1);  // k << 1 | sign
-                // below the lane's first record the gap wraps, but k = 0 there: an empty entry
-                const uint32_t e = rtab[(((q0 + c - prev) << 6) | kr) & (kRecordTab64 - 1)];
-                const uint32_t len = e & 31u;
-                w2 = __funnelshift_l(w1, w2, len);
-                w1 = __funnelshift_l(w0, w1, len);
-                w0 = (w0 << len) | (e >> 5);
-                nbits += len;
-                prev = kr > 1u ? q0 + c : prev;
+                for (int q = 0; q < NC; ++q) {
+                    ss = __fmaf_rn(x[q], x[q], ss);
+                    mx = fmaxf(mx, fabsf(x[q]));
+                    nan |= isnan(x[q]);
+                }
             }
-            if (nzm) {  // omega(gap of the first record) in front of the string
-                const uint32_t ge = otab[q0 + cf - prev_in];  // gap <= d <= 1024
-                const uint32_t gl = ge & 0xFFu, gc = ge >> 8;
-                if (nbits + gl <= 96u) {
-                    const uint32_t sh = nbits & 31u;  // gc lands at bit nbits
-                    const uint32_t lo = sh ? gc << sh : gc, hi = sh ? gc >> (32u - sh) : 0u;
-                    if (nbits < 32u) {
-                        w0 |= lo;
-                        w1 |= hi;
-                    } else if (nbits < 64u) {
-                        w1 |= lo;
-                        w2 |= hi;
-                    } else {
-                        w2 |= lo;
+            float norm;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                ss = __fadd_rn(ss, __shfl_xor_sync(kAll, ss, o));
+                mx = fmaxf(mx, __shfl_xor_sync(kAll, mx, o));
+            }
+            if (a.norm_kind == QSGD_NORM_MAX) {
+                norm = __any_sync(kAll, nan) ? __uint_as_float(0x7FC00000u) : mx;
+            } else {
+                norm = __fsqrt_rn(ss);
+                if (needs_rescale(ss) && !isnan(ss)) {  // uniform in the warp
+                    if (isinf(mx)) {
+                        norm = mx;
+                    } else if (mx > 0.f) {  // squares outside the normal range: scaled by a power of two
+                        float unscale;
+                        const float scale = pow2_scale(mx, unscale);
+                        float s2 = 0.f;
+                        for (uint32_t lo = 0; lo < m; lo += kChunkCoords) {
+                            load_contig<V>(a.in + base, lo + ql, m, x);
+                            if constexpr (kEF) {
+                                load_contig<V>(a.ef + base, lo + ql, m, ev);
+#pragma unroll
+                                for (int q = 0; q < NC; ++q) x[q] = __fadd_rn(ev[q], x[q]);
+                            }
+#pragma unroll
+                            for (int q = 0; q < NC; ++q) {
+                                const float y = __fmul_rn(x[q], scale);
+                                s2 = __fmaf_rn(y, y, s2);
+                            }
+                        }
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1) s2 = __fadd_rn(s2, __shfl_xor_sync(kAll, s2, o));
+                        norm = __fmul_rn(__fsqrt_rn(s2), unscale);
                     }
                 }
-                nbits += gl;
             }
-        }
-        // --- the lane's first bit in the bucket: scan of the bit counts ---------------
-        uint32_t incl = nbits;
+            const BucketScale sc = bucket_scale(norm, a.s, true, a.status, lane == 0);
+            // --- then chunk by chunk: levels and records ------------------------------------
+            for (uint32_t lo = 0; lo < m; lo += kChunkCoords) {
+                load_contig<V>(a.in + base, lo + ql, m, x);
+                if constexpr (kEF) {
+                    load_contig<V>(a.ef + base, lo + ql, m, ev);
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t t = __shfl_up_sync(kAll, incl, o);
-            if (lane >= o) incl += t;
-        }
-        const uint32_t P = 32u + incl - nbits;
-        const uint32_t total = 32u + __shfl_sync(kAll, incl, 31);
-        if (lane == 0) buf[0] = __float_as_uint(sc.sent);
-        if (!__any_sync(kAll, nbits > 96u)) {
-            if (nbits != 0u) {
-                // left-align the string in 96 bits, then OR it in at bit P
-                const uint32_t sa = 96u - nbits, bsh = sa & 31u, wsh = sa >> 5;
-                const uint32_t t2 = __funnelshift_l(w1, w2, bsh), t1 = __funnelshift_l(w0, w1, bsh), t0 = w0 << bsh;
-                const uint32_t L0 = wsh == 0 ? t2 : wsh == 1 ? t1 : t0;
-                const uint32_t L1 = wsh == 0 ? t1 : wsh == 1 ? t0 : 0u;
-                const uint32_t L2 = wsh == 0 ? t0 : 0u;
-                const uint32_t wp = P >> 5, sh = P & 31u;
-                const uint32_t nw = (sh + nbits + 31u) >> 5;  // 1..4
-                atomicOr(&buf[wp], L0 >> sh);
-                if (nw > 1) atomicOr(&buf[wp + 1], __funnelshift_r(L1, L0, sh));
-                if (nw > 2) atomicOr(&buf[wp + 2], __funnelshift_r(L2, L1, sh));
-                if (nw > 3) atomicOr(&buf[wp + 3], __funnelshift_r(0u, L2, sh));
-            }
-        } else {  // some lane's string is longer than 96 bits: record by record
-            int32_t prev = prev_in;
-            uint32_t p = P;
-#pragma unroll
-            for (int c = 0; c < NC; ++c) {
-                const uint32_t kv = kq[c];
-                if ((kv & 0x7FFFFFFFu) != 0u) {
-                    uint32_t code, len;
-                    short_record(rtab, otab, static_cast<uint32_t>(static_cast<int32_t>(q0 + c) - prev), kv, code, len);
-                    prev = static_cast<int32_t>(q0 + c);
-                    put_bits(buf, p, code, len);
-                    p += len;
+                    for (int q = 0; q < NC; ++q) x[q] = __fadd_rn(ev[q], x[q]);
                 }
+                if (!sc.good) {  // sent as a zero bucket; the memory keeps p
+                    if constexpr (kEF) store_contig<V>(a.ef + base, lo + ql, m, x);
+#pragma unroll
+                    for (int q = 0; q < NC; ++q) x[q] = 0.f;
+                }
+                code_chunk<V, kEF>(a, rtab, otab, buf, x, ev, sc, base, lo, m, lane, carry, pos);
             }
+            if (lane == 0) buf[0] = __float_as_uint(sc.sent);
         }
         __syncwarp();
-        // --- the bucket's bits into its staging slot; the buffer cleared again -------
+        // --- the bucket's bits into its staging slot; the buffer cleared again -----------
+        const uint32_t total = pos;
         uint32_t* const slot = a.stage + b * a.slot_words;
         const uint32_t nw = (total + 31u) >> 5;
         for (uint32_t i = lane; i < nw; i += 32) {

@@ -110,8 +110,9 @@ struct StageLayout {
 };
 StageLayout stage_layout(uint64_t n, uint32_t d, uint32_t s);
 
-// Float4s per lane of the bucket coder (a power of two >= d/128).
-inline uint32_t stage_v(uint32_t d) { return fast_v(d); }
+// Float4s per lane of the bucket coder (a power of two >= d/128; 4 for buckets of
+// several 512-coordinate chunks).
+inline uint32_t stage_v(uint32_t d) { return d <= 1024 ? fast_v(d) : 4; }
 // Dynamic shared memory of the bucket coder: omega table | record table (s <= 31) |
 // one bucket buffer per warp.
 inline size_t stage_smem_bytes(uint32_t s, uint32_t buf_words) {
@@ -119,7 +120,9 @@ inline size_t stage_smem_bytes(uint32_t s, uint32_t buf_words) {
             static_cast<size_t>(kStageWarps) * buf_words) *
            sizeof(uint32_t);
 }
-inline bool stage_shape(uint32_t d) { return d >= kStageMinD && d <= kStageMaxD && d % 4 == 0; }
+// Whether the two-launch encoder takes (d, s) (alignment aside): the shapes above,
+// with one bucket buffer per warp within the shared memory.
+bool stage_shape(uint32_t d, uint32_t s);
 cudaError_t launch_encode_stage(const StageArgs& a, cudaStream_t stream);
 
 // The encode entry behind qsgd_encode_ex and qsgd_encode_ef (d_ef null or the

@@ -44,8 +44,9 @@ constexpr int kFastBlock = 32 * kFastWarps;
 __host__ __device__ constexpr int enc_depth(unsigned v) { return v <= 4 ? QSGD_ENC_DEPTH : 1; }
 constexpr int kFastMinBlocks = QSGD_FAST_MIN_BLOCKS;
 
-// Two-launch encoder (bucket coder + compaction): 4 <= d <= 1024, d % 4 == 0,
-// 16-byte aligned input; one warp per bucket, kStageWarps warps per CTA; the
+// Two-launch encoder (bucket coder + compaction): d % 4 == 0, 4 <= d <= 1024 (or
+// 16384 for s <= 31), 16-byte aligned input; one warp per bucket, kStageWarps warps
+// per CTA; the
 // compaction takes kCompactBlock buckets per CTA.  Whole-record table for s <= 31.
 constexpr int kStageWarps = 8;
 constexpr int kStageBlock = 32 * kStageWarps;
@@ -54,7 +55,8 @@ constexpr int kStageBlock = 32 * kStageWarps;
 #endif
 constexpr int kCompactBlock = QSGD_COMPACT_BLOCK;
 constexpr uint32_t kStageMinD = 4;
-constexpr uint32_t kStageMaxD = 1024;
+constexpr uint32_t kStageMaxD = 1024;        // s > 31: one chunk of 128V coordinates per bucket
+constexpr uint32_t kStageShortMaxD = 16384;  // s <= 31: buckets of several 512-coordinate chunks
 constexpr uint32_t kStageShortMaxS = 31;
 
 // One-stream decoder with byte codes staged in whole bucket rows: d % 4 == 0,

@@ -96,6 +96,10 @@ CASES = [
     (5_000, 384, 3000, 1, "normal"),
     (6_000, 1000, 31, 2, "layered"),
     (1, 512, 16, 1, "normal"),
+    # buckets of several 512-coordinate chunks (s <= 31): whole, ragged and partial chunks
+    (60_001, 8192, 1, 2, "heavy_tailed_sparse"),
+    (40_003, 3000, 16, 2, "layered"),
+    (50_000, 16384, 4, 2, "normal"),
 ]
 
 
@@ -112,7 +116,7 @@ def test_stage_encoder_matches_oracle(stage_exe, tmp_path, oracle_lib, n, d, s, 
     assert np.array_equal(words, r_words)
 
 
-@pytest.mark.parametrize("d,s", [(512, 16), (128, 3), (256, 100)])
+@pytest.mark.parametrize("d,s", [(512, 16), (128, 3), (256, 100), (4096, 8)])
 def test_stage_encoder_max_norm_matches_oracle(stage_exe, tmp_path, oracle_lib, d, s):
     v = W.layered(20_000, 4)
     words, offsets, status, _ = _run(stage_exe, tmp_path, v, d, s, 8, 2, norm_kind=1)
@@ -120,7 +124,7 @@ def test_stage_encoder_max_norm_matches_oracle(stage_exe, tmp_path, oracle_lib, 
     assert status == rst and np.array_equal(offsets, r_offsets) and np.array_equal(words, r_words)
 
 
-@pytest.mark.parametrize("d,s", [(512, 16), (256, 40), (100, 5)])
+@pytest.mark.parametrize("d,s", [(512, 16), (256, 40), (100, 5), (2048, 3)])
 def test_stage_error_feedback_matches_oracle(stage_exe, tmp_path, oracle_lib, d, s):
     g = W.layered(30_001, 6)
     e = W.normal(30_001, 7) * np.float32(0.05)
@@ -143,7 +147,7 @@ def test_stage_special_values(stage_exe, tmp_path, oracle_lib):
     v[1600:2048] = 1e-30
     v[2048:2560] = 3e38
     v[3000:3512] = -0.0
-    for d in (512, 500):
+    for d in (512, 500, 4096):
         words, offsets, status, _ = _run(stage_exe, tmp_path, v, d, 16, 1, 2)
         _, _, own_norms, own_status = oracle_lib.encode(v, d, 16, 1)
         assert status == own_status
