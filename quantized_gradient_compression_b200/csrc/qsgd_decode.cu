@@ -844,6 +844,8 @@ cudaError_t launch_decode(const DecodeArgs& a, bool accumulate, cudaStream_t str
         if (a.K == 1) return launch_decode_rows(a, accumulate, stream);
     }
     if (a.start_zero || a.div != 0.f) return fast ? launch_multi(a, stream) : cudaErrorInvalidValue;
+    // buckets larger than the rows: a fill of the output, then the records
+    if (decode_sparse_shape(a.d, a.out)) return launch_decode_sparse(a, accumulate, stream);
     if (!fast) return accumulate ? launch<true>(a, stream) : launch<false>(a, stream);
 #ifndef QSGD_MULTI
 #define QSGD_MULTI 1

@@ -632,6 +632,110 @@ __global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows_multi(const __
     }
 }
 
+// ---------------------------------------------------------------------------
+// Large buckets (d > 1024): a CTA takes 32 buckets.  All its threads first write the
+// buckets' output range with 16-byte stores where it is aligned: zeros (decode), or
+// the output + 0 (decode-accumulate; +0 turns -0.0 into +0.0 as the add of a zero
+// term does).  After a CTA barrier, lane L of warp 0 parses bucket 32g + L of every
+// stream in order and stores each record's value (decode) or adds it (accumulate)
+// at its coordinate.  The outputs of such gradients are mostly zeros, so the fill
+// carries the traffic; the records are few.
+// ---------------------------------------------------------------------------
+template <bool kAcc>
+__global__ void __launch_bounds__(kSparseBlock) decode_sparse(const __grid_constant__ DecodeArgs a) {
+    __shared__ uint32_t lut[kLutSize];
+    const int tid = threadIdx.x, lane = tid & 31;
+    build_rows_lut(lut, min(a.s, 127u), tid, kSparseBlock);
+    __syncthreads();
+    const float fs = __uint2float_rn(a.s);
+    const uint64_t d = a.d;
+    const uint64_t ngroups = (a.nb + 31) / 32;
+    for (uint64_t g = blockIdx.x; g < ngroups; g += gridDim.x) {
+        // --- the fill: [g*32*d, min(n, (g+1)*32*d)) ----------------------------------
+        const uint64_t c0 = g * 32 * d, c1 = min(a.n, (g + 1) * 32 * d);
+        float* const out = a.out;
+        const uint64_t head = min(c1, (c0 + 3) & ~uint64_t(3));  // aligned start of the body (out is 16-byte aligned)
+        const uint64_t tail = max(head, c1 & ~uint64_t(3));
+        for (uint64_t i = c0 + tid; i < head; i += kSparseBlock) out[i] = kAcc ? __fadd_rn(out[i], 0.0f) : 0.0f;
+        for (uint64_t i = tail + tid; i < c1; i += kSparseBlock) out[i] = kAcc ? __fadd_rn(out[i], 0.0f) : 0.0f;
+        for (uint64_t i = head + 4 * static_cast<uint64_t>(tid); i < tail; i += 4 * kSparseBlock) {
+            float4* p4 = reinterpret_cast<float4*>(out + i);
+            if constexpr (kAcc) {
+                float4 v = *p4;
+                v.x = __fadd_rn(v.x, 0.0f);
+                v.y = __fadd_rn(v.y, 0.0f);
+                v.z = __fadd_rn(v.z, 0.0f);
+                v.w = __fadd_rn(v.w, 0.0f);
+                *p4 = v;
+            } else {
+                __stcs(p4, make_float4(0.f, 0.f, 0.f, 0.f));
+            }
+        }
+        __syncthreads();
+        // --- the records: lane L of warp 0 takes bucket 32g + L of every stream -------
+        if (tid < 32) {
+            const uint64_t b = g * 32 + lane;
+            const bool live = b < a.nb;
+            const uint32_t m = live ? static_cast<uint32_t>(min(d, a.n - b * d)) : 0u;
+            float* const row = out + b * d;
+            bool bad = false;
+            for (int j = 0; j < a.K && live; ++j) {
+                const StreamRef st = a.streams[j];
+                const uint64_t begin = st.offsets[b];
+                const uint64_t end = st.offsets[b + 1];
+                if (!(end >= begin && end - begin >= 32 && end <= st.num_words * 32 && end - begin < (1ull << 31))) {
+                    bad = true;
+                    continue;
+                }
+                RowReader r;
+                r.init(st.words, st.num_words, begin, static_cast<uint32_t>(end - begin));
+                const uint32_t nbits = r.peek();
+                r.advance(32);
+                const float norm = __uint_as_float(nbits);
+                float scale = 0.f;
+                if (nbits == 0) {
+                    bad = bad || r.left != 0;
+                    continue;
+                } else if (!(isfinite(norm) && norm > 0.f)) {
+                    bad = true;
+                    continue;
+                }
+                scale = __fdiv_rn(norm, fs);
+                if (!(scale > 0.f) && r.left != 0) {  // a zero scale carries no records
+                    bad = true;
+                    continue;
+                }
+                uint32_t next = 0;
+                for (uint32_t it = 0; r.left > 0; ++it) {
+                    uint32_t gap, sign, k;
+                    const uint32_t e = lut[r.peek() >> (32 - kLutBits)];
+                    const uint32_t len1 = e & 15u;
+                    if (len1 != 0u && it < kParseGuard) {  // the first record of the window
+                        gap = (e >> 8) & 15u;
+                        sign = (e >> 23) & 1u;
+                        k = (e >> 16) & 0x7Fu;
+                        r.advance(len1);
+                    } else if (it >= kParseGuard || !slow_record(r, a.s, gap, sign, k)) {
+                        bad = true;
+                        break;
+                    }
+                    next += gap;
+                    if (next > m) {
+                        bad = true;
+                        break;
+                    }
+                    const float q = __fmul_rn(scale, __uint2float_rn(k));
+                    const float v = sign ? -q : q;
+                    row[next - 1] = kAcc ? __fadd_rn(row[next - 1], v) : v;
+                }
+                if (r.left != 0) bad = true;
+            }
+            if (bad) atomicOr(a.status, QSGD_ST_BAD_STREAM);
+        }
+        __syncthreads();
+    }
+}
+
 // Words of one staging row: room for d codes and a padding code, rounded so that
 // consecutive rows start on different banks: stride = 1 mod 32 for byte codes;
 // for 16-bit codes even (the write-back reads 8 bytes a lane) and 2 mod 32.
@@ -698,7 +802,28 @@ cudaError_t launch_rows_t(const DecodeArgs& a, bool accumulate, cudaStream_t str
     }
 }
 
+cudaError_t launch_sparse(const DecodeArgs& a, bool accumulate, cudaStream_t stream) {
+    int dev = 0, sms = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const uint64_t groups = (a.nb + 31) / 32;
+    const uint64_t blocks = std::max<uint64_t>(1, std::min<uint64_t>(groups, static_cast<uint64_t>(sms) * 8));
+    if (accumulate)
+        decode_sparse<true><<<static_cast<unsigned>(blocks), kSparseBlock, 0, stream>>>(a);
+    else
+        decode_sparse<false><<<static_cast<unsigned>(blocks), kSparseBlock, 0, stream>>>(a);
+    return cudaGetLastError();
+}
+
 }  // namespace
+
+bool decode_sparse_shape(uint32_t d, const float* out) {
+    return d > kRowsMaxD && (reinterpret_cast<uintptr_t>(out) & 15u) == 0;
+}
+
+cudaError_t launch_decode_sparse(const DecodeArgs& a, bool accumulate, cudaStream_t stream) {
+    return launch_sparse(a, accumulate, stream);
+}
 
 bool decode_rows_shape(uint32_t d, uint32_t s, const float* out) {
     return d % 4 == 0 && d >= 4 && d <= kRowsMaxD && s <= kRowsMaxS && (reinterpret_cast<uintptr_t>(out) & 15u) == 0;

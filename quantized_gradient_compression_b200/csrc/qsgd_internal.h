@@ -160,6 +160,10 @@ bool decode_rows_shape(uint32_t d, uint32_t s, const float* out);
 cudaError_t launch_decode_rows(const DecodeArgs& a, bool accumulate, cudaStream_t stream);
 // Several streams (decode-accumulate and the mean) on the same shapes (qsgd_decode_rows.cu).
 cudaError_t launch_decode_rows_multi(const DecodeArgs& a, cudaStream_t stream);
+// Buckets larger than the row decoders take (qsgd_decode_rows.cu): decode and
+// decode-accumulate (K <= 16 streams to a launch, in order).
+bool decode_sparse_shape(uint32_t d, const float* out);
+cudaError_t launch_decode_sparse(const DecodeArgs& a, bool accumulate, cudaStream_t stream);
 // Whether the one-lane-per-bucket decoders (and the several-stream kernel, which
 // start_zero / div need) take this shape.
 bool decode_fast_shape(uint32_t d, uint32_t s, const float* out);

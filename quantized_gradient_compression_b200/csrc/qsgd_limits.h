@@ -68,6 +68,10 @@ constexpr uint32_t kRowsMaxD = 1024;
 constexpr uint32_t kRowsMaxS8 = 127;     // byte codes up to here, 16-bit codes above
 constexpr uint32_t kRowsMaxS = 32767;
 
+// Large-bucket decoder (d > kRowsMaxD, 16-byte aligned output): a CTA fills the
+// output of 32 buckets, then one lane per bucket stores the records.
+constexpr int kSparseBlock = 256;
+
 constexpr int kDecodeBlock = 128;
 constexpr int kMaxStreamsPerLaunch = 16;  // decode-accumulate streams per launch
 

@@ -110,6 +110,32 @@ int main(int argc, char** argv) {
     std::vector<float> out(n + 4);
     std::memcpy(out.data(), xb.data(), 4 * n);
     uint32_t status = 0;
+    if (d > qsgd::kRowsMaxD) {  // the large-bucket decoder, 16 streams to a launch
+        std::vector<std::vector<unsigned char>> ws(K), os(K);
+        for (int j = 0; j < K; ++j) {
+            ws[j] = slurp(dir + "/w" + std::to_string(j) + ".bin");
+            os[j] = slurp(dir + "/o" + std::to_string(j) + ".bin");
+        }
+        for (int j0 = 0; j0 < K; j0 += qsgd::kMaxStreamsPerLaunch) {
+            qsgd::DecodeArgs a{};
+            a.n = n; a.d = d; a.s = s; a.nb = nb; a.out = out.data(); a.status = &status;
+            a.K = std::min(K - j0, qsgd::kMaxStreamsPerLaunch);
+            a.first_group = j0 == 0;
+            for (int j = 0; j < a.K; ++j) {
+                a.streams[j].words = reinterpret_cast<const uint32_t*>(ws[j0 + j].data());
+                a.streams[j].num_words = ws[j0 + j].size() / 4;
+                a.streams[j].offsets = reinterpret_cast<const uint64_t*>(os[j0 + j].data());
+            }
+            if (acc)
+                run_grid(grid, qsgd::kSparseBlock, 0, [&] { qsgd::decode_sparse<true>(a); });
+            else
+                run_grid(grid, qsgd::kSparseBlock, 0, [&] { qsgd::decode_sparse<false>(a); });
+            if (g_emu_error) return 4;
+        }
+        spit(dir + "/out.bin", out.data(), 4 * n);
+        std::printf("status %u\n", status);
+        return 0;
+    }
     if (K > 1 || mean) {
         std::vector<std::vector<unsigned char>> ws(K), os(K);
         for (int j = 0; j < K; ++j) {

@@ -204,3 +204,41 @@ def test_row_multi_decoder_corrupt_stream(rows_exe, tmp_path, oracle_lib):
             keep[b * d:min(n, (b + 1) * d)] = False
     assert keep.any() and not keep.all()
     assert np.array_equal(got[keep].view(np.uint32), ref[keep].view(np.uint32))
+
+
+# decode_sparse: buckets larger than the rows (d > 1024), decode and decode-accumulate
+# of several streams in order; ragged last bucket, d not a multiple of four, long gaps
+# (bit-serial records), s above the table's levels
+SPARSE = [
+    (60_001, 8192, 1, 1, False, "heavy_tailed_sparse"),
+    (40_003, 3001, 16, 1, False, "layered"),
+    (30_000, 2048, 300, 3, True, "normal"),
+    (20_000, 4096, 4, 17, True, "small_normal"),
+]
+
+
+@pytest.mark.parametrize("n,d,s,K,acc,kind", SPARSE, ids=["n%d-d%d-s%d-K%d-acc%d-%s" % c for c in SPARSE])
+def test_large_bucket_decoder_matches_oracle(rows_exe, tmp_path, oracle_lib, n, d, s, K, acc, kind):
+    streams = []
+    for j in range(K):
+        w, o, _, st = oracle_lib.encode(W.GENERATORS[kind](n, 90 + j), d, s, seed=j)
+        assert st == 0
+        streams.append((w, o))
+    for j, (w, o) in enumerate(streams):
+        np.concatenate([w, np.zeros(1, np.uint32)]).tofile(tmp_path / ("w%d.bin" % j))
+        o.astype(np.uint64).tofile(tmp_path / ("o%d.bin" % j))
+    base = _base(n, d, acc)
+    base.tofile(tmp_path / "out_in.bin")
+    np.array([n, d, s], np.uint64).tofile(tmp_path / "params.bin")
+    r = subprocess.run([rows_exe, str(tmp_path), "1" if acc else "0", "2", "1", str(K), "0"],
+                       capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, (r.stdout[-500:], r.stderr[-2000:])
+    got, status = np.fromfile(tmp_path / "out.bin", np.float32), int(r.stdout.split()[-1])
+    assert status == 0
+    if acc:
+        ref = base.copy()
+        _, rst = oracle_lib.decode_accumulate(streams, n, d, s, ref)
+    else:
+        ref, rst = oracle_lib.decode(streams[0][0], streams[0][1], n, d, s)
+    assert rst == 0
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
