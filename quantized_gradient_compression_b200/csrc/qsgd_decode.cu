@@ -837,11 +837,13 @@ bool decode_fast_shape(uint32_t d, uint32_t s, const float* out) {
 cudaError_t launch_decode(const DecodeArgs& a, bool accumulate, cudaStream_t stream) {
     if (a.nb == 0) return cudaSuccess;
     const bool fast = decode_fast_shape(a.d, a.s, a.out);
-    // the row decoders when the shape allows: one stream staged as codes, several
-    // streams (and the mean) added onto fp32 tiles in stream order
+    // the row decoders when the shape allows: one stream staged as codes; several
+    // streams (and the mean) added onto fp32 tiles in stream order where the
+    // several-stream kernel below, which decodes the streams side by side, does not
+    // take the levels (s >= 1024)
     if (decode_rows_shape(a.d, a.s, a.out)) {
-        if (a.start_zero || a.div != 0.f || (accumulate && a.K >= 2)) return launch_decode_rows_multi(a, stream);
-        if (a.K == 1) return launch_decode_rows(a, accumulate, stream);
+        if (a.K == 1 && !a.start_zero && a.div == 0.f) return launch_decode_rows(a, accumulate, stream);
+        if (!fast) return launch_decode_rows_multi(a, stream);
     }
     if (a.start_zero || a.div != 0.f) return fast ? launch_multi(a, stream) : cudaErrorInvalidValue;
     // buckets larger than the rows: a fill of the output, then the records

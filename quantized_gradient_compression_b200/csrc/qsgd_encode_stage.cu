@@ -844,8 +844,9 @@ __global__ void __launch_bounds__(kCompactBlock) compact_stream(const __grid_con
     release_control(a.ctrl);
 }
 
-template <class Kernel>
-cudaError_t launch_coder(Kernel kernel, const StageArgs& a, cudaStream_t stream) {
+// One instance per kernel, so that each kernel gets its own shared-memory attribute.
+template <auto kernel>
+cudaError_t launch_coder(const StageArgs& a, cudaStream_t stream) {
     const size_t smem = stage_smem_bytes(a.s, a.buf_words);
     static bool attr_set[64] = {};
     int dev = 0;
@@ -868,9 +869,9 @@ cudaError_t launch_coder(Kernel kernel, const StageArgs& a, cudaStream_t stream)
 template <int V, bool kShort, bool kEF>
 cudaError_t launch_code(const StageArgs& a, cudaStream_t stream) {
     if constexpr (kShort)
-        return launch_coder(code_buckets_short<V, kEF>, a, stream);
+        return launch_coder<code_buckets_short<V, kEF>>(a, stream);
     else
-        return launch_coder(code_buckets<V, false, kEF>, a, stream);
+        return launch_coder<code_buckets<V, false, kEF>>(a, stream);
 }
 
 template <int V>

@@ -22,8 +22,9 @@ def _base(n, seed):
     return b
 
 
-# (n, d, s, K): split decoder with P = 2 / 4 / 8, the one-lane fast decoder (d < 128),
-# the general decoder (odd d, d > 4096), and K beyond one launch's 16 streams
+# (n, d, s, K): the one-stream row decoder (K = 1), the several-stream row decoder
+# (d <= 1024, d a multiple of 4), the large-bucket decoder (d > 1024), the one-lane
+# decoders (d < 4 or d not a multiple of 4), and K beyond one launch's 16 streams
 CASES = [
     (40_000, 132, 3, 3),
     (100_003, 512, 16, 1),
@@ -69,8 +70,8 @@ def test_accumulate_matches_oracle(oracle_lib, n, d, s, K):
 
 @pytest.mark.parametrize("d", [512, 2048, 132])
 def test_decode_of_oracle_streams(oracle_lib, d):
-    """Plain decode of oracle-made streams (layered data, so many buckets are too
-    sparse to split and some need the bit-serial path)."""
+    """Plain decode of oracle-made streams (layered data: many buckets are nearly
+    empty and some records need the bit-serial path)."""
     import torch
     from quantized_gradient_compression_b200 import binding as B
 

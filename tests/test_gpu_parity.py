@@ -13,7 +13,11 @@ def vec(kind, n, seed):
     return W.GENERATORS[kind](n, seed)
 
 
-# (kind, n, d, s): several tiles and a ragged tail on both encoder paths
+# (kind, n, d, s): several tiles and a ragged tail on every encoder and decoder path:
+# the staged short coder (s <= 31, d <= 16384, one or several 512-coordinate chunks),
+# the staged lane-strided coder (s > 31, d <= 1024), the one-pass coder (other shapes),
+# the row decoder with byte codes (s <= 127) and 16-bit codes, the large-bucket
+# decoder (d > 1024) and the one-lane decoders (d not a multiple of 4)
 CASES = [
     ("layered", 2_000_001, 512, 16),       # fast path, ragged last bucket (129)
     ("layered", 1_000_000, 512, 16),
@@ -37,8 +41,7 @@ CASES = [
     ("normal", 513, 512, 16),
     ("normal", 20_000, 512, 1 << 22),      # largest s
     ("normal", 20_000, 100, 7),            # d < 128: general
-    # decoder with P lanes per bucket: P = 2 (d < 256, d not a multiple of 64),
-    # P = 8 (d >= 1024), and sparse buckets too short to split (decoded whole)
+    # d not a multiple of 64, a large bucket with s > 31, sparse buckets
     ("normal", 100_000, 132, 3),
     ("normal", 200_000, 2048, 64),
     ("heavy_tailed_sparse", 300_000, 512, 2),

@@ -37,7 +37,7 @@ def _build(tmp_path_factory, name, extra=()):
         shutil.copy(os.path.join(CSRC, h), src_dir / h)
     (src_dir / "qsgd_device.cuh").write_text(_host_source(open(os.path.join(CSRC, "qsgd_device.cuh")).read()))
     enc = open(os.path.join(CSRC, "qsgd_encode_stage.cu")).read()
-    cut = enc.index("template <class Kernel>\ncudaError_t launch_coder")
+    cut = enc.index("// One instance per kernel, so that each kernel gets its own shared-memory attribute.")
     (src_dir / "stage_emu.inc").write_text(_host_source(enc[:cut]) + "}  // namespace\n}  // namespace qsgd\n")
     exe = d / "stage_main"
     r = subprocess.run(["g++", "-O1", "-std=c++17", "-ffp-contract=off", "-pthread", *extra, "-I", EMU, "-I",
