@@ -10,9 +10,11 @@
 //
 // Work layout: each lane of a warp parses one bucket (buckets are independent
 // prefix-code streams located by the offsets header), 32 consecutive buckets to a
-// warp.  Records are decoded through a shared-memory table of the whole records at
-// the start of a 12-bit window (up to two per entry), two lookups a step; longer
-// records take a bit-serial path.  The lane stores the
+// warp.  With byte codes, records are decoded through a shared-memory table of the
+// whole records at the start of a 12-bit window (up to two per entry), two lookups
+// a step; with 16-bit codes (large s, where nearly every coordinate has a record),
+// through a table of omega codes, one lookup for the gap and one for the level.
+// Longer records take a bit-serial path.  The lane stores the
 // record's code (sign << 7 | k in a byte for s <= 127, sign << 15 | k in 16 bits for
 // s <= 32767) at its index in its bucket's row of a zeroed staging area: 32 rows of d
 // codes, padded so that the rows start on different banks.  No lane waits for another while parsing.  Then the warp converts
@@ -35,8 +37,11 @@ constexpr int kLutBits = 12;
 constexpr int kLutSize = 1 << kLutBits;
 constexpr uint32_t kParseGuard = 1u << 20;  // a second, explicit bound of the parse loop
 
+// Decoding tables, computed at compile time and copied into shared memory by every
+// CTA.  Both read windows MSB-first; a window is the next 12 bits of the stream.
+
 // One omega code from the top of an n-bit window w, starting at bit pos (MSB = 0).
-__device__ __forceinline__ bool window_omega(uint32_t w, int nbits, int& pos, uint32_t& value) {
+constexpr bool window_omega(uint32_t w, int nbits, int& pos, uint32_t& value) {
     uint32_t v = 1;
     for (;;) {
         if (pos >= nbits) return false;
@@ -53,31 +58,37 @@ __device__ __forceinline__ bool window_omega(uint32_t w, int nbits, int& pos, ui
     }
 }
 
-// One whole record (omega(gap) | sign | omega(k)) at bit pos of a 12-bit window with
-// gap <= 15 and 1 <= k <= min(s, 127): its gap, code sign << 7 | k and the bit after it.
-__device__ __forceinline__ bool window_record(uint32_t w, int& pos, uint32_t s, uint32_t& gap, uint32_t& code) {
+// One whole record (omega(gap) | sign | omega(k)) at bit pos of a 12-bit window: its
+// gap, code sign << 7 | k and the bit after it.  Within 12 bits, gap <= 15 and k <= 15.
+constexpr bool window_record(uint32_t w, int& pos, uint32_t& gap, uint32_t& code) {
     uint32_t k = 0;
     if (!window_omega(w, kLutBits, pos, gap) || pos >= kLutBits) return false;
     const uint32_t sign = (w >> (kLutBits - 1 - pos)) & 1u;
     ++pos;
-    if (!window_omega(w, kLutBits, pos, k) || k > s || k > 127u || gap > 15u) return false;
+    if (!window_omega(w, kLutBits, pos, k)) return false;
     code = (sign << 7) | k;
     return true;
 }
 
-// Table of the whole records at the start of a 12-bit window, up to two: [3:0] length
-// of the first (0: none, take the bit-serial path), [7:4] length of both (the first's
-// when there is no second), [11:8] first gap, [15:12] second gap, [23:16] first code,
-// [31:24] second code (0: none; a code is never 0, since k >= 1).
-__device__ void build_rows_lut(uint32_t* lut, uint32_t s, int tid, int nthreads) {
-    for (int w = tid; w < kLutSize; w += nthreads) {
+// The whole records at the start of a 12-bit window, up to two: [3:0] length of the
+// first (0: none, take the bit-serial path), [7:4] length of both (the first's when
+// there is no second), [11:8] first gap, [15:12] second gap, [23:16] first code,
+// [31:24] second code (0: none; a code is never 0, since k >= 1).  For s >= 15 the
+// table is the same for every s; a smaller s drops the records with k > s when the
+// table is copied (rows_lut_fill).
+struct alignas(16) RowsLut {  // read with 16-byte loads
+    uint32_t v[kLutSize];
+};
+constexpr RowsLut make_rows_lut() {
+    RowsLut t{};
+    for (uint32_t w = 0; w < static_cast<uint32_t>(kLutSize); ++w) {
         int pos = 0;
         uint32_t g1 = 0, c1 = 0, e = 0;
-        if (window_record(static_cast<uint32_t>(w), pos, s, g1, c1)) {
+        if (window_record(w, pos, g1, c1)) {
             const int len1 = pos;
             uint32_t g2 = 0, c2 = 0;
             int len2 = len1;
-            if (!window_record(static_cast<uint32_t>(w), len2, s, g2, c2)) {
+            if (!window_record(w, len2, g2, c2)) {
                 g2 = 0;
                 c2 = 0;
                 len2 = len1;
@@ -85,8 +96,49 @@ __device__ void build_rows_lut(uint32_t* lut, uint32_t s, int tid, int nthreads)
             e = static_cast<uint32_t>(len1) | (static_cast<uint32_t>(len2) << 4) | (g1 << 8) | (g2 << 12) |
                 (c1 << 16) | (c2 << 24);
         }
-        lut[w] = e;
+        t.v[w] = e;
     }
+    return t;
+}
+__device__ const RowsLut kRowsLutGlobal = make_rows_lut();
+
+// The omega code at the top of a 12-bit window: [3:0] length (0: longer than 12
+// bits), [9:4] value (<= 63, as every code of at most 12 bits).
+struct alignas(16) OmegaLut {  // read with 16-byte loads
+    uint16_t v[kLutSize];
+};
+constexpr OmegaLut make_omega_lut() {
+    OmegaLut t{};
+    for (uint32_t w = 0; w < static_cast<uint32_t>(kLutSize); ++w) {
+        int pos = 0;
+        uint32_t val = 0;
+        t.v[w] = window_omega(w, kLutBits, pos, val) ? static_cast<uint16_t>(static_cast<uint32_t>(pos) | (val << 4)) : 0;
+    }
+    return t;
+}
+__device__ const OmegaLut kOmegaLutGlobal = make_omega_lut();
+
+// The record table for levels up to s, in shared memory (16-byte loads).
+__device__ __forceinline__ void rows_lut_fill(uint32_t* lut, uint32_t s, int tid, int nthreads) {
+    const uint4* src = reinterpret_cast<const uint4*>(kRowsLutGlobal.v);
+    for (int i = tid; i < kLutSize / 4; i += nthreads) {
+        uint4 q = src[i];
+        if (s < 15u) {
+            uint32_t* e = &q.x;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                if (((e[j] >> 16) & 0x7Fu) > s)
+                    e[j] = 0u;  // the first record's level is beyond s: bit-serial path
+                else if ((e[j] >> 24 & 0x7Fu) > s)
+                    e[j] = (e[j] & 0x00FF0F0Fu) | ((e[j] & 15u) << 4);  // keep the first record only
+            }
+        }
+        reinterpret_cast<uint4*>(lut)[i] = q;
+    }
+}
+__device__ __forceinline__ void omega_lut_fill(uint16_t* olut, int tid, int nthreads) {
+    const uint4* src = reinterpret_cast<const uint4*>(kOmegaLutGlobal.v);
+    for (int i = tid; i < kLutSize / 8; i += nthreads) reinterpret_cast<uint4*>(olut)[i] = src[i];
 }
 
 // MSB-first reader of one bucket over two stream words: the next unread bits are
@@ -191,7 +243,13 @@ __global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows(const __grid_c
     const int W = blockDim.x >> 5;
     uint32_t* const rows = smem + kLutSize + static_cast<uint32_t>(warp) * 32u * stride_w;
     T* const myrow = reinterpret_cast<T*>(rows + static_cast<uint32_t>(lane) * stride_w);
-    build_rows_lut(lut, a.s, tid, blockDim.x);
+    // byte codes (s <= 127): the two-record table; 16-bit codes: the omega table,
+    // looked up for the gap and then for the level
+    const uint16_t* const olut = reinterpret_cast<const uint16_t*>(smem);
+    if constexpr (sizeof(T) == 1)
+        rows_lut_fill(lut, a.s, tid, blockDim.x);
+    else
+        omega_lut_fill(reinterpret_cast<uint16_t*>(smem), tid, blockDim.x);
     __syncthreads();
     const StreamRef st = a.streams[0];
     const float fs = __uint2float_rn(a.s);
@@ -242,7 +300,7 @@ __global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows(const __grid_c
             }
         }
         __syncwarp();
-        // --- parse: every record's code into the lane's row, up to two a lookup ----
+        // --- parse: every record's code into the lane's row -------------------------
         uint32_t next = 0;  // bucket-local index after the last record
         if (bad) r.left = 0;
         for (uint32_t it = 0; __any_sync(kWarpAll, r.left > 0); ++it) {
@@ -250,7 +308,32 @@ __global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows(const __grid_c
                 bad = bad || r.left > 0;
                 break;
             }
-            if (r.left > 0) {
+            if constexpr (sizeof(T) == 2) {
+                // one record a step: omega(gap) (<= 12 bits), the sign, omega(k) (<= 12
+                // bits) from the 32 bits at the cursor; k <= 63 < s, so no level check
+                if (r.left > 0) {
+                    const uint32_t w = r.peek();
+                    const uint32_t ge = olut[w >> (32 - kLutBits)];
+                    const uint32_t gl = ge & 15u;
+                    const uint32_t w2 = w << gl;
+                    const uint32_t ke = olut[(w2 << 1) >> (32 - kLutBits)];
+                    const uint32_t kl = ke & 15u;
+                    if (gl != 0u && kl != 0u) {
+                        next += ge >> 4;
+                        myrow[min(next - 1u, d)] = row_code<T>(w2 >> 31, ke >> 4);
+                        r.advance(gl + 1u + kl);
+                    } else {
+                        uint32_t gap = 0, sign = 0, k = 0;
+                        if (slow_record(r, a.s, gap, sign, k)) {
+                            next += gap;
+                            myrow[min(next - 1u, d)] = row_code<T>(sign, k);
+                        } else {
+                            bad = true;
+                            r.left = 0;
+                        }
+                    }
+                }
+            } else if (r.left > 0) {
                 // up to two table entries a step, each up to two records: the 32 bits at
                 // the cursor hold both 12-bit windows (the first takes at most 12 bits);
                 // a record is taken only when it ends inside the bucket
@@ -375,37 +458,13 @@ __global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows(const __grid_c
 // decode-accumulate, and a stream adds nothing off its support.  The tile is then
 // written back (divided by K in the last launch of a mean).  Between segments each
 // stream's parse state (reader, next index, the record read past the segment, the
-// bucket's scale) waits in shared memory.  Records are read through a table of omega
-// gap codes (12-bit window) and one of sign | omega(k) (8-bit window), so gaps up to
-// 63 and levels up to 15 take two lookups; others take the bit-serial path.
+// bucket's scale) waits in shared memory.  Records are read through the omega table,
+// once for the gap and once for the level, so gaps and levels up to 63 take two
+// lookups; others take the bit-serial path.
 // ---------------------------------------------------------------------------
 constexpr int kMSeg = 64;          // columns per segment
 constexpr int kMTile = kMSeg + 1;  // tile row stride (odd: lanes' rows on different banks)
 constexpr uint32_t kNoPend = 0xFFFFFFFFu;
-
-// omega(gap) at the top of a 12-bit window: [3:0] length (0: not within 12 bits),
-// [9:4] gap (<= 63).
-__device__ void build_gap_lut(uint16_t* glut, int tid, int nthreads) {
-    for (int w = tid; w < kLutSize; w += nthreads) {
-        int pos = 0;
-        uint32_t g = 0;
-        uint32_t e = 0;
-        if (window_omega(static_cast<uint32_t>(w), kLutBits, pos, g) && g <= 63u) e = static_cast<uint32_t>(pos) | (g << 4);
-        glut[w] = static_cast<uint16_t>(e);
-    }
-}
-// sign | omega(k) at the top of an 8-bit window: [3:0] length (0: not within 8 bits,
-// or k > s), [8:4] k (<= 15), [15] sign.
-__device__ void build_level_lut(uint16_t* klut, uint32_t s, int tid, int nthreads) {
-    for (int w = tid; w < 256; w += nthreads) {
-        const uint32_t sign = static_cast<uint32_t>(w) >> 7;
-        int pos = 1;
-        uint32_t k = 0, e = 0;
-        if (window_omega(static_cast<uint32_t>(w), 8, pos, k) && k <= s && k <= 15u)
-            e = static_cast<uint32_t>(pos) | (k << 4) | (sign << 15);
-        klut[w] = static_cast<uint16_t>(e);
-    }
-}
 
 // Parse state of one stream of one bucket, kept in registers while the stream is
 // decoded and in shared memory (one array per field, [stream][lane]) in between.
@@ -478,17 +537,15 @@ __device__ __forceinline__ bool ms_omega(MsReader& r, const StreamRef& st, uint3
 
 __global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows_multi(const __grid_constant__ DecodeArgs a) {
     extern __shared__ __align__(16) uint32_t smem[];
-    uint16_t* const glut = reinterpret_cast<uint16_t*>(smem);
-    uint16_t* const klut = glut + kLutSize;
+    uint16_t* const olut = reinterpret_cast<uint16_t*>(smem);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int W = blockDim.x >> 5;
-    char* const wbase = reinterpret_cast<char*>(smem) + (kLutSize + 256) * sizeof(uint16_t) +
+    char* const wbase = reinterpret_cast<char*>(smem) + kLutSize * sizeof(uint16_t) +
                         static_cast<size_t>(warp) * (sizeof(MsState) + 32 * kMTile * sizeof(float));
     MsState& S = *reinterpret_cast<MsState*>(wbase);
     float* const tile = reinterpret_cast<float*>(wbase + sizeof(MsState));
     float* const myrow = tile + lane * kMTile;
-    build_gap_lut(glut, tid, blockDim.x);
-    build_level_lut(klut, a.s, tid, blockDim.x);
+    omega_lut_fill(olut, tid, blockDim.x);
     __syncthreads();
     const float fs = __uint2float_rn(a.s);
     const uint32_t d = a.d;
@@ -569,15 +626,16 @@ __global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows_multi(const __
                         uint32_t gap = 0, k = 0, sign = 0;
                         bool ok = false;
                         const uint32_t w = ms_peek(r);
-                        const uint32_t ge = glut[w >> (32 - kLutBits)];
+                        const uint32_t ge = olut[w >> (32 - kLutBits)];
                         const uint32_t gl = ge & 15u;
-                        const uint32_t ke = gl ? klut[(w << gl) >> 24] : 0u;
+                        const uint32_t w2 = w << gl;
+                        const uint32_t ke = olut[(w2 << 1) >> (32 - kLutBits)];
                         const uint32_t kl = ke & 15u;
-                        if (kl != 0u) {
-                            gap = (ge >> 4) & 63u;
-                            k = (ke >> 4) & 31u;
-                            sign = ke >> 15;
-                            ms_advance(r, st, gl + kl);
+                        if (gl != 0u && kl != 0u && (ke >> 4) <= a.s) {
+                            gap = ge >> 4;
+                            k = ke >> 4;
+                            sign = w2 >> 31;
+                            ms_advance(r, st, gl + 1u + kl);
                             ok = r.left >= 0;
                         } else if (ms_omega(r, st, gap) && r.left > 0 && gap <= 0xFFFFu) {
                             sign = ms_peek(r) >> 31;
@@ -643,9 +701,9 @@ __global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows_multi(const __
 // ---------------------------------------------------------------------------
 template <bool kAcc>
 __global__ void __launch_bounds__(kSparseBlock) decode_sparse(const __grid_constant__ DecodeArgs a) {
-    __shared__ uint32_t lut[kLutSize];
+    __shared__ __align__(16) uint32_t lut[kLutSize];
     const int tid = threadIdx.x, lane = tid & 31;
-    build_rows_lut(lut, min(a.s, 127u), tid, kSparseBlock);
+    rows_lut_fill(lut, a.s, tid, kSparseBlock);
     __syncthreads();
     const float fs = __uint2float_rn(a.s);
     const uint64_t d = a.d;
@@ -776,7 +834,7 @@ cudaError_t launch_rows_multi(const DecodeArgs& a, cudaStream_t stream) {
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     const size_t per_warp = sizeof(MsState) + 32 * kMTile * sizeof(float);
-    const size_t luts = (kLutSize + 256) * sizeof(uint16_t);
+    const size_t luts = kLutSize * sizeof(uint16_t);
     const int W_fit = static_cast<int>(std::min<size_t>(kRowsMaxWarps, (static_cast<size_t>(optin) - luts - 1024) / per_warp));
     if (W_fit < 1) return cudaErrorInvalidConfiguration;
     const uint64_t groups = (a.nb + 31) / 32;

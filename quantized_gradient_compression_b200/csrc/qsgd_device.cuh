@@ -251,7 +251,7 @@ __device__ __forceinline__ void omega_compute(uint64_t N, uint64_t& code, uint32
 
 // Table of omega codes for N < kOmegaTab: entry = (code << 8) | len (entry 0 is
 // unused).  Built at compile time by the same rule as omega_compute.
-struct OmegaTable {
+struct alignas(16) OmegaTable {  // read with 16-byte loads
     uint32_t v[kOmegaTab];
 };
 constexpr OmegaTable make_omega_table() {
@@ -282,7 +282,7 @@ __device__ __forceinline__ void omega_table_fill(uint32_t* tab, int tid, int nth
 
 // Whole records omega(gap) | sign | omega(k) for gap < 64 and k < 16, indexed by
 // gap << 5 | k << 1 | sign: entry = code << 5 | length (length <= 20 bits).
-struct RecordTable {
+struct alignas(16) RecordTable {  // read with 16-byte loads
     uint32_t v[kRecordTab];
 };
 constexpr RecordTable make_record_table() {

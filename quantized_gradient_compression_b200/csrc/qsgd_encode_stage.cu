@@ -38,7 +38,7 @@ constexpr uint32_t kAll = 0xFFFFFFFFu;
 // Whole records omega(gap) | sign | omega(k) for gap < 64 and k < 32, indexed by
 // gap << 6 | k << 1 | sign: entry = code << 5 | length (length <= 24 bits).  Gap 0
 // holds the record without its gap, sign | omega(k); k = 0 entries are empty.
-struct RecordTable64 {
+struct alignas(16) RecordTable64 {  // read with 16-byte loads
     uint32_t v[kRecordTab64];
 };
 constexpr RecordTable64 make_record_table64() {

@@ -26,6 +26,7 @@ def host_source(text: str) -> str:
         (r'asm volatile\("prefetch\.global\.L2 \[%0\];" ::"l"\([^;]*\);', ";"),
         (r"extern __shared__ __align__\(16\) uint32_t smem\[\];",
          "uint32_t* smem = reinterpret_cast<uint32_t*>(emu_smem());"),
+        (r"__shared__ __align__\(16\) ", "__shared__ "),
         (r"__shared__\s+([\w:<> ]+?)\s+(\w+)\s*(\[[^\]]*\])?\s*;", r"auto& \2 = emu_shared<\1\3>(__LINE__);"),
     ]
     for pat, rep in reps:

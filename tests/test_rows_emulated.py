@@ -111,7 +111,8 @@ def test_row_decoder_matches_oracle(rows_exe, tmp_path, oracle_lib, n, d, s, acc
     assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
 
 
-@pytest.mark.parametrize("d,accumulate,s", [(512, False, 16), (128, True, 16), (1000, False, 16), (512, True, 300)])
+@pytest.mark.parametrize("d,accumulate,s", [(512, False, 16), (128, True, 16), (1000, False, 16), (512, True, 300),
+                                          (256, False, 2)])
 def test_row_decoder_corrupt_streams(rows_exe, tmp_path, oracle_lib, d, accumulate, s):
     n = 30_000
     v = W.normal(n, 5)
