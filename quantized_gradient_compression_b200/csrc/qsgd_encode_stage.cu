@@ -13,13 +13,13 @@
 //    bucket's bits (norm, then the records in index order) into the bucket's own
 //    slot of a staging area in the workspace, at bucket-local bit offsets, together
 //    with the bucket's bit count.  A slot holds the bucket's largest possible size.
-// 2. compact_stream: one CTA per 256 buckets scans the bit counts (a block scan and a
-//    decoupled look-back over the CTAs, Merrill & Garland 2016, read a whole CTA of
-//    predecessors at a time), writes the offsets
-//    header, and moves every bucket's bits to their stream position with funnel
-//    shifts.  An output word belongs to the bucket that holds its first bit; that
-//    bucket's warp also reads the first bits of the next bucket, so every word has
-//    exactly one writer and the output needs no clearing.
+// 2. compact_stream: a CTA of 512 threads per tile of 256 buckets scans the bit
+//    counts (a block scan and a decoupled look-back over the tiles, Merrill &
+//    Garland 2016, reading 512 predecessors at a time), writes the offsets header,
+//    and moves every bucket's bits to their stream position with funnel shifts, one
+//    warp per bucket.  An output word belongs to the bucket that holds its first
+//    bit; that bucket's warp also reads the first bits of the next bucket, so every
+//    word has exactly one writer and the output needs no clearing.
 // The staging costs two extra passes over the compressed bytes (a few percent of
 // the input bytes) and buys an encoder with no inter-CTA waits in its long kernel.
 #include <cuda_runtime.h>
@@ -694,22 +694,23 @@ __device__ __forceinline__ void release_control(ScanControl* ctrl) {
 // ---------------------------------------------------------------------------
 // 2. Compaction: offsets header and the stream at its final bit positions.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kCompactBlock) compact_stream(const __grid_constant__ StageArgs a) {
+__global__ void __launch_bounds__(kCompactThreads, 2) compact_stream(const __grid_constant__ StageArgs a) {
+    constexpr int kWarps = kCompactThreads / 32;
     __shared__ uint32_t s_R[kCompactBlock];
     __shared__ uint32_t s_L[kCompactBlock];
-    __shared__ uint32_t s_warp[kCompactBlock / 32];
+    __shared__ uint32_t s_warp[kWarps];
     __shared__ uint32_t s_tile;
     __shared__ uint64_t s_X;
     __shared__ int s_ok;
     __shared__ uint32_t s_first;
-    __shared__ uint64_t s_part[kCompactBlock / 32];
+    __shared__ uint64_t s_part[kWarps];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) s_tile = atomicAdd(&a.ctrl->ticket, 1u);  // tiles in scheduling order
     __syncthreads();
     const uint64_t tile = s_tile;
     const uint64_t b0 = tile * kCompactBlock;
     const uint64_t b = b0 + tid;
-    const uint32_t L = b < a.nb ? a.bits[b] : 0u;
+    const uint32_t L = tid < kCompactBlock && b < a.nb ? a.bits[b] : 0u;
     // block scan of the bucket sizes (a tile is at most 256 * 2^21 bits... far below 2^32)
     uint32_t incl = L;
 #pragma unroll
@@ -721,7 +722,7 @@ __global__ void __launch_bounds__(kCompactBlock) compact_stream(const __grid_con
     __syncthreads();
     uint32_t before = 0, total = 0;
 #pragma unroll
-    for (int w = 0; w < kCompactBlock / 32; ++w) {
+    for (int w = 0; w < kWarps; ++w) {
         const uint32_t x = s_warp[w];
         before += w < warp ? x : 0u;
         total += x;
@@ -729,7 +730,7 @@ __global__ void __launch_bounds__(kCompactBlock) compact_stream(const __grid_con
     const uint32_t excl = before + incl - L;
     if (tid == 0) st_release(&a.cdesc[tile], make_desc(0, tile == 0 ? kStatePrefix : kStateAggregate, total));
     // look-back by the whole CTA: thread i reads the descriptor of tile (window end -
-    // i), so one read covers kCompactBlock predecessors; the nearest one holding its
+    // i), so one read covers kCompactThreads predecessors; the nearest one holding its
     // inclusive prefix ends the walk, and every tile between must have published its
     // bit count.  Bounded: an abort or kMaxPolls empty reads end it with an error.
     uint64_t Xacc = 0;
@@ -746,7 +747,7 @@ __global__ void __launch_bounds__(kCompactBlock) compact_stream(const __grid_con
                 val = desc_value(dsc);
             }
             // nearest prefix: the smallest thread index holding one
-            if (tid == 0) s_first = kCompactBlock;
+            if (tid == 0) s_first = kCompactThreads;
             __syncthreads();
             if (st == kStatePrefix) atomicMin(&s_first, static_cast<uint32_t>(tid));
             __syncthreads();
@@ -770,10 +771,10 @@ __global__ void __launch_bounds__(kCompactBlock) compact_stream(const __grid_con
             if (lane == 0) s_part[warp] = c;
             __syncthreads();
 #pragma unroll
-            for (int w = 0; w < kCompactBlock / 32; ++w) Xacc += s_part[w];
+            for (int w = 0; w < kWarps; ++w) Xacc += s_part[w];
             __syncthreads();
-            if (first < kCompactBlock) break;
-            wend -= kCompactBlock;
+            if (first < kCompactThreads) break;
+            wend -= kCompactThreads;
         }
         if (tid == 0 && ok) st_release(&a.cdesc[tile], make_desc(0, kStatePrefix, Xacc + total));
     }
@@ -791,52 +792,41 @@ __global__ void __launch_bounds__(kCompactBlock) compact_stream(const __grid_con
         return;
     }
     const uint64_t X = s_X;
-    const uint64_t F = X + excl;
-    s_R[tid] = excl;  // tile-relative start of each bucket
-    s_L[tid] = L;
-    if (b < a.nb) a.offsets[b] = F;
-    if (b + 1 == a.nb) a.offsets[a.nb] = F + L;
+    if (tid < kCompactBlock) {
+        const uint64_t F = X + excl;
+        s_R[tid] = excl;  // tile-relative start of each bucket
+        s_L[tid] = L;
+        if (b < a.nb) a.offsets[b] = F;
+        if (b + 1 == a.nb) a.offsets[a.nb] = F + L;
+    }
     __syncthreads();
-    // Every thread takes output words w = wb + tid + kCompactBlock i of the tile: the
-    // words whose first bit lies in one of its buckets.  A word's bucket comes from a
-    // binary search over the buckets' starts; its bits are that bucket's staged bits
-    // from the word's offset on, and, past the bucket's end, the first bits of the
-    // next bucket (always >= 32 bits, so one word of it suffices).
+    // A warp per bucket, its lanes over the output words whose first bit lies in the
+    // bucket: word k is bits [delta + 32 k, + 32) of the bucket's staged bits, delta
+    // the distance from the bucket's start to the next word boundary; a word that runs
+    // past the bucket's end takes the first bits of the next bucket (always >= 32
+    // bits, so one word of it suffices).  Every output word has exactly one writer.
     const uint32_t nt = static_cast<uint32_t>(min(static_cast<uint64_t>(kCompactBlock), a.nb - b0));
-    const uint64_t wb = (X + 31u) >> 5, we = (X + total + 31u) >> 5;
-    constexpr int kUnroll = 8;
-    for (uint64_t w0 = wb + tid; w0 < we; w0 += kUnroll * kCompactBlock) {
-        uint32_t v[kUnroll];
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const uint64_t w = w0 + static_cast<uint64_t>(u) * kCompactBlock;
-            v[u] = 0u;
-            if (w >= we) continue;
-            const uint32_t g = static_cast<uint32_t>(32u * w - X);  // tile-relative bit of the word
-            uint32_t lo = 0, hi = nt - 1;  // the last bucket with start <= g
-            while (lo < hi) {
-                const uint32_t mid = (lo + hi + 1) >> 1;
-                if (s_R[mid] <= g) lo = mid; else hi = mid - 1;
-            }
-            const uint64_t bb = b0 + lo;
-            const uint32_t Lb = s_L[lo];
-            const uint32_t r = g - s_R[lo];
-            const uint32_t q = r >> 5, sh = r & 31u;
-            const uint32_t* src = a.stage + bb * a.slot_words;
-            const uint32_t a0 = src[q];
-            const uint32_t a1 = q + 1 < ((Lb + 31u) >> 5) ? src[q + 1] : 0u;
-            v[u] = __funnelshift_l(a1, a0, sh);
-            if (r + 32u > Lb) {  // the word runs into the next bucket: its first bits
+    for (uint32_t i = warp; i < nt; i += kWarps) {
+        const uint64_t bb = b0 + i;
+        const uint32_t Lb = s_L[i];
+        const uint64_t F = X + s_R[i];
+        const uint64_t wf = (F + 31u) >> 5;
+        const uint32_t cnt = static_cast<uint32_t>(((F + Lb + 31u) >> 5) - wf);
+        const uint32_t delta = static_cast<uint32_t>((wf << 5) - F);
+        const uint32_t nw = (Lb + 31u) >> 5;
+        const uint32_t* src = a.stage + bb * a.slot_words;
+        for (uint32_t k = lane; k < cnt; k += 32) {
+            const uint32_t r = delta + 32u * k;  // bucket-relative bit of the word (< Lb)
+            const uint32_t a0 = src[k];
+            const uint32_t a1 = k + 1 < nw ? src[k + 1] : 0u;
+            uint32_t v = __funnelshift_l(a1, a0, delta);
+            if (r + 32u > Lb) {  // 1 <= Lb - r <= 31
                 const uint32_t hd = bb + 1 < a.nb ? a.stage[(bb + 1) * a.slot_words] : 0u;
-                v[u] |= hd >> (Lb - r);
+                v |= hd >> (Lb - r);
             }
-        }
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const uint64_t w = w0 + static_cast<uint64_t>(u) * kCompactBlock;
-            if (w >= we) continue;
+            const uint64_t w = wf + k;
             if (w < a.cap_words)
-                a.words[w] = v[u];
+                a.words[w] = v;
             else
                 report(a.status, QSGD_ST_OVERFLOW);
         }
@@ -892,7 +882,7 @@ cudaError_t launch_encode_stage(const StageArgs& a, cudaStream_t stream) {
         default: e = launch_code_v<8>(a, stream); break;
     }
     if (e != cudaSuccess) return e;
-    compact_stream<<<static_cast<unsigned>(a.ntiles), kCompactBlock, 0, stream>>>(a);
+    compact_stream<<<static_cast<unsigned>(a.ntiles), kCompactThreads, 0, stream>>>(a);
     return cudaGetLastError();
 }
 

@@ -46,14 +46,15 @@ constexpr int kFastMinBlocks = QSGD_FAST_MIN_BLOCKS;
 
 // Two-launch encoder (bucket coder + compaction): d % 4 == 0, 4 <= d <= 1024 (or
 // 16384 for s <= 31), 16-byte aligned input; one warp per bucket, kStageWarps warps
-// per CTA; the
-// compaction takes kCompactBlock buckets per CTA.  Whole-record table for s <= 31.
+// per CTA; the compaction takes a tile of kCompactBlock buckets per CTA of
+// kCompactThreads threads.  Whole-record table for s <= 31.
 constexpr int kStageWarps = 8;
 constexpr int kStageBlock = 32 * kStageWarps;
 #ifndef QSGD_COMPACT_BLOCK
 #define QSGD_COMPACT_BLOCK 256
 #endif
 constexpr int kCompactBlock = QSGD_COMPACT_BLOCK;
+constexpr int kCompactThreads = 2 * kCompactBlock;
 constexpr uint32_t kStageMinD = 4;
 constexpr uint32_t kStageMaxD = 1024;        // s > 31: one chunk of 128V coordinates per bucket
 constexpr uint32_t kStageShortMaxD = 16384;  // s <= 31: buckets of several 512-coordinate chunks

@@ -48,23 +48,14 @@ static void run_grid(unsigned grid, unsigned block, size_t smem, Kernel k) {
     for (auto& x : th) x.join();
 }
 
-template <int V, class T>
-static void run(const qsgd::DecodeArgs& a, bool acc, unsigned grid, unsigned W, uint32_t stride, size_t smem) {
-    if (acc)
-        run_grid(grid, 32 * W, smem, [&] { qsgd::decode_rows<V, true, T>(a, stride); });
-    else
-        run_grid(grid, 32 * W, smem, [&] { qsgd::decode_rows<V, false, T>(a, stride); });
-}
 template <class T>
 static void run_t(const qsgd::DecodeArgs& a, bool acc, unsigned grid, unsigned W) {
-    const uint32_t stride = qsgd::rows_stride_words(a.d, sizeof(T));
+    const uint32_t stride = qsgd::rows_stride_words(sizeof(T));
     const size_t smem = 4 * (size_t)qsgd::kLutSize + (size_t)W * 32 * stride * 4;
-    switch (qsgd::fast_v(a.d)) {
-        case 1: run<1, T>(a, acc, grid, W, stride, smem); break;
-        case 2: run<2, T>(a, acc, grid, W, stride, smem); break;
-        case 4: run<4, T>(a, acc, grid, W, stride, smem); break;
-        default: run<8, T>(a, acc, grid, W, stride, smem); break;
-    }
+    if (acc)
+        run_grid(grid, 32 * W, smem, [&] { qsgd::decode_rows<true, T>(a, stride); });
+    else
+        run_grid(grid, 32 * W, smem, [&] { qsgd::decode_rows<false, T>(a, stride); });
 }
 
 // Several streams: decode_rows_multi over K streams, 16 to a launch as the library

@@ -36,7 +36,7 @@ def rows_exe(tmp_path_factory):
         shutil.copy(os.path.join(CSRC, h), src_dir / h)
     (src_dir / "qsgd_device.cuh").write_text(_host_source(open(os.path.join(CSRC, "qsgd_device.cuh")).read()))
     src = open(os.path.join(CSRC, "qsgd_decode_rows.cu")).read()
-    cut = src.index("template <int V, bool kAcc, class T>\ncudaError_t launch_rows_v")
+    cut = src.index("template <bool kAcc, class T>\ncudaError_t launch_rows_t")
     (src_dir / "rows_emu.inc").write_text(_host_source(src[:cut]) + "}  // namespace\n}  // namespace qsgd\n")
     exe = d / "rows_main"
     r = subprocess.run(["g++", "-O1", "-std=c++17", "-ffp-contract=off", "-pthread", "-I", EMU, "-I", str(src_dir),
@@ -86,6 +86,9 @@ CASES = [
     (3_001, 4, 2, False, 2, 2, "normal"),
     (6_000, 1000, 127, False, 1, 2, "layered"),
     (1, 512, 16, True, 1, 1, "normal"),
+    # gaps past the ring of two segments (records held back until their segment)
+    (20_000, 1024, 1, False, 2, 2, "heavy_tailed_sparse"),
+    (20_000, 1024, 200, True, 2, 2, "heavy_tailed_sparse"),
     # 16-bit codes (s > 127): large levels, and records the table never holds
     (20_000, 512, 256, False, 2, 2, "normal"),
     (20_000, 512, 256, True, 2, 2, "layered"),
@@ -108,6 +111,25 @@ def test_row_decoder_matches_oracle(rows_exe, tmp_path, oracle_lib, n, d, s, acc
     else:
         ref, rst = oracle_lib.decode(words, offsets, n, d, s)
     assert rst == 0
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("d,s", [(1024, 16), (1000, 300)])
+def test_row_decoder_far_records(rows_exe, tmp_path, oracle_lib, d, s):
+    """Buckets whose first record lies more than two segments ahead (a bit-serial
+    gap, held back until its segment), next to dense buckets."""
+    n = 64 * d
+    rng = np.random.default_rng(d)
+    v = np.zeros(n, np.float32)
+    for b in range(0, 64, 2):
+        pos = rng.integers(300, d, size=2)
+        v[b * d + pos] = rng.standard_normal(2).astype(np.float32)
+        v[(b + 1) * d:(b + 2) * d] = rng.standard_normal(d).astype(np.float32)
+    words, offsets, _, st = oracle_lib.encode(v, d, s, seed=4)
+    assert st == 0
+    got, status = _run(rows_exe, tmp_path, words, offsets, n, d, s, False, 2, 2, _base(n, d, False))
+    ref, rst = oracle_lib.decode(words, offsets, n, d, s)
+    assert status == 0 and rst == 0
     assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
 
 
