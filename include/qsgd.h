@@ -94,11 +94,17 @@ QSGD_API uint64_t qsgd_num_buckets(uint64_t n, uint32_t d);
  * bits and the gaps of a bucket sum to at most m_b.  Returns 0 for invalid d or s. */
 QSGD_API uint64_t qsgd_max_encoded_words(uint64_t n, uint32_t d, uint32_t s);
 
-/* Bytes of device workspace qsgd_encode needs for (n, d, s).  The workspace holds
- * the scan state of the single-pass encoder (tile descriptors, tail words, per-bucket
- * norms for large buckets).  It must be zero-filled once before its first use
- * (qsgd_workspace_init); every encode leaves it ready for the next one.  One
- * workspace must not be used by two encodes that may run at the same time. */
+/* Bytes of device workspace qsgd_encode (and _ex, _ef) needs for (n, d, s).  The
+ * workspace holds, for the shapes the two-launch encoder takes (d % 4 == 0,
+ * 4 <= d <= 1024, or d <= 16384 for s <= 31, 16-byte aligned input): a control
+ * block, one scan descriptor per 256 buckets, each bucket's bit count and a staging
+ * slot per bucket of the bucket's largest possible size; for the other shapes, the
+ * scan state of the one-pass encoder (control block, tile descriptors, tail words,
+ * per-bucket norms for large buckets).  The size is the larger of the two, so one
+ * workspace serves every encoder for (n, d, s).  It must be zero-filled once before
+ * its first use (qsgd_workspace_init); every encode leaves it ready for the next
+ * one, whichever encoder ran before.  One workspace must not be used by two encodes
+ * that may run at the same time. */
 QSGD_API size_t qsgd_encode_workspace_bytes(uint64_t n, uint32_t d, uint32_t s);
 
 /* Zero-fills a workspace (cudaMemsetAsync on `stream`). */
@@ -106,8 +112,10 @@ QSGD_API int qsgd_workspace_init(void* d_ws, size_t ws_bytes, cudaStream_t strea
 
 /* Encoder: QSGD-quantises d_in[0..n) bucket by bucket and writes the Elias-omega
  * stream.  (Definition paragraph and the two claims cited above.)
- *   d_in            fp32[n], any alignment (16-byte alignment and d % 4 == 0 take
- *                   the fast path)
+ *   d_in            fp32[n], any alignment (16-byte alignment with d % 4 == 0 and
+ *                   d within the limits above takes the two-launch encoder: a
+ *                   bucket coder into the staging slots, then a compaction that
+ *                   scans the bit counts and moves the bits to their offsets)
  *   seed            Philox key of the stochastic rounding
  *   d_words         uint32[words_capacity]; words past ceil(offsets[nb]/32) are
  *                   not written
@@ -169,10 +177,13 @@ QSGD_API int qsgd_decode(const uint32_t* d_words, uint64_t num_words, const uint
  *   h_words, h_num_words, h_offsets  host arrays of K entries holding device
  *                                    pointers / word counts (copied at the call)
  *   1 <= K <= 1024
- * Status bits as for qsgd_decode.  Two or more streams (d % 4 == 0, d <= 4096,
- * s < 1024, 16-byte aligned d_out) are decoded side by side, up to 16 to a launch, and
- * d_out is read and written once per eight streams.  Other cases take one launch per
- * stream.  The result is the same either way. */
+ * Status bits as for qsgd_decode.  Up to 16 streams go to one launch (launches in
+ * stream order).  With a 16-byte aligned d_out and d % 4 == 0: for d <= 4096 and
+ * s < 1024 the streams are decoded side by side (a warp per stream) and d_out is read
+ * and written once per eight streams; for d <= 1024 and larger s they are added onto
+ * fp32 tiles one after another; for d > 1024 the launch fills the buckets' outputs
+ * with +0-added values and then adds each stream's records in order.  One stream on
+ * d <= 1024 takes the one-stream row decoder.  The result is the same on every path. */
 QSGD_API int qsgd_decode_accumulate(const uint32_t* const* h_words, const uint64_t* h_num_words,
                            const uint64_t* const* h_offsets, int K, uint64_t n, uint32_t d,
                            uint32_t s, float* d_out, uint32_t* d_status, cudaStream_t stream);
@@ -205,9 +216,10 @@ QSGD_API int qsgd_decode_mean(const uint32_t* const* h_words, const uint64_t* h_
  * is bit-identical to qsgd_encode's for the same (d_in, n, d, s, seed).
  *   - The array is qsgd_static_workspace_limit() bytes (4 MiB).  Every GPU that
  *     loads the library holds it until the process exits.  A problem whose
- *     qsgd_encode_workspace_bytes(n, d, s) exceeds it is rejected with
- *     QSGD_ERR_STATIC_LIMIT before anything is enqueued (about 1.4 million
- *     buckets at d = 512).
+ *     one-pass scan state does not fit is rejected with QSGD_ERR_STATIC_LIMIT
+ *     before anything is enqueued (about 1.4 million buckets at d = 512).  A
+ *     problem whose staging slots also fit takes the two-launch encoder; the
+ *     others take the one-pass encoder.  The stream is the same either way.
  *   - The first call on a device looks up the array's device address (once per
  *     device, with that device current).  Make that first call before any stream
  *     capture.

@@ -9,18 +9,22 @@
 // receiver in "distributed data-parallel optimization", same paragraph) adds the
 // decoded stream onto the output: out_i <- fl(out_i + q_i).
 //
-// One stream (decode_rows): each lane of a warp parses one bucket (buckets are
-// independent prefix-code streams located by the offsets header), 32 consecutive
-// buckets to a warp.  With byte codes, records are decoded through a shared-memory
-// table of the whole records at the start of a 12-bit window (up to two per entry),
-// two lookups a step; with 16-bit codes (large s, where nearly every coordinate has
-// a record), through a table of omega codes, one lookup for the gap and one for the
-// level.  Longer records take a bit-serial path.  The lane stores each record's code
-// (sign << 7 | k in a byte for s <= 127, sign << 15 | k in 16 bits for s <= 32767)
-// in its bucket's row of a zeroed ring of codes; no lane waits for another while
-// parsing.  Segment by segment, the warp converts the rows to fp32 and writes each
-// bucket's columns with coalesced 16-byte stores (decode-accumulate first reads the
-// output, which a prefetch to L2 issued before the parse has brought in).
+// One stream: each lane of a warp parses one bucket (buckets are independent
+// prefix-code streams located by the offsets header), 32 consecutive buckets to a
+// warp, and stores each record's code at its index in its bucket's row of a zeroed
+// staging area in shared memory; no lane waits for another while parsing.  The warp
+// then converts the rows to fp32 and writes each bucket with coalesced 16-byte
+// stores (decode-accumulate first reads the output, which a prefetch to L2 issued
+// before the parse has brought in).
+//   - decode_rows (s <= 127): byte codes sign << 7 | k in whole rows of d codes;
+//     records through a table of the whole records at the start of a 12-bit window
+//     (up to two per entry), two lookups a step.
+//   - decode_rows_ring (127 < s <= 32767, where nearly every coordinate has a
+//     record): 16-bit codes sign << 15 | k in a ring of two 128-column segments per
+//     row, written back segment by segment (half the shared memory of whole rows,
+//     twice the warps); records through a table of omega codes, one lookup for the
+//     gap and one for the level.
+// Longer records take a bit-serial path.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -207,6 +211,200 @@ template <class T>
 __device__ __forceinline__ T row_code(uint32_t sign, uint32_t k) {
     return static_cast<T>((sign << (8 * sizeof(T) - 1)) | k);
 }
+// The output of bucket bb as lane `lane` reads it in the write-back: float4 i is
+// coordinates 4 (lane + 32 i) .. + 3, zeros past the bucket's end.
+template <int V>
+__device__ __forceinline__ void load_row(const DecodeArgs& a, uint64_t bb, int lane, float4 (&o)[V]) {
+    const uint32_t mm = static_cast<uint32_t>(min(static_cast<uint64_t>(a.d), a.n - bb * a.d));
+    const float* gp = a.out + bb * a.d;
+#pragma unroll
+    for (int i = 0; i < V; ++i) {
+        const uint32_t c = 4u * (static_cast<uint32_t>(lane) + 32u * i);
+        o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (c + 4 <= mm) {
+            o[i] = __ldcs(reinterpret_cast<const float4*>(gp + c));
+        } else if (c < mm) {
+            o[i].x = gp[c];
+            if (c + 1 < mm) o[i].y = gp[c + 1];
+            if (c + 2 < mm) o[i].z = gp[c + 2];
+        }
+    }
+}
+
+template <int V, bool kAcc>
+__global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows(const __grid_constant__ DecodeArgs a,
+                                                                   uint32_t stride_w) {
+    extern __shared__ __align__(16) uint32_t smem[];
+    uint32_t* const lut = smem;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int W = blockDim.x >> 5;
+    uint32_t* const rows = smem + kLutSize + static_cast<uint32_t>(warp) * 32u * stride_w;
+    uint8_t* const myrow = reinterpret_cast<uint8_t*>(rows + static_cast<uint32_t>(lane) * stride_w);
+    rows_lut_fill(lut, a.s, tid, blockDim.x);
+    __syncthreads();
+    const StreamRef st = a.streams[0];
+    const float fs = __uint2float_rn(a.s);
+    const uint32_t d = a.d;
+    const uint64_t ngroups = (a.nb + 31) / 32;
+    for (uint64_t g = blockIdx.x + static_cast<uint64_t>(gridDim.x) * warp; g < ngroups;
+         g += static_cast<uint64_t>(gridDim.x) * W) {
+        const uint64_t b = g * 32 + lane;
+        const bool live = b < a.nb;
+        const uint32_t m = live ? static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - b * d)) : 0u;
+        if constexpr (kAcc) {  // bring the group's output into L2 while the records are parsed
+            const float* gp = a.out + g * 32 * d;
+            const uint64_t gbytes = 4 * (min(a.n, (g + 1) * 32 * d) - g * 32 * d);
+            for (uint64_t off = static_cast<uint64_t>(lane) * 128; off < gbytes; off += 32 * 128)
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const char*>(gp) + off));
+        }
+        // zero the warp's rows (32 * stride_w words, a multiple of four)
+        for (uint32_t q = lane; q < 8u * stride_w; q += 32)
+            reinterpret_cast<uint4*>(rows)[q] = make_uint4(0u, 0u, 0u, 0u);
+        // open this lane's bucket: header checks and the norm
+        bool bad = false;
+        RowReader r;
+        r.left = 0;
+        float scale = 0.f;
+        if (live) {
+            const uint64_t begin = st.offsets[b];
+            const uint64_t end = st.offsets[b + 1];
+            if (!(end >= begin && end - begin >= 32 && end <= st.num_words * 32 && end - begin < (1ull << 30))) {
+                bad = true;
+            } else {
+                r.init(st.words, st.num_words, begin, static_cast<uint32_t>(end - begin));
+                const uint32_t nbits = r.peek();
+                r.advance(32);
+                const float norm = __uint_as_float(nbits);
+                if (nbits == 0) {
+                    bad = r.left != 0;
+                    r.left = 0;
+                } else if (!(isfinite(norm) && norm > 0.f)) {
+                    bad = true;
+                    r.left = 0;
+                } else {
+                    scale = __fdiv_rn(norm, fs);
+                    if (!(scale > 0.f) && r.left != 0) {  // a zero scale carries no records
+                        bad = true;
+                        r.left = 0;
+                    }
+                }
+            }
+        }
+        __syncwarp();
+        // --- parse: every record's code into the lane's row -------------------------
+        uint32_t next = 0;  // bucket-local index after the last record
+        if (bad) r.left = 0;
+        for (uint32_t it = 0; __any_sync(kWarpAll, r.left > 0); ++it) {
+            if (it == kParseGuard) {
+                bad = bad || r.left > 0;
+                break;
+            }
+            if (r.left > 0) {
+                // up to two table entries a step, each up to two records: the 32 bits at
+                // the cursor hold both 12-bit windows (the first takes at most 12 bits);
+                // a record is taken only when it ends inside the bucket
+                const uint32_t w = r.peek();
+                const uint32_t e = lut[w >> (32 - kLutBits)];
+                const uint32_t len1 = e & 15u;
+                if (len1 != 0u) {
+                    const uint32_t len2 = (e >> 4) & 15u;
+                    const bool two = static_cast<int32_t>(len2) <= r.left;
+                    uint32_t used = two ? len2 : len1;
+                    next += (e >> 8) & 15u;
+                    myrow[min(next - 1u, d)] = static_cast<uint8_t>((e >> 16) & 0xFFu);
+                    const uint32_t c2 = e >> 24;
+                    if (two && c2 != 0u) {
+                        next += (e >> 12) & 15u;
+                        myrow[min(next - 1u, d)] = static_cast<uint8_t>(c2);
+                    }
+                    if (two) {
+                        const uint32_t f = lut[(w << used) >> (32 - kLutBits)];
+                        const uint32_t flen1 = f & 15u;
+                        if (flen1 != 0u && static_cast<int32_t>(used + flen1) <= r.left) {
+                            const uint32_t flen2 = (f >> 4) & 15u;
+                            const bool ftwo = static_cast<int32_t>(used + flen2) <= r.left;
+                            next += (f >> 8) & 15u;
+                            myrow[min(next - 1u, d)] = static_cast<uint8_t>((f >> 16) & 0xFFu);
+                            const uint32_t fc2 = f >> 24;
+                            if (ftwo && fc2 != 0u) {
+                                next += (f >> 12) & 15u;
+                                myrow[min(next - 1u, d)] = static_cast<uint8_t>(fc2);
+                            }
+                            used += ftwo ? flen2 : flen1;
+                        }
+                    }
+                    r.advance(used);
+                } else {
+                    uint32_t gap = 0, sign = 0, k = 0;
+                    if (slow_record(r, a.s, gap, sign, k)) {
+                        next += gap;
+                        myrow[min(next - 1u, d)] = row_code<uint8_t>(sign, k);
+                    } else {
+                        bad = true;
+                        r.left = 0;
+                    }
+                }
+            }
+        }
+        // every record index below m, and the bucket consumed exactly (a record that
+        // overran leaves left negative; an index past m lands in the row's padding)
+        if (live && !bad && (next > m || r.left != 0)) bad = true;
+        __syncwarp();
+        // --- write the rows back: row rr is bucket g*32 + rr -----------------------
+        // (decode-accumulate reads the next row's output before it stores this row's,
+        // so that two rows of loads are in flight)
+        const int nrows = static_cast<int>(min(static_cast<uint64_t>(32), a.nb - g * 32));
+        float4 cur[kAcc ? V : 1], nxt[kAcc ? V : 1];
+        if constexpr (kAcc) load_row<V>(a, g * 32, lane, cur);
+        for (int rr = 0; rr < nrows; ++rr) {
+            const uint64_t bb = g * 32 + rr;
+            const float sc = __shfl_sync(kWarpAll, scale, rr);
+            if constexpr (kAcc) {
+                if (rr + 1 < nrows) load_row<V>(a, bb + 1, lane, nxt);
+            }
+            const uint32_t mm = static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - bb * d));
+            const uint32_t* rowp = rows + static_cast<uint32_t>(rr) * stride_w;
+            float* gp = a.out + bb * d;
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                const uint32_t q = static_cast<uint32_t>(lane) + 32u * i;
+                const uint32_t c = 4u * q;
+                if (c < mm) {
+                    uint32_t code[4];
+                    const uint32_t w = rowp[q];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) code[j] = ((w >> (8 * j)) & 0x7Fu) | (((w >> (8 * j)) & 0x80u) << 24);
+                    float v[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        // code[j] = k | sign << 31: k as fp32 through the 2^23 offset (exact
+                        // for k < 2^23), times the step, the sign last
+                        const float kf = __fsub_rn(__uint_as_float(0x4B000000u | (code[j] & 0x7FFFFFFFu)), 8388608.0f);
+                        v[j] = __uint_as_float(__float_as_uint(__fmul_rn(sc, kf)) | (code[j] & 0x80000000u));
+                    }
+                    if constexpr (kAcc) {
+                        v[0] = __fadd_rn(cur[i].x, v[0]);
+                        v[1] = __fadd_rn(cur[i].y, v[1]);
+                        v[2] = __fadd_rn(cur[i].z, v[2]);
+                        v[3] = __fadd_rn(cur[i].w, v[3]);
+                    }
+                    if (c + 4 <= mm) {
+                        __stcs(reinterpret_cast<float4*>(gp + c), make_float4(v[0], v[1], v[2], v[3]));
+                    } else {
+                        for (uint32_t j = 0; j < 4 && c + j < mm; ++j) gp[c + j] = v[j];
+                    }
+                }
+            }
+            if constexpr (kAcc) {
+#pragma unroll
+                for (int i = 0; i < V; ++i) cur[i] = nxt[i];
+            }
+        }
+        if (bad) atomicOr(a.status, QSGD_ST_BAD_STREAM);
+        __syncwarp();
+    }
+}
+
 // Segments and the ring of codes: the warp decodes its 32 buckets kRSeg columns at a
 // time and writes each segment back as soon as every lane has parsed past it, so
 // the output stores of one segment overlap the parse of the next.  A row holds two
@@ -221,23 +419,19 @@ constexpr uint32_t kRSeg = QSGD_ROWS_SEG;
 constexpr uint32_t kRRing = 2 * kRSeg;
 static_assert(kRSeg % 128 == 0 && kRSeg >= 128, "a segment is whole float4 columns of the warp");
 constexpr int kRVec = static_cast<int>(kRSeg / 128);  // float4 per lane per row per segment
+constexpr int kRBatch = 8;                             // rows whose output is loaded together
 
-template <bool kAcc, class T>
-__global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows(const __grid_constant__ DecodeArgs a,
+template <bool kAcc>
+__global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows_ring(const __grid_constant__ DecodeArgs a,
                                                                    uint32_t stride_w) {
     extern __shared__ __align__(16) uint32_t smem[];
-    uint32_t* const lut = smem;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int W = blockDim.x >> 5;
     uint32_t* const rows = smem + kLutSize + static_cast<uint32_t>(warp) * 32u * stride_w;
-    T* const myrow = reinterpret_cast<T*>(rows + static_cast<uint32_t>(lane) * stride_w);
-    // byte codes (s <= 127): the two-record table; 16-bit codes: the omega table,
-    // looked up for the gap and then for the level
-    const uint16_t* const olut = reinterpret_cast<const uint16_t*>(smem);
-    if constexpr (sizeof(T) == 1)
-        rows_lut_fill(lut, a.s, tid, blockDim.x);
-    else
-        omega_lut_fill(reinterpret_cast<uint16_t*>(smem), tid, blockDim.x);
+    uint16_t* const myrow = reinterpret_cast<uint16_t*>(rows + static_cast<uint32_t>(lane) * stride_w);
+    // the omega table, looked up for the gap and then for the level
+    uint16_t* const olut = reinterpret_cast<uint16_t*>(smem);
+    omega_lut_fill(olut, tid, blockDim.x);
     __syncthreads();
     const StreamRef st = a.streams[0];
     const float fs = __uint2float_rn(a.s);
@@ -297,7 +491,7 @@ __global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows(const __grid_c
         for (uint32_t lo = 0; lo < d; lo += kRSeg) {
             const uint32_t hi = lo + kRSeg;
             if (pend && pidx < hi + kRSeg) {
-                myrow[pidx & (kRRing - 1u)] = static_cast<T>(pcode);
+                myrow[pidx & (kRRing - 1u)] = static_cast<uint16_t>(pcode);
                 pend = false;
             }
             // --- parse until every lane has passed column hi (or ended) ---------------
@@ -312,60 +506,21 @@ __global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows(const __grid_c
                     continue;
                 }
                 if (!act) continue;
-                if constexpr (sizeof(T) == 2) {
-                    // one record a step: omega(gap) (<= 12 bits), the sign, omega(k)
-                    // (<= 12 bits) from the 32 bits at the cursor; k <= 63 < s
-                    const uint32_t w = r.peek();
-                    const uint32_t ge = olut[w >> (32 - kLutBits)];
-                    const uint32_t gl = ge & 15u;
-                    const uint32_t w2 = w << gl;
-                    const uint32_t ke = olut[(w2 << 1) >> (32 - kLutBits)];
-                    const uint32_t kl = ke & 15u;
-                    if (gl != 0u && kl != 0u) {
-                        next += ge >> 4;
-                        myrow[min(next - 1u, d) & (kRRing - 1u)] = row_code<T>(w2 >> 31, ke >> 4);
-                        r.advance(gl + 1u + kl);
-                        continue;
-                    }
-                } else {
-                    // up to two table entries a step, each up to two records: the 32 bits
-                    // at the cursor hold both 12-bit windows (the first takes at most 12
-                    // bits); a second record is taken only when it ends inside the bucket
-                    const uint32_t w = r.peek();
-                    const uint32_t e = lut[w >> (32 - kLutBits)];
-                    const uint32_t len1 = e & 15u;
-                    if (len1 != 0u) {
-                        const uint32_t len2 = (e >> 4) & 15u;
-                        const bool two = static_cast<int32_t>(len2) <= r.left;
-                        uint32_t used = two ? len2 : len1;
-                        next += (e >> 8) & 15u;
-                        myrow[min(next - 1u, d) & (kRRing - 1u)] = static_cast<T>((e >> 16) & 0xFFu);
-                        const uint32_t c2 = e >> 24;
-                        if (two && c2 != 0u) {
-                            next += (e >> 12) & 15u;
-                            myrow[min(next - 1u, d) & (kRRing - 1u)] = static_cast<T>(c2);
-                        }
-                        if (two) {
-                            const uint32_t f = lut[(w << used) >> (32 - kLutBits)];
-                            const uint32_t flen1 = f & 15u;
-                            if (flen1 != 0u && static_cast<int32_t>(used + flen1) <= r.left) {
-                                const uint32_t flen2 = (f >> 4) & 15u;
-                                const bool ftwo = static_cast<int32_t>(used + flen2) <= r.left;
-                                next += (f >> 8) & 15u;
-                                myrow[min(next - 1u, d) & (kRRing - 1u)] = static_cast<T>((f >> 16) & 0xFFu);
-                                const uint32_t fc2 = f >> 24;
-                                if (ftwo && fc2 != 0u) {
-                                    next += (f >> 12) & 15u;
-                                    myrow[min(next - 1u, d) & (kRRing - 1u)] = static_cast<T>(fc2);
-                                }
-                                used += ftwo ? flen2 : flen1;
-                            }
-                        }
-                        r.advance(used);
-                        continue;
-                    }
+                // one record a step: omega(gap) (<= 12 bits), the sign, omega(k) (<= 12
+                // bits) from the 32 bits at the cursor; k <= 63 < s, so no level check
+                const uint32_t w = r.peek();
+                const uint32_t ge = olut[w >> (32 - kLutBits)];
+                const uint32_t gl = ge & 15u;
+                const uint32_t w2 = w << gl;
+                const uint32_t ke = olut[(w2 << 1) >> (32 - kLutBits)];
+                const uint32_t kl = ke & 15u;
+                if (gl != 0u && kl != 0u) {
+                    next += ge >> 4;
+                    myrow[min(next - 1u, d) & (kRRing - 1u)] = row_code<uint16_t>(w2 >> 31, ke >> 4);
+                    r.advance(gl + 1u + kl);
+                    continue;
                 }
-                // a record the tables do not hold, bit by bit
+                // a record the table does not hold, bit by bit
                 uint32_t gap = 0, sign = 0, k = 0;
                 if (slow_record(r, a.s, gap, sign, k)) {
                     next += gap;
@@ -373,9 +528,9 @@ __global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows(const __grid_c
                     if (idx >= hi + kRSeg) {
                         pend = true;
                         pidx = idx;
-                        pcode = row_code<T>(sign, k);
+                        pcode = row_code<uint16_t>(sign, k);
                     } else {
-                        myrow[idx & (kRRing - 1u)] = row_code<T>(sign, k);
+                        myrow[idx & (kRRing - 1u)] = row_code<uint16_t>(sign, k);
                     }
                 } else {
                     bad = true;
@@ -384,80 +539,75 @@ __global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows(const __grid_c
             }
             __syncwarp();
             // --- write back columns [lo, hi) of the 32 rows, and clear them ----------
-            // (decode-accumulate reads the next row's output before it stores this
-            // row's, so that two rows of loads are in flight)
-            float4 cur[kAcc ? kRVec : 1], nxt[kAcc ? kRVec : 1];
-            auto load_seg = [&](int rr, float4 (&o)[kAcc ? kRVec : 1]) {
-                const uint64_t bb = g * 32 + rr;
-                const uint32_t mm = static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - bb * d));
-                const float* gp = a.out + bb * d;
+            // (decode-accumulate loads the output of kRBatch rows at a time, so that
+            // their loads are in flight together)
+            for (int r0 = 0; r0 < nrows; r0 += kRBatch) {
+                float4 o[kAcc ? kRBatch * kRVec : 1];
+                if constexpr (kAcc) {
 #pragma unroll
-                for (int i = 0; i < kRVec; ++i) {
-                    const uint32_t c = lo + 4u * (static_cast<uint32_t>(lane) + 32u * i);
-                    o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-                    if (c + 4 <= mm) {
-                        o[i] = __ldcs(reinterpret_cast<const float4*>(gp + c));
-                    } else if (c < mm) {
-                        o[i].x = gp[c];
-                        if (c + 1 < mm) o[i].y = gp[c + 1];
-                        if (c + 2 < mm) o[i].z = gp[c + 2];
+                    for (int t = 0; t < kRBatch; ++t) {
+                        const int rr = r0 + t;
+                        const uint64_t bb = g * 32 + rr;
+                        const uint32_t mm = rr < nrows ? static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - bb * d)) : 0u;
+                        const float* gp = a.out + bb * d;
+#pragma unroll
+                        for (int i = 0; i < kRVec; ++i) {
+                            const uint32_t c = lo + 4u * (static_cast<uint32_t>(lane) + 32u * i);
+                            float4& x = o[t * kRVec + i];
+                            x = make_float4(0.f, 0.f, 0.f, 0.f);
+                            if (c + 4 <= mm) {
+                                x = __ldcs(reinterpret_cast<const float4*>(gp + c));
+                            } else if (c < mm) {
+                                x.x = gp[c];
+                                if (c + 1 < mm) x.y = gp[c + 1];
+                                if (c + 2 < mm) x.z = gp[c + 2];
+                            }
+                        }
                     }
                 }
-            };
-            if constexpr (kAcc) load_seg(0, cur);
-            for (int rr = 0; rr < nrows; ++rr) {
-                const uint64_t bb = g * 32 + rr;
-                const float sc = __shfl_sync(kWarpAll, scale, rr);
-                if constexpr (kAcc) {
-                    if (rr + 1 < nrows) load_seg(rr + 1, nxt);
-                }
-                const uint32_t mm = static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - bb * d));
-                uint32_t* const rowp = rows + static_cast<uint32_t>(rr) * stride_w;
-                float* const gp = a.out + bb * d;
 #pragma unroll
-                for (int i = 0; i < kRVec; ++i) {
-                    const uint32_t c = lo + 4u * (static_cast<uint32_t>(lane) + 32u * i);
-                    if (c < mm) {
-                        const uint32_t q = (c & (kRRing - 1u)) >> 2;  // four codes
-                        uint32_t code[4];
-                        if constexpr (sizeof(T) == 1) {
-                            const uint32_t w = rowp[q];
-                            rowp[q] = 0u;
+                for (int t = 0; t < kRBatch; ++t) {
+                    const int rr = r0 + t;
+                    if (rr >= nrows) break;
+                    const uint64_t bb = g * 32 + rr;
+                    const float sc = __shfl_sync(kWarpAll, scale, rr);
+                    const uint32_t mm = static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - bb * d));
+                    uint32_t* const rowp = rows + static_cast<uint32_t>(rr) * stride_w;
+                    float* const gp = a.out + bb * d;
 #pragma unroll
-                            for (int j = 0; j < 4; ++j)
-                                code[j] = ((w >> (8 * j)) & 0x7Fu) | (((w >> (8 * j)) & 0x80u) << 24);
-                        } else {
+                    for (int i = 0; i < kRVec; ++i) {
+                        const uint32_t c = lo + 4u * (static_cast<uint32_t>(lane) + 32u * i);
+                        if (c < mm) {
+                            const uint32_t q = (c & (kRRing - 1u)) >> 2;  // four codes
                             const uint2 w = reinterpret_cast<const uint2*>(rowp)[q];
                             reinterpret_cast<uint2*>(rowp)[q] = make_uint2(0u, 0u);
+                            uint32_t code[4];
                             code[0] = (w.x & 0x7FFFu) | ((w.x & 0x8000u) << 16);
                             code[1] = (w.x >> 16 & 0x7FFFu) | (w.x & 0x80000000u);
                             code[2] = (w.y & 0x7FFFu) | ((w.y & 0x8000u) << 16);
                             code[3] = (w.y >> 16 & 0x7FFFu) | (w.y & 0x80000000u);
-                        }
-                        float v[4];
+                            float v[4];
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            // code[j] = k | sign << 31: k as fp32 through the 2^23 offset
-                            // (exact for k < 2^23), times the step, the sign last
-                            const float kf = __fsub_rn(__uint_as_float(0x4B000000u | (code[j] & 0x7FFFFFFFu)), 8388608.0f);
-                            v[j] = __uint_as_float(__float_as_uint(__fmul_rn(sc, kf)) | (code[j] & 0x80000000u));
-                        }
-                        if constexpr (kAcc) {
-                            v[0] = __fadd_rn(cur[i].x, v[0]);
-                            v[1] = __fadd_rn(cur[i].y, v[1]);
-                            v[2] = __fadd_rn(cur[i].z, v[2]);
-                            v[3] = __fadd_rn(cur[i].w, v[3]);
-                        }
-                        if (c + 4 <= mm) {
-                            __stcs(reinterpret_cast<float4*>(gp + c), make_float4(v[0], v[1], v[2], v[3]));
-                        } else {
-                            for (uint32_t j = 0; j < 4 && c + j < mm; ++j) gp[c + j] = v[j];
+                            for (int j = 0; j < 4; ++j) {
+                                // code[j] = k | sign << 31: k as fp32 through the 2^23
+                                // offset (exact for k < 2^23), times the step, the sign last
+                                const float kf = __fsub_rn(__uint_as_float(0x4B000000u | (code[j] & 0x7FFFFFFFu)), 8388608.0f);
+                                v[j] = __uint_as_float(__float_as_uint(__fmul_rn(sc, kf)) | (code[j] & 0x80000000u));
+                            }
+                            if constexpr (kAcc) {
+                                const float4& x = o[t * kRVec + i];
+                                v[0] = __fadd_rn(x.x, v[0]);
+                                v[1] = __fadd_rn(x.y, v[1]);
+                                v[2] = __fadd_rn(x.z, v[2]);
+                                v[3] = __fadd_rn(x.w, v[3]);
+                            }
+                            if (c + 4 <= mm) {
+                                __stcs(reinterpret_cast<float4*>(gp + c), make_float4(v[0], v[1], v[2], v[3]));
+                            } else {
+                                for (uint32_t j = 0; j < 4 && c + j < mm; ++j) gp[c + j] = v[j];
+                            }
                         }
                     }
-                }
-                if constexpr (kAcc) {
-#pragma unroll
-                    for (int i = 0; i < kRVec; ++i) cur[i] = nxt[i];
                 }
             }
             __syncwarp();
@@ -817,16 +967,20 @@ __global__ void __launch_bounds__(kSparseBlock) decode_sparse(const __grid_const
     }
 }
 
-// Words of one staging row: a ring of kRRing codes, padded so that consecutive rows
-// start on different banks: stride = 1 mod 32 for byte codes; for 16-bit codes even
-// (the write-back reads 8 bytes a lane) and 2 mod 32.
-uint32_t rows_stride_words(uint32_t code_bytes) {
-    return kRRing * code_bytes / 4 + (code_bytes == 1 ? 1u : 2u);
+// Words of one row of byte codes: d codes and a padding code (where an index past the
+// bucket is parked), rounded to 1 mod 32 so that consecutive rows start on different
+// banks.
+uint32_t rows_stride_words(uint32_t d) {
+    const uint32_t need = (d + 1 + 3) / 4;
+    return ((need + 30) / 32) * 32 + 1;
 }
+// Words of one row of the ring of 16-bit codes: kRRing codes, even (the write-back
+// reads 8 bytes a lane) and 2 mod 32.
+constexpr uint32_t ring_stride_words() { return kRRing * 2 / 4 + 2; }
 
-template <bool kAcc, class T>
-cudaError_t launch_rows_t(const DecodeArgs& a, cudaStream_t stream) {
-    const uint32_t stride = rows_stride_words(sizeof(T));
+// One CTA per SM, its warps one group each where the groups allow: every SM busy.
+template <class Kernel>
+cudaError_t launch_row_kernel(Kernel kernel, bool& attr_done, const DecodeArgs& a, uint32_t stride, cudaStream_t stream) {
     int dev = 0, sms = 0, optin = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -835,18 +989,44 @@ cudaError_t launch_rows_t(const DecodeArgs& a, cudaStream_t stream) {
     const size_t lut_bytes = static_cast<size_t>(kLutSize) * sizeof(uint32_t);
     const int W_fit = static_cast<int>(std::min<size_t>(kRowsMaxWarps, (static_cast<size_t>(optin) - lut_bytes - 1024) / per_warp));
     if (W_fit < 1) return cudaErrorInvalidConfiguration;
-    // one CTA per SM, its warps one group each where the groups allow: every SM busy
     const uint64_t groups = (a.nb + 31) / 32;
     const int W = static_cast<int>(std::max<uint64_t>(1, std::min<uint64_t>(W_fit, (groups + sms - 1) / sms)));
     const size_t smem = lut_bytes + W * per_warp;
-    static bool attr_set[64] = {};
-    if (dev < 64 && !attr_set[dev]) {
-        cudaFuncSetAttribute(decode_rows<kAcc, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
-        attr_set[dev] = true;
+    if (!attr_done) {
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+        attr_done = true;
     }
     const uint64_t blocks = std::max<uint64_t>(1, std::min<uint64_t>(static_cast<uint64_t>(sms), (groups + W - 1) / W));
-    decode_rows<kAcc, T><<<static_cast<unsigned>(blocks), 32 * W, smem, stream>>>(a, stride);
+    kernel<<<static_cast<unsigned>(blocks), 32 * W, smem, stream>>>(a, stride);
     return cudaGetLastError();
+}
+
+template <int V, bool kAcc>
+cudaError_t launch_rows_v(const DecodeArgs& a, cudaStream_t stream) {
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    bool scratch = false;
+    return launch_row_kernel(decode_rows<V, kAcc>, dev < 64 ? attr_set[dev] : scratch, a, rows_stride_words(a.d), stream);
+}
+
+template <bool kAcc>
+cudaError_t launch_rows_ring(const DecodeArgs& a, cudaStream_t stream) {
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    bool scratch = false;
+    return launch_row_kernel(decode_rows_ring<kAcc>, dev < 64 ? attr_set[dev] : scratch, a, ring_stride_words(), stream);
+}
+
+template <bool kAcc>
+cudaError_t launch_rows_bytes(const DecodeArgs& a, cudaStream_t stream) {
+    switch (fast_v(a.d)) {
+        case 1: return launch_rows_v<1, kAcc>(a, stream);
+        case 2: return launch_rows_v<2, kAcc>(a, stream);
+        case 4: return launch_rows_v<4, kAcc>(a, stream);
+        default: return launch_rows_v<8, kAcc>(a, stream);
+    }
 }
 
 cudaError_t launch_rows_multi(const DecodeArgs& a, cudaStream_t stream) {
@@ -901,9 +1081,8 @@ bool decode_rows_shape(uint32_t d, uint32_t s, const float* out) {
 cudaError_t launch_decode_rows_multi(const DecodeArgs& a, cudaStream_t stream) { return launch_rows_multi(a, stream); }
 
 cudaError_t launch_decode_rows(const DecodeArgs& a, bool accumulate, cudaStream_t stream) {
-    if (a.s <= kRowsMaxS8)
-        return accumulate ? launch_rows_t<true, uint8_t>(a, stream) : launch_rows_t<false, uint8_t>(a, stream);
-    return accumulate ? launch_rows_t<true, uint16_t>(a, stream) : launch_rows_t<false, uint16_t>(a, stream);
+    if (a.s <= kRowsMaxS8) return accumulate ? launch_rows_bytes<true>(a, stream) : launch_rows_bytes<false>(a, stream);
+    return accumulate ? launch_rows_ring<true>(a, stream) : launch_rows_ring<false>(a, stream);
 }
 
 }  // namespace qsgd

@@ -16,8 +16,8 @@
 // 2. compact_stream: a CTA of 512 threads per tile of 256 buckets scans the bit
 //    counts (a block scan and a decoupled look-back over the tiles, Merrill &
 //    Garland 2016, reading 512 predecessors at a time), writes the offsets header,
-//    and moves every bucket's bits to their stream position with funnel shifts, one
-//    warp per bucket.  An output word belongs to the bucket that holds its first
+//    and moves every bucket's bits to their stream position with funnel shifts, 8 to
+//    32 lanes per bucket.  An output word belongs to the bucket that holds its first
 //    bit; that bucket's warp also reads the first bits of the next bucket, so every
 //    word has exactly one writer and the output needs no clearing.
 // The staging costs two extra passes over the compressed bytes (a few percent of
@@ -800,35 +800,70 @@ __global__ void __launch_bounds__(kCompactThreads, 2) compact_stream(const __gri
         if (b + 1 == a.nb) a.offsets[a.nb] = F + L;
     }
     __syncthreads();
-    // A warp per bucket, its lanes over the output words whose first bit lies in the
-    // bucket: word k is bits [delta + 32 k, + 32) of the bucket's staged bits, delta
-    // the distance from the bucket's start to the next word boundary; a word that runs
-    // past the bucket's end takes the first bits of the next bucket (always >= 32
-    // bits, so one word of it suffices).  Every output word has exactly one writer.
+    // G lanes per bucket (G = 8, 16 or 32, from the tile's mean bucket size), over the
+    // output words whose first bit lies in the bucket: word k is bits [delta + 32 k,
+    // + 32) of the bucket's staged bits, delta the distance from the bucket's start to
+    // the next word boundary; a word that runs past the bucket's end takes the first
+    // bits of the next bucket (always >= 32 bits, so one word of it suffices).  Every
+    // output word has exactly one writer.
     const uint32_t nt = static_cast<uint32_t>(min(static_cast<uint64_t>(kCompactBlock), a.nb - b0));
-    for (uint32_t i = warp; i < nt; i += kWarps) {
-        const uint64_t bb = b0 + i;
-        const uint32_t Lb = s_L[i];
-        const uint64_t F = X + s_R[i];
-        const uint64_t wf = (F + 31u) >> 5;
-        const uint32_t cnt = static_cast<uint32_t>(((F + Lb + 31u) >> 5) - wf);
-        const uint32_t delta = static_cast<uint32_t>((wf << 5) - F);
-        const uint32_t nw = (Lb + 31u) >> 5;
-        const uint32_t* src = a.stage + bb * a.slot_words;
-        for (uint32_t k = lane; k < cnt; k += 32) {
-            const uint32_t r = delta + 32u * k;  // bucket-relative bit of the word (< Lb)
-            const uint32_t a0 = src[k];
-            const uint32_t a1 = k + 1 < nw ? src[k + 1] : 0u;
-            uint32_t v = __funnelshift_l(a1, a0, delta);
-            if (r + 32u > Lb) {  // 1 <= Lb - r <= 31
-                const uint32_t hd = bb + 1 < a.nb ? a.stage[(bb + 1) * a.slot_words] : 0u;
-                v |= hd >> (Lb - r);
+    const uint32_t mean_words = total / (32u * nt);
+    const uint32_t G = mean_words < 8u ? 8u : mean_words < 16u ? 16u : 32u;
+    const uint32_t per_warp = 32u / G, sub = static_cast<uint32_t>(lane) / G, sl = static_cast<uint32_t>(lane) % G;
+    const uint32_t step = kWarps * per_warp;
+    // four buckets at a time, so that their loads are in flight together
+    constexpr int kU = 4;
+    for (uint32_t i0 = static_cast<uint32_t>(warp) * per_warp + sub; i0 < nt; i0 += kU * step) {
+        uint32_t cnt[kU], delta[kU], nw[kU], Lb[kU];
+        uint64_t wf[kU];
+        const uint32_t* src[kU];
+        uint32_t hd[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const uint32_t i = i0 + static_cast<uint32_t>(u) * step;
+            cnt[u] = 0u;
+            delta[u] = nw[u] = Lb[u] = hd[u] = 0u;
+            wf[u] = 0u;
+            src[u] = a.stage;
+            if (i < nt) {
+                const uint64_t bb = b0 + i;
+                Lb[u] = s_L[i];
+                const uint64_t F = X + s_R[i];
+                wf[u] = (F + 31u) >> 5;
+                cnt[u] = static_cast<uint32_t>(((F + Lb[u] + 31u) >> 5) - wf[u]);
+                delta[u] = static_cast<uint32_t>((wf[u] << 5) - F);
+                nw[u] = (Lb[u] + 31u) >> 5;
+                src[u] = a.stage + bb * a.slot_words;
+                // the next bucket's first word, for the word that runs past this one's end
+                if (bb + 1 < a.nb) hd[u] = a.stage[(bb + 1) * a.slot_words];
             }
-            const uint64_t w = wf + k;
-            if (w < a.cap_words)
-                a.words[w] = v;
-            else
-                report(a.status, QSGD_ST_OVERFLOW);
+        }
+        for (uint32_t k = sl;; k += G) {
+            uint32_t v[kU];
+            bool more = false;
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                v[u] = 0u;
+                if (k < cnt[u]) {
+                    const uint32_t r = delta[u] + 32u * k;  // bucket-relative bit of the word (< Lb)
+                    const uint32_t a0 = src[u][k];
+                    const uint32_t a1 = k + 1 < nw[u] ? src[u][k + 1] : 0u;
+                    v[u] = __funnelshift_l(a1, a0, delta[u]);
+                    if (r + 32u > Lb[u]) v[u] |= hd[u] >> (Lb[u] - r);  // 1 <= Lb - r <= 31
+                }
+                more = more || k + G < cnt[u];
+            }
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                if (k < cnt[u]) {
+                    const uint64_t w = wf[u] + k;
+                    if (w < a.cap_words)
+                        a.words[w] = v[u];
+                    else
+                        report(a.status, QSGD_ST_OVERFLOW);
+                }
+            }
+            if (!more) break;
         }
     }
     release_control(a.ctrl);

@@ -48,14 +48,32 @@ static void run_grid(unsigned grid, unsigned block, size_t smem, Kernel k) {
     for (auto& x : th) x.join();
 }
 
+template <int V>
+static void run_v(const qsgd::DecodeArgs& a, bool acc, unsigned grid, unsigned W, uint32_t stride, size_t smem) {
+    if (acc)
+        run_grid(grid, 32 * W, smem, [&] { qsgd::decode_rows<V, true>(a, stride); });
+    else
+        run_grid(grid, 32 * W, smem, [&] { qsgd::decode_rows<V, false>(a, stride); });
+}
 template <class T>
 static void run_t(const qsgd::DecodeArgs& a, bool acc, unsigned grid, unsigned W) {
-    const uint32_t stride = qsgd::rows_stride_words(sizeof(T));
+    if constexpr (sizeof(T) == 2) {
+        const uint32_t stride = qsgd::ring_stride_words();
+        const size_t smem = 4 * (size_t)qsgd::kLutSize + (size_t)W * 32 * stride * 4;
+        if (acc)
+            run_grid(grid, 32 * W, smem, [&] { qsgd::decode_rows_ring<true>(a, stride); });
+        else
+            run_grid(grid, 32 * W, smem, [&] { qsgd::decode_rows_ring<false>(a, stride); });
+        return;
+    }
+    const uint32_t stride = qsgd::rows_stride_words(a.d);
     const size_t smem = 4 * (size_t)qsgd::kLutSize + (size_t)W * 32 * stride * 4;
-    if (acc)
-        run_grid(grid, 32 * W, smem, [&] { qsgd::decode_rows<true, T>(a, stride); });
-    else
-        run_grid(grid, 32 * W, smem, [&] { qsgd::decode_rows<false, T>(a, stride); });
+    switch (qsgd::fast_v(a.d)) {
+        case 1: run_v<1>(a, acc, grid, W, stride, smem); break;
+        case 2: run_v<2>(a, acc, grid, W, stride, smem); break;
+        case 4: run_v<4>(a, acc, grid, W, stride, smem); break;
+        default: run_v<8>(a, acc, grid, W, stride, smem); break;
+    }
 }
 
 // Several streams: decode_rows_multi over K streams, 16 to a launch as the library

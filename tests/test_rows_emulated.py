@@ -36,7 +36,7 @@ def rows_exe(tmp_path_factory):
         shutil.copy(os.path.join(CSRC, h), src_dir / h)
     (src_dir / "qsgd_device.cuh").write_text(_host_source(open(os.path.join(CSRC, "qsgd_device.cuh")).read()))
     src = open(os.path.join(CSRC, "qsgd_decode_rows.cu")).read()
-    cut = src.index("template <bool kAcc, class T>\ncudaError_t launch_rows_t")
+    cut = src.index("// One CTA per SM, its warps one group each where the groups allow: every SM busy.")
     (src_dir / "rows_emu.inc").write_text(_host_source(src[:cut]) + "}  // namespace\n}  // namespace qsgd\n")
     exe = d / "rows_main"
     r = subprocess.run(["g++", "-O1", "-std=c++17", "-ffp-contract=off", "-pthread", "-I", EMU, "-I", str(src_dir),
