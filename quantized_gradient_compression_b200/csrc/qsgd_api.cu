@@ -367,7 +367,7 @@ int qsgd_decode_mean(const uint32_t* const* h_words, const uint64_t* h_num_words
         if (!h_words[j] || !h_offsets[j] || (reinterpret_cast<uintptr_t>(h_offsets[j]) & 7u) != 0)
             return QSGD_ERR_ARG;
     // the several-stream kernel: sum from +0 in stream order, divided in its last launch
-    if (decode_fast_shape(d, s, d_out) && K >= kMultiMinStreams)
+    if (decode_multi_shape(d, s, d_out) && K >= kMultiMinStreams)
         return decode_impl(h_words, h_num_words, h_offsets, K, n, d, s, d_out, d_status, stream, true, true);
     // other shapes and a few streams: stream 0 decoded into d_out, the others added in
     // order, then the division

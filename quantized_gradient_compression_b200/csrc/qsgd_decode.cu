@@ -1,4 +1,5 @@
-// QSGD decoder and decode-accumulate kernels (sm_100a).
+// QSGD decoders for the shapes the row decoders do not take, and the several-stream
+// kernel (sm_100a).
 //
 // Method: "QSGD (Quantized Stochastic Gradient Descent) with Elias Coding" (AIMech
 // curated entry).  The definition paragraph calls the coding "lossless prefix
@@ -10,13 +11,18 @@
 //
 // Layout of the work: buckets are independent prefix-code streams located by the
 // offsets header, so each lane of a warp parses one bucket.  The decoded values of
-// a segment of kSeg coordinates of each of the warp's 32 buckets are scattered into
-// a shared-memory staging tile (zero-filled, or loaded from the output for
-// decode-accumulate) and the tile is written back with coalesced 16-byte stores.
-// A record is normally decoded with one lookup of its first 12 bits in a
-// shared-memory table of complete records; longer records take a bit-serial path.
-// Every read is bounded by the bucket's [offsets[b], offsets[b+1]) range and by
-// the stream length.
+// a segment of coordinates of each of the warp's 32 buckets are scattered into a
+// shared-memory staging tile (zero-filled, or loaded from the output for
+// decode-accumulate) and the tile is written back.  A record is normally decoded
+// with one lookup of its first 12 bits in a shared-memory table of complete
+// records; longer records take a bit-serial path.  Every read is bounded by the
+// bucket's [offsets[b], offsets[b+1]) range and by the stream length.
+//   - decode_warp: any shape (d % 4 != 0, unaligned output), up to 16 streams a
+//     launch, each lane's per-stream state in shared memory.
+//   - decode_multi: two or more streams (and the mean) with d % 4 == 0, d <= 4096,
+//     s < 1024 and an aligned output, a warp per stream, side by side.
+// The launch routing (launch_decode) sends one stream with d <= 1024 to the row
+// decoders and d > 1024 to the large-bucket decoder (qsgd_decode_rows.cu).
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -318,8 +324,8 @@ __global__ void __launch_bounds__(kDecodeBlock) decode_warp(const __grid_constan
 }
 
 // ---------------------------------------------------------------------------
-// Fast decoder (one stream; d % 4 == 0, d <= kFastDecodeMaxD, s < 1024, 16-byte
-// aligned output), plain or accumulating.
+// Bit reader and record step of the several-stream kernel (d % 4 == 0,
+// d <= kMultiMaxD, s < 1024, 16-byte aligned output).
 //
 // Reader: a 64-bit left-aligned bit buffer -- the next unread bits of the bucket
 // are the top `valid` bits of `buf` (valid >= 32 after every refill) -- plus the
@@ -328,7 +334,7 @@ __global__ void __launch_bounds__(kDecodeBlock) decode_warp(const __grid_constan
 // detected when the bucket ends (the staging writes stay inside the segment by
 // construction), so the common path has no per-record bounds checks.
 // ---------------------------------------------------------------------------
-constexpr uint32_t kFastDecodeMaxD = 4096;
+constexpr uint32_t kMultiMaxD = 4096;
 constexpr uint32_t kFullMask = 0xFFFFFFFFu;
 
 struct BitBuf {
@@ -432,151 +438,6 @@ __device__ __forceinline__ bool slow_next(BitBuf& r, uint32_t s, float scale, ui
     idx = next - 1;
     vbits = __float_as_uint(__fmul_rn(scale, __uint2float_rn(k))) | sign;
     return true;
-}
-
-template <bool kAccumulate>
-__global__ void __launch_bounds__(kDecodeBlock) decode_fast(const __grid_constant__ DecodeArgs a) {
-    extern __shared__ __align__(16) uint32_t smem[];
-    uint32_t* lut = smem;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    float* stage = reinterpret_cast<float*>(smem + kLut) + warp * 32 * kStride;
-    build_record_lut(lut, a.s, tid, kDecodeBlock);
-    __syncthreads();
-    const StreamRef st = a.streams[0];
-    const float fs = __uint2float_rn(a.s);
-    const uint32_t d = a.d;
-    const uint64_t ngroups = (a.nb + 31) / 32;
-    const uint64_t gwarps = static_cast<uint64_t>(gridDim.x) * kDecWarps;
-    // write-back geometry: step i moves row 2i + (lane >> 4), columns 4 (lane & 15) .. +3
-    const uint32_t wrow = static_cast<uint32_t>(lane >> 4), wcol = static_cast<uint32_t>(lane & 15) * 4;
-    float* row = stage + lane * kStride;
-    for (uint64_t g = static_cast<uint64_t>(blockIdx.x) * kDecWarps + warp; g < ngroups; g += gwarps) {
-        const uint64_t b = g * 32 + lane;
-        const bool live = b < a.nb;
-        const uint32_t m = live ? static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - b * d)) : 0u;
-        // every row of the group is a whole bucket of d: no masks in the staging
-        const bool full = (g + 1) * 32 <= a.nb && (g + 1) * 32 * static_cast<uint64_t>(d) <= a.n;
-        bool bad = false;
-        BitBuf r;
-        r.left = 0;
-        float scale = 0.f;
-        if (live) {
-            const uint64_t begin = st.offsets[b];
-            const uint64_t end = st.offsets[b + 1];
-            if (!(end >= begin && end - begin >= 32 && end <= st.num_words * 32 && end - begin < (1ull << 30))) {
-                bad = true;
-            } else {
-                r.init(st.words, st.num_words, begin, static_cast<uint32_t>(end - begin));
-                const uint32_t nbits = r.top(32);
-                r.consume(32);
-                const float norm = __uint_as_float(nbits);
-                if (nbits == 0) {
-                    bad = r.left != 0;
-                    r.left = 0;
-                } else if (!(isfinite(norm) && norm > 0.f)) {
-                    bad = true;
-                    r.left = 0;
-                } else {
-                    scale = __fdiv_rn(norm, fs);
-                    if (!(scale > 0.f) && r.left != 0) {  // a zero scale carries no records
-                        bad = true;
-                        r.left = 0;
-                    }
-                }
-            }
-        }
-        uint32_t next = 0, pidx = kNoRecord, pval = 0;
-        if (!bad) table_next(r, lut, scale, next, pidx, pval);
-        for (uint32_t lo = 0; lo < d; lo += kSeg) {
-            // --- staging tile: zeros, or the current output ---------------------
-            // Step i covers row 2i + wrow (bucket g*32 + 2i + wrow), columns
-            // lo + wcol .. +3.  Rows past the last bucket and columns past a
-            // bucket's end are neither read nor written back (the ragged last
-            // group takes the same unrolled path, only masked).
-            if (kAccumulate) {
-                uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(stage + wrow * kStride + wcol));
-                const uint32_t c = lo + wcol;
-#pragma unroll
-                for (int i = 0; i < 16; ++i, dst += 2 * kStride * sizeof(float)) {
-                    const uint64_t bb = g * 32 + wrow + 2 * i;
-                    const uint32_t mm = full ? d : bb < a.nb ? static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - bb * d)) : 0u;
-                    if (c + 4 <= mm) {
-                        const float* src = a.out + bb * d + c;
-                        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src) : "memory");
-                    } else if (c < mm) {
-                        float* sp = stage + (wrow + 2 * i) * kStride + wcol;
-                        for (uint32_t e = 0; e < 4; ++e)
-                            if (c + e < mm) sp[e] = a.out[bb * d + c + e];
-                    }
-                }
-                asm volatile("cp.async.wait_all;\n" ::: "memory");
-            } else {
-                for (int q = lane; q < 32 * kStride / 4; q += 32)
-                    reinterpret_cast<float4*>(stage)[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-            __syncwarp();
-            // --- scatter this segment's records -------------------------------
-            // Lanes whose next record is too long for the table park; the
-            // bit-serial path runs only when no lane has table work left, so the
-            // parked lanes of a warp are resolved together.
-            const uint32_t hi = lo + kSeg;
-            for (uint32_t it = 0;; ++it) {
-                const bool place = pidx < hi;
-                if (it == kLoopGuard) {
-                    bad = true;
-                    pidx = kNoRecord;
-                }
-                if (__any_sync(kFullMask, place) && it < kLoopGuard) {
-                    if (place) {
-                        float* dst = row + (pidx - lo);
-                        *dst = kAccumulate ? __fadd_rn(*dst, __uint_as_float(pval)) : __uint_as_float(pval);
-                        table_next(r, lut, scale, next, pidx, pval);
-                    }
-                } else if (__any_sync(kFullMask, pidx == kParked)) {
-                    if (pidx == kParked && !slow_next(r, a.s, scale, next, pidx, pval)) {
-                        bad = true;
-                        pidx = kNoRecord;
-                    }
-                } else {
-                    break;
-                }
-            }
-            __syncwarp();
-            // --- write the tile back (the first stream of an accumulation adds +0.0:
-            // (x + 0) + v == (x + v) + 0 for every x and v, -0.0 included) ------
-            {
-                const float* sp = stage + wrow * kStride + wcol;
-                const uint32_t c = lo + wcol;
-                const bool plus_zero = kAccumulate && a.first_group;
-#pragma unroll 4
-                for (int i = 0; i < 16; ++i, sp += 2 * kStride) {
-                    const uint64_t bb = g * 32 + wrow + 2 * i;
-                    const uint32_t mm = full ? d : bb < a.nb ? static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - bb * d)) : 0u;
-                    if (c < mm) {
-                        float4 v = *reinterpret_cast<const float4*>(sp);
-                        if (plus_zero) {
-                            v.x = __fadd_rn(v.x, 0.0f);
-                            v.y = __fadd_rn(v.y, 0.0f);
-                            v.z = __fadd_rn(v.z, 0.0f);
-                            v.w = __fadd_rn(v.w, 0.0f);
-                        }
-                        float* gp = a.out + bb * d + c;
-                        if (c + 4 <= mm) {
-                            *reinterpret_cast<float4*>(gp) = v;
-                        } else {
-                            const float e4[4] = {v.x, v.y, v.z, v.w};
-                            for (uint32_t e = 0; e < 4; ++e)
-                                if (c + e < mm) gp[e] = e4[e];
-                        }
-                    }
-                }
-            }
-            __syncwarp();
-        }
-        // every record index below m, and the bucket consumed exactly
-        if (live && !bad && (next > m || r.left != 0 || pidx != kNoRecord)) bad = true;
-        if (bad) atomicOr(a.status, QSGD_ST_BAD_STREAM);
-    }
 }
 
 // ---------------------------------------------------------------------------
@@ -743,48 +604,6 @@ __global__ void __launch_bounds__(kMultiBlock) decode_multi(const __grid_constan
     }
 }
 
-// Dynamic shared memory for a one-wave launch of `blocks` CTAs that needs `base`
-// bytes: padded so that no SM can hold more than ceil(blocks / SMs) CTAs.  The
-// hardware otherwise stacks up to the occupancy limit on some SMs and leaves
-// others short, and those SMs' issue-bound warps set the kernel's time.
-inline size_t balanced_smem(size_t base, uint64_t blocks, int dev, int sms, int per_sm) {
-    if (sms <= 0 || per_sm <= 1 || blocks == 0) return base;
-    const uint64_t target = (blocks + sms - 1) / sms;
-    if (target >= static_cast<uint64_t>(per_sm)) return base;
-    int per_sm_bytes = 0, reserved = 0;
-    cudaDeviceGetAttribute(&per_sm_bytes, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
-    cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
-    // target + 1 CTAs must not fit; target CTAs must
-    const size_t pad = static_cast<size_t>(per_sm_bytes) / (target + 1) - static_cast<size_t>(reserved) + 1;
-    if (pad <= base || target * (pad + reserved) > static_cast<size_t>(per_sm_bytes)) return base;
-    return pad;
-}
-
-template <bool kAccumulate>
-cudaError_t launch_fast_decode(const DecodeArgs& a, cudaStream_t stream) {
-    const size_t smem = kLut * sizeof(uint32_t) + static_cast<size_t>(kDecWarps) * 32 * kStride * sizeof(float);
-    static bool attr_set[64] = {};
-    int dev = 0, sms = 0, per_sm = 0;
-    cudaGetDevice(&dev);
-    if (dev < 64 && !attr_set[dev]) {
-        cudaFuncSetAttribute(decode_fast<kAccumulate>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-        attr_set[dev] = true;
-    }
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_fast<kAccumulate>, kDecodeBlock, smem);
-    if (e != cudaSuccess) return e;
-    if (per_sm < 1) return cudaErrorInvalidConfiguration;
-    const uint64_t groups = (a.nb + 31) / 32;
-    const uint64_t blocks = std::min<uint64_t>((groups + kDecWarps - 1) / kDecWarps, static_cast<uint64_t>(sms) * per_sm);
-#ifndef QSGD_NO_BALANCE
-    const size_t smem_launch = balanced_smem(smem, blocks, dev, sms, per_sm);
-#else
-    const size_t smem_launch = smem;
-#endif
-    decode_fast<kAccumulate><<<static_cast<unsigned>(blocks), kDecodeBlock, smem_launch, stream>>>(a);
-    return cudaGetLastError();
-}
-
 cudaError_t launch_multi(const DecodeArgs& a, cudaStream_t stream) {
     const size_t smem = kLut * sizeof(uint32_t) + static_cast<size_t>(kMultiWarps) * 32 * kMStride * sizeof(float);
     static bool attr_set[64] = {};
@@ -830,46 +649,29 @@ cudaError_t launch(const DecodeArgs& a, cudaStream_t stream) {
 
 }  // namespace
 
-bool decode_fast_shape(uint32_t d, uint32_t s, const float* out) {
-    return d % 4 == 0 && d <= kFastDecodeMaxD && s < 1024 && (reinterpret_cast<uintptr_t>(out) & 15u) == 0;
+bool decode_multi_shape(uint32_t d, uint32_t s, const float* out) {
+    return d % 4 == 0 && d <= kMultiMaxD && s < 1024 && (reinterpret_cast<uintptr_t>(out) & 15u) == 0;
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, bool accumulate, cudaStream_t stream) {
     if (a.nb == 0) return cudaSuccess;
-    const bool fast = decode_fast_shape(a.d, a.s, a.out);
+    const bool multi = decode_multi_shape(a.d, a.s, a.out);
     // the row decoders when the shape allows: one stream staged as codes; several
     // streams (and the mean) added onto fp32 tiles in stream order where the
     // several-stream kernel below, which decodes the streams side by side, does not
     // take the levels (s >= 1024)
     if (decode_rows_shape(a.d, a.s, a.out)) {
         if (a.K == 1 && !a.start_zero && a.div == 0.f) return launch_decode_rows(a, accumulate, stream);
-        if (!fast) return launch_decode_rows_multi(a, stream);
+        if (!multi) return launch_decode_rows_multi(a, stream);
     }
-    if (a.start_zero || a.div != 0.f) return fast ? launch_multi(a, stream) : cudaErrorInvalidValue;
+    // the mean in one pass: streams decoded side by side, the sum divided at the end
+    if (a.start_zero || a.div != 0.f) return multi ? launch_multi(a, stream) : cudaErrorInvalidValue;
     // buckets larger than the rows: a fill of the output, then the records
     if (decode_sparse_shape(a.d, a.out)) return launch_decode_sparse(a, accumulate, stream);
-    if (!fast) return accumulate ? launch<true>(a, stream) : launch<false>(a, stream);
-#ifndef QSGD_MULTI
-#define QSGD_MULTI 1
-#endif
-    // several streams: decoded side by side, the output moved once
-    if (QSGD_MULTI && accumulate && a.K >= 2) return launch_multi(a, stream);
-    auto one = [&](const DecodeArgs& x) -> cudaError_t {
-        return accumulate ? launch_fast_decode<true>(x, stream) : launch_fast_decode<false>(x, stream);
-    };
-    if (a.K == 1) return one(a);
-    // several streams (decode-accumulate): one launch per stream, in stream order
-    // on the one CUDA stream, so every coordinate still sees its adds left to
-    // right; between launches the output stays in L2
-    DecodeArgs o = a;
-    o.K = 1;
-    for (int j = 0; j < a.K; ++j) {
-        o.streams[0] = a.streams[j];
-        o.first_group = a.first_group && j == 0;
-        const cudaError_t e = one(o);
-        if (e != cudaSuccess) return e;
-    }
-    return cudaSuccess;
+    // several streams on the rows' shapes: decoded side by side, the output moved once
+    if (multi && accumulate && a.K >= 2) return launch_multi(a, stream);
+    // every other shape (d % 4 != 0, an unaligned output): one warp per 32 buckets
+    return accumulate ? launch<true>(a, stream) : launch<false>(a, stream);
 }
 
 }  // namespace qsgd

@@ -164,9 +164,9 @@ cudaError_t launch_decode_rows_multi(const DecodeArgs& a, cudaStream_t stream);
 // decode-accumulate (K <= 16 streams to a launch, in order).
 bool decode_sparse_shape(uint32_t d, const float* out);
 cudaError_t launch_decode_sparse(const DecodeArgs& a, bool accumulate, cudaStream_t stream);
-// Whether the one-lane-per-bucket decoders (and the several-stream kernel, which
-// start_zero / div need) take this shape.
-bool decode_fast_shape(uint32_t d, uint32_t s, const float* out);
+// Whether the several-stream kernel (decode_multi, which start_zero / div need)
+// takes this shape.
+bool decode_multi_shape(uint32_t d, uint32_t s, const float* out);
 
 // Fixed-width b-bit variant (b in {2, 4, 8}, checked by the caller).
 cudaError_t launch_bbit_encode(const float* in, float* ef, uint64_t n, uint32_t d, uint32_t b, uint64_t seed,

@@ -1,11 +1,10 @@
-// Runs the decoder kernels decode_fast (P = 0), decode_multi (P = -1) and
-// decode_warp (P = -2), compiled for the host under warp_emu.h, over
-// streams read from files.  argv: dir P accumulate [grid [mean]]
+// Runs the decoder kernels decode_multi (P = -1) and decode_warp (P = -2), compiled
+// for the host under warp_emu.h, over streams read from files.
+// argv: dir P accumulate [grid [mean]]
 // dir holds params.bin (u64 n, d, s, K), out_in.bin (fp32[n]), w<j>.bin / o<j>.bin
 // (words, offsets of stream j); the result goes to out.bin and the status to stdout.
-// For P = 0 the K streams are decoded one launch each, in order.  For P < 0 they
-// go 16 to a launch, as the library sends them; with mean = 1 (decode_multi only)
-// the first launch starts from +0 and the last divides by K.
+// The K streams go 16 to a launch, as the library sends them; with mean = 1
+// (decode_multi only) the first launch starts from +0 and the last divides by K.
 #include "warp_emu.h"
 thread_local dim3e threadIdx, blockIdx;
 dim3e gridDim, blockDim;
@@ -39,28 +38,6 @@ static std::vector<unsigned char> slurp(const std::string& p) {
     if (n && std::fread(b.data(), 1, n, f) != (size_t)n) std::exit(2);
     std::fclose(f);
     return b;
-}
-// decode_fast (one lane per bucket, staged segments).
-template <bool A> void run_kernel(const qsgd::DecodeArgs& a, unsigned grid) {
-    const int kBlock = qsgd::kDecodeBlock;
-    const size_t smem = qsgd::kLut * 4 + (size_t)qsgd::kDecWarps * 32 * qsgd::kStride * 4;
-    gridDim = {grid, 1, 1};
-    blockDim = {(unsigned)kBlock, 1, 1};
-    std::vector<unsigned char> sm(smem + 64);
-    std::vector<WarpSync> warps(kBlock / 32);
-    for (unsigned b = 0; b < grid; ++b) {
-        g_emu_smem = sm.data();
-        std::memset(sm.data(), 0xAB, sm.size());  // garbage, like real shared memory
-        g_warps = warps.data();
-        std::vector<std::thread> th;
-        for (int t = 0; t < kBlock; ++t)
-            th.emplace_back([&, t, b] {
-                threadIdx = {(unsigned)t, 0, 0};
-                blockIdx = {b, 0, 0};
-                qsgd::decode_fast<A>(a);
-            });
-        for (auto& x : th) x.join();
-    }
 }
 template <bool A> static void run_warp(const qsgd::DecodeArgs& a, unsigned grid) {
     const int kBlock = qsgd::kDecodeBlock;
@@ -123,7 +100,8 @@ int main(int argc, char** argv) {
     std::memcpy(out.data(), outb.data(), 4 * n);
     uint32_t status = 0;
     std::vector<std::vector<unsigned char>> ws(K), os(K);
-    if (P < 0) {
+    if (P != -1 && P != -2) return 2;
+    {
         const bool mean = argc > 5 && std::atoi(argv[5]) != 0;
         for (int j = 0; j < K; ++j) {
             ws[j] = slurp(dir + "/w" + std::to_string(j) + ".bin");
@@ -155,24 +133,4 @@ int main(int argc, char** argv) {
         std::printf("status %u\n", status);
         return 0;
     }
-    for (int j = 0; j < K; ++j) {
-        ws[j] = slurp(dir + "/w" + std::to_string(j) + ".bin");
-        os[j] = slurp(dir + "/o" + std::to_string(j) + ".bin");
-        qsgd::DecodeArgs a{};
-        a.n = n; a.d = d; a.s = s; a.nb = (n + d - 1) / d; a.out = out.data(); a.status = &status; a.K = 1;
-        a.first_group = acc ? (j == 0) : 1;
-        a.streams[0].words = reinterpret_cast<const uint32_t*>(ws[j].data());
-        a.streams[0].num_words = ws[j].size() / 4;
-        a.streams[0].offsets = reinterpret_cast<const uint64_t*>(os[j].data());
-        if (acc)
-            run_kernel<true>(a, grid);
-        else
-            run_kernel<false>(a, grid);
-        if (g_emu_error) return 4;
-    }
-    FILE* f = std::fopen((dir + "/out.bin").c_str(), "wb");
-    std::fwrite(out.data(), 4, n, f);
-    std::fclose(f);
-    std::printf("status %u\n", status);
-    return 0;
 }

@@ -1,13 +1,12 @@
 """The decoders' kernel source run on the CPU under a warp emulator (no GPU).
 
-`tests/emu/inc/warp_emu.h` stands in for the CUDA features `decode_fast` (P = 0
-below), `decode_multi` (P = -1) and `decode_warp` (P = -2) use:
-every thread of a block is a host thread, and each warp primitive gathers the 32
-lanes and checks that they call the same primitive at the same source line.  A lane
-that skips a primitive the others wait in (a deadlock on a GPU) fails the test here,
-as does any mismatch with the oracle.  Shared memory starts as garbage, as on the
-device.  The kernel text is taken from `qsgd_decode.cu` as it stands; only the
-launch helpers are cut and the two `cp.async` statements are mapped to copies.
+`tests/emu/inc/warp_emu.h` stands in for the CUDA features `decode_multi` (P = -1
+below) and `decode_warp` (P = -2) use: every thread of a block is a host thread, and
+each warp primitive gathers the 32 lanes and checks that they call the same primitive
+at the same source line.  A lane that skips a primitive the others wait in (a
+deadlock on a GPU) fails the test here, as does any mismatch with the oracle.
+Shared memory starts as garbage, as on the device.  The kernel text is taken from
+`qsgd_decode.cu` as it stands; only the launch helpers are cut.
 
 The streams are made by the oracle; the checks are bit-exact.
 """
@@ -30,16 +29,13 @@ CSRC = os.path.join(ROOT, "quantized_gradient_compression_b200", "csrc")
 def _kernel_source() -> str:
     src = open(os.path.join(CSRC, "qsgd_decode.cu")).read()
     # everything from the first host-side launch helper on is cut
-    cut = src.index("// Dynamic shared memory for a one-wave launch")
+    cut = src.index("cudaError_t launch_multi(const DecodeArgs& a, cudaStream_t stream) {")
     s = src[:cut] + "}  // namespace\n}  // namespace qsgd\n"
     s = s.replace('#include "../../include/qsgd.h"', '#include "%s"' % os.path.join(ROOT, "include", "qsgd.h"))
     s = s.replace('#include "qsgd_internal.h"', '#include "%s"' % os.path.join(CSRC, "qsgd_internal.h"))
     s = s.replace("extern __shared__ __align__(16) uint32_t smem[];",
                   "uint32_t* smem = reinterpret_cast<uint32_t*>(g_emu_smem);")
-    s, copies = re.subn(r'asm volatile\("cp\.async\.cg\.shared\.global \[%0\], \[%1\], 16;\\n" ::"r"\((\w+)\), '
-                        r'"l"\(([^)]*)\)\s*:\s*"memory"\);', r"emu_cp16(\1, \2);", s)
-    s, waits = re.subn(r'asm volatile\("cp\.async\.wait_all;\\n" ::: "memory"\);', ";", s)
-    assert copies >= 1 and waits >= 1 and "asm" not in s
+    assert "asm" not in s
     return s
 
 
@@ -93,16 +89,17 @@ def _run(exe, tmp, oracle_lib, n, d, s, K, P, accumulate, kind, corrupt=False, m
     return got, status, streams, base
 
 
-# (n, d, s, K, P, accumulate, input): P = 0, the one-lane staged decoder
-# (decode_fast): ragged last group, d % 64 != 0, several streams one launch each
+# (n, d, s, K, P, accumulate, input): P = -2, the any-shape decoder (decode_warp),
+# on the shapes the row decoders take on the GPU: ragged last group, d % 64 != 0,
+# several streams in one launch
 CASES = [
-    (30_001, 512, 16, 1, 0, False, "layered"),
-    (30_001, 512, 16, 2, 0, True, "layered"),
-    (20_000, 100, 7, 2, 0, True, "normal"),
-    (9_000, 132, 3, 1, 0, False, "normal"),
-    (20_000, 512, 2, 1, 0, False, "heavy_tailed_sparse"),
-    (9_001, 4096, 1000, 1, 0, False, "normal"),
-    (513, 512, 16, 2, 0, True, "normal"),
+    (30_001, 512, 16, 1, -2, False, "layered"),
+    (30_001, 512, 16, 2, -2, True, "layered"),
+    (20_000, 100, 7, 2, -2, True, "normal"),
+    (9_000, 132, 3, 1, -2, False, "normal"),
+    (20_000, 512, 2, 1, -2, False, "heavy_tailed_sparse"),
+    (9_001, 4096, 1000, 1, -2, False, "normal"),
+    (513, 512, 16, 2, -2, True, "normal"),
 ]
 
 
@@ -125,7 +122,7 @@ def test_staged_decoder_corrupt_streams(emu_exe, tmp_path, oracle_lib, d):
     """Bit flips in some buckets: the kernel finishes (no lane waits alone), flags
     the stream, and every bucket without a flip decodes as the oracle decodes it."""
     n, s = 30_000, 16
-    got, status, streams, _ = _run(emu_exe, tmp_path, oracle_lib, n, d, s, 1, 0, False, "normal", corrupt=True)
+    got, status, streams, _ = _run(emu_exe, tmp_path, oracle_lib, n, d, s, 1, -2, False, "normal", corrupt=True)
     assert status & 2
     words, offsets, _, _ = oracle_lib.encode(W.GENERATORS["normal"](n, 300), d, s, seed=77)
     ref, _ = oracle_lib.decode(words, offsets, n, d, s)

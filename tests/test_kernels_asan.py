@@ -1,11 +1,15 @@
 """The kernels' source under AddressSanitizer on the CPU emulators (no GPU).
 
-- Decoders (decode_fast, decode_multi, decode_warp) on damaged input:
-  random bit flips anywhere (norm fields included), scrambled offsets headers, and
-  word arrays cut short.  They may flag the input, but they must read and write
-  nothing outside their buffers, and must end.
-- Encoders (encode_fast, encode_general) at ragged shapes and special values: every
-  access stays in bounds, and the stream still matches the oracle."""
+- Decoders on damaged input: random bit flips anywhere (norm fields included),
+  scrambled offsets headers, and word arrays cut short -- decode_multi and
+  decode_warp, and the row decoders (decode_rows, decode_rows_ring,
+  decode_rows_multi) with the large-bucket decoder (decode_sparse).  They may flag
+  the input, but they must read and write nothing outside their buffers, and must
+  end.
+- Encoders at ragged shapes and special values -- the one-pass encode_fast and
+  encode_general, and the two-launch encoder (code_buckets_short, code_buckets,
+  compact_stream): every access stays in bounds, and the stream still matches the
+  oracle."""
 
 import os
 import shutil
@@ -55,7 +59,7 @@ def test_decoders_on_damaged_input(dec_asan, tmp_path, oracle_lib):
         d = int(rng.choice([4, 64, 100, 128, 512, 1000, 4096]))
         s = int(rng.choice([1, 3, 16, 100, 1023]))
         K = int(rng.integers(1, 4))
-        P = int(rng.choice([0, -1, -2]))
+        P = int(rng.choice([-1, -2]))
         acc = bool(rng.integers(0, 2)) or P == -1
         t = tmp_path / ("t%d" % trial)
         t.mkdir()
@@ -117,6 +121,83 @@ def test_encoders_stay_in_bounds(enc_asan, tmp_path, oracle_lib, n, d, s, mode, 
         v[1500:1800] = 3e38
     words, offsets, status, _ = E._run(enc_asan, tmp_path, v, d, s, 2, mode, 2)
     own_words, own_offsets, own_norms, own_status = oracle_lib.encode(v, d, s, 2)
+    assert status == own_status
+    gn = stream_norms(words, offsets)
+    check_norms(gn, own_norms)
+    r_words, r_offsets, _, _ = oracle_lib.encode(v, d, s, 2, norms_in=gn)
+    assert np.array_equal(offsets, r_offsets) and np.array_equal(words, r_words)
+
+
+# --- the row decoders, the several-stream tiles and the large-bucket decoder --------
+@pytest.fixture(scope="module")
+def rows_asan(tmp_path_factory):
+    d = tmp_path_factory.mktemp("rowsasan")
+    if not _have_asan(d):
+        pytest.skip("no AddressSanitizer")
+    import test_rows_emulated as R
+
+    return R.build_rows_exe(d / "b", ASAN)
+
+
+def test_row_decoders_on_damaged_input(rows_asan, tmp_path, oracle_lib):
+    """decode_rows (byte codes), decode_rows_ring (16-bit codes), decode_rows_multi
+    (K > 1) and decode_sparse (d > 1024) on bit flips, scrambled offsets and cut word
+    arrays: they may flag the input, but touch nothing outside their buffers."""
+    rng = np.random.default_rng(77)
+    for trial in range(30):
+        n = int(rng.integers(1, 6000))
+        d = int(rng.choice([4, 100, 512, 1000, 1024, 2048, 3001]))
+        s = int(rng.choice([1, 3, 16, 127, 300, 32767]))
+        K = int(rng.integers(1, 4)) if d <= 1024 else int(rng.integers(1, 3))
+        acc = bool(rng.integers(0, 2))
+        t = tmp_path / ("t%d" % trial)
+        t.mkdir()
+        for j in range(K):
+            words, offsets, _, _ = oracle_lib.encode(W.normal(n, trial * 10 + j), d, s, seed=j)
+            mode = rng.integers(0, 4)
+            if mode == 0 and words.size:
+                for pos in rng.integers(0, words.size * 32, size=8):
+                    words[pos >> 5] ^= np.uint32(1) << np.uint32(31 - (pos & 31))
+            elif mode == 1:
+                offsets = offsets.copy()
+                idx = rng.integers(0, offsets.size, size=3)
+                offsets[idx] = rng.integers(0, max(1, int(offsets[-1]) * 2 + 64), size=3).astype(np.uint64)
+            elif mode == 2 and words.size > 2:
+                words = words[: max(1, words.size // 2)]
+            words.astype(np.uint32).tofile(t / ("w%d.bin" % j))
+            offsets.astype(np.uint64).tofile(t / ("o%d.bin" % j))
+        np.zeros(n, np.float32).tofile(t / "out_in.bin")
+        np.array([n, d, s], np.uint64).tofile(t / "params.bin")
+        r = subprocess.run([rows_asan, str(t), "1" if acc else "0", "2", "2", str(K), "0"], capture_output=True,
+                           text=True, timeout=600)
+        assert r.returncode == 0 and "AddressSanitizer" not in r.stderr, (trial, n, d, s, K, r.stderr[-2000:])
+
+
+# --- the two-launch encoder (bucket coders and compaction) ----------------------------
+@pytest.fixture(scope="module")
+def stage_asan(tmp_path_factory):
+    d = tmp_path_factory.mktemp("stageasan")
+    if not _have_asan(d):
+        pytest.skip("no AddressSanitizer")
+    import test_stage_emulated as S
+
+    return S._build(tmp_path_factory, "stageasanb", ASAN)
+
+
+@pytest.mark.parametrize("n,d,s,special", [(5_003, 512, 16, True), (3_001, 128, 40, False), (9_001, 4096, 2, True),
+                                           (2_501, 4, 9, False), (1, 512, 16, False), (20_000, 1000, 31, False)])
+def test_staged_encoder_stays_in_bounds(stage_asan, tmp_path, oracle_lib, n, d, s, special):
+    import test_stage_emulated as S
+
+    v = W.normal(n, 5)
+    if special and n > 1800:
+        v[:300] = 0.0
+        v[400] = np.inf
+        v[900] = np.nan
+        v[1200:1500] = 1e-30
+        v[1500:1800] = 3e38
+    words, offsets, status, _ = S._run(stage_asan, tmp_path, v, d, s, 2, 2)
+    _, _, own_norms, own_status = oracle_lib.encode(v, d, s, 2)
     assert status == own_status
     gn = stream_norms(words, offsets)
     check_norms(gn, own_norms)

@@ -24,11 +24,8 @@ CSRC = os.path.join(ROOT, "quantized_gradient_compression_b200", "csrc")
 EMU = os.path.join(HERE, "emu", "enc")
 
 
-@pytest.fixture(scope="module")
-def rows_exe(tmp_path_factory):
-    if shutil.which("g++") is None:
-        pytest.skip("g++ not available")
-    d = tmp_path_factory.mktemp("rowsemu")
+def build_rows_exe(d, extra=()):
+    """Builds the row decoders' host program in directory d (extra: g++ flags)."""
     src_dir = d / "pkg" / "csrc"
     src_dir.mkdir(parents=True)
     shutil.copytree(os.path.join(ROOT, "include"), d / "include")
@@ -39,10 +36,18 @@ def rows_exe(tmp_path_factory):
     cut = src.index("// One CTA per SM, its warps one group each where the groups allow: every SM busy.")
     (src_dir / "rows_emu.inc").write_text(_host_source(src[:cut]) + "}  // namespace\n}  // namespace qsgd\n")
     exe = d / "rows_main"
-    r = subprocess.run(["g++", "-O1", "-std=c++17", "-ffp-contract=off", "-pthread", "-I", EMU, "-I", str(src_dir),
+    flags = list(extra) or ["-O1"]
+    r = subprocess.run(["g++", *flags, "-std=c++17", "-ffp-contract=off", "-pthread", "-I", EMU, "-I", str(src_dir),
                         os.path.join(EMU, "rows_main.cpp"), "-o", str(exe)], capture_output=True, text=True)
     assert r.returncode == 0, r.stderr[-4000:]
     return str(exe)
+
+
+@pytest.fixture(scope="module")
+def rows_exe(tmp_path_factory):
+    if shutil.which("g++") is None:
+        pytest.skip("g++ not available")
+    return build_rows_exe(tmp_path_factory.mktemp("rowsemu"))
 
 
 def _flip_bits(words, offsets, rng):
