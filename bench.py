@@ -37,14 +37,21 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM traffic per launch of each phase's kernel (dram__bytes_read.sum +
 # dram__bytes_write.sum) from one ncu capture of this workload, with the hash of
 # the kernel sources it was taken on; reported as null once the sources differ.
-TRAFFIC_SOURCES = ("qsgd_decode.cu", "qsgd_device.cuh", "qsgd_encode.cu", "qsgd_limits.h")
+TRAFFIC_SOURCES = ("qsgd_encode_stage.cu", "qsgd_decode_rows.cu", "qsgd_device.cuh", "qsgd_limits.h")
 TRAFFIC = {"bytes_per_launch": {"encode": 106337792, "decode": 51031296, "decode_accumulate": 155691776},
            "sources_sha256": "bdf6cc90cd42717cabba452c2a57cfcd2968e52b3595eea9b8a83c04c9075922"}
 
 
+# The kernels behind each phase of the c2 step (d = 512, s = 16, aligned buffers).
+KERNELS = {"encode": "code_buckets_short<4, false> + compact_stream (qsgd_encode, two launches)",
+           "decode": "decode_rows<4, false> (qsgd_decode)",
+           "decode_accumulate": "decode_rows<4, true> (qsgd_decode_accumulate, K = 1)"}
+
+
 def sources_sha256() -> str:
-    """Hash of the files that hold the device code of the profiled kernels
-    (encode_fast, decode_fast): the traffic figures above are void once it changes."""
+    """Hash of the files that hold the device code of the profiled kernels (the
+    bucket coder, the compaction and the row decoder): the traffic figures above are
+    void once it changes."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "quantized_gradient_compression_b200", "csrc")
     for name in TRAFFIC_SOURCES:
@@ -72,7 +79,56 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5],
                     help="workload: 2 (default, the headline line) or another of the five configs")
+    ap.add_argument("--profile-step", action="store_true",
+                    help="no timing: run the config's step three times (two as warm-up) and exit, for a "
+                         "profiler's capture of the third; c2 / c5 take --s")
+    ap.add_argument("--s", type=int, default=None, help="levels for --profile-step on c2 or c5")
+    ap.add_argument("--bbit", type=int, default=None, choices=[2, 4, 8],
+                    help="--profile-step on c2 with the fixed-width b-bit codec instead")
     return ap.parse_args()
+
+
+def profile_step(args):
+    """Three passes of one config's device work, untimed: c1 / c2 / c3 / c5 (at --s)
+    qsgd_encode, qsgd_decode and qsgd_decode_accumulate (K = 1); c4 the sixteen
+    senders' encodes and the K = 16 qsgd_decode_accumulate; with --bbit, the b-bit
+    encode, decode and decode-accumulate on c2.  Launches per pass: two for each
+    encode on the two-launch shapes, one for each decode."""
+    import torch
+    from quantized_gradient_compression_b200 import binding as B
+    from quantized_gradient_compression_b200 import workloads as W
+
+    cfg = args.config
+    if args.bbit is not None:
+        w = W.C2
+        x = torch.from_numpy(w.generate()).cuda()
+        acc = torch.zeros(w.n, dtype=torch.float32, device="cuda")
+        for _ in range(3):
+            enc = B.bbit_encode(x, w.d, args.bbit, w.seed)
+            B.bbit_decode(enc)
+            B.bbit_decode_accumulate([enc], acc)
+        torch.cuda.synchronize()
+        return
+    if cfg == 4:
+        senders = W.c4_streams()
+        xs = [torch.from_numpy(w.generate()).cuda() for w in senders]
+        acc = torch.zeros(senders[0].n, dtype=torch.float32, device="cuda")
+        for _ in range(3):
+            encs = [B.encode(x, w.d, w.s, w.seed) for x, w in zip(xs, senders)]
+            B.decode_accumulate(encs, acc)
+        torch.cuda.synchronize()
+        return
+    w = {1: W.C1, 2: W.C2, 3: W.C3, 5: W.c5(16)}[cfg]
+    s = args.s if args.s is not None and cfg in (2, 5) else w.s
+    x = torch.from_numpy(w.generate()).cuda()
+    acc = torch.zeros(w.n, dtype=torch.float32, device="cuda")
+    for _ in range(3):
+        enc = B.encode(x, w.d, s, w.seed)
+        out, st = B.decode(enc)
+        B.decode_accumulate([enc], acc)
+    torch.cuda.synchronize()
+    if int(enc.status.item()) != 0 or int(st.item()) != 0:
+        raise RuntimeError("device status %d / %d" % (int(enc.status.item()), int(st.item())))
 
 
 def workload():
@@ -575,9 +631,7 @@ def run_ours(args, w):
         "bits_per_coord": total_bits / n,
         "compressed_bytes": comp_bytes,
         "phases": phases,
-        "roofline": {"bound": "hbm", "kernel": {"encode": "encode_fast<4, true, false> (qsgd_encode)",
-                                                  "decode": "decode_fast<false> (qsgd_decode)",
-                                                  "decode_accumulate": "decode_fast<true> (qsgd_decode_accumulate)"}[dominant],
+        "roofline": {"bound": "hbm", "kernel": KERNELS[dominant],
                      "achieved": dom["algorithmic_gbs"], "peak": peak, "unit": "GB/s",
                      "frac": dom["algorithmic_gbs"] / peak, "traffic": traffic,
                      "peak_source": "%s hbm_gbs (burst copy)" % peak_kind,
@@ -588,7 +642,7 @@ def run_ours(args, w):
                 "ms_per_step": t_e2e,
                 "how": "qsgd_encode/decode/decode_accumulate on host-pinned data; per step H2D of the "
                        "input and D2H of the result, pipelined over copy-in / compute / copy-out streams"},
-        "gpu_launches": 3 * K,
+        "gpu_launches": 4 * K,  # per step: the encoder's coder and compaction, the decode, the accumulate
         "bbit": bbit,
         "qsgdinf": qsgdinf,
         "error_feedback": error_feedback,
@@ -804,6 +858,9 @@ def run_config(args, cfg: int):
 def main():
     args = parse_args()
     w = workload()
+    if args.profile_step:
+        profile_step(args)
+        return
     if args.impl == "reference":
         if args.config != 2:
             w = config_workloads(args.config)[2 if args.config == 5 else 0]

@@ -811,56 +811,59 @@ __global__ void __launch_bounds__(kCompactThreads, 2) compact_stream(const __gri
     const uint32_t G = mean_words < 8u ? 8u : mean_words < 16u ? 16u : 32u;
     const uint32_t per_warp = 32u / G, sub = static_cast<uint32_t>(lane) / G, sl = static_cast<uint32_t>(lane) % G;
     const uint32_t step = kWarps * per_warp;
-    // four buckets at a time, so that their loads are in flight together
-    constexpr int kU = 4;
+    // four buckets at a time and two words a lane of each, all loaded before any is
+    // stored, so that their loads are in flight together
+    constexpr int kU = 4, kC = 2;
     for (uint32_t i0 = static_cast<uint32_t>(warp) * per_warp + sub; i0 < nt; i0 += kU * step) {
-        uint32_t cnt[kU], delta[kU], nw[kU], Lb[kU];
-        uint64_t wf[kU];
-        const uint32_t* src[kU];
-        uint32_t hd[kU];
+        uint32_t Lb[kU], hd[kU];
+        uint64_t F[kU];
 #pragma unroll
         for (int u = 0; u < kU; ++u) {
             const uint32_t i = i0 + static_cast<uint32_t>(u) * step;
-            cnt[u] = 0u;
-            delta[u] = nw[u] = Lb[u] = hd[u] = 0u;
-            wf[u] = 0u;
-            src[u] = a.stage;
+            Lb[u] = hd[u] = 0u;
+            F[u] = 0u;
             if (i < nt) {
-                const uint64_t bb = b0 + i;
                 Lb[u] = s_L[i];
-                const uint64_t F = X + s_R[i];
-                wf[u] = (F + 31u) >> 5;
-                cnt[u] = static_cast<uint32_t>(((F + Lb[u] + 31u) >> 5) - wf[u]);
-                delta[u] = static_cast<uint32_t>((wf[u] << 5) - F);
-                nw[u] = (Lb[u] + 31u) >> 5;
-                src[u] = a.stage + bb * a.slot_words;
+                F[u] = X + s_R[i];
                 // the next bucket's first word, for the word that runs past this one's end
-                if (bb + 1 < a.nb) hd[u] = a.stage[(bb + 1) * a.slot_words];
+                if (b0 + i + 1 < a.nb) hd[u] = a.stage[(b0 + i + 1) * a.slot_words];
             }
         }
-        for (uint32_t k = sl;; k += G) {
-            uint32_t v[kU];
+        for (uint32_t kb = sl;; kb += kC * G) {
+            uint32_t a0[kU][kC], a1[kU][kC];
             bool more = false;
 #pragma unroll
             for (int u = 0; u < kU; ++u) {
-                v[u] = 0u;
-                if (k < cnt[u]) {
-                    const uint32_t r = delta[u] + 32u * k;  // bucket-relative bit of the word (< Lb)
-                    const uint32_t a0 = src[u][k];
-                    const uint32_t a1 = k + 1 < nw[u] ? src[u][k + 1] : 0u;
-                    v[u] = __funnelshift_l(a1, a0, delta[u]);
-                    if (r + 32u > Lb[u]) v[u] |= hd[u] >> (Lb[u] - r);  // 1 <= Lb - r <= 31
+                const uint64_t wf = (F[u] + 31u) >> 5;
+                const uint32_t cnt = static_cast<uint32_t>(((F[u] + Lb[u] + 31u) >> 5) - wf);
+                const uint32_t nw = (Lb[u] + 31u) >> 5;
+                const uint32_t* src = a.stage + (b0 + i0 + static_cast<uint32_t>(u) * step) * a.slot_words;
+#pragma unroll
+                for (int c = 0; c < kC; ++c) {
+                    const uint32_t k = kb + static_cast<uint32_t>(c) * G;
+                    a0[u][c] = k < cnt ? src[k] : 0u;
+                    a1[u][c] = k + 1 < nw && k < cnt ? src[k + 1] : 0u;
                 }
-                more = more || k + G < cnt[u];
+                more = more || kb + kC * G < cnt;
             }
 #pragma unroll
             for (int u = 0; u < kU; ++u) {
-                if (k < cnt[u]) {
-                    const uint64_t w = wf[u] + k;
-                    if (w < a.cap_words)
-                        a.words[w] = v[u];
-                    else
-                        report(a.status, QSGD_ST_OVERFLOW);
+                const uint64_t wf = (F[u] + 31u) >> 5;
+                const uint32_t cnt = static_cast<uint32_t>(((F[u] + Lb[u] + 31u) >> 5) - wf);
+                const uint32_t delta = static_cast<uint32_t>((wf << 5) - F[u]);
+#pragma unroll
+                for (int c = 0; c < kC; ++c) {
+                    const uint32_t k = kb + static_cast<uint32_t>(c) * G;
+                    if (k < cnt) {
+                        const uint32_t r = delta + 32u * k;  // bucket-relative bit of the word (< Lb)
+                        uint32_t v = __funnelshift_l(a1[u][c], a0[u][c], delta);
+                        if (r + 32u > Lb[u]) v |= hd[u] >> (Lb[u] - r);  // 1 <= Lb - r <= 31
+                        const uint64_t w = wf + k;
+                        if (w < a.cap_words)
+                            a.words[w] = v;
+                        else
+                            report(a.status, QSGD_ST_OVERFLOW);
+                    }
                 }
             }
             if (!more) break;
