@@ -34,12 +34,14 @@ sys.path.insert(0, ROOT)
 METRIC = "QSGD encode & decode GB/s of fp32 gradient input; % of B200 HBM roofline"
 FALLBACK_HBM_GBS = 6650.0
 
-# DRAM traffic per launch of each phase's kernel (dram__bytes_read.sum +
-# dram__bytes_write.sum) from one ncu capture of this workload, with the hash of
-# the kernel sources it was taken on; reported as null once the sources differ.
+# DRAM traffic per call of each phase (dram__bytes_read.sum + dram__bytes_write.sum,
+# summed over the call's launches: the encode's coder and compaction) from one ncu
+# capture of this workload (ncu --set full over bench.py --profile-step), with the
+# hash of the kernel sources it was taken on; reported as null once the sources
+# differ.
 TRAFFIC_SOURCES = ("qsgd_encode_stage.cu", "qsgd_decode_rows.cu", "qsgd_device.cuh", "qsgd_limits.h")
-TRAFFIC = {"bytes_per_launch": {"encode": 106337792, "decode": 51031296, "decode_accumulate": 155691776},
-           "sources_sha256": "bdf6cc90cd42717cabba452c2a57cfcd2968e52b3595eea9b8a83c04c9075922"}
+TRAFFIC = {"bytes_per_launch": {"encode": 122624768, "decode": 50971392, "decode_accumulate": 153777664},
+           "sources_sha256": "0cfc6eb06a5d22ac8b8ca8238c2e6a8ebe89140fdfecddeee4c8134be8c1d9c0"}
 
 
 # The kernels behind each phase of the c2 step (d = 512, s = 16, aligned buffers).
