@@ -384,6 +384,18 @@ __global__ void __launch_bounds__(kStageBlock, (V <= 4 ? 4 : 2)) code_buckets_sh
         uint32_t pos = 32u;
         if (m <= kChunkCoords) {
             // --- one chunk: the values stay in registers ---------------------------------
+#ifndef QSGD_STAGE_PREFETCH
+#define QSGD_STAGE_PREFETCH 0
+#endif
+            if (QSGD_STAGE_PREFETCH && b + gwarps < a.nb) {  // the warp's next bucket into L2
+                const uint64_t nbase = (b + gwarps) * d;
+                const uint64_t nend = min(a.n, nbase + d);
+                const uint64_t line = (nbase * 4u & ~uint64_t(127)) + 128u * static_cast<uint32_t>(lane);
+                if (line < nend * 4u) {
+                    const char* pf = reinterpret_cast<const char*>(a.in) + line;
+                    asm volatile("prefetch.global.L2 [%0];" ::"l"(pf));
+                }
+            }
             load_contig<V>(a.in + base, ql, m, x);
             if constexpr (kEF) {  // p = e + g
                 load_contig<V>(a.ef + base, ql, m, ev);
@@ -696,9 +708,12 @@ __device__ __forceinline__ void release_control(ScanControl* ctrl) {
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kCompactThreads, 2) compact_stream(const __grid_constant__ StageArgs a) {
     constexpr int kWarps = kCompactThreads / 32;
+    extern __shared__ __align__(16) uint32_t smem[];  // the tile's staged words (gather)
     __shared__ uint32_t s_R[kCompactBlock];
     __shared__ uint32_t s_L[kCompactBlock];
+    __shared__ uint32_t s_RW[kCompactBlock + 1];
     __shared__ uint32_t s_warp[kWarps];
+    __shared__ uint32_t s_wwarp[kWarps];
     __shared__ uint32_t s_tile;
     __shared__ uint64_t s_X;
     __shared__ int s_ok;
@@ -729,6 +744,44 @@ __global__ void __launch_bounds__(kCompactThreads, 2) compact_stream(const __gri
     }
     const uint32_t excl = before + incl - L;
     if (tid == 0) st_release(&a.cdesc[tile], make_desc(0, tile == 0 ? kStatePrefix : kStateAggregate, total));
+    // the staged words of each bucket: a scan of their counts places them in shared
+    // memory, where they are gathered (cp.async) while the look-back runs
+    const uint32_t NW = (L + 31u) >> 5;
+    uint32_t wincl = NW;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t t = __shfl_up_sync(kAll, wincl, o);
+        if (lane >= o) wincl += t;
+    }
+    if (lane == 31) s_wwarp[warp] = wincl;
+    if (tid < kCompactBlock) {
+        s_R[tid] = excl;  // tile-relative start of each bucket
+        s_L[tid] = L;
+    }
+    __syncthreads();
+    uint32_t wbefore = 0, wtotal = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+        const uint32_t x = s_wwarp[w];
+        wbefore += w < warp ? x : 0u;
+        wtotal += x;
+    }
+    if (tid <= kCompactBlock) s_RW[tid] = wbefore + wincl - NW;  // s_RW[kCompactBlock] = wtotal
+    const bool gather = wtotal <= kCompactSmemWords;
+    const uint32_t nt = static_cast<uint32_t>(min(static_cast<uint64_t>(kCompactBlock), a.nb - b0));
+    __syncthreads();
+    if (gather) {
+        for (uint32_t i = warp; i < nt; i += kWarps) {
+            const uint32_t nw = (s_L[i] + 31u) >> 5, rw = s_RW[i];
+            const uint32_t* src0 = a.stage + (b0 + i) * a.slot_words;
+            for (uint32_t k = lane; k < nw; k += 32) {
+                const uint32_t saddr = static_cast<uint32_t>(__cvta_generic_to_shared(smem + rw + k));
+                const uint32_t* src = src0 + k;
+                asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(saddr), "l"(src) : "memory");
+            }
+        }
+        asm volatile("cp.async.commit_group;\n" ::: "memory");
+    }
     // look-back by the whole CTA: thread i reads the descriptor of tile (window end -
     // i), so one read covers kCompactThreads predecessors; the nearest one holding its
     // inclusive prefix ends the walk, and every tile between must have published its
@@ -788,29 +841,57 @@ __global__ void __launch_bounds__(kCompactThreads, 2) compact_stream(const __gri
     }
     __syncthreads();
     if (!s_ok) {
+        if (gather) asm volatile("cp.async.wait_all;\n" ::: "memory");  // no copy outlives the CTA
         release_control(a.ctrl);
         return;
     }
     const uint64_t X = s_X;
     if (tid < kCompactBlock) {
         const uint64_t F = X + excl;
-        s_R[tid] = excl;  // tile-relative start of each bucket
-        s_L[tid] = L;
         if (b < a.nb) a.offsets[b] = F;
         if (b + 1 == a.nb) a.offsets[a.nb] = F + L;
     }
-    __syncthreads();
+    if (gather) {
+        asm volatile("cp.async.wait_all;\n" ::: "memory");
+        __syncthreads();
+    }
     // G lanes per bucket (G = 8, 16 or 32, from the tile's mean bucket size), over the
     // output words whose first bit lies in the bucket: word k is bits [delta + 32 k,
     // + 32) of the bucket's staged bits, delta the distance from the bucket's start to
     // the next word boundary; a word that runs past the bucket's end takes the first
     // bits of the next bucket (always >= 32 bits, so one word of it suffices).  Every
     // output word has exactly one writer.
-    const uint32_t nt = static_cast<uint32_t>(min(static_cast<uint64_t>(kCompactBlock), a.nb - b0));
     const uint32_t mean_words = total / (32u * nt);
     const uint32_t G = mean_words < 8u ? 8u : mean_words < 16u ? 16u : 32u;
     const uint32_t per_warp = 32u / G, sub = static_cast<uint32_t>(lane) / G, sl = static_cast<uint32_t>(lane) % G;
     const uint32_t step = kWarps * per_warp;
+    if (gather) {  // the words are in shared memory
+        for (uint32_t i = static_cast<uint32_t>(warp) * per_warp + sub; i < nt; i += step) {
+            const uint32_t Lb = s_L[i], rw = s_RW[i];
+            const uint64_t F = X + s_R[i];
+            const uint64_t wf = (F + 31u) >> 5;
+            const uint32_t cnt = static_cast<uint32_t>(((F + Lb + 31u) >> 5) - wf);
+            const uint32_t delta = static_cast<uint32_t>((wf << 5) - F);
+            const uint32_t nw = (Lb + 31u) >> 5;
+            // the next bucket's first word, for the word that runs past this one's end
+            const uint32_t hd = i + 1 < nt ? smem[s_RW[i + 1]]
+                                : b0 + i + 1 < a.nb ? a.stage[(b0 + i + 1) * a.slot_words] : 0u;
+            for (uint32_t k = sl; k < cnt; k += G) {
+                const uint32_t r = delta + 32u * k;  // bucket-relative bit of the word (< Lb)
+                const uint32_t a0 = smem[rw + k];
+                const uint32_t a1 = k + 1 < nw ? smem[rw + k + 1] : 0u;
+                uint32_t v = __funnelshift_l(a1, a0, delta);
+                if (r + 32u > Lb) v |= hd >> (Lb - r);  // 1 <= Lb - r <= 31
+                const uint64_t w = wf + k;
+                if (w < a.cap_words)
+                    a.words[w] = v;
+                else
+                    report(a.status, QSGD_ST_OVERFLOW);
+            }
+        }
+        release_control(a.ctrl);
+        return;
+    }
     // four buckets at a time and two words a lane of each, all loaded before any is
     // stored, so that their loads are in flight together
     constexpr int kU = 4, kC = 2;
@@ -920,7 +1001,15 @@ cudaError_t launch_encode_stage(const StageArgs& a, cudaStream_t stream) {
         default: e = launch_code_v<8>(a, stream); break;
     }
     if (e != cudaSuccess) return e;
-    compact_stream<<<static_cast<unsigned>(a.ntiles), kCompactThreads, 0, stream>>>(a);
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr_set[dev]) {
+        cudaFuncSetAttribute(compact_stream, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kCompactSmemWords * sizeof(uint32_t)));
+        attr_set[dev] = true;
+    }
+    compact_stream<<<static_cast<unsigned>(a.ntiles), kCompactThreads, kCompactSmemWords * sizeof(uint32_t), stream>>>(a);
     return cudaGetLastError();
 }
 

@@ -55,6 +55,13 @@ constexpr int kStageBlock = 32 * kStageWarps;
 #endif
 constexpr int kCompactBlock = QSGD_COMPACT_BLOCK;
 constexpr int kCompactThreads = 2 * kCompactBlock;
+// A tile whose staged words fit in this many words of shared memory is gathered
+// there while the compaction's look-back runs; a larger one is read from the
+// staging slots directly.
+#ifndef QSGD_COMPACT_SMEM_WORDS
+#define QSGD_COMPACT_SMEM_WORDS 16384
+#endif
+constexpr uint32_t kCompactSmemWords = QSGD_COMPACT_SMEM_WORDS;
 constexpr uint32_t kStageMinD = 4;
 constexpr uint32_t kStageMaxD = 1024;        // s > 31: one chunk of 128V coordinates per bucket
 constexpr uint32_t kStageShortMaxD = 16384;  // s <= 31: buckets of several 512-coordinate chunks

@@ -168,6 +168,7 @@ inline void emu_cp16z(uint32_t dst, const void* src, uint32_t src_bytes) {
     std::memcpy(emu_smem() + dst, src, src_bytes);
 }
 inline void emu_cp16(uint32_t dst, const void* src) { emu_cp16z(dst, src, 16); }
+inline void emu_cp4(uint32_t dst, const void* src) { std::memcpy(emu_smem() + dst, src, 4); }
 
 // op: 0 any, 1 ballot, 4 shfl_up, 5 shfl idx, 6 syncwarp, 7 shfl_xor
 inline uint64_t emu_warp(int op, int line, uint64_t v, int arg, int width) {

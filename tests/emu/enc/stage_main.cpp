@@ -140,7 +140,7 @@ int main(int argc, char** argv) {
     const unsigned grid = (unsigned)std::max<uint64_t>(1, std::min<uint64_t>((nb + qsgd::kStageWarps - 1) / qsgd::kStageWarps, grid_req));
     if (ef) code_any<true>(a, grid, smem); else code_any<false>(a, grid, smem);
     if (g_emu_error) return 4;
-    run_grid((unsigned)ntiles, qsgd::kCompactThreads, 0, [&] { qsgd::compact_stream(a); });
+    run_grid((unsigned)ntiles, qsgd::kCompactThreads, qsgd::kCompactSmemWords * 4, [&] { qsgd::compact_stream(a); });
     if (g_emu_error) return 4;
     spit(dir + "/words.bin", words.data(), 4 * cap);
     spit(dir + "/offsets.bin", offsets.data(), 8 * (nb + 1));

@@ -13,6 +13,8 @@ def host_source(text: str) -> str:
          r"emu_cp16(\1, \2);"),
         (r'asm volatile\("cp\.async\.cg\.shared\.global \[%0\], \[%1\], 16, %2;\\n" ::"r"\((\w+)\), "l"\((\w+)\), '
          r'"r"\((\w+)\)\s*:\s*"memory"\);', r"emu_cp16z(\1, \2, \3);"),
+        (r'asm volatile\("cp\.async\.ca\.shared\.global \[%0\], \[%1\], 4;\\n" ::"r"\((\w+)\), "l"\((\w+)\)\s*:\s*"memory"\);',
+         r"emu_cp4(\1, \2);"),
         (r'asm volatile\("cp\.async\.commit_group;\\n" ::: "memory"\);', ";"),
         (r'asm volatile\("cp\.async\.wait_all;\\n" ::: "memory"\);', ";"),
         (r'asm volatile\("st\.release\.gpu\.global\.u64 \[%0\], %1;" ::"l"\(p\), "l"\(v\) : "memory"\);',

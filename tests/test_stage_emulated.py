@@ -53,6 +53,13 @@ def stage_exe(tmp_path_factory):
 
 
 @pytest.fixture(scope="module")
+def stage_exe_direct(tmp_path_factory):
+    # a shared-memory gather of 64 words: nearly every tile reads the staging slots
+    # directly, the path of tiles too large to gather
+    return _build(tmp_path_factory, "stageemudirect", ["-DQSGD_COMPACT_SMEM_WORDS=64"])
+
+
+@pytest.fixture(scope="module")
 def stage_exe_small_tiles(tmp_path_factory):
     # compaction tiles of 32 buckets, so that the look-back walks several windows
     return _build(tmp_path_factory, "stageemu32", ["-DQSGD_COMPACT_BLOCK=32"])
@@ -116,6 +123,20 @@ def test_stage_encoder_matches_oracle(stage_exe, tmp_path, oracle_lib, n, d, s, 
     assert np.array_equal(words, r_words)
 
 
+@pytest.mark.parametrize("n,d,s,grid,kind", CASES[:6], ids=["n%d-d%d-s%d-g%d-%s" % c for c in CASES[:6]])
+def test_stage_encoder_direct_copy_matches_oracle(stage_exe_direct, tmp_path, oracle_lib, n, d, s, grid, kind):
+    """The compaction's copy from the staging slots (tiles too large for its
+    shared-memory gather)."""
+    v = W.GENERATORS[kind](n, n % 97)
+    words, offsets, status, _ = _run(stage_exe_direct, tmp_path, v, d, s, 5, grid)
+    _, _, own_norms, own_status = oracle_lib.encode(v, d, s, 5)
+    assert status == own_status
+    gn = stream_norms(words, offsets)
+    check_norms(gn, own_norms)
+    r_words, r_offsets, _, _ = oracle_lib.encode(v, d, s, 5, norms_in=gn)
+    assert np.array_equal(offsets, r_offsets) and np.array_equal(words, r_words)
+
+
 @pytest.mark.parametrize("d,s", [(512, 16), (128, 3), (256, 100), (4096, 8)])
 def test_stage_encoder_max_norm_matches_oracle(stage_exe, tmp_path, oracle_lib, d, s):
     v = W.layered(20_000, 4)
@@ -177,8 +198,9 @@ def test_stage_lane_strings_past_96_bits(stage_exe, tmp_path, oracle_lib):
 
 @pytest.mark.parametrize("n,d,s", [(12_000, 4, 3), (40_003, 128, 16)])
 def test_stage_lookback_over_several_windows(stage_exe_small_tiles, tmp_path, oracle_lib, n, d, s):
-    """Compaction tiles of 32 buckets: 94 and 10 tiles, so a tile's look-back reads
-    up to three windows of predecessors before it meets a prefix."""
+    """Compaction tiles of 32 buckets (CTAs of 64 threads): 94 and 10 tiles, so a
+    tile's look-back reads up to two windows of 64 predecessors before it meets a
+    prefix."""
     v = W.layered(n, 5)
     words, offsets, status, _ = _run(stage_exe_small_tiles, tmp_path, v, d, s, 4, 2)
     _, _, own_norms, own_status = oracle_lib.encode(v, d, s, 4)
