@@ -76,12 +76,10 @@ StageLayout stage_layout(uint64_t n, uint32_t d, uint32_t s) {
     const uint64_t slot_bits = 32u + static_cast<uint64_t>(d) * (2u + omega_len_host(s));
     L.slot_words = static_cast<uint32_t>(ceil_div(slot_bits, 32));
     L.ntiles = ceil_div(nb, kCompactBlock);
-    L.bits_off = 256;
+    L.desc_off = 256;
+    L.bits_off = L.desc_off + align256(sizeof(uint64_t) * L.ntiles);
     L.stage_off = L.bits_off + align256(sizeof(uint32_t) * nb);
-    const size_t stage_end = L.stage_off + align256(sizeof(uint32_t) * nb * L.slot_words);
-    L.desc_off = align256(std::max(stage_end, workspace_layout(n, d).total));
-    L.acc_off = L.desc_off + align256(sizeof(uint64_t) * L.ntiles);
-    L.total = L.acc_off + align256(sizeof(uint64_t) * L.ntiles);
+    L.total = L.stage_off + align256(sizeof(uint32_t) * nb * L.slot_words);
     return L;
 }
 
@@ -224,7 +222,6 @@ static StageArgs stage_args(const EncodeArgs& e, float* d_ef, uint64_t seed, voi
     a.offsets = e.offsets;
     a.ctrl = reinterpret_cast<ScanControl*>(ws);
     a.cdesc = reinterpret_cast<uint64_t*>(ws + L.desc_off);
-    a.cacc = reinterpret_cast<unsigned long long*>(ws + L.acc_off);
     a.ntiles = L.ntiles;
     return a;
 }

@@ -231,11 +231,6 @@ __device__ __forceinline__ void load_row(const DecodeArgs& a, uint64_t bb, int l
     }
 }
 
-#ifndef QSGD_ROWS_AHEAD
-#define QSGD_ROWS_AHEAD 1
-#endif
-constexpr int kRowsAhead = QSGD_ROWS_AHEAD;  // output rows in flight ahead (decode-accumulate)
-
 template <int V, bool kAcc>
 __global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows(const __grid_constant__ DecodeArgs a,
                                                                    uint32_t stride_w) {
@@ -356,60 +351,53 @@ __global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows(const __grid_c
         if (live && !bad && (next > m || r.left != 0)) bad = true;
         __syncwarp();
         // --- write the rows back: row rr is bucket g*32 + rr -----------------------
-        // (decode-accumulate keeps the output of kRowsAhead rows ahead in flight: a
-        // ring of kS = kRowsAhead + 1 slots, row rr in slot rr mod kS)
+        // (decode-accumulate reads the next row's output before it stores this row's,
+        // so that two rows of loads are in flight)
         const int nrows = static_cast<int>(min(static_cast<uint64_t>(32), a.nb - g * 32));
-        constexpr int kS = kAcc ? (V <= 4 ? kRowsAhead : 1) + 1 : 1;
-        float4 ring[kS][kAcc ? V : 1];
-        if constexpr (kAcc) {
+        float4 cur[kAcc ? V : 1], nxt[kAcc ? V : 1];
+        if constexpr (kAcc) load_row<V>(a, g * 32, lane, cur);
+        for (int rr = 0; rr < nrows; ++rr) {
+            const uint64_t bb = g * 32 + rr;
+            const float sc = __shfl_sync(kWarpAll, scale, rr);
+            if constexpr (kAcc) {
+                if (rr + 1 < nrows) load_row<V>(a, bb + 1, lane, nxt);
+            }
+            const uint32_t mm = static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - bb * d));
+            const uint32_t* rowp = rows + static_cast<uint32_t>(rr) * stride_w;
+            float* gp = a.out + bb * d;
 #pragma unroll
-            for (int t = 0; t + 1 < kS; ++t)
-                if (t < nrows) load_row<V>(a, g * 32 + t, lane, ring[t]);
-        }
-        for (int r0 = 0; r0 < nrows; r0 += kS) {
+            for (int i = 0; i < V; ++i) {
+                const uint32_t q = static_cast<uint32_t>(lane) + 32u * i;
+                const uint32_t c = 4u * q;
+                if (c < mm) {
+                    uint32_t code[4];
+                    const uint32_t w = rowp[q];
 #pragma unroll
-            for (int t = 0; t < kS; ++t) {
-                const int rr = r0 + t;
-                if (rr >= nrows) break;
-                const uint64_t bb = g * 32 + rr;
-                const float sc = __shfl_sync(kWarpAll, scale, rr);
-                if constexpr (kAcc) {
-                    if (rr + kS - 1 < nrows) load_row<V>(a, bb + kS - 1, lane, ring[(t + kS - 1) % kS]);
-                }
-                const uint32_t mm = static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - bb * d));
-                const uint32_t* rowp = rows + static_cast<uint32_t>(rr) * stride_w;
-                float* gp = a.out + bb * d;
+                    for (int j = 0; j < 4; ++j) code[j] = ((w >> (8 * j)) & 0x7Fu) | (((w >> (8 * j)) & 0x80u) << 24);
+                    float v[4];
 #pragma unroll
-                for (int i = 0; i < V; ++i) {
-                    const uint32_t q = static_cast<uint32_t>(lane) + 32u * i;
-                    const uint32_t c = 4u * q;
-                    if (c < mm) {
-                        uint32_t code[4];
-                        const uint32_t w = rowp[q];
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) code[j] = ((w >> (8 * j)) & 0x7Fu) | (((w >> (8 * j)) & 0x80u) << 24);
-                        float v[4];
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            // code[j] = k | sign << 31: k as fp32 through the 2^23 offset
-                            // (exact for k < 2^23), times the step, the sign last
-                            const float kf = __fsub_rn(__uint_as_float(0x4B000000u | (code[j] & 0x7FFFFFFFu)), 8388608.0f);
-                            v[j] = __uint_as_float(__float_as_uint(__fmul_rn(sc, kf)) | (code[j] & 0x80000000u));
-                        }
-                        if constexpr (kAcc) {
-                            const float4& x = ring[t][i];
-                            v[0] = __fadd_rn(x.x, v[0]);
-                            v[1] = __fadd_rn(x.y, v[1]);
-                            v[2] = __fadd_rn(x.z, v[2]);
-                            v[3] = __fadd_rn(x.w, v[3]);
-                        }
-                        if (c + 4 <= mm) {
-                            __stcs(reinterpret_cast<float4*>(gp + c), make_float4(v[0], v[1], v[2], v[3]));
-                        } else {
-                            for (uint32_t j = 0; j < 4 && c + j < mm; ++j) gp[c + j] = v[j];
-                        }
+                    for (int j = 0; j < 4; ++j) {
+                        // code[j] = k | sign << 31: k as fp32 through the 2^23 offset (exact
+                        // for k < 2^23), times the step, the sign last
+                        const float kf = __fsub_rn(__uint_as_float(0x4B000000u | (code[j] & 0x7FFFFFFFu)), 8388608.0f);
+                        v[j] = __uint_as_float(__float_as_uint(__fmul_rn(sc, kf)) | (code[j] & 0x80000000u));
+                    }
+                    if constexpr (kAcc) {
+                        v[0] = __fadd_rn(cur[i].x, v[0]);
+                        v[1] = __fadd_rn(cur[i].y, v[1]);
+                        v[2] = __fadd_rn(cur[i].z, v[2]);
+                        v[3] = __fadd_rn(cur[i].w, v[3]);
+                    }
+                    if (c + 4 <= mm) {
+                        __stcs(reinterpret_cast<float4*>(gp + c), make_float4(v[0], v[1], v[2], v[3]));
+                    } else {
+                        for (uint32_t j = 0; j < 4 && c + j < mm; ++j) gp[c + j] = v[j];
                     }
                 }
+            }
+            if constexpr (kAcc) {
+#pragma unroll
+                for (int i = 0; i < V; ++i) cur[i] = nxt[i];
             }
         }
         if (bad) atomicOr(a.status, QSGD_ST_BAD_STREAM);

@@ -13,12 +13,9 @@
 //    bucket's bits (norm, then the records in index order) into the bucket's own
 //    slot of a staging area in the workspace, at bucket-local bit offsets, together
 //    with the bucket's bit count.  A slot holds the bucket's largest possible size.
-//    The warp also adds the count to its tile's accumulator, and the warp that codes
-//    a tile's last bucket publishes the tile's total.
 // 2. compact_stream: a CTA of 512 threads per tile of 256 buckets scans the bit
-//    counts (a block scan, and a decoupled look-back over the tiles' published
-//    totals, Merrill & Garland 2016, reading 512 predecessors at a time, that never
-//    waits for another CTA), writes the offsets header,
+//    counts (a block scan and a decoupled look-back over the tiles, Merrill &
+//    Garland 2016, reading 512 predecessors at a time), writes the offsets header,
 //    and moves every bucket's bits to their stream position with funnel shifts, 8 to
 //    32 lanes per bucket.  An output word belongs to the bucket that holds its first
 //    bit; that bucket's warp also reads the first bits of the next bucket, so every
@@ -186,18 +183,6 @@ __device__ __forceinline__ void store_contig(float* p, uint32_t q0, uint32_t m, 
             if (i + 2 < m) __stcs(p + i + 2, v[4 * j + 2]);
         }
     }
-}
-
-// A coded bucket's bit count into its tile's accumulator (buckets << 40 | bits); the
-// warp that codes a tile's last bucket publishes the tile's total as the compaction's
-// look-back descriptor (tile 0's as its inclusive prefix), so that no compaction CTA
-// waits for another's scan.
-__device__ __forceinline__ void tile_add(const StageArgs& a, uint64_t b, uint32_t bits) {
-    const uint64_t t = b / kCompactBlock;
-    const uint64_t tn = min(static_cast<uint64_t>(kCompactBlock), a.nb - t * kCompactBlock);
-    const unsigned long long old = atomicAdd(&a.cacc[t], (1ull << 40) | bits);
-    if ((old >> 40) + 1 == tn)
-        st_release(&a.cdesc[t], make_desc(0, t == 0 ? kStatePrefix : kStateAggregate, (old & ((1ull << 40) - 1)) + bits));
 }
 
 // ---------------------------------------------------------------------------
@@ -381,6 +366,10 @@ __global__ void __launch_bounds__(kStageBlock, (V <= 4 ? 4 : 2)) code_buckets_sh
         for (int i = tid; i < kRecordTab64 / 4; i += kStageBlock) reinterpret_cast<uint4*>(rtab)[i] = src[i];
     }
     for (uint32_t i = lane; i < a.buf_words; i += 32) buf[i] = 0u;
+    {  // the compaction's scan state for this call: cleared here, before it runs
+        const uint64_t gt = static_cast<uint64_t>(blockIdx.x) * kStageBlock + tid;
+        for (uint64_t i = gt; i < a.ntiles; i += static_cast<uint64_t>(gridDim.x) * kStageBlock) a.cdesc[i] = 0;
+    }
     __syncthreads();
 
     const uint32_t d = a.d;
@@ -504,10 +493,7 @@ __global__ void __launch_bounds__(kStageBlock, (V <= 4 ? 4 : 2)) code_buckets_sh
             slot[i] = buf[i];
             buf[i] = 0u;
         }
-        if (lane == 0) {
-            a.bits[b] = total;
-            tile_add(a, b, total);
-        }
+        if (lane == 0) a.bits[b] = total;
         __syncwarp();
     }
 }
@@ -531,6 +517,11 @@ __global__ void __launch_bounds__(kStageBlock) code_buckets(const __grid_constan
         for (int i = tid; i < kRecordTab64 / 4; i += kStageBlock) reinterpret_cast<uint4*>(rtab)[i] = src[i];
     }
     for (uint32_t i = lane; i < a.buf_words; i += 32) buf[i] = 0u;
+    // the compaction's scan state for this call: cleared here, before it runs
+    {
+        const uint64_t gt = static_cast<uint64_t>(blockIdx.x) * kStageBlock + tid;
+        for (uint64_t i = gt; i < a.ntiles; i += static_cast<uint64_t>(gridDim.x) * kStageBlock) a.cdesc[i] = 0;
+    }
     __syncthreads();
 
     const uint32_t d = a.d;
@@ -692,37 +683,22 @@ __global__ void __launch_bounds__(kStageBlock) code_buckets(const __grid_constan
             slot[i] = buf[i];
             buf[i] = 0u;
         }
-        if (lane == 0) {
-            a.bits[b] = pos;
-            tile_add(a, b, pos);
-        }
+        if (lane == 0) a.bits[b] = pos;
         __syncwarp();
     }
 }
 
-// The end of a compaction CTA (every thread calls it).  The last CTA out returns the
-// workspace to its resting state for the next call of any encoder: the descriptors
-// and tile accumulators zero, the control block's ticket and completion count zero,
-// no abort.
-__device__ __forceinline__ void finish_compaction(const StageArgs& a, uint32_t& s_last) {
-    __syncthreads();  // every thread of the CTA is past its use of the scan state
+// The last compaction CTA out returns the control block to its resting state (ticket
+// and completion count zero, no abort), which every encoder of the library expects
+// at the start of a call on this workspace.
+__device__ __forceinline__ void release_control(ScanControl* ctrl) {
     if (threadIdx.x == 0) {
         __threadfence();
-        s_last = atomicAdd(&a.ctrl->done, 1u) == gridDim.x - 1 ? 1u : 0u;
-    }
-    __syncthreads();
-    if (s_last) {
-        __threadfence();
-        for (uint64_t i = threadIdx.x; i < a.ntiles; i += blockDim.x) {
-            a.cdesc[i] = 0;
-            a.cacc[i] = 0;
-        }
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            a.ctrl->ticket = 0;
-            a.ctrl->abort = 0;
+        if (atomicAdd(&ctrl->done, 1u) == gridDim.x - 1) {
+            ctrl->ticket = 0;
+            ctrl->abort = 0;
             __threadfence();
-            atomicExch(&a.ctrl->done, 0u);
+            atomicExch(&ctrl->done, 0u);
         }
     }
 }
@@ -742,7 +718,6 @@ __global__ void __launch_bounds__(kCompactThreads, 2) compact_stream(const __gri
     __shared__ uint64_t s_X;
     __shared__ int s_ok;
     __shared__ uint32_t s_first;
-    __shared__ uint32_t s_last;
     __shared__ uint64_t s_part[kWarps];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) s_tile = atomicAdd(&a.ctrl->ticket, 1u);  // tiles in scheduling order
@@ -768,7 +743,7 @@ __global__ void __launch_bounds__(kCompactThreads, 2) compact_stream(const __gri
         total += x;
     }
     const uint32_t excl = before + incl - L;
-    // (the bucket coder published the tile's total: see tile_add)
+    if (tid == 0) st_release(&a.cdesc[tile], make_desc(0, tile == 0 ? kStatePrefix : kStateAggregate, total));
     // the staged words of each bucket: a scan of their counts places them in shared
     // memory, where they are gathered (cp.async) while the look-back runs
     const uint32_t NW = (L + 31u) >> 5;
@@ -867,7 +842,7 @@ __global__ void __launch_bounds__(kCompactThreads, 2) compact_stream(const __gri
     __syncthreads();
     if (!s_ok) {
         if (gather) asm volatile("cp.async.wait_all;\n" ::: "memory");  // no copy outlives the CTA
-        finish_compaction(a, s_last);
+        release_control(a.ctrl);
         return;
     }
     const uint64_t X = s_X;
@@ -914,7 +889,7 @@ __global__ void __launch_bounds__(kCompactThreads, 2) compact_stream(const __gri
                     report(a.status, QSGD_ST_OVERFLOW);
             }
         }
-        finish_compaction(a, s_last);
+        release_control(a.ctrl);
         return;
     }
     // four buckets at a time and two words a lane of each, all loaded before any is
@@ -975,7 +950,7 @@ __global__ void __launch_bounds__(kCompactThreads, 2) compact_stream(const __gri
             if (!more) break;
         }
     }
-    finish_compaction(a, s_last);
+    release_control(a.ctrl);
 }
 
 // One instance per kernel, so that each kernel gets its own shared-memory attribute.

@@ -98,17 +98,13 @@ struct StageArgs {
     uint64_t* offsets;
     ScanControl* ctrl;
     uint64_t* cdesc;      // compaction scan descriptor per tile of kCompactBlock buckets
-    unsigned long long* cacc;  // per tile: buckets coded << 40 | their bits (bucket coder)
     uint64_t ntiles;
 };
 
-// Workspace of the two-launch encoder: [0, 256) control block; the bucket sizes; the
-// staging slots; then, past both the slots and the one-pass encoders' record area
-// (which those encoders clear before they run), the compaction's descriptors and the
-// per-tile accumulators.  Descriptors and accumulators are zero between calls: zeroed
-// by qsgd_workspace_init, and by the compaction's last CTA at the end of every call.
+// Workspace of the two-launch encoder: [0, 256) control block; the compaction's
+// descriptors; the bucket sizes; the staging slots.
 struct StageLayout {
-    size_t bits_off, stage_off, desc_off, acc_off, total;
+    size_t desc_off, bits_off, stage_off, total;
     uint64_t ntiles;
     uint32_t slot_words;
 };
