@@ -104,7 +104,8 @@ QSGD_API uint64_t qsgd_max_encoded_words(uint64_t n, uint32_t d, uint32_t s);
  * workspace serves every encoder for (n, d, s).  It must be zero-filled once before
  * its first use (qsgd_workspace_init); every encode leaves it ready for the next
  * one, whichever encoder ran before.  One workspace must not be used by two encodes
- * that may run at the same time. */
+ * that may run at the same time.  A call that returned an error after enqueueing
+ * work (QSGD_ERR_CUDA) may leave it mid-call: zero-fill it again before reusing it. */
 QSGD_API size_t qsgd_encode_workspace_bytes(uint64_t n, uint32_t d, uint32_t s);
 
 /* Zero-fills a workspace (cudaMemsetAsync on `stream`). */

@@ -384,18 +384,6 @@ __global__ void __launch_bounds__(kStageBlock, (V <= 4 ? 4 : 2)) code_buckets_sh
         uint32_t pos = 32u;
         if (m <= kChunkCoords) {
             // --- one chunk: the values stay in registers ---------------------------------
-#ifndef QSGD_STAGE_PREFETCH
-#define QSGD_STAGE_PREFETCH 0
-#endif
-            if (QSGD_STAGE_PREFETCH && b + gwarps < a.nb) {  // the warp's next bucket into L2
-                const uint64_t nbase = (b + gwarps) * d;
-                const uint64_t nend = min(a.n, nbase + d);
-                const uint64_t line = (nbase * 4u & ~uint64_t(127)) + 128u * static_cast<uint32_t>(lane);
-                if (line < nend * 4u) {
-                    const char* pf = reinterpret_cast<const char*>(a.in) + line;
-                    asm volatile("prefetch.global.L2 [%0];" ::"l"(pf));
-                }
-            }
             load_contig<V>(a.in + base, ql, m, x);
             if constexpr (kEF) {  // p = e + g
                 load_contig<V>(a.ef + base, ql, m, ev);

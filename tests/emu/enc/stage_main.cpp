@@ -7,6 +7,7 @@
 // status word.  The arguments and the workspace layout are those the library's host
 // code derives.
 #include "block_emu.h"
+#include <algorithm>
 thread_local dim3e threadIdx, blockIdx;
 dim3e gridDim, blockDim;
 thread_local BlockCtx* t_blk;
@@ -138,10 +139,30 @@ int main(int argc, char** argv) {
     a.ntiles = ntiles;
     const size_t smem = qsgd::stage_smem_bytes(s, a.buf_words);
     const unsigned grid = (unsigned)std::max<uint64_t>(1, std::min<uint64_t>((nb + qsgd::kStageWarps - 1) / qsgd::kStageWarps, grid_req));
-    if (ef) code_any<true>(a, grid, smem); else code_any<false>(a, grid, smem);
-    if (g_emu_error) return 4;
-    run_grid((unsigned)ntiles, qsgd::kCompactThreads, qsgd::kCompactSmemWords * 4, [&] { qsgd::compact_stream(a); });
-    if (g_emu_error) return 4;
+    // two calls on the one workspace, the second over the first's leftovers; each call
+    // must leave the control block at rest, and without memory the second call's
+    // stream must equal the first's
+    std::vector<uint32_t> first_words;
+    std::vector<uint64_t> first_offsets;
+    for (int call = 0; call < (ef ? 1 : 2); ++call) {
+        if (ef) code_any<true>(a, grid, smem); else code_any<false>(a, grid, smem);
+        if (g_emu_error) return 4;
+        run_grid((unsigned)ntiles, qsgd::kCompactThreads, qsgd::kCompactSmemWords * 4, [&] { qsgd::compact_stream(a); });
+        if (g_emu_error) return 4;
+        const qsgd::ScanControl* c = reinterpret_cast<const qsgd::ScanControl*>(wsp);
+        if (c->ticket != 0 || c->done != 0 || c->abort != 0) {
+            std::fprintf(stderr, "control block not at rest after a call\n");
+            return 5;
+        }
+        if (call == 0 && !ef) {
+            first_words = words;
+            first_offsets = offsets;
+            std::fill(words.begin(), words.end(), 0xDEADBEEFu);
+        } else if (call == 1 && (words != first_words || offsets != first_offsets)) {
+            std::fprintf(stderr, "the second call's stream differs\n");
+            return 6;
+        }
+    }
     spit(dir + "/words.bin", words.data(), 4 * cap);
     spit(dir + "/offsets.bin", offsets.data(), 8 * (nb + 1));
     if (ef) spit(dir + "/e_out.bin", e.data(), 4 * n);
