@@ -40,8 +40,8 @@ FALLBACK_HBM_GBS = 6650.0
 # hash of the kernel sources it was taken on; reported as null once the sources
 # differ.
 TRAFFIC_SOURCES = ("qsgd_encode_stage.cu", "qsgd_decode_rows.cu", "qsgd_device.cuh", "qsgd_limits.h")
-TRAFFIC = {"bytes_per_launch": {"encode": 122624768, "decode": 50971392, "decode_accumulate": 153777664},
-           "sources_sha256": "0cfc6eb06a5d22ac8b8ca8238c2e6a8ebe89140fdfecddeee4c8134be8c1d9c0"}
+TRAFFIC = {"bytes_per_launch": {"encode": 121600512, "decode": 52798976, "decode_accumulate": 153329920},
+           "sources_sha256": "efb98dc19330ffc8fece0b18c383cce2260fe6e82dff13e0d89435b111e4123a"}
 
 
 # The kernels behind each phase of the c2 step (d = 512, s = 16, aligned buffers).
@@ -85,6 +85,9 @@ def parse_args():
                     help="no timing: run the config's step three times (two as warm-up) and exit, for a "
                          "profiler's capture of the third; c2 / c5 take --s")
     ap.add_argument("--s", type=int, default=None, help="levels for --profile-step on c2 or c5")
+    ap.add_argument("--d", type=int, default=None,
+                    help="bucket size for --profile-step on c2 (d % 4 != 0 takes the general encoder and the "
+                         "any-shape decoder)")
     ap.add_argument("--bbit", type=int, default=None, choices=[2, 4, 8],
                     help="--profile-step on c2 with the fixed-width b-bit codec instead")
     return ap.parse_args()
@@ -122,10 +125,11 @@ def profile_step(args):
         return
     w = {1: W.C1, 2: W.C2, 3: W.C3, 5: W.c5(16)}[cfg]
     s = args.s if args.s is not None and cfg in (2, 5) else w.s
+    d = args.d if args.d is not None and cfg == 2 else w.d
     x = torch.from_numpy(w.generate()).cuda()
     acc = torch.zeros(w.n, dtype=torch.float32, device="cuda")
     for _ in range(3):
-        enc = B.encode(x, w.d, s, w.seed)
+        enc = B.encode(x, d, s, w.seed)
         out, st = B.decode(enc)
         B.decode_accumulate([enc], acc)
     torch.cuda.synchronize()
