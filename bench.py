@@ -39,9 +39,9 @@ FALLBACK_HBM_GBS = 6650.0
 # capture of this workload (ncu --set full over bench.py --profile-step), with the
 # hash of the kernel sources it was taken on; reported as null once the sources
 # differ.
-TRAFFIC_SOURCES = ("qsgd_encode_stage.cu", "qsgd_decode_rows.cu", "qsgd_device.cuh", "qsgd_limits.h")
+TRAFFIC_SOURCES = ("qsgd_encode_stage.cu", "qsgd_decode_rows.cu", "qsgd_tables.cuh", "qsgd_device.cuh", "qsgd_limits.h")
 TRAFFIC = {"bytes_per_launch": {"encode": 121600512, "decode": 52798976, "decode_accumulate": 153329920},
-           "sources_sha256": "efb98dc19330ffc8fece0b18c383cce2260fe6e82dff13e0d89435b111e4123a"}
+           "sources_sha256": "013a97a0bac78a94a6fe26c364c0b4ecd526a10213b643e381922a10b79c8456"}
 
 
 # The kernels behind each phase of the c2 step (d = 512, s = 16, aligned buffers).

@@ -14,7 +14,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libqsgd_b200.so")
 SOURCES = ["qsgd_api.cu", "qsgd_encode.cu", "qsgd_decode.cu", "qsgd_static_ws.cu", "qsgd_bbit.cu", "qsgd_ef.cu", "qsgd_mean.cu", "qsgd_encode_stage.cu", "qsgd_decode_rows.cu"]
-HEADERS = ["qsgd_device.cuh", "qsgd_internal.h", "qsgd_limits.h"]
+HEADERS = ["qsgd_device.cuh", "qsgd_internal.h", "qsgd_limits.h", "qsgd_tables.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

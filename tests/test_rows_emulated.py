@@ -32,6 +32,7 @@ def build_rows_exe(d, extra=()):
     for h in ("qsgd_internal.h", "qsgd_limits.h"):
         shutil.copy(os.path.join(CSRC, h), src_dir / h)
     (src_dir / "qsgd_device.cuh").write_text(_host_source(open(os.path.join(CSRC, "qsgd_device.cuh")).read()))
+    (src_dir / "qsgd_tables.cuh").write_text(_host_source(open(os.path.join(CSRC, "qsgd_tables.cuh")).read()))
     src = open(os.path.join(CSRC, "qsgd_decode_rows.cu")).read()
     cut = src.index("// One CTA per SM, its warps one group each where the groups allow: every SM busy.")
     (src_dir / "rows_emu.inc").write_text(_host_source(src[:cut]) + "}  // namespace\n}  // namespace qsgd\n")
