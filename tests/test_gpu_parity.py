@@ -135,3 +135,14 @@ def test_one_workspace_serves_every_encoder(oracle_lib):
     for n, d, s, seed in ((70_001, 512, 16, 1), (30_001, 3, 4, 2), (70_001, 512, 16, 3),
                           (50_000, 8192, 1, 4), (10_000, 128, 64, 5)):
         check_parity(oracle_lib, W.layered(n, seed), d, s, seed)
+
+
+def test_compaction_tiles_on_both_paths(oracle_lib):
+    """Tiles of 256 buckets at s = 48: full tiles hold about 16,920 staged words,
+    more than the compaction gathers into shared memory, so they copy from the
+    staging slots; tiles with zero buckets hold fewer and are gathered."""
+    n = 6 * 256 * 512
+    v = W.normal(n, 3)
+    v[256 * 512:256 * 512 + 60 * 512] = 0.0
+    v[3 * 256 * 512:3 * 256 * 512 + 128 * 512] = 0.0
+    check_parity(oracle_lib, v, 512, 48, seed=1)

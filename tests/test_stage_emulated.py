@@ -209,3 +209,20 @@ def test_stage_lookback_over_several_windows(stage_exe_small_tiles, tmp_path, or
     check_norms(gn, own_norms)
     r_words, r_offsets, _, _ = oracle_lib.encode(v, d, s, 4, norms_in=gn)
     assert np.array_equal(offsets, r_offsets) and np.array_equal(words, r_words)
+
+
+def test_stage_compaction_tiles_on_both_paths(stage_exe, tmp_path, oracle_lib):
+    """Tiles of 256 buckets at s = 48: full tiles hold about 16,920 staged words,
+    more than the compaction's shared-memory gather, so they copy from the staging
+    slots; tiles with zero buckets hold fewer and are gathered."""
+    n = 3 * 256 * 512
+    v = W.normal(n, 3)
+    v[256 * 512:256 * 512 + 60 * 512] = 0.0
+    words, offsets, status, _ = _run(stage_exe, tmp_path, v, 512, 48, 1, 3)
+    _, _, own_norms, own_status = oracle_lib.encode(v, 512, 48, 1)
+    assert status == own_status
+    gn = stream_norms(words, offsets)
+    check_norms(gn, own_norms)
+    r_words, r_offsets, _, _ = oracle_lib.encode(v, 512, 48, 1, norms_in=gn)
+    assert np.array_equal(offsets, r_offsets) and np.array_equal(words, r_words)
+
