@@ -74,7 +74,8 @@ StageLayout stage_layout(uint64_t n, uint32_t d, uint32_t s) {
     StageLayout L{};
     const uint64_t nb = n ? ceil_div(n, d) : 0;
     const uint64_t slot_bits = 32u + static_cast<uint64_t>(d) * (2u + omega_len_host(s));
-    L.slot_words = static_cast<uint32_t>(ceil_div(slot_bits, 32));
+    // a whole number of 16-byte units, so that every slot starts 16-byte aligned
+    L.slot_words = static_cast<uint32_t>(ceil_div(ceil_div(slot_bits, 32), 4) * 4);
     L.ntiles = ceil_div(nb, kCompactBlock);
     L.desc_off = 256;
     L.bits_off = L.desc_off + align256(sizeof(uint64_t) * L.ntiles);

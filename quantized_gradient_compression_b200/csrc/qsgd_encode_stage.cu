@@ -734,7 +734,9 @@ __global__ void __launch_bounds__(kCompactThreads, 2) compact_stream(const __gri
     if (tid == 0) st_release(&a.cdesc[tile], make_desc(0, tile == 0 ? kStatePrefix : kStateAggregate, total));
     // the staged words of each bucket: a scan of their counts places them in shared
     // memory, where they are gathered (cp.async) while the look-back runs
-    const uint32_t NW = (L + 31u) >> 5;
+    // (in whole 16-byte units: a slot starts 16-byte aligned, so its words are
+    // gathered 16 bytes a copy, up to three words past the bucket's last)
+    const uint32_t NW = ((L + 127u) >> 7) << 2;
     uint32_t wincl = NW;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -760,12 +762,12 @@ __global__ void __launch_bounds__(kCompactThreads, 2) compact_stream(const __gri
     __syncthreads();
     if (gather) {
         for (uint32_t i = warp; i < nt; i += kWarps) {
-            const uint32_t nw = (s_L[i] + 31u) >> 5, rw = s_RW[i];
+            const uint32_t nw4 = ((s_L[i] + 127u) >> 7) << 2, rw = s_RW[i];
             const uint32_t* src0 = a.stage + (b0 + i) * a.slot_words;
-            for (uint32_t k = lane; k < nw; k += 32) {
+            for (uint32_t k = 4u * lane; k < nw4; k += 128u) {
                 const uint32_t saddr = static_cast<uint32_t>(__cvta_generic_to_shared(smem + rw + k));
                 const uint32_t* src = src0 + k;
-                asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(saddr), "l"(src) : "memory");
+                asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(saddr), "l"(src) : "memory");
             }
         }
         asm volatile("cp.async.commit_group;\n" ::: "memory");

@@ -164,6 +164,7 @@ inline uint32_t __cvta_generic_to_shared(const void* p) {
 }
 // cp.async with its source size: the first `src_bytes` bytes copied, the rest zeroed
 inline void emu_cp16z(uint32_t dst, const void* src, uint32_t src_bytes) {
+    if ((dst & 15u) != 0 || (reinterpret_cast<uintptr_t>(src) & 15u) != 0) emu_fail("cp.async of 16 bytes not 16-byte aligned", __LINE__);
     std::memset(emu_smem() + dst, 0, 16);
     std::memcpy(emu_smem() + dst, src, src_bytes);
 }
