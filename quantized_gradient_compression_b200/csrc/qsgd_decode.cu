@@ -30,48 +30,45 @@
 #include "../../include/qsgd.h"
 #include "qsgd_device.cuh"
 #include "qsgd_internal.h"
+#include "qsgd_tables.cuh"
 
 namespace qsgd {
 namespace {
 
-constexpr int kLutBits = 12;
-constexpr int kLut = 1 << kLutBits;
+constexpr int kLut = kLutSize;
 
 // Record table entry for a 12-bit window: [4:0] record length (0: not complete in
-// 12 bits or k > s), [5] the window holds a complete record with k > s, [15:6] gap,
-// [25:16] k, [31] sign.
-__device__ __forceinline__ bool omega_from_window(uint32_t w, int nbits, int& pos, uint32_t& value) {
-    uint32_t v = 1;
-    for (;;) {
-        if (pos >= nbits) return false;
-        const uint32_t bit = (w >> (nbits - 1 - pos)) & 1u;
-        ++pos;
-        if (bit == 0) {
-            value = v;
-            return true;
-        }
-        if (pos + static_cast<int>(v) > nbits) return false;
-        const uint32_t rest = (w >> (nbits - pos - v)) & ((1u << v) - 1u);
-        pos += v;
-        v = (1u << v) | rest;
-    }
-}
-
-__device__ void build_record_lut(uint32_t* lut, uint32_t s, int tid, int nthreads) {
-    for (int w = tid; w < kLut; w += nthreads) {
+// 12 bits, or k > s), [5] the window holds a complete record with k > s, [15:6] gap,
+// [25:16] k, [31] sign.  Computed at compile time for every level (within 12 bits,
+// gap <= 15 and k <= 15); the copy into shared memory marks levels above s.
+struct alignas(16) RecordLut {  // read with 16-byte loads
+    uint32_t v[kLutSize];
+};
+constexpr RecordLut make_record_lut() {
+    RecordLut t{};
+    for (uint32_t w = 0; w < static_cast<uint32_t>(kLutSize); ++w) {
         int pos = 0;
         uint32_t gap = 0, k = 0, e = 0;
-        if (omega_from_window(static_cast<uint32_t>(w), kLutBits, pos, gap) && pos < kLutBits) {
-            const uint32_t sign = (static_cast<uint32_t>(w) >> (kLutBits - 1 - pos)) & 1u;
+        if (window_omega(w, kLutBits, pos, gap) && pos < kLutBits) {
+            const uint32_t sign = (w >> (kLutBits - 1 - pos)) & 1u;
             ++pos;
-            if (omega_from_window(static_cast<uint32_t>(w), kLutBits, pos, k)) {
-                if (k <= s && gap < 1024 && k < 1024)
-                    e = static_cast<uint32_t>(pos) | (gap << 6) | (k << 16) | (sign << 31);
-                else if (k > s)
-                    e = 32u;
-            }
+            if (window_omega(w, kLutBits, pos, k)) e = static_cast<uint32_t>(pos) | (gap << 6) | (k << 16) | (sign << 31);
         }
-        lut[w] = e;
+        t.v[w] = e;
+    }
+    return t;
+}
+__device__ const RecordLut kRecordLutGlobal = make_record_lut();
+
+__device__ __forceinline__ void record_lut_fill(uint32_t* lut, uint32_t s, int tid, int nthreads) {
+    const uint4* src = reinterpret_cast<const uint4*>(kRecordLutGlobal.v);
+    for (int i = tid; i < kLutSize / 4; i += nthreads) {
+        uint4 q = src[i];
+        uint32_t* e = &q.x;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            if ((e[j] & 31u) != 0u && ((e[j] >> 16) & 1023u) > s) e[j] = 32u;  // a level above s
+        reinterpret_cast<uint4*>(lut)[i] = q;
     }
 }
 
@@ -191,7 +188,7 @@ __global__ void __launch_bounds__(kDecodeBlock) decode_warp(const __grid_constan
     float* stage = reinterpret_cast<float*>(smem + kLut) + warp * 32 * kStride;
     LaneStream* lstate = reinterpret_cast<LaneStream*>(smem + kLut + kDecWarps * 32 * kStride) +
                          (warp * 32 + lane) * a.K;
-    build_record_lut(lut, a.s, tid, kDecodeBlock);
+    record_lut_fill(lut, a.s, tid, kDecodeBlock);
     __syncthreads();
 
     const uint64_t ngroups = (a.nb + 31) / 32;
@@ -470,7 +467,7 @@ __global__ void __launch_bounds__(kMultiBlock) decode_multi(const __grid_constan
     float* const tiles = reinterpret_cast<float*>(smem + kLut);
     float* const stage = tiles + warp * 32 * kMStride;
     float* const row = stage + lane * kMStride;
-    build_record_lut(lut, a.s, tid, kMultiBlock);
+    record_lut_fill(lut, a.s, tid, kMultiBlock);
     __syncthreads();
     const float fs = __uint2float_rn(a.s);
     const uint32_t d = a.d;

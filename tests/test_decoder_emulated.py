@@ -33,6 +33,7 @@ def _kernel_source() -> str:
     s = src[:cut] + "}  // namespace\n}  // namespace qsgd\n"
     s = s.replace('#include "../../include/qsgd.h"', '#include "%s"' % os.path.join(ROOT, "include", "qsgd.h"))
     s = s.replace('#include "qsgd_internal.h"', '#include "%s"' % os.path.join(CSRC, "qsgd_internal.h"))
+    s = s.replace('#include "qsgd_tables.cuh"', '#include "%s"' % os.path.join(CSRC, "qsgd_tables.cuh"))
     s = s.replace("extern __shared__ __align__(16) uint32_t smem[];",
                   "uint32_t* smem = reinterpret_cast<uint32_t*>(g_emu_smem);")
     assert "asm" not in s
