@@ -832,28 +832,57 @@ __global__ void __launch_bounds__(kSparseBlock) decode_sparse(const __grid_const
                     continue;
                 }
                 uint32_t next = 0;
-                for (uint32_t it = 0; r.left > 0; ++it) {
-                    uint32_t gap, sign, k;
-                    const uint32_t e = lut[r.peek() >> (32 - kLutBits)];
-                    const uint32_t len1 = e & 15u;
-                    if (len1 != 0u && it < kParseGuard) {  // the first record of the window
-                        gap = (e >> 8) & 15u;
-                        sign = (e >> 23) & 1u;
-                        k = (e >> 16) & 0x7Fu;
-                        r.advance(len1);
-                    } else if (it >= kParseGuard || !slow_record(r, a.s, gap, sign, k)) {
-                        bad = true;
-                        break;
-                    }
+                // the records: up to two table entries a step, each up to two records
+                // (a second record or entry only when it ends inside the bucket)
+                bool ok = true;
+                auto put = [&](uint32_t gap, uint32_t sign, uint32_t k) {
                     next += gap;
                     if (next > m) {
-                        bad = true;
-                        break;
+                        ok = false;
+                        return;
                     }
                     const float q = __fmul_rn(scale, __uint2float_rn(k));
                     const float v = sign ? -q : q;
                     row[next - 1] = kAcc ? __fadd_rn(row[next - 1], v) : v;
+                };
+                for (uint32_t it = 0; r.left > 0 && ok; ++it) {
+                    if (it >= kParseGuard) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t w = r.peek();
+                    const uint32_t e = lut[w >> (32 - kLutBits)];
+                    const uint32_t len1 = e & 15u;
+                    if (len1 == 0u) {  // a record the table does not hold, bit by bit
+                        uint32_t gap, sign, k;
+                        if (!slow_record(r, a.s, gap, sign, k)) {
+                            ok = false;
+                            break;
+                        }
+                        put(gap, sign, k);
+                        continue;
+                    }
+                    const uint32_t len2 = (e >> 4) & 15u;
+                    const bool two = static_cast<int32_t>(len2) <= r.left;
+                    uint32_t used = two ? len2 : len1;
+                    put((e >> 8) & 15u, (e >> 23) & 1u, (e >> 16) & 0x7Fu);  // table codes: sign << 7 | k
+                    const uint32_t c2 = e >> 24;
+                    if (ok && two && c2 != 0u) put((e >> 12) & 15u, c2 >> 7, c2 & 0x7Fu);
+                    if (ok && two) {
+                        const uint32_t f = lut[(w << used) >> (32 - kLutBits)];
+                        const uint32_t flen1 = f & 15u;
+                        if (flen1 != 0u && static_cast<int32_t>(used + flen1) <= r.left) {
+                            const uint32_t flen2 = (f >> 4) & 15u;
+                            const bool ftwo = static_cast<int32_t>(used + flen2) <= r.left;
+                            put((f >> 8) & 15u, (f >> 23) & 1u, (f >> 16) & 0x7Fu);
+                            const uint32_t fc2 = f >> 24;
+                            if (ok && ftwo && fc2 != 0u) put((f >> 12) & 15u, fc2 >> 7, fc2 & 0x7Fu);
+                            used += ftwo ? flen2 : flen1;
+                        }
+                    }
+                    r.advance(used);
                 }
+                if (!ok) bad = true;
                 if (r.left != 0) bad = true;
             }
             if (bad) atomicOr(a.status, QSGD_ST_BAD_STREAM);

@@ -243,6 +243,8 @@ SPARSE = [
     (40_003, 3001, 16, 1, False, "layered"),
     (30_000, 2048, 300, 3, True, "normal"),
     (20_000, 4096, 4, 17, True, "small_normal"),
+    (20_000, 2048, 1 << 20, 1, False, "normal"),  # levels past 16 bits (bit-serial)
+    (65_536, 65_536, 256, 1, False, "normal"),    # one bucket (the small workload's shape)
 ]
 
 
