@@ -757,7 +757,10 @@ __global__ void __launch_bounds__(kCompactThreads, 2) compact_stream(const __gri
         wtotal += x;
     }
     if (tid <= kCompactBlock) s_RW[tid] = wbefore + wincl - NW;  // s_RW[kCompactBlock] = wtotal
-    const bool gather = wtotal <= kCompactSmemWords;
+    // (the 16-byte copies need 16-byte aligned slots: a workspace laid out otherwise
+    // takes the direct copy)
+    const bool gather = wtotal <= kCompactSmemWords && (a.slot_words & 3u) == 0u &&
+                        (reinterpret_cast<uintptr_t>(a.stage) & 15u) == 0u;
     const uint32_t nt = static_cast<uint32_t>(min(static_cast<uint64_t>(kCompactBlock), a.nb - b0));
     __syncthreads();
     if (gather) {

@@ -7,6 +7,7 @@
 // status word.  The arguments and the workspace layout are those the library's host
 // code derives.
 #include "block_emu.h"
+#include <cstdlib>
 #include <algorithm>
 thread_local dim3e threadIdx, blockIdx;
 dim3e gridDim, blockDim;
@@ -110,7 +111,10 @@ int main(int argc, char** argv) {
     // workspace as the host code lays it out: control block, descriptors, sizes, slots;
     // zeroed once, then filled with garbage where the kernels must not rely on zeros
     const uint64_t slot_bits = 32u + (uint64_t)d * (2u + qsgd::omega_len_host(s));
-    const uint32_t slot_words = (uint32_t)(((slot_bits + 31) / 32 + 3) / 4 * 4);  // whole 16-byte units
+    // whole 16-byte units, as the library lays them out; STAGE_UNPADDED=1 lays them out
+    // word by word, which the compaction must notice (it then copies without gathering)
+    const bool unpadded = std::getenv("STAGE_UNPADDED") != nullptr;
+    const uint32_t slot_words = unpadded ? (uint32_t)((slot_bits + 31) / 32) : (uint32_t)(((slot_bits + 31) / 32 + 3) / 4 * 4);
     const uint64_t ntiles = (nb + qsgd::kCompactBlock - 1) / qsgd::kCompactBlock;
     const size_t desc_off = 256, bits_off = desc_off + align256(8 * ntiles), stage_off = bits_off + align256(4 * nb);
     const size_t total = stage_off + align256(4 * nb * (size_t)slot_words);

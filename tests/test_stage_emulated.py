@@ -226,3 +226,19 @@ def test_stage_compaction_tiles_on_both_paths(stage_exe, tmp_path, oracle_lib):
     r_words, r_offsets, _, _ = oracle_lib.encode(v, 512, 48, 1, norms_in=gn)
     assert np.array_equal(offsets, r_offsets) and np.array_equal(words, r_words)
 
+
+def test_stage_compaction_with_unaligned_slots(stage_exe, tmp_path, oracle_lib, monkeypatch):
+    """Staging slots laid out word by word (not the library's layout): the compaction
+    must not gather them 16 bytes a copy (the emulator rejects an unaligned 16-byte
+    copy) and must still place every bit."""
+    monkeypatch.setenv("STAGE_UNPADDED", "1")
+    n, d, s = 20_003, 100, 7  # 32 + 100 * (2 + 6) bits: 26 words a slot
+    v = W.normal(n, 8)
+    words, offsets, status, _ = _run(stage_exe, tmp_path, v, d, s, 2, 2)
+    _, _, own_norms, own_status = oracle_lib.encode(v, d, s, 2)
+    assert status == own_status
+    gn = stream_norms(words, offsets)
+    check_norms(gn, own_norms)
+    r_words, r_offsets, _, _ = oracle_lib.encode(v, d, s, 2, norms_in=gn)
+    assert np.array_equal(offsets, r_offsets) and np.array_equal(words, r_words)
+
