@@ -700,8 +700,6 @@ __global__ void __launch_bounds__(kCompactThreads, 2) compact_stream(const __gri
     __shared__ uint32_t s_R[kCompactBlock];
     __shared__ uint32_t s_L[kCompactBlock];
     __shared__ uint32_t s_RW[kCompactBlock + 1];
-    __shared__ uint32_t s_warp[kWarps];
-    __shared__ uint32_t s_wwarp[kWarps];
     __shared__ uint32_t s_tile;
     __shared__ uint64_t s_X;
     __shared__ int s_ok;
@@ -714,49 +712,35 @@ __global__ void __launch_bounds__(kCompactThreads, 2) compact_stream(const __gri
     const uint64_t b0 = tile * kCompactBlock;
     const uint64_t b = b0 + tid;
     const uint32_t L = tid < kCompactBlock && b < a.nb ? a.bits[b] : 0u;
-    // block scan of the bucket sizes (a tile is at most 256 * 2^21 bits... far below 2^32)
-    uint32_t incl = L;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t t = __shfl_up_sync(kAll, incl, o);
-        if (lane >= o) incl += t;
-    }
-    if (lane == 31) s_warp[warp] = incl;
-    __syncthreads();
-    uint32_t before = 0, total = 0;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-        const uint32_t x = s_warp[w];
-        before += w < warp ? x : 0u;
-        total += x;
-    }
-    const uint32_t excl = before + incl - L;
-    if (tid == 0) st_release(&a.cdesc[tile], make_desc(0, tile == 0 ? kStatePrefix : kStateAggregate, total));
-    // the staged words of each bucket: a scan of their counts places them in shared
-    // memory, where they are gathered (cp.async) while the look-back runs
-    // (in whole 16-byte units: a slot starts 16-byte aligned, so its words are
-    // gathered 16 bytes a copy, up to three words past the bucket's last)
+    // one block scan of two counts at once: the bucket's bits (low half; a tile is at
+    // most 256 * 2^21 bits, far below 2^32) and its staged words in whole 16-byte
+    // units (high half: a slot starts 16-byte aligned, so its words are gathered 16
+    // bytes a copy, up to three words past the bucket's last)
     const uint32_t NW = ((L + 127u) >> 7) << 2;
-    uint32_t wincl = NW;
+    const uint64_t pair = static_cast<uint64_t>(NW) << 32 | L;
+    uint64_t pincl = pair;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t t = __shfl_up_sync(kAll, wincl, o);
-        if (lane >= o) wincl += t;
+        const uint64_t t = __shfl_up_sync(kAll, pincl, o);
+        if (lane >= o) pincl += t;
     }
-    if (lane == 31) s_wwarp[warp] = wincl;
-    if (tid < kCompactBlock) {
-        s_R[tid] = excl;  // tile-relative start of each bucket
-        s_L[tid] = L;
-    }
+    if (lane == 31) s_part[warp] = pincl;
+    if (tid < kCompactBlock) s_L[tid] = L;
     __syncthreads();
-    uint32_t wbefore = 0, wtotal = 0;
+    uint64_t pbefore = 0, ptotal = 0;
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) {
-        const uint32_t x = s_wwarp[w];
-        wbefore += w < warp ? x : 0u;
-        wtotal += x;
+        const uint64_t x = s_part[w];
+        pbefore += w < warp ? x : 0u;
+        ptotal += x;
     }
-    if (tid <= kCompactBlock) s_RW[tid] = wbefore + wincl - NW;  // s_RW[kCompactBlock] = wtotal
+    const uint32_t total = static_cast<uint32_t>(ptotal);
+    const uint32_t excl = static_cast<uint32_t>(pbefore + pincl - pair);
+    if (tid == 0) st_release(&a.cdesc[tile], make_desc(0, tile == 0 ? kStatePrefix : kStateAggregate, total));
+    if (tid < kCompactBlock) s_R[tid] = excl;  // tile-relative start of each bucket
+    const uint32_t wincl = static_cast<uint32_t>((pbefore + pincl) >> 32), wtotal = static_cast<uint32_t>(ptotal >> 32);
+    const uint32_t wbefore = wincl - NW;
+    if (tid <= kCompactBlock) s_RW[tid] = wbefore;  // tile-relative first staged word; s_RW[kCompactBlock] = wtotal
     // (the 16-byte copies need 16-byte aligned slots: a workspace laid out otherwise
     // takes the direct copy)
     const bool gather = wtotal <= kCompactSmemWords && (a.slot_words & 3u) == 0u &&
@@ -764,10 +748,15 @@ __global__ void __launch_bounds__(kCompactThreads, 2) compact_stream(const __gri
     const uint32_t nt = static_cast<uint32_t>(min(static_cast<uint64_t>(kCompactBlock), a.nb - b0));
     __syncthreads();
     if (gather) {
-        for (uint32_t i = warp; i < nt; i += kWarps) {
+        // gG lanes per bucket (4, 8, 16 or 32: the fewest that cover the tile's mean
+        // count of 16-byte units), each lane one unit a pass
+        const uint32_t mc = (wtotal / 4u + nt - 1u) / nt;
+        const uint32_t gG = mc <= 4u ? 4u : mc <= 8u ? 8u : mc <= 16u ? 16u : 32u;
+        const uint32_t gsub = static_cast<uint32_t>(lane) / gG, gl = static_cast<uint32_t>(lane) % gG;
+        for (uint32_t i = static_cast<uint32_t>(warp) * (32u / gG) + gsub; i < nt; i += kWarps * (32u / gG)) {
             const uint32_t nw4 = ((s_L[i] + 127u) >> 7) << 2, rw = s_RW[i];
             const uint32_t* src0 = a.stage + (b0 + i) * a.slot_words;
-            for (uint32_t k = 4u * lane; k < nw4; k += 128u) {
+            for (uint32_t k = 4u * gl; k < nw4; k += 4u * gG) {
                 const uint32_t saddr = static_cast<uint32_t>(__cvta_generic_to_shared(smem + rw + k));
                 const uint32_t* src = src0 + k;
                 asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(saddr), "l"(src) : "memory");
