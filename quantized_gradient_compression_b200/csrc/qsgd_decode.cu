@@ -20,9 +20,11 @@
 //   - decode_warp: any shape (d % 4 != 0, unaligned output), up to 16 streams a
 //     launch, each lane's per-stream state in shared memory.
 //   - decode_multi: two or more streams (and the mean) with d % 4 == 0, d <= 4096,
-//     s < 1024 and an aligned output, a warp per stream, side by side.
-// The launch routing (launch_decode) sends one stream with d <= 1024 to the row
-// decoders and d > 1024 to the large-bucket decoder (qsgd_decode_rows.cu).
+//     s < 1024 and an aligned output, a warp per stream, side by side; the row
+//     decoders' side-by-side kernel takes d <= 1024 with s <= 127.
+// The launch routing (launch_decode) sends one stream with d <= 1024, and several
+// streams with d <= 1024 and s <= 127, to the row decoders, and d > 1024 to the
+// large-bucket decoder (qsgd_decode_rows.cu).
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -654,11 +656,12 @@ cudaError_t launch_decode(const DecodeArgs& a, bool accumulate, cudaStream_t str
     if (a.nb == 0) return cudaSuccess;
     const bool multi = decode_multi_shape(a.d, a.s, a.out);
     // the row decoders when the shape allows: one stream staged as codes; several
-    // streams (and the mean) added onto fp32 tiles in stream order where the
-    // several-stream kernel below, which decodes the streams side by side, does not
-    // take the levels (s >= 1024)
+    // streams (and the mean) parsed side by side as byte codes (s <= 127), or added
+    // onto fp32 tiles in stream order where the several-stream kernel below, which
+    // decodes the streams side by side, does not take the levels (s >= 1024)
     if (decode_rows_shape(a.d, a.s, a.out)) {
         if (a.K == 1 && !a.start_zero && a.div == 0.f) return launch_decode_rows(a, accumulate, stream);
+        if (a.s <= kRowsMaxS8 && (accumulate || a.start_zero)) return launch_decode_rows_side(a, stream);
         if (!multi) return launch_decode_rows_multi(a, stream);
     }
     // the mean in one pass: streams decoded side by side, the sum divided at the end

@@ -1,5 +1,5 @@
-// QSGD row decoders: one stream staged as level codes, several streams added onto
-// fp32 tiles, and large buckets (sm_100a).
+// QSGD row decoders: one stream staged as level codes, several streams parsed side by
+// side or added onto fp32 tiles, and large buckets (sm_100a).
 //
 // Method: "QSGD (Quantized Stochastic Gradient Descent) with Elias Coding" (AIMech
 // curated entry).  The definition paragraph calls the coding "lossless prefix
@@ -24,6 +24,13 @@
 //     row, written back segment by segment (half the shared memory of whole rows,
 //     twice the warps); records through a table of omega codes, one lookup for the
 //     gap and one for the level.
+// Several streams (decode-accumulate, K >= 2, and the mean):
+//   - decode_rows_side (s <= 127): a warp a stream, the streams of a chunk side by
+//     side in one CTA, each parsed as decode_rows does into a ring of byte codes; the
+//     CTA adds a segment's values onto the output in stream order once every warp has
+//     passed it.
+//   - decode_rows_multi (larger s where the other several-stream kernel does not
+//     take the levels): the streams one after another onto an fp32 tile.
 // Longer records take a bit-serial path.
 #include <cuda_runtime.h>
 
@@ -126,16 +133,73 @@ __device__ __forceinline__ void load_row(const DecodeArgs& a, uint64_t bb, int l
     }
 }
 
+// One parse step through the whole-record table (byte codes): up to two table
+// entries, each up to two records.  The 32 bits at the cursor hold both 12-bit
+// windows (the first entry's records take at most 12 bits); a record is taken only
+// when it ends inside the bucket.  A record longer than the window whose gap code
+// fits it (gap <= 63) is read as the entry's gap, the sign and a level from the
+// level table (k <= 15 and k <= s); that record ends within 20 bits of the cursor.
+// put(index, code) stores a record's code (sign << 7 | k) at its bucket-local index.
+// Returns false, having read nothing, when the record at the cursor is neither (the
+// bit-serial path takes it).
+template <class Put>
+__device__ __forceinline__ bool rows_table_step(RowReader& r, const uint32_t* lut, const uint8_t* klut, uint32_t s,
+                                                uint32_t& next, const Put& put) {
+    const uint32_t w = r.peek();
+    const uint32_t e = lut[w >> (32 - kLutBits)];
+    const uint32_t len1 = e & 15u;
+    if (len1 == 0u) {
+        const uint32_t gl = (e >> 4) & 15u;
+        const uint32_t kc = klut[(w << (gl + 1u)) >> (32 - kKLutBits)];
+        const uint32_t kl = kc & 15u;
+        if (gl == 0u || kl == 0u || (kc >> 4) > s) return false;
+        next += (e >> 8) & 63u;
+        put(next - 1u, (((w << gl) >> 31) << 7) | (kc >> 4));
+        r.advance(gl + 1u + kl);
+        return true;
+    }
+    const uint32_t len2 = (e >> 4) & 15u;
+    const bool two = static_cast<int32_t>(len2) <= r.left;
+    uint32_t used = two ? len2 : len1;
+    next += (e >> 8) & 15u;
+    put(next - 1u, (e >> 16) & 0xFFu);
+    const uint32_t c2 = e >> 24;
+    if (two && c2 != 0u) {
+        next += (e >> 12) & 15u;
+        put(next - 1u, c2);
+    }
+    if (two) {
+        const uint32_t f = lut[(w << used) >> (32 - kLutBits)];
+        const uint32_t flen1 = f & 15u;
+        if (flen1 != 0u && static_cast<int32_t>(used + flen1) <= r.left) {
+            const uint32_t flen2 = (f >> 4) & 15u;
+            const bool ftwo = static_cast<int32_t>(used + flen2) <= r.left;
+            next += (f >> 8) & 15u;
+            put(next - 1u, (f >> 16) & 0xFFu);
+            const uint32_t fc2 = f >> 24;
+            if (ftwo && fc2 != 0u) {
+                next += (f >> 12) & 15u;
+                put(next - 1u, fc2);
+            }
+            used += ftwo ? flen2 : flen1;
+        }
+    }
+    r.advance(used);
+    return true;
+}
+
 template <int V, bool kAcc>
 __global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows(const __grid_constant__ DecodeArgs a,
                                                                    uint32_t stride_w) {
     extern __shared__ __align__(16) uint32_t smem[];
     uint32_t* const lut = smem;
+    uint8_t* const klut = reinterpret_cast<uint8_t*>(smem + kLutSize);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int W = blockDim.x >> 5;
-    uint32_t* const rows = smem + kLutSize + static_cast<uint32_t>(warp) * 32u * stride_w;
+    uint32_t* const rows = smem + kLutSize + kKLutWords + static_cast<uint32_t>(warp) * 32u * stride_w;
     uint8_t* const myrow = reinterpret_cast<uint8_t*>(rows + static_cast<uint32_t>(lane) * stride_w);
     rows_lut_fill(lut, a.s, tid, blockDim.x);
+    k_lut_fill(klut, tid, blockDim.x);
     __syncthreads();
     const StreamRef st = a.streams[0];
     const float fs = __uint2float_rn(a.s);
@@ -195,41 +259,8 @@ __global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows(const __grid_c
                 break;
             }
             if (r.left > 0) {
-                // up to two table entries a step, each up to two records: the 32 bits at
-                // the cursor hold both 12-bit windows (the first takes at most 12 bits);
-                // a record is taken only when it ends inside the bucket
-                const uint32_t w = r.peek();
-                const uint32_t e = lut[w >> (32 - kLutBits)];
-                const uint32_t len1 = e & 15u;
-                if (len1 != 0u) {
-                    const uint32_t len2 = (e >> 4) & 15u;
-                    const bool two = static_cast<int32_t>(len2) <= r.left;
-                    uint32_t used = two ? len2 : len1;
-                    next += (e >> 8) & 15u;
-                    myrow[min(next - 1u, d)] = static_cast<uint8_t>((e >> 16) & 0xFFu);
-                    const uint32_t c2 = e >> 24;
-                    if (two && c2 != 0u) {
-                        next += (e >> 12) & 15u;
-                        myrow[min(next - 1u, d)] = static_cast<uint8_t>(c2);
-                    }
-                    if (two) {
-                        const uint32_t f = lut[(w << used) >> (32 - kLutBits)];
-                        const uint32_t flen1 = f & 15u;
-                        if (flen1 != 0u && static_cast<int32_t>(used + flen1) <= r.left) {
-                            const uint32_t flen2 = (f >> 4) & 15u;
-                            const bool ftwo = static_cast<int32_t>(used + flen2) <= r.left;
-                            next += (f >> 8) & 15u;
-                            myrow[min(next - 1u, d)] = static_cast<uint8_t>((f >> 16) & 0xFFu);
-                            const uint32_t fc2 = f >> 24;
-                            if (ftwo && fc2 != 0u) {
-                                next += (f >> 12) & 15u;
-                                myrow[min(next - 1u, d)] = static_cast<uint8_t>(fc2);
-                            }
-                            used += ftwo ? flen2 : flen1;
-                        }
-                    }
-                    r.advance(used);
-                } else {
+                const auto put = [&](uint32_t idx, uint32_t code) { myrow[min(idx, d)] = static_cast<uint8_t>(code); };
+                if (!rows_table_step(r, lut, klut, a.s, next, put)) {
                     uint32_t gap = 0, sign = 0, k = 0;
                     if (slow_record(r, a.s, gap, sign, k)) {
                         next += gap;
@@ -759,6 +790,221 @@ __global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows_multi(const __
 }
 
 // ---------------------------------------------------------------------------
+// Several streams side by side, byte codes (decode-accumulate with K >= 2 and the
+// mean of K >= 1 streams, s <= 127).
+//
+// The kSideWarps warps of a CTA take W = min(K, kSideWarps) streams at a time (a
+// chunk) and G = kSideWarps / W groups of 32 buckets: warp w parses stream
+// c0 + (w mod W) of group w div W, a bucket a lane, into a ring of byte codes
+// (sign << 7 | k) of two kSSeg-column segments a row, with the whole-record table (up
+// to two records a lookup, two lookups a step).  Once every lane of every warp has
+// passed a segment, the CTA adds the chunk's values there onto the output, each
+// coordinate in stream order: v = out + 0 (+0 for the first chunk of a mean), then
+// v = v + q_j for every stream j of the chunk, v / div in the last chunk of a mean.
+// The first add makes a -0.0 output +0.0 as the first stream's add would; after it
+// adding a zero code's +0 leaves v as it is, as the sum in stream order does.  The
+// add clears the codes it reads for the ring's next turn; the output is read and
+// written once per chunk.  A step of table records moves at most 60 columns and a
+// long record through the level table at most 63, so the records of a lane still
+// short of the segment's end land in the ring; a bit-serial one further ahead waits
+// in registers until its segment.  Segments of 64 columns keep a CTA at 51 KB of
+// shared memory, four CTAs an SM.
+// ---------------------------------------------------------------------------
+#ifndef QSGD_SIDE_SEG
+#define QSGD_SIDE_SEG 64
+#endif
+constexpr int kSideWarps = 8;
+constexpr uint32_t kSSeg = QSGD_SIDE_SEG;         // columns a segment
+constexpr uint32_t kSRing = 2 * kSSeg;            // codes (bytes) a ring row
+constexpr uint32_t kSStride = kSRing / 4 + 1;     // words a ring row: 1 mod 32, rows on different banks
+constexpr uint32_t kSSegWords = kSSeg / 4;        // words of a row's segment
+constexpr uint32_t kSRowsPerWarp = 32 / kSSegWords;  // rows a warp's 32 threads add at once
+// (a step of table records moves at most 60 columns, a long record through the
+// level table at most 63)
+static_assert(kSSeg == 64 || kSSeg == 128, "a segment holds a step of records and a warp whole rows");
+
+// The value of one byte code (sign << 7 | k) of a bucket with step sc: fl(sc * k),
+// the sign last.
+__device__ __forceinline__ float side_value(uint32_t code, float sc) {
+    const float kf = __fsub_rn(__uint_as_float(0x4B000000u | (code & 0x7Fu)), 8388608.0f);
+    return __uint_as_float(__float_as_uint(__fmul_rn(sc, kf)) | ((code & 0x80u) << 24));
+}
+
+__global__ void __launch_bounds__(32 * kSideWarps, 2) decode_rows_side(const __grid_constant__ DecodeArgs a) {
+    extern __shared__ __align__(16) uint32_t smem[];
+    constexpr int kThreads = 32 * kSideWarps;
+    uint32_t* const lut = smem;
+    uint8_t* const klut = reinterpret_cast<uint8_t*>(smem + kLutSize);
+    float* const s_scale = reinterpret_cast<float*>(smem + kLutSize + kKLutWords);  // [warp][lane]
+    uint32_t* const rings = smem + kLutSize + kKLutWords + kThreads;                // [warp][row][kSStride]
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    uint8_t* const myrow = reinterpret_cast<uint8_t*>(rings + static_cast<uint32_t>(tid) * kSStride);
+    rows_lut_fill(lut, a.s, tid, kThreads);
+    k_lut_fill(klut, tid, kThreads);
+    for (uint32_t q = static_cast<uint32_t>(tid); q < kThreads * kSStride; q += kThreads) rings[q] = 0u;
+    __syncthreads();
+    const float fs = __uint2float_rn(a.s);
+    const uint32_t d = a.d;
+    const uint64_t ngroups = (a.nb + 31) / 32;
+    const int W = min(a.K, kSideWarps);  // streams to a chunk
+    const int G = kSideWarps / W;        // groups a CTA takes at once
+    const int gi = warp / W;             // this warp's group of the G (G when idle)
+    const int wj = warp - gi * W;        // this warp's stream within a chunk
+    for (uint64_t g0 = static_cast<uint64_t>(blockIdx.x) * G; g0 < ngroups; g0 += static_cast<uint64_t>(gridDim.x) * G) {
+        const uint64_t g = g0 + gi;
+        const uint64_t b = g * 32 + lane;
+        const bool live = gi < G && b < a.nb;
+        const uint32_t m = live ? static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - b * d)) : 0u;
+        for (int c0 = 0; c0 < a.K; c0 += W) {
+            const int nt = min(W, a.K - c0);                     // streams in this chunk
+            const bool mine = gi < G && g < ngroups && wj < nt;  // uniform in the warp
+            const bool from_zero = a.start_zero && c0 == 0;
+            const bool divide = c0 + nt == a.K && a.div != 0.f;
+            // --- open this lane's bucket of stream c0 + wj: header checks, the norm ----
+            bool bad = false;
+            RowReader r;
+            r.left = 0;
+            float scale = 0.f;
+            if (mine && live) {
+                const StreamRef st = a.streams[c0 + wj];
+                const uint64_t begin = st.offsets[b];
+                const uint64_t end = st.offsets[b + 1];
+                if (!(end >= begin && end - begin >= 32 && end <= st.num_words * 32 && end - begin < (1ull << 30))) {
+                    bad = true;
+                } else {
+                    r.init(st.words, st.num_words, begin, static_cast<uint32_t>(end - begin));
+                    const uint32_t nbits = r.peek();
+                    r.advance(32);
+                    const float norm = __uint_as_float(nbits);
+                    if (nbits == 0) {
+                        bad = r.left != 0;
+                        r.left = 0;
+                    } else if (!(isfinite(norm) && norm > 0.f)) {
+                        bad = true;
+                        r.left = 0;
+                    } else {
+                        scale = __fdiv_rn(norm, fs);
+                        if (!(scale > 0.f) && r.left != 0) {  // a zero scale carries no records
+                            bad = true;
+                            r.left = 0;
+                        }
+                    }
+                }
+            }
+            if (bad) r.left = 0;
+            s_scale[tid] = scale;
+            uint32_t next = 0;  // bucket-local index after the last record
+            bool pend = false;  // a bit-serial record beyond the ring, held here
+            uint32_t pidx = 0, pcode = 0;
+            uint32_t it = 0;  // parse steps over the whole bucket (an explicit bound)
+            const auto put = [&](uint32_t idx, uint32_t code) {
+                myrow[idx & (kSRing - 1u)] = static_cast<uint8_t>(code);
+            };
+            for (uint32_t lo = 0; lo < d; lo += kSSeg) {
+                const uint32_t hi = lo + kSSeg;
+                if (mine) {
+                    if (pend && pidx < hi + kSSeg) {
+                        put(pidx, pcode);
+                        pend = false;
+                    }
+                    // --- parse until every lane has passed column hi (or ended) -------
+                    for (;; ++it) {
+                        const bool act = r.left > 0 && !pend && next < hi;
+                        if (!__any_sync(kWarpAll, act)) break;
+                        if (it >= kParseGuard) {  // never reached by a well-formed stream
+                            if (act) {
+                                bad = true;
+                                r.left = 0;
+                            }
+                            continue;
+                        }
+                        if (!act || rows_table_step(r, lut, klut, a.s, next, put)) continue;
+                        // a record the table does not hold, bit by bit
+                        uint32_t gap = 0, sign = 0, k = 0;
+                        if (slow_record(r, a.s, gap, sign, k)) {
+                            next += gap;
+                            const uint32_t idx = min(next - 1u, d);
+                            if (idx >= hi + kSSeg) {
+                                pend = true;
+                                pidx = idx;
+                                pcode = row_code<uint8_t>(sign, k);
+                            } else {
+                                put(idx, row_code<uint8_t>(sign, k));
+                            }
+                        } else {
+                            bad = true;
+                            r.left = 0;
+                        }
+                    }
+                }
+                __syncthreads();  // every warp's codes of [lo, hi) are in its ring, the scales too
+                // --- the chunk's values of [lo, hi) onto the output, in stream order ---
+                const uint32_t slot0 = (lo & (kSRing - 1u)) >> 2;  // the segment's first word in a ring row
+                for (uint32_t q = static_cast<uint32_t>(tid); q < static_cast<uint32_t>(G) * 32u * kSSegWords;
+                     q += kThreads) {
+                    // a warp's threads take rows i and i + 32 / kSRowsPerWarp: their ring
+                    // words lie on different banks
+                    const uint32_t qg = q / (32u * kSSegWords);
+                    const uint32_t qi = q % (32u * kSSegWords);
+                    const uint32_t cw = qi % kSSegWords;
+                    const uint32_t rr = qi / 32u + (qi % 32u) / kSSegWords * (32u / kSRowsPerWarp);
+                    const uint32_t c = lo + 4u * cw;
+                    const uint64_t bb = (g0 + qg) * 32 + rr;
+                    const uint32_t mm = bb < a.nb ? static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - bb * d)) : 0u;
+                    float* const gp = a.out + bb * d + c;
+                    float v[4] = {0.f, 0.f, 0.f, 0.f};
+                    if (c < mm && !from_zero) {
+                        if (c + 4 <= mm) {
+                            const float4 o = *reinterpret_cast<const float4*>(gp);
+                            v[0] = o.x;
+                            v[1] = o.y;
+                            v[2] = o.z;
+                            v[3] = o.w;
+                        } else {  // c < mm <= c + 3
+                            v[0] = gp[0];
+                            if (c + 1 < mm) v[1] = gp[1];
+                            if (c + 2 < mm) v[2] = gp[2];
+                        }
+                    }
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) v[e] = __fadd_rn(v[e], 0.f);  // -0.0 -> +0.0, as a first add of +0
+                    const uint32_t row0 = (qg * static_cast<uint32_t>(W) * 32u + rr) * kSStride + slot0 + cw;
+                    for (int t = 0; t < nt; ++t) {
+                        uint32_t* const p = rings + row0 + static_cast<uint32_t>(t) * 32u * kSStride;
+                        const uint32_t w = *p;
+                        *p = 0u;
+                        const float sc = s_scale[(qg * static_cast<uint32_t>(W) + static_cast<uint32_t>(t)) * 32u + rr];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) v[e] = __fadd_rn(v[e], side_value(w >> (8 * e), sc));
+                    }
+                    if (c >= mm) continue;
+                    if (divide) {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) v[e] = __fdiv_rn(v[e], a.div);
+                    }
+                    if (c + 4 <= mm) {
+                        *reinterpret_cast<float4*>(gp) = make_float4(v[0], v[1], v[2], v[3]);
+                    } else {
+                        gp[0] = v[0];
+                        if (c + 1 < mm) gp[1] = v[1];
+                        if (c + 2 < mm) gp[2] = v[2];
+                    }
+                }
+                __syncthreads();  // the ring's words of [lo, hi) are clear again
+            }
+            // every record index below m, the bucket consumed exactly, nothing held back
+            if (mine && live && !bad && (next > m || r.left != 0 || pend)) bad = true;
+            if (mine && bad) atomicOr(a.status, QSGD_ST_BAD_STREAM);
+            // a malformed bucket may have left codes past its segments: clear the ring
+            if (__syncthreads_or(mine && bad)) {
+                for (uint32_t q = static_cast<uint32_t>(tid); q < kThreads * kSStride; q += kThreads) rings[q] = 0u;
+                __syncthreads();
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Large buckets (d > 1024): a CTA takes 32 buckets.  All its threads first write the
 // buckets' output range with 16-byte stores where it is aligned: zeros (decode), or
 // the output + 0 (decode-accumulate; +0 turns -0.0 into +0.0 as the add of a zero
@@ -910,7 +1156,9 @@ cudaError_t launch_row_kernel(Kernel kernel, bool& attr_done, const DecodeArgs& 
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     const size_t per_warp = static_cast<size_t>(32) * stride * sizeof(uint32_t);
-    const size_t lut_bytes = static_cast<size_t>(kLutSize) * sizeof(uint32_t);
+    // the record table and the level table (the ring kernel uses the first half of
+    // the record table's room for its omega table, and the level table's not at all)
+    const size_t lut_bytes = static_cast<size_t>(kLutSize + kKLutWords) * sizeof(uint32_t);
     const int W_fit = static_cast<int>(std::min<size_t>(kRowsMaxWarps, (static_cast<size_t>(optin) - lut_bytes - 1024) / per_warp));
     if (W_fit < 1) return cudaErrorInvalidConfiguration;
     const uint64_t groups = (a.nb + 31) / 32;
@@ -975,6 +1223,28 @@ cudaError_t launch_rows_multi(const DecodeArgs& a, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
+cudaError_t launch_rows_side(const DecodeArgs& a, cudaStream_t stream) {
+    constexpr int kThreads = 32 * kSideWarps;
+    const size_t smem =
+        (static_cast<size_t>(kLutSize) + kKLutWords + kThreads + static_cast<size_t>(kThreads) * kSStride) * sizeof(uint32_t);
+    static bool attr_set[64] = {};
+    int dev = 0, sms = 0, per_sm = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 64 || !attr_set[dev]) {
+        cudaFuncSetAttribute(decode_rows_side, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (dev < 64) attr_set[dev] = true;
+    }
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_rows_side, kThreads, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    const uint64_t G = static_cast<uint64_t>(kSideWarps / std::min(a.K, kSideWarps));  // groups a CTA takes at once
+    const uint64_t sets = ((a.nb + 31) / 32 + G - 1) / G;
+    const uint64_t blocks = std::max<uint64_t>(1, std::min<uint64_t>(sets, static_cast<uint64_t>(sms) * per_sm));
+    decode_rows_side<<<static_cast<unsigned>(blocks), kThreads, smem, stream>>>(a);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_sparse(const DecodeArgs& a, bool accumulate, cudaStream_t stream) {
     int dev = 0, sms = 0;
     cudaGetDevice(&dev);
@@ -1003,6 +1273,8 @@ bool decode_rows_shape(uint32_t d, uint32_t s, const float* out) {
 }
 
 cudaError_t launch_decode_rows_multi(const DecodeArgs& a, cudaStream_t stream) { return launch_rows_multi(a, stream); }
+
+cudaError_t launch_decode_rows_side(const DecodeArgs& a, cudaStream_t stream) { return launch_rows_side(a, stream); }
 
 cudaError_t launch_decode_rows(const DecodeArgs& a, bool accumulate, cudaStream_t stream) {
     if (a.s <= kRowsMaxS8) return accumulate ? launch_rows_bytes<true>(a, stream) : launch_rows_bytes<false>(a, stream);

@@ -158,8 +158,11 @@ cudaError_t launch_decode(const DecodeArgs& a, bool accumulate, cudaStream_t str
 // The one-stream decoder with whole rows staged as byte codes (qsgd_decode_rows.cu).
 bool decode_rows_shape(uint32_t d, uint32_t s, const float* out);
 cudaError_t launch_decode_rows(const DecodeArgs& a, bool accumulate, cudaStream_t stream);
-// Several streams (decode-accumulate and the mean) on the same shapes (qsgd_decode_rows.cu).
+// Several streams (decode-accumulate and the mean) on the same shapes (qsgd_decode_rows.cu):
+// added onto fp32 tiles one stream after another (any s), or parsed side by side as
+// byte codes (s <= 127).
 cudaError_t launch_decode_rows_multi(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_decode_rows_side(const DecodeArgs& a, cudaStream_t stream);
 // Buckets larger than the row decoders take (qsgd_decode_rows.cu): decode and
 // decode-accumulate (K <= 16 streams to a launch, in order).
 bool decode_sparse_shape(uint32_t d, const float* out);

@@ -49,11 +49,13 @@ constexpr bool window_record(uint32_t w, int& pos, uint32_t& gap, uint32_t& code
 }
 
 // The whole records at the start of a 12-bit window, up to two: [3:0] length of the
-// first (0: none, take the bit-serial path), [7:4] length of both (the first's when
-// there is no second), [11:8] first gap, [15:12] second gap, [23:16] first code,
-// [31:24] second code (0: none; a code is never 0, since k >= 1).  For s >= 15 the
-// table is the same for every s; a smaller s drops the records with k > s when the
-// table is copied (rows_lut_fill).
+// first, [7:4] length of both (the first's when there is no second), [11:8] first
+// gap, [15:12] second gap, [23:16] first code, [31:24] second code (0: none; a code
+// is never 0, since k >= 1).  A window that holds no whole record has [3:0] = 0 and,
+// when the gap's omega code fits the window, [7:4] its length and [13:8] the gap
+// (<= 63, as every omega code of at most 12 bits); the sign and the level follow it
+// (the level through kKLut).  For s >= 15 the table is the same for every s; a
+// smaller s drops the records with k > s when the table is copied (rows_lut_fill).
 struct alignas(16) RowsLut {  // read with 16-byte loads
     uint32_t v[kLutSize];
 };
@@ -73,12 +75,38 @@ constexpr RowsLut make_rows_lut() {
             }
             e = static_cast<uint32_t>(len1) | (static_cast<uint32_t>(len2) << 4) | (g1 << 8) | (g2 << 12) |
                 (c1 << 16) | (c2 << 24);
+        } else {
+            int gpos = 0;
+            uint32_t gap = 0;
+            if (window_omega(w, kLutBits, gpos, gap)) e = (static_cast<uint32_t>(gpos) << 4) | (gap << 8);
         }
         t.v[w] = e;
     }
     return t;
 }
 __device__ const RowsLut kRowsLutGlobal = make_rows_lut();
+
+// The omega code of a level at the top of a 7-bit window: [3:0] length (0: longer
+// than 7 bits), [7:4] value (<= 15, as every code of at most 7 bits).
+constexpr int kKLutBits = 7;
+constexpr int kKLutWords = (1 << kKLutBits) / 4;  // its size in shared memory, in words
+struct alignas(16) KLut {  // read with 16-byte loads
+    uint8_t v[1 << kKLutBits];
+};
+constexpr KLut make_k_lut() {
+    KLut t{};
+    for (uint32_t w = 0; w < (1u << kKLutBits); ++w) {
+        int pos = 0;
+        uint32_t val = 0;
+        t.v[w] = window_omega(w, kKLutBits, pos, val) ? static_cast<uint8_t>(static_cast<uint32_t>(pos) | (val << 4)) : 0;
+    }
+    return t;
+}
+__device__ const KLut kKLutGlobal = make_k_lut();
+__device__ __forceinline__ void k_lut_fill(uint8_t* klut, int tid, int nthreads) {
+    const uint4* src = reinterpret_cast<const uint4*>(kKLutGlobal.v);
+    for (int i = tid; i < (1 << kKLutBits) / 16; i += nthreads) reinterpret_cast<uint4*>(klut)[i] = src[i];
+}
 
 // The omega code at the top of a 12-bit window: [3:0] length (0: longer than 12
 // bits), [9:4] value (<= 63, as every code of at most 12 bits).

@@ -1,9 +1,10 @@
-// Runs the one-stream row decoder decode_rows, compiled for the host under
-// block_emu.h, with all its CTAs at once.
-// argv: dir accumulate grid warps
-// dir holds params.bin (u64 n, d, s), w0.bin (u32 stream words), o0.bin (u64[nb+1])
-// and out_in.bin (fp32[n], the output before the call).  It writes out.bin and
-// prints the status word.
+// Runs the row decoders (decode_rows, decode_rows_ring, decode_rows_multi,
+// decode_rows_side, decode_sparse), compiled for the host under block_emu.h, with all
+// their CTAs at once.
+// argv: dir accumulate grid warps [K [mean [side]]]
+// dir holds params.bin (u64 n, d, s), w<j>.bin (u32 stream words), o<j>.bin
+// (u64[nb+1]) and out_in.bin (fp32[n], the output before the call).  It writes
+// out.bin and prints the status word.
 #include "block_emu.h"
 thread_local dim3e threadIdx, blockIdx;
 dim3e gridDim, blockDim;
@@ -59,7 +60,7 @@ template <class T>
 static void run_t(const qsgd::DecodeArgs& a, bool acc, unsigned grid, unsigned W) {
     if constexpr (sizeof(T) == 2) {
         const uint32_t stride = qsgd::ring_stride_words();
-        const size_t smem = 4 * (size_t)qsgd::kLutSize + (size_t)W * 32 * stride * 4;
+        const size_t smem = 4 * (size_t)(qsgd::kLutSize + qsgd::kKLutWords) + (size_t)W * 32 * stride * 4;
         if (acc)
             run_grid(grid, 32 * W, smem, [&] { qsgd::decode_rows_ring<true>(a, stride); });
         else
@@ -67,7 +68,7 @@ static void run_t(const qsgd::DecodeArgs& a, bool acc, unsigned grid, unsigned W
         return;
     }
     const uint32_t stride = qsgd::rows_stride_words(a.d);
-    const size_t smem = 4 * (size_t)qsgd::kLutSize + (size_t)W * 32 * stride * 4;
+    const size_t smem = 4 * (size_t)(qsgd::kLutSize + qsgd::kKLutWords) + (size_t)W * 32 * stride * 4;
     switch (qsgd::fast_v(a.d)) {
         case 1: run_v<1>(a, acc, grid, W, stride, smem); break;
         case 2: run_v<2>(a, acc, grid, W, stride, smem); break;
@@ -77,11 +78,15 @@ static void run_t(const qsgd::DecodeArgs& a, bool acc, unsigned grid, unsigned W
 }
 
 // Several streams: decode_rows_multi over K streams, 16 to a launch as the library
-// sends them (a mean starts the first launch from +0 and divides in the last).
+// sends them (a mean starts the first launch from +0 and divides in the last); with
+// side, decode_rows_side (a CTA of kSideWarps warps, the streams side by side).
 static void run_multi(qsgd::DecodeArgs a, const std::vector<std::vector<unsigned char>>& ws,
-                      const std::vector<std::vector<unsigned char>>& os, bool mean, unsigned grid, unsigned W) {
+                      const std::vector<std::vector<unsigned char>>& os, bool mean, unsigned grid, unsigned W,
+                      bool side) {
     const int K = (int)ws.size();
-    const size_t smem = (qsgd::kLutSize + 256) * 2 + (size_t)W * (sizeof(qsgd::MsState) + 32 * qsgd::kMTile * 4);
+    const size_t smem = side ? (qsgd::kLutSize + qsgd::kKLutWords + 32 * qsgd::kSideWarps +
+                                (size_t)32 * qsgd::kSideWarps * qsgd::kSStride) * 4
+                             : (qsgd::kLutSize + 256) * 2 + (size_t)W * (sizeof(qsgd::MsState) + 32 * qsgd::kMTile * 4);
     for (int j0 = 0; j0 < K; j0 += qsgd::kMaxStreamsPerLaunch) {
         a.K = std::min(K - j0, qsgd::kMaxStreamsPerLaunch);
         a.first_group = j0 == 0;
@@ -92,7 +97,10 @@ static void run_multi(qsgd::DecodeArgs a, const std::vector<std::vector<unsigned
             a.streams[j].num_words = ws[j0 + j].size() / 4;
             a.streams[j].offsets = reinterpret_cast<const uint64_t*>(os[j0 + j].data());
         }
-        run_grid(grid, 32 * W, smem, [&] { qsgd::decode_rows_multi(a); });
+        if (side)
+            run_grid(grid, 32 * qsgd::kSideWarps, smem, [&] { qsgd::decode_rows_side(a); });
+        else
+            run_grid(grid, 32 * W, smem, [&] { qsgd::decode_rows_multi(a); });
         if (g_emu_error) return;
     }
 }
@@ -103,6 +111,7 @@ int main(int argc, char** argv) {
     const unsigned grid = std::atoi(argv[3]), W = std::atoi(argv[4]);
     const int K = argc > 5 ? std::atoi(argv[5]) : 1;
     const bool mean = argc > 6 && std::atoi(argv[6]) != 0;
+    const bool side = argc > 7 && std::atoi(argv[7]) != 0;
     auto prm = slurp(dir + "/params.bin");
     uint64_t q[3];
     std::memcpy(q, prm.data(), sizeof q);
@@ -153,7 +162,7 @@ int main(int argc, char** argv) {
         }
         qsgd::DecodeArgs a{};
         a.n = n; a.d = d; a.s = s; a.nb = nb; a.out = out.data(); a.status = &status;
-        run_multi(a, ws, os, mean, grid, W);
+        run_multi(a, ws, os, mean, grid, W, side);
         if (g_emu_error) return 4;
         spit(dir + "/out.bin", out.data(), 4 * n);
         std::printf("status %u\n", status);

@@ -141,10 +141,11 @@ def rows_asan(tmp_path_factory):
 
 def test_row_decoders_on_damaged_input(rows_asan, tmp_path, oracle_lib):
     """decode_rows (byte codes), decode_rows_ring (16-bit codes), decode_rows_multi
-    (K > 1) and decode_sparse (d > 1024) on bit flips, scrambled offsets and cut word
-    arrays: they may flag the input, but touch nothing outside their buffers."""
+    and decode_rows_side (K > 1), and decode_sparse (d > 1024) on bit flips, scrambled
+    offsets and cut word arrays: they may flag the input, but touch nothing outside
+    their buffers."""
     rng = np.random.default_rng(77)
-    for trial in range(30):
+    for trial in range(40):
         n = int(rng.integers(1, 6000))
         d = int(rng.choice([4, 100, 512, 1000, 1024, 2048, 3001]))
         s = int(rng.choice([1, 3, 16, 127, 300, 32767]))
@@ -168,8 +169,9 @@ def test_row_decoders_on_damaged_input(rows_asan, tmp_path, oracle_lib):
             offsets.astype(np.uint64).tofile(t / ("o%d.bin" % j))
         np.zeros(n, np.float32).tofile(t / "out_in.bin")
         np.array([n, d, s], np.uint64).tofile(t / "params.bin")
-        r = subprocess.run([rows_asan, str(t), "1" if acc else "0", "2", "2", str(K), "0"], capture_output=True,
-                           text=True, timeout=600)
+        side = d <= 1024 and s <= 127 and K > 1 and trial % 2 == 1
+        r = subprocess.run([rows_asan, str(t), "1" if acc else "0", "2", "2", str(K), "0", "1" if side else "0"],
+                           capture_output=True, text=True, timeout=600)
         assert r.returncode == 0 and "AddressSanitizer" not in r.stderr, (trial, n, d, s, K, r.stderr[-2000:])
 
 

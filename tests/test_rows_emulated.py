@@ -177,14 +177,14 @@ MULTI = [
 ]
 
 
-def _run_multi(exe, tmp, streams, n, d, s, mean, base, grid=2, warps=2):
+def _run_multi(exe, tmp, streams, n, d, s, mean, base, grid=2, warps=2, side=False):
     for j, (w, o) in enumerate(streams):
         np.concatenate([w, np.zeros(1, np.uint32)]).tofile(tmp / ("w%d.bin" % j))
         o.astype(np.uint64).tofile(tmp / ("o%d.bin" % j))
     base.tofile(tmp / "out_in.bin")
     np.array([n, d, s], np.uint64).tofile(tmp / "params.bin")
-    r = subprocess.run([exe, str(tmp), "1", str(grid), str(warps), str(len(streams)), "1" if mean else "0"],
-                       capture_output=True, text=True, timeout=900)
+    r = subprocess.run([exe, str(tmp), "1", str(grid), str(warps), str(len(streams)), "1" if mean else "0",
+                        "1" if side else "0"], capture_output=True, text=True, timeout=900)
     assert r.returncode == 0, (r.stdout[-500:], r.stderr[-2000:])
     return np.fromfile(tmp / "out.bin", np.float32), int(r.stdout.split()[-1])
 
@@ -232,6 +232,156 @@ def test_row_multi_decoder_corrupt_stream(rows_exe, tmp_path, oracle_lib):
         if flipped[w0:w1].any():
             keep[b * d:min(n, (b + 1) * d)] = False
     assert keep.any() and not keep.all()
+    assert np.array_equal(got[keep].view(np.uint32), ref[keep].view(np.uint32))
+
+
+# decode_rows_side: K streams parsed side by side (a warp a stream) into rings of byte
+# codes, added onto the output in stream order after each segment.  K from one (the
+# mean) past a chunk of eight warps and past one launch of 16; every d % 128 class and
+# a ragged last bucket; grids that leave CTAs several sets of groups (the rings are
+# reused); sparse streams with gaps past the ring (bit-serial records held back).
+SIDE = [
+    (20_003, 512, 4, 2, False, 1, "small_normal"),
+    (20_003, 512, 16, 3, True, 2, "layered"),
+    (9_001, 128, 4, 17, False, 2, "small_normal"),
+    (7_000, 100, 7, 5, True, 1, "normal"),
+    (6_000, 1000, 127, 8, False, 2, "layered"),
+    (6_000, 1024, 16, 9, True, 1, "normal"),
+    (3_000, 512, 1, 18, True, 2, "heavy_tailed_sparse"),
+    (4_000, 4, 2, 4, False, 1, "normal"),
+    (12_000, 200, 16, 1, True, 1, "layered"),
+    (30_000, 1024, 1, 2, False, 1, "heavy_tailed_sparse"),
+    (1, 512, 16, 2, False, 1, "normal"),
+]
+
+
+@pytest.mark.parametrize("n,d,s,K,mean,grid,kind", SIDE, ids=["n%d-d%d-s%d-K%d-mean%d-g%d-%s" % c for c in SIDE])
+def test_side_decoder_matches_oracle(rows_exe, tmp_path, oracle_lib, n, d, s, K, mean, grid, kind):
+    streams = []
+    for j in range(K):
+        v = W.GENERATORS[kind](n, 90 + j)
+        w, o, _, st = oracle_lib.encode(v, d, s, seed=3 + j)
+        assert st == 0
+        streams.append((w, o))
+    base = _base(n, d, True)
+    got, status = _run_multi(rows_exe, tmp_path, streams, n, d, s, mean, base, grid=grid, side=True)
+    assert status == 0
+    if mean:
+        ref, rst = oracle_lib.decode_mean(streams, n, d, s)
+    else:
+        ref = base.copy()
+        _, rst = oracle_lib.decode_accumulate(streams, n, d, s, ref)
+    assert rst == 0
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+
+
+@pytest.fixture(scope="module")
+def rows_exe_seg128(tmp_path_factory):
+    if shutil.which("g++") is None:
+        pytest.skip("g++ not available")
+    return build_rows_exe(tmp_path_factory.mktemp("rowsemu128"), ("-O1", "-DQSGD_SIDE_SEG=128"))
+
+
+@pytest.mark.parametrize("n,d,s,K,mean,grid,kind", [SIDE[1], SIDE[6], SIDE[9]],
+                         ids=["n%d-d%d-s%d-K%d-mean%d-g%d-%s" % c for c in (SIDE[1], SIDE[6], SIDE[9])])
+def test_side_decoder_128_column_segments(rows_exe_seg128, tmp_path, oracle_lib, n, d, s, K, mean, grid, kind):
+    """The same kernel built with segments of 128 columns (two CTAs an SM)."""
+    test_side_decoder_matches_oracle(rows_exe_seg128, tmp_path, oracle_lib, n, d, s, K, mean, grid, kind)
+
+
+def test_side_decoder_far_records(rows_exe, tmp_path, oracle_lib):
+    """Buckets whose records lie more than two segments ahead (bit-serial gaps held
+    back until their segment), next to dense buckets, in three streams."""
+    d, s = 1024, 16
+    n = 64 * d
+    streams = []
+    for j in range(3):
+        rng = np.random.default_rng(40 + j)
+        v = np.zeros(n, np.float32)
+        for b in range(64):
+            if (b + j) % 2 == 0:  # two records, both far into the bucket
+                v[b * d + rng.integers(300, d, size=2)] = rng.standard_normal(2).astype(np.float32)
+            else:
+                v[b * d:(b + 1) * d] = rng.standard_normal(d).astype(np.float32)
+        w, o, _, st = oracle_lib.encode(v, d, s, seed=5 + j)
+        assert st == 0
+        streams.append((w, o))
+    base = _base(n, d, True)
+    got, status = _run_multi(rows_exe, tmp_path, streams, n, d, s, False, base, grid=1, side=True)
+    assert status == 0
+    ref = base.copy()
+    _, rst = oracle_lib.decode_accumulate(streams, n, d, s, ref)
+    assert rst == 0
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("K", [3, 10])
+def test_side_decoder_corrupt_stream(rows_exe, tmp_path, oracle_lib, K):
+    """Bit flips in stream 1: the input is flagged, and every bucket no flip touched
+    equals the oracle's sum, in later groups of the same CTA too (one CTA: its rings
+    are reused after the malformed buckets)."""
+    n, d, s = 40_000, 512, 4
+    intact, streams = [], []
+    for j in range(K):
+        w, o, _, _ = oracle_lib.encode(W.small_normal(n, 70 + j), d, s, seed=j)
+        intact.append((w, o))
+        w2 = w.copy()
+        if j == 1:
+            _flip_bits(w2, o, np.random.default_rng(9))
+        streams.append((w2, o))
+    base = _base(n, d, True)
+    got, status = _run_multi(rows_exe, tmp_path, streams, n, d, s, False, base, grid=1, side=True)
+    assert status & 2
+    ref = base.copy()
+    oracle_lib.decode_accumulate(intact, n, d, s, ref)
+    keep = np.ones(n, dtype=bool)
+    flipped = streams[1][0] != intact[1][0]
+    offs = intact[1][1]
+    for b in range(offs.size - 1):
+        w0, w1 = int(offs[b]) >> 5, (int(offs[b + 1]) + 31) >> 5
+        if flipped[w0:w1].any():
+            keep[b * d:min(n, (b + 1) * d)] = False
+    assert keep.any() and not keep.all()
+    assert np.array_equal(got[keep].view(np.uint32), ref[keep].view(np.uint32))
+
+
+def _bucket_bits(words, offsets, b):
+    """Bucket b's bits (MSB-first) as a numpy array of 0/1."""
+    bits = np.unpackbits(words.astype(">u4").view(np.uint8))
+    return bits[int(offsets[b]):int(offsets[b + 1])]
+
+
+def _assemble(buckets):
+    """A stream (words, offsets) from a list of per-bucket bit arrays."""
+    offsets = np.zeros(len(buckets) + 1, np.uint64)
+    offsets[1:] = np.cumsum([x.size for x in buckets])
+    allbits = np.concatenate(buckets + [np.zeros((-int(offsets[-1])) % 32, np.uint8)])
+    return np.packbits(allbits).view(">u4").astype(np.uint32), offsets
+
+
+def test_side_decoder_overlong_bucket(rows_exe, tmp_path, oracle_lib):
+    """A bucket whose records run past d (a well-formed bucket of 1024 coordinates in a
+    stream of d = 512): flagged, and the codes it left beyond its row's last segment
+    must not reach the buckets decoded after it by the same CTA."""
+    n, d, s, K = 8 * 32 * 512, 512, 16, 3  # eight groups: four sets of two for one CTA
+    streams = []
+    for j in range(K):
+        w, o, _, st = oracle_lib.encode(W.normal(n, 20 + j), d, s, seed=j)
+        assert st == 0
+        streams.append((w, o))
+    long_w, long_o, _, _ = oracle_lib.encode(W.normal(1024, 5), 1024, s, seed=9)
+    w1, o1 = streams[1]
+    buckets = [_bucket_bits(w1, o1, b) for b in range(o1.size - 1)]
+    buckets[3] = _bucket_bits(long_w, long_o, 0)
+    streams[1] = _assemble(buckets)
+    base = _base(n, d, True)
+    got, status = _run_multi(rows_exe, tmp_path, streams, n, d, s, False, base, grid=1, side=True)
+    assert status & 2
+    intact = [streams[0], (w1, o1), streams[2]]
+    ref = base.copy()
+    oracle_lib.decode_accumulate(intact, n, d, s, ref)
+    keep = np.ones(n, dtype=bool)
+    keep[3 * d:4 * d] = False
     assert np.array_equal(got[keep].view(np.uint32), ref[keep].view(np.uint32))
 
 
