@@ -808,7 +808,8 @@ __global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows_multi(const __
 // long record through the level table at most 63, so the records of a lane still
 // short of the segment's end land in the ring; a bit-serial one further ahead waits
 // in registers until its segment.  Segments of 64 columns keep a CTA at 51 KB of
-// shared memory, four CTAs an SM.
+// shared memory; three CTAs an SM (76 registers a thread) measured faster than four
+// (64 registers, with spills) or two (segments of 128 columns).
 // ---------------------------------------------------------------------------
 #ifndef QSGD_SIDE_SEG
 #define QSGD_SIDE_SEG 64
@@ -822,6 +823,7 @@ constexpr uint32_t kSRowsPerWarp = 32 / kSSegWords;  // rows a warp's 32 threads
 // (a step of table records moves at most 60 columns, a long record through the
 // level table at most 63)
 static_assert(kSSeg == 64 || kSSeg == 128, "a segment holds a step of records and a warp whole rows");
+static_assert((32 * kSSegWords) % (2 * 32 * kSideWarps) == 0, "a group's items come in pairs a thread");
 
 // The value of one byte code (sign << 7 | k) of a bucket with step sc: fl(sc * k),
 // the sign last.
@@ -830,7 +832,10 @@ __device__ __forceinline__ float side_value(uint32_t code, float sc) {
     return __uint_as_float(__float_as_uint(__fmul_rn(sc, kf)) | ((code & 0x80u) << 24));
 }
 
-__global__ void __launch_bounds__(32 * kSideWarps, 2) decode_rows_side(const __grid_constant__ DecodeArgs a) {
+#ifndef QSGD_SIDE_MINB
+#define QSGD_SIDE_MINB 3
+#endif
+__global__ void __launch_bounds__(32 * kSideWarps, QSGD_SIDE_MINB) decode_rows_side(const __grid_constant__ DecodeArgs a) {
     extern __shared__ __align__(16) uint32_t smem[];
     constexpr int kThreads = 32 * kSideWarps;
     uint32_t* const lut = smem;
@@ -860,6 +865,12 @@ __global__ void __launch_bounds__(32 * kSideWarps, 2) decode_rows_side(const __g
             const bool mine = gi < G && g < ngroups && wj < nt;  // uniform in the warp
             const bool from_zero = a.start_zero && c0 == 0;
             const bool divide = c0 + nt == a.K && a.div != 0.f;
+            if (c0 == 0 && !from_zero) {  // bring the groups' output into L2 while the records are parsed
+                const uint64_t i0 = g0 * 32 * d, i1 = min(a.n, (g0 + G) * 32 * d);
+                const char* const gpb = reinterpret_cast<const char*>(a.out + i0);
+                for (uint64_t off = static_cast<uint64_t>(tid) * 128; off < 4 * (i1 - i0); off += kThreads * 128)
+                    asm volatile("prefetch.global.L2 [%0];" ::"l"(gpb + off));
+            }
             // --- open this lane's bucket of stream c0 + wj: header checks, the norm ----
             bool bad = false;
             RowReader r;
@@ -940,54 +951,67 @@ __global__ void __launch_bounds__(32 * kSideWarps, 2) decode_rows_side(const __g
                 __syncthreads();  // every warp's codes of [lo, hi) are in its ring, the scales too
                 // --- the chunk's values of [lo, hi) onto the output, in stream order ---
                 const uint32_t slot0 = (lo & (kSRing - 1u)) >> 2;  // the segment's first word in a ring row
-                for (uint32_t q = static_cast<uint32_t>(tid); q < static_cast<uint32_t>(G) * 32u * kSSegWords;
-                     q += kThreads) {
-                    // a warp's threads take rows i and i + 32 / kSRowsPerWarp: their ring
-                    // words lie on different banks
-                    const uint32_t qg = q / (32u * kSSegWords);
-                    const uint32_t qi = q % (32u * kSSegWords);
-                    const uint32_t cw = qi % kSSegWords;
-                    const uint32_t rr = qi / 32u + (qi % 32u) / kSSegWords * (32u / kSRowsPerWarp);
-                    const uint32_t c = lo + 4u * cw;
-                    const uint64_t bb = (g0 + qg) * 32 + rr;
-                    const uint32_t mm = bb < a.nb ? static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - bb * d)) : 0u;
-                    float* const gp = a.out + bb * d + c;
-                    float v[4] = {0.f, 0.f, 0.f, 0.f};
-                    if (c < mm && !from_zero) {
-                        if (c + 4 <= mm) {
-                            const float4 o = *reinterpret_cast<const float4*>(gp);
-                            v[0] = o.x;
-                            v[1] = o.y;
-                            v[2] = o.z;
-                            v[3] = o.w;
-                        } else {  // c < mm <= c + 3
-                            v[0] = gp[0];
-                            if (c + 1 < mm) v[1] = gp[1];
-                            if (c + 2 < mm) v[2] = gp[2];
+                // two items (four coordinates of a row) a thread at a time, both outputs
+                // loaded before either is added; a warp's threads take rows i and
+                // i + 32 / kSRowsPerWarp, whose ring words lie on different banks
+                for (uint32_t q0 = static_cast<uint32_t>(tid); q0 < static_cast<uint32_t>(G) * 32u * kSSegWords;
+                     q0 += 2u * kThreads) {
+                    uint32_t c[2], mm[2], row0[2], sc0[2];
+                    float* gp[2];
+                    float v[2][4];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const uint32_t q = q0 + static_cast<uint32_t>(u) * kThreads;
+                        const uint32_t qg = q / (32u * kSSegWords);
+                        const uint32_t qi = q % (32u * kSSegWords);
+                        const uint32_t cw = qi % kSSegWords;
+                        const uint32_t rr = qi / 32u + (qi % 32u) / kSSegWords * (32u / kSRowsPerWarp);
+                        const uint64_t bb = (g0 + qg) * 32 + rr;
+                        c[u] = lo + 4u * cw;
+                        mm[u] = bb < a.nb ? static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - bb * d)) : 0u;
+                        gp[u] = a.out + bb * d + c[u];
+                        row0[u] = (qg * static_cast<uint32_t>(W) * 32u + rr) * kSStride + slot0 + cw;
+                        sc0[u] = qg * static_cast<uint32_t>(W) * 32u + rr;
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) v[u][e] = 0.f;
+                        if (c[u] < mm[u] && !from_zero) {
+                            if (c[u] + 4 <= mm[u]) {
+                                const float4 o = *reinterpret_cast<const float4*>(gp[u]);
+                                v[u][0] = o.x;
+                                v[u][1] = o.y;
+                                v[u][2] = o.z;
+                                v[u][3] = o.w;
+                            } else {  // c < mm <= c + 3
+                                v[u][0] = gp[u][0];
+                                if (c[u] + 1 < mm[u]) v[u][1] = gp[u][1];
+                                if (c[u] + 2 < mm[u]) v[u][2] = gp[u][2];
+                            }
                         }
                     }
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) v[e] = __fadd_rn(v[e], 0.f);  // -0.0 -> +0.0, as a first add of +0
-                    const uint32_t row0 = (qg * static_cast<uint32_t>(W) * 32u + rr) * kSStride + slot0 + cw;
-                    for (int t = 0; t < nt; ++t) {
-                        uint32_t* const p = rings + row0 + static_cast<uint32_t>(t) * 32u * kSStride;
-                        const uint32_t w = *p;
-                        *p = 0u;
-                        const float sc = s_scale[(qg * static_cast<uint32_t>(W) + static_cast<uint32_t>(t)) * 32u + rr];
+                    for (int u = 0; u < 2; ++u) {
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) v[e] = __fadd_rn(v[e], side_value(w >> (8 * e), sc));
-                    }
-                    if (c >= mm) continue;
-                    if (divide) {
+                        for (int e = 0; e < 4; ++e) v[u][e] = __fadd_rn(v[u][e], 0.f);  // -0.0 -> +0.0, as a first add of +0
+                        for (int t = 0; t < nt; ++t) {
+                            uint32_t* const p = rings + row0[u] + static_cast<uint32_t>(t) * 32u * kSStride;
+                            const uint32_t w = *p;
+                            *p = 0u;
+                            const float sc = s_scale[sc0[u] + static_cast<uint32_t>(t) * 32u];
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) v[e] = __fdiv_rn(v[e], a.div);
-                    }
-                    if (c + 4 <= mm) {
-                        *reinterpret_cast<float4*>(gp) = make_float4(v[0], v[1], v[2], v[3]);
-                    } else {
-                        gp[0] = v[0];
-                        if (c + 1 < mm) gp[1] = v[1];
-                        if (c + 2 < mm) gp[2] = v[2];
+                            for (int e = 0; e < 4; ++e) v[u][e] = __fadd_rn(v[u][e], side_value(w >> (8 * e), sc));
+                        }
+                        if (c[u] >= mm[u]) continue;
+                        if (divide) {
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) v[u][e] = __fdiv_rn(v[u][e], a.div);
+                        }
+                        if (c[u] + 4 <= mm[u]) {
+                            *reinterpret_cast<float4*>(gp[u]) = make_float4(v[u][0], v[u][1], v[u][2], v[u][3]);
+                        } else {
+                            gp[u][0] = v[u][0];
+                            if (c[u] + 1 < mm[u]) gp[u][1] = v[u][1];
+                            if (c[u] + 2 < mm[u]) gp[u][2] = v[u][2];
+                        }
                     }
                 }
                 __syncthreads();  // the ring's words of [lo, hi) are clear again
