@@ -98,7 +98,8 @@ def profile_step(args):
     qsgd_encode, qsgd_decode and qsgd_decode_accumulate (K = 1); c4 the sixteen
     senders' encodes and the K = 16 qsgd_decode_accumulate; with --bbit, the b-bit
     encode, decode and decode-accumulate on c2.  Launches per pass: two for each
-    encode on the two-launch shapes, one for each decode."""
+    encode on the two-launch shapes, two for the decode of buckets past 1024
+    coordinates (a fill, then the records), one for every other decode."""
     import torch
     from quantized_gradient_compression_b200 import binding as B
     from quantized_gradient_compression_b200 import workloads as W

@@ -99,10 +99,11 @@ struct RowReader {
     }
 };
 
-// A record the table does not hold, bit by bit: false when it is malformed (or its
-// level exceeds s).
-__device__ __forceinline__ bool slow_record(RowReader& r, uint32_t s, uint32_t& gap, uint32_t& sign, uint32_t& k) {
-    if (!r.omega(gap) || r.left <= 0 || gap > 0xFFFFu) return false;
+// A record the table does not hold, bit by bit: false when it is malformed (its gap
+// beyond the bucket length d, or its level beyond s).
+__device__ __forceinline__ bool slow_record(RowReader& r, uint32_t s, uint32_t d, uint32_t& gap, uint32_t& sign,
+                                            uint32_t& k) {
+    if (!r.omega(gap) || r.left <= 0 || gap > d) return false;
     sign = r.peek() >> 31;
     r.advance(1);
     return r.omega(k) && k <= s;
@@ -135,13 +136,12 @@ __device__ __forceinline__ void load_row(const DecodeArgs& a, uint64_t bb, int l
 
 // One parse step through the whole-record table (byte codes): up to two table
 // entries, each up to two records.  The 32 bits at the cursor hold both 12-bit
-// windows (the first entry's records take at most 12 bits); a record is taken only
-// when it ends inside the bucket.  A record longer than the window whose gap code
-// fits it (gap <= 63) is read as the entry's gap, the sign and a level from the
-// level table (k <= 15 and k <= s); that record ends within 20 bits of the cursor.
-// put(index, code) stores a record's code (sign << 7 | k) at its bucket-local index.
-// Returns false, having read nothing, when the record at the cursor is neither (the
-// bit-serial path takes it).
+// windows (the first entry's records take at most 12 bits, so a step moves at most
+// 60 columns); a record is taken only when it ends inside the bucket.  A record
+// longer than the window whose gap's code fits it goes through near_long_record
+// (gap <= 63, k <= 15 and k <= s; at most 63 columns).  put(index, code) stores a
+// record's code (sign << 7 | k) at its bucket-local index.  Returns false, having
+// read nothing, when the record at the cursor is neither (far_record takes it).
 template <class Put>
 __device__ __forceinline__ bool rows_table_step(RowReader& r, const uint32_t* lut, const uint8_t* klut, uint32_t s,
                                                 uint32_t& next, const Put& put) {
@@ -149,13 +149,12 @@ __device__ __forceinline__ bool rows_table_step(RowReader& r, const uint32_t* lu
     const uint32_t e = lut[w >> (32 - kLutBits)];
     const uint32_t len1 = e & 15u;
     if (len1 == 0u) {
-        const uint32_t gl = (e >> 4) & 15u;
-        const uint32_t kc = klut[(w << (gl + 1u)) >> (32 - kKLutBits)];
-        const uint32_t kl = kc & 15u;
-        if (gl == 0u || kl == 0u || (kc >> 4) > s) return false;
-        next += (e >> 8) & 63u;
-        put(next - 1u, (((w << gl) >> 31) << 7) | (kc >> 4));
-        r.advance(gl + 1u + kl);
+        uint32_t gap = 0, code = 0;
+        const uint32_t len = near_long_record(w, e, klut, gap, code);
+        if (len == 0u || (code & 0x7Fu) > s) return false;
+        next += gap;
+        put(next - 1u, code);
+        r.advance(len);
         return true;
     }
     const uint32_t len2 = (e >> 4) & 15u;
@@ -188,18 +187,36 @@ __device__ __forceinline__ bool rows_table_step(RowReader& r, const uint32_t* lu
     return true;
 }
 
+// A record the table step does not take: far_long_record (gap < 2^16, k <= 15),
+// else bit by bit.  Returns false when it is malformed (gap beyond d, level beyond
+// s); else its gap, sign and level, the reader past it.
+__device__ __forceinline__ bool far_record(RowReader& r, const uint8_t* plut, const uint8_t* klut, uint32_t s,
+                                           uint32_t d, uint32_t& gap, uint32_t& sign, uint32_t& k) {
+    uint32_t code = 0;
+    const uint32_t len = far_long_record(r.peek(), plut, klut, gap, code);
+    if (len != 0u && (code & 0x7Fu) <= s) {
+        r.advance(len);
+        sign = code >> 7;
+        k = code & 0x7Fu;
+        return true;
+    }
+    return slow_record(r, s, d, gap, sign, k);
+}
+
 template <int V, bool kAcc>
 __global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows(const __grid_constant__ DecodeArgs a,
                                                                    uint32_t stride_w) {
     extern __shared__ __align__(16) uint32_t smem[];
     uint32_t* const lut = smem;
     uint8_t* const klut = reinterpret_cast<uint8_t*>(smem + kLutSize);
+    uint8_t* const plut = reinterpret_cast<uint8_t*>(smem + kLutSize + kKLutWords);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int W = blockDim.x >> 5;
-    uint32_t* const rows = smem + kLutSize + kKLutWords + static_cast<uint32_t>(warp) * 32u * stride_w;
+    uint32_t* const rows = smem + kLutSize + kSmallLutWords + static_cast<uint32_t>(warp) * 32u * stride_w;
     uint8_t* const myrow = reinterpret_cast<uint8_t*>(rows + static_cast<uint32_t>(lane) * stride_w);
     rows_lut_fill(lut, a.s, tid, blockDim.x);
     k_lut_fill(klut, tid, blockDim.x);
+    p_lut_fill(plut, tid, blockDim.x);
     __syncthreads();
     const StreamRef st = a.streams[0];
     const float fs = __uint2float_rn(a.s);
@@ -262,9 +279,9 @@ __global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows(const __grid_c
                 const auto put = [&](uint32_t idx, uint32_t code) { myrow[min(idx, d)] = static_cast<uint8_t>(code); };
                 if (!rows_table_step(r, lut, klut, a.s, next, put)) {
                     uint32_t gap = 0, sign = 0, k = 0;
-                    if (slow_record(r, a.s, gap, sign, k)) {
+                    if (far_record(r, plut, klut, a.s, d, gap, sign, k)) {
                         next += gap;
-                        myrow[min(next - 1u, d)] = row_code<uint8_t>(sign, k);
+                        put(next - 1u, row_code<uint8_t>(sign, k));
                     } else {
                         bad = true;
                         r.left = 0;
@@ -448,7 +465,7 @@ __global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows_ring(const __g
                 }
                 // a record the table does not hold, bit by bit
                 uint32_t gap = 0, sign = 0, k = 0;
-                if (slow_record(r, a.s, gap, sign, k)) {
+                if (slow_record(r, a.s, a.d, gap, sign, k)) {
                     next += gap;
                     const uint32_t idx = min(next - 1u, d);
                     if (idx >= hi + kRSeg) {
@@ -804,10 +821,9 @@ __global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows_multi(const __
 // The first add makes a -0.0 output +0.0 as the first stream's add would; after it
 // adding a zero code's +0 leaves v as it is, as the sum in stream order does.  The
 // add clears the codes it reads for the ring's next turn; the output is read and
-// written once per chunk.  A step of table records moves at most 60 columns and a
-// long record through the level table at most 63, so the records of a lane still
-// short of the segment's end land in the ring; a bit-serial one further ahead waits
-// in registers until its segment.  Segments of 64 columns keep a CTA at 51 KB of
+// written once per chunk.  A step of table records moves at most 60 columns, so the
+// records of a lane still short of the segment's end land in the ring; a longer
+// record further ahead waits in registers until its segment.  Segments of 64 columns keep a CTA at 51 KB of
 // shared memory; three CTAs an SM (76 registers a thread) measured faster than four
 // (64 registers, with spills) or two (segments of 128 columns).
 // ---------------------------------------------------------------------------
@@ -820,8 +836,7 @@ constexpr uint32_t kSRing = 2 * kSSeg;            // codes (bytes) a ring row
 constexpr uint32_t kSStride = kSRing / 4 + 1;     // words a ring row: 1 mod 32, rows on different banks
 constexpr uint32_t kSSegWords = kSSeg / 4;        // words of a row's segment
 constexpr uint32_t kSRowsPerWarp = 32 / kSSegWords;  // rows a warp's 32 threads add at once
-// (a step of table records moves at most 60 columns, a long record through the
-// level table at most 63)
+// (a step of table records moves at most 60 columns)
 static_assert(kSSeg == 64 || kSSeg == 128, "a segment holds a step of records and a warp whole rows");
 static_assert((32 * kSSegWords) % (2 * 32 * kSideWarps) == 0, "a group's items come in pairs a thread");
 
@@ -840,12 +855,14 @@ __global__ void __launch_bounds__(32 * kSideWarps, QSGD_SIDE_MINB) decode_rows_s
     constexpr int kThreads = 32 * kSideWarps;
     uint32_t* const lut = smem;
     uint8_t* const klut = reinterpret_cast<uint8_t*>(smem + kLutSize);
-    float* const s_scale = reinterpret_cast<float*>(smem + kLutSize + kKLutWords);  // [warp][lane]
-    uint32_t* const rings = smem + kLutSize + kKLutWords + kThreads;                // [warp][row][kSStride]
+    uint8_t* const plut = reinterpret_cast<uint8_t*>(smem + kLutSize + kKLutWords);
+    float* const s_scale = reinterpret_cast<float*>(smem + kLutSize + kSmallLutWords);  // [warp][lane]
+    uint32_t* const rings = smem + kLutSize + kSmallLutWords + kThreads;                // [warp][row][kSStride]
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     uint8_t* const myrow = reinterpret_cast<uint8_t*>(rings + static_cast<uint32_t>(tid) * kSStride);
     rows_lut_fill(lut, a.s, tid, kThreads);
     k_lut_fill(klut, tid, kThreads);
+    p_lut_fill(plut, tid, kThreads);
     for (uint32_t q = static_cast<uint32_t>(tid); q < kThreads * kSStride; q += kThreads) rings[q] = 0u;
     __syncthreads();
     const float fs = __uint2float_rn(a.s);
@@ -908,9 +925,9 @@ __global__ void __launch_bounds__(32 * kSideWarps, QSGD_SIDE_MINB) decode_rows_s
             bool pend = false;  // a bit-serial record beyond the ring, held here
             uint32_t pidx = 0, pcode = 0;
             uint32_t it = 0;  // parse steps over the whole bucket (an explicit bound)
-            const auto put = [&](uint32_t idx, uint32_t code) {
-                myrow[idx & (kSRing - 1u)] = static_cast<uint8_t>(code);
-            };
+            // a table step's record into the ring (it lies less than 64 columns past the
+            // segment's end)
+            const auto put = [&](uint32_t idx, uint32_t code) { myrow[idx & (kSRing - 1u)] = static_cast<uint8_t>(code); };
             for (uint32_t lo = 0; lo < d; lo += kSSeg) {
                 const uint32_t hi = lo + kSSeg;
                 if (mine) {
@@ -930,9 +947,10 @@ __global__ void __launch_bounds__(32 * kSideWarps, QSGD_SIDE_MINB) decode_rows_s
                             continue;
                         }
                         if (!act || rows_table_step(r, lut, klut, a.s, next, put)) continue;
-                        // a record the table does not hold, bit by bit
+                        // a longer record; held here when it lies past the ring (the lane
+                        // then waits for its segment)
                         uint32_t gap = 0, sign = 0, k = 0;
-                        if (slow_record(r, a.s, gap, sign, k)) {
+                        if (far_record(r, plut, klut, a.s, d, gap, sign, k)) {
                             next += gap;
                             const uint32_t idx = min(next - 1u, d);
                             if (idx >= hi + kSSeg) {
@@ -1029,134 +1047,183 @@ __global__ void __launch_bounds__(32 * kSideWarps, QSGD_SIDE_MINB) decode_rows_s
 }
 
 // ---------------------------------------------------------------------------
-// Large buckets (d > 1024): a CTA takes 32 buckets.  All its threads first write the
-// buckets' output range with 16-byte stores where it is aligned: zeros (decode), or
-// the output + 0 (decode-accumulate; +0 turns -0.0 into +0.0 as the add of a zero
-// term does).  After a CTA barrier, lane L of warp 0 parses bucket 32g + L of every
-// stream in order and stores each record's value (decode) or adds it (accumulate)
-// at its coordinate.  The outputs of such gradients are mostly zeros, so the fill
-// carries the traffic; the records are few.
+// Large buckets (d > 1024).  The outputs of such gradients are mostly zeros (c3:
+// 0.107 bits a coordinate), so writing the output carries the traffic and the records
+// are few.  The output is first written whole with 16-byte stores where it is
+// aligned: zeros (decode), or the output + 0 (decode-accumulate; +0 turns -0.0 into
+// +0.0 as the add of a zero term does).  Then one lane a bucket parses the bucket of
+// every stream in order and stores each record's value (decode) or adds it
+// (accumulate) at its coordinate.
+//   - decode: sparse_fill over the whole output (every SM, no barrier), then
+//     sparse_records, a lane a bucket;
+//   - decode-accumulate: decode_sparse_acc, a CTA a group of kSparseGroup buckets, its
+//     threads adding +0 to the group's output and, after a CTA barrier, lane L of
+//     warp 0 parsing bucket L of the group, whose output the CTA has just brought
+//     into L2.
 // ---------------------------------------------------------------------------
+
+// The records of bucket b of every stream onto its output row (the row written
+// before): a record's value is stored, or added with kAcc.  Returns false when a
+// stream's bucket is malformed.
 template <bool kAcc>
-__global__ void __launch_bounds__(kSparseBlock) decode_sparse(const __grid_constant__ DecodeArgs a) {
-    __shared__ __align__(16) uint32_t lut[kLutSize];
-    const int tid = threadIdx.x, lane = tid & 31;
-    rows_lut_fill(lut, a.s, tid, kSparseBlock);
-    __syncthreads();
+__device__ __forceinline__ bool sparse_bucket(const DecodeArgs& a, const uint32_t* lut, const uint8_t* plut,
+                                              const uint8_t* klut, uint64_t b) {
     const float fs = __uint2float_rn(a.s);
+    const uint32_t m = static_cast<uint32_t>(min(static_cast<uint64_t>(a.d), a.n - b * a.d));
+    float* const row = a.out + b * a.d;
+    bool bad = false;
+    for (int j = 0; j < a.K; ++j) {
+        const StreamRef st = a.streams[j];
+        const uint64_t begin = st.offsets[b];
+        const uint64_t end = st.offsets[b + 1];
+        if (!(end >= begin && end - begin >= 32 && end <= st.num_words * 32 && end - begin < (1ull << 31))) {
+            bad = true;
+            continue;
+        }
+        RowReader r;
+        r.init(st.words, st.num_words, begin, static_cast<uint32_t>(end - begin));
+        const uint32_t nbits = r.peek();
+        r.advance(32);
+        const float norm = __uint_as_float(nbits);
+        float scale = 0.f;
+        if (nbits == 0) {
+            bad = bad || r.left != 0;
+            continue;
+        } else if (!(isfinite(norm) && norm > 0.f)) {
+            bad = true;
+            continue;
+        }
+        scale = __fdiv_rn(norm, fs);
+        if (!(scale > 0.f) && r.left != 0) {  // a zero scale carries no records
+            bad = true;
+            continue;
+        }
+        uint32_t next = 0;
+        // the records: up to two table entries a step, each up to two records
+        // (a second record or entry only when it ends inside the bucket)
+        bool ok = true;
+        auto put = [&](uint32_t gap, uint32_t sign, uint32_t k) {
+            next += gap;
+            if (next > m) {
+                ok = false;
+                return;
+            }
+            const float q = __fmul_rn(scale, __uint2float_rn(k));
+            const float v = sign ? -q : q;
+            row[next - 1] = kAcc ? __fadd_rn(row[next - 1], v) : v;
+        };
+        for (uint32_t it = 0; r.left > 0 && ok; ++it) {
+            if (it >= kParseGuard) {
+                ok = false;
+                break;
+            }
+            const uint32_t w = r.peek();
+            const uint32_t e = lut[w >> (32 - kLutBits)];
+            const uint32_t len1 = e & 15u;
+            if (len1 == 0u) {  // a record longer than the window
+                // (such buckets are sparse: the gap's code is mostly past the window)
+                uint32_t gap = 0, code = 0, sign = 0, k = 0;
+                uint32_t len = far_long_record(w, plut, klut, gap, code);
+                if (len == 0u) len = near_long_record(w, e, klut, gap, code);
+                if (len != 0u && (code & 0x7Fu) <= a.s) {
+                    r.advance(len);
+                    sign = code >> 7;
+                    k = code & 0x7Fu;
+                } else if (!slow_record(r, a.s, a.d, gap, sign, k)) {
+                    ok = false;
+                    break;
+                }
+                put(gap, sign, k);
+                continue;
+            }
+            const uint32_t len2 = (e >> 4) & 15u;
+            const bool two = static_cast<int32_t>(len2) <= r.left;
+            uint32_t used = two ? len2 : len1;
+            put((e >> 8) & 15u, (e >> 23) & 1u, (e >> 16) & 0x7Fu);  // table codes: sign << 7 | k
+            const uint32_t c2 = e >> 24;
+            if (ok && two && c2 != 0u) put((e >> 12) & 15u, c2 >> 7, c2 & 0x7Fu);
+            if (ok && two) {
+                const uint32_t f = lut[(w << used) >> (32 - kLutBits)];
+                const uint32_t flen1 = f & 15u;
+                if (flen1 != 0u && static_cast<int32_t>(used + flen1) <= r.left) {
+                    const uint32_t flen2 = (f >> 4) & 15u;
+                    const bool ftwo = static_cast<int32_t>(used + flen2) <= r.left;
+                    put((f >> 8) & 15u, (f >> 23) & 1u, (f >> 16) & 0x7Fu);
+                    const uint32_t fc2 = f >> 24;
+                    if (ok && ftwo && fc2 != 0u) put((f >> 12) & 15u, fc2 >> 7, fc2 & 0x7Fu);
+                    used += ftwo ? flen2 : flen1;
+                }
+            }
+            r.advance(used);
+        }
+        if (!ok) bad = true;
+        if (r.left != 0) bad = true;
+    }
+    return !bad;
+}
+
+// Writes out[c0, c1) (out 16-byte aligned): zeros, or out + 0 with kAcc; thread t of
+// nthreads takes every nthreads-th float4 of the aligned body.
+template <bool kAcc>
+__device__ __forceinline__ void sparse_fill_range(float* out, uint64_t c0, uint64_t c1, uint64_t t, uint64_t nthreads) {
+    const uint64_t head = min(c1, (c0 + 3) & ~uint64_t(3));  // aligned start of the body
+    const uint64_t tail = max(head, c1 & ~uint64_t(3));
+    for (uint64_t i = c0 + t; i < head; i += nthreads) out[i] = kAcc ? __fadd_rn(out[i], 0.0f) : 0.0f;
+    for (uint64_t i = tail + t; i < c1; i += nthreads) out[i] = kAcc ? __fadd_rn(out[i], 0.0f) : 0.0f;
+    for (uint64_t i = head + 4 * t; i < tail; i += 4 * nthreads) {
+        float4* p4 = reinterpret_cast<float4*>(out + i);
+        if constexpr (kAcc) {
+            float4 v = *p4;
+            v.x = __fadd_rn(v.x, 0.0f);
+            v.y = __fadd_rn(v.y, 0.0f);
+            v.z = __fadd_rn(v.z, 0.0f);
+            v.w = __fadd_rn(v.w, 0.0f);
+            *p4 = v;
+        } else {
+            __stcs(p4, make_float4(0.f, 0.f, 0.f, 0.f));
+        }
+    }
+}
+
+// The decode's fill: zeros over the whole output.
+__global__ void __launch_bounds__(kSparseBlock) sparse_fill(float* out, uint64_t n) {
+    sparse_fill_range<false>(out, 0, n, static_cast<uint64_t>(blockIdx.x) * kSparseBlock + threadIdx.x,
+                             static_cast<uint64_t>(gridDim.x) * kSparseBlock);
+}
+
+// The decode's records: thread t of the grid takes bucket t.
+__global__ void __launch_bounds__(kSparseRecBlock) sparse_records(const __grid_constant__ DecodeArgs a) {
+    __shared__ __align__(16) uint32_t lut[kLutSize];
+    __shared__ __align__(16) uint8_t plut[1 << kPLutBits];
+    __shared__ __align__(16) uint8_t klut[1 << kKLutBits];
+    rows_lut_fill(lut, a.s, threadIdx.x, kSparseRecBlock);
+    p_lut_fill(plut, threadIdx.x, kSparseRecBlock);
+    k_lut_fill(klut, threadIdx.x, kSparseRecBlock);
+    __syncthreads();
+    const uint64_t b = static_cast<uint64_t>(blockIdx.x) * kSparseRecBlock + threadIdx.x;
+    if (b < a.nb && !sparse_bucket<false>(a, lut, plut, klut, b)) atomicOr(a.status, QSGD_ST_BAD_STREAM);
+}
+
+// Decode-accumulate: a CTA a group of kSparseGroup buckets, the fill by all its
+// threads, then the records by lanes 0 .. kSparseGroup - 1 of warp 0.
+__global__ void __launch_bounds__(kSparseBlock) decode_sparse_acc(const __grid_constant__ DecodeArgs a) {
+    __shared__ __align__(16) uint32_t lut[kLutSize];
+    __shared__ __align__(16) uint8_t plut[1 << kPLutBits];
+    __shared__ __align__(16) uint8_t klut[1 << kKLutBits];
+    const int tid = threadIdx.x;
+    rows_lut_fill(lut, a.s, tid, kSparseBlock);
+    p_lut_fill(plut, tid, kSparseBlock);
+    k_lut_fill(klut, tid, kSparseBlock);
+    __syncthreads();
     const uint64_t d = a.d;
-    const uint64_t ngroups = (a.nb + 31) / 32;
+    const uint64_t ngroups = (a.nb + kSparseGroup - 1) / kSparseGroup;
     for (uint64_t g = blockIdx.x; g < ngroups; g += gridDim.x) {
-        // --- the fill: [g*32*d, min(n, (g+1)*32*d)) ----------------------------------
-        const uint64_t c0 = g * 32 * d, c1 = min(a.n, (g + 1) * 32 * d);
-        float* const out = a.out;
-        const uint64_t head = min(c1, (c0 + 3) & ~uint64_t(3));  // aligned start of the body (out is 16-byte aligned)
-        const uint64_t tail = max(head, c1 & ~uint64_t(3));
-        for (uint64_t i = c0 + tid; i < head; i += kSparseBlock) out[i] = kAcc ? __fadd_rn(out[i], 0.0f) : 0.0f;
-        for (uint64_t i = tail + tid; i < c1; i += kSparseBlock) out[i] = kAcc ? __fadd_rn(out[i], 0.0f) : 0.0f;
-        for (uint64_t i = head + 4 * static_cast<uint64_t>(tid); i < tail; i += 4 * kSparseBlock) {
-            float4* p4 = reinterpret_cast<float4*>(out + i);
-            if constexpr (kAcc) {
-                float4 v = *p4;
-                v.x = __fadd_rn(v.x, 0.0f);
-                v.y = __fadd_rn(v.y, 0.0f);
-                v.z = __fadd_rn(v.z, 0.0f);
-                v.w = __fadd_rn(v.w, 0.0f);
-                *p4 = v;
-            } else {
-                __stcs(p4, make_float4(0.f, 0.f, 0.f, 0.f));
-            }
-        }
+        sparse_fill_range<true>(a.out, g * kSparseGroup * d, min(a.n, (g + 1) * kSparseGroup * d),
+                                static_cast<uint64_t>(tid), kSparseBlock);
         __syncthreads();
-        // --- the records: lane L of warp 0 takes bucket 32g + L of every stream -------
-        if (tid < 32) {
-            const uint64_t b = g * 32 + lane;
-            const bool live = b < a.nb;
-            const uint32_t m = live ? static_cast<uint32_t>(min(d, a.n - b * d)) : 0u;
-            float* const row = out + b * d;
-            bool bad = false;
-            for (int j = 0; j < a.K && live; ++j) {
-                const StreamRef st = a.streams[j];
-                const uint64_t begin = st.offsets[b];
-                const uint64_t end = st.offsets[b + 1];
-                if (!(end >= begin && end - begin >= 32 && end <= st.num_words * 32 && end - begin < (1ull << 31))) {
-                    bad = true;
-                    continue;
-                }
-                RowReader r;
-                r.init(st.words, st.num_words, begin, static_cast<uint32_t>(end - begin));
-                const uint32_t nbits = r.peek();
-                r.advance(32);
-                const float norm = __uint_as_float(nbits);
-                float scale = 0.f;
-                if (nbits == 0) {
-                    bad = bad || r.left != 0;
-                    continue;
-                } else if (!(isfinite(norm) && norm > 0.f)) {
-                    bad = true;
-                    continue;
-                }
-                scale = __fdiv_rn(norm, fs);
-                if (!(scale > 0.f) && r.left != 0) {  // a zero scale carries no records
-                    bad = true;
-                    continue;
-                }
-                uint32_t next = 0;
-                // the records: up to two table entries a step, each up to two records
-                // (a second record or entry only when it ends inside the bucket)
-                bool ok = true;
-                auto put = [&](uint32_t gap, uint32_t sign, uint32_t k) {
-                    next += gap;
-                    if (next > m) {
-                        ok = false;
-                        return;
-                    }
-                    const float q = __fmul_rn(scale, __uint2float_rn(k));
-                    const float v = sign ? -q : q;
-                    row[next - 1] = kAcc ? __fadd_rn(row[next - 1], v) : v;
-                };
-                for (uint32_t it = 0; r.left > 0 && ok; ++it) {
-                    if (it >= kParseGuard) {
-                        ok = false;
-                        break;
-                    }
-                    const uint32_t w = r.peek();
-                    const uint32_t e = lut[w >> (32 - kLutBits)];
-                    const uint32_t len1 = e & 15u;
-                    if (len1 == 0u) {  // a record the table does not hold, bit by bit
-                        uint32_t gap, sign, k;
-                        if (!slow_record(r, a.s, gap, sign, k)) {
-                            ok = false;
-                            break;
-                        }
-                        put(gap, sign, k);
-                        continue;
-                    }
-                    const uint32_t len2 = (e >> 4) & 15u;
-                    const bool two = static_cast<int32_t>(len2) <= r.left;
-                    uint32_t used = two ? len2 : len1;
-                    put((e >> 8) & 15u, (e >> 23) & 1u, (e >> 16) & 0x7Fu);  // table codes: sign << 7 | k
-                    const uint32_t c2 = e >> 24;
-                    if (ok && two && c2 != 0u) put((e >> 12) & 15u, c2 >> 7, c2 & 0x7Fu);
-                    if (ok && two) {
-                        const uint32_t f = lut[(w << used) >> (32 - kLutBits)];
-                        const uint32_t flen1 = f & 15u;
-                        if (flen1 != 0u && static_cast<int32_t>(used + flen1) <= r.left) {
-                            const uint32_t flen2 = (f >> 4) & 15u;
-                            const bool ftwo = static_cast<int32_t>(used + flen2) <= r.left;
-                            put((f >> 8) & 15u, (f >> 23) & 1u, (f >> 16) & 0x7Fu);
-                            const uint32_t fc2 = f >> 24;
-                            if (ok && ftwo && fc2 != 0u) put((f >> 12) & 15u, fc2 >> 7, fc2 & 0x7Fu);
-                            used += ftwo ? flen2 : flen1;
-                        }
-                    }
-                    r.advance(used);
-                }
-                if (!ok) bad = true;
-                if (r.left != 0) bad = true;
-            }
-            if (bad) atomicOr(a.status, QSGD_ST_BAD_STREAM);
-        }
+        const uint64_t b = g * kSparseGroup + static_cast<uint64_t>(tid);
+        if (tid < kSparseGroup && b < a.nb && !sparse_bucket<true>(a, lut, plut, klut, b))
+            atomicOr(a.status, QSGD_ST_BAD_STREAM);
         __syncthreads();
     }
 }
@@ -1180,9 +1247,9 @@ cudaError_t launch_row_kernel(Kernel kernel, bool& attr_done, const DecodeArgs& 
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     const size_t per_warp = static_cast<size_t>(32) * stride * sizeof(uint32_t);
-    // the record table and the level table (the ring kernel uses the first half of
-    // the record table's room for its omega table, and the level table's not at all)
-    const size_t lut_bytes = static_cast<size_t>(kLutSize + kKLutWords) * sizeof(uint32_t);
+    // the record table and the small tables (the ring kernel uses the first half of
+    // the record table's room for its omega table, and the small tables' not at all)
+    const size_t lut_bytes = static_cast<size_t>(kLutSize + kSmallLutWords) * sizeof(uint32_t);
     const int W_fit = static_cast<int>(std::min<size_t>(kRowsMaxWarps, (static_cast<size_t>(optin) - lut_bytes - 1024) / per_warp));
     if (W_fit < 1) return cudaErrorInvalidConfiguration;
     const uint64_t groups = (a.nb + 31) / 32;
@@ -1250,7 +1317,7 @@ cudaError_t launch_rows_multi(const DecodeArgs& a, cudaStream_t stream) {
 cudaError_t launch_rows_side(const DecodeArgs& a, cudaStream_t stream) {
     constexpr int kThreads = 32 * kSideWarps;
     const size_t smem =
-        (static_cast<size_t>(kLutSize) + kKLutWords + kThreads + static_cast<size_t>(kThreads) * kSStride) * sizeof(uint32_t);
+        (static_cast<size_t>(kLutSize) + kSmallLutWords + kThreads + static_cast<size_t>(kThreads) * kSStride) * sizeof(uint32_t);
     static bool attr_set[64] = {};
     int dev = 0, sms = 0, per_sm = 0;
     cudaGetDevice(&dev);
@@ -1273,12 +1340,18 @@ cudaError_t launch_sparse(const DecodeArgs& a, bool accumulate, cudaStream_t str
     int dev = 0, sms = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const uint64_t groups = (a.nb + 31) / 32;
+    if (!accumulate) {  // the fill over every SM, then a lane a bucket
+        const uint64_t fill_threads = (a.n + 3) / 4;
+        const uint64_t fill_blocks = std::max<uint64_t>(
+            1, std::min<uint64_t>((fill_threads + kSparseBlock - 1) / kSparseBlock, static_cast<uint64_t>(sms) * 8));
+        sparse_fill<<<static_cast<unsigned>(fill_blocks), kSparseBlock, 0, stream>>>(a.out, a.n);
+        const uint64_t rec_blocks = (a.nb + kSparseRecBlock - 1) / kSparseRecBlock;
+        sparse_records<<<static_cast<unsigned>(rec_blocks), kSparseRecBlock, 0, stream>>>(a);
+        return cudaGetLastError();
+    }
+    const uint64_t groups = (a.nb + kSparseGroup - 1) / kSparseGroup;
     const uint64_t blocks = std::max<uint64_t>(1, std::min<uint64_t>(groups, static_cast<uint64_t>(sms) * 8));
-    if (accumulate)
-        decode_sparse<true><<<static_cast<unsigned>(blocks), kSparseBlock, 0, stream>>>(a);
-    else
-        decode_sparse<false><<<static_cast<unsigned>(blocks), kSparseBlock, 0, stream>>>(a);
+    decode_sparse_acc<<<static_cast<unsigned>(blocks), kSparseBlock, 0, stream>>>(a);
     return cudaGetLastError();
 }
 

@@ -79,6 +79,8 @@ constexpr uint32_t kRowsMaxS = 32767;
 // Large-bucket decoder (d > kRowsMaxD, 16-byte aligned output): a CTA fills the
 // output of 32 buckets, then one lane per bucket stores the records.
 constexpr int kSparseBlock = 256;
+constexpr int kSparseGroup = 8;     // buckets a CTA of the large-bucket decode-accumulate takes at once
+constexpr int kSparseRecBlock = 64;  // threads (buckets) a CTA of the large-bucket decode's records
 
 constexpr int kDecodeBlock = 128;
 constexpr int kMaxStreamsPerLaunch = 16;  // decode-accumulate streams per launch

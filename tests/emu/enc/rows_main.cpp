@@ -1,5 +1,6 @@
 // Runs the row decoders (decode_rows, decode_rows_ring, decode_rows_multi,
-// decode_rows_side, decode_sparse), compiled for the host under block_emu.h, with all
+// decode_rows_side, and for large buckets sparse_fill with sparse_records or
+// decode_sparse_acc), compiled for the host under block_emu.h, with all
 // their CTAs at once.
 // argv: dir accumulate grid warps [K [mean [side]]]
 // dir holds params.bin (u64 n, d, s), w<j>.bin (u32 stream words), o<j>.bin
@@ -60,7 +61,7 @@ template <class T>
 static void run_t(const qsgd::DecodeArgs& a, bool acc, unsigned grid, unsigned W) {
     if constexpr (sizeof(T) == 2) {
         const uint32_t stride = qsgd::ring_stride_words();
-        const size_t smem = 4 * (size_t)(qsgd::kLutSize + qsgd::kKLutWords) + (size_t)W * 32 * stride * 4;
+        const size_t smem = 4 * (size_t)(qsgd::kLutSize + qsgd::kSmallLutWords) + (size_t)W * 32 * stride * 4;
         if (acc)
             run_grid(grid, 32 * W, smem, [&] { qsgd::decode_rows_ring<true>(a, stride); });
         else
@@ -68,7 +69,7 @@ static void run_t(const qsgd::DecodeArgs& a, bool acc, unsigned grid, unsigned W
         return;
     }
     const uint32_t stride = qsgd::rows_stride_words(a.d);
-    const size_t smem = 4 * (size_t)(qsgd::kLutSize + qsgd::kKLutWords) + (size_t)W * 32 * stride * 4;
+    const size_t smem = 4 * (size_t)(qsgd::kLutSize + qsgd::kSmallLutWords) + (size_t)W * 32 * stride * 4;
     switch (qsgd::fast_v(a.d)) {
         case 1: run_v<1>(a, acc, grid, W, stride, smem); break;
         case 2: run_v<2>(a, acc, grid, W, stride, smem); break;
@@ -84,7 +85,7 @@ static void run_multi(qsgd::DecodeArgs a, const std::vector<std::vector<unsigned
                       const std::vector<std::vector<unsigned char>>& os, bool mean, unsigned grid, unsigned W,
                       bool side) {
     const int K = (int)ws.size();
-    const size_t smem = side ? (qsgd::kLutSize + qsgd::kKLutWords + 32 * qsgd::kSideWarps +
+    const size_t smem = side ? (qsgd::kLutSize + qsgd::kSmallLutWords + 32 * qsgd::kSideWarps +
                                 (size_t)32 * qsgd::kSideWarps * qsgd::kSStride) * 4
                              : (qsgd::kLutSize + 256) * 2 + (size_t)W * (sizeof(qsgd::MsState) + 32 * qsgd::kMTile * 4);
     for (int j0 = 0; j0 < K; j0 += qsgd::kMaxStreamsPerLaunch) {
@@ -144,10 +145,14 @@ int main(int argc, char** argv) {
                 a.streams[j].num_words = ws[j0 + j].size() / 4;
                 a.streams[j].offsets = reinterpret_cast<const uint64_t*>(os[j0 + j].data());
             }
-            if (acc)
-                run_grid(grid, qsgd::kSparseBlock, 0, [&] { qsgd::decode_sparse<true>(a); });
-            else
-                run_grid(grid, qsgd::kSparseBlock, 0, [&] { qsgd::decode_sparse<false>(a); });
+            if (acc) {
+                run_grid(grid, qsgd::kSparseBlock, 0, [&] { qsgd::decode_sparse_acc(a); });
+            } else {  // the fill (grid CTAs, grid-stride), then a lane a bucket
+                run_grid(grid, qsgd::kSparseBlock, 0, [&] { qsgd::sparse_fill(a.out, a.n); });
+                if (g_emu_error) return 4;
+                run_grid((unsigned)((nb + qsgd::kSparseRecBlock - 1) / qsgd::kSparseRecBlock), qsgd::kSparseRecBlock, 0,
+                         [&] { qsgd::sparse_records(a); });
+            }
             if (g_emu_error) return 4;
         }
         spit(dir + "/out.bin", out.data(), 4 * n);

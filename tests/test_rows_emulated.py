@@ -423,3 +423,31 @@ def test_large_bucket_decoder_matches_oracle(rows_exe, tmp_path, oracle_lib, n, 
         ref, rst = oracle_lib.decode(streams[0][0], streams[0][1], n, d, s)
     assert rst == 0
     assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("acc", [False, True])
+def test_large_bucket_decoder_gap_boundaries(rows_exe, tmp_path, oracle_lib, acc):
+    """Gaps at the edges of the long-record path (the gap-prefix table reads at most
+    one 16-bit group): 63, 64, 2^15 - 1, 2^15, 2^16 - 1 take it; 2^16 and more take
+    the bit-serial path.  Levels 15 (the level table's last) and 16 (past it)."""
+    d, s = 70_000, 20
+    gaps = [63, 64, 2 ** 15 - 1, 2 ** 15, 2 ** 16 - 1, 2 ** 16, 69_000]
+    n = len(gaps) * d
+    v = np.zeros(n, np.float32)
+    for b, gap in enumerate(gaps):
+        v[b * d] = 1.0  # the first record: gap 1
+        v[b * d + gap] = -0.75 if b % 2 else 0.75
+    words, offsets, _, st = oracle_lib.encode(v, d, s, seed=3)
+    assert st == 0
+    base = _base(n, d, acc)
+    got, status = _run(rows_exe, tmp_path, words, offsets, n, d, s, acc, 2, 1, base)
+    assert status == 0
+    if acc:
+        ref = base.copy()
+        _, rst = oracle_lib.decode_accumulate([(words, offsets)], n, d, s, ref)
+    else:
+        ref, rst = oracle_lib.decode(words, offsets, n, d, s)
+    assert rst == 0
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+    if not acc:
+        assert np.flatnonzero(ref).size == 2 * len(gaps)  # every far record decoded to a value
