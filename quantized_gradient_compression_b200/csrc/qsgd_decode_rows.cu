@@ -50,11 +50,14 @@ constexpr uint32_t kParseGuard = 1u << 20;  // a second, explicit bound of the p
 // MSB-first reader of one bucket over two stream words: the next unread bits are
 // the top bits of funnelshift(nx, cur, off) (0 <= off < 32); `left` counts the bits
 // of the bucket not yet consumed (negative, as int32, after a record that overran).
-struct RowReader {
+// kAhead: one more word held, loaded a word ahead of its use (the large-bucket
+// decoders, whose few warps per SM wait on each refill otherwise).
+template <bool kAhead>
+struct RowReaderT {
     const uint32_t* base;  // word holding the bucket's first bit
     uint32_t wi;           // next word to fetch, relative to base
     uint32_t wlim;         // words available from base to the end of the stream
-    uint32_t cur, nx, off;
+    uint32_t cur, nx, nx2, off;
     int32_t left;
     __device__ __forceinline__ uint32_t fetch() {
         const uint32_t w = wi < wlim ? __ldg(base + wi) : 0u;
@@ -68,6 +71,7 @@ struct RowReader {
         wi = 0;
         cur = fetch();
         nx = fetch();
+        if (kAhead) nx2 = fetch();
         off = static_cast<uint32_t>(begin & 31u);
         left = static_cast<int32_t>(nbits);
     }
@@ -77,7 +81,12 @@ struct RowReader {
         left -= static_cast<int32_t>(n);
         if (off >= 32u) {
             cur = nx;
-            nx = fetch();
+            if (kAhead) {
+                nx = nx2;
+                nx2 = fetch();
+            } else {
+                nx = fetch();
+            }
             off -= 32u;
         }
     }
@@ -98,10 +107,12 @@ struct RowReader {
         }
     }
 };
+using RowReader = RowReaderT<false>;
 
 // A record the table does not hold, bit by bit: false when it is malformed (its gap
 // beyond the bucket length d, or its level beyond s).
-__device__ __forceinline__ bool slow_record(RowReader& r, uint32_t s, uint32_t d, uint32_t& gap, uint32_t& sign,
+template <class Reader>
+__device__ __forceinline__ bool slow_record(Reader& r, uint32_t s, uint32_t d, uint32_t& gap, uint32_t& sign,
                                             uint32_t& k) {
     if (!r.omega(gap) || r.left <= 0 || gap > d) return false;
     sign = r.peek() >> 31;
@@ -190,7 +201,8 @@ __device__ __forceinline__ bool rows_table_step(RowReader& r, const uint32_t* lu
 // A record the table step does not take: far_long_record (gap < 2^16, k <= 15),
 // else bit by bit.  Returns false when it is malformed (gap beyond d, level beyond
 // s); else its gap, sign and level, the reader past it.
-__device__ __forceinline__ bool far_record(RowReader& r, const uint8_t* plut, const uint8_t* klut, uint32_t s,
+template <class Reader>
+__device__ __forceinline__ bool far_record(Reader& r, const uint8_t* plut, const uint8_t* klut, uint32_t s,
                                            uint32_t d, uint32_t& gap, uint32_t& sign, uint32_t& k) {
     uint32_t code = 0;
     const uint32_t len = far_long_record(r.peek(), plut, klut, gap, code);
@@ -1080,7 +1092,7 @@ __device__ __forceinline__ bool sparse_bucket(const DecodeArgs& a, const uint32_
             bad = true;
             continue;
         }
-        RowReader r;
+        RowReaderT<true> r;
         r.init(st.words, st.num_words, begin, static_cast<uint32_t>(end - begin));
         const uint32_t nbits = r.peek();
         r.advance(32);
@@ -1191,7 +1203,9 @@ __global__ void __launch_bounds__(kSparseBlock) sparse_fill(float* out, uint64_t
                              static_cast<uint64_t>(gridDim.x) * kSparseBlock);
 }
 
-// The decode's records: thread t of the grid takes bucket t.
+// The decode's records: lanes 0 .. kSparseRecLanes - 1 of every warp take a bucket
+// each (fewer chains a warp, so less of the warp's time goes to paths that only
+// some of its lanes take, and more warps an SM to hide each chain's latency).
 __global__ void __launch_bounds__(kSparseRecBlock) sparse_records(const __grid_constant__ DecodeArgs a) {
     __shared__ __align__(16) uint32_t lut[kLutSize];
     __shared__ __align__(16) uint8_t plut[1 << kPLutBits];
@@ -1200,8 +1214,10 @@ __global__ void __launch_bounds__(kSparseRecBlock) sparse_records(const __grid_c
     p_lut_fill(plut, threadIdx.x, kSparseRecBlock);
     k_lut_fill(klut, threadIdx.x, kSparseRecBlock);
     __syncthreads();
-    const uint64_t b = static_cast<uint64_t>(blockIdx.x) * kSparseRecBlock + threadIdx.x;
-    if (b < a.nb && !sparse_bucket<false>(a, lut, plut, klut, b)) atomicOr(a.status, QSGD_ST_BAD_STREAM);
+    const uint32_t lane = threadIdx.x & 31u;
+    const uint64_t b = static_cast<uint64_t>(blockIdx.x) * kSparseRecBuckets + (threadIdx.x >> 5) * kSparseRecLanes + lane;
+    if (lane < kSparseRecLanes && b < a.nb && !sparse_bucket<false>(a, lut, plut, klut, b))
+        atomicOr(a.status, QSGD_ST_BAD_STREAM);
 }
 
 // Decode-accumulate: a CTA a group of kSparseGroup buckets, the fill by all its
@@ -1345,7 +1361,7 @@ cudaError_t launch_sparse(const DecodeArgs& a, bool accumulate, cudaStream_t str
         const uint64_t fill_blocks = std::max<uint64_t>(
             1, std::min<uint64_t>((fill_threads + kSparseBlock - 1) / kSparseBlock, static_cast<uint64_t>(sms) * 8));
         sparse_fill<<<static_cast<unsigned>(fill_blocks), kSparseBlock, 0, stream>>>(a.out, a.n);
-        const uint64_t rec_blocks = (a.nb + kSparseRecBlock - 1) / kSparseRecBlock;
+        const uint64_t rec_blocks = (a.nb + kSparseRecBuckets - 1) / kSparseRecBuckets;
         sparse_records<<<static_cast<unsigned>(rec_blocks), kSparseRecBlock, 0, stream>>>(a);
         return cudaGetLastError();
     }

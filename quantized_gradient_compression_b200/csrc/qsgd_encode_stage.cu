@@ -837,14 +837,16 @@ __global__ void __launch_bounds__(kCompactThreads, 2) compact_stream(const __gri
         asm volatile("cp.async.wait_all;\n" ::: "memory");
         __syncthreads();
     }
-    // G lanes per bucket (G = 8, 16 or 32, from the tile's mean bucket size), over the
+    // G lanes per bucket (G = 4 below 16 words a bucket on the tile's mean, else 8: a
+    // quarter of the lanes that would cover a mean bucket at once, so that one setup
+    // serves several words a lane), over the
     // output words whose first bit lies in the bucket: word k is bits [delta + 32 k,
     // + 32) of the bucket's staged bits, delta the distance from the bucket's start to
     // the next word boundary; a word that runs past the bucket's end takes the first
     // bits of the next bucket (always >= 32 bits, so one word of it suffices).  Every
     // output word has exactly one writer.
     const uint32_t mean_words = total / (32u * nt);
-    const uint32_t G = mean_words < 8u ? 8u : mean_words < 16u ? 16u : 32u;
+    const uint32_t G = mean_words < 16u ? 4u : 8u;
     const uint32_t per_warp = 32u / G, sub = static_cast<uint32_t>(lane) / G, sl = static_cast<uint32_t>(lane) % G;
     const uint32_t step = kWarps * per_warp;
     if (gather) {  // the words are in shared memory

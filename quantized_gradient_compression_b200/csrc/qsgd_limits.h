@@ -80,7 +80,12 @@ constexpr uint32_t kRowsMaxS = 32767;
 // output of 32 buckets, then one lane per bucket stores the records.
 constexpr int kSparseBlock = 256;
 constexpr int kSparseGroup = 8;     // buckets a CTA of the large-bucket decode-accumulate takes at once
-constexpr int kSparseRecBlock = 64;  // threads (buckets) a CTA of the large-bucket decode's records
+#ifndef QSGD_SPARSE_REC_LANES
+#define QSGD_SPARSE_REC_LANES 4
+#endif
+constexpr int kSparseRecBlock = 256;                      // threads a CTA of the large-bucket decode's records
+constexpr int kSparseRecLanes = QSGD_SPARSE_REC_LANES;    // lanes of a warp there that take a bucket
+constexpr int kSparseRecBuckets = kSparseRecBlock / 32 * kSparseRecLanes;  // buckets a CTA
 
 constexpr int kDecodeBlock = 128;
 constexpr int kMaxStreamsPerLaunch = 16;  // decode-accumulate streams per launch

@@ -150,7 +150,7 @@ int main(int argc, char** argv) {
             } else {  // the fill (grid CTAs, grid-stride), then a lane a bucket
                 run_grid(grid, qsgd::kSparseBlock, 0, [&] { qsgd::sparse_fill(a.out, a.n); });
                 if (g_emu_error) return 4;
-                run_grid((unsigned)((nb + qsgd::kSparseRecBlock - 1) / qsgd::kSparseRecBlock), qsgd::kSparseRecBlock, 0,
+                run_grid((unsigned)((nb + qsgd::kSparseRecBuckets - 1) / qsgd::kSparseRecBuckets), qsgd::kSparseRecBlock, 0,
                          [&] { qsgd::sparse_records(a); });
             }
             if (g_emu_error) return 4;
