@@ -179,12 +179,14 @@ QSGD_API int qsgd_decode(const uint32_t* d_words, uint64_t num_words, const uint
  *                                    pointers / word counts (copied at the call)
  *   1 <= K <= 1024
  * Status bits as for qsgd_decode.  Up to 16 streams go to one launch (launches in
- * stream order).  With a 16-byte aligned d_out and d % 4 == 0: for d <= 4096 and
- * s < 1024 the streams are decoded side by side (a warp per stream) and d_out is read
- * and written once per eight streams; for d <= 1024 and larger s they are added onto
- * fp32 tiles one after another; for d > 1024 the launch fills the buckets' outputs
- * with +0-added values and then adds each stream's records in order.  One stream on
- * d <= 1024 takes the one-stream row decoder.  The result is the same on every path. */
+ * stream order).  With a 16-byte aligned d_out and d % 4 == 0: for d <= 1024 and
+ * s <= 127 the streams are parsed side by side (a warp per stream) into byte codes
+ * and added segment by segment, d_out read and written once per eight streams; for
+ * d <= 4096 and s < 1024 otherwise they are decoded side by side onto fp32 tiles; for
+ * d <= 1024 and larger s they are added onto fp32 tiles one after another; for
+ * d > 1024 the launch adds +0 to the buckets' outputs and then each stream's records
+ * in order.  One stream on d <= 1024 takes the one-stream row decoder.  The result is
+ * the same on every path. */
 QSGD_API int qsgd_decode_accumulate(const uint32_t* const* h_words, const uint64_t* h_num_words,
                            const uint64_t* const* h_offsets, int K, uint64_t n, uint32_t d,
                            uint32_t s, float* d_out, uint32_t* d_status, cudaStream_t stream);
