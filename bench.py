@@ -41,7 +41,7 @@ FALLBACK_HBM_GBS = 6650.0
 # differ.
 TRAFFIC_SOURCES = ("qsgd_encode_stage.cu", "qsgd_decode_rows.cu", "qsgd_tables.cuh", "qsgd_device.cuh", "qsgd_limits.h")
 TRAFFIC = {"bytes_per_launch": {"encode": 121254656, "decode": 50603008, "decode_accumulate": 153385728},
-           "sources_sha256": "fe42761f461d4d61a992a4bd6a90e9402da35d130677325cf96d3484aa515254"}
+           "sources_sha256": "ea15be31703e96903cf2ee56a299e9385d1b9203cd9f34b2038203f6d778a144"}
 
 
 # The kernels behind each phase of the c2 step (d = 512, s = 16, aligned buffers).

@@ -36,7 +36,8 @@ constexpr int kFastBlock = 32 * kFastWarps;
 // Fast encoder pipeline: a CTA gathers the prefix of (and stores) the tile it coded
 // enc_depth(V) iterations earlier, with enc_depth(V) + 1 tile buffers (V = float4s
 // per lane).  Depth 1 by default: depth 2 (QSGD_ENC_DEPTH=2, for V <= 4) measured
-// the same on c2.  V = 8 always uses depth 1, so that its larger tiles leave room
+// the same on the 25.6 M coordinate gradient at d = 512.  V = 8 always uses depth 1,
+// so that its larger tiles leave room
 // for two CTAs per SM.
 #ifndef QSGD_ENC_DEPTH
 #define QSGD_ENC_DEPTH 1
