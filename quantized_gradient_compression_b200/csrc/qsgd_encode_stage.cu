@@ -114,6 +114,32 @@ __device__ __forceinline__ void put_bits64(uint32_t* buf, uint32_t pos, uint64_t
     put_bits(buf, pos, static_cast<uint32_t>(code), len);
 }
 
+// Appends len (0..31) bits of code, right-aligned, to the 96-bit register string
+// (w2:w1:w0), right-aligned too.
+__device__ __forceinline__ void string_append(uint32_t& w0, uint32_t& w1, uint32_t& w2, uint32_t code, uint32_t len) {
+    w2 = __funnelshift_l(w1, w2, len);
+    w1 = __funnelshift_l(w0, w1, len);
+    w0 = (w0 << len) | code;
+}
+
+// ORs the right-aligned nbits (1..96) bits of the register string (w2:w1:w0) into the
+// zeroed bit buffer at bit position pos: left-aligned in 96 bits, then at most four
+// word atomics.
+__device__ __forceinline__ void string_or(uint32_t* buf, uint32_t pos, uint32_t w0, uint32_t w1, uint32_t w2,
+                                          uint32_t nbits) {
+    const uint32_t sa = 96u - nbits, bsh = sa & 31u, wsh = sa >> 5;
+    const uint32_t t2 = __funnelshift_l(w1, w2, bsh), t1 = __funnelshift_l(w0, w1, bsh), t0 = w0 << bsh;
+    const uint32_t L0 = wsh == 0 ? t2 : wsh == 1 ? t1 : t0;
+    const uint32_t L1 = wsh == 0 ? t1 : wsh == 1 ? t0 : 0u;
+    const uint32_t L2 = wsh == 0 ? t0 : 0u;
+    const uint32_t wp = pos >> 5, sh = pos & 31u;
+    const uint32_t nw = (sh + nbits + 31u) >> 5;  // 1..4
+    atomicOr(&buf[wp], L0 >> sh);
+    if (nw > 1) atomicOr(&buf[wp + 1], __funnelshift_r(L1, L0, sh));
+    if (nw > 2) atomicOr(&buf[wp + 2], __funnelshift_r(L2, L1, sh));
+    if (nw > 3) atomicOr(&buf[wp + 3], __funnelshift_r(0u, L2, sh));
+}
+
 // Stores one lane's 4V values (float4 L + 32j of a bucket of m values at p) with
 // streaming stores; nothing past m is written.
 template <int V>
@@ -253,9 +279,7 @@ __device__ __forceinline__ void code_chunk(const StageArgs& a, const uint32_t* r
             // below the lane's first record the gap wraps, but k = 0 there: an empty entry
             const uint32_t e = rtab[(((q0 + c - prev) << 6) | kr) & (kRecordTab64 - 1)];
             const uint32_t len = e & 31u;
-            w2 = __funnelshift_l(w1, w2, len);
-            w1 = __funnelshift_l(w0, w1, len);
-            w0 = (w0 << len) | (e >> 5);
+            string_append(w0, w1, w2, e >> 5, len);
             nbits += len;
             prev = kr > 1u ? q0 + c : prev;
         }
@@ -297,20 +321,7 @@ __device__ __forceinline__ void code_chunk(const StageArgs& a, const uint32_t* r
     const uint32_t P = pos + incl - nbits;
     pos += __shfl_sync(kAll, incl, 31);
     if (!__any_sync(kAll, nbits > 96u)) {
-        if (nbits != 0u) {
-            // left-align the string in 96 bits, then OR it in at bit P
-            const uint32_t sa = 96u - nbits, bsh = sa & 31u, wsh = sa >> 5;
-            const uint32_t t2 = __funnelshift_l(w1, w2, bsh), t1 = __funnelshift_l(w0, w1, bsh), t0 = w0 << bsh;
-            const uint32_t L0 = wsh == 0 ? t2 : wsh == 1 ? t1 : t0;
-            const uint32_t L1 = wsh == 0 ? t1 : wsh == 1 ? t0 : 0u;
-            const uint32_t L2 = wsh == 0 ? t0 : 0u;
-            const uint32_t wp = P >> 5, sh = P & 31u;
-            const uint32_t nw = (sh + nbits + 31u) >> 5;  // 1..4
-            atomicOr(&buf[wp], L0 >> sh);
-            if (nw > 1) atomicOr(&buf[wp + 1], __funnelshift_r(L1, L0, sh));
-            if (nw > 2) atomicOr(&buf[wp + 2], __funnelshift_r(L2, L1, sh));
-            if (nw > 3) atomicOr(&buf[wp + 3], __funnelshift_r(0u, L2, sh));
-        }
+        if (nbits != 0u) string_or(buf, P, w0, w1, w2, nbits);
     } else {  // some lane's string is longer than 96 bits: record by record
         int32_t prev = prev_in;
         uint32_t p = P;
@@ -487,23 +498,22 @@ __global__ void __launch_bounds__(kStageBlock, (V <= 4 ? 4 : 2)) code_buckets_sh
 }
 
 // ---------------------------------------------------------------------------
-// 1. Bucket coder.  kShort: s <= 31, records of gap < 64 through the whole-record
-// table (the others from the omega table), every record <= 30 bits.  Otherwise every
-// record from the omega table (or computed for k >= 2048), up to 18 + 1 + 34 bits.
+// 1b. Bucket coder for s > 31 (d <= 1024): lane L holds the float4s L + 32j of its
+// bucket, coded run by run (run j is coordinates [128j, 128j + 128)).  Every record
+// is omega(gap) | sign from the omega table, then omega(k) from the omega table (or
+// computed for k >= 2048), up to 18 + 1 + 34 bits.  A lane appends its run's records
+// to a 96-bit register string and ORs it into the bucket buffer once its position is
+// known; a run where some lane's string is longer, or a level's code longer than 31
+// bits, is placed record by record.
 // ---------------------------------------------------------------------------
-template <int V, bool kShort, bool kEF>
+template <int V, bool kEF>
 __global__ void __launch_bounds__(kStageBlock) code_buckets(const __grid_constant__ StageArgs a) {
     extern __shared__ __align__(16) uint32_t smem[];
     constexpr int NC = 4 * V;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    uint32_t* const otab = smem;                                                  // omega table
-    uint32_t* const rtab = smem + kOmegaTab;                                      // record table (kShort)
-    uint32_t* const buf = smem + kOmegaTab + (kShort ? kRecordTab64 : 0) + warp * a.buf_words;  // this warp's bucket bits
+    uint32_t* const otab = smem;                                    // omega table
+    uint32_t* const buf = smem + kOmegaTab + warp * a.buf_words;    // this warp's bucket bits
     omega_table_fill(otab, tid, kStageBlock);
-    if constexpr (kShort) {
-        const uint4* src = reinterpret_cast<const uint4*>(kRecordTable64Global.v);
-        for (int i = tid; i < kRecordTab64 / 4; i += kStageBlock) reinterpret_cast<uint4*>(rtab)[i] = src[i];
-    }
     for (uint32_t i = lane; i < a.buf_words; i += 32) buf[i] = 0u;
     // the compaction's scan state for this call: cleared here, before it runs
     {
@@ -595,52 +605,38 @@ __global__ void __launch_bounds__(kStageBlock) code_buckets(const __grid_constan
             const uint32_t B = __ballot_sync(kAll, m4 != 0u);
             const uint32_t lower = B & ((1u << lane) - 1u);
             const int32_t pv = __shfl_sync(kAll, last, lower ? 31 - __clz(lower) : 0);
-            int32_t prev = lower ? pv : carry;
+            const int32_t prev_in = lower ? pv : carry;
             carry = B ? __shfl_sync(kAll, last, 31 - __clz(B)) : carry;
-            // the lane's records of this run: codes and their total length
-            uint32_t code[4], len[4];
-            uint64_t kcode[kShort ? 1 : 4];
-            uint32_t klen[kShort ? 1 : 4];
-            uint32_t lbits = 0;
+            // the lane's records of this run, appended to the register string while
+            // every piece is at most 31 bits
+            uint32_t w0 = 0, w1 = 0, w2 = 0, lbits = 0;
+            bool fits = true;
+            {
+                int32_t prev = prev_in;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const uint32_t kv = kq[4 * j + c];
-                const uint32_t k = kv & 0x7FFFFFFFu;
-                const uint32_t gap = static_cast<uint32_t>(static_cast<int32_t>(qb + c) - prev);
-                code[c] = 0;
-                len[c] = 0;
-                if constexpr (!kShort) {
-                    kcode[c] = 0;
-                    klen[c] = 0;
-                }
-                if (k != 0u) {
-                    prev = static_cast<int32_t>(qb + c);
-                    if constexpr (kShort) {
-                        if (gap < 64u) {
-                            const uint32_t e = rtab[(gap << 6) | __funnelshift_l(kv, kv, 1)];
-                            code[c] = e >> 5;
-                            len[c] = e & 31u;
-                        } else {  // omega(gap) from the table (gap <= d <= 1024), then sign, omega(k)
-                            const uint32_t ge = otab[gap], ke = otab[k];
-                            const uint32_t kl = ke & 0xFFu;
-                            code[c] = ((((ge >> 8) << 1) | (kv >> 31)) << kl) | (ke >> 8);
-                            len[c] = (ge & 0xFFu) + 1u + kl;
-                        }
-                    } else {
-                        const uint32_t ge = otab[gap];
-                        code[c] = ((ge >> 8) << 1) | (kv >> 31);
-                        len[c] = (ge & 0xFFu) + 1u;
+                for (int c = 0; c < 4; ++c) {
+                    const uint32_t kv = kq[4 * j + c];
+                    const uint32_t k = kv & 0x7FFFFFFFu;
+                    if (k != 0u) {
+                        const uint32_t gap = static_cast<uint32_t>(static_cast<int32_t>(qb + c) - prev);
+                        prev = static_cast<int32_t>(qb + c);
+                        const uint32_t ge = otab[gap];  // gap <= d <= 1024
+                        const uint32_t glen = (ge & 0xFFu) + 1u;
+                        string_append(w0, w1, w2, ((ge >> 8) << 1) | (kv >> 31), glen);
+                        uint64_t kcode;
+                        uint32_t klen;
                         if (k < static_cast<uint32_t>(kOmegaTab)) {
                             const uint32_t ke = otab[k];
-                            kcode[c] = ke >> 8;
-                            klen[c] = ke & 0xFFu;
+                            kcode = ke >> 8;
+                            klen = ke & 0xFFu;
                         } else {
-                            omega_compute(k, kcode[c], klen[c]);
+                            omega_compute(k, kcode, klen);
                         }
+                        fits = fits && klen <= 31u;
+                        string_append(w0, w1, w2, static_cast<uint32_t>(kcode), klen <= 31u ? klen : 0u);
+                        lbits += glen + klen;
                     }
                 }
-                lbits += len[c];
-                if constexpr (!kShort) lbits += klen[c];
             }
             // the lane's first bit in the run: exclusive scan of the lane lengths
             uint32_t incl = lbits;
@@ -649,15 +645,34 @@ __global__ void __launch_bounds__(kStageBlock) code_buckets(const __grid_constan
                 const uint32_t t = __shfl_up_sync(kAll, incl, o);
                 if (lane >= o) incl += t;
             }
-            uint32_t p = pos + incl - lbits;
+            const uint32_t p0 = pos + incl - lbits;
+            if (!__any_sync(kAll, !fits || lbits > 96u)) {
+                if (lbits != 0u) string_or(buf, p0, w0, w1, w2, lbits);
+            } else {  // some lane's string is longer than 96 bits: record by record
+                int32_t prev = prev_in;
+                uint32_t p = p0;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                if (len[c] != 0u) {
-                    put_bits(buf, p, code[c], len[c]);
-                    p += len[c];
-                    if constexpr (!kShort) {
-                        put_bits64(buf, p, kcode[c], klen[c]);
-                        p += klen[c];
+                for (int c = 0; c < 4; ++c) {
+                    const uint32_t kv = kq[4 * j + c];
+                    const uint32_t k = kv & 0x7FFFFFFFu;
+                    if (k != 0u) {
+                        const uint32_t gap = static_cast<uint32_t>(static_cast<int32_t>(qb + c) - prev);
+                        prev = static_cast<int32_t>(qb + c);
+                        const uint32_t ge = otab[gap];
+                        const uint32_t glen = (ge & 0xFFu) + 1u;
+                        put_bits(buf, p, ((ge >> 8) << 1) | (kv >> 31), glen);
+                        p += glen;
+                        uint64_t kcode;
+                        uint32_t klen;
+                        if (k < static_cast<uint32_t>(kOmegaTab)) {
+                            const uint32_t ke = otab[k];
+                            kcode = ke >> 8;
+                            klen = ke & 0xFFu;
+                        } else {
+                            omega_compute(k, kcode, klen);
+                        }
+                        put_bits64(buf, p, kcode, klen);
+                        p += klen;
                     }
                 }
             }
@@ -964,7 +979,7 @@ cudaError_t launch_code(const StageArgs& a, cudaStream_t stream) {
     if constexpr (kShort)
         return launch_coder<code_buckets_short<V, kEF>>(a, stream);
     else
-        return launch_coder<code_buckets<V, false, kEF>>(a, stream);
+        return launch_coder<code_buckets<V, kEF>>(a, stream);
 }
 
 template <int V>

@@ -70,7 +70,7 @@ static void code(const qsgd::StageArgs& a, unsigned grid, size_t smem) {
     if constexpr (kShort)
         run_grid(grid, qsgd::kStageBlock, smem, [&] { qsgd::code_buckets_short<V, kEF>(a); });
     else
-        run_grid(grid, qsgd::kStageBlock, smem, [&] { qsgd::code_buckets<V, false, kEF>(a); });
+        run_grid(grid, qsgd::kStageBlock, smem, [&] { qsgd::code_buckets<V, kEF>(a); });
 }
 template <int V, bool kEF>
 static void code_v(const qsgd::StageArgs& a, unsigned grid, size_t smem) {

@@ -101,6 +101,9 @@ CASES = [
     (70_001, 200, 7, 2, "normal"),
     (3_001, 4, 2, 1, "normal"),
     (5_000, 384, 3000, 1, "normal"),
+    # levels whose codes make a lane's run longer than 96 bits, and codes past 31 bits
+    (4_000, 128, 1 << 20, 1, "normal"),
+    (4_000, 256, 1 << 22, 1, "normal"),
     (6_000, 1000, 31, 2, "layered"),
     (1, 512, 16, 1, "normal"),
     # buckets of several 512-coordinate chunks (s <= 31): whole, ragged and partial chunks
