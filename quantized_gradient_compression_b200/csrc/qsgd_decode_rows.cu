@@ -372,9 +372,11 @@ __global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows(const __grid_c
 #endif
 constexpr uint32_t kRSeg = QSGD_ROWS_SEG;
 constexpr uint32_t kRRing = 2 * kRSeg;
-static_assert(kRSeg % 128 == 0 && kRSeg >= 128, "a segment is whole float4 columns of the warp");
-constexpr int kRVec = static_cast<int>(kRSeg / 128);  // float4 per lane per row per segment
-constexpr int kRBatch = 8;                             // rows whose output is loaded together
+static_assert(kRSeg == 64 || (kRSeg % 128 == 0 && kRSeg >= 128), "a segment is half a warp's or whole float4 columns");
+constexpr uint32_t kRLanesPerRow = kRSeg / 4 < 32 ? kRSeg / 4 : 32;  // lanes on one row of a segment
+constexpr uint32_t kRRowsPerPass = 32 / kRLanesPerRow;               // rows a warp writes at once
+constexpr int kRVec = kRSeg / 128 > 0 ? static_cast<int>(kRSeg / 128) : 1;  // float4 per lane per row
+constexpr int kRBatch = 8;  // passes whose output is loaded together
 
 template <bool kAcc>
 __global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows_ring(const __grid_constant__ DecodeArgs a,
@@ -494,20 +496,23 @@ __global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows_ring(const __g
             }
             __syncwarp();
             // --- write back columns [lo, hi) of the 32 rows, and clear them ----------
-            // (decode-accumulate loads the output of kRBatch rows at a time, so that
-            // their loads are in flight together)
-            for (int r0 = 0; r0 < nrows; r0 += kRBatch) {
+            // (kRRowsPerPass rows a pass, kRLanesPerRow lanes a row; decode-accumulate
+            // loads the output of kRBatch passes at a time, so that their loads are in
+            // flight together)
+            const uint32_t wsub = static_cast<uint32_t>(lane) / kRLanesPerRow;
+            const uint32_t wcol = static_cast<uint32_t>(lane) % kRLanesPerRow;
+            for (int r0 = 0; r0 < nrows; r0 += kRBatch * static_cast<int>(kRRowsPerPass)) {
                 float4 o[kAcc ? kRBatch * kRVec : 1];
                 if constexpr (kAcc) {
 #pragma unroll
                     for (int t = 0; t < kRBatch; ++t) {
-                        const int rr = r0 + t;
+                        const int rr = r0 + t * static_cast<int>(kRRowsPerPass) + static_cast<int>(wsub);
                         const uint64_t bb = g * 32 + rr;
                         const uint32_t mm = rr < nrows ? static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - bb * d)) : 0u;
                         const float* gp = a.out + bb * d;
 #pragma unroll
                         for (int i = 0; i < kRVec; ++i) {
-                            const uint32_t c = lo + 4u * (static_cast<uint32_t>(lane) + 32u * i);
+                            const uint32_t c = lo + 4u * (wcol + kRLanesPerRow * i);
                             float4& x = o[t * kRVec + i];
                             x = make_float4(0.f, 0.f, 0.f, 0.f);
                             if (c + 4 <= mm) {
@@ -522,16 +527,16 @@ __global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows_ring(const __g
                 }
 #pragma unroll
                 for (int t = 0; t < kRBatch; ++t) {
-                    const int rr = r0 + t;
-                    if (rr >= nrows) break;
+                    const int rr = r0 + t * static_cast<int>(kRRowsPerPass) + static_cast<int>(wsub);
+                    const float sc = __shfl_sync(kWarpAll, scale, rr & 31);
+                    if (rr >= nrows) continue;
                     const uint64_t bb = g * 32 + rr;
-                    const float sc = __shfl_sync(kWarpAll, scale, rr);
                     const uint32_t mm = static_cast<uint32_t>(min(static_cast<uint64_t>(d), a.n - bb * d));
                     uint32_t* const rowp = rows + static_cast<uint32_t>(rr) * stride_w;
                     float* const gp = a.out + bb * d;
 #pragma unroll
                     for (int i = 0; i < kRVec; ++i) {
-                        const uint32_t c = lo + 4u * (static_cast<uint32_t>(lane) + 32u * i);
+                        const uint32_t c = lo + 4u * (wcol + kRLanesPerRow * i);
                         if (c < mm) {
                             const uint32_t q = (c & (kRRing - 1u)) >> 2;  // four codes
                             const uint2 w = reinterpret_cast<const uint2*>(rowp)[q];

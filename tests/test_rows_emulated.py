@@ -289,6 +289,22 @@ def test_side_decoder_128_column_segments(rows_exe_seg128, tmp_path, oracle_lib,
     test_side_decoder_matches_oracle(rows_exe_seg128, tmp_path, oracle_lib, n, d, s, K, mean, grid, kind)
 
 
+@pytest.fixture(scope="module")
+def rows_exe_ring64(tmp_path_factory):
+    if shutil.which("g++") is None:
+        pytest.skip("g++ not available")
+    return build_rows_exe(tmp_path_factory.mktemp("rowsemuring64"), ("-O1", "-DQSGD_ROWS_SEG=64"))
+
+
+RING = [c for c in CASES if c[2] > 127]
+
+
+@pytest.mark.parametrize("n,d,s,accumulate,grid,warps,kind", RING, ids=["n%d-d%d-s%d-acc%d-g%d-w%d-%s" % c for c in RING])
+def test_ring_decoder_64_column_segments(rows_exe_ring64, tmp_path, oracle_lib, n, d, s, accumulate, grid, warps, kind):
+    """The 16-bit ring decoder built with segments of 64 columns (two rows a pass)."""
+    test_row_decoder_matches_oracle(rows_exe_ring64, tmp_path, oracle_lib, n, d, s, accumulate, grid, warps, kind)
+
+
 def test_side_decoder_far_records(rows_exe, tmp_path, oracle_lib):
     """Buckets whose records lie more than two segments ahead (bit-serial gaps held
     back until their segment), next to dense buckets, in three streams."""
