@@ -22,14 +22,18 @@ def _base(n, seed):
     return b
 
 
-# (n, d, s, K): the one-stream row decoder (K = 1), the several-stream row decoder
-# (d <= 1024, d a multiple of 4), the large-bucket decoder (d > 1024), the one-lane
-# decoders (d < 4 or d not a multiple of 4), and K beyond one launch's 16 streams
+# (n, d, s, K): the one-stream row decoder (K = 1), the several-stream decoders on
+# d <= 1024 (byte codes side by side for s <= 127, fp32 tiles side by side below
+# s = 1024, fp32 tiles one stream after another above), the large-bucket decoder
+# (d > 1024), the one-lane decoders (d < 4 or d not a multiple of 4), and K beyond one
+# launch's 16 streams
 CASES = [
     (40_000, 132, 3, 3),
     (100_003, 512, 16, 1),
     (100_003, 512, 16, 3),
     (60_000, 512, 4, 17),
+    (40_000, 512, 300, 3),
+    (20_000, 512, 2000, 2),
     (50_000, 2048, 64, 2),
     (30_000, 100, 7, 3),
     (30_001, 8192, 2, 2),
