@@ -109,6 +109,85 @@ struct RowReaderT {
 };
 using RowReader = RowReaderT<false>;
 
+// The 16-bit ring decoder's reader: the bucket's stream words pass through a ring of
+// eight words a lane in shared memory, refilled four words at a time with cp.async
+// while the lane parses the other four.  (That kernel's shared memory leaves L1 little
+// room, so a word loaded straight from the stream waits on L2 at every refill.)  Same
+// bit order and interface as RowReaderT.
+struct StagedReader {
+    const uint32_t* base;  // word holding the bucket's first bit
+    uint32_t* sbuf;        // this lane's eight words (word w in slot w mod 8)
+    uint32_t wi;           // next word to read, relative to base
+    uint32_t wlim;         // words available from base to the end of the stream
+    uint32_t cur, nx, off;
+    int32_t left;
+    // words w0 .. w0 + 3 into their slots (zeros past the stream), one commit group
+    __device__ __forceinline__ void copy_half(uint32_t w0) {
+#pragma unroll
+        for (uint32_t i = 0; i < 4u; ++i) {
+            const uint32_t w = w0 + i;
+            uint32_t* const dst = sbuf + (w & 7u);
+            if (w < wlim) {
+                const uint32_t saddr = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+                const uint32_t* const src = base + w;
+                asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(saddr), "l"(src) : "memory");
+            } else {
+                *dst = 0u;
+            }
+        }
+        asm volatile("cp.async.commit_group;\n" ::: "memory");
+    }
+    __device__ __forceinline__ uint32_t fetch() {
+        if ((wi & 3u) == 0u) {  // entering a half: its words have landed; refill the half just left
+            asm volatile("cp.async.wait_all;\n" ::: "memory");
+            copy_half(wi + 4u);
+        }
+        const uint32_t w = sbuf[wi & 7u];
+        ++wi;
+        return w;
+    }
+    __device__ __forceinline__ void init(const uint32_t* words, uint64_t num_words, uint64_t begin, uint32_t nbits) {
+        asm volatile("cp.async.wait_all;\n" ::: "memory");  // no copy of an earlier bucket is still landing
+        const uint64_t w0 = begin >> 5;
+        base = words + w0;
+        wlim = static_cast<uint32_t>(min(num_words - w0, static_cast<uint64_t>(0xFFFFFFFFu)));
+        copy_half(0u);
+        copy_half(4u);
+        asm volatile("cp.async.wait_all;\n" ::: "memory");
+        cur = sbuf[0];
+        nx = sbuf[1];
+        wi = 2;
+        off = static_cast<uint32_t>(begin & 31u);
+        left = static_cast<int32_t>(nbits);
+    }
+    __device__ __forceinline__ uint32_t peek() const { return __funnelshift_l(nx, cur, off); }
+    __device__ __forceinline__ void advance(uint32_t n) {  // n <= 32
+        off += n;
+        left -= static_cast<int32_t>(n);
+        if (off >= 32u) {
+            cur = nx;
+            nx = fetch();
+            off -= 32u;
+        }
+    }
+    __device__ __forceinline__ bool omega(uint32_t& N) {  // bit-serial, any length up to 2^32 - 1
+        uint32_t v = 1;
+        for (;;) {
+            if (left <= 0) return false;
+            const uint32_t bit = peek() >> 31;
+            advance(1);
+            if (bit == 0) {
+                N = v;
+                return true;
+            }
+            if (v > 31 || left < static_cast<int32_t>(v)) return false;
+            const uint32_t rest = peek() >> (32 - v);
+            advance(v);
+            v = (1u << v) | rest;
+        }
+    }
+};
+
 // A record the table does not hold, bit by bit: false when it is malformed (its gap
 // beyond the bucket length d, or its level beyond s).
 template <class Reader>
@@ -153,8 +232,8 @@ __device__ __forceinline__ void load_row(const DecodeArgs& a, uint64_t bb, int l
 // (gap <= 63, k <= 15 and k <= s; at most 63 columns).  put(index, code) stores a
 // record's code (sign << 7 | k) at its bucket-local index.  Returns false, having
 // read nothing, when the record at the cursor is neither (far_record takes it).
-template <class Put>
-__device__ __forceinline__ bool rows_table_step(RowReader& r, const uint32_t* lut, const uint8_t* klut, uint32_t s,
+template <class Reader, class Put>
+__device__ __forceinline__ bool rows_table_step(Reader& r, const uint32_t* lut, const uint8_t* klut, uint32_t s,
                                                 uint32_t& next, const Put& put) {
     const uint32_t w = r.peek();
     const uint32_t e = lut[w >> (32 - kLutBits)];
@@ -386,6 +465,8 @@ __global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows_ring(const __g
     const int W = blockDim.x >> 5;
     uint32_t* const rows = smem + kLutSize + static_cast<uint32_t>(warp) * 32u * stride_w;
     uint16_t* const myrow = reinterpret_cast<uint16_t*>(rows + static_cast<uint32_t>(lane) * stride_w);
+    // this lane's ring of stream words (after every warp's rows)
+    uint32_t* const sbuf = smem + kLutSize + static_cast<uint32_t>(W) * 32u * stride_w + static_cast<uint32_t>(tid) * 8u;
     // the omega table, looked up for the gap and then for the level
     uint16_t* const olut = reinterpret_cast<uint16_t*>(smem);
     omega_lut_fill(olut, tid, blockDim.x);
@@ -411,7 +492,8 @@ __global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows_ring(const __g
             reinterpret_cast<uint4*>(rows)[q] = make_uint4(0u, 0u, 0u, 0u);
         // open this lane's bucket: header checks and the norm
         bool bad = false;
-        RowReader r;
+        StagedReader r;
+        r.sbuf = sbuf;
         r.left = 0;
         float scale = 0.f;
         if (live) {
@@ -578,6 +660,7 @@ __global__ void __launch_bounds__(32 * kRowsMaxWarps) decode_rows_ring(const __g
         if (bad) atomicOr(a.status, QSGD_ST_BAD_STREAM);
         __syncwarp();
     }
+    asm volatile("cp.async.wait_all;\n" ::: "memory");  // no copy outlives the CTA
 }
 
 // ---------------------------------------------------------------------------
@@ -1262,12 +1345,13 @@ constexpr uint32_t ring_stride_words() { return kRRing * 2 / 4 + 2; }
 
 // One CTA per SM, its warps one group each where the groups allow: every SM busy.
 template <class Kernel>
-cudaError_t launch_row_kernel(Kernel kernel, bool& attr_done, const DecodeArgs& a, uint32_t stride, cudaStream_t stream) {
+cudaError_t launch_row_kernel(Kernel kernel, bool& attr_done, const DecodeArgs& a, uint32_t stride, cudaStream_t stream,
+                              size_t extra_per_warp = 0) {
     int dev = 0, sms = 0, optin = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-    const size_t per_warp = static_cast<size_t>(32) * stride * sizeof(uint32_t);
+    const size_t per_warp = static_cast<size_t>(32) * stride * sizeof(uint32_t) + extra_per_warp;
     // the record table and the small tables (the ring kernel uses the first half of
     // the record table's room for its omega table, and the small tables' not at all)
     const size_t lut_bytes = static_cast<size_t>(kLutSize + kSmallLutWords) * sizeof(uint32_t);
@@ -1300,7 +1384,8 @@ cudaError_t launch_rows_ring(const DecodeArgs& a, cudaStream_t stream) {
     int dev = 0;
     cudaGetDevice(&dev);
     bool scratch = false;
-    return launch_row_kernel(decode_rows_ring<kAcc>, dev < 64 ? attr_set[dev] : scratch, a, ring_stride_words(), stream);
+    return launch_row_kernel(decode_rows_ring<kAcc>, dev < 64 ? attr_set[dev] : scratch, a, ring_stride_words(), stream,
+                             32 * 8 * sizeof(uint32_t));
 }
 
 template <bool kAcc>

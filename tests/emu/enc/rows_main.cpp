@@ -61,7 +61,8 @@ template <class T>
 static void run_t(const qsgd::DecodeArgs& a, bool acc, unsigned grid, unsigned W) {
     if constexpr (sizeof(T) == 2) {
         const uint32_t stride = qsgd::ring_stride_words();
-        const size_t smem = 4 * (size_t)(qsgd::kLutSize + qsgd::kSmallLutWords) + (size_t)W * 32 * stride * 4;
+        const size_t smem = 4 * (size_t)(qsgd::kLutSize + qsgd::kSmallLutWords) + (size_t)W * 32 * stride * 4 +
+                            (size_t)W * 32 * 8 * 4;
         if (acc)
             run_grid(grid, 32 * W, smem, [&] { qsgd::decode_rows_ring<true>(a, stride); });
         else
